@@ -1,0 +1,400 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself (brute force, closed forms, invariants, textbook routines, hand-derived
+examples).  Rules cited from "AdaCluster: Adaptive Query-Key Clustering for
+Sparse Attention in Video Generation" (Tan et al.)."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from clustered_sparse_attention_head_b200 import workloads as W
+
+
+def _gmm(n, d, comps, seed, sigma=0.3):
+    rng = np.random.default_rng(seed)
+    mu = rng.standard_normal((comps, d)).astype(np.float32)
+    lab = rng.integers(0, comps, n)
+    return (mu[lab] + sigma * rng.standard_normal((n, d))).astype(np.float32)
+
+
+# ---------------------------------------------------------------- assignment
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_assign_euclid_bruteforce_with_ties(orc, seed):
+    """§3.2.1: keys go to the Euclidean-closest centre.  Small integers make
+    every distance exact, duplicated centroids force exact ties -> lowest id."""
+    rng = np.random.default_rng(seed)
+    n, k, d = 40, 7, 3
+    x = rng.integers(-3, 4, (n, d)).astype(np.float32)
+    c = rng.integers(-3, 4, (k, d)).astype(np.float32)
+    c[5] = c[2]
+    ids, dist, obj = orc.assign(x.astype(np.float64), c, orc.EUCLID)
+    for i in range(n):
+        d2 = [sum((float(x[i, t]) - float(c[j, t])) ** 2 for t in range(d)) for j in range(k)]
+        best = min(range(k), key=lambda j: (d2[j], j))
+        assert ids[i] == best
+        assert dist[i] == math.sqrt(d2[best])
+    assert 5 not in ids.tolist()
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_assign_sphere_bruteforce(orc, seed):
+    """§3.1: normalised queries go to the centre of largest cosine; for unit
+    centroids that is also the Euclidean-closest centre on the sphere."""
+    rng = np.random.default_rng(seed)
+    n, k, d = 50, 6, 4
+    x = rng.standard_normal((n, d)).astype(np.float32)
+    c = rng.standard_normal((k, d))
+    c = (c / np.linalg.norm(c, axis=1, keepdims=True)).astype(np.float32)
+    c[4] = c[1]
+    xs, nrm = orc.prepare(x, orc.SPHERE)
+    ids, dist, _ = orc.assign(xs, c, orc.SPHERE)
+    for i in range(n):
+        xi = [float(v) for v in x[i]]
+        r = math.sqrt(sum(v * v for v in xi))
+        cos = [sum(xi[t] / r * float(c[j, t]) for t in range(d)) for j in range(k)]
+        eu = [sum((xi[t] / r - float(c[j, t])) ** 2 for t in range(d)) for j in range(k)]
+        best = max(range(k), key=lambda j: (cos[j], -j))
+        assert ids[i] == best
+        assert min(range(k), key=lambda j: (eu[j], j)) == best or abs(eu[best] - min(eu)) < 1e-12
+        assert abs(dist[i] - math.sqrt(eu[best])) < 1e-12
+    assert 4 not in ids.tolist()
+
+
+def test_normalise_unit_and_zero(orc):
+    """§3.1 normalisation: unit length, a zero query stays zero (and ties every
+    centroid, so it lands in cluster 0)."""
+    x = _gmm(30, 8, 3, 5)
+    x[7] = 0
+    xs, nrm = orc.prepare(x, orc.SPHERE)
+    np.testing.assert_allclose(np.linalg.norm(xs, axis=1)[np.arange(30) != 7], 1.0, atol=1e-15)
+    assert np.all(xs[7] == 0) and nrm[7] == 0
+    c = xs[[0, 10, 20]].astype(np.float32)
+    ids, _, _ = orc.assign(xs, c, orc.SPHERE)
+    assert ids[7] == 0
+
+
+def test_sphere_scale_invariance(orc):
+    """§3.1: the ranking of q.k over keys does not depend on ||q||, so query
+    clusters must not either.  Power-of-two scalings keep q/||q|| bit-identical."""
+    x = _gmm(400, 16, 6, 11)
+    s = (2.0 ** np.random.default_rng(3).integers(-6, 7, 400)).astype(np.float32)
+    a = orc.kmeans(orc.prepare(x, orc.SPHERE)[0], 6, 8, orc.SPHERE)
+    b = orc.kmeans(orc.prepare(x * s[:, None], orc.SPHERE)[0], 6, 8, orc.SPHERE)
+    assert np.array_equal(a.assign, b.assign)
+    assert np.array_equal(a.cent, b.cent)
+
+
+# ------------------------------------------------------------------- k-means
+@pytest.mark.parametrize("mode", [0, 1])
+def test_kmeans_objective_monotone(orc, mode):
+    """Lloyd's algorithm never increases its objective (assign and update both
+    minimise it); fp32 storage of centroids allows a relative 1e-6 slack."""
+    x = _gmm(3000, 32, 12, 21, sigma=0.8)
+    xs, _ = orc.prepare(x, mode)
+    r = orc.kmeans(xs, 20, 10, mode, trace=True)
+    tr = r.trace
+    assert np.all(np.diff(tr) <= 1e-6 * np.abs(tr[:-1]) + 1e-9), tr
+
+
+def test_kmeans_k1_closed_form(orc):
+    """k = 1: the Euclidean centre is the mean; the spherical centre is the
+    normalised sum of the unit vectors (textbook closed forms)."""
+    x = _gmm(500, 12, 3, 8)
+    r = orc.kmeans(x.astype(np.float64), 1, 3, orc.EUCLID)
+    np.testing.assert_array_equal(r.cent[0], x.astype(np.float64).mean(0).astype(np.float32))
+    xs, _ = orc.prepare(x, orc.SPHERE)
+    r2 = orc.kmeans(xs, 1, 3, orc.SPHERE)
+    u = x / np.linalg.norm(x.astype(np.float64), axis=1, keepdims=True)
+    s = u.sum(0)
+    np.testing.assert_allclose(r2.cent[0], (s / np.linalg.norm(s)).astype(np.float32), rtol=0, atol=1e-7)
+    assert np.all(r.assign == 0) and r.count[0] == 500
+
+
+def test_kmeans_separated_recovers_components(orc):
+    """Well-separated components with one seed per component: k-means returns the
+    component means (each centre = its component's sample mean)."""
+    rng = np.random.default_rng(4)
+    d, comps, per = 8, 5, 60
+    mu = 20.0 * rng.standard_normal((comps, d))
+    x = np.concatenate([mu[c] + 0.1 * rng.standard_normal((per, d)) for c in range(comps)]).astype(np.float32)
+    r = orc.kmeans(x.astype(np.float64), comps, 5, orc.EUCLID)
+    for c in range(comps):
+        np.testing.assert_array_equal(r.assign[c * per:(c + 1) * per], c)
+        np.testing.assert_allclose(r.cent[c], x[c * per:(c + 1) * per].astype(np.float64).mean(0), rtol=1e-6)
+
+
+def test_update_empty_cluster_keeps_centroid(orc):
+    x = _gmm(200, 4, 2, 9)
+    c = np.array([x[0], x[100], [1e4, 1e4, 1e4, 1e4]], np.float32)
+    ids, _, _ = orc.assign(x.astype(np.float64), c, orc.EUCLID)
+    c2, cnt = orc.update(x.astype(np.float64), ids, c, orc.EUCLID)
+    assert cnt[2] == 0 and np.array_equal(c2[2], c[2])
+
+
+def test_cauchy_schwarz_bound(orc):
+    """§3.2.1: |q.c(k) - q.k| <= ||q|| ||k - c(k)|| for every key and query."""
+    k = _gmm(800, 16, 8, 2)
+    q = _gmm(50, 16, 8, 3)
+    r = orc.kmeans(k.astype(np.float64), 8, 6, orc.EUCLID)
+    c = r.cent[r.assign].astype(np.float64)
+    lhs = np.abs(q.astype(np.float64) @ (c - k).T)
+    rhs = np.linalg.norm(q, axis=1)[:, None] * r.dist[None, :]
+    assert np.all(lhs <= rhs * (1 + 1e-12) + 1e-12)
+    np.testing.assert_allclose(r.dist, np.linalg.norm(k - c, axis=1), rtol=1e-12)
+
+
+# -------------------------------------------------------------- Algorithm 1
+def _four_groups():
+    """Three tight groups of 100 (spread 0.5) and a far pair, in 2-D."""
+    rng = np.random.default_rng(7)
+    cen = [(0.0, 0.0), (10.0, 0.0), (0.0, 10.0)]
+    pts = [np.array(c) + rng.uniform(-0.25, 0.25, (100, 2)) for c in cen]
+    pts.append(np.array([[30.0, 25.0], [31.0, 25.0]]))
+    return np.concatenate(pts).astype(np.float32)
+
+
+def test_multistage_hand_trace(orc):
+    """Algorithm 1 on a hand-built case (the Figure 5 idea): stage 0 (m0 = 3)
+    finds the three groups (the far pair joins the group at (10,0), whose centre
+    moves by < 0.6, so every group point stays within tau = 3); only the far pair
+    is left in U; stage 1 uses m_1 = ceil(3*2/302) = 1 cluster, whose centre is
+    the pair's midpoint (distance 0.5 < tau), so U empties: |C| = 4, F = False,
+    two stages; the final reassignment gives counts 100/100/100/2."""
+    x = _four_groups()
+    r = orc.multistage(x.astype(np.float64), 3, 10, orc.TAU_ABS, 3.0, 50, orc.EUCLID)
+    assert (r.nclusters, r.dense, r.nstages) == (4, 0, 2)
+    np.testing.assert_array_equal(np.sort(r.count), [2, 100, 100, 100])
+    for g in range(3):
+        assert len(set(r.assign[100 * g:100 * (g + 1)].tolist())) == 1
+    assert r.assign[300] == r.assign[301] == 3
+    np.testing.assert_allclose(r.cent[3], [30.5, 25.0], atol=1e-6)
+
+
+def test_multistage_nmax_sets_flag(orc):
+    """Algorithm 1 lines 5-7: U is non-empty after stage 0 and |C| = 3 >= N_max = 3,
+    so F is set and no further stage runs."""
+    x = _four_groups()
+    r = orc.multistage(x.astype(np.float64), 3, 10, orc.TAU_ABS, 3.0, 3, orc.EUCLID)
+    assert (r.nclusters, r.dense, r.nstages) == (3, 1, 1)
+
+
+def test_multistage_tau_zero_closed_form(orc):
+    """tau = 0 removes nothing (d_i < 0 never holds), so each stage adds m0
+    clusters until |C| >= N_max: ceil(N_max / m0) stages, F = True."""
+    x = _gmm(500, 6, 5, 1)
+    for m0, nmax in [(4, 10), (5, 5), (7, 30)]:
+        r = orc.multistage(x.astype(np.float64), m0, 3, orc.TAU_ABS, 0.0, nmax, orc.EUCLID)
+        st = -(-nmax // m0)
+        assert (r.nstages, r.nclusters, r.dense) == (st, st * m0, 1)
+
+
+def test_multistage_tau_inf_is_plain_kmeans(orc):
+    """tau = +inf empties U after stage 0: one stage of k-means with m0 centres,
+    F = False, and the final reassignment equals k-means' own final assignment."""
+    x = _gmm(600, 8, 6, 2)
+    for mode in (0, 1):
+        xs, _ = orc.prepare(x, mode)
+        r = orc.multistage(xs, 6, 5, orc.TAU_ABS, np.inf, 100, mode)
+        k = orc.kmeans(xs, 6, 5, mode)
+        assert (r.nclusters, r.dense, r.nstages) == (6, 0, 1)
+        assert np.array_equal(r.assign, k.assign) and np.array_equal(r.cent, k.cent)
+
+
+def test_multistage_terminates_and_partitions(orc):
+    """Every stage adds >= 1 centre, so the loop ends; the final assignment
+    covers every token and ids are < |C|; the capacity bound N_max + m0 holds."""
+    x = _gmm(2000, 16, 30, 6, sigma=1.0)
+    for rule, val in [(orc.TAU_MEAN_X, 1.0), (orc.TAU_MEDIAN_RADIUS_X, 0.5), (orc.TAU_ABS, 2.0)]:
+        r = orc.multistage(x.astype(np.float64), 16, 4, rule, val, 120, orc.EUCLID)
+        assert r.nclusters <= 120 + 16 and r.count.sum() == 2000
+        assert r.assign.min() >= 0 and r.assign.max() < r.nclusters
+        assert r.dense == (1 if r.nclusters >= 120 else 0) or r.dense == 0
+
+
+def test_tau_mean_rule_matches_stage0(orc):
+    """§4.1: tau = 1.5 x the mean token-to-centre distance of the first stage.
+    Stage 0 is plain k-means with m0 centres, so tau must equal 1.5 x the mean
+    of that run's distances, and rerunning with that tau as an absolute value
+    must reproduce the result."""
+    x = _gmm(1500, 16, 20, 8, sigma=0.7)
+    xs = x.astype(np.float64)
+    r = orc.multistage(xs, 10, 5, orc.TAU_MEAN_X, 1.5, 200, orc.EUCLID)
+    k0 = orc.kmeans(xs, 10, 5, orc.EUCLID)
+    assert r.tau == pytest.approx(1.5 * k0.dist.mean(), rel=1e-12)
+    r2 = orc.multistage(xs, 10, 5, orc.TAU_ABS, r.tau, 200, orc.EUCLID)
+    assert np.array_equal(r.assign, r2.assign) and r.nclusters == r2.nclusters
+
+
+def test_tau_median_radius_rule(orc):
+    x = _gmm(1500, 16, 20, 8, sigma=0.7)
+    xs = x.astype(np.float64)
+    r = orc.multistage(xs, 10, 5, orc.TAU_MEDIAN_RADIUS_X, 0.5, 200, orc.EUCLID)
+    k0 = orc.kmeans(xs, 10, 5, orc.EUCLID)
+    radii = sorted(k0.dist[k0.assign == j].mean() for j in range(10) if np.any(k0.assign == j))
+    assert r.tau == pytest.approx(0.5 * radii[(len(radii) - 1) // 2], rel=1e-12)
+
+
+# ---------------------------------------------------------------- selection
+def _sel(orc, t, counts, top_p, rbar=2.0, qcount=1):
+    """One query cluster with centroid e_0, mean norm rbar, d = 4 (so
+    s_b = rbar * t_b / 2), key centroids t_b * e_0."""
+    d = 4
+    qc = np.zeros((1, d), np.float32)
+    qc[0, 0] = 1
+    kc = np.zeros((len(t), d), np.float32)
+    kc[:, 0] = t
+    s, c = orc.select(qc, np.array([rbar], np.float32), np.array([qcount], np.int32), kc,
+                      np.array(counts, np.int32), top_p)
+    return sorted(s[0, :c[0]].tolist())
+
+
+def test_select_hand_example_sizes(orc):
+    """Equal scores: p_b is the size share n_b / sum n = [.1,.2,.3,.4]."""
+    assert _sel(orc, [0, 0, 0, 0], [1, 2, 3, 4], 0.5) == [2, 3]
+    assert _sel(orc, [0, 0, 0, 0], [1, 2, 3, 4], 0.4) == [3]
+    assert _sel(orc, [0, 0, 0, 0], [1, 2, 3, 4], 0.71) == [1, 2, 3]
+    assert _sel(orc, [0, 0, 0, 0], [1, 2, 3, 4], 1.0) == [0, 1, 2, 3]
+
+
+def test_select_hand_example_scores(orc):
+    """Scores s_b = t_b (rbar = 2, sqrt(d) = 2), unit sizes:
+    p = e^{t-2} / sum = [0.0900, 0.2447, 0.6652]."""
+    e = [math.exp(t - 2) for t in (0, 1, 2)]
+    p = [v / sum(e) for v in e]
+    assert abs(p[2] - 0.6652) < 1e-4
+    assert _sel(orc, [0, 1, 2], [1, 1, 1], 0.6) == [2]
+    assert _sel(orc, [0, 1, 2], [1, 1, 1], 0.7) == [1, 2]
+    assert _sel(orc, [0, 1, 2], [1, 1, 1], 0.9) == [1, 2]
+    assert _sel(orc, [0, 1, 2], [1, 1, 1], 0.95) == [0, 1, 2]
+    # doubling rbar doubles the temperature-free scores: p = e^{2t-4}/sum
+    assert _sel(orc, [0, 1, 2], [1, 1, 1], 0.85, rbar=4.0) == [2]
+
+
+def test_select_ties_lower_index_first(orc):
+    """Equal p: the lower cluster id is visited first."""
+    assert _sel(orc, [0, 0, 0], [2, 2, 1], 0.3) == [0]
+    assert _sel(orc, [0, 0, 0], [1, 2, 2], 0.3) == [1]
+
+
+def test_select_empty_clusters(orc):
+    assert _sel(orc, [5, 0, 0], [0, 1, 1], 1.0) == [1, 2]
+    assert _sel(orc, [0, 0], [1, 1], 1.0, qcount=0) == []
+
+
+def test_select_invariants(orc):
+    """top_p = 1 keeps every non-empty key cluster; the kept set grows with
+    top_p; one key cluster is always kept."""
+    rng = np.random.default_rng(0)
+    kq, kk, d = 20, 60, 16
+    qc = rng.standard_normal((kq, d)).astype(np.float32)
+    qc /= np.linalg.norm(qc, axis=1, keepdims=True)
+    kc = rng.standard_normal((kk, d)).astype(np.float32)
+    qn = rng.uniform(1, 8, kq).astype(np.float32)
+    qcnt = rng.integers(0, 30, kq).astype(np.int32)
+    kcnt = rng.integers(0, 30, kk).astype(np.int32)
+    prev = None
+    for p in [0.1, 0.5, 0.8, 0.9, 0.99, 1.0]:
+        s, c = orc.select(qc, qn, qcnt, kc, kcnt, p)
+        sets = [set(s[a, :c[a]].tolist()) for a in range(kq)]
+        for a in range(kq):
+            assert all(kcnt[b] > 0 for b in sets[a])
+            assert (len(sets[a]) == 0) == (qcnt[a] == 0)
+            if prev is not None:
+                assert prev[a] <= sets[a]
+        prev = sets
+    for a in range(kq):
+        if qcnt[a]:
+            assert prev[a] == {b for b in range(kk) if kcnt[b] > 0}
+    s, c = orc.select(qc, qn, qcnt, kc[:1], np.array([5], np.int32), 0.5)
+    assert all(c[a] == (1 if qcnt[a] else 0) for a in range(kq))
+
+
+# ---------------------------------------------------------------- attention
+def _np_attention(q, k, v):
+    s = (q.astype(np.float64) @ k.astype(np.float64).T) / math.sqrt(q.shape[1])
+    s -= s.max(1, keepdims=True)
+    e = np.exp(s)
+    return (e @ v.astype(np.float64)) / e.sum(1, keepdims=True)
+
+
+def test_attention_select_all_is_dense(orc):
+    """Algorithm 3: with every key cluster selected (or F set) the sparse
+    attention equals dense softmax attention (textbook definition in numpy)."""
+    rng = np.random.default_rng(1)
+    n, d = 300, 32
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    ref = _np_attention(q, k, v)
+    rows = np.arange(n)
+    out = orc.attention_rows(q, k, v, None, None, 0, None, None, 1, rows)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    qa = rng.integers(0, 5, n)
+    ka = rng.integers(0, 7, n)
+    sel = np.tile(np.arange(7, dtype=np.int32), (5, 1))
+    out2 = orc.attention_rows(q, k, v, qa, ka, 7, sel, np.full(5, 7, np.int32), 0, rows)
+    np.testing.assert_allclose(out2, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_subset_is_attention_over_subset(orc):
+    """Algorithm 3 lines 8-9: attention over K* = K[Index], V* = V[Index]."""
+    rng = np.random.default_rng(2)
+    n, d, kq, kk = 400, 16, 6, 9
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    qa = rng.integers(0, kq, n).astype(np.int32)
+    ka = rng.integers(0, kk, n).astype(np.int32)
+    sel = np.full((kq, kk), -1, np.int32)
+    cnt = np.zeros(kq, np.int32)
+    for a in range(kq):
+        s = np.sort(rng.choice(kk, rng.integers(1, kk + 1), replace=False))
+        sel[a, :len(s)] = s
+        cnt[a] = len(s)
+    rows = np.arange(0, n, 7)
+    out = orc.attention_rows(q, k, v, qa, ka, kk, sel, cnt, 0, rows)
+    for r, i in enumerate(rows):
+        keys = np.isin(ka, sel[qa[i], :cnt[qa[i]]])
+        np.testing.assert_allclose(out[r], _np_attention(q[i:i + 1], k[keys], v[keys])[0], rtol=1e-12,
+                                   atol=1e-12)
+
+
+def test_attention_single_key(orc):
+    rng = np.random.default_rng(3)
+    n, d = 50, 8
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    ka = np.arange(n, dtype=np.int32)
+    qa = np.zeros(n, np.int32)
+    sel = np.array([[17]], np.int32)
+    out = orc.attention_rows(q, k, v, qa, ka, n, sel, np.array([1], np.int32), 0, np.arange(n))
+    np.testing.assert_array_equal(out, np.tile(v[17].astype(np.float64), (n, 1)))
+
+
+# --------------------------------------------------------------------- sort
+def test_cluster_sort_is_stable_argsort(orc):
+    rng = np.random.default_rng(5)
+    ids = rng.integers(0, 37, 5000).astype(np.int32)
+    ids[ids == 11] = 12  # an empty cluster
+    perm, off = orc.cluster_sort(ids, 37)
+    np.testing.assert_array_equal(perm, np.argsort(ids, kind="stable"))
+    np.testing.assert_array_equal(off, np.concatenate([[0], np.cumsum(np.bincount(ids, minlength=37))]))
+
+
+# --------------------------------------------------------- composed forward
+def test_forward_head_top_p_one_is_dense(orc):
+    """Algorithm 3 end to end: top_p = 1 selects every non-empty key cluster,
+    so each row's output is dense attention."""
+    w = W.small(W.WORKLOADS["gmm16-n2048-d64-f32"], 512)
+    h = W.head_inputs(w, 0)
+    spec = orc.HeadSpec(kq=8, kk=16, iters=4, top_p=1.0)
+    r = orc.forward_head(h.q, h.k, h.v, spec, rows=np.arange(0, 512, 5))
+    np.testing.assert_allclose(r.out_rows, _np_attention(h.q[::5], h.k, h.v), rtol=1e-10, atol=1e-12)
+    assert r.dense == 0
+
+
+def test_forward_head_dense_flag(orc):
+    """Algorithm 3 lines 3-4: F set (N_max reached) -> full attention."""
+    w = W.small(W.WORKLOADS["gmm16-n2048-d64-f32"], 400)
+    h = W.head_inputs(w, 0)
+    spec = orc.HeadSpec(kq=8, kk=16, iters=3, top_p=0.5, adaptive_k=True, tau_rule=orc.TAU_ABS,
+                        tau_value=0.0, nmax_k=16)
+    r = orc.forward_head(h.q, h.k, h.v, spec, rows=np.arange(0, 400, 9))
+    assert r.dense == 1
+    np.testing.assert_allclose(r.out_rows, _np_attention(h.q[::9], h.k, h.v), rtol=1e-10, atol=1e-12)
