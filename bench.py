@@ -1,0 +1,353 @@
+#!/usr/bin/env python
+"""Benchmark of the AdaCluster clustered sparse attention call (ac_forward).
+
+One step = one ac_forward call over the whole workload (Q clustering, K
+clustering, critical-cluster selection, cluster sort + gather, block-sparse
+attention) on the Wan-2.1-shaped workload: 40 heads x 75,600 tokens x d=128,
+bf16, 250 query / 500 key clusters, 10 k-means iterations, top-p 0.9.
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle on a
+bounded sample of the same workload instead.  Under torchrun every rank runs
+its own independent call (heads and calls share nothing), so scaling is weak
+and value = calls over all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from clustered_sparse_attention_head_b200 import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "wan21-n75600-h40-d128"
+METRIC = "clustered sparse-attn calls/s & achieved TFLOPS at 75.6K tokens vs dense attn"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.ORDER)
+    ap.add_argument("--top-p", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None, help="fewer heads (profiling captures only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def gen_inputs(w, heads=None):
+    """Seeded inputs, all heads (threads: numpy releases the GIL in bulk draws)."""
+    from concurrent.futures import ThreadPoolExecutor
+    hs = list(range(w.heads)) if heads is None else heads
+    with ThreadPoolExecutor(max_workers=min(16, len(hs))) as ex:
+        res = list(ex.map(lambda h: W.head_inputs(w, h), hs))
+    return res
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except Exception:
+            self.p.kill()
+            out = ""
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ cpu baseline
+def oracle_sample(w, hi, rows_sample: int):
+    """Time the oracle on one head: full Q and K clustering and selection, and
+    attention for `rows_sample` query rows; extrapolate to one whole call."""
+    import oracle
+    oracle.build()
+    spec = oracle.HeadSpec(kq=w.kq, kk=w.kk, iters=w.iters, top_p=w.top_p, adaptive_q=w.adaptive_q,
+                           adaptive_k=w.adaptive_k, tau_rule=w.tau_rule, tau_value=w.tau_value, nmax_q=w.nmax_q,
+                           nmax_k=w.nmax_k)
+    t0 = time.perf_counter()
+    rq, qmn = oracle.cluster_q(hi.q, spec)
+    rk = oracle.cluster_k(hi.k, spec)
+    dense = int(rq.dense or rk.dense)
+    if dense:
+        sel, cnt = np.zeros((rq.nclusters, max(rk.nclusters, 1)), np.int32), np.zeros(rq.nclusters, np.int32)
+    else:
+        sel, cnt = oracle.select(rq.cent, qmn, rq.count, rk.cent, rk.count, spec.top_p)
+    t1 = time.perf_counter()
+    rows = np.linspace(0, w.n - 1, rows_sample).astype(np.int32)
+    oracle.attention_rows(hi.q, hi.k, hi.v, rq.assign, rk.assign, rk.nclusters, sel, cnt, dense, rows)
+    t2 = time.perf_counter()
+    per_call = w.heads * ((t1 - t0) + (t2 - t1) * w.n / rows_sample)
+    return per_call, t2 - t0
+
+
+def omp_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
+
+
+def cpu_baseline_obj(w, hi, rows_sample=128):
+    per_call, wall = oracle_sample(w, hi, rows_sample)
+    return {"value": 1.0 / per_call, "unit": "calls/s", "cores": omp_threads(), "kind": "oracle",
+            "sample": (f"head 0 of {w.heads}: Q and K clustering and selection in full, attention for "
+                       f"{rows_sample} of {w.n} query rows; extrapolated x{w.heads} heads and x{w.n}/{rows_sample} "
+                       f"rows ({wall:.1f} s of CPU time measured)")}
+
+
+# -------------------------------------------------------------- reference
+def run_reference(a, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    hi = W.head_inputs(w, 0)
+    rows = 64
+    times = []
+    for i in range(a.warmup + a.steps):
+        per_call, _ = oracle_sample(w, hi, rows)
+        if i >= a.warmup:
+            times.append(per_call)
+    per_call = statistics.mean(times)
+    v = 1.0 / per_call
+    line = {"metric": METRIC, "value": v, "unit": "calls/s", "n_gpus": 0, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": per_call * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "heads": w.heads, "n": w.n, "d": w.d, "kq": w.kq, "kk": w.kk,
+                       "iters": w.iters, "top_p": w.top_p},
+            "cpu_baseline": {"value": v, "unit": "calls/s", "cores": omp_threads(), "kind": "oracle",
+                             "sample": f"per step: head 0 clustered and selected in full, attention for {rows} of "
+                                       f"{w.n} rows, extrapolated to {w.heads} heads x {w.n} rows"},
+            "e2e": {"value": v, "unit": "calls/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- ours
+def main():
+    a = parse()
+    w = W.WORKLOADS[a.workload]
+    from dataclasses import replace
+    if a.top_p is not None:
+        w = replace(w, top_p=a.top_p)
+    if a.heads is not None:
+        w = replace(w, heads=a.heads)
+    if a.impl == "reference":
+        return run_reference(a, w)
+
+    rank, world, local = dist_env()
+    # the oracle sample needs no GPU; run it before CUDA starts
+    hs = gen_inputs(w)
+    cpu_base = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu_base = cpu_baseline_obj(w, hs[0])
+
+    import torch
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    from clustered_sparse_attention_head_b200 import _abi
+    from clustered_sparse_attention_head_b200.api import AdaCluster, Config
+
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q_h = torch.from_numpy(np.stack([h.q for h in hs])).to(tdt)
+    k_h = torch.from_numpy(np.stack([h.k for h in hs])).to(tdt)
+    v_h = torch.from_numpy(np.stack([h.v for h in hs])).to(tdt)
+    del hs
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    cfg = Config.from_workload(w)
+    cfg.flags = _abi.AC_FLAG_PROFILE
+    ac = AdaCluster(cfg, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # warm-up, then one call with statistics (pairs, dense heads)
+    for _ in range(max(a.warmup, 3) - 1):
+        ac.ac_forward(q, k, v, out=out)
+    _, st = ac.ac_forward(q, k, v, out=out, stats=True)
+    status = ac.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
+    ac.profile_read()
+
+    # timed region: inputs (774 MB per tensor) exceed the 126 MB L2, so no flush
+    sampler = ClockSampler(local)
+    barrier()
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        ac.ac_forward(q, k, v, out=out)
+    e1.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / a.steps
+    prof = ac.profile_read()
+    status = ac.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
+    t_max = ms
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    calls_per_s = world * 1000.0 / t_max
+    flops = 4.0 * w.d * st["pairs"]
+    tflops_call = flops / (ms * 1e-3) / 1e12
+    attn_ms = prof["ms_attn_kernel"]
+    tflops_attn = flops / (attn_ms * 1e-3) / 1e12
+
+    # end to end through the same call with host buffers (pinned), copies timed
+    e2e = None
+    if not a.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        op = torch.empty_like(qp).pin_memory()
+        for _ in range(2):
+            q.copy_(qp, non_blocking=True); k.copy_(kp, non_blocking=True); v.copy_(vp, non_blocking=True)
+            ac.ac_forward(q, k, v, out=out)
+            op.copy_(out, non_blocking=True)
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        n_e2e = max(1, min(a.steps, 5))
+        for _ in range(n_e2e):
+            q.copy_(qp, non_blocking=True); k.copy_(kp, non_blocking=True); v.copy_(vp, non_blocking=True)
+            ac.ac_forward(q, k, v, out=out)
+            op.copy_(out, non_blocking=True)
+        s1.record(stream)
+        barrier()
+        ms_e2e = s0.elapsed_time(s1) / n_e2e
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nb = q.numel() * q.element_size()
+        e2e = {"value": world * 1000.0 / ms_e2e, "unit": "calls/s", "h2d_bytes_per_step": 3 * nb,
+               "d2h_bytes_per_step": nb, "ms_per_step": ms_e2e}
+        ac.profile_read()
+
+    # dense comparator: torch SDPA at the same shape (40 heads x 75.6K x 128)
+    dense = None
+    if not a.no_dense and rank == 0:
+        import torch.nn.functional as F
+        qd, kd, vd = (t.unsqueeze(0) for t in (q, k, v))
+        for _ in range(2):
+            F.scaled_dot_product_attention(qd, kd, vd)
+        torch.cuda.synchronize(dev)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(3):
+            F.scaled_dot_product_attention(qd, kd, vd)
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dms = d0.elapsed_time(d1) / 3
+        dense = {"impl": "torch.nn.functional.scaled_dot_product_attention", "ms": dms,
+                 "tflops": w.dense_flops() / (dms * 1e-3) / 1e12, "speedup_of_clustered_call": dms / ms}
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    peak = peaks.get("bf16_tflops_sustained") or 1390.6
+    peak_src = "measured (MEASURED_PEAKS.json bf16_tflops_sustained)" if peaks else "fallback"
+    roof = {"kernel": "attn_kernel (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": tflops_attn,
+            "peak": peak, "unit": "TFLOP/s", "frac": tflops_attn / peak, "traffic": None,
+            "peak_source": peak_src, "ms_per_launch": attn_ms,
+            "flops_per_launch": flops, "flops_rule": "4 * d * computed (query, key) pairs"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": calls_per_s, "unit": "calls/s", "n_gpus": world, "steps": a.steps,
+                "warmup": max(a.warmup, 3), "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+                "config": {"workload": w.name, "heads": w.heads, "n": w.n, "d": w.d, "kq": w.kq, "kk": w.kk,
+                           "iters": w.iters, "top_p": w.top_p, "parallelism": f"dp{world} (independent calls)",
+                           "l2": "inputs larger than L2 (774 MB per tensor), no flush"},
+                "tflops_effective_call": tflops_call, "tflops_effective_attn": tflops_attn,
+                "pairs": st["pairs"], "density": st["pairs"] / (w.heads * float(w.n) ** 2),
+                "dense_heads": st["dense_heads"],
+                "stage_ms": {k2: prof[k2] for k2 in ("ms_cluster_q", "ms_cluster_k", "ms_select", "ms_prep",
+                                                     "ms_attn_kernel", "ms_total")},
+                "roofline": roof, "dense_attention": dense,
+                "cpu_baseline": cpu_base, "e2e": e2e,
+                "gpu_launches": int(prof["launches"]) if e2e is None else None, "clocks": clocks}
+        if line["gpu_launches"] is None:
+            line["gpu_launches"] = launches_per_call(ac, q, k, v, out) * a.steps
+        print(json.dumps(line), flush=True)
+    ac.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def launches_per_call(ac, q, k, v, out):
+    ac.profile_read()
+    ac.ac_forward(q, k, v, out=out)
+    return int(ac.profile_read()["launches"])
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,167 @@
+"""Python front end of the C ABI with the same call names (ac_cluster_q, ...).
+
+``AdaCluster`` owns one ``ac_ctx`` and a workspace tensor.  Each method passes
+torch CUDA tensors straight to the matching C call; outputs are allocated with
+torch (device memory is torch's, the work is the library's kernels).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _abi
+from ._abi import check, ptr, stream_ptr
+
+
+@dataclass
+class Config:
+    heads: int
+    n: int
+    d: int
+    dtype: str = "bf16"          # "bf16" | "f32"
+    kq: int = 100
+    kk: int = 200
+    iters: int = 10
+    adaptive_q: bool = False
+    adaptive_k: bool = False
+    tau_rule: int = _abi.AC_TAU_ABS
+    tau_value: float = 0.0
+    nmax_q: int = 0
+    nmax_k: int = 0
+    top_p: float = 0.9
+    flags: int = 0
+
+    def to_c(self) -> _abi.ac_config:
+        return _abi.ac_config(self.heads, self.n, self.d, _abi.AC_BF16 if self.dtype == "bf16" else _abi.AC_F32,
+                              self.kq, self.kk, self.iters, int(self.adaptive_q), int(self.adaptive_k),
+                              self.tau_rule, float(self.tau_value), self.nmax_q, self.nmax_k, float(self.top_p),
+                              self.flags)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    @staticmethod
+    def from_workload(w) -> "Config":
+        return Config(heads=w.heads, n=w.n, d=w.d, dtype=w.dtype, kq=w.kq, kk=w.kk, iters=w.iters,
+                      adaptive_q=w.adaptive_q, adaptive_k=w.adaptive_k, tau_rule=w.tau_rule,
+                      tau_value=w.tau_value, nmax_q=w.nmax_q, nmax_k=w.nmax_k, top_p=w.top_p)
+
+
+class AdaCluster:
+    def __init__(self, cfg: Config, device="cuda", workspace: torch.Tensor | None = None):
+        self.cfg = cfg
+        self.lib = _abi.load()
+        self._ctx = ctypes.c_void_p()
+        c = cfg.to_c()
+        check("ac_create", self.lib.ac_create(ctypes.byref(c), ctypes.byref(self._ctx)))
+        kq, kk = ctypes.c_int(), ctypes.c_int()
+        check("ac_capacities", self.lib.ac_capacities(self._ctx, ctypes.byref(kq), ctypes.byref(kk)))
+        self.kq_cap, self.kk_cap = kq.value, kk.value
+        nb = ctypes.c_size_t()
+        check("ac_workspace_size", self.lib.ac_workspace_size(self._ctx, ctypes.byref(nb)))
+        self.ws_bytes = nb.value
+        self.device = torch.device(device)
+        self.ws = workspace if workspace is not None else torch.empty(self.ws_bytes + 256, dtype=torch.uint8,
+                                                                      device=self.device)
+        off = (-self.ws.data_ptr()) % 256
+        self._ws = self.ws[off:off + self.ws_bytes]
+
+    def close(self):
+        if self._ctx:
+            self.lib.ac_destroy(self._ctx)
+            self._ctx = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # --------------------------------------------------------------- helpers
+    def _i32(self, *shape):
+        return torch.empty(*shape, dtype=torch.int32, device=self.device)
+
+    def _f32(self, *shape):
+        return torch.empty(*shape, dtype=torch.float32, device=self.device)
+
+    def _args_ws(self):
+        return ptr(self._ws), ctypes.c_size_t(self.ws_bytes)
+
+    def profile_read(self) -> dict:
+        p = _abi.ac_profile()
+        check("ac_profile_read", self.lib.ac_profile_read(self._ctx, ctypes.byref(p)))
+        return {f: getattr(p, f) for f, _ in _abi.ac_profile._fields_}
+
+    def get_status(self, stream=None) -> int:
+        return self.lib.ac_get_status(self._ctx, stream_ptr(stream))
+
+    # ------------------------------------------------------------ the calls
+    def ac_cluster_q(self, q, init_cent=None, stream=None):
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        out = dict(assign=self._i32(H, N), cent=self._f32(H, self.kq_cap, D).zero_(),
+                   count=self._i32(H, self.kq_cap), mean_norm=self._f32(H, self.kq_cap), nclusters=self._i32(H),
+                   dense_flag=torch.empty(H, dtype=torch.uint8, device=self.device))
+        ws, nb = self._args_ws()
+        check("ac_cluster_q", self.lib.ac_cluster_q(
+            self._ctx, ptr(q), ptr(init_cent), ptr(out["assign"]), ptr(out["cent"]), ptr(out["count"]),
+            ptr(out["mean_norm"]), ptr(out["nclusters"]), ptr(out["dense_flag"]), ws, nb, stream_ptr(stream)))
+        return out
+
+    def ac_cluster_k(self, k, init_cent=None, stream=None):
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        out = dict(assign=self._i32(H, N), cent=self._f32(H, self.kk_cap, D).zero_(),
+                   count=self._i32(H, self.kk_cap), nclusters=self._i32(H),
+                   dense_flag=torch.empty(H, dtype=torch.uint8, device=self.device))
+        ws, nb = self._args_ws()
+        check("ac_cluster_k", self.lib.ac_cluster_k(
+            self._ctx, ptr(k), ptr(init_cent), ptr(out["assign"]), ptr(out["cent"]), ptr(out["count"]),
+            ptr(out["nclusters"]), ptr(out["dense_flag"]), ws, nb, stream_ptr(stream)))
+        return out
+
+    def ac_select(self, q_cent, q_mean_norm, q_count, k_cent, k_count, nq=None, nk=None, dense_flag=None,
+                  stream=None):
+        H = self.cfg.heads
+        sel = torch.full((H, self.kq_cap, self.kk_cap), -1, dtype=torch.int32, device=self.device)
+        cnt = self._i32(H, self.kq_cap)
+        ws, nb = self._args_ws()
+        check("ac_select", self.lib.ac_select(
+            self._ctx, ptr(q_cent), ptr(q_mean_norm), ptr(q_count), ptr(k_cent), ptr(k_count), ptr(nq), ptr(nk),
+            ptr(dense_flag), ptr(sel), ptr(cnt), ws, nb, stream_ptr(stream)))
+        return sel, cnt
+
+    def ac_cluster_sort(self, assign, cap, ncl=None, stream=None):
+        H, N = self.cfg.heads, self.cfg.n
+        perm = self._i32(H, N)
+        off = self._i32(H, cap + 1)
+        ws, nb = self._args_ws()
+        check("ac_cluster_sort", self.lib.ac_cluster_sort(self._ctx, ptr(assign), cap, ptr(ncl), ptr(perm),
+                                                          ptr(off), ws, nb, stream_ptr(stream)))
+        return perm, off
+
+    def ac_sparse_attn(self, q, k, v, q_assign, k_assign, sel_idx, sel_cnt, nq=None, nk=None, dense_flag=None,
+                       lse=False, out=None, stream=None):
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        if out is None:
+            out = torch.empty(H, N, D, dtype=self.cfg.torch_dtype, device=self.device)
+        lse_t = self._f32(H, N) if lse else None
+        ws, nb = self._args_ws()
+        check("ac_sparse_attn", self.lib.ac_sparse_attn(
+            self._ctx, ptr(q), ptr(k), ptr(v), ptr(q_assign), ptr(k_assign), ptr(sel_idx), ptr(sel_cnt), ptr(nq),
+            ptr(nk), ptr(dense_flag), ptr(out), ptr(lse_t), ws, nb, stream_ptr(stream)))
+        return (out, lse_t) if lse else out
+
+    def ac_forward(self, q, k, v, q_cent_io=None, k_cent_io=None, out=None, stats=False, stream=None):
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        if out is None:
+            out = torch.empty(H, N, D, dtype=self.cfg.torch_dtype, device=self.device)
+        st = _abi.ac_stats() if stats else None
+        ws, nb = self._args_ws()
+        check("ac_forward", self.lib.ac_forward(
+            self._ctx, ptr(q), ptr(k), ptr(v), ptr(q_cent_io), ptr(k_cent_io), ptr(out),
+            ctypes.byref(st) if st is not None else None, ws, nb, stream_ptr(stream)))
+        if stats:
+            return out, {f: getattr(st, f) for f, _ in _abi.ac_stats._fields_}
+        return out

@@ -1,0 +1,568 @@
+// C ABI of libadacluster.so: argument checks, workspace layout and the host
+// orchestration of AdaCluster's Algorithm 3 ("AdaCluster: Adaptive Query-Key
+// Clustering for Sparse Attention in Video Generation", §3.3).  All compute
+// runs in the kernels of this directory; this file only launches them.
+#include <atomic>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "adacluster.h"
+#include "ac_kernels.cuh"
+#include "ac_multistage.cuh"
+
+using namespace ac;
+
+void ac_or_flags(int H, const uint8_t *a, uint8_t *b, cudaStream_t st);
+
+static std::atomic<long long> g_launches{0};
+namespace ac {
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+long long launches_total() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace ac
+
+constexpr int PROF_RING = 256;
+constexpr int PROF_EV = 6;
+
+struct ac_ctx {
+    ac_config cfg;
+    int kq_cap, kk_cap, cap_max;
+    int elt;
+    int *d_status;     // [8] device status words
+    int32_t *d_info;   // [8] device -> host control summary
+    int32_t *h_info;   // [8] pinned host mirror
+    int num_sms;
+    void *encode_fn;
+    cudaEvent_t ev[8];
+    cudaEvent_t *prof;     // [PROF_RING][PROF_EV]
+    long long prof_n;      // calls recorded since the last read
+    long long launch_base;
+};
+
+// ------------------------------------------------------------ workspace
+namespace {
+struct Bump {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        size_t o = off;
+        off += (bytes + 255) & ~(size_t)255;
+        return o;
+    }
+};
+
+struct Ws {
+    // clustering scratch
+    size_t norm, U0, U1, passign, dist, rank, hist, cnt, off, perm, amb, ambc, cn2, cmax, seg, ms;
+    // ac_forward internals
+    size_t qa, ka, qc, kc, qcount, kcount, qmn, nq, nk, dq, dk, sel, selc;
+    // attention
+    size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
+    size_t total;
+};
+
+Ws layout(const ac_ctx *c) {
+    const ac_config &g = c->cfg;
+    const size_t H = g.heads, N = g.n, D = g.d;
+    const size_t HN = H * N;
+    const size_t capm = c->cap_max;
+    Bump b;
+    Ws w;
+    w.norm = b.take(HN * 8);
+    w.U0 = b.take(HN * 4);
+    w.U1 = b.take(HN * 4);
+    w.passign = b.take(HN * 4);
+    w.dist = b.take(HN * 8);
+    w.rank = b.take(HN * 4);
+    w.hist = b.take(sort_hist_elems((int)H, (int)N, (int)capm) * 4);
+    w.cnt = b.take(H * capm * 4);
+    w.off = b.take(H * (capm + 1) * 4);
+    w.perm = b.take(HN * 4);
+    w.amb = b.take(HN * 4);
+    w.ambc = b.take(H * 4);
+    w.cn2 = b.take(H * capm * 4);
+    w.cmax = b.take(H * 4);
+    w.seg = b.take(H * sizeof(HeadSeg));
+    w.ms = b.take(H * sizeof(MsHead));
+    w.qa = b.take(HN * 4);
+    w.ka = b.take(HN * 4);
+    w.qc = b.take(H * c->kq_cap * D * 4);
+    w.kc = b.take(H * c->kk_cap * D * 4);
+    w.qcount = b.take(H * c->kq_cap * 4);
+    w.kcount = b.take(H * c->kk_cap * 4);
+    w.qmn = b.take(H * c->kq_cap * 4);
+    w.nq = b.take(H * 4);
+    w.nk = b.take(H * 4);
+    w.dq = b.take(H);
+    w.dk = b.take(H);
+    w.sel = b.take(H * (size_t)c->kq_cap * c->kk_cap * 4);
+    w.selc = b.take(H * c->kq_cap * 4);
+    w.qperm = b.take(HN * 4);
+    w.kperm = b.take(HN * 4);
+    w.qoff = b.take(H * (c->kq_cap + 1) * 4);
+    w.koff = b.take(H * (c->kk_cap + 1) * 4);
+    w.qg = b.take(HN * D * c->elt);
+    w.kg = b.take(HN * D * c->elt);
+    w.vg = b.take(HN * D * c->elt);
+    w.items = b.take((size_t)attn_max_items((int)H, (int)N, c->kq_cap) * sizeof(AttnItem));
+    w.nitems = b.take(16);
+    w.pairs = b.take(16);
+    w.cnt2 = b.take(H * capm * 4);
+    w.segq = b.take(H * sizeof(HeadSeg));
+    w.segk = b.take(H * sizeof(HeadSeg));
+    w.total = b.off;
+    return w;
+}
+
+template <typename P> P *at(void *ws, size_t off) { return reinterpret_cast<P *>(static_cast<char *>(ws) + off); }
+
+#define AC_CUDA(call)                                                                    \
+    do {                                                                                 \
+        cudaError_t e_ = (call);                                                         \
+        if (e_ != cudaSuccess) {                                                         \
+            fprintf(stderr, "adacluster: %s failed: %s\n", #call, cudaGetErrorString(e_)); \
+            return AC_ERR_CUDA;                                                          \
+        }                                                                                \
+    } while (0)
+
+ac_status launch_check() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        fprintf(stderr, "adacluster: kernel launch failed: %s\n", cudaGetErrorString(e));
+        return AC_ERR_CUDA;
+    }
+    return AC_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ac_status check_ws(const ac_ctx *c, void *ws, size_t ws_bytes) {
+    if (!ws) return AC_ERR_WORKSPACE;
+    if (ws_bytes < layout(c).total) return AC_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return AC_ERR_WORKSPACE;
+    return AC_OK;
+}
+
+// ------------------------------------------------------ clustering driver
+// One k-means run per head (fixed count) or Algorithm 1 (adaptive), all heads
+// batched in every launch.
+ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int32_t *assign, float *cent,
+                      int32_t *count, float *mean_norm, int32_t *ncl, uint8_t *flag, void *ws, cudaStream_t st,
+                      int *max_stages) {
+    const ac_config &g = c->cfg;
+    const int H = g.heads, N = g.n, D = g.d;
+    const int dt = g.dtype == AC_BF16 ? DT_BF16 : DT_F32;
+    const bool q = (mode == MODE_SPHERE);
+    const int cap = q ? c->kq_cap : c->kk_cap;
+    const int k = q ? g.kq : g.kk;
+    const bool adaptive = q ? g.adaptive_q : g.adaptive_k;
+    const int nmax = q ? g.nmax_q : g.nmax_k;
+    Ws w = layout(c);
+    double *norm = at<double>(ws, w.norm);
+    HeadSeg *seg = at<HeadSeg>(ws, w.seg);
+    int32_t *perm = at<int32_t>(ws, w.perm), *off = at<int32_t>(ws, w.off);
+    int32_t *rank = at<int32_t>(ws, w.rank), *hist = at<int32_t>(ws, w.hist);
+    int32_t *cnt = at<int32_t>(ws, w.cnt);
+    float *cn2 = at<float>(ws, w.cn2), *cmax = at<float>(ws, w.cmax);
+    int32_t *amb = at<int32_t>(ws, w.amb), *ambc = at<int32_t>(ws, w.ambc);
+    int *status = c->d_status;
+
+    k_row_norm(x, dt, H, N, D, norm, (g.flags & AC_FLAG_CHECK_FINITE) ? 1 : 0, status, st);
+    if (!adaptive) {
+        k_seg_uniform(H, N, k, seg, ncl, flag, st);
+        if (init) AC_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * H * cap * D, cudaMemcpyDeviceToDevice, st));
+        else k_init_cent(x, dt, H, N, D, nullptr, norm, seg, k, mode, cent, cap, st);
+        for (int it = 0; it < g.iters; it++) {
+            k_assign(x, dt, H, N, D, nullptr, seg, N, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+            k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, cnt, off, perm, status, st);
+            k_update(x, dt, H, N, D, seg, k, perm, off, cap, norm, mode, cent, st);
+        }
+        k_assign(x, dt, H, N, D, nullptr, seg, N, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+        k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
+        if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
+        if (max_stages) *max_stages = 1;
+        return launch_check();
+    }
+    // ---- Algorithm 1
+    int32_t *U = at<int32_t>(ws, w.U0), *Un = at<int32_t>(ws, w.U1);
+    int32_t *pa = at<int32_t>(ws, w.passign);
+    double *dist = at<double>(ws, w.dist);
+    MsHead *ms = at<MsHead>(ws, w.ms);
+    k_ms_init(H, N, ms, U, st);
+    int stages = 0;
+    for (int t = 0;; t++) {
+        k_ms_control(H, N, k, nmax, cap, ms, seg, c->d_info, status, st);
+        AC_CUDA(cudaMemcpyAsync(c->h_info, c->d_info, 8 * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+        AC_CUDA(cudaStreamSynchronize(st));
+        if (c->h_info[4]) return AC_ERR_CAPACITY;
+        if (c->h_info[0] == 0) break;
+        const int mnu = c->h_info[1], mmt = c->h_info[2];
+        stages = t + 1;
+        k_init_cent(x, dt, H, N, D, U, norm, seg, mmt, mode, cent, cap, st);
+        for (int it = 0; it < g.iters; it++) {
+            k_assign(x, dt, H, N, D, U, seg, mnu, cent, cap, cn2, cmax, norm, mode, pa, amb, ambc, st);
+            k_sort(pa, U, seg, H, N, mnu, cap, rank, hist, cnt, off, perm, status, st);
+            k_update(x, dt, H, N, D, seg, mmt, perm, off, cap, norm, mode, cent, st);
+        }
+        k_assign(x, dt, H, N, D, U, seg, mnu, cent, cap, cn2, cmax, norm, mode, pa, amb, ambc, st);
+        k_dist(x, dt, H, N, D, U, seg, mnu, cent, cap, norm, mode, pa, dist, st);
+        if (t == 0) {
+            if (g.tau_rule == AC_TAU_MEDIAN_RADIUS_X)
+                k_sort(pa, U, seg, H, N, mnu, cap, rank, hist, cnt, off, perm, status, st);
+            k_ms_tau(H, N, (int)g.tau_rule, (double)g.tau_value, seg, dist, perm, off, cap, mmt, ms, st);
+        }
+        k_ms_remove(H, N, seg, dist, U, Un, ms, st);
+        int32_t *tmp = U;
+        U = Un;
+        Un = tmp;
+        AC_CUDA(cudaGetLastError());
+    }
+    k_ms_final(H, N, ms, seg, ncl, flag, c->d_info, st);
+    k_assign(x, dt, H, N, D, nullptr, seg, N, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+    k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
+    if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
+    if (max_stages) *max_stages = stages;
+    return launch_check();
+}
+
+ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v, const int32_t *qa,
+                         const int32_t *ka, const int32_t *sel, const int32_t *selc, const int32_t *nq,
+                         const int32_t *nk, const uint8_t *dense, void *out, float *lse, void *ws, cudaStream_t st,
+                         int64_t *pairs_dev, cudaEvent_t *ev_kernel = nullptr) {
+    const ac_config &g = c->cfg;
+    const int H = g.heads, N = g.n, D = g.d;
+    Ws w = layout(c);
+    HeadSeg *sq = at<HeadSeg>(ws, w.segq), *sk = at<HeadSeg>(ws, w.segk);
+    int32_t *rank = at<int32_t>(ws, w.rank), *hist = at<int32_t>(ws, w.hist), *cnt = at<int32_t>(ws, w.cnt2);
+    int32_t *qperm = at<int32_t>(ws, w.qperm), *kperm = at<int32_t>(ws, w.kperm);
+    int32_t *qoff = at<int32_t>(ws, w.qoff), *koff = at<int32_t>(ws, w.koff);
+    void *qg = at<void>(ws, w.qg), *kg = at<void>(ws, w.kg), *vg = at<void>(ws, w.vg);
+    AttnItem *items = at<AttnItem>(ws, w.items);
+    int32_t *nitems = at<int32_t>(ws, w.nitems);
+    k_seg_from_counts(H, N, nq, g.kq, sq, st);
+    k_seg_from_counts(H, N, nk, g.kk, sk, st);
+    k_sort(qa, nullptr, sq, H, N, N, c->kq_cap, rank, hist, cnt, qoff, qperm, c->d_status, st);
+    k_sort(ka, nullptr, sk, H, N, N, c->kk_cap, rank, hist, cnt, koff, kperm, c->d_status, st);
+    const int rb = D * c->elt;
+    k_gather_rows(q, qg, qperm, H, N, rb, st);
+    k_gather_rows(k, kg, kperm, H, N, rb, st);
+    k_gather_rows(v, vg, kperm, H, N, rb, st);
+    k_build_items(H, N, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items, nitems, pairs_dev, st);
+    if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
+    int rc = k_attention(g.dtype == AC_BF16 ? DT_BF16 : DT_F32, D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel,
+                         c->kq_cap, selc, items, nitems, attn_max_items(H, N, c->kq_cap), out, lse, c->d_status,
+                         c->num_sms, c->encode_fn, st);
+    if (rc != 0) return AC_ERR_CUDA;
+    if (ev_kernel) cudaEventRecord(ev_kernel[1], st);
+    return launch_check();
+}
+
+ac_status validate(const ac_config *g) {
+    if (!g) return AC_ERR_INVALID_ARG;
+    if (g->heads < 1 || g->n < 1 || g->iters < 0) return AC_ERR_INVALID_ARG;
+    if (g->d != 64 && g->d != 128) return AC_ERR_UNSUPPORTED;
+    if (g->dtype != AC_F32 && g->dtype != AC_BF16) return AC_ERR_INVALID_ARG;
+    if (g->kq < 1 || g->kk < 1 || g->kq > g->n || g->kk > g->n) return AC_ERR_INVALID_ARG;
+    if (!(g->top_p > 0.0)) return AC_ERR_INVALID_ARG;
+    if ((long long)g->heads * g->n > 0x7fffffffLL / 2) return AC_ERR_UNSUPPORTED;
+    if (g->adaptive_q && g->nmax_q < 1) return AC_ERR_INVALID_ARG;
+    if (g->adaptive_k && g->nmax_k < 1) return AC_ERR_INVALID_ARG;
+    if ((g->adaptive_q || g->adaptive_k) &&
+        (g->tau_rule < AC_TAU_ABS || g->tau_rule > AC_TAU_MEDIAN_RADIUS_X || !(g->tau_value >= 0.0)))
+        return AC_ERR_INVALID_ARG;
+    return AC_OK;
+}
+}  // namespace
+
+// ------------------------------------------------------------------ ABI
+extern "C" {
+
+const char *ac_status_string(ac_status s) {
+    switch (s) {
+    case AC_OK: return "ok";
+    case AC_ERR_INVALID_ARG: return "invalid argument";
+    case AC_ERR_UNSUPPORTED: return "unsupported configuration";
+    case AC_ERR_CUDA: return "CUDA error";
+    case AC_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case AC_ERR_TIMEOUT: return "device wait timed out";
+    case AC_ERR_NONFINITE: return "non-finite input";
+    case AC_ERR_CAPACITY: return "adaptive clustering exceeded its capacity";
+    }
+    return "unknown status";
+}
+
+ac_status ac_create(const ac_config *cfg, ac_ctx **out) {
+    if (!out) return AC_ERR_INVALID_ARG;
+    *out = nullptr;
+    ac_status v = validate(cfg);
+    if (v != AC_OK) return v;
+    ac_ctx *c = (ac_ctx *)calloc(1, sizeof(ac_ctx));
+    if (!c) return AC_ERR_INVALID_ARG;
+    c->cfg = *cfg;
+    c->kq_cap = cfg->adaptive_q ? cfg->nmax_q + cfg->kq : cfg->kq;
+    c->kk_cap = cfg->adaptive_k ? cfg->nmax_k + cfg->kk : cfg->kk;
+    c->cap_max = c->kq_cap > c->kk_cap ? c->kq_cap : c->kk_cap;
+    c->elt = cfg->dtype == AC_BF16 ? 2 : 4;
+    if (c->cap_max > 8192) {
+        free(c);
+        return AC_ERR_UNSUPPORTED;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaMalloc(&c->d_status, 8 * sizeof(int)) != cudaSuccess) {
+        free(c);
+        return AC_ERR_CUDA;
+    }
+    if (cudaMalloc(&c->d_info, 8 * sizeof(int32_t)) != cudaSuccess ||
+        cudaMallocHost(&c->h_info, 8 * sizeof(int32_t)) != cudaSuccess ||
+        cudaMemset(c->d_status, 0, 8 * sizeof(int)) != cudaSuccess) {
+        ac_destroy(c);
+        return AC_ERR_CUDA;
+    }
+    for (int i = 0; i < 8; i++)
+        if (cudaEventCreate(&c->ev[i]) != cudaSuccess) {
+            ac_destroy(c);
+            return AC_ERR_CUDA;
+        }
+    c->prof = (cudaEvent_t *)calloc((size_t)PROF_RING * PROF_EV, sizeof(cudaEvent_t));
+    if (!c->prof) {
+        ac_destroy(c);
+        return AC_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < PROF_RING * PROF_EV; i++)
+        if (cudaEventCreate(&c->prof[i]) != cudaSuccess) {
+            ac_destroy(c);
+            return AC_ERR_CUDA;
+        }
+    c->launch_base = launches_total();
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &c->encode_fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || !c->encode_fn) {
+        ac_destroy(c);
+        return AC_ERR_CUDA;
+    }
+    *out = c;
+    return AC_OK;
+}
+
+void ac_destroy(ac_ctx *c) {
+    if (!c) return;
+    if (c->d_status) cudaFree(c->d_status);
+    if (c->d_info) cudaFree(c->d_info);
+    if (c->h_info) cudaFreeHost(c->h_info);
+    for (int i = 0; i < 8; i++)
+        if (c->ev[i]) cudaEventDestroy(c->ev[i]);
+    if (c->prof) {
+        for (int i = 0; i < PROF_RING * PROF_EV; i++)
+            if (c->prof[i]) cudaEventDestroy(c->prof[i]);
+        free(c->prof);
+    }
+    free(c);
+}
+
+ac_status ac_profile_read(ac_ctx *c, ac_profile *out) {
+    if (!c || !out) return AC_ERR_INVALID_ARG;
+    memset(out, 0, sizeof(*out));
+    long long n = c->prof_n < PROF_RING ? c->prof_n : PROF_RING;
+    long long first = c->prof_n - n;
+    double acc[6] = {0, 0, 0, 0, 0, 0};
+    for (long long i = first; i < c->prof_n; i++) {
+        cudaEvent_t *e = c->prof + (size_t)(i % PROF_RING) * PROF_EV;
+        AC_CUDA(cudaEventSynchronize(e[5]));
+        float ms;
+        const int a[6][2] = {{0, 1}, {1, 2}, {2, 3}, {3, 4}, {4, 5}, {0, 5}};
+        for (int j = 0; j < 6; j++) {
+            AC_CUDA(cudaEventElapsedTime(&ms, e[a[j][0]], e[a[j][1]]));
+            acc[j] += ms;
+        }
+    }
+    out->calls = (int)n;
+    if (n > 0) {
+        out->ms_cluster_q = acc[0] / n;
+        out->ms_cluster_k = acc[1] / n;
+        out->ms_select = acc[2] / n;
+        out->ms_prep = acc[3] / n;
+        out->ms_attn_kernel = acc[4] / n;
+        out->ms_total = acc[5] / n;
+    }
+    long long now = launches_total();
+    out->launches = now - c->launch_base;
+    c->launch_base = now;
+    c->prof_n = 0;
+    return AC_OK;
+}
+
+ac_status ac_capacities(const ac_ctx *c, int *kq_cap, int *kk_cap) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    if (kq_cap) *kq_cap = c->kq_cap;
+    if (kk_cap) *kk_cap = c->kk_cap;
+    return AC_OK;
+}
+
+ac_status ac_workspace_size(const ac_ctx *c, size_t *bytes) {
+    if (!c || !bytes) return AC_ERR_INVALID_ARG;
+    *bytes = layout(c).total;
+    return AC_OK;
+}
+
+ac_status ac_cluster_q(ac_ctx *c, const void *q, const float *init_cent, int32_t *assign, float *cent,
+                       int32_t *count, float *mean_norm, int32_t *nclusters, uint8_t *dense_flag, void *ws,
+                       size_t ws_bytes, void *stream) {
+    if (!c || !q || !assign || !cent || !count || !mean_norm || !nclusters || !dense_flag) return AC_ERR_INVALID_ARG;
+    if (!aligned16(q) || (init_cent && c->cfg.adaptive_q)) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    return run_cluster(c, MODE_SPHERE, q, init_cent, assign, cent, count, mean_norm, nclusters, dense_flag, ws,
+                       (cudaStream_t)stream, nullptr);
+}
+
+ac_status ac_cluster_k(ac_ctx *c, const void *k, const float *init_cent, int32_t *assign, float *cent,
+                       int32_t *count, int32_t *nclusters, uint8_t *dense_flag, void *ws, size_t ws_bytes,
+                       void *stream) {
+    if (!c || !k || !assign || !cent || !count || !nclusters || !dense_flag) return AC_ERR_INVALID_ARG;
+    if (!aligned16(k) || (init_cent && c->cfg.adaptive_k)) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    return run_cluster(c, MODE_EUCLID, k, init_cent, assign, cent, count, nullptr, nclusters, dense_flag, ws,
+                       (cudaStream_t)stream, nullptr);
+}
+
+ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, const int32_t *q_count,
+                    const float *k_cent, const int32_t *k_count, const int32_t *nq, const int32_t *nk,
+                    const uint8_t *dense_flag, int32_t *sel_idx, int32_t *sel_cnt, void *ws, size_t ws_bytes,
+                    void *stream) {
+    if (!c || !q_cent || !q_mean_norm || !q_count || !k_cent || !k_count || !sel_idx || !sel_cnt)
+        return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    const ac_config &g = c->cfg;
+    k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, c->kk_cap, nq, nk, g.kq, g.kk,
+             dense_flag, g.top_p, sel_idx, sel_cnt, (cudaStream_t)stream);
+    return launch_check();
+}
+
+ac_status ac_cluster_sort(ac_ctx *c, const int32_t *assign, int cap, const int32_t *ncl, int32_t *perm,
+                          int32_t *offsets, void *ws, size_t ws_bytes, void *stream) {
+    if (!c || !assign || !perm || !offsets || cap < 1 || cap > c->cap_max) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    const ac_config &g = c->cfg;
+    Ws w = layout(c);
+    cudaStream_t st = (cudaStream_t)stream;
+    HeadSeg *seg = at<HeadSeg>(ws, w.seg);
+    k_seg_from_counts(g.heads, g.n, ncl, cap, seg, st);
+    k_sort(assign, nullptr, seg, g.heads, g.n, g.n, cap, at<int32_t>(ws, w.rank), at<int32_t>(ws, w.hist),
+           at<int32_t>(ws, w.cnt), offsets, perm, c->d_status, st);
+    return launch_check();
+}
+
+ac_status ac_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v, const int32_t *q_assign,
+                         const int32_t *k_assign, const int32_t *sel_idx, const int32_t *sel_cnt,
+                         const int32_t *nq, const int32_t *nk, const uint8_t *dense_flag, void *out, float *lse,
+                         void *ws, size_t ws_bytes, void *stream) {
+    if (!c || !q || !k || !v || !q_assign || !k_assign || !sel_idx || !sel_cnt || !out) return AC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    Ws w = layout(c);
+    return do_sparse_attn(c, q, k, v, q_assign, k_assign, sel_idx, sel_cnt, nq, nk, dense_flag, out, lse, ws,
+                          (cudaStream_t)stream, at<int64_t>(ws, w.pairs));
+}
+
+ac_status ac_forward(ac_ctx *c, const void *q, const void *k, const void *v, float *q_cent_io, float *k_cent_io,
+                     void *out, ac_stats *stats, void *ws, size_t ws_bytes, void *stream) {
+    if (!c || !q || !k || !v || !out) return AC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return AC_ERR_INVALID_ARG;
+    const ac_config &g = c->cfg;
+    const bool warm = (g.flags & AC_FLAG_WARM_START) != 0;
+    if (warm && ((q_cent_io && g.adaptive_q) || (k_cent_io && g.adaptive_k))) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    Ws w = layout(c);
+    float *qc = q_cent_io ? q_cent_io : at<float>(ws, w.qc);
+    float *kc = k_cent_io ? k_cent_io : at<float>(ws, w.kc);
+    int32_t *qa = at<int32_t>(ws, w.qa), *ka = at<int32_t>(ws, w.ka);
+    int32_t *qn = at<int32_t>(ws, w.qcount), *kn = at<int32_t>(ws, w.kcount);
+    float *qmn = at<float>(ws, w.qmn);
+    int32_t *nq = at<int32_t>(ws, w.nq), *nk = at<int32_t>(ws, w.nk);
+    uint8_t *dq = at<uint8_t>(ws, w.dq), *dk = at<uint8_t>(ws, w.dk);
+    int32_t *sel = at<int32_t>(ws, w.sel), *selc = at<int32_t>(ws, w.selc);
+    int sq = 1, sk = 1;
+    cudaEvent_t *pe = nullptr;
+    if (g.flags & AC_FLAG_PROFILE) {
+        pe = c->prof + (size_t)(c->prof_n % PROF_RING) * PROF_EV;
+        c->prof_n++;
+        AC_CUDA(cudaEventRecord(pe[0], st));
+    }
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[0], st));
+    s = run_cluster(c, MODE_SPHERE, q, (warm && q_cent_io) ? q_cent_io : nullptr, qa, qc, qn, qmn, nq, dq, ws, st,
+                    &sq);
+    if (s != AC_OK) return s;
+    if (pe) AC_CUDA(cudaEventRecord(pe[1], st));
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[1], st));
+    s = run_cluster(c, MODE_EUCLID, k, (warm && k_cent_io) ? k_cent_io : nullptr, ka, kc, kn, nullptr, nk, dk, ws,
+                    st, &sk);
+    if (s != AC_OK) return s;
+    if (pe) AC_CUDA(cudaEventRecord(pe[2], st));
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[2], st));
+    // a head is dense when either clustering set its flag F
+    uint8_t *dense = dk;
+    if (g.adaptive_q) ac_or_flags(g.heads, dq, dk, st);
+    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, c->kk_cap, nq, nk, g.kq, g.kk, dense, g.top_p, sel, selc,
+             st);
+    if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
+    s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
+                       pe ? pe + 4 : nullptr);
+    if (s != AC_OK) return s;
+    if (stats) {
+        AC_CUDA(cudaEventRecord(c->ev[4], st));
+        AC_CUDA(cudaEventSynchronize(c->ev[4]));
+        float ms[4];
+        cudaEventElapsedTime(&ms[0], c->ev[0], c->ev[1]);
+        cudaEventElapsedTime(&ms[1], c->ev[1], c->ev[2]);
+        cudaEventElapsedTime(&ms[2], c->ev[2], c->ev[3]);
+        cudaEventElapsedTime(&ms[3], c->ev[3], c->ev[4]);
+        memset(stats, 0, sizeof(*stats));
+        stats->ms_cluster_q = ms[0];
+        stats->ms_cluster_k = ms[1];
+        stats->ms_select = ms[2];
+        stats->ms_attn = ms[3];
+        stats->ms_total = ms[0] + ms[1] + ms[2] + ms[3];
+        int64_t pairs = 0;
+        AC_CUDA(cudaMemcpy(&pairs, at<int64_t>(ws, w.pairs), sizeof(pairs), cudaMemcpyDeviceToHost));
+        stats->pairs = pairs;
+        uint8_t *hd = (uint8_t *)malloc(g.heads);
+        if (hd) {
+            AC_CUDA(cudaMemcpy(hd, dense, g.heads, cudaMemcpyDeviceToHost));
+            for (int h = 0; h < g.heads; h++) stats->dense_heads += hd[h] ? 1 : 0;
+            free(hd);
+        }
+        stats->max_stages_q = sq;
+        stats->max_stages_k = sk;
+    }
+    return launch_check();
+}
+
+ac_status ac_get_status(ac_ctx *c, void *stream) {
+    if (!c) return AC_ERR_INVALID_ARG;
+    AC_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+    int h[8];
+    AC_CUDA(cudaMemcpy(h, c->d_status, sizeof(h), cudaMemcpyDeviceToHost));
+    AC_CUDA(cudaMemset(c->d_status, 0, sizeof(h)));
+    return (ac_status)h[0];
+}
+
+}  // extern "C"
+
+__global__ void or_flags_kernel(int H, const uint8_t *a, uint8_t *b) {
+    int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h < H) b[h] = (uint8_t)(a[h] | b[h]);
+}
+void ac_or_flags(int H, const uint8_t *a, uint8_t *b, cudaStream_t st) {
+    or_flags_kernel<<<(H + 127) / 128, 128, 0, st>>>(H, a, b); note_launch();
+}

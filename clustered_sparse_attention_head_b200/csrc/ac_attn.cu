@@ -1,0 +1,609 @@
+// Block-sparse exact softmax attention over selected key clusters (AdaCluster,
+// Algorithm 3 line 9; line 4 for dense heads) on sm_100a tensor cores.
+//
+// Inputs are gathered into cluster order (ac_sort.cu): the rows of query
+// cluster a are contiguous in Qg, the keys/values of key cluster b contiguous
+// in Kg/Vg.  A work item is one tile of up to 128 query rows of one query
+// cluster (or of a dense head); it walks the key rows of every selected key
+// cluster in chunks of up to BN rows.
+//
+// Per CTA (persistent, one per SM): warp 0 issues TMA loads (Q tile once per
+// item, K/V chunks into a 2-stage ring, 32-row boxes so a short cluster tail
+// costs only the rows it needs); lane 0 of warp 1 issues tcgen05.mma:
+// S = Q K^T into one of two TMEM buffers, O += P V into a TMEM accumulator;
+// warps 2-5 (one thread per query row = TMEM lane) run the online softmax
+// from TMEM, write P (bf16, or tf32 for fp32 inputs) to shared memory in the
+// 128-byte-swizzled K-major layout, and do the epilogue (O / l, scatter rows
+// back to token order).  The running max is only moved (and O rescaled in
+// TMEM) when it grows by more than 2^8, so most chunks skip the rescale.
+// Every mbarrier wait is bounded; on expiry the CTA records ST_TIMEOUT,
+// drains its own copies and MMAs, frees TMEM and returns.
+#include "ac_kernels.cuh"
+
+namespace ac {
+
+template <typename T, int D> struct AttnCfg {
+    static constexpr int ELT = sizeof(T);
+    static constexpr int BM = 128;
+    static constexpr int BN = (ELT == 4 && D == 128) ? 64 : 128;
+    static constexpr int EPR = 128 / ELT;          // elements per 128-byte swizzle row
+    static constexpr int DB = D / EPR;             // 128-byte column blocks of a Q/K/V row
+    static constexpr int KSTEP = 32 / ELT;         // K of one MMA instruction
+    static constexpr int BOX = 32;                 // rows per K/V TMA box
+    static constexpr int Q_BYTES = BM * D * ELT;
+    static constexpr int KV_BYTES = BN * D * ELT;  // one stage of K (or of V)
+    static constexpr int P_BYTES = BM * BN * ELT;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
+    static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    // + alignment slack; at least 116 KB so that two CTAs never share an SM
+    // (each allocates all 512 TMEM columns)
+    static constexpr int SMEM_RAW = OFF_BAR + 256 + 1024;
+    static constexpr int SMEM = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
+    static constexpr int FMT = (ELT == 2) ? 1 : 2;     // bf16 / tf32
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int TM_S0 = 0, TM_S1 = BN, TM_O = 2 * BN;
+    static_assert(TM_O + D <= (int)TMEM_COLS, "TMEM budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct AttnParams {
+    int H, N;
+    const int32_t *qperm;
+    const int32_t *koff;
+    int kk_cap;
+    const int32_t *sel_idx;
+    const int32_t *sel_cnt;
+    int kq_cap;
+    const AttnItem *items;
+    const int32_t *n_items;
+    void *out;
+    float *lse;
+    int *status;
+    float scale_log2;
+};
+
+// Walks the key chunks of one work item: every selected key cluster's rows
+// [koff[b], koff[b+1]) (all rows [0, N) for a dense head) in pieces of <= BN.
+struct ChunkIter {
+    const int32_t *koff, *sel;
+    int nsel, si, cur, end, bn;
+    __device__ void init(const AttnParams &p, const AttnItem &it, int bn_) {
+        bn = bn_;
+        koff = p.koff + (size_t)it.h * (p.kk_cap + 1);
+        if (it.a < 0) {
+            sel = nullptr;
+            nsel = 1;
+        } else {
+            sel = p.sel_idx + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
+            nsel = p.sel_cnt[(size_t)it.h * p.kq_cap + it.a];
+        }
+        si = -1;
+        cur = end = 0;
+        (void)p;
+        dense_n = p.N;
+    }
+    int dense_n;
+    __device__ bool next(int &start, int &len) {
+        while (cur >= end) {
+            if (++si >= nsel) return false;
+            if (sel) {
+                int b = sel[si];
+                cur = koff[b];
+                end = koff[b + 1];
+            } else {
+                cur = 0;
+                end = dense_n;
+            }
+        }
+        start = cur;
+        len = min(bn, end - cur);
+        cur += len;
+        return true;
+    }
+    __device__ int count(const AttnParams &p, const AttnItem &it) {
+        init(p, it, bn);
+        int n = 0, s, l;
+        while (next(s, l)) n++;
+        init(p, it, bn);
+        return n;
+    }
+};
+
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
+    bool ok = mbar_wait(bar, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag (used to drain own copies / MMAs).
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+    uint64_t t0 = gtimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (gtimer() - t0 > 200000000ull) break;
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    using C = AttnCfg<T, D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                          ~(uintptr_t)1023);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
+    uint64_t *q_full = bars + 0, *q_empty = bars + 1;
+    uint64_t *k_full = bars + 2, *v_full = bars + 4, *kv_empty = bars + 6;
+    uint64_t *s_full = bars + 8, *s_empty = bars + 10;
+    uint64_t *p_full = bars + 12, *o_done = bars + 13, *o_free = bars + 14, *drain = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(k_full + i, 1);
+            mbar_init(v_full + i, 1);
+            mbar_init(kv_empty + i, 1);
+            mbar_init(s_full + i, 1);
+            mbar_init(s_empty + i, 128);
+        }
+        mbar_init(p_full, 128);
+        mbar_init(o_done, 1);
+        mbar_init(o_free, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_items = *p.n_items;
+
+    if (warp == 0) {
+        // ------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            uint32_t g = 0, qi = 0;
+            int last_kv[2] = {-1, -1};
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+                AttnItem it = p.items[item];
+                ChunkIter ci;
+                ci.bn = C::BN;
+                if (ci.count(p, it) == 0) continue;
+                if (qi >= 1 && !mbar_wait(q_empty, (qi - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+                const int qrow = it.h * p.N + it.q_start;
+                for (int kb = 0; kb < C::DB; kb++)
+                    tma_load_2d(sm + C::OFF_Q + kb * (C::BM * 128), &tmQ, q_full, kb * C::EPR, qrow);
+                qi++;
+                int start, len;
+                while (ci.next(start, len)) {
+                    const int st = g & 1;
+                    const uint32_t u = g >> 1;
+                    if (u >= 1 && !mbar_wait(kv_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    const int nb = (len + C::BOX - 1) / C::BOX;
+                    const uint32_t bytes = (uint32_t)nb * C::BOX * 128 * C::DB;
+                    const int krow = it.h * p.N + start;
+                    mbar_arrive_expect_tx(k_full + st, bytes);
+                    for (int kb = 0; kb < C::DB; kb++)
+                        for (int b = 0; b < nb; b++)
+                            tma_load_2d(sm + C::OFF_K + st * C::KV_BYTES + kb * (C::BN * 128) + b * (C::BOX * 128),
+                                        &tmK, k_full + st, kb * C::EPR, krow + b * C::BOX);
+                    mbar_arrive_expect_tx(v_full + st, bytes);
+                    for (int kb = 0; kb < C::DB; kb++)
+                        for (int b = 0; b < nb; b++)
+                            tma_load_2d(sm + C::OFF_V + st * C::KV_BYTES + kb * (C::BN * 128) + b * (C::BOX * 128),
+                                        &tmV, v_full + st, kb * C::EPR, krow + b * C::BOX);
+                    last_kv[st] = (int)u;
+                    g++;
+                }
+            }
+            if (!ok) {
+                // drain the copies this thread issued before leaving
+                if (qi >= 1) drain_wait(q_full, (qi - 1) & 1);
+                for (int st = 0; st < 2; st++)
+                    if (last_kv[st] >= 0) {
+                        drain_wait(k_full + st, last_kv[st] & 1);
+                        drain_wait(v_full + st, last_kv[st] & 1);
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_o = idesc_make(128, D, C::FMT, true);
+            uint32_t g = 0, qi = 0;
+            bool ok = true;
+            auto issue_pv = [&](uint32_t gp, int lenp, bool first) -> bool {
+                if (!mbar_wait(p_full, gp & 1, abort_flag, p.status)) return false;
+                if (!mbar_wait(v_full + (gp & 1), (gp >> 1) & 1, abort_flag, p.status)) return false;
+                if (first && qi >= 2 && !mbar_wait(o_free, (qi - 2) & 1, abort_flag, p.status)) return false;
+                tc_fence_after();
+                const int np = (lenp + 31) & ~31;
+                const uint32_t vbase = smem_u32(sm + C::OFF_V + (gp & 1) * C::KV_BYTES);
+                const uint32_t pbase = smem_u32(sm + C::OFF_P);
+                for (int ks = 0; ks < np / C::KSTEP; ks++) {
+                    const int kofs = ks * C::KSTEP;
+                    const uint64_t a = sdesc_sw128(pbase + (kofs / C::EPR) * (C::BM * 128) + (kofs % C::EPR) * C::ELT,
+                                                   16, 1024);
+                    // V is MN-major (d contiguous): 128-byte blocks along d at
+                    // LBO; 8-row (bf16) or 4-row (tf32, 32-byte atoms) K groups at SBO
+                    const uint64_t b = sdesc_make(vbase + kofs * 128, C::BN * 128, C::ELT == 2 ? 1024 : 512,
+                                                  C::ELT == 2 ? 2u : 1u);
+                    if (C::FMT == 1) umma_f16(tmem + C::TM_O, a, b, idesc_o, (!first || ks > 0) ? 1u : 0u);
+                    else umma_tf32(tmem + C::TM_O, a, b, idesc_o, (!first || ks > 0) ? 1u : 0u);
+                }
+                umma_commit(o_done);
+                umma_commit(kv_empty + (gp & 1));
+                return true;
+            };
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+                AttnItem it = p.items[item];
+                ChunkIter ci;
+                ci.bn = C::BN;
+                const int nch = ci.count(p, it);
+                if (nch == 0) continue;
+                if (!mbar_wait(q_full, qi & 1, abort_flag, p.status)) { ok = false; break; }
+                qi++;
+                int start, len, c = 0, prev_len = 0;
+                while (ci.next(start, len)) {
+                    const int st = g & 1;
+                    const uint32_t u = g >> 1;
+                    if (!mbar_wait(k_full + st, u & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (u >= 1 && !mbar_wait(s_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const int ncol = (len + 31) & ~31;
+                    const uint32_t idesc_s = idesc_make(128, ncol, C::FMT, false);
+                    const uint32_t qbase = smem_u32(sm + C::OFF_Q);
+                    const uint32_t kbase = smem_u32(sm + C::OFF_K + st * C::KV_BYTES);
+                    const uint32_t dS = tmem + (st ? C::TM_S1 : C::TM_S0);
+                    for (int ks = 0; ks < D / C::KSTEP; ks++) {
+                        const int kofs = ks * C::KSTEP;
+                        const uint32_t boff = (kofs % C::EPR) * C::ELT;
+                        const uint64_t a = sdesc_sw128(qbase + (kofs / C::EPR) * (C::BM * 128) + boff, 16, 1024);
+                        const uint64_t b = sdesc_sw128(kbase + (kofs / C::EPR) * (C::BN * 128) + boff, 16, 1024);
+                        if (C::FMT == 1) umma_f16(dS, a, b, idesc_s, ks > 0 ? 1u : 0u);
+                        else umma_tf32(dS, a, b, idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    umma_commit(s_full + st);
+                    if (c == nch - 1) umma_commit(q_empty);
+                    if (c > 0 && !issue_pv(g - 1, prev_len, c == 1)) { ok = false; break; }
+                    prev_len = len;
+                    c++;
+                    g++;
+                }
+                if (!ok) break;
+                if (!issue_pv(g - 1, prev_len, nch == 1)) { ok = false; break; }
+            }
+            if (!ok) {
+                umma_commit(drain);
+                drain_wait(drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax + epilogue
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        uint32_t g = 0;
+        bool ok = true;
+        unsigned char *prow = sm + C::OFF_P + row * 128;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            AttnItem it = p.items[item];
+            ChunkIter ci;
+            ci.bn = C::BN;
+            const int nch = ci.count(p, it);
+            float m_ref = -INFINITY, l = 0.f;
+            int start, len, c = 0;
+            while (nch > 0 && ci.next(start, len)) {
+                const int st = g & 1;
+                const uint32_t u = g >> 1;
+                if (!wait_all(s_full + st, u & 1, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sadr = tmem + lane_addr + (st ? C::TM_S1 : C::TM_S0);
+                const int npc = (len + 31) >> 5;
+                float mx = -INFINITY;
+                uint32_t r[32];
+                for (int pc = 0; pc < npc; pc++) {
+                    tmem_ld32(sadr + pc * 32, r);
+#pragma unroll
+                    for (int i = 0; i < 32; i++)
+                        if (pc * 32 + i < len) mx = fmaxf(mx, __uint_as_float(r[i]));
+                }
+                const float m_new = mx * p.scale_log2;
+                if (c == 0) m_ref = m_new;
+                if (g >= 1 && !wait_all(o_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                // Move the reference max (and rescale O) only when it grew by
+                // more than 2^8.  The TMEM accesses are warp-collective, so the
+                // decision is taken per warp; rows that did not grow use f = 1.
+                if (c > 0 && __any_sync(0xffffffffu, m_new > m_ref + 8.f)) {
+                    const float m_to = fmaxf(m_ref, m_new);
+                    const float f = ex2_approx(m_ref - m_to);
+                    l *= f;
+                    tc_fence_after();
+                    for (int pc = 0; pc < D / 32; pc++) {
+                        tmem_ld32(tmem + lane_addr + C::TM_O + pc * 32, r);
+#pragma unroll
+                        for (int i = 0; i < 32; i++) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+                        tmem_st32(tmem + lane_addr + C::TM_O + pc * 32, r);
+                    }
+                    tmem_st_wait();
+                    m_ref = m_to;
+                }
+                const int ncol = npc * 32;
+                for (int pc = 0; pc < npc; pc++) {
+                    tmem_ld32(sadr + pc * 32, r);
+                    float pv[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i++) {
+                        float e = (pc * 32 + i < len) ? ex2_approx(fmaf(__uint_as_float(r[i]), p.scale_log2, -m_ref))
+                                                      : 0.f;
+                        pv[i] = e;
+                    }
+                    if (C::ELT == 2) {
+                        // 32 bf16 = 4 x 16-byte chunks of the row's 128-byte block
+                        const int kb = (pc * 32) / C::EPR;
+                        const int ch0 = ((pc * 32) % C::EPR) / 8;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; q4++) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; e2++) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[q4 * 8 + e2 * 2], pv[q4 * 8 + e2 * 2 + 1]);
+                                float2 back = __bfloat1622float2(b2);
+                                l += back.x + back.y;
+                                w[e2] = *reinterpret_cast<uint32_t *>(&b2);
+                            }
+                            const int chunk = (ch0 + q4) ^ (row & 7);
+                            *reinterpret_cast<uint4 *>(prow + kb * (C::BM * 128) + chunk * 16) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    } else {
+                        // 32 fp32 (rounded to tf32) = one whole 128-byte block
+                        const int kb = pc;
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; q4++) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; e2++) {
+                                uint32_t tf;
+                                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(tf) : "f"(pv[q4 * 4 + e2]));
+                                l += __uint_as_float(tf);
+                                w[e2] = tf;
+                            }
+                            const int chunk = q4 ^ (row & 7);
+                            *reinterpret_cast<uint4 *>(prow + kb * (C::BM * 128) + chunk * 16) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                (void)ncol;
+                tc_fence_before();
+                mbar_arrive(s_empty + st);
+                fence_proxy_async_smem();
+                mbar_arrive(p_full);
+                c++;
+                g++;
+            }
+            if (!ok) break;
+            // epilogue: out row = O / l, scattered back to token order
+            const bool valid = row < it.q_len;
+            int tok = 0;
+            if (valid) tok = p.qperm[(size_t)it.h * p.N + it.q_start + row];
+            const size_t orow = ((size_t)it.h * p.N + tok) * D;
+            if (nch > 0) {
+                if (!wait_all(o_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const float inv = 1.f / l;
+                for (int pc = 0; pc < D / 32; pc++) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_addr + C::TM_O + pc * 32, r);
+                    if (valid) {
+                        if (C::ELT == 2) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int i = 0; i < 16; i++) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * inv,
+                                                                          __uint_as_float(r[2 * i + 1]) * inv);
+                                w[i] = *reinterpret_cast<uint32_t *>(&b2);
+                            }
+                            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow + pc * 32);
+#pragma unroll
+                            for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                        } else {
+                            float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + orow + pc * 32);
+#pragma unroll
+                            for (int i = 0; i < 8; i++)
+                                dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                                                     __uint_as_float(r[4 * i + 2]) * inv,
+                                                     __uint_as_float(r[4 * i + 3]) * inv);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(o_free);
+                if (valid && p.lse) p.lse[(size_t)it.h * p.N + tok] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+            } else if (valid) {
+                for (int t = 0; t < D; t++) {
+                    if (C::ELT == 2) reinterpret_cast<__nv_bfloat16 *>(p.out)[orow + t] = __float2bfloat16(0.f);
+                    else reinterpret_cast<float *>(p.out)[orow + t] = 0.f;
+                }
+                if (p.lse) p.lse[(size_t)it.h * p.N + tok] = -INFINITY;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------ work items
+// One CTA: for each head, query tiles of 128 rows per non-empty query cluster
+// (or over all rows of a dense head), plus the number of (query, key) pairs.
+__global__ void build_items_kernel(int H, int N, int kq_cap, int kk_cap, const int32_t *__restrict__ qoff,
+                                   const int32_t *__restrict__ nq, const uint8_t *__restrict__ dense, int kq_fixed,
+                                   const int32_t *__restrict__ koff, const int32_t *__restrict__ sel_idx,
+                                   const int32_t *__restrict__ sel_cnt, AttnItem *__restrict__ items,
+                                   int32_t *__restrict__ n_items, int64_t *__restrict__ pairs) {
+    __shared__ int wsum[32];
+    __shared__ int base;
+    __shared__ unsigned long long pairs_acc;
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, w = tid >> 5;
+    if (tid == 0) {
+        base = 0;
+        pairs_acc = 0ull;
+    }
+    __syncthreads();
+    for (int h = 0; h < H; h++) {
+        const bool dn = dense && dense[h];
+        const int nqh = dn ? 1 : (nq ? nq[h] : kq_fixed);
+        const int32_t *qo = qoff + (size_t)h * (kq_cap + 1);
+        const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
+        for (int a0 = 0; a0 < nqh; a0 += nt) {
+            const int a = a0 + tid;
+            int qs = 0, qn = 0, tiles = 0;
+            if (a < nqh) {
+                if (dn) { qs = 0; qn = N; }
+                else { qs = qo[a]; qn = qo[a + 1] - qs; }
+                tiles = (qn + 127) / 128;
+                if (!dn && qn > 0) {
+                    long long keys = 0;
+                    const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
+                    const int ns = sel_cnt[(size_t)h * kq_cap + a];
+                    for (int c = 0; c < ns; c++) keys += ko[sl[c] + 1] - ko[sl[c]];
+                    atomicAdd(&pairs_acc, (unsigned long long)(keys * qn));
+                } else if (dn) {
+                    atomicAdd(&pairs_acc, (unsigned long long)N * (unsigned long long)N);
+                }
+            }
+            int x = tiles;
+            for (int d = 1; d < 32; d <<= 1) {
+                int y = __shfl_up_sync(0xffffffffu, x, d);
+                if (lane >= d) x += y;
+            }
+            if (lane == 31) wsum[w] = x;
+            __syncthreads();
+            if (w == 0) {
+                int t = lane < nt / 32 ? wsum[lane] : 0;
+                for (int d = 1; d < 32; d <<= 1) {
+                    int y = __shfl_up_sync(0xffffffffu, t, d);
+                    if (lane >= d) t += y;
+                }
+                if (lane < nt / 32) wsum[lane] = t;
+            }
+            __syncthreads();
+            const int excl = base + x - tiles + (w > 0 ? wsum[w - 1] : 0);
+            for (int t = 0; t < tiles; t++) {
+                AttnItem itm;
+                itm.h = h;
+                itm.a = dn ? -1 : a;
+                itm.q_start = qs + t * 128;
+                itm.q_len = min(128, qn - t * 128);
+                items[excl + t] = itm;
+            }
+            __syncthreads();
+            if (tid == 0) base += wsum[nt / 32 - 1];
+            __syncthreads();
+        }
+    }
+    if (tid == 0) {
+        *n_items = base;
+        if (pairs) *pairs = (int64_t)pairs_acc;
+    }
+}
+
+int attn_max_items(int H, int N, int kq_cap) { return H * ((N + 127) / 128 + kq_cap); }
+
+void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
+                   const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
+                   const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, cudaStream_t st) {
+    build_items_kernel<<<1, 1024, 0, st>>>(H, N, kq_cap, kk_cap, qoff, nq, dense, kq_fixed, koff, sel_idx, sel_cnt,
+                                           items, n_items, pairs); note_launch();
+}
+
+// ------------------------------------------------------------ launcher
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static int make_map(EncodeTiledFn enc, CUtensorMap *m, const void *base, int elt, int rows, int cols, int box_rows,
+                    CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * elt};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / elt), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, elt == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+template <typename T, int D>
+static int launch_attn(const void *qg, const void *kg, const void *vg, const AttnParams &p, int max_items,
+                       int num_sms, void *encode_fn, cudaStream_t st) {
+    using C = AttnCfg<T, D>;
+    EncodeTiledFn enc = (EncodeTiledFn)encode_fn;
+    CUtensorMap mq, mk, mv;
+    const int rows = p.H * p.N;
+    if (make_map(enc, &mq, qg, C::ELT, rows, D, C::BM) || make_map(enc, &mk, kg, C::ELT, rows, D, C::BOX) ||
+        make_map(enc, &mv, vg, C::ELT, rows, D, C::BOX,
+                 C::ELT == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
+        return -1;
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(attn_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        attr = true;
+    }
+    int grid = max_items < num_sms ? max_items : num_sms;
+    if (grid < 1) grid = 1;
+    attn_kernel<T, D><<<grid, 192, C::SMEM, st>>>(mq, mk, mv, p); note_launch();
+    return 0;
+}
+
+int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
+                const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
+                const int32_t *sel_cnt, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
+                float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st) {
+    AttnParams p;
+    p.H = H;
+    p.N = N;
+    p.qperm = qperm;
+    p.koff = koff;
+    p.kk_cap = kk_cap;
+    p.sel_idx = sel_idx;
+    p.sel_cnt = sel_cnt;
+    p.kq_cap = kq_cap;
+    p.items = items;
+    p.n_items = n_items;
+    p.out = out;
+    p.lse = lse;
+    p.status = status;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    if (dtype == DT_BF16) {
+        if (D == 64) return launch_attn<__nv_bfloat16, 64>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+        return launch_attn<__nv_bfloat16, 128>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+    }
+    if (D == 64) return launch_attn<float, 64>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+    return launch_attn<float, 128>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+}
+
+}  // namespace ac

@@ -1,0 +1,61 @@
+// Internal launch interface between the C ABI (ac_api.cu) and the kernels.
+#pragma once
+#include "ac_common.cuh"
+
+namespace ac {
+
+enum { MODE_EUCLID = 0, MODE_SPHERE = 1 };
+enum { DT_F32 = 0, DT_BF16 = 1 };
+constexpr int SORT_TILE = 256;  // positions per rank/histogram tile (one warp)
+
+// Host-side count of kernels this library has launched (profiling).
+void note_launch();
+long long launches_total();
+
+// ---- ac_kmeans.cu
+void k_row_norm(const void *x, int dtype, int H, int N, int D, double *norm, int check, int *status,
+                cudaStream_t st);
+void k_init_cent(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const double *norm,
+                 const HeadSeg *seg, int kmax, int mode, float *cent, int cap, cudaStream_t st);
+void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
+              int nrows_max, const float *cent, int cap, float *cn2, float *cmax, const double *norm, int mode,
+              int32_t *assign, int32_t *amb_list, int32_t *amb_count, cudaStream_t st);
+void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
+            int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
+            double *dist, cudaStream_t st);
+void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg, int kmax, const int32_t *perm,
+              const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st);
+void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const int32_t *off, int cap,
+                 const double *norm, float *mean_norm, cudaStream_t st);
+
+// ---- ac_sort.cu
+// Stable counting sort of positions 0..seg.nrows-1 by id (< seg.k): perm gets
+// rows[pos] (or pos), off [H, cap+1] the cluster offsets, cnt [H, cap] the sizes.
+void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, int N, int nrows_max, int cap,
+            int32_t *rank, int32_t *hist, int32_t *cnt, int32_t *off, int32_t *perm, int *status, cudaStream_t st);
+size_t sort_hist_elems(int H, int N, int cap);
+void k_gather_rows(const void *src, void *dst, const int32_t *perm, int H, int N, int row_bytes, cudaStream_t st);
+
+// ---- ac_multistage.cu
+struct MsState;  // device-side Algorithm 1 state, see ac_multistage.cu
+
+// ---- ac_select.cu
+void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const int32_t *q_count, int kq_cap,
+              const float *k_cent, const int32_t *k_count, int kk_cap, const int32_t *nq, const int32_t *nk,
+              int kq_fixed, int kk_fixed, const uint8_t *dense, double top_p, int32_t *sel_idx, int32_t *sel_cnt,
+              cudaStream_t st);
+
+// ---- ac_attn.cu
+struct AttnItem {
+    int h, a, q_start, q_len;  // a < 0: dense head (all keys)
+};
+void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
+                   const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
+                   const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, cudaStream_t st);
+int attn_max_items(int H, int N, int kq_cap);
+int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
+                const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
+                const int32_t *sel_cnt, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
+                float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st);
+
+}  // namespace ac

@@ -1,0 +1,470 @@
+// k-means kernels of AdaCluster ("AdaCluster: Adaptive Query-Key Clustering for
+// Sparse Attention in Video Generation"): spherical k-means on normalised
+// queries (§3.1) and Euclidean k-means on keys (§3.2.1), used per stage by
+// Algorithm 1 (§3.2.2).
+//
+// Decisions (which centroid is closest) are made in double precision with the
+// same operation order as a plain sequential loop, so that they are exact up
+// to the input values: a fp32 screening pass finds the best two candidates of
+// every row and a rigorous rounding bound; only rows whose top-2 gap lies
+// within that bound are re-scored exactly (a warp per row).  Centroid sums are
+// per-cluster double sums in token order over the cluster-sorted permutation,
+// which makes the update deterministic.
+#include "ac_kernels.cuh"
+
+namespace ac {
+
+// ---------------------------------------------------------------- row norms
+// norm[h,i] = sqrt(sum_t x_t^2) (double, sequential).  With check_finite,
+// a NaN/Inf element records ST_NONFINITE.
+template <typename T>
+__global__ void row_norm_kernel(const T *__restrict__ x, int N, int D, double *__restrict__ norm, int check,
+                                int *status) {
+    int h = blockIdx.y;
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    const T *xi = x + ((size_t)h * N + i) * D;
+    double ss = 0.0;
+    bool bad = false;
+    for (int t = 0; t < D; t++) {
+        double v = (double)to_f(xi[t]);
+        if (check && !isfinite(v)) bad = true;
+        ss = dadd(ss, dmul(v, v));
+    }
+    if (bad) set_status(status, ST_NONFINITE);
+    norm[(size_t)h * N + i] = sqrt(ss);
+}
+
+// Working value of element t of token tok: x (EUCLID) or x/||x|| (SPHERE).
+template <typename T>
+__device__ __forceinline__ double work_val(const T *xi, int t, int mode, double nrm) {
+    double v = (double)to_f(xi[t]);
+    if (mode == MODE_SPHERE) return nrm > 0.0 ? ddiv(v, nrm) : 0.0;
+    return v;
+}
+
+// ------------------------------------------------------------------- init
+// Centroid j of the pass = working vector of listed row floor(j * nrows / k).
+template <typename T>
+__global__ void init_cent_kernel(const T *__restrict__ x, int N, int D, const int32_t *__restrict__ rows,
+                                 const double *__restrict__ norm, const HeadSeg *__restrict__ seg, int mode,
+                                 float *__restrict__ cent, int cap) {
+    int h = blockIdx.y, j = blockIdx.x;
+    HeadSeg s = seg[h];
+    if (s.nrows <= 0 || j >= s.k) return;
+    int r = (int)(((int64_t)j * s.nrows) / s.k);
+    int tok = rows ? rows[(size_t)h * N + r] : r;
+    const T *xi = x + ((size_t)h * N + tok) * D;
+    double nrm = norm[(size_t)h * N + tok];
+    float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
+    for (int t = threadIdx.x; t < D; t += blockDim.x) c[t] = (float)work_val(xi, t, mode, nrm);
+}
+
+// ||c_j||^2 as fp32 (from double) and max_j ||c_j|| (rounded up) per head.
+__global__ void cent_prep_kernel(const float *__restrict__ cent, int cap, int D, const HeadSeg *__restrict__ seg,
+                                 float *__restrict__ cn2, float *__restrict__ cmax) {
+    int h = blockIdx.x;
+    HeadSeg s = seg[h];
+    __shared__ float red[32];
+    float mx = 0.f;
+    for (int j = threadIdx.x; j < s.k; j += blockDim.x) {
+        const float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
+        double ss = 0.0;
+        for (int t = 0; t < D; t++) ss += (double)c[t] * (double)c[t];
+        cn2[(size_t)h * cap + j] = (float)ss;
+        float nr = (float)(sqrt(ss) * (1.0 + 1e-6));
+        mx = fmaxf(mx, nr);
+    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); w++) m = fmaxf(m, red[w]);
+        cmax[h] = m;
+    }
+}
+
+// ---------------------------------------------------------- fp32 screening
+// CTA tile: 128 rows x 64 centroids per step, 256 threads, thread = 8 rows x 4
+// centroids.  Screening score (smaller is closer):
+//   EUCLID: ||c||^2 - 2 x.c      SPHERE: -(x.mu)   (x unnormalised: the argmax
+//   of x_hat.mu equals that of x.mu since ||x|| > 0; zero rows tie everywhere).
+// Each score is within E of its exact value, E = (D+8) 2^-23 (2||x|| Cmax +
+// Cmax^2) for EUCLID and (D+8) 2^-23 ||x|| Cmax for SPHERE (twice the standard
+// bound for a length-D fp32 dot product, plus the final combination).  A row
+// whose best two scores are more than 2E apart has a certain winner; the
+// others go to the exact pass.
+constexpr int SCR_ROWS = 128, SCR_COLS = 64, SCR_XS = SCR_ROWS + 4, SCR_CS = SCR_COLS + 4;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) assign_screen_kernel(
+    const T *__restrict__ x, int N, const int32_t *__restrict__ rows, const HeadSeg *__restrict__ seg,
+    const float *__restrict__ cent, int cap, const float *__restrict__ cn2, const float *__restrict__ cmax, int mode,
+    int32_t *__restrict__ assign, int32_t *__restrict__ amb_list, int32_t *__restrict__ amb_count) {
+    extern __shared__ __align__(16) float smf[];
+    float *Xs = smf;                 // [D][SCR_XS]
+    float *Cs = smf + D * SCR_XS;    // [D][SCR_CS]
+    int h = blockIdx.y;
+    HeadSeg s = seg[h];
+    int r0 = blockIdx.x * SCR_ROWS;
+    if (r0 >= s.nrows || s.k <= 0) return;
+    const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
+    const float *ch = cent + ((size_t)h * cap + s.cent_off) * D;
+    const float *cn = cn2 + (size_t)h * cap;
+
+    for (int idx = tid; idx < SCR_ROWS * D; idx += 256) {
+        int rr = idx / D, t = idx - rr * D;
+        int pos = r0 + rr;
+        float v = 0.f;
+        if (pos < s.nrows) {
+            int tok = rows ? rows[(size_t)h * N + pos] : pos;
+            v = to_f(x[((size_t)h * N + tok) * D + t]);
+        }
+        Xs[t * SCR_XS + rr] = v;
+    }
+
+    __syncthreads();
+    float xn_row = 0.f;
+    if (tid < SCR_ROWS) {
+        float xx = 0.f;
+        for (int t = 0; t < D; t++) xx = fmaf(Xs[t * SCR_XS + tid], Xs[t * SCR_XS + tid], xx);
+        xn_row = sqrtf(xx) * 1.001f;
+    }
+
+    float b1[8], b2[8];
+    int i1[8];
+#pragma unroll
+    for (int a = 0; a < 8; a++) { b1[a] = INFINITY; b2[a] = INFINITY; i1[a] = 0; }
+
+    for (int j0 = 0; j0 < s.k; j0 += SCR_COLS) {
+        __syncthreads();
+        for (int idx = tid; idx < SCR_COLS * D; idx += 256) {
+            int jj = idx / D, t = idx - jj * D;
+            int j = j0 + jj;
+            Cs[t * SCR_CS + jj] = (j < s.k) ? ch[(size_t)j * D + t] : 0.f;
+        }
+        __syncthreads();
+        float acc[8][4];
+#pragma unroll
+        for (int a = 0; a < 8; a++)
+#pragma unroll
+            for (int b = 0; b < 4; b++) acc[a][b] = 0.f;
+#pragma unroll 4
+        for (int t = 0; t < D; t++) {
+            float4 xa = *reinterpret_cast<const float4 *>(&Xs[t * SCR_XS + tr * 8]);
+            float4 xb = *reinterpret_cast<const float4 *>(&Xs[t * SCR_XS + tr * 8 + 4]);
+            float4 cc = *reinterpret_cast<const float4 *>(&Cs[t * SCR_CS + tc * 4]);
+            float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            float cv[4] = {cc.x, cc.y, cc.z, cc.w};
+#pragma unroll
+            for (int a = 0; a < 8; a++)
+#pragma unroll
+                for (int b = 0; b < 4; b++) acc[a][b] = fmaf(xv[a], cv[b], acc[a][b]);
+        }
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+            int j = j0 + tc * 4 + b;
+            if (j < s.k) {
+                float c2 = (mode == MODE_EUCLID) ? cn[j] : 0.f;
+#pragma unroll
+                for (int a = 0; a < 8; a++) {
+                    float sc = (mode == MODE_EUCLID) ? (c2 - 2.f * acc[a][b]) : -acc[a][b];
+                    if (sc < b1[a]) { b2[a] = b1[a]; b1[a] = sc; i1[a] = j; }
+                    else if (sc < b2[a]) b2[a] = sc;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    // reduce the 16 column groups of every row (buffers overwrite the X tile)
+    float *R1 = smf;                        // [128][16]
+    float *R2 = smf + SCR_ROWS * 16;        // [128][16]
+    int *RI = reinterpret_cast<int *>(smf + 2 * SCR_ROWS * 16);
+#pragma unroll
+    for (int a = 0; a < 8; a++) {
+        int rr = tr * 8 + a;
+        R1[rr * 16 + tc] = b1[a];
+        R2[rr * 16 + tc] = b2[a];
+        RI[rr * 16 + tc] = i1[a];
+    }
+    __syncthreads();
+    if (tid < SCR_ROWS) {
+        int rr = tid, pos = r0 + rr;
+        if (pos < s.nrows) {
+            float B1 = INFINITY, B2 = INFINITY;
+            int I1 = 0x7fffffff;
+            for (int g = 0; g < 16; g++) {
+                float v1 = R1[rr * 16 + g], v2 = R2[rr * 16 + g];
+                int iv = RI[rr * 16 + g];
+                if (v1 < B1 || (v1 == B1 && iv < I1)) {
+                    B2 = fminf(B2, B1);
+                    B1 = v1;
+                    I1 = iv;
+                } else {
+                    B2 = fminf(B2, v1);
+                }
+                B2 = fminf(B2, v2);
+            }
+            float xn = xn_row;
+            float cm = cmax[h];
+            float E = (float)(D + 8) * 1.1920929e-7f *
+                      ((mode == MODE_EUCLID) ? (2.f * xn * cm + cm * cm) : (xn * cm));
+            if (s.k > 1 && !(B2 - B1 > 2.f * E)) {
+                int slot = atomicAdd(&amb_count[h], 1);
+                amb_list[(size_t)h * N + slot] = pos;
+            } else {
+                assign[(size_t)h * N + pos] = I1;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------- exact pass
+// One warp per ambiguous row: every centroid is scored in double with the
+// sequential order of a plain loop (EUCLID: sum (x-c)^2; SPHERE: sum x_hat*mu),
+// and the best score wins, ties to the lowest id.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) assign_exact_kernel(
+    const T *__restrict__ x, int N, const int32_t *__restrict__ rows, const HeadSeg *__restrict__ seg,
+    const float *__restrict__ cent, int cap, const double *__restrict__ norm, int mode,
+    const int32_t *__restrict__ amb_list, const int32_t *__restrict__ amb_count, int32_t *__restrict__ assign) {
+    __shared__ double xs[8][D];
+    int h = blockIdx.y;
+    HeadSeg s = seg[h];
+    int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int na = amb_count[h];
+    const float *ch = cent + ((size_t)h * cap + s.cent_off) * D;
+    for (int a = blockIdx.x * 8 + warp; a < na; a += gridDim.x * 8) {
+        int pos = amb_list[(size_t)h * N + a];
+        int tok = rows ? rows[(size_t)h * N + pos] : pos;
+        const T *xi = x + ((size_t)h * N + tok) * D;
+        double nrm = norm[(size_t)h * N + tok];
+        __syncwarp();
+        for (int t = lane; t < D; t += 32) xs[warp][t] = work_val(xi, t, mode, nrm);
+        __syncwarp();
+        double best = (mode == MODE_EUCLID) ? INFINITY : -INFINITY;
+        int bj = 0x7fffffff;
+        for (int j = lane; j < s.k; j += 32) {
+            const float *c = ch + (size_t)j * D;
+            double acc = 0.0;
+            if (mode == MODE_EUCLID) {
+                for (int t = 0; t < D; t++) {
+                    double df = dsub(xs[warp][t], (double)c[t]);
+                    acc = dadd(acc, dmul(df, df));
+                }
+                if (acc < best) { best = acc; bj = j; }
+            } else {
+                for (int t = 0; t < D; t++) acc = dadd(acc, dmul(xs[warp][t], (double)c[t]));
+                if (acc > best) { best = acc; bj = j; }
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            double ob = __shfl_xor_sync(0xffffffffu, best, o);
+            int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+            bool better = (mode == MODE_EUCLID) ? (ob < best) : (ob > best);
+            if (better || (ob == best && oj < bj)) { best = ob; bj = oj; }
+        }
+        if (lane == 0) assign[(size_t)h * N + pos] = bj;
+    }
+}
+
+// ------------------------------------------------------------- distances
+// dist[h,pos] = ||x' - c_assign||_2 in double (x' = working vector).
+template <typename T, int D>
+__global__ void dist_kernel(const T *__restrict__ x, int N, const int32_t *__restrict__ rows,
+                            const HeadSeg *__restrict__ seg, const float *__restrict__ cent, int cap,
+                            const double *__restrict__ norm, int mode, const int32_t *__restrict__ assign,
+                            double *__restrict__ dist) {
+    int h = blockIdx.y;
+    HeadSeg s = seg[h];
+    int pos = blockIdx.x * blockDim.x + threadIdx.x;
+    if (pos >= s.nrows) return;
+    int tok = rows ? rows[(size_t)h * N + pos] : pos;
+    const T *xi = x + ((size_t)h * N + tok) * D;
+    double nrm = norm[(size_t)h * N + tok];
+    const float *c = cent + ((size_t)h * cap + s.cent_off + assign[(size_t)h * N + pos]) * D;
+    double acc = 0.0;
+    for (int t = 0; t < D; t++) {
+        double df = dsub(work_val(xi, t, mode, nrm), (double)c[t]);
+        acc = dadd(acc, dmul(df, df));
+    }
+    dist[(size_t)h * N + pos] = sqrt(acc);
+}
+
+// ----------------------------------------------------------------- update
+// Cluster j of head h (grid x = j, y = h; blockDim = D): members are
+// perm[off[j] .. off[j+1]) in token order; thread t sums element t of their
+// working vectors in double in that order.  EUCLID: c = sum / count.
+// SPHERE: mu = sum / ||sum||.  Empty clusters (or a zero sum) keep their centroid.
+template <typename T, int D>
+__global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__restrict__ seg,
+                              const int32_t *__restrict__ perm, const int32_t *__restrict__ off, int cap,
+                              const double *__restrict__ norm, int mode, float *__restrict__ cent) {
+    __shared__ double ssum[D];
+    __shared__ double snr;
+    int h = blockIdx.y, j = blockIdx.x, t = threadIdx.x;
+    HeadSeg s = seg[h];
+    if (s.nrows <= 0 || j >= s.k) return;
+    const int32_t *o = off + (size_t)h * (cap + 1);
+    int b = o[j], e = o[j + 1];
+    if (e <= b) return;
+    const int32_t *ph = perm + (size_t)h * N;
+    double acc = 0.0;
+    int r = b;
+    for (; r + 4 <= e; r += 4) {
+        int t0 = ph[r], t1 = ph[r + 1], t2 = ph[r + 2], t3 = ph[r + 3];
+        double v0 = work_val(x + ((size_t)h * N + t0) * D, t, mode, norm[(size_t)h * N + t0]);
+        double v1 = work_val(x + ((size_t)h * N + t1) * D, t, mode, norm[(size_t)h * N + t1]);
+        double v2 = work_val(x + ((size_t)h * N + t2) * D, t, mode, norm[(size_t)h * N + t2]);
+        double v3 = work_val(x + ((size_t)h * N + t3) * D, t, mode, norm[(size_t)h * N + t3]);
+        acc = dadd(acc, v0);
+        acc = dadd(acc, v1);
+        acc = dadd(acc, v2);
+        acc = dadd(acc, v3);
+    }
+    for (; r < e; r++) {
+        int tk = ph[r];
+        acc = dadd(acc, work_val(x + ((size_t)h * N + tk) * D, t, mode, norm[(size_t)h * N + tk]));
+    }
+    float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
+    if (mode == MODE_EUCLID) {
+        c[t] = (float)ddiv(acc, (double)(e - b));
+        return;
+    }
+    ssum[t] = acc;
+    __syncthreads();
+    if (t == 0) {
+        double ss = 0.0;
+        for (int u = 0; u < D; u++) ss = dadd(ss, dmul(ssum[u], ssum[u]));
+        snr = sqrt(ss);
+    }
+    __syncthreads();
+    if (snr > 0.0) c[t] = (float)ddiv(acc, snr);
+}
+
+// Mean ||q|| over the members of each cluster (sequential double sum in
+// token order); 0 for empty clusters.
+__global__ void mean_norm_kernel(int N, const HeadSeg *__restrict__ seg, const int32_t *__restrict__ perm,
+                                 const int32_t *__restrict__ off, int cap, const double *__restrict__ norm,
+                                 float *__restrict__ mean_norm) {
+    int h = blockIdx.y;
+    int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= cap) return;
+    HeadSeg s = seg[h];
+    float out = 0.f;
+    if (j < s.k) {
+        const int32_t *o = off + (size_t)h * (cap + 1);
+        int b = o[j], e = o[j + 1];
+        double acc = 0.0;
+        for (int r = b; r < e; r++) acc = dadd(acc, norm[(size_t)h * N + perm[(size_t)h * N + r]]);
+        if (e > b) out = (float)ddiv(acc, (double)(e - b));
+    }
+    mean_norm[(size_t)h * cap + j] = out;
+}
+
+// ------------------------------------------------------------- launchers
+template <typename T>
+static void launch_row_norm(const void *x, int H, int N, int D, double *norm, int check, int *status,
+                            cudaStream_t st) {
+    dim3 g((N + 255) / 256, H);
+    row_norm_kernel<T><<<g, 256, 0, st>>>((const T *)x, N, D, norm, check, status); note_launch();
+}
+
+void k_row_norm(const void *x, int dtype, int H, int N, int D, double *norm, int check, int *status,
+                cudaStream_t st) {
+    if (dtype == DT_BF16) launch_row_norm<__nv_bfloat16>(x, H, N, D, norm, check, status, st);
+    else launch_row_norm<float>(x, H, N, D, norm, check, status, st);
+}
+
+void k_init_cent(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const double *norm,
+                 const HeadSeg *seg, int kmax, int mode, float *cent, int cap, cudaStream_t st) {
+    dim3 g(kmax, H);
+    if (dtype == DT_BF16)
+        init_cent_kernel<__nv_bfloat16><<<g, 128, 0, st>>>((const __nv_bfloat16 *)x, N, D, rows, norm, seg, mode,
+                                                             cent, cap);
+    else
+        init_cent_kernel<float><<<g, 128, 0, st>>>((const float *)x, N, D, rows, norm, seg, mode, cent, cap);
+    note_launch();
+}
+
+template <typename T, int D>
+static void launch_assign(const void *x, int H, int N, const int32_t *rows, const HeadSeg *seg, int nrows_max,
+                          const float *cent, int cap, const float *cn2, const float *cmax, const double *norm,
+                          int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, cudaStream_t st) {
+    size_t smem = (size_t)D * (SCR_XS + SCR_CS) * sizeof(float);
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaFuncSetAttribute(assign_screen_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        attr_set = true;
+    }
+    dim3 g((nrows_max + SCR_ROWS - 1) / SCR_ROWS, H);
+    assign_screen_kernel<T, D><<<g, 256, smem, st>>>((const T *)x, N, rows, seg, cent, cap, cn2, cmax, mode, assign,
+                                                      amb_list, amb_count); note_launch();
+    dim3 g2(64, H);
+    assign_exact_kernel<T, D><<<g2, 256, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, amb_list,
+                                                   amb_count, assign); note_launch();
+}
+
+void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
+              int nrows_max, const float *cent, int cap, float *cn2, float *cmax, const double *norm, int mode,
+              int32_t *assign, int32_t *amb_list, int32_t *amb_count, cudaStream_t st) {
+    cudaMemsetAsync(amb_count, 0, sizeof(int32_t) * H, st);
+    cent_prep_kernel<<<H, 256, 0, st>>>(cent, cap, D, seg, cn2, cmax); note_launch();
+    if (dtype == DT_BF16) {
+        if (D == 64)
+            launch_assign<__nv_bfloat16, 64>(x, H, N, rows, seg, nrows_max, cent, cap, cn2, cmax, norm, mode, assign,
+                                             amb_list, amb_count, st);
+        else
+            launch_assign<__nv_bfloat16, 128>(x, H, N, rows, seg, nrows_max, cent, cap, cn2, cmax, norm, mode,
+                                              assign, amb_list, amb_count, st);
+    } else {
+        if (D == 64)
+            launch_assign<float, 64>(x, H, N, rows, seg, nrows_max, cent, cap, cn2, cmax, norm, mode, assign,
+                                     amb_list, amb_count, st);
+        else
+            launch_assign<float, 128>(x, H, N, rows, seg, nrows_max, cent, cap, cn2, cmax, norm, mode, assign,
+                                      amb_list, amb_count, st);
+    }
+}
+
+void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
+            int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
+            double *dist, cudaStream_t st) {
+    dim3 g((nrows_max + 127) / 128, H);
+#define AC_DIST(T, DD) \
+    dist_kernel<T, DD><<<g, 128, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, assign, dist)
+    if (dtype == DT_BF16) {
+        if (D == 64) AC_DIST(__nv_bfloat16, 64);
+        else AC_DIST(__nv_bfloat16, 128);
+    } else {
+        if (D == 64) AC_DIST(float, 64);
+        else AC_DIST(float, 128);
+    }
+#undef AC_DIST
+    note_launch();
+}
+
+void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg, int kmax, const int32_t *perm,
+              const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st) {
+    dim3 g(kmax, H);
+#define AC_UPD(T, DD) \
+    update_kernel<T, DD><<<g, DD, 0, st>>>((const T *)x, N, seg, perm, off, cap, norm, mode, cent)
+    if (dtype == DT_BF16) {
+        if (D == 64) AC_UPD(__nv_bfloat16, 64);
+        else AC_UPD(__nv_bfloat16, 128);
+    } else {
+        if (D == 64) AC_UPD(float, 64);
+        else AC_UPD(float, 128);
+    }
+#undef AC_UPD
+    note_launch();
+}
+
+void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const int32_t *off, int cap,
+                 const double *norm, float *mean_norm, cudaStream_t st) {
+    dim3 g((cap + 127) / 128, H);
+    mean_norm_kernel<<<g, 128, 0, st>>>(N, seg, perm, off, cap, norm, mean_norm); note_launch();
+}
+
+}  // namespace ac

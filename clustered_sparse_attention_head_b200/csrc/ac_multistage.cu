@@ -1,0 +1,273 @@
+// Device-side control of Algorithm 1 (MultiStageClustering, AdaCluster §3.2.2):
+// per-head stage decisions, the tau rules of the first stage, and the removal
+// of tokens within tau of their centre from the remaining set U.
+//
+// Readings of the algorithm (the paper leaves these open):
+//  - U starts as all tokens; stage t clusters U into m_t clusters with
+//    m_0 = m0 and m_t = min(|U|, ceil(m0 |U| / N)) for t >= 1.
+//  - |C| >= N_max is tested before a stage; then F is set and the loop stops.
+//  - A token of U leaves U when its distance to its centre is < tau.
+//  - tau (MEAN_X / MEDIAN_RADIUS_X) is fixed from the first stage.
+#include "ac_kernels.cuh"
+#include "ac_multistage.cuh"
+
+namespace ac {
+
+__global__ void ms_init_kernel(int H, int N, MsHead *__restrict__ st, int32_t *__restrict__ U) {
+    int h = blockIdx.y;
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < N) U[(size_t)h * N + i] = i;
+    if (i == 0) {
+        MsHead s;
+        s.nc = 0;
+        s.nu = N;
+        s.stage = 0;
+        s.flag = 0;
+        s.mt = 0;
+        s.done = 0;
+        s.tau = 0.0;
+        st[h] = s;
+    }
+}
+
+// Decide the next stage of every head; writes the pass descriptors and a
+// summary {active heads, max |U|, max m_t, max |C|, capacity error} for the host.
+__global__ void ms_control_kernel(int H, int N, int m0, int nmax, int cap, MsHead *__restrict__ st,
+                                  HeadSeg *__restrict__ seg, int32_t *__restrict__ info, int *status) {
+    __shared__ int act, mnu, mmt, mnc, err;
+    if (threadIdx.x == 0) { act = 0; mnu = 0; mmt = 0; mnc = 0; err = 0; }
+    __syncthreads();
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        MsHead s = st[h];
+        HeadSeg g;
+        g.nrows = 0;
+        g.k = 0;
+        g.cent_off = s.nc;
+        g.pad = 0;
+        if (!s.done) {
+            if (s.nu <= 0) {
+                s.done = 1;
+            } else if (s.nc >= nmax) {
+                s.flag = 1;
+                s.done = 1;
+            } else {
+                int mt;
+                if (s.stage == 0) mt = m0;
+                else {
+                    long long num = (long long)m0 * s.nu;
+                    long long c = (num + N - 1) / N;
+                    mt = (int)(c < s.nu ? c : s.nu);
+                }
+                if (mt > s.nu) mt = s.nu;
+                if (s.nc + mt > cap) {
+                    atomicExch(&err, 1);
+                    set_status(status, ST_CAPACITY);
+                    s.done = 1;
+                } else {
+                    s.mt = mt;
+                    g.nrows = s.nu;
+                    g.k = mt;
+                    atomicAdd(&act, 1);
+                    atomicMax(&mnu, s.nu);
+                    atomicMax(&mmt, mt);
+                }
+            }
+        }
+        atomicMax(&mnc, s.nc + (g.nrows > 0 ? s.mt : 0));
+        st[h] = s;
+        seg[h] = g;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        info[0] = act;
+        info[1] = mnu;
+        info[2] = mmt;
+        info[3] = mnc;
+        info[4] = err;
+    }
+}
+
+// tau of the first stage (one CTA per head; positions = tokens at stage 0).
+//  ABS: tau = x.
+//  MEAN_X: x * (sequential sum of distances in token order) / |U|.
+//  MEDIAN_RADIUS_X: x * lower median over non-empty clusters of the
+//  sequential (token-order) mean member distance.
+__global__ void ms_tau_kernel(int N, int rule, double x, const HeadSeg *__restrict__ seg,
+                              const double *__restrict__ dist, const int32_t *__restrict__ perm,
+                              const int32_t *__restrict__ off, int cap, MsHead *__restrict__ st) {
+    extern __shared__ double rad[];  // [n2]
+    __shared__ int nrad;
+    int h = blockIdx.x;
+    HeadSeg g = seg[h];
+    if (g.nrows <= 0 || st[h].stage != 0) return;
+    const double *dh = dist + (size_t)h * N;
+    if (rule == 0) {
+        if (threadIdx.x == 0) st[h].tau = x;
+        return;
+    }
+    if (rule == 1) {
+        if (threadIdx.x == 0) {
+            double s = 0.0;
+            for (int i = 0; i < g.nrows; i++) s = dadd(s, dh[i]);
+            st[h].tau = dmul(x, ddiv(s, (double)g.nrows));
+        }
+        return;
+    }
+    int n2 = 1;
+    while (n2 < g.k) n2 <<= 1;
+    if (threadIdx.x == 0) nrad = 0;
+    __syncthreads();
+    const int32_t *o = off + (size_t)h * (cap + 1);
+    for (int j = threadIdx.x; j < n2; j += blockDim.x) rad[j] = INFINITY;
+    __syncthreads();
+    for (int j = threadIdx.x; j < g.k; j += blockDim.x) {
+        int b = o[j], e = o[j + 1];
+        if (e > b) {
+            double s = 0.0;
+            for (int r = b; r < e; r++) s = dadd(s, dh[perm[(size_t)h * N + r]]);
+            rad[j] = ddiv(s, (double)(e - b));
+            atomicAdd(&nrad, 1);
+        }
+    }
+    __syncthreads();
+    for (int k = 2; k <= n2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+                int l = i ^ j;
+                if (l > i) {
+                    double a = rad[i], b = rad[l];
+                    bool up = (i & k) == 0;
+                    if (up ? (a > b) : (a < b)) { rad[i] = b; rad[l] = a; }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (threadIdx.x == 0) st[h].tau = dmul(x, rad[(nrad - 1) / 2]);
+}
+
+// Keep the positions of U whose distance is not < tau (order preserved), then
+// advance the head's stage: |C| += m_t.  One CTA per head.
+__global__ void ms_remove_kernel(int N, const HeadSeg *__restrict__ seg, const double *__restrict__ dist,
+                                 const int32_t *__restrict__ U, int32_t *__restrict__ Unext, MsHead *__restrict__ st) {
+    __shared__ int wsum[32];
+    __shared__ int base;
+    int h = blockIdx.x;
+    HeadSeg g = seg[h];
+    if (g.nrows <= 0) return;
+    const double tau = st[h].tau;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+    if (tid == 0) base = 0;
+    __syncthreads();
+    for (int p0 = 0; p0 < g.nrows; p0 += blockDim.x) {
+        int pos = p0 + tid;
+        int keep = (pos < g.nrows) && !(dist[(size_t)h * N + pos] < tau);
+        unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) wsum[w] = __popc(bal);
+        __syncthreads();
+        int before = base;
+        for (int u = 0; u < w; u++) before += wsum[u];
+        if (keep) Unext[(size_t)h * N + before + __popc(bal & ((1u << lane) - 1u))] = U[(size_t)h * N + pos];
+        __syncthreads();
+        if (tid == 0) {
+            int t = 0;
+            for (int u = 0; u < nw; u++) t += wsum[u];
+            base += t;
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        MsHead s = st[h];
+        s.nu = base;
+        s.nc += s.mt;
+        s.stage += 1;
+        st[h] = s;
+    }
+}
+
+// Final pass over all tokens with every centre of C; also publishes
+// nclusters and the flag F.
+__global__ void ms_final_kernel(int H, int N, const MsHead *__restrict__ st, HeadSeg *__restrict__ seg,
+                                int32_t *__restrict__ ncl, uint8_t *__restrict__ flag, int32_t *__restrict__ info) {
+    __shared__ int mnc;
+    if (threadIdx.x == 0) mnc = 0;
+    __syncthreads();
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        MsHead s = st[h];
+        HeadSeg g;
+        g.nrows = s.nc > 0 ? N : 0;
+        g.k = s.nc;
+        g.cent_off = 0;
+        g.pad = 0;
+        seg[h] = g;
+        if (ncl) ncl[h] = s.nc;
+        if (flag) flag[h] = (uint8_t)s.flag;
+        atomicMax(&mnc, s.nc);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) info[5] = mnc;
+}
+
+__global__ void seg_uniform_kernel(int H, int nrows, int k, HeadSeg *__restrict__ seg, int32_t *__restrict__ ncl,
+                                   uint8_t *__restrict__ flag) {
+    int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    HeadSeg g;
+    g.nrows = nrows;
+    g.k = k;
+    g.cent_off = 0;
+    g.pad = 0;
+    seg[h] = g;
+    if (ncl) ncl[h] = k;
+    if (flag) flag[h] = 0;
+}
+
+// Per-head pass descriptors from device cluster counts (nk may be NULL).
+__global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restrict__ ncl, int kfix,
+                                       HeadSeg *__restrict__ seg) {
+    int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    HeadSeg g;
+    g.nrows = nrows;
+    g.k = ncl ? ncl[h] : kfix;
+    g.cent_off = 0;
+    g.pad = 0;
+    seg[h] = g;
+}
+
+void k_ms_init(int H, int N, MsHead *st, int32_t *U, cudaStream_t s) {
+    dim3 g((N + 255) / 256, H);
+    ms_init_kernel<<<g, 256, 0, s>>>(H, N, st, U); note_launch();
+}
+void k_ms_control(int H, int N, int m0, int nmax, int cap, MsHead *st, HeadSeg *seg, int32_t *info, int *status,
+                  cudaStream_t s) {
+    ms_control_kernel<<<1, 256, 0, s>>>(H, N, m0, nmax, cap, st, seg, info, status); note_launch();
+}
+void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double *dist, const int32_t *perm,
+              const int32_t *off, int cap, int kmax, MsHead *st, cudaStream_t s) {
+    int n2 = 1;
+    while (n2 < kmax) n2 <<= 1;
+    size_t smem = (size_t)n2 * sizeof(double);
+    static size_t smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+        cudaFuncSetAttribute(ms_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        smem_set = smem;
+    }
+    ms_tau_kernel<<<H, 256, smem, s>>>(N, rule, x, seg, dist, perm, off, cap, st); note_launch();
+}
+void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int32_t *U, int32_t *Unext, MsHead *st,
+                 cudaStream_t s) {
+    ms_remove_kernel<<<H, 1024, 0, s>>>(N, seg, dist, U, Unext, st); note_launch();
+}
+void k_ms_final(int H, int N, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
+                cudaStream_t s) {
+    ms_final_kernel<<<1, 256, 0, s>>>(H, N, st, seg, ncl, flag, info); note_launch();
+}
+void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s) {
+    seg_uniform_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, k, seg, ncl, flag); note_launch();
+}
+void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s) {
+    seg_from_counts_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, ncl, kfix, seg); note_launch();
+}
+
+}  // namespace ac

@@ -1,0 +1,29 @@
+// Algorithm 1 per-head state and launchers (see ac_multistage.cu).
+#pragma once
+#include "ac_common.cuh"
+
+namespace ac {
+
+struct MsHead {
+    int nc;      // |C|: clusters created so far
+    int nu;      // |U|: tokens still to be clustered
+    int stage;   // t
+    int flag;    // F
+    int mt;      // m_t of the stage in progress
+    int done;
+    double tau;
+};
+
+void k_ms_init(int H, int N, MsHead *st, int32_t *U, cudaStream_t s);
+void k_ms_control(int H, int N, int m0, int nmax, int cap, MsHead *st, HeadSeg *seg, int32_t *info, int *status,
+                  cudaStream_t s);
+void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double *dist, const int32_t *perm,
+              const int32_t *off, int cap, int kmax, MsHead *st, cudaStream_t s);
+void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int32_t *U, int32_t *Unext, MsHead *st,
+                 cudaStream_t s);
+void k_ms_final(int H, int N, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
+                cudaStream_t s);
+void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s);
+void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s);
+
+}  // namespace ac

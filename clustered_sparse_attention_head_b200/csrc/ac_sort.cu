@@ -1,0 +1,172 @@
+// Cluster-sort permutation and gather (Algorithm 3 line 8, "K* = K[Index]"):
+// a stable counting sort of tokens by cluster id, so every cluster's tokens are
+// contiguous and in increasing token order, then a 16-byte vectorised row
+// gather into cluster order.
+//
+// Stable ranks: each warp owns a tile of 256 positions and walks it in order,
+// 32 at a time; __match_any_sync groups equal ids within the 32 and a
+// shared-memory counter per id gives each position its rank among equal ids
+// of the tile.  Tile histograms are then scanned per cluster (over tiles) and
+// per head (over clusters) to place every position.
+#include "ac_kernels.cuh"
+
+namespace ac {
+
+__global__ void rank_hist_kernel(const int32_t *__restrict__ ids, const HeadSeg *__restrict__ seg, int N,
+                                 int cap, int ntiles_max, int32_t *__restrict__ rank, int32_t *__restrict__ hist,
+                                 int *status) {
+    extern __shared__ int32_t sh[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    HeadSeg s = seg[h];
+    const int tile = blockIdx.x * 4 + warp;
+    const int base = tile * SORT_TILE;
+    int32_t *cnt = sh + warp * cap;
+    if (base >= s.nrows || tile >= ntiles_max) return;
+    for (int j = lane; j < s.k; j += 32) cnt[j] = 0;
+    __syncwarp();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c = 0; c < SORT_TILE; c += 32) {
+        int pos = base + c + lane;
+        bool valid = pos < s.nrows;
+        int id = valid ? ids[(size_t)h * N + pos] : -1;
+        if (valid && (id < 0 || id >= s.k)) {
+            set_status(status, 1);
+            id = -1;
+            valid = false;
+        }
+        unsigned m = __match_any_sync(0xffffffffu, id);
+        int r = 0;
+        if (valid) r = cnt[id] + __popc(m & lt);
+        __syncwarp();
+        if (valid && lane == __ffs(m) - 1) cnt[id] += __popc(m);
+        __syncwarp();
+        if (valid) rank[(size_t)h * N + pos] = r;
+    }
+    int32_t *hh = hist + ((size_t)h * ntiles_max + tile) * cap;
+    for (int j = lane; j < s.k; j += 32) hh[j] = cnt[j];
+}
+
+// Per cluster j: exclusive scan over tiles (in place) and the cluster size.
+__global__ void scan_tiles_kernel(const HeadSeg *__restrict__ seg, int cap, int ntiles_max,
+                                  int32_t *__restrict__ hist, int32_t *__restrict__ cnt) {
+    int h = blockIdx.y;
+    int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= cap) return;
+    HeadSeg s = seg[h];
+    int run = 0;
+    if (j < s.k && s.nrows > 0) {
+        int nt = (s.nrows + SORT_TILE - 1) / SORT_TILE;
+        int32_t *p = hist + (size_t)h * ntiles_max * cap + j;
+        for (int t = 0; t < nt; t++) {
+            int v = p[(size_t)t * cap];
+            p[(size_t)t * cap] = run;
+            run += v;
+        }
+    }
+    cnt[(size_t)h * cap + j] = run;
+}
+
+// Per head: exclusive scan of cluster sizes -> offsets [cap + 1].
+__global__ void scan_clusters_kernel(const int32_t *__restrict__ cnt, int cap, int32_t *__restrict__ off) {
+    __shared__ int32_t warp_tot[32];
+    __shared__ int32_t carry;
+    int h = blockIdx.x;
+    const int32_t *c = cnt + (size_t)h * cap;
+    int32_t *o = off + (size_t)h * (cap + 1);
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int b = 0; b < cap; b += blockDim.x) {
+        int j = b + threadIdx.x;
+        int v = j < cap ? c[j] : 0;
+        int x = v;
+        int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        for (int d = 1; d < 32; d <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        if (lane == 31) warp_tot[w] = x;
+        __syncthreads();
+        if (w == 0) {
+            int nw = blockDim.x >> 5;
+            int t = lane < nw ? warp_tot[lane] : 0;
+            for (int d = 1; d < 32; d <<= 1) {
+                int y = __shfl_up_sync(0xffffffffu, t, d);
+                if (lane >= d) t += y;
+            }
+            if (lane < nw) warp_tot[lane] = t;
+        }
+        __syncthreads();
+        int incl = x + (w > 0 ? warp_tot[w - 1] : 0) + carry;
+        if (j < cap) o[j] = incl - v;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = incl;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) o[cap] = carry;
+}
+
+__global__ void scatter_kernel(const int32_t *__restrict__ ids, const int32_t *__restrict__ rows,
+                               const HeadSeg *__restrict__ seg, int N, int cap, int ntiles_max,
+                               const int32_t *__restrict__ rank, const int32_t *__restrict__ hist,
+                               const int32_t *__restrict__ off, int32_t *__restrict__ perm) {
+    int h = blockIdx.y;
+    HeadSeg s = seg[h];
+    int pos = blockIdx.x * blockDim.x + threadIdx.x;
+    if (pos >= s.nrows) return;
+    int id = ids[(size_t)h * N + pos];
+    if (id < 0 || id >= s.k) return;
+    int tile = pos / SORT_TILE;
+    int p = off[(size_t)h * (cap + 1) + id] + hist[((size_t)h * ntiles_max + tile) * cap + id] +
+            rank[(size_t)h * N + pos];
+    perm[(size_t)h * N + p] = rows ? rows[(size_t)h * N + pos] : pos;
+}
+
+size_t sort_hist_elems(int H, int N, int cap) {
+    size_t nt = (size_t)(N + SORT_TILE - 1) / SORT_TILE;
+    return (size_t)H * nt * cap;
+}
+
+void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, int N, int nrows_max, int cap,
+            int32_t *rank, int32_t *hist, int32_t *cnt, int32_t *off, int32_t *perm, int *status, cudaStream_t st) {
+    int ntiles_max = (N + SORT_TILE - 1) / SORT_TILE;
+    int nt = (nrows_max + SORT_TILE - 1) / SORT_TILE;
+    size_t smem = (size_t)4 * cap * sizeof(int32_t);
+    static size_t smem_set = 0;
+    if (smem > 48 * 1024 && smem > smem_set) {
+        cudaFuncSetAttribute(rank_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        smem_set = smem;
+    }
+    if (nt > 0) {
+        dim3 g1((nt + 3) / 4, H);
+        rank_hist_kernel<<<g1, 128, smem, st>>>(ids, seg, N, cap, ntiles_max, rank, hist, status); note_launch();
+    }
+    dim3 g2((cap + 127) / 128, H);
+    scan_tiles_kernel<<<g2, 128, 0, st>>>(seg, cap, ntiles_max, hist, cnt); note_launch();
+    scan_clusters_kernel<<<H, 1024, 0, st>>>(cnt, cap, off); note_launch();
+    if (nrows_max > 0) {
+        dim3 g3((nrows_max + 255) / 256, H);
+        scatter_kernel<<<g3, 256, 0, st>>>(ids, rows, seg, N, cap, ntiles_max, rank, hist, off, perm); note_launch();
+    }
+}
+
+// dst[h, p, :] = src[h, perm[h, p], :], 16 bytes per thread.
+__global__ void gather_rows_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst,
+                                   const int32_t *__restrict__ perm, int N, int vec_per_row) {
+    int h = blockIdx.y;
+    size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    size_t tot = (size_t)N * vec_per_row;
+    if (idx >= tot) return;
+    int p = (int)(idx / vec_per_row), v = (int)(idx - (size_t)p * vec_per_row);
+    int tok = perm[(size_t)h * N + p];
+    dst[((size_t)h * N + p) * vec_per_row + v] = src[((size_t)h * N + tok) * vec_per_row + v];
+}
+
+void k_gather_rows(const void *src, void *dst, const int32_t *perm, int H, int N, int row_bytes, cudaStream_t st) {
+    int vpr = row_bytes / 16;
+    size_t tot = (size_t)N * vpr;
+    dim3 g((unsigned)((tot + 255) / 256), H);
+    gather_rows_kernel<<<g, 256, 0, st>>>((const uint4 *)src, (uint4 *)dst, perm, N, vpr); note_launch();
+}
+
+}  // namespace ac

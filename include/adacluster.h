@@ -1,0 +1,206 @@
+/*
+ * adacluster.h -- C ABI of libadacluster.so, a CUDA (sm_100a) implementation of
+ * the AdaCluster clustered sparse attention hot path.
+ *
+ * Method: "AdaCluster: Adaptive Query-Key Clustering for Sparse Attention in
+ * Video Generation" (Tan et al., arXiv 2604.18348), Algorithm 3 (§3.3):
+ *   A_q, C_q    <- KMeans(Normalize(Q))                         (§3.1)
+ *   A_k, C_k, F <- MultiStageClustering(K, tau, N_max)          (§3.2.2, Algorithm 1)
+ *   F ? dense attention : attention over the selected key clusters only.
+ * Cluster selection uses centroid-centroid scores weighted by key-cluster size
+ * with a top-p cut (the centroid-based significance estimate of §2.3).
+ *
+ * Conventions shared by every call
+ *  - Every function returns ac_status.  Argument errors are detected on the host
+ *    and returned synchronously; nothing is launched in that case.
+ *  - Work is enqueued asynchronously on the given CUDA stream (cudaStream_t
+ *    passed as void*; NULL = legacy default stream).  Device-side errors (a
+ *    bounded wait that timed out, a non-finite input, a capacity overflow) set a
+ *    status word inside the context; ac_get_status() synchronises the stream and
+ *    returns and clears it.
+ *  - All tensor pointers are caller-owned DEVICE memory.  The library allocates
+ *    device memory only in ac_create (a small status block); every other buffer,
+ *    including the scratch workspace `ws`, is passed in.  Pointers must be
+ *    16-byte aligned; tensors are dense row-major.
+ *  - Layouts (H = heads, N = tokens, d = head dim in {64, 128}):
+ *      q, k, v, out   [H, N, d]   element type = config dtype (fp32 or bf16)
+ *      assign         [H, N]      int32 cluster id of each token
+ *      cent           [H, cap, d] fp32 centroids
+ *      count          [H, cap]    int32 members per cluster
+ *      mean_norm      [H, kq_cap] fp32 mean ||q|| over a query cluster's members
+ *      nclusters      [H]         int32 clusters in use (== kq/kk unless adaptive)
+ *      dense_flag     [H]         uint8 1 = head takes dense attention (flag F)
+ *      sel_idx        [H, kq_cap, kk_cap] int32 selected key-cluster ids, ascending
+ *      sel_cnt        [H, kq_cap] int32 number of selected key clusters
+ *    with cap = kq_cap for queries and kk_cap for keys (ac_capacities()).
+ *  - Cluster ids are int32; ties in every argmin/argmax go to the lowest id.
+ *  - Concurrent calls on one context must not overlap on the GPU: the context's
+ *    status word and the workspace are shared by the calls that use them.
+ */
+#ifndef ADACLUSTER_H
+#define ADACLUSTER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AC_API __attribute__((visibility("default")))
+#else
+#define AC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AC_OK = 0,
+    AC_ERR_INVALID_ARG = 1,  /* bad pointer, shape, or parameter              */
+    AC_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not 64/128) */
+    AC_ERR_CUDA = 3,         /* a CUDA runtime call failed                    */
+    AC_ERR_WORKSPACE = 4,    /* workspace pointer NULL or too small           */
+    AC_ERR_TIMEOUT = 5,      /* a bounded device wait expired                 */
+    AC_ERR_NONFINITE = 6,    /* NaN or Inf in an input                        */
+    AC_ERR_CAPACITY = 7      /* adaptive clustering outgrew its capacity      */
+} ac_status;
+
+typedef enum { AC_F32 = 0, AC_BF16 = 1 } ac_dtype;
+
+/* How tau of Algorithm 1 is obtained.  ABS: tau = tau_value.  MEAN_X: tau =
+ * tau_value x the mean token-to-centre distance of the first stage (§4.1 uses
+ * 1.5).  MEDIAN_RADIUS_X: tau = tau_value x the lower median, over non-empty
+ * first-stage clusters, of the mean member-to-centre distance.              */
+typedef enum { AC_TAU_ABS = 0, AC_TAU_MEAN_X = 1, AC_TAU_MEDIAN_RADIUS_X = 2 } ac_tau_rule;
+
+/* ac_config.flags */
+#define AC_FLAG_WARM_START 1u    /* ac_forward: seed k-means from q_cent_io/k_cent_io */
+#define AC_FLAG_CHECK_FINITE 2u  /* scan inputs for NaN/Inf (AC_ERR_NONFINITE)        */
+#define AC_FLAG_PROFILE 4u       /* ac_forward records per-stage CUDA events (no sync);
+                                    read them with ac_profile_read                     */
+
+typedef struct {
+    int heads, n, d;        /* H, N, d (d in {64, 128}); batch is folded into heads   */
+    ac_dtype dtype;         /* element type of q, k, v and out                         */
+    int kq, kk;             /* cluster counts, or the first-stage count m0 if adaptive */
+    int iters;              /* k-means iterations (assign + update) per stage          */
+    int adaptive_q;         /* 1 = Algorithm 1 on normalised queries                   */
+    int adaptive_k;         /* 1 = Algorithm 1 on keys                                 */
+    ac_tau_rule tau_rule;
+    double tau_value;
+    int nmax_q, nmax_k;     /* Algorithm 1's N_max for queries / keys                  */
+    double top_p;           /* (0, 1]; >= 1 keeps every non-empty key cluster          */
+    unsigned flags;
+} ac_config;
+
+/* Per-call statistics filled by ac_forward when `stats` is non-NULL (the call
+ * then synchronises the stream before returning). */
+typedef struct {
+    double ms_cluster_q, ms_cluster_k, ms_select, ms_sort, ms_attn, ms_total;
+    int64_t pairs;          /* (query, key) pairs the attention computed, all heads   */
+    int dense_heads;        /* heads that took dense attention                        */
+    int max_stages_q, max_stages_k;
+} ac_stats;
+
+/* Averages over the ac_forward calls recorded with AC_FLAG_PROFILE since the
+ * last ac_profile_read (at most the last 256 calls). */
+typedef struct {
+    int calls;
+    double ms_cluster_q, ms_cluster_k, ms_select;
+    double ms_prep;          /* cluster sort, gather and work list of the attention */
+    double ms_attn_kernel;   /* the block-sparse attention kernel alone             */
+    double ms_total;
+    long long launches;      /* kernels this library launched since the last read   */
+} ac_profile;
+
+typedef struct ac_ctx ac_ctx;
+
+/* Create a context for one problem shape.  Validates the configuration and
+ * allocates the context's small device status block.  *out = NULL on error.  */
+AC_API ac_status ac_create(const ac_config *cfg, ac_ctx **out);
+AC_API void ac_destroy(ac_ctx *ctx);
+
+/* Capacities of the cluster dimension: kq/kk, or N_max + m0 in adaptive mode
+ * (Algorithm 1 tests |C| >= N_max before a stage, so the last stage may add up
+ * to m0 clusters beyond N_max). */
+AC_API ac_status ac_capacities(const ac_ctx *ctx, int *kq_cap, int *kk_cap);
+
+/* Bytes of scratch workspace that every call below needs (one size for all). */
+AC_API ac_status ac_workspace_size(const ac_ctx *ctx, size_t *bytes);
+
+/* Query clustering (§3.1, Algorithm 3 line 1): q_hat = q/||q|| (zero stays
+ * zero), then spherical k-means: assign each q_hat to the centroid of largest
+ * q_hat.mu (equivalently the closest unit centroid), update mu_j = s_j/||s_j||
+ * with s_j the member sum (empty clusters keep their centroid); `iters`
+ * rounds, then a final assignment.  With adaptive_q, Algorithm 1 runs on q_hat
+ * with the chordal distance.  Initial centroids: init_cent [H, kq, d] if non-NULL,
+ * else q_hat of tokens floor(j*N/kq).  Outputs assign, cent, count, mean_norm,
+ * nclusters, dense_flag (any may not be NULL).                              */
+AC_API ac_status ac_cluster_q(ac_ctx *ctx, const void *q, const float *init_cent, int32_t *assign,
+                       float *cent, int32_t *count, float *mean_norm, int32_t *nclusters,
+                       uint8_t *dense_flag, void *ws, size_t ws_bytes, void *stream);
+
+/* Key clustering (§3.2.1; Algorithm 1 of §3.2.2 when adaptive_k): Euclidean
+ * k-means, assign by smallest ||k - c||^2, update c_j = member mean.  Same
+ * initialisation, iteration and output rules as ac_cluster_q.              */
+AC_API ac_status ac_cluster_k(ac_ctx *ctx, const void *k, const float *init_cent, int32_t *assign,
+                       float *cent, int32_t *count, int32_t *nclusters, uint8_t *dense_flag,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* Critical-cluster selection.  For each non-empty query cluster a of a head
+ * whose dense_flag is 0:
+ *   s_ab = mean_norm_a * (mu_a . c_b) / sqrt(d)  over non-empty key clusters b,
+ *   p_ab = count_b exp(s_ab - max_b s_ab) / sum_b (...),
+ * then key clusters are taken in decreasing p (ties: lower b) until the taken
+ * mass reaches top_p.  sel_idx lists them in ascending id.  Empty query
+ * clusters and dense heads get sel_cnt = 0.  nq/nk/dense_flag may be NULL
+ * (then kq/kk and 0 are used).                                              */
+AC_API ac_status ac_select(ac_ctx *ctx, const float *q_cent, const float *q_mean_norm,
+                    const int32_t *q_count, const float *k_cent, const int32_t *k_count,
+                    const int32_t *nq, const int32_t *nk, const uint8_t *dense_flag,
+                    int32_t *sel_idx, int32_t *sel_cnt, void *ws, size_t ws_bytes, void *stream);
+
+/* Stable counting sort of token ids by cluster id (per head): perm [H, N]
+ * lists tokens of cluster 0 in increasing token order, then cluster 1, ...;
+ * offsets [H, cap + 1] holds each cluster's first position and offsets[cap]
+ * = N (clusters >= nclusters are empty).  ncl may be NULL (then cap).       */
+AC_API ac_status ac_cluster_sort(ac_ctx *ctx, const int32_t *assign, int cap, const int32_t *ncl,
+                          int32_t *perm, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
+
+/* Exact softmax attention over the selected key clusters (Algorithm 3 lines
+ * 8-9; line 4 for heads with dense_flag = 1):
+ *   out_i = sum_{j: assign_k(j) in S(assign_q(i))} softmax_j(q_i.k_j / sqrt(d)) v_j.
+ * Tokens are gathered into cluster order internally; rows are written back in
+ * token order.  A query whose selected set is empty gets zeros.  lse [H, N]
+ * (natural-log log-sum-exp of the scaled scores) is written when non-NULL.
+ * nq/nk/dense_flag may be NULL.  Computes in bf16 (fp32 accumulation) for bf16
+ * inputs and in tf32 (fp32 accumulation) for fp32 inputs.                   */
+AC_API ac_status ac_sparse_attn(ac_ctx *ctx, const void *q, const void *k, const void *v,
+                         const int32_t *q_assign, const int32_t *k_assign, const int32_t *sel_idx,
+                         const int32_t *sel_cnt, const int32_t *nq, const int32_t *nk,
+                         const uint8_t *dense_flag, void *out, float *lse, void *ws,
+                         size_t ws_bytes, void *stream);
+
+/* The whole of Algorithm 3 for every head: ac_cluster_q, ac_cluster_k,
+ * ac_select, ac_sparse_attn.  q_cent_io / k_cent_io ([H, cap, d], nullable):
+ * with AC_FLAG_WARM_START they seed k-means (§3.2.2 "Efficient
+ * initialization"); when non-NULL they receive the final centroids.
+ * Adaptive clustering reads one int per head back to the host per stage; the
+ * fixed-count path never synchronises unless `stats` is non-NULL.          */
+AC_API ac_status ac_forward(ac_ctx *ctx, const void *q, const void *k, const void *v, float *q_cent_io,
+                     float *k_cent_io, void *out, ac_stats *stats, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/* Wait for the recorded events, fill *out (averages per call) and reset the
+ * record.  Events are recorded on the stream each ac_forward call used. */
+AC_API ac_status ac_profile_read(ac_ctx *ctx, ac_profile *out);
+
+/* Synchronise `stream`, return the first device-side error recorded since the
+ * last call (AC_OK if none) and clear it. */
+AC_API ac_status ac_get_status(ac_ctx *ctx, void *stream);
+
+AC_API const char *ac_status_string(ac_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ADACLUSTER_H */

@@ -1,0 +1,75 @@
+"""The C-ABI library loads on a machine without a GPU and exports every entry
+point that include/adacluster.h declares; the product package never imports
+the oracle."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "adacluster.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ac_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from clustered_sparse_attention_head_b200 import build
+    path = build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for n in ["ac_cluster_q", "ac_cluster_k", "ac_select", "ac_sparse_attn", "ac_forward"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from clustered_sparse_attention_head_b200 import _abi
+    names = declared()
+    assert sorted(_abi.EXPORTS) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    lib.ac_status_string.restype = ctypes.c_char_p
+    for code in range(8):
+        s = lib.ac_status_string(code).decode()
+        assert s and s != "unknown status"
+
+
+def test_nothing_but_declared_symbols_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True).stdout
+    syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert {s for s in syms if s.startswith("ac_")} == set(declared())
+
+
+def test_create_rejects_bad_config_without_launching(lib):
+    from clustered_sparse_attention_head_b200 import _abi
+    L = _abi.load()
+    ctx = ctypes.c_void_p()
+    bad = _abi.ac_config(1, 100, 96, 1, 4, 4, 1, 0, 0, 0, 0.0, 0, 0, 0.9, 0)   # d = 96
+    assert L.ac_create(ctypes.byref(bad), ctypes.byref(ctx)) == _abi.AC_ERR_UNSUPPORTED
+    bad = _abi.ac_config(1, 100, 64, 1, 0, 4, 1, 0, 0, 0, 0.0, 0, 0, 0.9, 0)   # kq = 0
+    assert L.ac_create(ctypes.byref(bad), ctypes.byref(ctx)) == _abi.AC_ERR_INVALID_ARG
+    bad = _abi.ac_config(1, 100, 64, 1, 4, 4, 1, 0, 0, 0, 0.0, 0, 0, 0.0, 0)   # top_p = 0
+    assert L.ac_create(ctypes.byref(bad), ctypes.byref(ctx)) == _abi.AC_ERR_INVALID_ARG
+    bad = _abi.ac_config(1, 100, 64, 1, 4, 4, 1, 0, 1, 0, 0.0, 0, 0, 0.9, 0)   # adaptive, nmax 0
+    assert L.ac_create(ctypes.byref(bad), ctypes.byref(ctx)) == _abi.AC_ERR_INVALID_ARG
+    assert not ctx.value
+
+
+def test_product_does_not_import_oracle():
+    code = ("import sys; import clustered_sparse_attention_head_b200 as p; "
+            "from clustered_sparse_attention_head_b200 import api, _abi; "
+            "assert 'oracle' not in sys.modules, 'oracle imported'")
+    subprocess.check_call([sys.executable, "-c", code], cwd=ROOT)
