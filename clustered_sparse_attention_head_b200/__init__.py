@@ -7,7 +7,7 @@ from . import workloads  # noqa: F401
 
 
 def build(force: bool = False) -> str:
-    from .build import build as _b
+    from ._build import build as _b
     return _b(force=force)
 
 
