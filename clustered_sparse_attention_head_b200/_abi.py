@@ -22,7 +22,7 @@ AC_FLAG_WARM_START, AC_FLAG_CHECK_FINITE, AC_FLAG_PROFILE = 1, 2, 4
 
 # every entry point declared in include/adacluster.h
 EXPORTS = ["ac_create", "ac_destroy", "ac_capacities", "ac_workspace_size", "ac_cluster_q", "ac_cluster_k",
-           "ac_select", "ac_cluster_sort", "ac_sparse_attn", "ac_forward", "ac_profile_read", "ac_get_status",
+           "ac_select", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_profile_read", "ac_get_status",
            "ac_status_string"]
 
 
@@ -72,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ac_cluster_k": ([P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_select": ([P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_cluster_sort": ([P, P, c_int, P, P, P, P, c_size_t, P], c_int),
+        "ac_cluster_sort_static": ([P, c_int, c_int, c_int, P, P, P, P], c_int),
         "ac_sparse_attn": ([P, P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_forward": ([P, P, P, P, P, P, P, POINTER(ac_stats), P, c_size_t, P], c_int),
         "ac_profile_read": ([P, POINTER(ac_profile)], c_int),

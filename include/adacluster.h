@@ -166,6 +166,29 @@ AC_API ac_status ac_select(ac_ctx *ctx, const float *q_cent, const float *q_mean
 AC_API ac_status ac_cluster_sort(ac_ctx *ctx, const int32_t *assign, int cap, const int32_t *ncl,
                           int32_t *perm, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
 
+/* Allocation-free cluster sort.  The paper has no counterpart: this is a
+ * convenience for callers that cannot allocate device memory where they need
+ * the sort.  Examples are an engine plugin limited to memory reserved before
+ * execution, or a host loop whose memory budget is fixed at start-up.
+ * Same result as ac_cluster_sort (assign [heads, n], ncl [heads] or NULL,
+ * perm [heads, n], offsets [heads, cap + 1]), but no context, no workspace,
+ * and no cudaMalloc/cudaFree or other allocating call.
+ *  - Scratch is a 16 MiB array in the library's own device memory; every GPU
+ *    that loads the library holds it until the process exits.  A problem
+ *    needs 256 + 16*heads + 4*heads*n + 4*heads*cap + 4*heads*ceil(n/256)*cap
+ *    bytes (each term rounded up to 256); larger problems, or cap > 8192,
+ *    return AC_ERR_UNSUPPORTED without launching anything.
+ *  - The first call on each device looks up that device's address of the
+ *    array (cudaGetSymbolAddress, with the device current); make that first
+ *    call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents;
+ *    calls that overlap on the GPU (different streams without ordering) race,
+ *    so order them.
+ *  - ids outside [0, ncl[h]) are skipped and leave their perm slots unwritten.
+ * Returns AC_ERR_INVALID_ARG for NULL pointers or non-positive sizes.         */
+AC_API ac_status ac_cluster_sort_static(const int32_t *assign, int heads, int n, int cap, const int32_t *ncl,
+                                        int32_t *perm, int32_t *offsets, void *stream);
+
 /* Exact softmax attention over the selected key clusters (Algorithm 3 lines
  * 8-9; line 4 for heads with dense_flag = 1):
  *   out_i = sum_{j: assign_k(j) in S(assign_q(i))} softmax_j(q_i.k_j / sqrt(d)) v_j.
