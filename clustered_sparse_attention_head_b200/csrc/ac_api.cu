@@ -60,6 +60,9 @@ struct Ws {
     size_t qa, ka, qc, kc, qcount, kcount, qmn, nq, nk, dq, dk, sel, selc;
     // attention
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
+    // tensor-core screen: split centroids and per-stage gathered rows
+    size_t chi, clo, xu;
+    int kpad;
     size_t total;
 };
 
@@ -112,6 +115,10 @@ Ws layout(const ac_ctx *c) {
     w.cnt2 = b.take(H * capm * 4);
     w.segq = b.take(H * sizeof(HeadSeg));
     w.segk = b.take(H * sizeof(HeadSeg));
+    w.kpad = (int)((capm + 127) / 128 * 128);
+    w.chi = b.take(H * (size_t)w.kpad * D * 2);
+    w.clo = b.take(H * (size_t)w.kpad * D * 2);
+    w.xu = b.take(HN * D * c->elt);
     w.total = b.off;
     return w;
 }
@@ -145,6 +152,35 @@ ac_status check_ws(const ac_ctx *c, void *ws, size_t ws_bytes) {
     return AC_OK;
 }
 
+// One assignment step: tensor-core screen for bf16 inputs (rows of the pass
+// contiguous in xc), fp32 screen otherwise; the exact pass resolves near-ties.
+ac_status assign_step(ac_ctx *c, const Ws &w, void *ws, const void *x, const void *xc, const int32_t *rows,
+                      const HeadSeg *seg, int nrows_max, const float *cent, int cap, int mode, int32_t *assign,
+                      cudaStream_t st) {
+    const ac_config &g = c->cfg;
+    const int H = g.heads, N = g.n, D = g.d;
+    float *cn2 = at<float>(ws, w.cn2), *cmax = at<float>(ws, w.cmax);
+    int32_t *amb = at<int32_t>(ws, w.amb), *ambc = at<int32_t>(ws, w.ambc);
+    const double *norm = at<double>(ws, w.norm);
+    if (g.dtype == AC_BF16) {
+        AC_CUDA(cudaMemsetAsync(ambc, 0, sizeof(int32_t) * H, st));
+        if (k_assign_tc(xc, H, N, D, rows, seg, nrows_max, cent, cap, w.kpad, at<void>(ws, w.chi),
+                        at<void>(ws, w.clo), cn2, cmax, norm, mode, assign, amb, ambc, c->d_status, c->encode_fn,
+                        st) != 0)
+            return AC_ERR_CUDA;
+        k_assign_exact(x, DT_BF16, H, N, D, rows, seg, cent, cap, norm, mode, amb, ambc, assign, st);
+    } else {
+        k_assign(x, DT_F32, H, N, D, rows, seg, nrows_max, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+    }
+    return AC_OK;
+}
+
+#define AC_TRY(expr)                   \
+    do {                               \
+        ac_status s_ = (expr);         \
+        if (s_ != AC_OK) return s_;    \
+    } while (0)
+
 // ------------------------------------------------------ clustering driver
 // One k-means run per head (fixed count) or Algorithm 1 (adaptive), all heads
 // batched in every launch.
@@ -175,11 +211,11 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         if (init) AC_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * H * cap * D, cudaMemcpyDeviceToDevice, st));
         else k_init_cent(x, dt, H, N, D, nullptr, norm, seg, k, mode, cent, cap, st);
         for (int it = 0; it < g.iters; it++) {
-            k_assign(x, dt, H, N, D, nullptr, seg, N, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+            AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
             k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, cnt, off, perm, status, st);
             k_update(x, dt, H, N, D, seg, k, perm, off, cap, norm, mode, cent, st);
         }
-        k_assign(x, dt, H, N, D, nullptr, seg, N, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+        AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
         k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
         if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
         if (max_stages) *max_stages = 1;
@@ -190,7 +226,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
     int32_t *pa = at<int32_t>(ws, w.passign);
     double *dist = at<double>(ws, w.dist);
     MsHead *ms = at<MsHead>(ws, w.ms);
-    k_ms_init(H, N, ms, U, st);
+    k_ms_init(H, N, ms, U, Un, st);
     int stages = 0;
     for (int t = 0;; t++) {
         k_ms_control(H, N, k, nmax, cap, ms, seg, c->d_info, status, st);
@@ -201,12 +237,14 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         const int mnu = c->h_info[1], mmt = c->h_info[2];
         stages = t + 1;
         k_init_cent(x, dt, H, N, D, U, norm, seg, mmt, mode, cent, cap, st);
+        void *xu = at<void>(ws, w.xu);
+        if (dt == DT_BF16) k_gather_rows(x, xu, U, H, N, D * c->elt, st);
         for (int it = 0; it < g.iters; it++) {
-            k_assign(x, dt, H, N, D, U, seg, mnu, cent, cap, cn2, cmax, norm, mode, pa, amb, ambc, st);
+            AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
             k_sort(pa, U, seg, H, N, mnu, cap, rank, hist, cnt, off, perm, status, st);
             k_update(x, dt, H, N, D, seg, mmt, perm, off, cap, norm, mode, cent, st);
         }
-        k_assign(x, dt, H, N, D, U, seg, mnu, cent, cap, cn2, cmax, norm, mode, pa, amb, ambc, st);
+        AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
         k_dist(x, dt, H, N, D, U, seg, mnu, cent, cap, norm, mode, pa, dist, st);
         if (t == 0) {
             if (g.tau_rule == AC_TAU_MEDIAN_RADIUS_X)
@@ -220,7 +258,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         AC_CUDA(cudaGetLastError());
     }
     k_ms_final(H, N, ms, seg, ncl, flag, c->d_info, st);
-    k_assign(x, dt, H, N, D, nullptr, seg, N, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
+    AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
     k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
     if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
     if (max_stages) *max_stages = stages;

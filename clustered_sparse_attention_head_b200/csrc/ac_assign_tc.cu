@@ -1,0 +1,323 @@
+// Tensor-core screening pass of the k-means assignment (AdaCluster §3.1 and
+// §3.2.1: queries to the centroid of largest q_hat.mu, keys to the closest
+// centroid) for bf16 inputs on sm_100a.
+//
+// Each fp32 centroid is split into two bf16 parts, c = c_hi + c_lo + r with
+// |r| <= 2^-18 |c| elementwise, and the CTA computes X (C_hi + C_lo)^T for a
+// 128-row tile of X against 128-centroid chunks with tcgen05.mma (both parts
+// accumulate into one fp32 TMEM tile; bf16 x bf16 products are exact).  The
+// four epilogue warps (one row per thread) read the tile from TMEM and keep
+// each row's best score, its index and the second-best score:
+//   EUCLID: ||c||^2 - 2 x.c        SPHERE: -(x.mu)   (smaller is closer)
+// Error bound of a dot product: |x.r| <= 2^-18 ||x|| ||c|| plus fp32
+// accumulation of 2d exact products, <= 2d 2^-23 ||x|| ||c||; the pass uses
+// E_dot = 2^-13 ||x|| Cmax (>= 2x that bound for d <= 128).  A row whose best
+// two scores are within 2E goes to the exact double pass (assign_exact_kernel),
+// so the final decision equals the exact one.
+//
+// Warp 0 issues TMA (X tile once, then C_hi/C_lo chunks), lane 0 of warp 1
+// issues the MMAs into two TMEM accumulators (double buffer), warps 2-5 run
+// the epilogue.  All waits are bounded.
+#include "ac_kernels.cuh"
+
+namespace ac {
+
+template <int D> struct TcCfg {
+    static constexpr int ROWS = 128, COLS = 128;
+    static constexpr int DB = D / 64;                        // 128-byte column blocks
+    static constexpr int STAGES = D == 128 ? 1 : 2;
+    static constexpr int X_BYTES = ROWS * D * 2;
+    static constexpr int C_BYTES = COLS * D * 2;              // one part (hi or lo)
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_C = X_BYTES;                      // stage s: hi at +2s*C, lo at +(2s+1)*C
+    static constexpr int OFF_BAR = OFF_C + STAGES * 2 * C_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static constexpr uint32_t TMEM_COLS = 256;
+};
+
+struct TcParams {
+    int N, cap, kpad;
+    const int32_t *rows;
+    const HeadSeg *seg;
+    const float *cn2, *cmax;
+    const double *norm;
+    int mode;
+    int32_t *assign, *amb_list, *amb_count;
+    int *status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 2)
+    assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmChi,
+                     const __grid_constant__ CUtensorMap tmClo, const TcParams p) {
+    using C = TcCfg<D>;
+    const int h = blockIdx.y;
+    const HeadSeg s = p.seg[h];
+    const int r0 = blockIdx.x * C::ROWS;
+    if (r0 >= s.nrows || s.k <= 0) return;  // whole CTA
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                          ~(uintptr_t)1023);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
+    uint64_t *x_full = bars, *c_full = bars + 1, *c_empty = bars + 3, *d_full = bars + 5, *d_empty = bars + 7;
+    uint64_t *drain = bars + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nch = (s.k + C::COLS - 1) / C::COLS;
+
+    if (threadIdx.x == 0) {
+        mbar_init(x_full, 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(c_full + i, 1);
+            mbar_init(c_empty + i, 1);
+            mbar_init(d_full + i, 1);
+            mbar_init(d_empty + i, 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            bool ok = true;
+            int issued = -1;
+            mbar_arrive_expect_tx(x_full, C::X_BYTES);
+            for (int kb = 0; kb < C::DB; kb++)
+                tma_load_2d(sm + C::OFF_X + kb * (C::ROWS * 128), &tmX, x_full, kb * 64, h * p.N + r0);
+            const int crow0 = h * p.kpad;
+            for (int j = 0; j < nch && ok; j++) {
+                const int st = j % C::STAGES;
+                const int u = j / C::STAGES;
+                if (u >= 1 && !mbar_wait(c_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                mbar_arrive_expect_tx(c_full + st, 2 * C::C_BYTES);
+                unsigned char *hi = sm + C::OFF_C + (2 * st) * C::C_BYTES;
+                unsigned char *lo = sm + C::OFF_C + (2 * st + 1) * C::C_BYTES;
+                for (int kb = 0; kb < C::DB; kb++) {
+                    tma_load_2d(hi + kb * (C::COLS * 128), &tmChi, c_full + st, kb * 64, crow0 + j * C::COLS);
+                    tma_load_2d(lo + kb * (C::COLS * 128), &tmClo, c_full + st, kb * 64, crow0 + j * C::COLS);
+                }
+                issued = j;
+            }
+            if (!ok) {
+                // wait (bounded) for this thread's copies before the CTA leaves
+                uint64_t t0 = gtimer();
+                while (!mbar_try_wait(x_full, 0) && gtimer() - t0 < 200000000ull) {
+                }
+                for (int j = issued - C::STAGES + 1; j <= issued; j++) {
+                    if (j < 0) continue;
+                    t0 = gtimer();
+                    while (!mbar_try_wait(c_full + (j % C::STAGES), (j / C::STAGES) & 1) &&
+                           gtimer() - t0 < 200000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = mbar_wait(x_full, 0, abort_flag, p.status);
+            const uint32_t idesc = idesc_make(128, C::COLS, 1, false);
+            const uint32_t xb = smem_u32(sm + C::OFF_X);
+            for (int j = 0; j < nch && ok; j++) {
+                const int st = j % C::STAGES;
+                const int b = j & 1;
+                if (!mbar_wait(c_full + st, (j / C::STAGES) & 1, abort_flag, p.status)) { ok = false; break; }
+                if (j >= 2 && !mbar_wait(d_empty + b, ((j >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t hb = smem_u32(sm + C::OFF_C + (2 * st) * C::C_BYTES);
+                const uint32_t lb = smem_u32(sm + C::OFF_C + (2 * st + 1) * C::C_BYTES);
+                const uint32_t dcol = tmem + b * C::COLS;
+                for (int ks = 0; ks < D / 16; ks++) {
+                    const uint32_t off = (ks / 4) * 0 + (ks % 4) * 32;
+                    const uint64_t a = sdesc_sw128(xb + (ks / 4) * (C::ROWS * 128) + off, 16, 1024);
+                    umma_f16(dcol, a, sdesc_sw128(hb + (ks / 4) * (C::COLS * 128) + off, 16, 1024), idesc,
+                             ks > 0 ? 1u : 0u);
+                }
+                for (int ks = 0; ks < D / 16; ks++) {
+                    const uint32_t off = (ks % 4) * 32;
+                    const uint64_t a = sdesc_sw128(xb + (ks / 4) * (C::ROWS * 128) + off, 16, 1024);
+                    umma_f16(dcol, a, sdesc_sw128(lb + (ks / 4) * (C::COLS * 128) + off, 16, 1024), idesc, 1u);
+                }
+                umma_commit(c_empty + st);
+                umma_commit(d_full + b);
+            }
+            if (!ok) {
+                umma_commit(drain);
+                uint64_t t0 = gtimer();
+                while (!mbar_try_wait(drain, 0) && gtimer() - t0 < 200000000ull) {
+                }
+            }
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const float *cn = p.cn2 + (size_t)h * p.cap;
+        float b1 = INFINITY, b2 = INFINITY;
+        int i1 = 0;
+        bool ok = true;
+        for (int j = 0; j < nch; j++) {
+            const int b = j & 1;
+            bool w = mbar_wait(d_full + b, (j >> 1) & 1, abort_flag, p.status);
+            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+            tc_fence_after();
+            for (int pc = 0; pc < C::COLS / 32; pc++) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_addr + b * C::COLS + pc * 32, r);
+                const int c0 = j * C::COLS + pc * 32;
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const int col = c0 + i;
+                    if (col < s.k) {
+                        const float v = __uint_as_float(r[i]);
+                        const float sc = (p.mode == MODE_EUCLID) ? fmaf(-2.f, v, cn[col]) : -v;
+                        if (sc < b1) { b2 = b1; b1 = sc; i1 = col; }
+                        else if (sc < b2) b2 = sc;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(d_empty + b);
+        }
+        const int pos = r0 + row;
+        if (ok && pos < s.nrows) {
+            const int tok = p.rows ? p.rows[(size_t)h * p.N + pos] : pos;
+            const float xn = (float)(p.norm[(size_t)h * p.N + tok] * (1.0 + 1e-6));
+            const float cm = p.cmax[h];
+            const float edot = 1.220703125e-4f * xn * cm;  // 2^-13 ||x|| Cmax
+            const float E = (p.mode == MODE_EUCLID) ? 2.f * edot + 2.384185791e-7f * (cm * cm + 2.f * xn * cm) : edot;
+            if (s.k > 1 && !(b2 - b1 > 2.f * E)) {
+                const int slot = atomicAdd(&p.amb_count[h], 1);
+                p.amb_list[(size_t)h * p.N + slot] = pos;
+            } else {
+                p.assign[(size_t)h * p.N + pos] = i1;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// C_hi / C_lo (bf16, [H, kpad, D], zero rows beyond k), ||c||^2 (fp32 of a
+// double sum) and max ||c|| (rounded up) for the centroids of the pass.
+template <int D>
+__global__ void cent_split_kernel(const float *__restrict__ cent, int cap, int kpad, const HeadSeg *__restrict__ seg,
+                                  __nv_bfloat16 *__restrict__ chi, __nv_bfloat16 *__restrict__ clo,
+                                  float *__restrict__ cn2, float *__restrict__ cmax) {
+    __shared__ float red[32];
+    const int h = blockIdx.x;
+    const HeadSeg s = seg[h];
+    float mx = 0.f;
+    for (int j = threadIdx.x; j < kpad; j += blockDim.x) {
+        __nv_bfloat16 *ph = chi + ((size_t)h * kpad + j) * D;
+        __nv_bfloat16 *pl = clo + ((size_t)h * kpad + j) * D;
+        if (j < s.k) {
+            const float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
+            double ss = 0.0;
+            for (int t = 0; t < D; t++) {
+                const float v = c[t];
+                const __nv_bfloat16 vh = __float2bfloat16_rn(v);
+                ph[t] = vh;
+                pl[t] = __float2bfloat16_rn(v - __bfloat162float(vh));
+                ss += (double)v * (double)v;
+            }
+            cn2[(size_t)h * cap + j] = (float)ss;
+            mx = fmaxf(mx, (float)(sqrt(ss) * (1.0 + 1e-6)));
+        } else {
+            for (int t = 0; t < D; t++) {
+                ph[t] = __float2bfloat16_rn(0.f);
+                pl[t] = __float2bfloat16_rn(0.f);
+            }
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); w++) m = fmaxf(m, red[w]);
+        cmax[h] = m;
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static int bf16_map(EncodeTiledFn enc, CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+               ? 0
+               : -1;
+}
+
+template <int D>
+static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const HeadSeg *seg, int nrows_max,
+                     const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
+                     const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count,
+                     int *status, void *encode_fn, cudaStream_t st) {
+    using C = TcCfg<D>;
+    EncodeTiledFn enc = (EncodeTiledFn)encode_fn;
+    cent_split_kernel<D><<<H, 256, 0, st>>>(cent, cap, kpad, seg, (__nv_bfloat16 *)chi, (__nv_bfloat16 *)clo, cn2,
+                                            cmax);
+    note_launch();
+    CUtensorMap mx, mh, ml;
+    if (bf16_map(enc, &mx, xc, H * N, D, C::ROWS) || bf16_map(enc, &mh, chi, H * kpad, D, C::COLS) ||
+        bf16_map(enc, &ml, clo, H * kpad, D, C::COLS))
+        return -1;
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        attr = true;
+    }
+    TcParams p;
+    p.N = N;
+    p.cap = cap;
+    p.kpad = kpad;
+    p.rows = rows;
+    p.seg = seg;
+    p.cn2 = cn2;
+    p.cmax = cmax;
+    p.norm = norm;
+    p.mode = mode;
+    p.assign = assign;
+    p.amb_list = amb_list;
+    p.amb_count = amb_count;
+    p.status = status;
+    dim3 g((nrows_max + C::ROWS - 1) / C::ROWS, H);
+    assign_tc_kernel<D><<<g, 192, C::SMEM, st>>>(mx, mh, ml, p);
+    note_launch();
+    return 0;
+}
+
+int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const HeadSeg *seg, int nrows_max,
+                const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
+                const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int *status,
+                void *encode_fn, cudaStream_t st) {
+    if (D == 64)
+        return launch_tc<64>(xc, H, N, rows, seg, nrows_max, cent, cap, kpad, chi, clo, cn2, cmax, norm, mode, assign,
+                             amb_list, amb_count, status, encode_fn, st);
+    return launch_tc<128>(xc, H, N, rows, seg, nrows_max, cent, cap, kpad, chi, clo, cn2, cmax, norm, mode, assign,
+                          amb_list, amb_count, status, encode_fn, st);
+}
+
+}  // namespace ac

@@ -20,6 +20,9 @@ void k_init_cent(const void *x, int dtype, int H, int N, int D, const int32_t *r
 void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
               int nrows_max, const float *cent, int cap, float *cn2, float *cmax, const double *norm, int mode,
               int32_t *assign, int32_t *amb_list, int32_t *amb_count, cudaStream_t st);
+void k_assign_exact(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
+                    const float *cent, int cap, const double *norm, int mode, const int32_t *amb_list,
+                    const int32_t *amb_count, int32_t *assign, cudaStream_t st);
 void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
             int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
             double *dist, cudaStream_t st);
@@ -27,6 +30,12 @@ void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg,
               const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st);
 void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const int32_t *off, int cap,
                  const double *norm, float *mean_norm, cudaStream_t st);
+
+// ---- ac_assign_tc.cu (bf16 inputs): tcgen05 screen; the exact pass follows
+int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const HeadSeg *seg, int nrows_max,
+                const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
+                const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int *status,
+                void *encode_fn, cudaStream_t st);
 
 // ---- ac_sort.cu
 // Stable counting sort of positions 0..seg.nrows-1 by id (< seg.k): perm gets

@@ -428,6 +428,24 @@ void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows
     }
 }
 
+void k_assign_exact(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
+                    const float *cent, int cap, const double *norm, int mode, const int32_t *amb_list,
+                    const int32_t *amb_count, int32_t *assign, cudaStream_t st) {
+    dim3 g2(64, H);
+#define AC_EXACT(T, DD)                                                                                          \
+    assign_exact_kernel<T, DD><<<g2, 256, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, amb_list, \
+                                                    amb_count, assign)
+    if (dtype == DT_BF16) {
+        if (D == 64) AC_EXACT(__nv_bfloat16, 64);
+        else AC_EXACT(__nv_bfloat16, 128);
+    } else {
+        if (D == 64) AC_EXACT(float, 64);
+        else AC_EXACT(float, 128);
+    }
+#undef AC_EXACT
+    note_launch();
+}
+
 void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
             int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
             double *dist, cudaStream_t st) {

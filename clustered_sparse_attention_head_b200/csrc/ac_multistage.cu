@@ -13,10 +13,16 @@
 
 namespace ac {
 
-__global__ void ms_init_kernel(int H, int N, MsHead *__restrict__ st, int32_t *__restrict__ U) {
+// Both U buffers start as the identity, so every entry is a valid token id
+// (entries past |U| are never used as members, but row gathers read them).
+__global__ void ms_init_kernel(int H, int N, MsHead *__restrict__ st, int32_t *__restrict__ U,
+                               int32_t *__restrict__ U2) {
     int h = blockIdx.y;
     int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < N) U[(size_t)h * N + i] = i;
+    if (i < N) {
+        U[(size_t)h * N + i] = i;
+        U2[(size_t)h * N + i] = i;
+    }
     if (i == 0) {
         MsHead s;
         s.nc = 0;
@@ -235,9 +241,9 @@ __global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restri
     seg[h] = g;
 }
 
-void k_ms_init(int H, int N, MsHead *st, int32_t *U, cudaStream_t s) {
+void k_ms_init(int H, int N, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s) {
     dim3 g((N + 255) / 256, H);
-    ms_init_kernel<<<g, 256, 0, s>>>(H, N, st, U); note_launch();
+    ms_init_kernel<<<g, 256, 0, s>>>(H, N, st, U, U2); note_launch();
 }
 void k_ms_control(int H, int N, int m0, int nmax, int cap, MsHead *st, HeadSeg *seg, int32_t *info, int *status,
                   cudaStream_t s) {

@@ -14,7 +14,7 @@ struct MsHead {
     double tau;
 };
 
-void k_ms_init(int H, int N, MsHead *st, int32_t *U, cudaStream_t s);
+void k_ms_init(int H, int N, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s);
 void k_ms_control(int H, int N, int m0, int nmax, int cap, MsHead *st, HeadSeg *seg, int32_t *info, int *status,
                   cudaStream_t s);
 void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double *dist, const int32_t *perm,

@@ -202,3 +202,60 @@ def test_forward_end_to_end_small(orc):
     r = orc.forward_head(q[0], k[0], v[0], spec)
     attn_close(out[0].float().cpu().numpy(), r.out_rows, "forward/f32")
     assert st["pairs"] == orc.pairs(r.q.count, r.k.count, r.sel_idx, r.sel_cnt)
+
+
+ADAPTIVE = [
+    # (mode, tau_rule, tau_value, m0, nmax)
+    ("k", 1, 1.5, 16, 120),     # MEAN_X, the paper's 1.5 x mean distance
+    ("k", 2, 0.5, 16, 64),      # MEDIAN_RADIUS_X 0.5: expected to hit N_max (F = 1)
+    ("k", 0, 2.0, 12, 200),     # absolute tau
+    ("q", 1, 1.5, 10, 80),      # Algorithm 1 on normalised queries
+]
+
+
+@pytest.mark.parametrize("mode,rule,val,m0,nmax", ADAPTIVE)
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_multistage_parity(orc, mode, rule, val, m0, nmax, dt):
+    """Algorithm 1 (MultiStageClustering): |C|, F, the final assignment and the
+    counts bit-exact, centroids within 1e-5 relative, against the oracle."""
+    base = W.WORKLOADS["wan21-n75600-h40-d128"] if dt == "bf16" else W.WORKLOADS["gmm16-n2048-d64-f32"]
+    w = W.small(base, 1999, heads=2, seed=9)
+    q, k, v = stack_heads(w)
+    x = q if mode == "q" else k
+    om = orc.SPHERE if mode == "q" else orc.EUCLID
+    over = dict(tau_rule=rule, tau_value=val, iters=5)
+    if mode == "q":
+        over.update(adaptive_q=True, kq=m0, nmax_q=nmax)
+    else:
+        over.update(adaptive_k=True, kk=m0, nmax_k=nmax)
+    ctx = _ctx(w, **over)
+    fn = ctx.ac_cluster_q if mode == "q" else ctx.ac_cluster_k
+    out = fn(to_dev(x, w.dtype))
+    torch.cuda.synchronize()
+    assert ctx.get_status() == 0
+    for h in range(w.heads):
+        xs, _ = orc.prepare(x[h], om)
+        r = orc.multistage(xs, m0, 5, rule, val, nmax, om)
+        nc = int(out["nclusters"][h])
+        print(f"{mode}/rule{rule}/h{h}: |C| {nc} (oracle {r.nclusters}), F {int(out['dense_flag'][h])} "
+              f"(oracle {r.dense}), stages {r.nstages}, tau {r.tau:.4f}")
+        assert nc == r.nclusters and int(out["dense_flag"][h]) == r.dense
+        assert_assign_equal(orc, xs, r.cent, om, out["assign"][h].cpu().numpy(), r.assign, f"ms/{mode}/h{h}")
+        np.testing.assert_array_equal(out["count"][h, :nc].cpu().numpy(), r.count)
+        np.testing.assert_allclose(out["cent"][h, :nc].cpu().numpy(), r.cent, rtol=CENT_RTOL, atol=1e-7)
+
+
+def test_forward_adaptive_dense_head(orc):
+    """A head whose Algorithm 1 sets F takes dense attention inside ac_forward."""
+    w = W.small(W.WORKLOADS["wan21-n75600-h40-d128"], 1200, heads=2, seed=3, kq=10, kk=8, iters=3,
+                adaptive_k=True, tau_rule=0, tau_value=0.0, nmax_k=16)
+    q, k, v = stack_heads(w)
+    ctx = _ctx(w)
+    out, st = ctx.ac_forward(to_dev(q, w.dtype), to_dev(k, w.dtype), to_dev(v, w.dtype), stats=True)
+    assert ctx.get_status() == 0
+    assert st["dense_heads"] == 2
+    got = out.float().cpu().numpy()
+    rows = np.arange(0, w.n, 7)
+    for h in range(w.heads):
+        ref = orc.attention_rows(q[h], k[h], v[h], None, None, 0, None, None, 1, rows)
+        attn_close(got[h][rows], ref, f"adaptive-dense/h{h}")
