@@ -61,7 +61,7 @@ struct Ws {
     // attention
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
-    size_t chi, clo, xu;
+    size_t chi, clo, xu, amb_cand, items_scr;
     int kpad;
     size_t total;
 };
@@ -119,6 +119,8 @@ Ws layout(const ac_ctx *c) {
     w.chi = b.take(H * (size_t)w.kpad * D * 2);
     w.clo = b.take(H * (size_t)w.kpad * D * 2);
     w.xu = b.take(HN * D * c->elt);
+    w.amb_cand = b.take(HN * 8);
+    w.items_scr = b.take(items_scratch_elems((int)H, c->kq_cap) * 4 + 16);
     w.total = b.off;
     return w;
 }
@@ -165,10 +167,11 @@ ac_status assign_step(ac_ctx *c, const Ws &w, void *ws, const void *x, const voi
     if (g.dtype == AC_BF16) {
         AC_CUDA(cudaMemsetAsync(ambc, 0, sizeof(int32_t) * H, st));
         if (k_assign_tc(xc, H, N, D, rows, seg, nrows_max, cent, cap, w.kpad, at<void>(ws, w.chi),
-                        at<void>(ws, w.clo), cn2, cmax, norm, mode, assign, amb, ambc, c->d_status, c->encode_fn,
-                        st) != 0)
+                        at<void>(ws, w.clo), cn2, cmax, norm, mode, assign, amb, ambc, at<int2>(ws, w.amb_cand),
+                        c->d_status, c->encode_fn, st) != 0)
             return AC_ERR_CUDA;
-        k_assign_exact(x, DT_BF16, H, N, D, rows, seg, cent, cap, norm, mode, amb, ambc, assign, st);
+        k_assign_exact(x, DT_BF16, H, N, D, rows, seg, cent, cap, norm, mode, amb, ambc, at<int2>(ws, w.amb_cand),
+                       assign, st);
     } else {
         k_assign(x, DT_F32, H, N, D, rows, seg, nrows_max, cent, cap, cn2, cmax, norm, mode, assign, amb, ambc, st);
     }
@@ -287,7 +290,8 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     k_gather_rows(q, qg, qperm, H, N, rb, st);
     k_gather_rows(k, kg, kperm, H, N, rb, st);
     k_gather_rows(v, vg, kperm, H, N, rb, st);
-    k_build_items(H, N, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items, nitems, pairs_dev, st);
+    k_build_items(H, N, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items, nitems, pairs_dev,
+                  at<int32_t>(ws, w.items_scr), st);
     if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
     int rc = k_attention(g.dtype == AC_BF16 ? DT_BF16 : DT_F32, D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel,
                          c->kq_cap, selc, items, nitems, attn_max_items(H, N, c->kq_cap), out, lse, c->d_status,

@@ -43,6 +43,7 @@ struct TcParams {
     const double *norm;
     int mode;
     int32_t *assign, *amb_list, *amb_count;
+    int2 *amb_cand;
     int *status;
 };
 
@@ -162,8 +163,8 @@ __global__ void __launch_bounds__(192, 2)
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const float *cn = p.cn2 + (size_t)h * p.cap;
-        float b1 = INFINITY, b2 = INFINITY;
-        int i1 = 0;
+        float b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
+        int i1 = 0, i2 = -1;
         bool ok = true;
         for (int j = 0; j < nch; j++) {
             const int b = j & 1;
@@ -180,8 +181,13 @@ __global__ void __launch_bounds__(192, 2)
                     if (col < s.k) {
                         const float v = __uint_as_float(r[i]);
                         const float sc = (p.mode == MODE_EUCLID) ? fmaf(-2.f, v, cn[col]) : -v;
-                        if (sc < b1) { b2 = b1; b1 = sc; i1 = col; }
-                        else if (sc < b2) b2 = sc;
+                        if (sc < b2) {
+                            b3 = b2;
+                            if (sc < b1) { b2 = b1; i2 = i1; b1 = sc; i1 = col; }
+                            else { b2 = sc; i2 = col; }
+                        } else {
+                            b3 = fminf(b3, sc);
+                        }
                     }
                 }
             }
@@ -196,8 +202,11 @@ __global__ void __launch_bounds__(192, 2)
             const float edot = 1.220703125e-4f * xn * cm;  // 2^-13 ||x|| Cmax
             const float E = (p.mode == MODE_EUCLID) ? 2.f * edot + 2.384185791e-7f * (cm * cm + 2.f * xn * cm) : edot;
             if (s.k > 1 && !(b2 - b1 > 2.f * E)) {
+                // Every centroid other than i1 and i2 scores >= b3; if b3 > b1 + 2E
+                // none of them can be the exact winner, so only the two are re-scored.
                 const int slot = atomicAdd(&p.amb_count[h], 1);
                 p.amb_list[(size_t)h * p.N + slot] = pos;
+                p.amb_cand[(size_t)h * p.N + slot] = (b3 - b1 > 2.f * E) ? make_int2(i1, i2) : make_int2(-1, -1);
             } else {
                 p.assign[(size_t)h * p.N + pos] = i1;
             }
@@ -217,40 +226,42 @@ __global__ void __launch_bounds__(192, 2)
 template <int D>
 __global__ void cent_split_kernel(const float *__restrict__ cent, int cap, int kpad, const HeadSeg *__restrict__ seg,
                                   __nv_bfloat16 *__restrict__ chi, __nv_bfloat16 *__restrict__ clo,
-                                  float *__restrict__ cn2, float *__restrict__ cmax) {
+                                  float *__restrict__ cn2) {
+    // one warp per centroid row: coalesced split, ||c||^2 from a double sum
+    const int h = blockIdx.y;
+    const HeadSeg s = seg[h];
+    const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (j >= kpad) return;
+    __nv_bfloat16 *ph = chi + ((size_t)h * kpad + j) * D;
+    __nv_bfloat16 *pl = clo + ((size_t)h * kpad + j) * D;
+    double ss = 0.0;
+    for (int t = lane; t < D; t += 32) {
+        float v = 0.f;
+        if (j < s.k) v = cent[((size_t)h * cap + s.cent_off + j) * D + t];
+        const __nv_bfloat16 vh = __float2bfloat16_rn(v);
+        ph[t] = vh;
+        pl[t] = __float2bfloat16_rn(v - __bfloat162float(vh));
+        ss += (double)v * (double)v;
+    }
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0 && j < s.k) cn2[(size_t)h * cap + j] = (float)ss;
+}
+
+// max_j ||c_j|| (rounded up) per head, from the ||c||^2 just written.
+__global__ void cent_max_kernel(int cap, const HeadSeg *__restrict__ seg, const float *__restrict__ cn2,
+                                float *__restrict__ cmax) {
     __shared__ float red[32];
     const int h = blockIdx.x;
     const HeadSeg s = seg[h];
     float mx = 0.f;
-    for (int j = threadIdx.x; j < kpad; j += blockDim.x) {
-        __nv_bfloat16 *ph = chi + ((size_t)h * kpad + j) * D;
-        __nv_bfloat16 *pl = clo + ((size_t)h * kpad + j) * D;
-        if (j < s.k) {
-            const float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
-            double ss = 0.0;
-            for (int t = 0; t < D; t++) {
-                const float v = c[t];
-                const __nv_bfloat16 vh = __float2bfloat16_rn(v);
-                ph[t] = vh;
-                pl[t] = __float2bfloat16_rn(v - __bfloat162float(vh));
-                ss += (double)v * (double)v;
-            }
-            cn2[(size_t)h * cap + j] = (float)ss;
-            mx = fmaxf(mx, (float)(sqrt(ss) * (1.0 + 1e-6)));
-        } else {
-            for (int t = 0; t < D; t++) {
-                ph[t] = __float2bfloat16_rn(0.f);
-                pl[t] = __float2bfloat16_rn(0.f);
-            }
-        }
-    }
+    for (int j = threadIdx.x; j < s.k; j += blockDim.x) mx = fmaxf(mx, cn2[(size_t)h * cap + j]);
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
     __syncthreads();
     if (threadIdx.x == 0) {
         float m = 0.f;
         for (int w = 0; w < (int)(blockDim.x >> 5); w++) m = fmaxf(m, red[w]);
-        cmax[h] = m;
+        cmax[h] = (float)(sqrt((double)m) * (1.0 + 1e-5));
     }
 }
 
@@ -274,11 +285,13 @@ template <int D>
 static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const HeadSeg *seg, int nrows_max,
                      const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
                      const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count,
-                     int *status, void *encode_fn, cudaStream_t st) {
+                     int2 *amb_cand, int *status, void *encode_fn, cudaStream_t st) {
     using C = TcCfg<D>;
     EncodeTiledFn enc = (EncodeTiledFn)encode_fn;
-    cent_split_kernel<D><<<H, 256, 0, st>>>(cent, cap, kpad, seg, (__nv_bfloat16 *)chi, (__nv_bfloat16 *)clo, cn2,
-                                            cmax);
+    cent_split_kernel<D><<<dim3(kpad / 8, H), 256, 0, st>>>(cent, cap, kpad, seg, (__nv_bfloat16 *)chi,
+                                                            (__nv_bfloat16 *)clo, cn2);
+    note_launch();
+    cent_max_kernel<<<H, 256, 0, st>>>(cap, seg, cn2, cmax);
     note_launch();
     CUtensorMap mx, mh, ml;
     if (bf16_map(enc, &mx, xc, H * N, D, C::ROWS) || bf16_map(enc, &mh, chi, H * kpad, D, C::COLS) ||
@@ -302,6 +315,7 @@ static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const He
     p.assign = assign;
     p.amb_list = amb_list;
     p.amb_count = amb_count;
+    p.amb_cand = amb_cand;
     p.status = status;
     dim3 g((nrows_max + C::ROWS - 1) / C::ROWS, H);
     assign_tc_kernel<D><<<g, 192, C::SMEM, st>>>(mx, mh, ml, p);
@@ -311,13 +325,13 @@ static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const He
 
 int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const HeadSeg *seg, int nrows_max,
                 const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
-                const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int *status,
-                void *encode_fn, cudaStream_t st) {
+                const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int2 *amb_cand,
+                int *status, void *encode_fn, cudaStream_t st) {
     if (D == 64)
         return launch_tc<64>(xc, H, N, rows, seg, nrows_max, cent, cap, kpad, chi, clo, cn2, cmax, norm, mode, assign,
-                             amb_list, amb_count, status, encode_fn, st);
+                             amb_list, amb_count, amb_cand, status, encode_fn, st);
     return launch_tc<128>(xc, H, N, rows, seg, nrows_max, cent, cap, kpad, chi, clo, cn2, cmax, norm, mode, assign,
-                          amb_list, amb_count, status, encode_fn, st);
+                          amb_list, amb_count, amb_cand, status, encode_fn, st);
 }
 
 }  // namespace ac

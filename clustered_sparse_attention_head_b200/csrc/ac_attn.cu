@@ -457,77 +457,106 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ------------------------------------------------------------ work items
-// One CTA: for each head, query tiles of 128 rows per non-empty query cluster
-// (or over all rows of a dense head), plus the number of (query, key) pairs.
-__global__ void build_items_kernel(int H, int N, int kq_cap, int kk_cap, const int32_t *__restrict__ qoff,
+// Work items are query tiles of 128 rows per non-empty query cluster (or over
+// all rows of a dense head).  Three launches: per head, tile counts and their
+// exclusive scan plus the head's (query, key) pairs; across heads, the bases;
+// per (cluster, head), the items themselves.
+__global__ void items_count_kernel(int N, int kq_cap, int kk_cap, const int32_t *__restrict__ qoff,
                                    const int32_t *__restrict__ nq, const uint8_t *__restrict__ dense, int kq_fixed,
                                    const int32_t *__restrict__ koff, const int32_t *__restrict__ sel_idx,
-                                   const int32_t *__restrict__ sel_cnt, AttnItem *__restrict__ items,
-                                   int32_t *__restrict__ n_items, int64_t *__restrict__ pairs) {
+                                   const int32_t *__restrict__ sel_cnt, int32_t *__restrict__ tile_off,
+                                   int32_t *__restrict__ head_tiles, unsigned long long *__restrict__ head_pairs) {
     __shared__ int wsum[32];
-    __shared__ int base;
-    __shared__ unsigned long long pairs_acc;
-    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, w = tid >> 5;
-    if (tid == 0) {
-        base = 0;
-        pairs_acc = 0ull;
-    }
+    __shared__ int carry;
+    __shared__ unsigned long long pacc;
+    const int h = blockIdx.x, tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, w = tid >> 5;
+    const bool dn = dense && dense[h];
+    const int nqh = dn ? 1 : (nq ? nq[h] : kq_fixed);
+    const int32_t *qo = qoff + (size_t)h * (kq_cap + 1);
+    const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
+    int32_t *to = tile_off + (size_t)h * (kq_cap + 1);
+    if (tid == 0) { carry = 0; pacc = 0ull; }
     __syncthreads();
-    for (int h = 0; h < H; h++) {
-        const bool dn = dense && dense[h];
-        const int nqh = dn ? 1 : (nq ? nq[h] : kq_fixed);
-        const int32_t *qo = qoff + (size_t)h * (kq_cap + 1);
-        const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
-        for (int a0 = 0; a0 < nqh; a0 += nt) {
-            const int a = a0 + tid;
-            int qs = 0, qn = 0, tiles = 0;
-            if (a < nqh) {
-                if (dn) { qs = 0; qn = N; }
-                else { qs = qo[a]; qn = qo[a + 1] - qs; }
-                tiles = (qn + 127) / 128;
-                if (!dn && qn > 0) {
-                    long long keys = 0;
-                    const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
-                    const int ns = sel_cnt[(size_t)h * kq_cap + a];
-                    for (int c = 0; c < ns; c++) keys += ko[sl[c] + 1] - ko[sl[c]];
-                    atomicAdd(&pairs_acc, (unsigned long long)(keys * qn));
-                } else if (dn) {
-                    atomicAdd(&pairs_acc, (unsigned long long)N * (unsigned long long)N);
-                }
+    for (int a0 = 0; a0 < nqh; a0 += nt) {
+        const int a = a0 + tid;
+        int tiles = 0;
+        if (a < nqh) {
+            const int qn = dn ? N : qo[a + 1] - qo[a];
+            tiles = (qn + 127) / 128;
+            unsigned long long pr = 0ull;
+            if (dn) {
+                pr = (unsigned long long)N * (unsigned long long)N;
+            } else if (qn > 0) {
+                long long keys = 0;
+                const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
+                const int ns = sel_cnt[(size_t)h * kq_cap + a];
+                for (int c = 0; c < ns; c++) keys += ko[sl[c] + 1] - ko[sl[c]];
+                pr = (unsigned long long)(keys * qn);
             }
-            int x = tiles;
-            for (int d = 1; d < 32; d <<= 1) {
-                int y = __shfl_up_sync(0xffffffffu, x, d);
-                if (lane >= d) x += y;
-            }
-            if (lane == 31) wsum[w] = x;
-            __syncthreads();
-            if (w == 0) {
-                int t = lane < nt / 32 ? wsum[lane] : 0;
-                for (int d = 1; d < 32; d <<= 1) {
-                    int y = __shfl_up_sync(0xffffffffu, t, d);
-                    if (lane >= d) t += y;
-                }
-                if (lane < nt / 32) wsum[lane] = t;
-            }
-            __syncthreads();
-            const int excl = base + x - tiles + (w > 0 ? wsum[w - 1] : 0);
-            for (int t = 0; t < tiles; t++) {
-                AttnItem itm;
-                itm.h = h;
-                itm.a = dn ? -1 : a;
-                itm.q_start = qs + t * 128;
-                itm.q_len = min(128, qn - t * 128);
-                items[excl + t] = itm;
-            }
-            __syncthreads();
-            if (tid == 0) base += wsum[nt / 32 - 1];
-            __syncthreads();
+            atomicAdd(&pacc, pr);
         }
+        int x = tiles;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
+        __syncthreads();
+        if (w == 0) {
+            int t = lane < nt / 32 ? wsum[lane] : 0;
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, t, d);
+                if (lane >= d) t += y;
+            }
+            if (lane < nt / 32) wsum[lane] = t;
+        }
+        __syncthreads();
+        if (a < nqh) to[a] = carry + x - tiles + (w > 0 ? wsum[w - 1] : 0);
+        __syncthreads();
+        if (tid == 0) carry += wsum[nt / 32 - 1];
+        __syncthreads();
     }
     if (tid == 0) {
-        *n_items = base;
-        if (pairs) *pairs = (int64_t)pairs_acc;
+        to[nqh] = carry;
+        head_tiles[h] = carry;
+        head_pairs[h] = pacc;
+    }
+}
+
+__global__ void items_base_kernel(int H, const int32_t *__restrict__ head_tiles,
+                                  const unsigned long long *__restrict__ head_pairs, int32_t *__restrict__ head_base,
+                                  int32_t *__restrict__ n_items, int64_t *__restrict__ pairs) {
+    if (threadIdx.x != 0) return;
+    int base = 0;
+    unsigned long long pr = 0ull;
+    for (int h = 0; h < H; h++) {
+        head_base[h] = base;
+        base += head_tiles[h];
+        pr += head_pairs[h];
+    }
+    *n_items = base;
+    if (pairs) *pairs = (int64_t)pr;
+}
+
+__global__ void items_write_kernel(int N, int kq_cap, const int32_t *__restrict__ qoff, const int32_t *__restrict__ nq,
+                                   const uint8_t *__restrict__ dense, int kq_fixed, const int32_t *__restrict__ tile_off,
+                                   const int32_t *__restrict__ head_base, AttnItem *__restrict__ items) {
+    const int h = blockIdx.y;
+    const int a = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool dn = dense && dense[h];
+    const int nqh = dn ? 1 : (nq ? nq[h] : kq_fixed);
+    if (a >= nqh) return;
+    const int32_t *qo = qoff + (size_t)h * (kq_cap + 1);
+    const int qs = dn ? 0 : qo[a];
+    const int qn = dn ? N : qo[a + 1] - qs;
+    const int base = head_base[h] + tile_off[(size_t)h * (kq_cap + 1) + a];
+    for (int t = 0; t * 128 < qn; t++) {
+        AttnItem itm;
+        itm.h = h;
+        itm.a = dn ? -1 : a;
+        itm.q_start = qs + t * 128;
+        itm.q_len = min(128, qn - t * 128);
+        items[base + t] = itm;
     }
 }
 
@@ -535,10 +564,24 @@ int attn_max_items(int H, int N, int kq_cap) { return H * ((N + 127) / 128 + kq_
 
 void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
-                   const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, cudaStream_t st) {
-    build_items_kernel<<<1, 1024, 0, st>>>(H, N, kq_cap, kk_cap, qoff, nq, dense, kq_fixed, koff, sel_idx, sel_cnt,
-                                           items, n_items, pairs); note_launch();
+                   const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
+                   cudaStream_t st) {
+    int32_t *tile_off = scratch;                                      // [H, kq_cap + 1]
+    int32_t *head_tiles = tile_off + (size_t)H * (kq_cap + 1);         // [H]
+    int32_t *head_base = head_tiles + H;                               // [H]
+    unsigned long long *head_pairs =
+        reinterpret_cast<unsigned long long *>(head_base + H + ((2 * H + (size_t)H * (kq_cap + 1)) & 1));  // [H]
+    items_count_kernel<<<H, 512, 0, st>>>(N, kq_cap, kk_cap, qoff, nq, dense, kq_fixed, koff, sel_idx, sel_cnt,
+                                          tile_off, head_tiles, head_pairs);
+    note_launch();
+    items_base_kernel<<<1, 32, 0, st>>>(H, head_tiles, head_pairs, head_base, n_items, pairs);
+    note_launch();
+    items_write_kernel<<<dim3((kq_cap + 127) / 128, H), 128, 0, st>>>(N, kq_cap, qoff, nq, dense, kq_fixed, tile_off,
+                                                                      head_base, items);
+    note_launch();
 }
+
+size_t items_scratch_elems(int H, int kq_cap) { return (size_t)H * (kq_cap + 1) + 2 * (size_t)H + 1 + 2 * (size_t)H; }
 
 // ------------------------------------------------------------ launcher
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,

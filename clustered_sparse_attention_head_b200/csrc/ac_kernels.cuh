@@ -6,7 +6,7 @@ namespace ac {
 
 enum { MODE_EUCLID = 0, MODE_SPHERE = 1 };
 enum { DT_F32 = 0, DT_BF16 = 1 };
-constexpr int SORT_TILE = 256;  // positions per rank/histogram tile (one warp)
+constexpr int SORT_TILE = 1024;  // positions per rank/histogram tile (one CTA of 4 warps)
 
 // Host-side count of kernels this library has launched (profiling).
 void note_launch();
@@ -22,7 +22,7 @@ void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows
               int32_t *assign, int32_t *amb_list, int32_t *amb_count, cudaStream_t st);
 void k_assign_exact(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
                     const float *cent, int cap, const double *norm, int mode, const int32_t *amb_list,
-                    const int32_t *amb_count, int32_t *assign, cudaStream_t st);
+                    const int32_t *amb_count, const int2 *amb_cand, int32_t *assign, cudaStream_t st);
 void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
             int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
             double *dist, cudaStream_t st);
@@ -34,8 +34,8 @@ void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const in
 // ---- ac_assign_tc.cu (bf16 inputs): tcgen05 screen; the exact pass follows
 int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const HeadSeg *seg, int nrows_max,
                 const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
-                const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int *status,
-                void *encode_fn, cudaStream_t st);
+                const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int2 *amb_cand,
+                int *status, void *encode_fn, cudaStream_t st);
 
 // ---- ac_sort.cu
 // Stable counting sort of positions 0..seg.nrows-1 by id (< seg.k): perm gets
@@ -60,7 +60,9 @@ struct AttnItem {
 };
 void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
-                   const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, cudaStream_t st);
+                   const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
+                   cudaStream_t st);
+size_t items_scratch_elems(int H, int kq_cap);
 int attn_max_items(int H, int N, int kq_cap);
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
                 const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,

@@ -20,19 +20,26 @@ namespace ac {
 template <typename T>
 __global__ void row_norm_kernel(const T *__restrict__ x, int N, int D, double *__restrict__ norm, int check,
                                 int *status) {
-    int h = blockIdx.y;
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= N) return;
-    const T *xi = x + ((size_t)h * N + i) * D;
-    double ss = 0.0;
+    // 64 rows per CTA: coalesced load into shared memory, then one thread per
+    // row sums its squares sequentially in double (the order of a plain loop).
+    __shared__ float tile[64 * 129];
+    const int h = blockIdx.y, r0 = blockIdx.x * 64;
+    const int nr = min(64, N - r0);
+    const T *xb = x + ((size_t)h * N + r0) * D;
     bool bad = false;
-    for (int t = 0; t < D; t++) {
-        double v = (double)to_f(xi[t]);
+    for (int idx = threadIdx.x; idx < nr * D; idx += blockDim.x) {
+        const float v = to_f(xb[idx]);
         if (check && !isfinite(v)) bad = true;
-        ss = dadd(ss, dmul(v, v));
+        tile[(idx / D) * 129 + (idx % D)] = v;
     }
     if (bad) set_status(status, ST_NONFINITE);
-    norm[(size_t)h * N + i] = sqrt(ss);
+    __syncthreads();
+    if ((int)threadIdx.x < nr) {
+        const float *row = tile + threadIdx.x * 129;
+        double ss = 0.0;
+        for (int t = 0; t < D; t++) ss = dadd(ss, dmul((double)row[t], (double)row[t]));
+        norm[(size_t)h * N + r0 + threadIdx.x] = sqrt(ss);
+    }
 }
 
 // Working value of element t of token tok: x (EUCLID) or x/||x|| (SPHERE).
@@ -228,7 +235,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) assign_exact_kernel(
     const T *__restrict__ x, int N, const int32_t *__restrict__ rows, const HeadSeg *__restrict__ seg,
     const float *__restrict__ cent, int cap, const double *__restrict__ norm, int mode,
-    const int32_t *__restrict__ amb_list, const int32_t *__restrict__ amb_count, int32_t *__restrict__ assign) {
+    const int32_t *__restrict__ amb_list, const int32_t *__restrict__ amb_count, const int2 *__restrict__ amb_cand,
+    int32_t *__restrict__ assign) {
     __shared__ double xs[8][D];
     int h = blockIdx.y;
     HeadSeg s = seg[h];
@@ -245,7 +253,11 @@ __global__ void __launch_bounds__(256) assign_exact_kernel(
         __syncwarp();
         double best = (mode == MODE_EUCLID) ? INFINITY : -INFINITY;
         int bj = 0x7fffffff;
-        for (int j = lane; j < s.k; j += 32) {
+        // shortlisted rows: only the two candidates the screen left open
+        const int2 cand = amb_cand ? amb_cand[(size_t)h * N + a] : make_int2(-1, -1);
+        const int jcount = cand.x >= 0 ? 2 : s.k;
+        for (int q = lane; q < jcount; q += 32) {
+            const int j = cand.x >= 0 ? (q == 0 ? cand.x : cand.y) : q;
             const float *c = ch + (size_t)j * D;
             double acc = 0.0;
             if (mode == MODE_EUCLID) {
@@ -303,29 +315,42 @@ __global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__r
                               const double *__restrict__ norm, int mode, float *__restrict__ cent) {
     __shared__ double ssum[D];
     __shared__ double snr;
+    __shared__ int toks[256];
+    __shared__ double nrms[256];
     int h = blockIdx.y, j = blockIdx.x, t = threadIdx.x;
     HeadSeg s = seg[h];
     if (s.nrows <= 0 || j >= s.k) return;
     const int32_t *o = off + (size_t)h * (cap + 1);
-    int b = o[j], e = o[j + 1];
+    const int b = o[j], e = o[j + 1];
     if (e <= b) return;
     const int32_t *ph = perm + (size_t)h * N;
+    const T *xh = x + (size_t)h * N * D;
     double acc = 0.0;
-    int r = b;
-    for (; r + 4 <= e; r += 4) {
-        int t0 = ph[r], t1 = ph[r + 1], t2 = ph[r + 2], t3 = ph[r + 3];
-        double v0 = work_val(x + ((size_t)h * N + t0) * D, t, mode, norm[(size_t)h * N + t0]);
-        double v1 = work_val(x + ((size_t)h * N + t1) * D, t, mode, norm[(size_t)h * N + t1]);
-        double v2 = work_val(x + ((size_t)h * N + t2) * D, t, mode, norm[(size_t)h * N + t2]);
-        double v3 = work_val(x + ((size_t)h * N + t3) * D, t, mode, norm[(size_t)h * N + t3]);
-        acc = dadd(acc, v0);
-        acc = dadd(acc, v1);
-        acc = dadd(acc, v2);
-        acc = dadd(acc, v3);
-    }
-    for (; r < e; r++) {
-        int tk = ph[r];
-        acc = dadd(acc, work_val(x + ((size_t)h * N + tk) * D, t, mode, norm[(size_t)h * N + tk]));
+    for (int r0 = b; r0 < e; r0 += 256) {
+        const int n = min(256, e - r0);
+        __syncthreads();
+        for (int i = t; i < n; i += D) {
+            const int tk = ph[r0 + i];
+            toks[i] = tk;
+            nrms[i] = (mode == MODE_SPHERE) ? norm[(size_t)h * N + tk] : 1.0;
+        }
+        __syncthreads();
+        int i = 0;
+        // members in order; 8 independent loads in flight, sums stay sequential
+        for (; i + 8 <= n; i += 8) {
+            double v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) v[u] = (double)to_f(xh[(size_t)toks[i + u] * D + t]);
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const double w = (mode == MODE_SPHERE) ? (nrms[i + u] > 0.0 ? ddiv(v[u], nrms[i + u]) : 0.0) : v[u];
+                acc = dadd(acc, w);
+            }
+        }
+        for (; i < n; i++) {
+            const double v = (double)to_f(xh[(size_t)toks[i] * D + t]);
+            acc = dadd(acc, (mode == MODE_SPHERE) ? (nrms[i] > 0.0 ? ddiv(v, nrms[i]) : 0.0) : v);
+        }
     }
     float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
     if (mode == MODE_EUCLID) {
@@ -367,7 +392,7 @@ __global__ void mean_norm_kernel(int N, const HeadSeg *__restrict__ seg, const i
 template <typename T>
 static void launch_row_norm(const void *x, int H, int N, int D, double *norm, int check, int *status,
                             cudaStream_t st) {
-    dim3 g((N + 255) / 256, H);
+    dim3 g((N + 63) / 64, H);
     row_norm_kernel<T><<<g, 256, 0, st>>>((const T *)x, N, D, norm, check, status); note_launch();
 }
 
@@ -403,7 +428,7 @@ static void launch_assign(const void *x, int H, int N, const int32_t *rows, cons
                                                       amb_list, amb_count); note_launch();
     dim3 g2(64, H);
     assign_exact_kernel<T, D><<<g2, 256, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, amb_list,
-                                                   amb_count, assign); note_launch();
+                                                   amb_count, nullptr, assign); note_launch();
 }
 
 void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
@@ -430,11 +455,11 @@ void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows
 
 void k_assign_exact(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
                     const float *cent, int cap, const double *norm, int mode, const int32_t *amb_list,
-                    const int32_t *amb_count, int32_t *assign, cudaStream_t st) {
+                    const int32_t *amb_count, const int2 *amb_cand, int32_t *assign, cudaStream_t st) {
     dim3 g2(64, H);
 #define AC_EXACT(T, DD)                                                                                          \
     assign_exact_kernel<T, DD><<<g2, 256, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, amb_list, \
-                                                    amb_count, assign)
+                                                    amb_count, amb_cand, assign)
     if (dtype == DT_BF16) {
         if (D == 64) AC_EXACT(__nv_bfloat16, 64);
         else AC_EXACT(__nv_bfloat16, 128);

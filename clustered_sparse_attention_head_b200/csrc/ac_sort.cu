@@ -12,22 +12,28 @@
 
 namespace ac {
 
-__global__ void rank_hist_kernel(const int32_t *__restrict__ ids, const HeadSeg *__restrict__ seg, int N,
-                                 int cap, int ntiles_max, int32_t *__restrict__ rank, int32_t *__restrict__ hist,
-                                 int *status) {
+__global__ void __launch_bounds__(128) rank_hist_kernel(const int32_t *__restrict__ ids, const HeadSeg *__restrict__ seg,
+                                                        int N, int cap, int ntiles_max, int32_t *__restrict__ rank,
+                                                        int32_t *__restrict__ hist, int *status) {
+    // A CTA tile holds SORT_TILE = 1024 positions, 256 per warp.  Each warp
+    // ranks its 256 positions in order with per-warp shared counters; the
+    // counters are then turned into per-warp prefixes (warp order = position
+    // order) so that a rank counts the equal ids earlier in the whole tile.
     extern __shared__ int32_t sh[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
-    HeadSeg s = seg[h];
-    const int tile = blockIdx.x * 4 + warp;
-    const int base = tile * SORT_TILE;
+    const HeadSeg s = seg[h];
+    const int tile = blockIdx.x;
+    const int base = tile * SORT_TILE + warp * (SORT_TILE / 4);
+    if (tile * SORT_TILE >= s.nrows || tile >= ntiles_max) return;  // whole CTA
     int32_t *cnt = sh + warp * cap;
-    if (base >= s.nrows || tile >= ntiles_max) return;
     for (int j = lane; j < s.k; j += 32) cnt[j] = 0;
     __syncwarp();
     const unsigned lt = (1u << lane) - 1u;
-    for (int c = 0; c < SORT_TILE; c += 32) {
-        int pos = base + c + lane;
+    int rk[8], idv[8];
+#pragma unroll
+    for (int c = 0; c < 8; c++) {
+        const int pos = base + c * 32 + lane;
         bool valid = pos < s.nrows;
         int id = valid ? ids[(size_t)h * N + pos] : -1;
         if (valid && (id < 0 || id >= s.k)) {
@@ -35,16 +41,33 @@ __global__ void rank_hist_kernel(const int32_t *__restrict__ ids, const HeadSeg 
             id = -1;
             valid = false;
         }
-        unsigned m = __match_any_sync(0xffffffffu, id);
+        const unsigned m = __match_any_sync(0xffffffffu, id);
         int r = 0;
         if (valid) r = cnt[id] + __popc(m & lt);
         __syncwarp();
         if (valid && lane == __ffs(m) - 1) cnt[id] += __popc(m);
         __syncwarp();
-        if (valid) rank[(size_t)h * N + pos] = r;
+        rk[c] = r;
+        idv[c] = id;
     }
+    __syncthreads();
     int32_t *hh = hist + ((size_t)h * ntiles_max + tile) * cap;
-    for (int j = lane; j < s.k; j += 32) hh[j] = cnt[j];
+    for (int j = threadIdx.x; j < s.k; j += blockDim.x) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+            const int v = sh[w * cap + j];
+            sh[w * cap + j] = run;
+            run += v;
+        }
+        hh[j] = run;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < 8; c++) {
+        const int pos = base + c * 32 + lane;
+        if (idv[c] >= 0) rank[(size_t)h * N + pos] = rk[c] + cnt[idv[c]];
+    }
 }
 
 // Per cluster j: exclusive scan over tiles (in place) and the cluster size.
@@ -138,7 +161,7 @@ void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, 
         smem_set = smem;
     }
     if (nt > 0) {
-        dim3 g1((nt + 3) / 4, H);
+        dim3 g1(nt, H);
         rank_hist_kernel<<<g1, 128, smem, st>>>(ids, seg, N, cap, ntiles_max, rank, hist, status); note_launch();
     }
     dim3 g2((cap + 127) / 128, H);

@@ -175,7 +175,7 @@ AC_API ac_status ac_cluster_sort(ac_ctx *ctx, const int32_t *assign, int cap, co
  * and no cudaMalloc/cudaFree or other allocating call.
  *  - Scratch is a 16 MiB array in the library's own device memory; every GPU
  *    that loads the library holds it until the process exits.  A problem
- *    needs 256 + 16*heads + 4*heads*n + 4*heads*cap + 4*heads*ceil(n/256)*cap
+ *    needs 256 + 16*heads + 4*heads*n + 4*heads*cap + 4*heads*ceil(n/1024)*cap
  *    bytes (each term rounded up to 256); larger problems, or cap > 8192,
  *    return AC_ERR_UNSUPPORTED without launching anything.
  *  - The first call on each device looks up that device's address of the
