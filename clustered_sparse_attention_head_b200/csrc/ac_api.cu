@@ -290,12 +290,17 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     k_gather_rows(q, qg, qperm, H, N, rb, st);
     k_gather_rows(k, kg, kperm, H, N, rb, st);
     k_gather_rows(v, vg, kperm, H, N, rb, st);
-    k_build_items(H, N, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items, nitems, pairs_dev,
-                  at<int32_t>(ws, w.items_scr), st);
+    const bool two_tiles = (g.dtype == AC_BF16);  // bf16: two query tiles per CTA (items of 256 rows)
+    k_build_items(H, N, two_tiles ? 256 : 128, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items,
+                  nitems, pairs_dev, at<int32_t>(ws, w.items_scr), st);
     if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
-    int rc = k_attention(g.dtype == AC_BF16 ? DT_BF16 : DT_F32, D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel,
-                         c->kq_cap, selc, items, nitems, attn_max_items(H, N, c->kq_cap), out, lse, c->d_status,
-                         c->num_sms, c->encode_fn, st);
+    int rc;
+    if (two_tiles)
+        rc = k_attention2(D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel, c->kq_cap, selc, items, nitems,
+                          attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
+    else
+        rc = k_attention(DT_F32, D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel, c->kq_cap, selc, items, nitems,
+                         attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
     if (rc != 0) return AC_ERR_CUDA;
     if (ev_kernel) cudaEventRecord(ev_kernel[1], st);
     return launch_check();

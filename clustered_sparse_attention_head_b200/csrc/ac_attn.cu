@@ -30,6 +30,9 @@ template <typename T, int D> struct AttnCfg {
     static constexpr int DB = D / EPR;             // 128-byte column blocks of a Q/K/V row
     static constexpr int KSTEP = 32 / ELT;         // K of one MMA instruction
     static constexpr int BOX = 32;                 // rows per K/V TMA box
+    static constexpr int NPB = ELT == 2 ? 2 : 1;   // P buffers (double-buffered for bf16)
+    static constexpr int SM_WARPS = 4;             // softmax warps: one per TMEM lane quarter
+    static constexpr int NTHREADS = (2 + SM_WARPS) * 32;
     static constexpr int Q_BYTES = BM * D * ELT;
     static constexpr int KV_BYTES = BN * D * ELT;  // one stage of K (or of V)
     static constexpr int P_BYTES = BM * BN * ELT;
@@ -37,7 +40,7 @@ template <typename T, int D> struct AttnCfg {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
     static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int OFF_BAR = OFF_P + NPB * P_BYTES;
     // + alignment slack; at least 116 KB so that two CTAs never share an SM
     // (each allocates all 512 TMEM columns)
     static constexpr int SMEM_RAW = OFF_BAR + 256 + 1024;
@@ -69,9 +72,8 @@ struct AttnParams {
 // [koff[b], koff[b+1]) (all rows [0, N) for a dense head) in pieces of <= BN.
 struct ChunkIter {
     const int32_t *koff, *sel;
-    int nsel, si, cur, end, bn;
-    __device__ void init(const AttnParams &p, const AttnItem &it, int bn_) {
-        bn = bn_;
+    int nsel, si, cur, end, bn, dense_n;
+    __device__ void init(const AttnParams &p, const AttnItem &it) {
         koff = p.koff + (size_t)it.h * (p.kk_cap + 1);
         if (it.a < 0) {
             sel = nullptr;
@@ -82,15 +84,13 @@ struct ChunkIter {
         }
         si = -1;
         cur = end = 0;
-        (void)p;
         dense_n = p.N;
     }
-    int dense_n;
     __device__ bool next(int &start, int &len) {
         while (cur >= end) {
             if (++si >= nsel) return false;
             if (sel) {
-                int b = sel[si];
+                const int b = sel[si];
                 cur = koff[b];
                 end = koff[b + 1];
             } else {
@@ -104,10 +104,10 @@ struct ChunkIter {
         return true;
     }
     __device__ int count(const AttnParams &p, const AttnItem &it) {
-        init(p, it, bn);
+        init(p, it);
         int n = 0, s, l;
         while (next(s, l)) n++;
-        init(p, it, bn);
+        init(p, it);
         return n;
     }
 };
@@ -125,8 +125,23 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// 2^x on the FMA pipe: x = n + f with n = rint(x) (magic-constant add),
+// f in [-1/2, 1/2]; 2^f by a cubic fitted (relative-error minimax on
+// Chebyshev nodes) to |rel err| < 7.5e-5, well below the bf16/tf32 rounding
+// P goes through; then n is added to the exponent.  x is clamped at -125.
+__device__ __forceinline__ float ex2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.0f;                  // 1.5 * 2^23: t - 1.5*2^23 = rint(x)
+    const int n = __float_as_int(t) - 0x4B400000;
+    const float f = x - (t - 12582912.0f);
+    float p = fmaf(0.0551716648042202f, f, 0.2426111251115799f);
+    p = fmaf(p, f, 0.6932609677314758f);
+    p = fmaf(p, f, 0.9999280571937561f);
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(AttnCfg<T, D>::NTHREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using C = AttnCfg<T, D>;
@@ -135,26 +150,28 @@ __global__ void __launch_bounds__(192, 1)
                                                           ~(uintptr_t)1023);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
     uint64_t *q_full = bars + 0, *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2, *v_full = bars + 4, *kv_empty = bars + 6;
+    uint64_t *k_full = bars + 2, *v_full = bars + 4, *k_empty = bars + 6, *v_empty = bars + 20;
     uint64_t *s_full = bars + 8, *s_empty = bars + 10;
-    uint64_t *p_full = bars + 12, *o_done = bars + 13, *o_free = bars + 14, *drain = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+    uint64_t *p_full = bars + 12, *pv_done = bars + 14, *o_free = bars + 16, *drain = bars + 17;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t NSM = C::SM_WARPS * 32;
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
         for (int i = 0; i < 2; i++) {
             mbar_init(k_full + i, 1);
             mbar_init(v_full + i, 1);
-            mbar_init(kv_empty + i, 1);
+            mbar_init(k_empty + i, 1);
+            mbar_init(v_empty + i, 1);
             mbar_init(s_full + i, 1);
-            mbar_init(s_empty + i, 128);
+            mbar_init(s_empty + i, NSM);
+            mbar_init(p_full + i, NSM);
+            mbar_init(pv_done + i, 1);
         }
-        mbar_init(p_full, 128);
-        mbar_init(o_done, 1);
-        mbar_init(o_free, 128);
+        mbar_init(o_free, NSM);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -181,7 +198,7 @@ __global__ void __launch_bounds__(192, 1)
             int last_kv[2] = {-1, -1};
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-                AttnItem it = p.items[item];
+                const AttnItem it = p.items[item];
                 ChunkIter ci;
                 ci.bn = C::BN;
                 if (ci.count(p, it) == 0) continue;
@@ -195,7 +212,9 @@ __global__ void __launch_bounds__(192, 1)
                 while (ci.next(start, len)) {
                     const int st = g & 1;
                     const uint32_t u = g >> 1;
-                    if (u >= 1 && !mbar_wait(kv_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    // K of stage st is free once S of its previous chunk is done,
+                    // V once that chunk's P.V is done
+                    if (u >= 1 && !mbar_wait(k_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
                     const int nb = (len + C::BOX - 1) / C::BOX;
                     const uint32_t bytes = (uint32_t)nb * C::BOX * 128 * C::DB;
                     const int krow = it.h * p.N + start;
@@ -204,6 +223,7 @@ __global__ void __launch_bounds__(192, 1)
                         for (int b = 0; b < nb; b++)
                             tma_load_2d(sm + C::OFF_K + st * C::KV_BYTES + kb * (C::BN * 128) + b * (C::BOX * 128),
                                         &tmK, k_full + st, kb * C::EPR, krow + b * C::BOX);
+                    if (u >= 1 && !mbar_wait(v_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
                     mbar_arrive_expect_tx(v_full + st, bytes);
                     for (int kb = 0; kb < C::DB; kb++)
                         for (int b = 0; b < nb; b++)
@@ -214,7 +234,6 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             if (!ok) {
-                // drain the copies this thread issued before leaving
                 if (qi >= 1) drain_wait(q_full, (qi - 1) & 1);
                 for (int st = 0; st < 2; st++)
                     if (last_kv[st] >= 0) {
@@ -229,14 +248,16 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t idesc_o = idesc_make(128, D, C::FMT, true);
             uint32_t g = 0, qi = 0;
             bool ok = true;
+            // O += P_gp V_gp; P from buffer gp % NPB, V from stage gp % 2
             auto issue_pv = [&](uint32_t gp, int lenp, bool first) -> bool {
-                if (!mbar_wait(p_full, gp & 1, abort_flag, p.status)) return false;
+                const int pb = gp % C::NPB;
+                if (!mbar_wait(p_full + pb, (gp / C::NPB) & 1, abort_flag, p.status)) return false;
                 if (!mbar_wait(v_full + (gp & 1), (gp >> 1) & 1, abort_flag, p.status)) return false;
                 if (first && qi >= 2 && !mbar_wait(o_free, (qi - 2) & 1, abort_flag, p.status)) return false;
                 tc_fence_after();
                 const int np = (lenp + 31) & ~31;
                 const uint32_t vbase = smem_u32(sm + C::OFF_V + (gp & 1) * C::KV_BYTES);
-                const uint32_t pbase = smem_u32(sm + C::OFF_P);
+                const uint32_t pbase = smem_u32(sm + C::OFF_P + pb * C::P_BYTES);
                 for (int ks = 0; ks < np / C::KSTEP; ks++) {
                     const int kofs = ks * C::KSTEP;
                     const uint64_t a = sdesc_sw128(pbase + (kofs / C::EPR) * (C::BM * 128) + (kofs % C::EPR) * C::ELT,
@@ -248,12 +269,12 @@ __global__ void __launch_bounds__(192, 1)
                     if (C::FMT == 1) umma_f16(tmem + C::TM_O, a, b, idesc_o, (!first || ks > 0) ? 1u : 0u);
                     else umma_tf32(tmem + C::TM_O, a, b, idesc_o, (!first || ks > 0) ? 1u : 0u);
                 }
-                umma_commit(o_done);
-                umma_commit(kv_empty + (gp & 1));
+                umma_commit(pv_done + pb);
+                umma_commit(v_empty + (gp & 1));
                 return true;
             };
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-                AttnItem it = p.items[item];
+                const AttnItem it = p.items[item];
                 ChunkIter ci;
                 ci.bn = C::BN;
                 const int nch = ci.count(p, it);
@@ -281,6 +302,7 @@ __global__ void __launch_bounds__(192, 1)
                         else umma_tf32(dS, a, b, idesc_s, ks > 0 ? 1u : 0u);
                     }
                     umma_commit(s_full + st);
+                    umma_commit(k_empty + st);
                     if (c == nch - 1) umma_commit(q_empty);
                     if (c > 0 && !issue_pv(g - 1, prev_len, c == 1)) { ok = false; break; }
                     prev_len = len;
@@ -297,14 +319,16 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ------------------------------------------------ softmax + epilogue
+        // One thread per query row (= TMEM lane).  Each chunk's scores come out
+        // of TMEM in one wide load; the S buffer is released right away, P goes
+        // to the buffer whose previous P.V has completed.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         uint32_t g = 0;
         bool ok = true;
-        unsigned char *prow = sm + C::OFF_P + row * 128;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-            AttnItem it = p.items[item];
+            const AttnItem it = p.items[item];
             ChunkIter ci;
             ci.bn = C::BN;
             const int nch = ci.count(p, it);
@@ -315,88 +339,96 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t u = g >> 1;
                 if (!wait_all(s_full + st, u & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sadr = tmem + lane_addr + (st ? C::TM_S1 : C::TM_S0);
-                const int npc = (len + 31) >> 5;
-                float mx = -INFINITY;
-                uint32_t r[32];
-                for (int pc = 0; pc < npc; pc++) {
-                    tmem_ld32(sadr + pc * 32, r);
+                uint32_t sr[C::BN];
+                if (C::BN == 128) tmem_ld128(tmem + lane_addr + (st ? C::TM_S1 : C::TM_S0), *reinterpret_cast<uint32_t (*)[128]>(sr));
+                else tmem_ld64(tmem + lane_addr + (st ? C::TM_S1 : C::TM_S0), *reinterpret_cast<uint32_t (*)[64]>(sr));
+                tc_fence_before();
+                mbar_arrive(s_empty + st);
+                // columns past the chunk's keys (rounded up to 32) do not count
+                if (len < C::BN) {
 #pragma unroll
-                    for (int i = 0; i < 32; i++)
-                        if (pc * 32 + i < len) mx = fmaxf(mx, __uint_as_float(r[i]));
+                    for (int i = 0; i < C::BN; i++)
+                        if (i >= len) sr[i] = __float_as_uint(-INFINITY);
                 }
+                float mx = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < C::BN; i++) mx = fmaxf(mx, __uint_as_float(sr[i]));
                 const float m_new = mx * p.scale_log2;
                 if (c == 0) m_ref = m_new;
-                if (g >= 1 && !wait_all(o_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
                 // Move the reference max (and rescale O) only when it grew by
                 // more than 2^8.  The TMEM accesses are warp-collective, so the
-                // decision is taken per warp; rows that did not grow use f = 1.
+                // decision is per warp; rows that did not grow use f = 1.
                 if (c > 0 && __any_sync(0xffffffffu, m_new > m_ref + 8.f)) {
+                    const uint32_t gq = g - 1;
+                    if (!wait_all(pv_done + gq % C::NPB, (gq / C::NPB) & 1, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
                     const float m_to = fmaxf(m_ref, m_new);
                     const float f = ex2_approx(m_ref - m_to);
                     l *= f;
-                    tc_fence_after();
+#pragma unroll
                     for (int pc = 0; pc < D / 32; pc++) {
-                        tmem_ld32(tmem + lane_addr + C::TM_O + pc * 32, r);
+                        uint32_t r[32];
+                        const uint32_t oa = tmem + lane_addr + C::TM_O + pc * 32;
+                        tmem_ld32(oa, r);
 #pragma unroll
                         for (int i = 0; i < 32; i++) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-                        tmem_st32(tmem + lane_addr + C::TM_O + pc * 32, r);
+                        tmem_st32(oa, r);
                     }
                     tmem_st_wait();
                     m_ref = m_to;
                 }
-                const int ncol = npc * 32;
-                for (int pc = 0; pc < npc; pc++) {
-                    tmem_ld32(sadr + pc * 32, r);
-                    float pv[32];
+                // P buffer g % NPB is free once the P.V of its previous use is done
+                const int pb = g % C::NPB;
+                const uint32_t pu = g / C::NPB;
+                if (pu >= 1 && !wait_all(pv_done + pb, (pu - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                unsigned char *prow = sm + C::OFF_P + pb * C::P_BYTES + row * 128;
+                const int npc = (len + 31) >> 5;
 #pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        float e = (pc * 32 + i < len) ? ex2_approx(fmaf(__uint_as_float(r[i]), p.scale_log2, -m_ref))
-                                                      : 0.f;
-                        pv[i] = e;
-                    }
-                    if (C::ELT == 2) {
-                        // 32 bf16 = 4 x 16-byte chunks of the row's 128-byte block
-                        const int kb = (pc * 32) / C::EPR;
-                        const int ch0 = ((pc * 32) % C::EPR) / 8;
+                for (int pc = 0; pc < C::BN / 32; pc++) {
+                    if (pc < npc) {
+                        float pv[32];
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; q4++) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; e2++) {
-                                __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[q4 * 8 + e2 * 2], pv[q4 * 8 + e2 * 2 + 1]);
-                                float2 back = __bfloat1622float2(b2);
-                                l += back.x + back.y;
-                                w[e2] = *reinterpret_cast<uint32_t *>(&b2);
-                            }
-                            const int chunk = (ch0 + q4) ^ (row & 7);
-                            *reinterpret_cast<uint4 *>(prow + kb * (C::BM * 128) + chunk * 16) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
+                        for (int i = 0; i < 32; i++) {
+                            const float x = fmaf(__uint_as_float(sr[pc * 32 + i]), p.scale_log2, -m_ref);
+                            pv[i] = (i & 3) == 3 ? ex2_poly(x) : ex2_approx(x);
+                            l += pv[i];
                         }
-                    } else {
-                        // 32 fp32 (rounded to tf32) = one whole 128-byte block
-                        const int kb = pc;
+                        if (C::ELT == 2) {
+                            const int kb = (pc * 32) / C::EPR;
+                            const int ch0 = ((pc * 32) % C::EPR) / 8;
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; q4++) {
-                            uint32_t w[4];
+                            for (int q4 = 0; q4 < 4; q4++) {
+                                uint32_t w[4];
 #pragma unroll
-                            for (int e2 = 0; e2 < 4; e2++) {
-                                uint32_t tf;
-                                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(tf) : "f"(pv[q4 * 4 + e2]));
-                                l += __uint_as_float(tf);
-                                w[e2] = tf;
+                                for (int e2 = 0; e2 < 4; e2++) {
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[q4 * 8 + e2 * 2], pv[q4 * 8 + e2 * 2 + 1]);
+                                    w[e2] = *reinterpret_cast<uint32_t *>(&b2);
+                                }
+                                const int chunk = (ch0 + q4) ^ (row & 7);
+                                *reinterpret_cast<uint4 *>(prow + kb * (C::BM * 128) + chunk * 16) =
+                                    make_uint4(w[0], w[1], w[2], w[3]);
                             }
-                            const int chunk = q4 ^ (row & 7);
-                            *reinterpret_cast<uint4 *>(prow + kb * (C::BM * 128) + chunk * 16) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
+                        } else {
+                            const int kb = pc;
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; q4++) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int e2 = 0; e2 < 4; e2++) {
+                                    uint32_t tf;
+                                    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(tf) : "f"(pv[q4 * 4 + e2]));
+                                    w[e2] = tf;
+                                }
+                                const int chunk = q4 ^ (row & 7);
+                                *reinterpret_cast<uint4 *>(prow + kb * (C::BM * 128) + chunk * 16) =
+                                    make_uint4(w[0], w[1], w[2], w[3]);
+                            }
                         }
                     }
                 }
-                (void)ncol;
-                tc_fence_before();
-                mbar_arrive(s_empty + st);
-                fence_proxy_async_smem();
-                mbar_arrive(p_full);
+                tc_fence_before();          // orders a rescale's tcgen05.st before the P.V
+                fence_proxy_async_smem();   // P (generic stores) visible to the MMA
+                mbar_arrive(p_full + pb);
                 c++;
                 g++;
             }
@@ -407,9 +439,11 @@ __global__ void __launch_bounds__(192, 1)
             if (valid) tok = p.qperm[(size_t)it.h * p.N + it.q_start + row];
             const size_t orow = ((size_t)it.h * p.N + tok) * D;
             if (nch > 0) {
-                if (!wait_all(o_done, (g - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                const uint32_t gq = g - 1;
+                if (!wait_all(pv_done + gq % C::NPB, (gq / C::NPB) & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
                 const float inv = 1.f / l;
+#pragma unroll
                 for (int pc = 0; pc < D / 32; pc++) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_addr + C::TM_O + pc * 32, r);
@@ -461,7 +495,7 @@ __global__ void __launch_bounds__(192, 1)
 // all rows of a dense head).  Three launches: per head, tile counts and their
 // exclusive scan plus the head's (query, key) pairs; across heads, the bases;
 // per (cluster, head), the items themselves.
-__global__ void items_count_kernel(int N, int kq_cap, int kk_cap, const int32_t *__restrict__ qoff,
+__global__ void items_count_kernel(int N, int rpi, int kq_cap, int kk_cap, const int32_t *__restrict__ qoff,
                                    const int32_t *__restrict__ nq, const uint8_t *__restrict__ dense, int kq_fixed,
                                    const int32_t *__restrict__ koff, const int32_t *__restrict__ sel_idx,
                                    const int32_t *__restrict__ sel_cnt, int32_t *__restrict__ tile_off,
@@ -482,7 +516,7 @@ __global__ void items_count_kernel(int N, int kq_cap, int kk_cap, const int32_t 
         int tiles = 0;
         if (a < nqh) {
             const int qn = dn ? N : qo[a + 1] - qo[a];
-            tiles = (qn + 127) / 128;
+            tiles = (qn + rpi - 1) / rpi;
             unsigned long long pr = 0ull;
             if (dn) {
                 pr = (unsigned long long)N * (unsigned long long)N;
@@ -538,7 +572,7 @@ __global__ void items_base_kernel(int H, const int32_t *__restrict__ head_tiles,
     if (pairs) *pairs = (int64_t)pr;
 }
 
-__global__ void items_write_kernel(int N, int kq_cap, const int32_t *__restrict__ qoff, const int32_t *__restrict__ nq,
+__global__ void items_write_kernel(int N, int rpi, int kq_cap, const int32_t *__restrict__ qoff, const int32_t *__restrict__ nq,
                                    const uint8_t *__restrict__ dense, int kq_fixed, const int32_t *__restrict__ tile_off,
                                    const int32_t *__restrict__ head_base, AttnItem *__restrict__ items) {
     const int h = blockIdx.y;
@@ -550,19 +584,19 @@ __global__ void items_write_kernel(int N, int kq_cap, const int32_t *__restrict_
     const int qs = dn ? 0 : qo[a];
     const int qn = dn ? N : qo[a + 1] - qs;
     const int base = head_base[h] + tile_off[(size_t)h * (kq_cap + 1) + a];
-    for (int t = 0; t * 128 < qn; t++) {
+    for (int t = 0; t * rpi < qn; t++) {
         AttnItem itm;
         itm.h = h;
         itm.a = dn ? -1 : a;
-        itm.q_start = qs + t * 128;
-        itm.q_len = min(128, qn - t * 128);
+        itm.q_start = qs + t * rpi;
+        itm.q_len = min(rpi, qn - t * rpi);
         items[base + t] = itm;
     }
 }
 
 int attn_max_items(int H, int N, int kq_cap) { return H * ((N + 127) / 128 + kq_cap); }
 
-void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
+void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
                    const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
                    cudaStream_t st) {
@@ -571,12 +605,12 @@ void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, co
     int32_t *head_base = head_tiles + H;                               // [H]
     unsigned long long *head_pairs =
         reinterpret_cast<unsigned long long *>(head_base + H + ((2 * H + (size_t)H * (kq_cap + 1)) & 1));  // [H]
-    items_count_kernel<<<H, 512, 0, st>>>(N, kq_cap, kk_cap, qoff, nq, dense, kq_fixed, koff, sel_idx, sel_cnt,
+    items_count_kernel<<<H, 512, 0, st>>>(N, rows_per_item, kq_cap, kk_cap, qoff, nq, dense, kq_fixed, koff, sel_idx, sel_cnt,
                                           tile_off, head_tiles, head_pairs);
     note_launch();
     items_base_kernel<<<1, 32, 0, st>>>(H, head_tiles, head_pairs, head_base, n_items, pairs);
     note_launch();
-    items_write_kernel<<<dim3((kq_cap + 127) / 128, H), 128, 0, st>>>(N, kq_cap, qoff, nq, dense, kq_fixed, tile_off,
+    items_write_kernel<<<dim3((kq_cap + 127) / 128, H), 128, 0, st>>>(N, rows_per_item, kq_cap, qoff, nq, dense, kq_fixed, tile_off,
                                                                       head_base, items);
     note_launch();
 }
@@ -618,7 +652,7 @@ static int launch_attn(const void *qg, const void *kg, const void *vg, const Att
     }
     int grid = max_items < num_sms ? max_items : num_sms;
     if (grid < 1) grid = 1;
-    attn_kernel<T, D><<<grid, 192, C::SMEM, st>>>(mq, mk, mv, p); note_launch();
+    attn_kernel<T, D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p); note_launch();
     return 0;
 }
 

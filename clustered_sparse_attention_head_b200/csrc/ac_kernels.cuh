@@ -58,12 +58,17 @@ void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const
 struct AttnItem {
     int h, a, q_start, q_len;  // a < 0: dense head (all keys)
 };
-void k_build_items(int H, int N, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
+void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
                    const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
                    cudaStream_t st);
 size_t items_scratch_elems(int H, int kq_cap);
 int attn_max_items(int H, int N, int kq_cap);
+// bf16: two 128-row query tiles per CTA (ac_attn2.cu); items of up to 256 rows
+int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
+                 const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap, const int32_t *sel_cnt,
+                 const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
+                 int num_sms, void *encode_fn, cudaStream_t st);
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
                 const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
                 const int32_t *sel_cnt, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
