@@ -66,37 +66,34 @@ struct AttnParams {
     float *lse;
     int *status;
     float scale_log2;
+    const int2 *segtab;
 };
 
 // Walks the key chunks of one work item: every selected key cluster's rows
 // [koff[b], koff[b+1]) (all rows [0, N) for a dense head) in pieces of <= BN.
 struct ChunkIter {
-    const int32_t *koff, *sel;
+    const int2 *seg;
     int nsel, si, cur, end, bn, dense_n;
+    int2 nxt;
     __device__ void init(const AttnParams &p, const AttnItem &it) {
-        koff = p.koff + (size_t)it.h * (p.kk_cap + 1);
         if (it.a < 0) {
-            sel = nullptr;
+            seg = nullptr;
             nsel = 1;
         } else {
-            sel = p.sel_idx + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
+            seg = p.segtab + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
             nsel = p.sel_cnt[(size_t)it.h * p.kq_cap + it.a];
         }
         si = -1;
         cur = end = 0;
         dense_n = p.N;
+        nxt = (seg && nsel > 0) ? seg[0] : make_int2(0, p.N);
     }
     __device__ bool next(int &start, int &len) {
         while (cur >= end) {
             if (++si >= nsel) return false;
-            if (sel) {
-                const int b = sel[si];
-                cur = koff[b];
-                end = koff[b + 1];
-            } else {
-                cur = 0;
-                end = dense_n;
-            }
+            cur = nxt.x;
+            end = nxt.y;
+            if (seg && si + 1 < nsel) nxt = seg[si + 1];  // one segment ahead
         }
         start = cur;
         len = min(bn, end - cur);
@@ -594,6 +591,29 @@ __global__ void items_write_kernel(int N, int rpi, int kq_cap, const int32_t *__
     }
 }
 
+// Segment table: for query cluster a of head h, entry c holds the key rows
+// [koff[b], koff[b+1]) of its c-th selected key cluster b, so the attention
+// kernels read one int2 per segment instead of two dependent loads.
+__global__ void seg_table_kernel(int kq_cap, int kk_cap, const int32_t *__restrict__ koff,
+                                 const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt,
+                                 int2 *__restrict__ segtab) {
+    const int h = blockIdx.y, a = blockIdx.x;
+    const int n = sel_cnt[(size_t)h * kq_cap + a];
+    const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
+    const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
+    int2 *out = segtab + ((size_t)h * kq_cap + a) * kk_cap;
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+        const int b = sl[c];
+        out[c] = make_int2(ko[b], ko[b + 1]);
+    }
+}
+
+void k_seg_table(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx,
+                 const int32_t *sel_cnt, int2 *segtab, cudaStream_t st) {
+    seg_table_kernel<<<dim3(kq_cap, H), 128, 0, st>>>(kq_cap, kk_cap, koff, sel_idx, sel_cnt, segtab);
+    note_launch();
+}
+
 int attn_max_items(int H, int N, int kq_cap) { return H * ((N + 127) / 128 + kq_cap); }
 
 void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
@@ -658,9 +678,10 @@ static int launch_attn(const void *qg, const void *kg, const void *vg, const Att
 
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
                 const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
-                const int32_t *sel_cnt, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
-                float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st) {
+                const int32_t *sel_cnt, const int2 *segtab, const AttnItem *items, const int32_t *n_items,
+                int max_items, void *out, float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st) {
     AttnParams p;
+    p.segtab = segtab;
     p.H = H;
     p.N = N;
     p.qperm = qperm;

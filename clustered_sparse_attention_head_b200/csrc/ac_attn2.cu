@@ -27,10 +27,13 @@ template <int D> struct A2Cfg {
     static constexpr int BM = 128, BN = 128, EPR = 64, DB = D / 64, BOX = 32, KSTEP = 16;
     static constexpr int Q_BYTES = BM * D * 2;     // one query tile
     static constexpr int KV_BYTES = BN * D * 2;    // one stage of K (or of V)
+    // K is consumed by S right away; V only after the softmax, so V gets the
+    // deeper ring (its loads must start further ahead of their use)
+    static constexpr int KST = 2, VST = 3;
     static constexpr int OFF_Q = 0;                // tile 1 at + Q_BYTES
     static constexpr int OFF_K = 2 * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
+    static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
     static constexpr int SMEM_RAW = OFF_BAR + 256 + 1024;
     // at least 116 KB so that two CTAs never share an SM (each takes all of TMEM)
     static constexpr int SMEM = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
@@ -58,37 +61,34 @@ struct A2Params {
     float *lse;
     int *status;
     float scale_log2;
+    const int2 *segtab;  // per (head, query cluster): key rows of each selected cluster
 };
 
 namespace {
 
 struct Chunks {
-    const int32_t *koff, *sel;
+    const int2 *seg;
     int nsel, si, cur, end, dense_n;
+    int2 nxt;
     __device__ void init(const A2Params &p, const AttnItem &it) {
-        koff = p.koff + (size_t)it.h * (p.kk_cap + 1);
         if (it.a < 0) {
-            sel = nullptr;
+            seg = nullptr;
             nsel = 1;
         } else {
-            sel = p.sel_idx + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
+            seg = p.segtab + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
             nsel = p.sel_cnt[(size_t)it.h * p.kq_cap + it.a];
         }
         si = -1;
         cur = end = 0;
         dense_n = p.N;
+        nxt = (seg && nsel > 0) ? seg[0] : make_int2(0, p.N);
     }
     __device__ bool next(int &start, int &len) {
         while (cur >= end) {
             if (++si >= nsel) return false;
-            if (sel) {
-                const int b = sel[si];
-                cur = koff[b];
-                end = koff[b + 1];
-            } else {
-                cur = 0;
-                end = dense_n;
-            }
+            cur = nxt.x;
+            end = nxt.y;
+            if (seg && si + 1 < nsel) nxt = seg[si + 1];  // one segment ahead
         }
         start = cur;
         len = min(128, end - cur);
@@ -185,28 +185,34 @@ __device__ __forceinline__ float ex2_fma(float x) {
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const A2Params p) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK128,
+                 const __grid_constant__ CUtensorMap tmV128, const A2Params p) {
     using C = A2Cfg<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                           ~(uintptr_t)1023);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
     uint64_t *q_full = bars + 0, *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2, *v_full = bars + 4, *k_empty = bars + 6, *v_empty = bars + 8;
-    uint64_t *s_full = bars + 10, *p_full = bars + 12, *pv_done = bars + 14, *o_free = bars + 16;
-    uint64_t *drain_bar = bars + 18;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
+    uint64_t *k_full = bars + 2, *k_empty = bars + 4;             // [KST]
+    uint64_t *v_full = bars + 6, *v_empty = bars + 9;             // [VST]
+    uint64_t *s_full = bars + 12, *p_full = bars + 14, *pv_done = bars + 16, *o_free = bars + 18;
+    uint64_t *drain_bar = bars + 20;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < C::KST; i++) {
             mbar_init(k_full + i, 1);
-            mbar_init(v_full + i, 1);
             mbar_init(k_empty + i, 1);
+        }
+        for (int i = 0; i < C::VST; i++) {
+            mbar_init(v_full + i, 1);
             mbar_init(v_empty + i, 1);
+        }
+        for (int i = 0; i < 2; i++) {
             mbar_init(s_full + i, 1);
             mbar_init(p_full + i, 128);
             mbar_init(pv_done + i, 1);
@@ -224,6 +230,8 @@ __global__ void __launch_bounds__(384, 1)
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
+        prefetch_tmap(&tmK128);
+        prefetch_tmap(&tmV128);
     }
     tc_fence_before();
     __syncthreads();
@@ -236,8 +244,13 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 8) {
         // ------------------------------------------------------- TMA producer
         if (lane == 0) {
+            // K/V rows are re-read by every query item of the head: keep them in
+            // L2; query tiles are read once: let them go first
+            const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
             uint32_t g = 0, qi = 0;
-            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+            int last_k[C::KST], last_v[C::VST];
+            for (int i = 0; i < C::KST; i++) last_k[i] = -1;
+            for (int i = 0; i < C::VST; i++) last_v[i] = -1;
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 const AttnItem it = p.items[item];
@@ -248,39 +261,49 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(q_full, nt * C::Q_BYTES);
                 for (int t = 0; t < nt; t++)
                     for (int kb = 0; kb < C::DB; kb++)
-                        tma_load_2d(sm + C::OFF_Q + t * C::Q_BYTES + kb * (C::BM * 128), &tmQ, q_full, kb * C::EPR,
-                                    it.h * p.N + it.q_start + t * 128);
+                        tma_load_2d_hint(sm + C::OFF_Q + t * C::Q_BYTES + kb * (C::BM * 128), &tmQ, q_full,
+                                         kb * C::EPR, it.h * p.N + it.q_start + t * 128, pol_stream);
                 qi++;
                 int start, len;
                 while (ci.next(start, len)) {
-                    const int st = g & 1;
-                    const uint32_t u = g >> 1;
+                    const int ks = g % C::KST, vs = g % C::VST;
+                    const uint32_t ku = g / C::KST, vu = g / C::VST;
                     const int nb = (len + C::BOX - 1) / C::BOX;
                     const uint32_t bytes = (uint32_t)nb * C::BOX * 128 * C::DB;
                     const int krow = it.h * p.N + start;
-                    if (u >= 1 && !mbar_wait(k_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(k_full + st, bytes);
-                    for (int kb = 0; kb < C::DB; kb++)
-                        for (int b = 0; b < nb; b++)
-                            tma_load_2d(sm + C::OFF_K + st * C::KV_BYTES + kb * (C::BN * 128) + b * (C::BOX * 128),
-                                        &tmK, k_full + st, kb * C::EPR, krow + b * C::BOX);
-                    last_k[st] = (int)u;
-                    if (u >= 1 && !mbar_wait(v_empty + st, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(v_full + st, bytes);
-                    for (int kb = 0; kb < C::DB; kb++)
-                        for (int b = 0; b < nb; b++)
-                            tma_load_2d(sm + C::OFF_V + st * C::KV_BYTES + kb * (C::BN * 128) + b * (C::BOX * 128),
-                                        &tmV, v_full + st, kb * C::EPR, krow + b * C::BOX);
-                    last_v[st] = (int)u;
+                    // a full chunk is one 128-row box per column block; a short
+                    // one is as many 32-row boxes as it needs
+                    if (ku >= 1 && !mbar_wait(k_empty + ks, (ku - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(k_full + ks, bytes);
+                    for (int kb = 0; kb < C::DB; kb++) {
+                        unsigned char *dst = sm + C::OFF_K + ks * C::KV_BYTES + kb * (C::BN * 128);
+                        if (nb == 4) tma_load_2d_hint(dst, &tmK128, k_full + ks, kb * C::EPR, krow, pol_keep);
+                        else
+                            for (int b = 0; b < nb; b++)
+                                tma_load_2d_hint(dst + b * (C::BOX * 128), &tmK, k_full + ks, kb * C::EPR,
+                                                 krow + b * C::BOX, pol_keep);
+                    }
+                    last_k[ks] = (int)ku;
+                    if (vu >= 1 && !mbar_wait(v_empty + vs, (vu - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(v_full + vs, bytes);
+                    for (int kb = 0; kb < C::DB; kb++) {
+                        unsigned char *dst = sm + C::OFF_V + vs * C::KV_BYTES + kb * (C::BN * 128);
+                        if (nb == 4) tma_load_2d_hint(dst, &tmV128, v_full + vs, kb * C::EPR, krow, pol_keep);
+                        else
+                            for (int b = 0; b < nb; b++)
+                                tma_load_2d_hint(dst + b * (C::BOX * 128), &tmV, v_full + vs, kb * C::EPR,
+                                                 krow + b * C::BOX, pol_keep);
+                    }
+                    last_v[vs] = (int)vu;
                     g++;
                 }
             }
             if (!ok) {
                 if (qi >= 1) drain(q_full, (qi - 1) & 1);
-                for (int st = 0; st < 2; st++) {
-                    if (last_k[st] >= 0) drain(k_full + st, last_k[st] & 1);
-                    if (last_v[st] >= 0) drain(v_full + st, last_v[st] & 1);
-                }
+                for (int i = 0; i < C::KST; i++)
+                    if (last_k[i] >= 0) drain(k_full + i, last_k[i] & 1);
+                for (int i = 0; i < C::VST; i++)
+                    if (last_v[i] >= 0) drain(v_full + i, last_v[i] & 1);
             }
         }
     } else if (warp == 9) {
@@ -291,27 +314,38 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t pph[2] = {0, 0};  // p_full phases consumed per tile
             uint32_t act[2] = {0, 0};  // items each tile was active in
             bool ok = true;
-            const uint32_t qbase = smem_u32(sm + C::OFF_Q);
-            // S_t = Q_t K^T for the chunk in ring slot st (ncol key columns)
-            auto issue_s = [&](int t, int st, int ncol) {
+            // Descriptors are built once; per MMA only the start-address field
+            // (16-byte units, bits 0-13) moves by a compile-time offset.  All
+            // shared-memory addresses here are < 256 KB, so the field never carries.
+            const uint64_t qdesc = sdesc_sw128(smem_u32(sm + C::OFF_Q), 16, 1024);
+            const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm + C::OFF_K), 16, 1024);
+            const uint64_t vdesc0 = sdesc_make(smem_u32(sm + C::OFF_V), C::BN * 128, 1024, 2u);
+            // S_t = Q_t K^T for the chunk in K ring slot ks_ (ncol key columns)
+            auto issue_s = [&](int t, int ks_, int ncol) {
                 const uint32_t idesc_s = idesc_make(128, ncol, 1, false);
-                const uint32_t kbase = smem_u32(sm + C::OFF_K + st * C::KV_BYTES);
-                const uint32_t qb = qbase + t * C::Q_BYTES;
-                for (int ks = 0; ks < D / C::KSTEP; ks++) {
-                    const uint32_t off = (ks % 4) * 32;
-                    const uint64_t a = sdesc_sw128(qb + (ks / 4) * (C::BM * 128) + off, 16, 1024);
-                    const uint64_t b = sdesc_sw128(kbase + (ks / 4) * (C::BN * 128) + off, 16, 1024);
-                    umma_f16(tmem + C::TM_S + t * 128, a, b, idesc_s, ks > 0 ? 1u : 0u);
+                const uint32_t d = tmem + C::TM_S + t * 128;
+                uint64_t a = qdesc + (uint64_t)((t * C::Q_BYTES) >> 4);
+                uint64_t b = kdesc0 + (uint64_t)((ks_ * C::KV_BYTES) >> 4);
+                for (int kb = 0; kb < C::DB; kb++) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; k4++)
+                        umma_f16(d, a + 2 * k4, b + 2 * k4, idesc_s, (kb | k4) ? 1u : 0u);
+                    a += (C::BM * 128) >> 4;
+                    b += (C::BN * 128) >> 4;
                 }
                 umma_commit(s_full + t);
             };
-            // O_t (+)= P_t V for ring slot st; P_t is bf16 in TMEM over S_t
-            auto issue_pv = [&](int t, int st, int ncol, bool first) {
-                const uint32_t vbase = smem_u32(sm + C::OFF_V + st * C::KV_BYTES);
-                for (int ks = 0; ks < ncol / C::KSTEP; ks++) {
-                    const uint64_t b = sdesc_make(vbase + ks * C::KSTEP * 128, C::BN * 128, 1024, 2u);
-                    umma_ts_f16(tmem + C::TM_O + t * 128, tmem + C::TM_S + t * 128 + ks * 8, b, idesc_o,
-                                (!first || ks > 0) ? 1u : 0u);
+            // O_t (+)= P_t V for V ring slot vs_; P_t is bf16 in TMEM over S_t
+            auto issue_pv = [&](int t, int vs_, int ncol, bool first) {
+                const uint64_t b0 = vdesc0 + (uint64_t)((vs_ * C::KV_BYTES) >> 4);
+                const uint32_t d = tmem + C::TM_O + t * 128;
+                const uint32_t a0 = tmem + C::TM_S + t * 128;
+                const int nk = ncol / C::KSTEP;
+#pragma unroll
+                for (int ks = 0; ks < C::BN / C::KSTEP; ks++) {
+                    if (ks < nk)
+                        umma_ts_f16(d, a0 + ks * 8, b0 + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc_o,
+                                    (!first || ks > 0) ? 1u : 0u);
                 }
             };
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -326,17 +360,17 @@ __global__ void __launch_bounds__(384, 1)
                 ci.next(start, len);
                 int ncol = (len + 31) & ~31;
                 // prologue: S_t(0)
-                if (!mbar_wait(k_full + (g & 1), (g >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                if (!mbar_wait(k_full + g % C::KST, (g / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
-                for (int t = 0; t < nt; t++) issue_s(t, g & 1, ncol);
-                umma_commit(k_empty + (g & 1));
+                for (int t = 0; t < nt; t++) issue_s(t, g % C::KST, ncol);
+                umma_commit(k_empty + g % C::KST);
                 if (nch == 1) umma_commit(q_empty);
                 for (int j = 0; j < nch && ok; j++) {
-                    const int st = g & 1;
+                    const int st = g % C::VST;
                     int nstart = 0, nlen = 0;
                     const bool more = (j + 1 < nch) && ci.next(nstart, nlen);
                     const int ncol_n = (nlen + 31) & ~31;
-                    if (!mbar_wait(v_full + st, (g >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait(v_full + st, (g / C::VST) & 1, abort_flag, p.status)) { ok = false; break; }
                     for (int t = 0; t < nt; t++) {
                         // PV_t(j) once softmax t has written P_t(j)
                         if (!mbar_wait(p_full + t, pph[t] & 1, abort_flag, p.status)) { ok = false; break; }
@@ -351,9 +385,9 @@ __global__ void __launch_bounds__(384, 1)
                         if (t + 1 == nt) umma_commit(v_empty + st);
                         // S_t(j+1) right behind PV_t(j)
                         if (more) {
-                            const int sn = (g + 1) & 1;
+                            const int sn = (g + 1) % C::KST;
                             if (t == 0 &&
-                                !mbar_wait(k_full + sn, ((g + 1) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                                !mbar_wait(k_full + sn, ((g + 1) / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
                             tc_fence_after();
                             issue_s(t, sn, ncol_n);
                             if (t + 1 == nt) {
@@ -486,7 +520,7 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + pc * 32);
 #pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int i = 0; i < 4; i++) __stcs(dst + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
                 }
             }
             tc_fence_before();
@@ -524,10 +558,11 @@ static int launch2(const void *qg, const void *kg, const void *vg, const A2Param
                    void *encode_fn, cudaStream_t st) {
     using C = A2Cfg<D>;
     EncodeTiledFn2 enc = (EncodeTiledFn2)encode_fn;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mk128, mv128;
     const int rows = p.H * p.N;
     if (bf16_map2(enc, &mq, qg, rows, D, 128) || bf16_map2(enc, &mk, kg, rows, D, C::BOX) ||
-        bf16_map2(enc, &mv, vg, rows, D, C::BOX))
+        bf16_map2(enc, &mv, vg, rows, D, C::BOX) || bf16_map2(enc, &mk128, kg, rows, D, 128) ||
+        bf16_map2(enc, &mv128, vg, rows, D, 128))
         return -1;
     static int checked = 0;  // 1 = ok, -1 = refused
     if (checked == 0) {
@@ -541,16 +576,17 @@ static int launch2(const void *qg, const void *kg, const void *vg, const A2Param
     if (checked != 1) return -1;
     int grid = max_items < num_sms ? max_items : num_sms;
     if (grid < 1) grid = 1;
-    attn2_kernel<D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);
+    attn2_kernel<D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, mk128, mv128, p);
     note_launch();
     return 0;
 }
 
 int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
                  const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap, const int32_t *sel_cnt,
-                 const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
-                 int num_sms, void *encode_fn, cudaStream_t st) {
+                 const int2 *segtab, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
+                 float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st) {
     A2Params p;
+    p.segtab = segtab;
     p.H = H;
     p.N = N;
     p.qperm = qperm;

@@ -67,11 +67,13 @@ int attn_max_items(int H, int N, int kq_cap);
 // bf16: two 128-row query tiles per CTA (ac_attn2.cu); items of up to 256 rows
 int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
                  const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap, const int32_t *sel_cnt,
-                 const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
-                 int num_sms, void *encode_fn, cudaStream_t st);
+                 const int2 *segtab, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
+                 float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st);
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
                 const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
-                const int32_t *sel_cnt, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
-                float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st);
+                const int32_t *sel_cnt, const int2 *segtab, const AttnItem *items, const int32_t *n_items,
+                int max_items, void *out, float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st);
+void k_seg_table(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx,
+                 const int32_t *sel_cnt, int2 *segtab, cudaStream_t st);
 
 }  // namespace ac

@@ -73,3 +73,9 @@ def test_product_does_not_import_oracle():
             "from clustered_sparse_attention_head_b200 import api, _abi; "
             "assert 'oracle' not in sys.modules, 'oracle imported'")
     subprocess.check_call([sys.executable, "-c", code], cwd=ROOT)
+
+
+def test_no_unresolved_internal_symbols(lib):
+    """Every internal launcher the entry points call is defined in the library."""
+    out = subprocess.run(["nm", "-D", "--undefined-only", lib._name], capture_output=True, text=True).stdout
+    assert not [l for l in out.splitlines() if "_ZN2ac" in l], out
