@@ -61,7 +61,7 @@ struct Ws {
     // attention
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
-    size_t chi, clo, xu, amb_cand, items_scr, segtab;
+    size_t chi, clo, xu, amb_cand, items_scr, runs, run_info;
     int kpad;
     size_t total;
 };
@@ -121,7 +121,8 @@ Ws layout(const ac_ctx *c) {
     w.xu = b.take(HN * D * c->elt);
     w.amb_cand = b.take(HN * 8);
     w.items_scr = b.take(items_scratch_elems((int)H, c->kq_cap) * 4 + 16);
-    w.segtab = b.take(H * (size_t)c->kq_cap * c->kk_cap * 8);
+    w.runs = b.take(H * (size_t)c->kq_cap * c->kk_cap * 8);
+    w.run_info = b.take(H * (size_t)c->kq_cap * 8);
     w.total = b.off;
     return w;
 }
@@ -294,16 +295,15 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     const bool two_tiles = (g.dtype == AC_BF16);  // bf16: two query tiles per CTA (items of 256 rows)
     k_build_items(H, N, two_tiles ? 256 : 128, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items,
                   nitems, pairs_dev, at<int32_t>(ws, w.items_scr), st);
-    int2 *segtab = at<int2>(ws, w.segtab);
-    k_seg_table(H, c->kq_cap, c->kk_cap, koff, sel, selc, segtab, st);
+    int2 *runs = at<int2>(ws, w.runs), *run_info = at<int2>(ws, w.run_info);
+    k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN2_CHUNK, runs, run_info, st);
     if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
     int rc;
     if (two_tiles)
-        rc = k_attention2(D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel, c->kq_cap, selc, segtab, items, nitems,
+        rc = k_attention2(D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, items, nitems,
                           attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
     else
-        rc = k_attention(DT_F32, D, H, N, qg, kg, vg, qperm, koff, c->kk_cap, sel, c->kq_cap, selc, segtab, items,
-                         nitems,
+        rc = k_attention(DT_F32, D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, items, nitems,
                          attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
     if (rc != 0) return AC_ERR_CUDA;
     if (ev_kernel) cudaEventRecord(ev_kernel[1], st);

@@ -55,22 +55,20 @@ template <typename T, int D> struct AttnCfg {
 struct AttnParams {
     int H, N;
     const int32_t *qperm;
-    const int32_t *koff;
-    int kk_cap;
-    const int32_t *sel_idx;
-    const int32_t *sel_cnt;
-    int kq_cap;
+    int kk_cap, kq_cap;
+    const int2 *runs;      // per (head, query cluster): ascending key-row runs
+    const int2 *run_info;  // per (head, query cluster): {runs, chunks}
     const AttnItem *items;
     const int32_t *n_items;
     void *out;
     float *lse;
     int *status;
     float scale_log2;
-    const int2 *segtab;
 };
 
-// Walks the key chunks of one work item: every selected key cluster's rows
-// [koff[b], koff[b+1]) (all rows [0, N) for a dense head) in pieces of <= BN.
+// Walks the key chunks of one work item: the rows of every key run (selected
+// key clusters, neighbours merged; all rows [0, N) for a dense head) in pieces
+// of <= BN.
 struct ChunkIter {
     const int2 *seg;
     int nsel, si, cur, end, bn, dense_n;
@@ -80,8 +78,8 @@ struct ChunkIter {
             seg = nullptr;
             nsel = 1;
         } else {
-            seg = p.segtab + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
-            nsel = p.sel_cnt[(size_t)it.h * p.kq_cap + it.a];
+            seg = p.runs + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
+            nsel = p.run_info[(size_t)it.h * p.kq_cap + it.a].x;
         }
         si = -1;
         cur = end = 0;
@@ -521,7 +519,10 @@ __global__ void items_count_kernel(int N, int rpi, int kq_cap, int kk_cap, const
                 long long keys = 0;
                 const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
                 const int ns = sel_cnt[(size_t)h * kq_cap + a];
-                for (int c = 0; c < ns; c++) keys += ko[sl[c] + 1] - ko[sl[c]];
+                for (int c = 0; c < ns; c++) {
+                    const int b = sl[c];
+                    if (b >= 0 && b < kk_cap) keys += ko[b + 1] - ko[b];
+                }
                 pr = (unsigned long long)(keys * qn);
             }
             atomicAdd(&pacc, pr);
@@ -591,26 +592,110 @@ __global__ void items_write_kernel(int N, int rpi, int kq_cap, const int32_t *__
     }
 }
 
-// Segment table: for query cluster a of head h, entry c holds the key rows
-// [koff[b], koff[b+1]) of its c-th selected key cluster b, so the attention
-// kernels read one int2 per segment instead of two dependent loads.
-__global__ void seg_table_kernel(int kq_cap, int kk_cap, const int32_t *__restrict__ koff,
-                                 const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt,
-                                 int2 *__restrict__ segtab) {
-    const int h = blockIdx.y, a = blockIdx.x;
-    const int n = sel_cnt[(size_t)h * kq_cap + a];
-    const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
-    const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
-    int2 *out = segtab + ((size_t)h * kq_cap + a) * kk_cap;
-    for (int c = threadIdx.x; c < n; c += blockDim.x) {
-        const int b = sl[c];
-        out[c] = make_int2(ko[b], ko[b + 1]);
+// Key runs of query cluster a of head h (one CTA each).  A bit set over the
+// key clusters marks the selected ones and the empty ones; each maximal run of
+// marked clusters b0..b1 becomes the row range [koff[b0], koff[b1+1]) of the
+// gathered K/V, in ascending order.  A run of empty clusters only has no rows
+// (the key stream skips it).  Every run's last piece is rounded up to 8 rows
+// and every chunk but the last is full, so the chunk count of KeyStream is
+// ceil(sum of rows rounded up to 8 / chunk_rows).
+constexpr int kRunWords = 8192 / 32;  // key-cluster capacity is at most 8192
+
+__device__ __forceinline__ int run_last(const uint32_t *m, int nw, int b) {
+    int w = b >> 5;
+    uint32_t z = ~m[w] & (~0u << (b & 31));  // unmarked clusters at or after b
+    while (z == 0) {
+        if (++w >= nw) return nw * 32 - 1;
+        z = ~m[w];
     }
+    return w * 32 + __ffs(z) - 2;
 }
 
-void k_seg_table(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx,
-                 const int32_t *sel_cnt, int2 *segtab, cudaStream_t st) {
-    seg_table_kernel<<<dim3(kq_cap, H), 128, 0, st>>>(kq_cap, kk_cap, koff, sel_idx, sel_cnt, segtab);
+__global__ void key_runs_kernel(int kq_cap, int kk_cap, const int32_t *__restrict__ koff,
+                                const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt,
+                                int chunk_rows, int2 *__restrict__ runs, int2 *__restrict__ info) {
+    __shared__ uint32_t m[kRunWords];
+    __shared__ int pre[kRunWords];
+    __shared__ int n_runs;
+    __shared__ unsigned long long slot_rows;
+    const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const int nw = (kk_cap + 31) >> 5;
+    const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
+    const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
+    const int n = min(sel_cnt[(size_t)h * kq_cap + a], kk_cap);
+    int2 *out = runs + ((size_t)h * kq_cap + a) * kk_cap;
+    if (n <= 0) {
+        if (tid == 0) info[(size_t)h * kq_cap + a] = make_int2(0, 0);
+        return;
+    }
+    for (int w = tid; w < nw; w += nt) {
+        uint32_t e = 0;
+        for (int i = 0; i < 32; i++) {
+            const int b = w * 32 + i;
+            if (b < kk_cap && ko[b + 1] == ko[b]) e |= 1u << i;
+        }
+        m[w] = e;
+    }
+    if (tid == 0) slot_rows = 0ull;
+    __syncthreads();
+    for (int c = tid; c < n; c += nt) {
+        const int b = sl[c];
+        if (b >= 0 && b < kk_cap) atomicOr(&m[b >> 5], 1u << (b & 31));
+    }
+    __syncthreads();
+    // run starts per word, exclusive prefix over words (warp 0, 8 words a lane)
+    if (tid < 32) {
+        int cnt[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int w = tid * 8 + i;
+            int c = 0;
+            if (w < nw) {
+                const uint32_t prev = w > 0 ? m[w - 1] >> 31 : 0u;
+                c = __popc(m[w] & ~((m[w] << 1) | prev));
+            }
+            cnt[i] = c;
+            sum += c;
+        }
+        int x = sum;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (tid >= d) x += y;
+        }
+        int base = x - sum;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int w = tid * 8 + i;
+            if (w < kRunWords) pre[w] = base;
+            base += cnt[i];
+        }
+        if (tid == 31) n_runs = x;
+    }
+    __syncthreads();
+    unsigned long long my_rows = 0ull;
+    for (int w = tid; w < nw; w += nt) {
+        const uint32_t prev = w > 0 ? m[w - 1] >> 31 : 0u;
+        uint32_t st = m[w] & ~((m[w] << 1) | prev);
+        int k = pre[w];
+        while (st) {
+            const int b = w * 32 + __ffs(st) - 1;
+            st &= st - 1;
+            const int e = run_last(m, nw, b);
+            const int r0 = ko[b], r1 = ko[e + 1];
+            out[k++] = make_int2(r0, r1);
+            my_rows += (unsigned long long)((r1 - r0 + 7) & ~7);
+        }
+    }
+    if (my_rows) atomicAdd(&slot_rows, my_rows);
+    __syncthreads();
+    if (tid == 0)
+        info[(size_t)h * kq_cap + a] =
+            make_int2(n_runs, (int)((slot_rows + (unsigned long long)chunk_rows - 1) / (unsigned long long)chunk_rows));
+}
+
+void k_key_runs(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx, const int32_t *sel_cnt,
+                int chunk_rows, int2 *runs, int2 *info, cudaStream_t st) {
+    key_runs_kernel<<<dim3(kq_cap, H), 128, 0, st>>>(kq_cap, kk_cap, koff, sel_idx, sel_cnt, chunk_rows, runs, info);
     note_launch();
 }
 
@@ -677,19 +762,17 @@ static int launch_attn(const void *qg, const void *kg, const void *vg, const Att
 }
 
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
-                const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
-                const int32_t *sel_cnt, const int2 *segtab, const AttnItem *items, const int32_t *n_items,
-                int max_items, void *out, float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st) {
+                const int32_t *qperm, int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info,
+                const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
+                int num_sms, void *encode_fn, cudaStream_t st) {
     AttnParams p;
-    p.segtab = segtab;
     p.H = H;
     p.N = N;
     p.qperm = qperm;
-    p.koff = koff;
     p.kk_cap = kk_cap;
-    p.sel_idx = sel_idx;
-    p.sel_cnt = sel_cnt;
     p.kq_cap = kq_cap;
+    p.runs = runs;
+    p.run_info = run_info;
     p.items = items;
     p.n_items = n_items;
     p.out = out;

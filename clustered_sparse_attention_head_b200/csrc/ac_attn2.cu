@@ -3,20 +3,20 @@
 // per CTA.
 //
 // A work item is up to 256 query rows of one query cluster (two 128-row
-// tiles) that share one key stream: the rows of every selected key cluster of
-// the gathered K/V, in chunks of <= 128 keys (TMA, 32-row boxes, 2-stage ring).
-// Per chunk j and tile t the single MMA thread issues S_t(j) = Q_t K_j^T into
-// TMEM and, once softmax warpgroup t has written P_t(j) (bf16) back into the
-// same TMEM columns, O_t += P_t(j) V_j with the A operand read from TMEM.  The
-// issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) lets each tile's softmax
-// run while the tensor core works on the other tile.
-//
+// tiles) that share one key stream (KeyStream): the rows of the cluster's key
+// runs packed into chunks of 64 keys, loaded by TMA into 4-stage K and V rings.
+// Each tile owns two S buffers in TMEM, so while softmax warpgroup t turns
+// S_t(j) into P_t(j) (bf16, written back over the same columns) the tensor
+// core already computes S_t(j+1) in the other buffer.  The single MMA thread
+// issues, per chunk j and tile t,
+//   O_t += P_t(j) V_j          (A operand read from TMEM) once P_t(j) is written,
+//   S_t(j+2) = Q_t K_{j+2}^T   into the buffer that P_t(j) occupied.
 // Ordering facts the protocol relies on (tcgen05 operations issued by one
-// thread complete in issue order, and a commit covers all earlier ones):
-//  - S_t(j+1) is issued after PV_t(j), so it never overwrites P_t(j) early;
-//  - the commit after S_t(j) also covers PV_t(j-1), so when S_t(j) is ready
-//    the softmax may both overwrite the P_t columns and rescale O_t;
-//  - only the epilogue waits for the item's last PV_t (pv_done[t]).
+// thread execute in issue order, and a commit covers all earlier ones):
+//  - S_t(j+2) is issued after PV_t(j), so it never overwrites P_t(j) early;
+//  - once S_t(j) is complete, so is PV_t(j-2), the last reader of its buffer;
+//  - PV_t(j-1) may still run while the softmax works on chunk j, so before it
+//    rescales O_t the softmax waits for the P.V barrier phase of chunk j-1.
 // Every mbarrier wait is bounded; on expiry the CTA records ST_TIMEOUT,
 // drains its copies and MMAs, frees TMEM and returns.
 #include "ac_kernels.cuh"
@@ -24,85 +24,63 @@
 namespace ac {
 
 template <int D> struct A2Cfg {
-    static constexpr int BM = 128, BN = 128, EPR = 64, DB = D / 64, BOX = 32, KSTEP = 16;
+    static constexpr int BM = 128, BN = ATTN2_CHUNK, DB = D / 64, KSTEP = 16;
     static constexpr int Q_BYTES = BM * D * 2;     // one query tile
     static constexpr int KV_BYTES = BN * D * 2;    // one stage of K (or of V)
-    // K is consumed by S right away; V only after the softmax, so V gets the
-    // deeper ring (its loads must start further ahead of their use)
-    static constexpr int KST = 2, VST = 3;
+    static constexpr int KST = 4, VST = 4;
     static constexpr int OFF_Q = 0;                // tile 1 at + Q_BYTES
     static constexpr int OFF_K = 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-    static constexpr int SMEM_RAW = OFF_BAR + 256 + 1024;
+    static constexpr int SMEM_RAW = OFF_BAR + 512 + 1024;
     // at least 116 KB so that two CTAs never share an SM (each takes all of TMEM)
     static constexpr int SMEM = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
     // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle:
     // three full warpgroups, so registers can move between them (setmaxnreg)
     static constexpr int NTHREADS = 384;
-    static constexpr int REGS_LAUNCH = 168, REGS_LOW = 56, REGS_HIGH = 224;
+    static constexpr int REGS_LAUNCH = 168, REGS_LOW = 88, REGS_HIGH = 208;
     static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= NTHREADS * REGS_LAUNCH, "register split");
-    static constexpr uint32_t TMEM_COLS = 512;     // S/P 0, S/P 1, O 0, O 1
-    static constexpr int TM_S = 0, TM_O = 256;     // + 128 t
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int TM_S = 0;                 // + 128 t + 64 buffer
+    static constexpr int TM_O = 256;               // + D t
+    static_assert(TM_O + 2 * D <= (int)TMEM_COLS, "TMEM budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct A2Params {
     int H, N;
     const int32_t *qperm;
-    const int32_t *koff;
-    int kk_cap;
-    const int32_t *sel_idx;
-    const int32_t *sel_cnt;
-    int kq_cap;
+    int kk_cap, kq_cap;
+    const int2 *runs;      // per (head, query cluster): ascending key-row runs
+    const int2 *run_info;  // per (head, query cluster): {runs, chunks}
     const AttnItem *items;
     const int32_t *n_items;
     __nv_bfloat16 *out;
     float *lse;
     int *status;
     float scale_log2;
-    const int2 *segtab;  // per (head, query cluster): key rows of each selected cluster
+};
+
+// K or V tensor maps of one operand, one per box height (64, 32, 16, 8 rows).
+struct KVMaps {
+    CUtensorMap m64, m32, m16, m8;
 };
 
 namespace {
 
-struct Chunks {
-    const int2 *seg;
-    int nsel, si, cur, end, dense_n;
-    int2 nxt;
-    __device__ void init(const A2Params &p, const AttnItem &it) {
-        if (it.a < 0) {
-            seg = nullptr;
-            nsel = 1;
-        } else {
-            seg = p.segtab + ((size_t)it.h * p.kq_cap + it.a) * p.kk_cap;
-            nsel = p.sel_cnt[(size_t)it.h * p.kq_cap + it.a];
-        }
-        si = -1;
-        cur = end = 0;
-        dense_n = p.N;
-        nxt = (seg && nsel > 0) ? seg[0] : make_int2(0, p.N);
+__device__ __forceinline__ int item_chunks(const A2Params &p, const AttnItem &it) {
+    if (it.a < 0) return (p.N + ATTN2_CHUNK - 1) / ATTN2_CHUNK;
+    return p.run_info[(size_t)it.h * p.kq_cap + it.a].y;
+}
+
+__device__ __forceinline__ void stream_init(KeyStream &ks, const A2Params &p, const AttnItem &it) {
+    if (it.a < 0) {
+        ks.init(nullptr, 1, p.N);
+    } else {
+        const size_t qa = (size_t)it.h * p.kq_cap + it.a;
+        ks.init(p.runs + qa * p.kk_cap, p.run_info[qa].x, p.N);
     }
-    __device__ bool next(int &start, int &len) {
-        while (cur >= end) {
-            if (++si >= nsel) return false;
-            cur = nxt.x;
-            end = nxt.y;
-            if (seg && si + 1 < nsel) nxt = seg[si + 1];  // one segment ahead
-        }
-        start = cur;
-        len = min(128, end - cur);
-        cur += len;
-        return true;
-    }
-    __device__ int count(const A2Params &p, const AttnItem &it) {
-        init(p, it);
-        int n = 0, s, l;
-        while (next(s, l)) n++;
-        init(p, it);
-        return n;
-    }
-};
+}
 
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
     const bool ok = mbar_wait(bar, parity, abort_flag, status);
@@ -115,7 +93,7 @@ __device__ __forceinline__ void drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
-// O += P V with A (P, bf16) read from TMEM columns a_col.. (two per 32-bit column).
+// O += P V with A (P, bf16) read from TMEM columns a_tmem.. (two per 32-bit column).
 __device__ __forceinline__ void umma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
@@ -123,24 +101,6 @@ __device__ __forceinline__ void umma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, ui
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
-        "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
-        "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
-        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
-        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]),
-        "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]),
-        "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]),
-        "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]),
-        "r"(r[63])
         : "memory");
 }
 
@@ -180,25 +140,91 @@ __device__ __forceinline__ float ex2_fma(float x) {
     return __int_as_float(__float_as_int(q) + (n << 23));
 }
 
+// `rows` (a multiple of 8, at most 64) rows from global row `grow` into rows
+// r0.. of one K or V stage: one box per set bit of `rows`, per 64-column block.
+template <int D>
+__device__ __forceinline__ void load_rows(unsigned char *stage, int r0, int grow, int rows, const KVMaps &m,
+                                          uint64_t *bar, uint64_t pol) {
+    using C = A2Cfg<D>;
+#pragma unroll
+    for (int kb = 0; kb < C::DB; kb++) {
+        unsigned char *dst = stage + kb * (C::BN * 128);
+        int r = r0, g = grow;
+        if (rows & 64) { tma_load_2d_hint(dst + r * 128, &m.m64, bar, kb * 64, g, pol); r += 64; g += 64; }
+        if (rows & 32) { tma_load_2d_hint(dst + r * 128, &m.m32, bar, kb * 64, g, pol); r += 32; g += 32; }
+        if (rows & 16) { tma_load_2d_hint(dst + r * 128, &m.m16, bar, kb * 64, g, pol); r += 16; g += 16; }
+        if (rows & 8) tma_load_2d_hint(dst + r * 128, &m.m8, bar, kb * 64, g, pol);
+    }
+}
+
+// The next chunk of the stream into one stage: each piece into its slot, and,
+// when the chunk ends on an odd multiple of 8 rows, 8 more rows after the last
+// piece (finite data under masked columns, so that 0 * V stays 0).
+template <int D>
+__device__ __forceinline__ void load_chunk(KeyStream &ks, unsigned char *stage, int row_base, const KVMaps &m,
+                                           uint64_t *bar, uint64_t pol) {
+    using C = A2Cfg<D>;
+    int fill = 0, start = 0, valid = 0, slot = 0, after = 0;
+    while (fill < C::BN && ks.piece(C::BN - fill, start, valid, slot)) {
+        load_rows<D>(stage, fill, row_base + start, slot, m, bar, pol);
+        fill += slot;
+        after = start + slot;
+    }
+    if (fill & 8) load_rows<D>(stage, fill, row_base + after, 8, m, bar, pol);
+}
+
+// S_t = Q_t K^T into TMEM columns d (ncol keys of one K stage)
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t d, uint64_t qdesc_t, uint64_t kdesc_stage, int ncol) {
+    using C = A2Cfg<D>;
+    // ncol >= 16 whenever the stream and the chunk count agree (they are built
+    // from the same runs); the clamp only keeps the instruction shape legal
+    const uint32_t idesc = idesc_make(128, ncol < 16 ? 16 : ncol, 1, false);
+    uint64_t a = qdesc_t, b = kdesc_stage;
+#pragma unroll
+    for (int kb = 0; kb < C::DB; kb++) {
+#pragma unroll
+        for (int k4 = 0; k4 < 4; k4++) umma_f16(d, a + 2 * k4, b + 2 * k4, idesc, (kb | k4) ? 1u : 0u);
+        a += (C::BM * 128) >> 4;
+        b += (C::BN * 128) >> 4;
+    }
+}
+
+// O_t (+)= P_t V for the first ncol keys of one V stage; P_t is bf16 in TMEM at a0
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t a0, uint64_t vdesc_stage, int ncol, bool first) {
+    using C = A2Cfg<D>;
+    const uint32_t idesc = idesc_make(128, D, 1, true);
+    const int nk = ncol / C::KSTEP;
+#pragma unroll
+    for (int ks = 0; ks < C::BN / C::KSTEP; ks++)
+        if (ks < nk)
+            umma_ts_f16(d, a0 + ks * 8, vdesc_stage + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc,
+                        (!first || ks > 0) ? 1u : 0u);
+}
+
 }  // namespace
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
-    attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK128,
-                 const __grid_constant__ CUtensorMap tmV128, const A2Params p) {
+    attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KVMaps mk,
+                 const __grid_constant__ KVMaps mv, const A2Params p) {
     using C = A2Cfg<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                           ~(uintptr_t)1023);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
     uint64_t *q_full = bars + 0, *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2, *k_empty = bars + 4;             // [KST]
-    uint64_t *v_full = bars + 6, *v_empty = bars + 9;             // [VST]
-    uint64_t *s_full = bars + 12, *p_full = bars + 14, *pv_done = bars + 16, *o_free = bars + 18;
-    uint64_t *drain_bar = bars + 20;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
+    uint64_t *k_full = bars + 2, *k_empty = k_full + C::KST;   // [KST]
+    uint64_t *v_full = k_empty + C::KST, *v_empty = v_full + C::VST;  // [VST]
+    uint64_t *s_full = v_empty + C::VST;    // [tile][buffer]
+    uint64_t *p_full = s_full + 4;          // [tile][buffer], 128 arrivals
+    uint64_t *pv_bar = p_full + 4;          // [tile]: one phase per P.V
+    uint64_t *o_free = pv_bar + 2;          // [tile], 128 arrivals
+    uint64_t *o_done = o_free + 2;          // [tile]: one phase per item, after its last P.V
+    uint64_t *drain_bar = o_done + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(drain_bar + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -212,11 +238,14 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(v_full + i, 1);
             mbar_init(v_empty + i, 1);
         }
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < 4; i++) {
             mbar_init(s_full + i, 1);
             mbar_init(p_full + i, 128);
-            mbar_init(pv_done + i, 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(pv_bar + i, 1);
             mbar_init(o_free + i, 128);
+            mbar_init(o_done + i, 1);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -228,10 +257,14 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (warp == 8 && lane == 0) {
         prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        prefetch_tmap(&tmK128);
-        prefetch_tmap(&tmV128);
+        prefetch_tmap(&mk.m64);
+        prefetch_tmap(&mk.m32);
+        prefetch_tmap(&mk.m16);
+        prefetch_tmap(&mk.m8);
+        prefetch_tmap(&mv.m64);
+        prefetch_tmap(&mv.m32);
+        prefetch_tmap(&mv.m16);
+        prefetch_tmap(&mv.m8);
     }
     tc_fence_before();
     __syncthreads();
@@ -248,70 +281,53 @@ __global__ void __launch_bounds__(384, 1)
             // L2; query tiles are read once: let them go first
             const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
             uint32_t g = 0, qi = 0;
-            int last_k[C::KST], last_v[C::VST];
-            for (int i = 0; i < C::KST; i++) last_k[i] = -1;
-            for (int i = 0; i < C::VST; i++) last_v[i] = -1;
+            uint32_t nk_loads = 0, nv_loads = 0;  // chunks whose K / V copies were issued
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 const AttnItem it = p.items[item];
-                Chunks ci;
-                if (ci.count(p, it) == 0) continue;
+                const int nch = item_chunks(p, it);
+                if (nch == 0) continue;
                 const int nt = it.q_len > 128 ? 2 : 1;
                 if (qi >= 1 && !mbar_wait(q_empty, (qi - 1) & 1, abort_flag, p.status)) { ok = false; break; }
                 mbar_arrive_expect_tx(q_full, nt * C::Q_BYTES);
                 for (int t = 0; t < nt; t++)
                     for (int kb = 0; kb < C::DB; kb++)
                         tma_load_2d_hint(sm + C::OFF_Q + t * C::Q_BYTES + kb * (C::BM * 128), &tmQ, q_full,
-                                         kb * C::EPR, it.h * p.N + it.q_start + t * 128, pol_stream);
+                                         kb * 64, it.h * p.N + it.q_start + t * 128, pol_stream);
                 qi++;
-                int start, len;
-                while (ci.next(start, len)) {
-                    const int ks = g % C::KST, vs = g % C::VST;
+                KeyStream ks;
+                stream_init(ks, p, it);
+                const int row_base = it.h * p.N;
+                for (int j = 0; j < nch; j++, g++) {
+                    KeyStream kk = ks, probe = ks;
+                    const uint32_t bytes = (uint32_t)probe.chunk(C::BN) * 128u * C::DB;
+                    const int kslot = g % C::KST, vslot = g % C::VST;
                     const uint32_t ku = g / C::KST, vu = g / C::VST;
-                    const int nb = (len + C::BOX - 1) / C::BOX;
-                    const uint32_t bytes = (uint32_t)nb * C::BOX * 128 * C::DB;
-                    const int krow = it.h * p.N + start;
-                    // a full chunk is one 128-row box per column block; a short
-                    // one is as many 32-row boxes as it needs
-                    if (ku >= 1 && !mbar_wait(k_empty + ks, (ku - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(k_full + ks, bytes);
-                    for (int kb = 0; kb < C::DB; kb++) {
-                        unsigned char *dst = sm + C::OFF_K + ks * C::KV_BYTES + kb * (C::BN * 128);
-                        if (nb == 4) tma_load_2d_hint(dst, &tmK128, k_full + ks, kb * C::EPR, krow, pol_keep);
-                        else
-                            for (int b = 0; b < nb; b++)
-                                tma_load_2d_hint(dst + b * (C::BOX * 128), &tmK, k_full + ks, kb * C::EPR,
-                                                 krow + b * C::BOX, pol_keep);
-                    }
-                    last_k[ks] = (int)ku;
-                    if (vu >= 1 && !mbar_wait(v_empty + vs, (vu - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(v_full + vs, bytes);
-                    for (int kb = 0; kb < C::DB; kb++) {
-                        unsigned char *dst = sm + C::OFF_V + vs * C::KV_BYTES + kb * (C::BN * 128);
-                        if (nb == 4) tma_load_2d_hint(dst, &tmV128, v_full + vs, kb * C::EPR, krow, pol_keep);
-                        else
-                            for (int b = 0; b < nb; b++)
-                                tma_load_2d_hint(dst + b * (C::BOX * 128), &tmV, v_full + vs, kb * C::EPR,
-                                                 krow + b * C::BOX, pol_keep);
-                    }
-                    last_v[vs] = (int)vu;
-                    g++;
+                    if (ku >= 1 && !mbar_wait(k_empty + kslot, (ku - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(k_full + kslot, bytes);
+                    load_chunk<D>(kk, sm + C::OFF_K + kslot * C::KV_BYTES, row_base, mk, k_full + kslot, pol_keep);
+                    nk_loads = g + 1;
+                    if (vu >= 1 && !mbar_wait(v_empty + vslot, (vu - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(v_full + vslot, bytes);
+                    load_chunk<D>(ks, sm + C::OFF_V + vslot * C::KV_BYTES, row_base, mv, v_full + vslot, pol_keep);
+                    nv_loads = g + 1;
                 }
             }
             if (!ok) {
+                // wait (bounded) for every copy in flight before the CTA exits
+                // (slot i last received chunk i + KST * ((loads - 1 - i) / KST))
                 if (qi >= 1) drain(q_full, (qi - 1) & 1);
-                for (int i = 0; i < C::KST; i++)
-                    if (last_k[i] >= 0) drain(k_full + i, last_k[i] & 1);
-                for (int i = 0; i < C::VST; i++)
-                    if (last_v[i] >= 0) drain(v_full + i, last_v[i] & 1);
+                for (uint32_t i = 0; i < (uint32_t)C::KST && i < nk_loads; i++)
+                    drain(k_full + i, ((nk_loads - 1 - i) / C::KST) & 1);
+                for (uint32_t i = 0; i < (uint32_t)C::VST && i < nv_loads; i++)
+                    drain(v_full + i, ((nv_loads - 1 - i) / C::VST) & 1);
             }
         }
     } else if (warp == 9) {
         // --------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_o = idesc_make(128, D, 1, true);
             uint32_t g = 0, qi = 0;
-            uint32_t pph[2] = {0, 0};  // p_full phases consumed per tile
+            uint32_t cnt[2] = {0, 0};  // chunks each tile has been through
             uint32_t act[2] = {0, 0};  // items each tile was active in
             bool ok = true;
             // Descriptors are built once; per MMA only the start-address field
@@ -320,86 +336,86 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t qdesc = sdesc_sw128(smem_u32(sm + C::OFF_Q), 16, 1024);
             const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm + C::OFF_K), 16, 1024);
             const uint64_t vdesc0 = sdesc_make(smem_u32(sm + C::OFF_V), C::BN * 128, 1024, 2u);
-            // S_t = Q_t K^T for the chunk in K ring slot ks_ (ncol key columns)
-            auto issue_s = [&](int t, int ks_, int ncol) {
-                const uint32_t idesc_s = idesc_make(128, ncol, 1, false);
-                const uint32_t d = tmem + C::TM_S + t * 128;
-                uint64_t a = qdesc + (uint64_t)((t * C::Q_BYTES) >> 4);
-                uint64_t b = kdesc0 + (uint64_t)((ks_ * C::KV_BYTES) >> 4);
-                for (int kb = 0; kb < C::DB; kb++) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; k4++)
-                        umma_f16(d, a + 2 * k4, b + 2 * k4, idesc_s, (kb | k4) ? 1u : 0u);
-                    a += (C::BM * 128) >> 4;
-                    b += (C::BN * 128) >> 4;
-                }
-                umma_commit(s_full + t);
-            };
-            // O_t (+)= P_t V for V ring slot vs_; P_t is bf16 in TMEM over S_t
-            auto issue_pv = [&](int t, int vs_, int ncol, bool first) {
-                const uint64_t b0 = vdesc0 + (uint64_t)((vs_ * C::KV_BYTES) >> 4);
-                const uint32_t d = tmem + C::TM_O + t * 128;
-                const uint32_t a0 = tmem + C::TM_S + t * 128;
-                const int nk = ncol / C::KSTEP;
-#pragma unroll
-                for (int ks = 0; ks < C::BN / C::KSTEP; ks++) {
-                    if (ks < nk)
-                        umma_ts_f16(d, a0 + ks * 8, b0 + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc_o,
-                                    (!first || ks > 0) ? 1u : 0u);
-                }
-            };
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 const AttnItem it = p.items[item];
-                Chunks ci;
-                const int nch = ci.count(p, it);
+                const int nch = item_chunks(p, it);
                 if (nch == 0) continue;
                 const int nt = it.q_len > 128 ? 2 : 1;
                 if (!mbar_wait(q_full, qi & 1, abort_flag, p.status)) { ok = false; break; }
                 qi++;
-                int start, len;
-                ci.next(start, len);
-                int ncol = (len + 31) & ~31;
-                // prologue: S_t(0)
-                if (!mbar_wait(k_full + g % C::KST, (g / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
-                tc_fence_after();
-                for (int t = 0; t < nt; t++) issue_s(t, g % C::KST, ncol);
-                umma_commit(k_empty + g % C::KST);
-                if (nch == 1) umma_commit(q_empty);
+                KeyStream ks;
+                stream_init(ks, p, it);
+                // prologue: S_t(0) and S_t(1)
+                int n0 = ks.chunk(C::BN), n1 = nch > 1 ? ks.chunk(C::BN) : 0, n2 = 0;
+                for (int jj = 0; jj < 2 && jj < nch && ok; jj++) {
+                    const uint32_t gk = g + jj;
+                    const int kslot = gk % C::KST;
+                    if (!mbar_wait(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int t = 0; t < 2; t++) {
+                        if (t >= nt) break;
+                        const int b = (cnt[t] + jj) & 1;
+                        issue_s<D>(tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
+                                   kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4), jj == 0 ? n0 : n1);
+                        umma_commit(s_full + 2 * t + b);
+                    }
+                    umma_commit(k_empty + kslot);
+                }
+                if (!ok) break;
+                if (nch <= 2) umma_commit(q_empty);
                 for (int j = 0; j < nch && ok; j++) {
-                    const int st = g % C::VST;
-                    int nstart = 0, nlen = 0;
-                    const bool more = (j + 1 < nch) && ci.next(nstart, nlen);
-                    const int ncol_n = (nlen + 31) & ~31;
-                    if (!mbar_wait(v_full + st, (g / C::VST) & 1, abort_flag, p.status)) { ok = false; break; }
-                    for (int t = 0; t < nt; t++) {
+                    const uint32_t gv = g + j;
+                    const int vslot = gv % C::VST;
+                    if (!mbar_wait(v_full + vslot, (gv / C::VST) & 1, abort_flag, p.status)) { ok = false; break; }
+                    const bool more = j + 2 < nch;
+                    if (more) n2 = ks.chunk(C::BN);
+                    const uint32_t gk = g + j + 2;
+                    const int kslot = gk % C::KST;
+#pragma unroll
+                    for (int t = 0; t < 2; t++) {
+                        if (t >= nt) break;
+                        const uint32_t c = cnt[t] + j;
+                        const int b = c & 1;
                         // PV_t(j) once softmax t has written P_t(j)
-                        if (!mbar_wait(p_full + t, pph[t] & 1, abort_flag, p.status)) { ok = false; break; }
-                        pph[t]++;
+                        if (!mbar_wait(p_full + 2 * t + b, (c >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
                         if (j == 0 && act[t] >= 1 && !mbar_wait(o_free + t, (act[t] - 1) & 1, abort_flag, p.status)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        issue_pv(t, st, ncol, j == 0);
-                        if (j + 1 == nch) umma_commit(pv_done + t);
-                        if (t + 1 == nt) umma_commit(v_empty + st);
-                        // S_t(j+1) right behind PV_t(j)
+                        issue_pv<D>(tmem + C::TM_O + t * D, tmem + C::TM_S + t * 128 + b * 64,
+                                    vdesc0 + (uint64_t)((vslot * C::KV_BYTES) >> 4), n0, j == 0);
+                        umma_commit(pv_bar + t);
+                        if (j + 1 == nch) umma_commit(o_done + t);
+                        // S_t(j+2) into the buffer P_t(j) occupied
                         if (more) {
-                            const int sn = (g + 1) % C::KST;
-                            if (t == 0 &&
-                                !mbar_wait(k_full + sn, ((g + 1) / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
-                            tc_fence_after();
-                            issue_s(t, sn, ncol_n);
-                            if (t + 1 == nt) {
-                                umma_commit(k_empty + sn);
-                                if (j + 2 == nch) umma_commit(q_empty);
+                            if (t == 0 && !mbar_wait(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) {
+                                ok = false;
+                                break;
                             }
+                            tc_fence_after();
+                            issue_s<D>(tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
+                                       kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4), n2);
+                            umma_commit(s_full + 2 * t + b);
                         }
                     }
-                    ncol = ncol_n;
-                    g++;
+                    if (!ok) break;
+                    umma_commit(v_empty + vslot);
+                    if (more) {
+                        umma_commit(k_empty + kslot);
+                        if (j + 3 == nch) umma_commit(q_empty);
+                    }
+                    n0 = n1;
+                    n1 = n2;
                 }
-                for (int t = 0; t < nt; t++) act[t]++;
+                g += nch;
+                cnt[0] += nch;
+                act[0]++;
+                if (nt > 1) {
+                    cnt[1] += nch;
+                    act[1]++;
+                }
             }
             if (!ok) {
                 umma_commit(drain_bar);
@@ -415,17 +431,17 @@ __global__ void __launch_bounds__(384, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const uint32_t s_addr = tmem + lane_addr + C::TM_S + t * 128;
-        const uint32_t o_addr = tmem + lane_addr + C::TM_O + t * 128;
+        const uint32_t s_base = tmem + lane_addr + C::TM_S + t * 128;
+        const uint32_t o_addr = tmem + lane_addr + C::TM_O + t * D;
         const float sc = p.scale_log2;
-        uint32_t sph = 0, act = 0;
+        uint32_t cnt = 0;         // chunks (= pv_bar phases) this tile has been through
+        uint32_t items_done = 0;  // items (= o_done phases) this tile has finished
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const AttnItem it = p.items[item];
             const int nt = it.q_len > 128 ? 2 : 1;
             if (t >= nt) continue;
-            Chunks ci;
-            const int nch = ci.count(p, it);
+            const int nch = item_chunks(p, it);
             const int r = t * 128 + row;
             const bool valid = r < it.q_len;
             int tok = 0;
@@ -438,30 +454,52 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 continue;
             }
+            KeyStream ks;
+            stream_init(ks, p, it);
             float m_ref = -INFINITY, l0 = 0.f, l1 = 0.f;
-            int start, len;
             for (int j = 0; j < nch; j++) {
-                ci.next(start, len);
-                if (!wait_warp(s_full + t, sph & 1, abort_flag, p.status)) { ok = false; break; }
-                sph++;
+                // valid rows per 8-row group of the chunk, 4 bits each (8 = all)
+                uint32_t gm = 0;
+                {
+                    int fill = 0, start, v, sl;
+                    while (fill < C::BN && ks.piece(C::BN - fill, start, v, sl)) {
+                        const int g0 = fill >> 3, nf = v >> 3;
+                        gm |= ((nf >= 8 ? 0xFFFFFFFFu : ((1u << (4 * nf)) - 1u)) & 0x88888888u) << (4 * g0);
+                        if (v & 7) gm |= (uint32_t)(v & 7) << (4 * (g0 + nf));
+                        fill += sl;
+                    }
+                }
+                const uint32_t c = cnt + j;
+                const int b = c & 1;
+                if (!wait_warp(s_full + 2 * t + b, (c >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t s[128];
-                tmem_ld128(s_addr, s);
-                if (len < 128) {
+                uint32_t s[64];
+                tmem_ld64(s_base + b * 64, s);
+                if (gm != 0x88888888u) {
 #pragma unroll
-                    for (int i = 0; i < 128; i++)
-                        if (i >= len) s[i] = __float_as_uint(-INFINITY);
+                    for (int gi = 0; gi < 8; gi++) {
+                        const uint32_t nv = (gm >> (4 * gi)) & 15u;
+                        if (nv != 8u) {
+#pragma unroll
+                            for (int i = 0; i < 8; i++)
+                                if ((uint32_t)i >= nv) s[8 * gi + i] = __float_as_uint(-INFINITY);
+                        }
+                    }
                 }
                 float mx = __uint_as_float(s[0]);
 #pragma unroll
-                for (int i = 1; i + 1 < 128; i += 2) mx = max3(mx, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-                mx = fmaxf(mx, __uint_as_float(s[127]));
+                for (int i = 1; i + 1 < 64; i += 2) mx = max3(mx, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+                mx = fmaxf(mx, __uint_as_float(s[63]));
                 const float m_new = mx * sc;
                 if (j == 0) m_ref = m_new;
                 // Move the reference max (and rescale O_t) only when it grew by
                 // more than 2^8; warp-uniform because TMEM access is collective.
-                // PV_t(j-1) is complete: the commit of S_t(j) covers it.
+                // PV_t(j-1) may still be accumulating into O_t: wait for it.  Its
+                // pv_bar phase is unambiguous here: PV_t(j-2) is complete (S_t(j)
+                // was issued after it) and PV_t(j) is not issued yet.
                 if (j > 0 && __any_sync(0xffffffffu, m_new > m_ref + 8.f)) {
+                    if (!wait_warp(pv_bar + t, (c - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
                     const float m_to = fmaxf(m_ref, m_new);
                     const float f = ex2_approx(m_ref - m_to);
                     l0 *= f;
@@ -478,31 +516,28 @@ __global__ void __launch_bounds__(384, 1)
                     m_ref = m_to;
                 }
                 const float nm = -m_ref;
+                uint32_t pk[32];
 #pragma unroll
-                for (int hh = 0; hh < 2; hh++) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        const int e = hh * 64 + 2 * i;
-                        float x0, x1;
-                        fma2(x0, x1, __uint_as_float(s[e]), __uint_as_float(s[e + 1]), sc, nm);
-                        const float e0 = ex2_approx(x0);
-                        const float e1 = (i & 1) ? ex2_fma(x1) : ex2_approx(x1);
-                        l0 += e0;
-                        l1 += e1;
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-                        pk[i] = *reinterpret_cast<uint32_t *>(&b2);
-                    }
-                    tmem_st32(s_addr + hh * 32, pk);
+                for (int i = 0; i < 32; i++) {
+                    float x0, x1;
+                    fma2(x0, x1, __uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]), sc, nm);
+                    const float e0 = ex2_approx(x0);
+                    const float e1 = (i & 1) ? ex2_fma(x1) : ex2_approx(x1);
+                    l0 += e0;
+                    l1 += e1;
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+                    pk[i] = *reinterpret_cast<uint32_t *>(&b2);
                 }
+                tmem_st32(s_base + b * 64, pk);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(p_full + t);
+                mbar_arrive(p_full + 2 * t + b);
             }
             if (!ok) break;
-            // epilogue: O_t / l, rows scattered back to token order
-            if (!wait_warp(pv_done + t, act & 1, abort_flag, p.status)) { ok = false; break; }
-            act++;
+            // epilogue: O_t / l once the last P.V is done, rows scattered back to
+            // token order.  (A parity wait on pv_bar cannot tell that phase from
+            // the one before it while P.V(j-1) may still run, hence o_done.)
+            if (!wait_warp(o_done + t, items_done & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
             const float lsum = l0 + l1;
             const float inv = 1.f / lsum;
@@ -526,6 +561,8 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before();
             mbar_arrive(o_free + t);
             if (valid && p.lse) p.lse[(size_t)it.h * p.N + tok] = (m_ref + __log2f(lsum)) * 0.69314718055994531f;
+            cnt += nch;
+            items_done++;
         }
     }
     tc_fence_before();
@@ -553,16 +590,22 @@ static int bf16_map2(EncodeTiledFn2 enc, CUtensorMap *m, const void *base, int r
                : -1;
 }
 
+static int kv_maps(EncodeTiledFn2 enc, KVMaps *m, const void *base, int rows, int cols) {
+    return (bf16_map2(enc, &m->m64, base, rows, cols, 64) || bf16_map2(enc, &m->m32, base, rows, cols, 32) ||
+            bf16_map2(enc, &m->m16, base, rows, cols, 16) || bf16_map2(enc, &m->m8, base, rows, cols, 8))
+               ? -1
+               : 0;
+}
+
 template <int D>
 static int launch2(const void *qg, const void *kg, const void *vg, const A2Params &p, int max_items, int num_sms,
                    void *encode_fn, cudaStream_t st) {
     using C = A2Cfg<D>;
     EncodeTiledFn2 enc = (EncodeTiledFn2)encode_fn;
-    CUtensorMap mq, mk, mv, mk128, mv128;
+    CUtensorMap mq;
+    KVMaps mk, mv;
     const int rows = p.H * p.N;
-    if (bf16_map2(enc, &mq, qg, rows, D, 128) || bf16_map2(enc, &mk, kg, rows, D, C::BOX) ||
-        bf16_map2(enc, &mv, vg, rows, D, C::BOX) || bf16_map2(enc, &mk128, kg, rows, D, 128) ||
-        bf16_map2(enc, &mv128, vg, rows, D, 128))
+    if (bf16_map2(enc, &mq, qg, rows, D, 128) || kv_maps(enc, &mk, kg, rows, D) || kv_maps(enc, &mv, vg, rows, D))
         return -1;
     static int checked = 0;  // 1 = ok, -1 = refused
     if (checked == 0) {
@@ -576,25 +619,23 @@ static int launch2(const void *qg, const void *kg, const void *vg, const A2Param
     if (checked != 1) return -1;
     int grid = max_items < num_sms ? max_items : num_sms;
     if (grid < 1) grid = 1;
-    attn2_kernel<D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, mk128, mv128, p);
+    attn2_kernel<D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);
     note_launch();
     return 0;
 }
 
 int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
-                 const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap, const int32_t *sel_cnt,
-                 const int2 *segtab, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
-                 float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st) {
+                 int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const AttnItem *items,
+                 const int32_t *n_items, int max_items, void *out, float *lse, int *status, int num_sms,
+                 void *encode_fn, cudaStream_t st) {
     A2Params p;
-    p.segtab = segtab;
     p.H = H;
     p.N = N;
     p.qperm = qperm;
-    p.koff = koff;
     p.kk_cap = kk_cap;
-    p.sel_idx = sel_idx;
-    p.sel_cnt = sel_cnt;
     p.kq_cap = kq_cap;
+    p.runs = runs;
+    p.run_info = run_info;
     p.items = items;
     p.n_items = n_items;
     p.out = reinterpret_cast<__nv_bfloat16 *>(out);

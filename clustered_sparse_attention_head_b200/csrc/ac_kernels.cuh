@@ -64,16 +64,62 @@ void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, cons
                    cudaStream_t st);
 size_t items_scratch_elems(int H, int kq_cap);
 int attn_max_items(int H, int N, int kq_cap);
-// bf16: two 128-row query tiles per CTA (ac_attn2.cu); items of up to 256 rows
+// Key runs of every (head, query cluster) (ac_attn.cu): the selected key
+// clusters in ascending order, neighbours merged into one range of rows of the
+// gathered K/V (empty clusters between them are absorbed).  runs [H, kq_cap,
+// kk_cap]; info [H, kq_cap] = {runs, chunks of `chunk_rows` rows as KeyStream
+// packs them}.  Cluster ids outside [0, kk_cap) are skipped.
+void k_key_runs(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx, const int32_t *sel_cnt,
+                int chunk_rows, int2 *runs, int2 *info, cudaStream_t st);
+// bf16: two 128-row query tiles per CTA, 64-key chunks (ac_attn2.cu); items of up to 256 rows
+constexpr int ATTN2_CHUNK = 64;
 int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
-                 const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap, const int32_t *sel_cnt,
-                 const int2 *segtab, const AttnItem *items, const int32_t *n_items, int max_items, void *out,
-                 float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st);
+                 int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const AttnItem *items,
+                 const int32_t *n_items, int max_items, void *out, float *lse, int *status, int num_sms,
+                 void *encode_fn, cudaStream_t st);
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
-                const int32_t *qperm, const int32_t *koff, int kk_cap, const int32_t *sel_idx, int kq_cap,
-                const int32_t *sel_cnt, const int2 *segtab, const AttnItem *items, const int32_t *n_items,
-                int max_items, void *out, float *lse, int *status, int num_sms, void *encode_fn, cudaStream_t st);
-void k_seg_table(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx,
-                 const int32_t *sel_cnt, int2 *segtab, cudaStream_t st);
+                const int32_t *qperm, int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info,
+                const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
+                int num_sms, void *encode_fn, cudaStream_t st);
+
+// The key rows of one work item as a stream of pieces: the rows of each run in
+// turn (all rows [0, dense_rows) of a dense head).  piece(room) hands out the
+// current run's next min(room, left) rows; their slot in the chunk is that
+// count rounded up to 8 rows.  A chunk takes pieces until its `cap` rows are
+// full or the stream ends, so every chunk but the last is exactly full; the
+// last is rounded up to 16 rows (the MMA's N and K granularity).  The
+// work-list builder and every role of the attention kernels step through the
+// same sequence.
+struct KeyStream {
+    const int2 *run;
+    int nrun, ri, cur, end;
+    int2 nxt;
+    __device__ __forceinline__ void init(const int2 *runs, int n, int dense_rows) {
+        run = runs;
+        nrun = runs ? n : 1;
+        ri = -1;
+        cur = end = 0;
+        nxt = runs ? (n > 0 ? runs[0] : make_int2(0, 0)) : make_int2(0, dense_rows);
+    }
+    __device__ __forceinline__ bool piece(int room, int &start, int &valid, int &slot) {
+        while (cur >= end) {
+            if (++ri >= nrun) return false;
+            cur = nxt.x;
+            end = nxt.y;
+            if (run && ri + 1 < nrun) nxt = run[ri + 1];  // one run ahead
+        }
+        start = cur;
+        valid = min(room, end - cur);
+        slot = (valid + 7) & ~7;
+        cur += valid;
+        return true;
+    }
+    // rows of the next chunk (0 at the end of the stream), rounded up to 16
+    __device__ __forceinline__ int chunk(int cap) {
+        int fill = 0, s, v, sl;
+        while (fill < cap && piece(cap - fill, s, v, sl)) fill += sl;
+        return (fill + 15) & ~15;
+    }
+};
 
 }  // namespace ac

@@ -170,6 +170,32 @@ def test_sparse_attention_from_oracle_selection(orc, name, top_p):
         attn_close(got[h], ref, f"{name}/p{top_p}/h{h}")
 
 
+@pytest.mark.parametrize("name", ["bf16-d64-ragged", "bf16-d128-ragged"])
+def test_sparse_attention_repeatable(orc, name):
+    """Five calls on the same inputs give bit-identical outputs and lse: every
+    reduction has a fixed order, so any difference would expose a race between
+    the kernel's TMA, MMA and softmax roles."""
+    w = _case(name)
+    q, k, v = stack_heads(w)
+    cl = _oracle_clusters(orc, w, q, k)
+    sels = [orc.select(rq.cent, qmn, rq.count, rk.cent, rk.count, 1.0) for rq, qmn, rk in cl]
+    ctx = _ctx(w, top_p=1.0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(np.stack(a))).cuda()
+    args = (to_dev(q, w.dtype), to_dev(k, w.dtype), to_dev(v, w.dtype), t([c[0].assign for c in cl]),
+            t([c[2].assign for c in cl]), t([s[0] for s in sels]), t([s[1] for s in sels]))
+    first = None
+    for _ in range(5):
+        out, lse = ctx.ac_sparse_attn(*args, lse=True)
+        torch.cuda.synchronize()
+        got = (out.view(torch.int16).cpu().numpy(), lse.cpu().numpy())
+        if first is None:
+            first = got
+        else:
+            np.testing.assert_array_equal(got[0], first[0])
+            np.testing.assert_array_equal(got[1], first[1])
+    assert ctx.get_status() == 0
+
+
 @pytest.mark.parametrize("name", ["f32-d64", "bf16-d128-ragged"])
 def test_dense_flag_gives_dense_attention(orc, name):
     w = _case(name)
