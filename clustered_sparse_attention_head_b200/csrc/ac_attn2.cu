@@ -17,6 +17,11 @@
 //  - once S_t(j) is complete, so is PV_t(j-2), the last reader of its buffer;
 //  - PV_t(j-1) may still run while the softmax works on chunk j, so before it
 //    rescales O_t the softmax waits for the P.V barrier phase of chunk j-1.
+// Every MMA covers a whole 64-key chunk, also for the short last chunk of an
+// item: the softmax masks the columns past its end (P = 0 there) and the V
+// ring is zeroed once at the start, so the stale K/V rows behind them are
+// finite.  A runtime guard per MMA instruction made the issue about 2.5x
+// slower on B200, and the MMA warp then needs no chunk sizes at all.
 // Every mbarrier wait is bounded; on expiry the CTA records ST_TIMEOUT,
 // drains its copies and MMAs, frees TMEM and returns.
 #include "ac_kernels.cuh"
@@ -38,7 +43,7 @@ template <int D> struct A2Cfg {
     // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle:
     // three full warpgroups, so registers can move between them (setmaxnreg)
     static constexpr int NTHREADS = 384;
-    static constexpr int REGS_LAUNCH = 168, REGS_LOW = 88, REGS_HIGH = 208;
+    static constexpr int REGS_LAUNCH = 168, REGS_LOW = 152, REGS_HIGH = 176;
     static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= NTHREADS * REGS_LAUNCH, "register split");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int TM_S = 0;                 // + 128 t + 64 buffer
@@ -91,17 +96,6 @@ __device__ __forceinline__ void drain(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = gtimer();
     while (!mbar_try_wait(bar, parity) && gtimer() - t0 < 200000000ull) {
     }
-}
-
-// O += P V with A (P, bf16) read from TMEM columns a_tmem.. (two per 32-bit column).
-__device__ __forceinline__ void umma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
 }
 
 template <int R> __device__ __forceinline__ void regs_dec() {
@@ -157,50 +151,51 @@ __device__ __forceinline__ void load_rows(unsigned char *stage, int r0, int grow
     }
 }
 
-// The next chunk of the stream into one stage: each piece into its slot, and,
-// when the chunk ends on an odd multiple of 8 rows, 8 more rows after the last
-// piece (finite data under masked columns, so that 0 * V stays 0).
+// The next chunk of the stream into one stage, each piece into its slot;
+// returns the rows loaded.
 template <int D>
-__device__ __forceinline__ void load_chunk(KeyStream &ks, unsigned char *stage, int row_base, const KVMaps &m,
-                                           uint64_t *bar, uint64_t pol) {
+__device__ __forceinline__ int load_chunk(KeyStream &ks, unsigned char *stage, int row_base, const KVMaps &m,
+                                          uint64_t *bar, uint64_t pol) {
     using C = A2Cfg<D>;
-    int fill = 0, start = 0, valid = 0, slot = 0, after = 0;
+    int fill = 0, start = 0, valid = 0, slot = 0;
     while (fill < C::BN && ks.piece(C::BN - fill, start, valid, slot)) {
         load_rows<D>(stage, fill, row_base + start, slot, m, bar, pol);
         fill += slot;
-        after = start + slot;
     }
-    if (fill & 8) load_rows<D>(stage, fill, row_base + after, 8, m, bar, pol);
+    return fill;
+}
+// Rows of the next chunk (the same pieces as load_chunk)
+__device__ __forceinline__ int chunk_rows(KeyStream &ks, int cap) {
+    int fill = 0, s, v, sl;
+    while (fill < cap && ks.piece(cap - fill, s, v, sl)) fill += sl;
+    return fill;
 }
 
-// S_t = Q_t K^T into TMEM columns d (ncol keys of one K stage)
+// S_t = Q_t K^T into TMEM columns d (the 64 keys of one K stage); whole warp
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t d, uint64_t qdesc_t, uint64_t kdesc_stage, int ncol) {
+__device__ __forceinline__ void issue_s(uint32_t d, uint64_t qdesc_t, uint64_t kdesc_stage) {
     using C = A2Cfg<D>;
-    // ncol >= 16 whenever the stream and the chunk count agree (they are built
-    // from the same runs); the clamp only keeps the instruction shape legal
-    const uint32_t idesc = idesc_make(128, ncol < 16 ? 16 : ncol, 1, false);
+    constexpr uint32_t idesc = idesc_make(128, C::BN, 1, false);
     uint64_t a = qdesc_t, b = kdesc_stage;
 #pragma unroll
     for (int kb = 0; kb < C::DB; kb++) {
 #pragma unroll
-        for (int k4 = 0; k4 < 4; k4++) umma_f16(d, a + 2 * k4, b + 2 * k4, idesc, (kb | k4) ? 1u : 0u);
+        for (int k4 = 0; k4 < 4; k4++) umma_f16_w(d, a + 2 * k4, b + 2 * k4, idesc, (kb | k4) ? 1u : 0u);
         a += (C::BM * 128) >> 4;
         b += (C::BN * 128) >> 4;
     }
 }
 
-// O_t (+)= P_t V for the first ncol keys of one V stage; P_t is bf16 in TMEM at a0
+// O_t (+)= P_t V over the 64 keys of one V stage; P_t is bf16 in TMEM at a0
+// (two keys per 32-bit column); whole warp
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t a0, uint64_t vdesc_stage, int ncol, bool first) {
+__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t a0, uint64_t vdesc_stage, bool first) {
     using C = A2Cfg<D>;
-    const uint32_t idesc = idesc_make(128, D, 1, true);
-    const int nk = ncol / C::KSTEP;
+    constexpr uint32_t idesc = idesc_make(128, D, 1, true);
 #pragma unroll
     for (int ks = 0; ks < C::BN / C::KSTEP; ks++)
-        if (ks < nk)
-            umma_ts_f16(d, a0 + ks * 8, vdesc_stage + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc,
-                        (!first || ks > 0) ? 1u : 0u);
+        umma_ts_f16_w(d, a0 + ks * 8, vdesc_stage + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc,
+                      (!first || ks > 0) ? 1u : 0u);
 }
 
 }  // namespace
@@ -227,6 +222,11 @@ __global__ void __launch_bounds__(384, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(drain_bar + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // zero the V ring once: rows of a stage past its chunk's end are read by
+    // P.V (with P = 0) and must hold finite values
+    for (int i = threadIdx.x; i < C::VST * C::KV_BYTES / 16; i += C::NTHREADS)
+        reinterpret_cast<uint4 *>(sm + C::OFF_V)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int row_base = it.h * p.N;
                 for (int j = 0; j < nch; j++, g++) {
                     KeyStream kk = ks, probe = ks;
-                    const uint32_t bytes = (uint32_t)probe.chunk(C::BN) * 128u * C::DB;
+                    const uint32_t bytes = (uint32_t)chunk_rows(probe, C::BN) * 128u * C::DB;
                     const int kslot = g % C::KST, vslot = g % C::VST;
                     const uint32_t ku = g / C::KST, vu = g / C::VST;
                     if (ku >= 1 && !mbar_wait(k_empty + kslot, (ku - 1) & 1, abort_flag, p.status)) { ok = false; break; }
@@ -325,7 +325,9 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp == 9) {
         // --------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop with identical values in every lane;
+        // each tcgen05 instruction is issued by one elected lane.
+        {
             uint32_t g = 0, qi = 0;
             uint32_t cnt[2] = {0, 0};  // chunks each tile has been through
             uint32_t act[2] = {0, 0};  // items each tile was active in
@@ -341,35 +343,31 @@ __global__ void __launch_bounds__(384, 1)
                 const int nch = item_chunks(p, it);
                 if (nch == 0) continue;
                 const int nt = it.q_len > 128 ? 2 : 1;
-                if (!mbar_wait(q_full, qi & 1, abort_flag, p.status)) { ok = false; break; }
+                if (!wait_warp(q_full, qi & 1, abort_flag, p.status)) { ok = false; break; }
                 qi++;
-                KeyStream ks;
-                stream_init(ks, p, it);
                 // prologue: S_t(0) and S_t(1)
-                int n0 = ks.chunk(C::BN), n1 = nch > 1 ? ks.chunk(C::BN) : 0, n2 = 0;
                 for (int jj = 0; jj < 2 && jj < nch && ok; jj++) {
                     const uint32_t gk = g + jj;
                     const int kslot = gk % C::KST;
-                    if (!mbar_wait(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_warp(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int t = 0; t < 2; t++) {
                         if (t >= nt) break;
                         const int b = (cnt[t] + jj) & 1;
                         issue_s<D>(tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
-                                   kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4), jj == 0 ? n0 : n1);
-                        umma_commit(s_full + 2 * t + b);
+                                   kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4));
+                        umma_commit_w(s_full + 2 * t + b);
                     }
-                    umma_commit(k_empty + kslot);
+                    umma_commit_w(k_empty + kslot);
                 }
                 if (!ok) break;
-                if (nch <= 2) umma_commit(q_empty);
+                if (nch <= 2) umma_commit_w(q_empty);
                 for (int j = 0; j < nch && ok; j++) {
                     const uint32_t gv = g + j;
                     const int vslot = gv % C::VST;
-                    if (!mbar_wait(v_full + vslot, (gv / C::VST) & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (!wait_warp(v_full + vslot, (gv / C::VST) & 1, abort_flag, p.status)) { ok = false; break; }
                     const bool more = j + 2 < nch;
-                    if (more) n2 = ks.chunk(C::BN);
                     const uint32_t gk = g + j + 2;
                     const int kslot = gk % C::KST;
 #pragma unroll
@@ -378,37 +376,38 @@ __global__ void __launch_bounds__(384, 1)
                         const uint32_t c = cnt[t] + j;
                         const int b = c & 1;
                         // PV_t(j) once softmax t has written P_t(j)
-                        if (!mbar_wait(p_full + 2 * t + b, (c >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                        if (j == 0 && act[t] >= 1 && !mbar_wait(o_free + t, (act[t] - 1) & 1, abort_flag, p.status)) {
+                        if (!wait_warp(p_full + 2 * t + b, (c >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                        if (j == 0 && act[t] >= 1 && !wait_warp(o_free + t, (act[t] - 1) & 1, abort_flag, p.status)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         issue_pv<D>(tmem + C::TM_O + t * D, tmem + C::TM_S + t * 128 + b * 64,
-                                    vdesc0 + (uint64_t)((vslot * C::KV_BYTES) >> 4), n0, j == 0);
-                        umma_commit(pv_bar + t);
-                        if (j + 1 == nch) umma_commit(o_done + t);
+                                    vdesc0 + (uint64_t)((vslot * C::KV_BYTES) >> 4), j == 0);
+                        umma_commit_w(pv_bar + t);
                         // S_t(j+2) into the buffer P_t(j) occupied
                         if (more) {
-                            if (t == 0 && !mbar_wait(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) {
+                            if (t == 0 && !wait_warp(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after();
                             issue_s<D>(tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
-                                       kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4), n2);
-                            umma_commit(s_full + 2 * t + b);
+                                       kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4));
+                            umma_commit_w(s_full + 2 * t + b);
                         }
                     }
                     if (!ok) break;
-                    umma_commit(v_empty + vslot);
+                    umma_commit_w(v_empty + vslot);
                     if (more) {
-                        umma_commit(k_empty + kslot);
-                        if (j + 3 == nch) umma_commit(q_empty);
+                        umma_commit_w(k_empty + kslot);
+                        if (j + 3 == nch) umma_commit_w(q_empty);
                     }
-                    n0 = n1;
-                    n1 = n2;
                 }
+                if (!ok) break;
+                // the item's last P.V of each tile is done once these arrive
+                umma_commit_w(o_done + 0);
+                if (nt > 1) umma_commit_w(o_done + 1);
                 g += nch;
                 cnt[0] += nch;
                 act[0]++;
@@ -418,7 +417,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             if (!ok) {
-                umma_commit(drain_bar);
+                umma_commit_w(drain_bar);
                 drain(drain_bar, 0);
             }
         }

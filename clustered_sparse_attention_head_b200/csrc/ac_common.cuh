@@ -168,6 +168,41 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                  : "memory");
 }
 
+// Warp-wide forms: called by all 32 lanes of a converged warp with identical
+// arguments; elect.sync picks the one lane that issues.  Issuing from a
+// converged warp is cheaper than from a lone lane inside a divergent branch
+// (measured on B200: ~48 vs ~58 cycles per M=128, N=64 MMA, and a commit costs
+// almost nothing instead of ~28 cycles), and the MMA pipe needs ~48-64 cycles
+// per instruction, so the lone-lane form is issue-bound for N <= 64.
+__device__ __forceinline__ void umma_f16_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// A operand from TMEM (a_tmem), B from shared memory.
+__device__ __forceinline__ void umma_ts_f16_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_w(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: lane i of the warp reads TMEM lane
 // (taddr.lane + i), columns taddr.col .. +31.  The wait for completion is in
 // the same asm statement, so no use of r can be scheduled before it.

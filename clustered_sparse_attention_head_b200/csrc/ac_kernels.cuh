@@ -86,10 +86,9 @@ int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, 
 // turn (all rows [0, dense_rows) of a dense head).  piece(room) hands out the
 // current run's next min(room, left) rows; their slot in the chunk is that
 // count rounded up to 8 rows.  A chunk takes pieces until its `cap` rows are
-// full or the stream ends, so every chunk but the last is exactly full; the
-// last is rounded up to 16 rows (the MMA's N and K granularity).  The
-// work-list builder and every role of the attention kernels step through the
-// same sequence.
+// full or the stream ends, so every chunk but the last is exactly full.  The
+// work-list builder and the roles of the attention kernel that need the
+// pieces step through the same sequence.
 struct KeyStream {
     const int2 *run;
     int nrun, ri, cur, end;
@@ -113,12 +112,6 @@ struct KeyStream {
         slot = (valid + 7) & ~7;
         cur += valid;
         return true;
-    }
-    // rows of the next chunk (0 at the end of the stream), rounded up to 16
-    __device__ __forceinline__ int chunk(int cap) {
-        int fill = 0, s, v, sl;
-        while (fill < cap && piece(cap - fill, s, v, sl)) fill += sl;
-        return (fill + 15) & ~15;
     }
 };
 
