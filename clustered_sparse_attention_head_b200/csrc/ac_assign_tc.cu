@@ -15,9 +15,12 @@
 // two scores are within 2E goes to the exact double pass (assign_exact_kernel),
 // so the final decision equals the exact one.
 //
-// Warp 0 issues TMA (X tile once, then C_hi/C_lo chunks), lane 0 of warp 1
-// issues the MMAs into two TMEM accumulators (double buffer), warps 2-5 run
-// the epilogue.  All waits are bounded.
+// Warp 0 issues TMA (X tile once, then C_hi/C_lo chunks), warp 1 issues the
+// MMAs into two TMEM accumulators (double buffer; whole warp, one elected
+// lane), warps 2-5 run the epilogue.  The epilogue keeps four independent
+// running top-3 lists per row (columns interleaved four ways, branch-free
+// updates) and merges them at the end: one serial list per row made the
+// kernel latency-bound.  All waits are bounded.
 #include "ac_kernels.cuh"
 
 namespace ac {
@@ -31,7 +34,9 @@ template <int D> struct TcCfg {
     static constexpr int OFF_X = 0;
     static constexpr int OFF_C = X_BYTES;                      // stage s: hi at +2s*C, lo at +(2s+1)*C
     static constexpr int OFF_BAR = OFF_C + STAGES * 2 * C_BYTES;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static constexpr int OFF_CN = OFF_BAR + 256;  // ||c||^2 of the head, kpad floats
+    // dynamic shared memory for a given kpad (plus 1 KB of alignment slack)
+    static constexpr int smem_bytes(int kpad) { return OFF_CN + kpad * 4 + 1024; }
     static constexpr uint32_t TMEM_COLS = 256;
 };
 
@@ -124,76 +129,123 @@ __global__ void __launch_bounds__(192, 2)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            bool ok = mbar_wait(x_full, 0, abort_flag, p.status);
-            const uint32_t idesc = idesc_make(128, C::COLS, 1, false);
-            const uint32_t xb = smem_u32(sm + C::OFF_X);
-            for (int j = 0; j < nch && ok; j++) {
-                const int st = j % C::STAGES;
-                const int b = j & 1;
-                if (!mbar_wait(c_full + st, (j / C::STAGES) & 1, abort_flag, p.status)) { ok = false; break; }
-                if (j >= 2 && !mbar_wait(d_empty + b, ((j >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t hb = smem_u32(sm + C::OFF_C + (2 * st) * C::C_BYTES);
-                const uint32_t lb = smem_u32(sm + C::OFF_C + (2 * st + 1) * C::C_BYTES);
-                const uint32_t dcol = tmem + b * C::COLS;
-                for (int ks = 0; ks < D / 16; ks++) {
-                    const uint32_t off = (ks / 4) * 0 + (ks % 4) * 32;
-                    const uint64_t a = sdesc_sw128(xb + (ks / 4) * (C::ROWS * 128) + off, 16, 1024);
-                    umma_f16(dcol, a, sdesc_sw128(hb + (ks / 4) * (C::COLS * 128) + off, 16, 1024), idesc,
-                             ks > 0 ? 1u : 0u);
-                }
-                for (int ks = 0; ks < D / 16; ks++) {
-                    const uint32_t off = (ks % 4) * 32;
-                    const uint64_t a = sdesc_sw128(xb + (ks / 4) * (C::ROWS * 128) + off, 16, 1024);
-                    umma_f16(dcol, a, sdesc_sw128(lb + (ks / 4) * (C::COLS * 128) + off, 16, 1024), idesc, 1u);
-                }
-                umma_commit(c_empty + st);
-                umma_commit(d_full + b);
+        // whole warp, identical values in every lane; one elected lane issues
+        bool ok = mbar_wait_warp(x_full, 0, abort_flag, p.status);
+        constexpr uint32_t idesc = idesc_make(128, C::COLS, 1, false);
+        const uint64_t xdesc = sdesc_sw128(smem_u32(sm + C::OFF_X), 16, 1024);
+        const uint64_t cdesc = sdesc_sw128(smem_u32(sm + C::OFF_C), 16, 1024);
+        for (int j = 0; j < nch && ok; j++) {
+            const int st = j % C::STAGES;
+            const int b = j & 1;
+            if (!mbar_wait_warp(c_full + st, (j / C::STAGES) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (j >= 2 && !mbar_wait_warp(d_empty + b, ((j >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t dcol = tmem + b * C::COLS;
+            // 16-byte units: hi part of stage st at 2st*C_BYTES, lo part at (2st+1)*C_BYTES
+            const uint64_t hdesc = cdesc + (uint64_t)(((2 * st) * C::C_BYTES) >> 4);
+            const uint64_t ldesc = cdesc + (uint64_t)(((2 * st + 1) * C::C_BYTES) >> 4);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ks++) {
+                const uint64_t a = xdesc + (uint64_t)(((ks / 4) * (C::ROWS * 128) + (ks % 4) * 32) >> 4);
+                const uint64_t bo = (uint64_t)(((ks / 4) * (C::COLS * 128) + (ks % 4) * 32) >> 4);
+                umma_f16_w(dcol, a, hdesc + bo, idesc, ks > 0 ? 1u : 0u);
             }
-            if (!ok) {
-                umma_commit(drain);
-                uint64_t t0 = gtimer();
-                while (!mbar_try_wait(drain, 0) && gtimer() - t0 < 200000000ull) {
-                }
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ks++) {
+                const uint64_t a = xdesc + (uint64_t)(((ks / 4) * (C::ROWS * 128) + (ks % 4) * 32) >> 4);
+                const uint64_t bo = (uint64_t)(((ks / 4) * (C::COLS * 128) + (ks % 4) * 32) >> 4);
+                umma_f16_w(dcol, a, ldesc + bo, idesc, 1u);
+            }
+            umma_commit_w(c_empty + st);
+            umma_commit_w(d_full + b);
+        }
+        if (!ok) {
+            umma_commit_w(drain);
+            uint64_t t0 = gtimer();
+            while (!mbar_try_wait(drain, 0) && gtimer() - t0 < 200000000ull) {
             }
         }
     } else {
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const float *cn = p.cn2 + (size_t)h * p.cap;
-        float b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
-        int i1 = 0, i2 = -1;
+        // ||c||^2 of this head's centroids (zero-padded to whole chunks) in
+        // shared memory; the four epilogue warps share a named barrier
+        float *cn_s = reinterpret_cast<float *>(sm + C::OFF_CN);
+        const int kpadc = nch * C::COLS;
+        for (int i = threadIdx.x - 64; i < kpadc; i += 128)
+            cn_s[i] = (p.mode == MODE_EUCLID && i < s.k) ? p.cn2[(size_t)h * p.cap + i] : 0.f;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // four running lists (columns col = 4m + q go to list q): best score and
+        // index, second best and index, third best score
+        float b1[4], b2[4], b3[4];
+        int i1[4], i2[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            b1[q] = b2[q] = b3[q] = INFINITY;
+            i1[q] = 0;
+            i2[q] = -1;
+        }
+        const float wv = (p.mode == MODE_EUCLID) ? -2.f : -1.f;
         bool ok = true;
         for (int j = 0; j < nch; j++) {
             const int b = j & 1;
-            bool w = mbar_wait(d_full + b, (j >> 1) & 1, abort_flag, p.status);
-            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+            if (!mbar_wait_warp(d_full + b, (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
+#pragma unroll
             for (int pc = 0; pc < C::COLS / 32; pc++) {
                 uint32_t r[32];
                 tmem_ld32(tmem + lane_addr + b * C::COLS + pc * 32, r);
                 const int c0 = j * C::COLS + pc * 32;
+                const float4 *cn4 = reinterpret_cast<const float4 *>(cn_s + c0);
 #pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const int col = c0 + i;
-                    if (col < s.k) {
-                        const float v = __uint_as_float(r[i]);
-                        const float sc = (p.mode == MODE_EUCLID) ? fmaf(-2.f, v, cn[col]) : -v;
-                        if (sc < b2) {
-                            b3 = b2;
-                            if (sc < b1) { b2 = b1; i2 = i1; b1 = sc; i1 = col; }
-                            else { b2 = sc; i2 = col; }
-                        } else {
-                            b3 = fminf(b3, sc);
-                        }
+                for (int i4 = 0; i4 < 8; i4++) {
+                    const float4 cv = cn4[i4];
+                    const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        const int col = c0 + 4 * i4 + q;
+                        // EUCLID: ||c||^2 - 2 x.c; SPHERE: -(x.mu); padding columns never win
+                        const float sc = col < s.k ? fmaf(wv, __uint_as_float(r[4 * i4 + q]), cc[q]) : INFINITY;
+                        const bool lt1 = sc < b1[q], lt2 = sc < b2[q];
+                        b3[q] = fminf(b3[q], fmaxf(sc, b2[q]));
+                        b2[q] = fminf(b2[q], fmaxf(sc, b1[q]));
+                        i2[q] = lt1 ? i1[q] : (lt2 ? col : i2[q]);
+                        i1[q] = lt1 ? col : i1[q];
+                        b1[q] = fminf(b1[q], sc);
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(d_empty + b);
         }
+        // merge lists 1-3 into list 0 (ties: the lower column index wins)
+        float B1 = b1[0], B2 = b2[0], B3 = b3[0];
+        int I1 = i1[0], I2 = i2[0];
+#pragma unroll
+        for (int q = 1; q < 4; q++) {
+            const float cs[3] = {b1[q], b2[q], b3[q]};
+            const int ci[3] = {i1[q], i2[q], 0x7fffffff};
+#pragma unroll
+            for (int e = 0; e < 3; e++) {
+                const float sc = cs[e];
+                const int col = ci[e];
+                const bool lt1 = sc < B1 || (sc == B1 && col < I1);
+                const bool lt2 = sc < B2 || (sc == B2 && col < I2);
+                B3 = fminf(B3, lt2 ? B2 : sc);
+                if (lt1) {
+                    B2 = B1;
+                    I2 = I1;
+                    B1 = sc;
+                    I1 = col;
+                } else if (lt2) {
+                    B2 = sc;
+                    I2 = col;
+                }
+            }
+        }
+        const float b1v = B1, b2v = B2, b3v = B3;
+        const int i1v = I1, i2v = I2;
         const int pos = r0 + row;
         if (ok && pos < s.nrows) {
             const int tok = p.rows ? p.rows[(size_t)h * p.N + pos] : pos;
@@ -201,14 +253,14 @@ __global__ void __launch_bounds__(192, 2)
             const float cm = p.cmax[h];
             const float edot = 1.220703125e-4f * xn * cm;  // 2^-13 ||x|| Cmax
             const float E = (p.mode == MODE_EUCLID) ? 2.f * edot + 2.384185791e-7f * (cm * cm + 2.f * xn * cm) : edot;
-            if (s.k > 1 && !(b2 - b1 > 2.f * E)) {
+            if (s.k > 1 && !(b2v - b1v > 2.f * E)) {
                 // Every centroid other than i1 and i2 scores >= b3; if b3 > b1 + 2E
                 // none of them can be the exact winner, so only the two are re-scored.
                 const int slot = atomicAdd(&p.amb_count[h], 1);
                 p.amb_list[(size_t)h * p.N + slot] = pos;
-                p.amb_cand[(size_t)h * p.N + slot] = (b3 - b1 > 2.f * E) ? make_int2(i1, i2) : make_int2(-1, -1);
+                p.amb_cand[(size_t)h * p.N + slot] = (b3v - b1v > 2.f * E) ? make_int2(i1v, i2v) : make_int2(-1, -1);
             } else {
-                p.assign[(size_t)h * p.N + pos] = i1;
+                p.assign[(size_t)h * p.N + pos] = i1v;
             }
         }
     }
@@ -297,9 +349,10 @@ static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const He
     if (bf16_map(enc, &mx, xc, H * N, D, C::ROWS) || bf16_map(enc, &mh, chi, H * kpad, D, C::COLS) ||
         bf16_map(enc, &ml, clo, H * kpad, D, C::COLS))
         return -1;
+    if (kpad > 8192) return -1;
     static bool attr = false;
     if (!attr) {
-        cudaFuncSetAttribute(assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaFuncSetAttribute(assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem_bytes(8192));
         attr = true;
     }
     TcParams p;
@@ -318,7 +371,7 @@ static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const He
     p.amb_cand = amb_cand;
     p.status = status;
     dim3 g((nrows_max + C::ROWS - 1) / C::ROWS, H);
-    assign_tc_kernel<D><<<g, 192, C::SMEM, st>>>(mx, mh, ml, p);
+    assign_tc_kernel<D><<<g, 192, C::smem_bytes(kpad), st>>>(mx, mh, ml, p);
     note_launch();
     return 0;
 }

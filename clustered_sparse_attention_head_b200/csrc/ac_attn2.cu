@@ -88,8 +88,7 @@ __device__ __forceinline__ void stream_init(KeyStream &ks, const A2Params &p, co
 }
 
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
-    const bool ok = mbar_wait(bar, parity, abort_flag, status);
-    return __all_sync(0xffffffffu, ok);
+    return mbar_wait_warp(bar, parity, abort_flag, status);
 }
 
 __device__ __forceinline__ void drain(uint64_t *bar, uint32_t parity) {
@@ -485,10 +484,17 @@ __global__ void __launch_bounds__(384, 1)
                         }
                     }
                 }
-                float mx = __uint_as_float(s[0]);
+                // row max: four independent chains of 3-input max (short dependences)
+                float mq[4];
 #pragma unroll
-                for (int i = 1; i + 1 < 64; i += 2) mx = max3(mx, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-                mx = fmaxf(mx, __uint_as_float(s[63]));
+                for (int q = 0; q < 4; q++) {
+                    float m = fmaxf(__uint_as_float(s[16 * q]), __uint_as_float(s[16 * q + 1]));
+#pragma unroll
+                    for (int i = 2; i < 16; i += 2)
+                        m = max3(m, __uint_as_float(s[16 * q + i]), __uint_as_float(s[16 * q + i + 1]));
+                    mq[q] = m;
+                }
+                const float mx = fmaxf(max3(mq[0], mq[1], mq[2]), mq[3]);
                 const float m_new = mx * sc;
                 if (j == 0) m_ref = m_new;
                 // Move the reference max (and rescale O_t) only when it grew by
@@ -516,17 +522,21 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 const float nm = -m_ref;
                 uint32_t pk[32];
+                // row sum in four partial sums (short dependences), folded into l0/l1
+                float la[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < 32; i++) {
                     float x0, x1;
                     fma2(x0, x1, __uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]), sc, nm);
                     const float e0 = ex2_approx(x0);
                     const float e1 = (i & 1) ? ex2_fma(x1) : ex2_approx(x1);
-                    l0 += e0;
-                    l1 += e1;
+                    la[2 * (i & 1)] += e0;
+                    la[2 * (i & 1) + 1] += e1;
                     __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
                     pk[i] = *reinterpret_cast<uint32_t *>(&b2);
                 }
+                l0 += la[0] + la[2];
+                l1 += la[1] + la[3];
                 tmem_st32(s_base + b * 64, pk);
                 tmem_st_wait();
                 tc_fence_before();
