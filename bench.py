@@ -54,6 +54,23 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks call this in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def calls_per_second(ms_max: float, world: int) -> float:
+    """Whole-job throughput: every rank completes one call per step, and the
+    job's step takes as long as its slowest rank."""
+    return world * 1000.0 / ms_max
+
+
 def gen_inputs(w, heads=None):
     """Seeded inputs, all heads (threads: numpy releases the GIL in bulk draws)."""
     from concurrent.futures import ThreadPoolExecutor
@@ -246,13 +263,8 @@ def main():
     status = ac.get_status()
     if status != 0:
         raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
-    t_max = ms
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-    calls_per_s = world * 1000.0 / t_max
+    t_max = max_over_ranks(ms, world, dev)
+    calls_per_s = calls_per_second(t_max, world)
     flops = 4.0 * w.d * st["pairs"]
     tflops_call = flops / (ms * 1e-3) / 1e12
     attn_ms = prof["ms_attn_kernel"]
@@ -277,14 +289,9 @@ def main():
             op.copy_(out, non_blocking=True)
         s1.record(stream)
         barrier()
-        ms_e2e = s0.elapsed_time(s1) / n_e2e
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world, dev)
         nb = q.numel() * q.element_size()
-        e2e = {"value": world * 1000.0 / ms_e2e, "unit": "calls/s", "h2d_bytes_per_step": 3 * nb,
+        e2e = {"value": calls_per_second(ms_e2e, world), "unit": "calls/s", "h2d_bytes_per_step": 3 * nb,
                "d2h_bytes_per_step": nb, "ms_per_step": ms_e2e}
         ac.profile_read()
 
