@@ -172,14 +172,14 @@ __device__ __forceinline__ int chunk_rows(KeyStream &ks, int cap) {
 
 // S_t = Q_t K^T into TMEM columns d (the 64 keys of one K stage); whole warp
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t d, uint64_t qdesc_t, uint64_t kdesc_stage) {
+__device__ __forceinline__ void issue_s(uint32_t ld, uint32_t d, uint64_t qdesc_t, uint64_t kdesc_stage) {
     using C = A2Cfg<D>;
     constexpr uint32_t idesc = idesc_make(128, C::BN, 1, false);
     uint64_t a = qdesc_t, b = kdesc_stage;
 #pragma unroll
     for (int kb = 0; kb < C::DB; kb++) {
 #pragma unroll
-        for (int k4 = 0; k4 < 4; k4++) umma_f16_w(d, a + 2 * k4, b + 2 * k4, idesc, (kb | k4) ? 1u : 0u);
+        for (int k4 = 0; k4 < 4; k4++) umma_f16_p(ld, d, a + 2 * k4, b + 2 * k4, idesc, (kb | k4) ? 1u : 0u);
         a += (C::BM * 128) >> 4;
         b += (C::BN * 128) >> 4;
     }
@@ -188,12 +188,12 @@ __device__ __forceinline__ void issue_s(uint32_t d, uint64_t qdesc_t, uint64_t k
 // O_t (+)= P_t V over the 64 keys of one V stage; P_t is bf16 in TMEM at a0
 // (two keys per 32-bit column); whole warp
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t a0, uint64_t vdesc_stage, bool first) {
+__device__ __forceinline__ void issue_pv(uint32_t ld, uint32_t d, uint32_t a0, uint64_t vdesc_stage, bool first) {
     using C = A2Cfg<D>;
     constexpr uint32_t idesc = idesc_make(128, D, 1, true);
 #pragma unroll
     for (int ks = 0; ks < C::BN / C::KSTEP; ks++)
-        umma_ts_f16_w(d, a0 + ks * 8, vdesc_stage + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc,
+        umma_ts_f16_p(ld, d, a0 + ks * 8, vdesc_stage + (uint64_t)((ks * C::KSTEP * 128) >> 4), idesc,
                       (!first || ks > 0) ? 1u : 0u);
 }
 
@@ -327,6 +327,8 @@ __global__ void __launch_bounds__(384, 1)
         // The whole warp runs this loop with identical values in every lane;
         // each tcgen05 instruction is issued by one elected lane.
         {
+            // the lane that issues every tcgen05 instruction, chosen once
+            const uint32_t leader = elect_leader();
             uint32_t g = 0, qi = 0;
             uint32_t cnt[2] = {0, 0};  // chunks each tile has been through
             uint32_t act[2] = {0, 0};  // items each tile was active in
@@ -354,14 +356,14 @@ __global__ void __launch_bounds__(384, 1)
                     for (int t = 0; t < 2; t++) {
                         if (t >= nt) break;
                         const int b = (cnt[t] + jj) & 1;
-                        issue_s<D>(tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
+                        issue_s<D>(leader, tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
                                    kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4));
-                        umma_commit_w(s_full + 2 * t + b);
+                        umma_commit_p(leader, s_full + 2 * t + b);
                     }
-                    umma_commit_w(k_empty + kslot);
+                    umma_commit_p(leader, k_empty + kslot);
                 }
                 if (!ok) break;
-                if (nch <= 2) umma_commit_w(q_empty);
+                if (nch <= 2) umma_commit_p(leader, q_empty);
                 for (int j = 0; j < nch && ok; j++) {
                     const uint32_t gv = g + j;
                     const int vslot = gv % C::VST;
@@ -381,9 +383,9 @@ __global__ void __launch_bounds__(384, 1)
                             break;
                         }
                         tc_fence_after();
-                        issue_pv<D>(tmem + C::TM_O + t * D, tmem + C::TM_S + t * 128 + b * 64,
+                        issue_pv<D>(leader, tmem + C::TM_O + t * D, tmem + C::TM_S + t * 128 + b * 64,
                                     vdesc0 + (uint64_t)((vslot * C::KV_BYTES) >> 4), j == 0);
-                        umma_commit_w(pv_bar + t);
+                        umma_commit_p(leader, pv_bar + t);
                         // S_t(j+2) into the buffer P_t(j) occupied
                         if (more) {
                             if (t == 0 && !wait_warp(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) {
@@ -391,22 +393,22 @@ __global__ void __launch_bounds__(384, 1)
                                 break;
                             }
                             tc_fence_after();
-                            issue_s<D>(tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
+                            issue_s<D>(leader, tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
                                        kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4));
-                            umma_commit_w(s_full + 2 * t + b);
+                            umma_commit_p(leader, s_full + 2 * t + b);
                         }
                     }
                     if (!ok) break;
-                    umma_commit_w(v_empty + vslot);
+                    umma_commit_p(leader, v_empty + vslot);
                     if (more) {
-                        umma_commit_w(k_empty + kslot);
-                        if (j + 3 == nch) umma_commit_w(q_empty);
+                        umma_commit_p(leader, k_empty + kslot);
+                        if (j + 3 == nch) umma_commit_p(leader, q_empty);
                     }
                 }
                 if (!ok) break;
                 // the item's last P.V of each tile is done once these arrive
-                umma_commit_w(o_done + 0);
-                if (nt > 1) umma_commit_w(o_done + 1);
+                umma_commit_p(leader, o_done + 0);
+                if (nt > 1) umma_commit_p(leader, o_done + 1);
                 g += nch;
                 cnt[0] += nch;
                 act[0]++;
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             if (!ok) {
-                umma_commit_w(drain_bar);
+                umma_commit_p(leader, drain_bar);
                 drain(drain_bar, 0);
             }
         }
