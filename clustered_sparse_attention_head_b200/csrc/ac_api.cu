@@ -61,7 +61,7 @@ struct Ws {
     // attention
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
-    size_t chi, clo, xu, amb_cand, items_scr, runs, run_info;
+    size_t chi, clo, xu, amb_cand, items_scr, runs, run_info, masks;
     int kpad;
     size_t total;
 };
@@ -123,6 +123,7 @@ Ws layout(const ac_ctx *c) {
     w.items_scr = b.take(items_scratch_elems((int)H, c->kq_cap) * 4 + 16);
     w.runs = b.take(H * (size_t)c->kq_cap * c->kk_cap * 8);
     w.run_info = b.take(H * (size_t)c->kq_cap * 8);
+    w.masks = b.take(H * (size_t)c->kq_cap * attn_max_chunks(c->cfg.n, c->kk_cap) * 4);
     w.total = b.off;
     return w;
 }
@@ -297,10 +298,14 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
                   nitems, pairs_dev, at<int32_t>(ws, w.items_scr), st);
     int2 *runs = at<int2>(ws, w.runs), *run_info = at<int2>(ws, w.run_info);
     k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN2_CHUNK, runs, run_info, st);
+    const int max_chunks = attn_max_chunks(N, c->kk_cap);
+    uint32_t *masks = at<uint32_t>(ws, w.masks);
+    if (two_tiles) k_chunk_masks(H, c->kq_cap, c->kk_cap, max_chunks, runs, run_info, masks, st);
     if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
     int rc;
     if (two_tiles)
-        rc = k_attention2(D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, items, nitems,
+        rc = k_attention2(D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, masks, max_chunks, items,
+                          nitems,
                           attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
     else
         rc = k_attention(DT_F32, D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, items, nitems,

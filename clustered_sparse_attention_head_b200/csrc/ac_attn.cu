@@ -699,6 +699,87 @@ void k_key_runs(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_
     note_launch();
 }
 
+// Chunk masks of every (head, query cluster): for chunk c of the key stream
+// (chunk_rows keys as KeyStream packs the runs) the number of valid rows in
+// each of its 8-row groups, 4 bits per group (chunk_rows = 64: 8 groups).  Run
+// r occupies stream positions [S_r, S_r + round8(len_r)) with S_r the prefix
+// sum of the rounded lengths, and its first len_r positions hold keys (a run
+// split at a chunk boundary is split at a multiple of 8, so this holds for
+// every piece).  One CTA per (query cluster, head): a block scan gives S, then
+// each thread fills chunks with a binary search per group.
+constexpr int kMaskMaxRuns = 8192;
+
+__global__ void chunk_masks_kernel(int kq_cap, int kk_cap, int max_chunks, const int2 *__restrict__ runs,
+                                   const int2 *__restrict__ info, uint32_t *__restrict__ masks) {
+    __shared__ int s_start[kMaskMaxRuns];
+    __shared__ int wsum[32];
+    const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const size_t qa = (size_t)h * kq_cap + a;
+    const int2 inf = info[qa];
+    const int nr = min(inf.x, kMaskMaxRuns), nch = min(inf.y, max_chunks);
+    if (nch <= 0) return;
+    const int2 *rr = runs + qa * kk_cap;
+    // exclusive scan of the rounded run lengths (runs processed in blocks of nt)
+    int carry = 0;
+    for (int b0 = 0; b0 < nr; b0 += nt) {
+        const int r = b0 + tid;
+        int len = 0;
+        if (r < nr) {
+            const int2 v = rr[r];
+            len = (v.y - v.x + 7) & ~7;
+        }
+        int x = len;
+        const int lane = tid & 31, w = tid >> 5;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
+        __syncthreads();
+        if (w == 0) {
+            int t = lane < nt / 32 ? wsum[lane] : 0;
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, t, d);
+                if (lane >= d) t += y;
+            }
+            if (lane < nt / 32) wsum[lane] = t;
+        }
+        __syncthreads();
+        if (r < nr) s_start[r] = carry + x - len + (w > 0 ? wsum[w - 1] : 0);
+        carry += wsum[nt / 32 - 1];
+        __syncthreads();
+    }
+    uint32_t *out = masks + qa * max_chunks;
+    for (int c = tid; c < nch; c += nt) {
+        uint32_t gm = 0;
+#pragma unroll 1
+        for (int g = 0; g < 8; g++) {
+            const int pos = c * 64 + 8 * g;
+            // last run with S_r <= pos
+            int lo = 0, hi = nr - 1, r = -1;
+            while (lo <= hi) {
+                const int mid = (lo + hi) >> 1;
+                if (s_start[mid] <= pos) { r = mid; lo = mid + 1; }
+                else hi = mid - 1;
+            }
+            if (r >= 0) {
+                const int2 v = rr[r];
+                const int left = s_start[r] + (v.y - v.x) - pos;
+                gm |= (uint32_t)(left <= 0 ? 0 : (left >= 8 ? 8 : left)) << (4 * g);
+            }
+        }
+        out[c] = gm;
+    }
+}
+
+int attn_max_chunks(int N, int kk_cap) { return (N + 7 * kk_cap + 63) / 64 + 1; }
+
+void k_chunk_masks(int H, int kq_cap, int kk_cap, int max_chunks, const int2 *runs, const int2 *info,
+                   uint32_t *masks, cudaStream_t st) {
+    chunk_masks_kernel<<<dim3(kq_cap, H), 256, 0, st>>>(kq_cap, kk_cap, max_chunks, runs, info, masks);
+    note_launch();
+}
+
 int attn_max_items(int H, int N, int kq_cap) { return H * ((N + 127) / 128 + kq_cap); }
 
 void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,

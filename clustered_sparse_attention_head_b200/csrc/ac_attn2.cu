@@ -58,6 +58,8 @@ struct A2Params {
     int kk_cap, kq_cap;
     const int2 *runs;      // per (head, query cluster): ascending key-row runs
     const int2 *run_info;  // per (head, query cluster): {runs, chunks}
+    const uint32_t *masks; // per (head, query cluster, chunk): valid rows per 8-row group
+    int max_chunks;
     const AttnItem *items;
     const int32_t *n_items;
     __nv_bfloat16 *out;
@@ -76,6 +78,21 @@ namespace {
 __device__ __forceinline__ int item_chunks(const A2Params &p, const AttnItem &it) {
     if (it.a < 0) return (p.N + ATTN2_CHUNK - 1) / ATTN2_CHUNK;
     return p.run_info[(size_t)it.h * p.kq_cap + it.a].y;
+}
+
+// Valid-row counts (4 bits per 8-row group) of a chunk whose first `rows` rows are keys.
+__device__ __forceinline__ uint32_t prefix_mask(int rows) {
+    const int nf = rows >> 3;
+    uint32_t gm = (nf >= 8 ? 0xFFFFFFFFu : ((1u << (4 * nf)) - 1u)) & 0x88888888u;
+    if (rows & 7) gm |= (uint32_t)(rows & 7) << (4 * nf);
+    return gm;
+}
+// Mask of chunk j of an item: from the precomputed table, or, for a dense head
+// (one run of all N rows), from the chunk's position.
+__device__ __forceinline__ uint32_t item_mask(const A2Params &p, const uint32_t *mrow, int j) {
+    if (mrow) return __ldg(mrow + j);
+    const int left = p.N - j * ATTN2_CHUNK;
+    return prefix_mask(left > ATTN2_CHUNK ? ATTN2_CHUNK : left);
 }
 
 __device__ __forceinline__ void stream_init(KeyStream &ks, const A2Params &p, const AttnItem &it) {
@@ -120,17 +137,13 @@ __device__ __forceinline__ void fma2(float &o0, float &o1, float a0, float a1, f
     asm("mov.b64 {%0, %1}, %2;" : "=f"(o0), "=f"(o1) : "l"(d));
 }
 
-// 2^x on the FMA pipe (see ac_attn.cu for the derivation): magic-constant
-// rounding, cubic minimax fit on [-1/2, 1/2] (|rel err| < 7.5e-5), exponent add.
-__device__ __forceinline__ float ex2_fma(float x) {
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.0f;
-    const int n = __float_as_int(t) - 0x4B400000;
-    const float f = x - (t - 12582912.0f);
-    float q = fmaf(0.0551716648042202f, f, 0.2426111251115799f);
-    q = fmaf(q, f, 0.6932609677314758f);
-    q = fmaf(q, f, 0.9999280571937561f);
-    return __int_as_float(__float_as_int(q) + (n << 23));
+// (a0, a1) + (b0, b1), one packed fp32 add
+__device__ __forceinline__ void add2(float &a0, float &a1, float b0, float b1) {
+    uint64_t a, b, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(d));
 }
 
 // `rows` (a multiple of 8, at most 64) rows from global row `grow` into rows
@@ -454,21 +467,14 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 continue;
             }
-            KeyStream ks;
-            stream_init(ks, p, it);
+            // valid rows per 8-row group of each chunk, 4 bits each (8 = all),
+            // precomputed from the key runs; the next chunk's mask is loaded ahead
+            const uint32_t *mrow = it.a < 0 ? nullptr : p.masks + ((size_t)it.h * p.kq_cap + it.a) * p.max_chunks;
+            uint32_t gm_next = item_mask(p, mrow, 0);
             float m_ref = -INFINITY, l0 = 0.f, l1 = 0.f;
             for (int j = 0; j < nch; j++) {
-                // valid rows per 8-row group of the chunk, 4 bits each (8 = all)
-                uint32_t gm = 0;
-                {
-                    int fill = 0, start, v, sl;
-                    while (fill < C::BN && ks.piece(C::BN - fill, start, v, sl)) {
-                        const int g0 = fill >> 3, nf = v >> 3;
-                        gm |= ((nf >= 8 ? 0xFFFFFFFFu : ((1u << (4 * nf)) - 1u)) & 0x88888888u) << (4 * g0);
-                        if (v & 7) gm |= (uint32_t)(v & 7) << (4 * (g0 + nf));
-                        fill += sl;
-                    }
-                }
+                const uint32_t gm = gm_next;
+                if (j + 1 < nch) gm_next = item_mask(p, mrow, j + 1);
                 const uint32_t c = cnt + j;
                 const int b = c & 1;
                 if (!wait_warp(s_full + 2 * t + b, (c >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
@@ -524,16 +530,18 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 const float nm = -m_ref;
                 uint32_t pk[32];
-                // row sum in four partial sums (short dependences), folded into l0/l1
+                // row sum in four partial sums (two packed pairs, short dependences),
+                // folded into l0/l1.  All exponentials go to the MUFU pipe: the
+                // softmax is issue-bound, and an FMA-pipe polynomial for part of
+                // them cost more issue slots than it saved (measured on B200).
                 float la[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < 32; i++) {
                     float x0, x1;
                     fma2(x0, x1, __uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]), sc, nm);
                     const float e0 = ex2_approx(x0);
-                    const float e1 = (i & 1) ? ex2_fma(x1) : ex2_approx(x1);
-                    la[2 * (i & 1)] += e0;
-                    la[2 * (i & 1) + 1] += e1;
+                    const float e1 = ex2_approx(x1);
+                    add2(la[2 * (i & 1)], la[2 * (i & 1) + 1], e0, e1);
                     __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
                     pk[i] = *reinterpret_cast<uint32_t *>(&b2);
                 }
@@ -636,7 +644,8 @@ static int launch2(const void *qg, const void *kg, const void *vg, const A2Param
 }
 
 int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
-                 int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const AttnItem *items,
+                 int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const uint32_t *masks,
+                 int max_chunks, const AttnItem *items,
                  const int32_t *n_items, int max_items, void *out, float *lse, int *status, int num_sms,
                  void *encode_fn, cudaStream_t st) {
     A2Params p;
@@ -647,6 +656,8 @@ int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void
     p.kq_cap = kq_cap;
     p.runs = runs;
     p.run_info = run_info;
+    p.masks = masks;
+    p.max_chunks = max_chunks;
     p.items = items;
     p.n_items = n_items;
     p.out = reinterpret_cast<__nv_bfloat16 *>(out);
