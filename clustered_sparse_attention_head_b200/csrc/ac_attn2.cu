@@ -8,9 +8,9 @@
 // Each tile owns two S buffers in TMEM, so while softmax warpgroup t turns
 // S_t(j) into P_t(j) (bf16, written back over the same columns) the tensor
 // core already computes S_t(j+1) in the other buffer.  The single MMA thread
-// issues, per chunk j and tile t,
-//   O_t += P_t(j) V_j          (A operand read from TMEM) once P_t(j) is written,
-//   S_t(j+2) = Q_t K_{j+2}^T   into the buffer that P_t(j) occupied.
+// issues, per chunk j,
+//   O_t += P_t(j) V_j          (A operand read from TMEM) once P_t(j) is written, t = 0, 1,
+//   S_t(j+2) = Q_t K_{j+2}^T   into the buffer that P_t(j) occupied, t = 0, 1.
 // Ordering facts the protocol relies on (tcgen05 operations issued by one
 // thread execute in issue order, and a commit covers all earlier ones):
 //  - S_t(j+2) is issued after PV_t(j), so it never overwrites P_t(j) early;
@@ -40,7 +40,7 @@ template <int D> struct A2Cfg {
     static constexpr int SMEM_RAW = OFF_BAR + 512 + 1024;
     // at least 116 KB so that two CTAs never share an SM (each takes all of TMEM)
     static constexpr int SMEM = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
-    // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle:
+    // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA (Q, K), 9 MMA, 10 TMA (V), 11 idle:
     // three full warpgroups, so registers can move between them (setmaxnreg)
     static constexpr int NTHREADS = 384;
     static constexpr int REGS_LAUNCH = 168, REGS_LOW = 152, REGS_HIGH = 176;
@@ -149,29 +149,29 @@ __device__ __forceinline__ void add2(float &a0, float &a1, float b0, float b1) {
 // `rows` (a multiple of 8, at most 64) rows from global row `grow` into rows
 // r0.. of one K or V stage: one box per set bit of `rows`, per 64-column block.
 template <int D>
-__device__ __forceinline__ void load_rows(unsigned char *stage, int r0, int grow, int rows, const KVMaps &m,
-                                          uint64_t *bar, uint64_t pol) {
+__device__ __forceinline__ void load_rows(uint32_t ld, unsigned char *stage, int r0, int grow, int rows,
+                                          const KVMaps &m, uint64_t *bar, uint64_t pol) {
     using C = A2Cfg<D>;
 #pragma unroll
     for (int kb = 0; kb < C::DB; kb++) {
         unsigned char *dst = stage + kb * (C::BN * 128);
         int r = r0, g = grow;
-        if (rows & 64) { tma_load_2d_hint(dst + r * 128, &m.m64, bar, kb * 64, g, pol); r += 64; g += 64; }
-        if (rows & 32) { tma_load_2d_hint(dst + r * 128, &m.m32, bar, kb * 64, g, pol); r += 32; g += 32; }
-        if (rows & 16) { tma_load_2d_hint(dst + r * 128, &m.m16, bar, kb * 64, g, pol); r += 16; g += 16; }
-        if (rows & 8) tma_load_2d_hint(dst + r * 128, &m.m8, bar, kb * 64, g, pol);
+        if (rows & 64) { tma_load_2d_hint_p(ld, dst + r * 128, &m.m64, bar, kb * 64, g, pol); r += 64; g += 64; }
+        if (rows & 32) { tma_load_2d_hint_p(ld, dst + r * 128, &m.m32, bar, kb * 64, g, pol); r += 32; g += 32; }
+        if (rows & 16) { tma_load_2d_hint_p(ld, dst + r * 128, &m.m16, bar, kb * 64, g, pol); r += 16; g += 16; }
+        if (rows & 8) tma_load_2d_hint_p(ld, dst + r * 128, &m.m8, bar, kb * 64, g, pol);
     }
 }
 
 // The next chunk of the stream into one stage, each piece into its slot;
 // returns the rows loaded.
 template <int D>
-__device__ __forceinline__ int load_chunk(KeyStream &ks, unsigned char *stage, int row_base, const KVMaps &m,
-                                          uint64_t *bar, uint64_t pol) {
+__device__ __forceinline__ int load_chunk(uint32_t ld, KeyStream &ks, unsigned char *stage, int row_base,
+                                          const KVMaps &m, uint64_t *bar, uint64_t pol) {
     using C = A2Cfg<D>;
     int fill = 0, start = 0, valid = 0, slot = 0;
     while (fill < C::BN && ks.piece(C::BN - fill, start, valid, slot)) {
-        load_rows<D>(stage, fill, row_base + start, slot, m, bar, pol);
+        load_rows<D>(ld, stage, fill, row_base + start, slot, m, bar, pol);
         fill += slot;
     }
     return fill;
@@ -286,54 +286,57 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp >= 8) {
     regs_dec<C::REGS_LOW>();
-    if (warp == 8) {
-        // ------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            // K/V rows are re-read by every query item of the head: keep them in
-            // L2; query tiles are read once: let them go first
-            const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
-            uint32_t g = 0, qi = 0;
-            uint32_t nk_loads = 0, nv_loads = 0;  // chunks whose K / V copies were issued
-            bool ok = true;
-            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-                const AttnItem it = p.items[item];
-                const int nch = item_chunks(p, it);
-                if (nch == 0) continue;
+    if (warp == 8 || warp == 10) {
+        // ------------------------------------------------------ TMA producers
+        // Warp 8 loads Q and K, warp 10 loads V.  Each runs its loop converged,
+        // with identical values in every lane, and one lane issues the copies.
+        // One lone thread loading K and V in turn could not keep up: the V
+        // ring frees slots late (after P.V), and each K load waited behind it.
+        const bool kq = warp == 8;
+        const uint32_t leader = elect_leader();
+        // K/V rows are re-read by every query item of the head: keep them in
+        // L2; query tiles are read once: let them go first
+        const uint64_t pol_keep = l2_policy_evict_last(), pol_stream = l2_policy_evict_first();
+        uint64_t *full = kq ? k_full : v_full, *empty = kq ? k_empty : v_empty;
+        constexpr int NST = C::KST;  // == C::VST
+        static_assert(C::KST == C::VST, "one ring depth for both producers");
+        unsigned char *ring = sm + (kq ? C::OFF_K : C::OFF_V);
+        const KVMaps &maps = kq ? mk : mv;
+        uint32_t g = 0, qi = 0, nloads = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            const AttnItem it = p.items[item];
+            const int nch = item_chunks(p, it);
+            if (nch == 0) continue;
+            if (kq) {
                 const int nt = it.q_len > 128 ? 2 : 1;
-                if (qi >= 1 && !mbar_wait(q_empty, (qi - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                mbar_arrive_expect_tx(q_full, nt * C::Q_BYTES);
+                if (qi >= 1 && !mbar_wait_warp(q_empty, (qi - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                mbar_arrive_expect_tx_p(leader, q_full, nt * C::Q_BYTES);
                 for (int t = 0; t < nt; t++)
                     for (int kb = 0; kb < C::DB; kb++)
-                        tma_load_2d_hint(sm + C::OFF_Q + t * C::Q_BYTES + kb * (C::BM * 128), &tmQ, q_full,
-                                         kb * 64, it.h * p.N + it.q_start + t * 128, pol_stream);
+                        tma_load_2d_hint_p(leader, sm + C::OFF_Q + t * C::Q_BYTES + kb * (C::BM * 128), &tmQ, q_full,
+                                           kb * 64, it.h * p.N + it.q_start + t * 128, pol_stream);
                 qi++;
-                KeyStream ks;
-                stream_init(ks, p, it);
-                const int row_base = it.h * p.N;
-                for (int j = 0; j < nch; j++, g++) {
-                    KeyStream kk = ks, probe = ks;
-                    const uint32_t bytes = (uint32_t)chunk_rows(probe, C::BN) * 128u * C::DB;
-                    const int kslot = g % C::KST, vslot = g % C::VST;
-                    const uint32_t ku = g / C::KST, vu = g / C::VST;
-                    if (ku >= 1 && !mbar_wait(k_empty + kslot, (ku - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(k_full + kslot, bytes);
-                    load_chunk<D>(kk, sm + C::OFF_K + kslot * C::KV_BYTES, row_base, mk, k_full + kslot, pol_keep);
-                    nk_loads = g + 1;
-                    if (vu >= 1 && !mbar_wait(v_empty + vslot, (vu - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(v_full + vslot, bytes);
-                    load_chunk<D>(ks, sm + C::OFF_V + vslot * C::KV_BYTES, row_base, mv, v_full + vslot, pol_keep);
-                    nv_loads = g + 1;
-                }
             }
-            if (!ok) {
-                // wait (bounded) for every copy in flight before the CTA exits
-                // (slot i last received chunk i + KST * ((loads - 1 - i) / KST))
-                if (qi >= 1) drain(q_full, (qi - 1) & 1);
-                for (uint32_t i = 0; i < (uint32_t)C::KST && i < nk_loads; i++)
-                    drain(k_full + i, ((nk_loads - 1 - i) / C::KST) & 1);
-                for (uint32_t i = 0; i < (uint32_t)C::VST && i < nv_loads; i++)
-                    drain(v_full + i, ((nv_loads - 1 - i) / C::VST) & 1);
+            KeyStream ks;
+            stream_init(ks, p, it);
+            const int row_base = it.h * p.N;
+            for (int j = 0; j < nch; j++, g++) {
+                KeyStream probe = ks;
+                const uint32_t bytes = (uint32_t)chunk_rows(probe, C::BN) * 128u * C::DB;
+                const int slot = g % NST;
+                const uint32_t u = g / NST;
+                if (u >= 1 && !mbar_wait_warp(empty + slot, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                mbar_arrive_expect_tx_p(leader, full + slot, bytes);
+                load_chunk<D>(leader, ks, ring + slot * C::KV_BYTES, row_base, maps, full + slot, pol_keep);
+                nloads = g + 1;
             }
+        }
+        if (!ok) {
+            // wait (bounded) for every copy in flight before the CTA exits
+            // (slot i last received chunk i + NST * ((loads - 1 - i) / NST))
+            if (kq && qi >= 1) drain(q_full, (qi - 1) & 1);
+            for (uint32_t i = 0; i < (uint32_t)NST && i < nloads; i++) drain(full + i, ((nloads - 1 - i) / NST) & 1);
         }
     } else if (warp == 9) {
         // --------------------------------------------------------- MMA issuer
@@ -399,13 +402,17 @@ __global__ void __launch_bounds__(384, 1)
                         issue_pv<D>(leader, tmem + C::TM_O + t * D, tmem + C::TM_S + t * 128 + b * 64,
                                     vdesc0 + (uint64_t)((vslot * C::KV_BYTES) >> 4), j == 0);
                         umma_commit_p(leader, pv_bar + t);
-                        // S_t(j+2) into the buffer P_t(j) occupied
-                        if (more) {
-                            if (t == 0 && !wait_warp(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
+                    }
+                    // S_t(j+2) into the buffers P_t(j) occupied, after both P.V
+                    // groups: the other tile's P.V runs between the reads of a
+                    // buffer and its overwrite
+                    if (ok && more) {
+                        if (!wait_warp(k_full + kslot, (gk / C::KST) & 1, abort_flag, p.status)) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int t = 0; t < 2; t++) {
+                            if (t >= nt) break;
+                            const int b = (cnt[t] + j) & 1;
                             issue_s<D>(leader, tmem + C::TM_S + t * 128 + b * 64, qdesc + (uint64_t)((t * C::Q_BYTES) >> 4),
                                        kdesc0 + (uint64_t)((kslot * C::KV_BYTES) >> 4));
                             umma_commit_p(leader, s_full + 2 * t + b);
