@@ -323,8 +323,16 @@ def main():
         pass
     peak = peaks.get("bf16_tflops_sustained") or 1390.6
     peak_src = "measured (MEASURED_PEAKS.json bf16_tflops_sustained)" if peaks else "fallback"
-    roof = {"kernel": "attn_kernel (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": tflops_attn,
-            "peak": peak, "unit": "TFLOP/s", "frac": tflops_attn / peak, "traffic": None,
+    # DRAM bytes of one attention launch, from an ncu capture of this kernel
+    # on the Wan-shaped workload cut to 8 heads (2.571 GB read + 0.146 GB
+    # written), scaled by heads; only for that workload and kernel version
+    traffic = None
+    if w.name == DEFAULT_WORKLOAD and w.top_p == 0.9:
+        traffic = 2.717e9 * w.heads / 8
+    roof = {"kernel": "attn2_kernel (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": tflops_attn,
+            "peak": peak, "unit": "TFLOP/s", "frac": tflops_attn / peak, "traffic": traffic,
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, 8-head capture scaled by heads"
+            if traffic else None,
             "peak_source": peak_src, "ms_per_launch": attn_ms,
             "flops_per_launch": flops, "flops_rule": "4 * d * computed (query, key) pairs"}
 
