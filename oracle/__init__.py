@@ -67,6 +67,9 @@ def _load():
         lib.orc_multistage.restype = i32
         lib.orc_cluster_mean_norm.argtypes = [i64, _P, _P, i32, _P]
         lib.orc_select.argtypes = [i32, i32, _P, _P, _P, i32, _P, _P, dbl, i32, _P, _P]
+        lib.orc_select2.argtypes = [i32, i32, _P, _P, _P, i32, _P, _P, _P, _P, i32, i32, dbl, i32, _P, _P]
+        lib.orc_key_bounds.argtypes = [i64, i32, _P, _P, i32, _P, _P]
+        lib.orc_scores.argtypes = [i32, i32, i32, _P, _P, i32, _P, _P, _P, _P]
         lib.orc_cluster_sort.argtypes = [i64, _P, i32, _P, _P]
         lib.orc_attention_rows.argtypes = [i64, i32, _P, _P, _P, _P, _P, i32, _P, _P, i32, i32, i64,
                                            _P, _P]
@@ -202,6 +205,50 @@ def select(q_cent, q_mean_norm, q_count, k_cent, k_count, top_p):
     return sel, cnt
 
 
+SCORE_CENTROID, SCORE_QUEST = 0, 1
+
+
+def key_bounds(k, ids, kk):
+    """Per key cluster and dimension: the largest and the smallest key value
+    (Quest's page bounds, §3.2.3 eq. (1)); zeros for clusters without members."""
+    k = _f32(k)
+    n, d = k.shape
+    kmax = np.empty((kk, d), np.float32)
+    kmin = np.empty((kk, d), np.float32)
+    _load().orc_key_bounds(n, d, _p(k), _p(_i32(ids)), kk, _p(kmax), _p(kmin))
+    return kmax, kmin
+
+
+def select2(q_cent, q_mean_norm, q_count, k_cent, k_count, top_p=0.9, score_mode=SCORE_CENTROID, top_k=0,
+            k_max=None, k_min=None):
+    """Selection with either score (centroid, or the Quest bound of eq. (1))
+    and either cut (top-p, or Algorithm 3's argtopk when top_k > 0)."""
+    q_cent, k_cent = _f32(q_cent), _f32(k_cent)
+    kq, d = q_cent.shape
+    kk = k_cent.shape[0]
+    sel = np.full((kq, max(kk, 1)), -1, np.int32)
+    cnt = np.zeros(kq, np.int32)
+    km = _f32(k_max) if k_max is not None else None
+    kn = _f32(k_min) if k_min is not None else None
+    _load().orc_select2(d, kq, _p(q_cent), _p(_f32(q_mean_norm)), _p(_i32(q_count)), kk, _p(k_cent),
+                        _p(_i32(k_count)), _p(km), _p(kn), int(score_mode), int(top_k), float(top_p), sel.shape[1],
+                        _p(sel), _p(cnt))
+    return sel, cnt
+
+
+def scores(q_cent, q_mean_norm, k_cent=None, score_mode=SCORE_CENTROID, k_max=None, k_min=None):
+    """The selection score s_ab of every (query cluster, key cluster) pair."""
+    q_cent = _f32(q_cent)
+    kq, d = q_cent.shape
+    kk = (k_cent if k_cent is not None else k_max).shape[0]
+    out = np.empty((kq, kk), np.float64)
+    _load().orc_scores(int(score_mode), d, kq, _p(q_cent), _p(_f32(q_mean_norm)), kk,
+                       _p(_f32(k_cent)) if k_cent is not None else None,
+                       _p(_f32(k_max)) if k_max is not None else None,
+                       _p(_f32(k_min)) if k_min is not None else None, _p(out))
+    return out
+
+
 def cluster_sort(ids, k):
     ids = _i32(ids)
     perm = np.empty(len(ids), np.int32)
@@ -252,6 +299,8 @@ class HeadSpec:
     tau_value: float = 0.0
     nmax_q: int = 0
     nmax_k: int = 0
+    score_mode: int = 0   # SCORE_CENTROID or SCORE_QUEST
+    top_k: int = 0        # > 0: argtopk instead of top-p
 
 
 @dataclass
@@ -292,7 +341,11 @@ def forward_head(q, k, v, spec: HeadSpec, rows=None):
         sel = np.zeros((rq.nclusters, max(rk.nclusters, 1)), np.int32)
         cnt = np.zeros(rq.nclusters, np.int32)
     else:
-        sel, cnt = select(rq.cent, qmn, rq.count, rk.cent, rk.count, spec.top_p)
+        kmax = kmin = None
+        if spec.score_mode == SCORE_QUEST:
+            kmax, kmin = key_bounds(k, rk.assign, rk.nclusters)
+        sel, cnt = select2(rq.cent, qmn, rq.count, rk.cent, rk.count, spec.top_p, spec.score_mode, spec.top_k,
+                           kmax, kmin)
     if rows is None:
         rows = np.arange(q.shape[0], dtype=np.int32)
     out = attention_rows(q, k, v, rq.assign, rk.assign, rk.nclusters, sel, cnt, dense, rows)

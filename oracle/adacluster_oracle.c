@@ -17,7 +17,10 @@
  * Cluster selection follows the centroid-centroid reading: score each key cluster
  * by its centroid against the query-cluster centroid, weight by cluster size,
  * keep the smallest top-p prefix (§2.3 names centroid-based significance
- * estimation; Algorithm 3 lines 6-7 is the select step it replaces).
+ * estimation; Algorithm 3 lines 6-7 is the select step it replaces).  The
+ * alternative score is Quest's per-page upper bound (§3.2.3, eq. (1)) of the
+ * representative query against each key cluster's per-dimension max/min, and
+ * the alternative cut is Algorithm 3's argtopk.
  *
  * Arithmetic: every input is fp32 (bf16 inputs arrive widened, which is exact)
  * and is widened to double.  All sums and products are double, evaluated in the
@@ -28,7 +31,10 @@
  * Parity pins (tests/test_oracle_pins.py): brute-force argmin on tiny inputs,
  * k-means objective monotonicity, k = 1 closed forms, Algorithm 1 closed-form
  * traces (tau = 0, tau = inf, N_max), selection invariants and a hand-derived
- * example, select-all attention = dense softmax attention, stable sort.
+ * example, select-all attention = dense softmax attention, stable sort; the
+ * Quest bound dominates every key of its page and is attained by a one-key page
+ * or by the page's corner key, per-page max/min equal numpy's, and argtopk on a
+ * hand example.
  * The score/weight reading of the selection rule is "parity unpinned" by the
  * paper itself (it is pinned only by invariants and a hand example).
  */
@@ -298,12 +304,44 @@ void orc_cluster_mean_norm(int64_t n, const double *norm, const int32_t *assign,
     free(c);
 }
 
-/* Critical-cluster selection (centroid-centroid scores weighted by size, top-p).
- * For each non-empty query cluster a:
- *   s_ab = (rbar_a * (mu_a . c_b)) * (1/sqrt(d))   for non-empty key clusters b,
- *   w_ab = n_b * exp(s_ab - max_b s_ab),  p_ab = w_ab / sum_b w_ab (sum in b order),
- *   visit b by p descending (ties: lower b first), accumulating p; keep b until
- *   the running sum reaches top_p.  top_p >= 1 keeps every non-empty b.
+/* Quest bounds of the key clusters (§3.2.3, eq. (1)): for cluster b and
+ * dimension t, kmax[b*d + t] is the largest k_i[t] over the members i of b and
+ * kmin[b*d + t] the smallest.  Clusters without members get 0.              */
+void orc_key_bounds(int64_t n, int d, const float *k, const int32_t *assign, int kk, float *kmax, float *kmin)
+{
+    char *seen = (char *)calloc((size_t)(kk > 0 ? kk : 1), 1);
+    for (int64_t j = 0; j < (int64_t)kk * d; j++) { kmax[j] = 0.0f; kmin[j] = 0.0f; }
+    for (int64_t i = 0; i < n; i++) {
+        const int b = assign[i];
+        const float *x = k + i * d;
+        float *M = kmax + (int64_t)b * d, *m = kmin + (int64_t)b * d;
+        if (!seen[b]) {
+            for (int t = 0; t < d; t++) { M[t] = x[t]; m[t] = x[t]; }
+            seen[b] = 1;
+        } else {
+            for (int t = 0; t < d; t++) {
+                if (x[t] > M[t]) M[t] = x[t];
+                if (x[t] < m[t]) m[t] = x[t];
+            }
+        }
+    }
+    free(seen);
+}
+
+/* Critical-cluster selection.  For each non-empty query cluster a and each
+ * non-empty key cluster b, a score s_ab:
+ *   score_mode 0 (centroid): s_ab = (rbar_a * (mu_a . c_b)) * (1/sqrt(d));
+ *   score_mode 1 (Quest, §3.2.3 eq. (1)): with the representative query
+ *     qbar = rbar_a * mu_a, s_ab = (sum_t max(qbar_t * M_bt, qbar_t * m_bt)) * (1/sqrt(d)),
+ *     M_b / m_b the per-dimension maximum / minimum of the keys of b (an upper
+ *     bound of qbar . k over every key k of b).
+ * Then either
+ *   top_k > 0 (Algorithm 3 line 7, argtopk): keep the top_k b of largest s_ab
+ *     (ties: lower b first), or all of them if fewer are non-empty;
+ *   else the top-p rule: w_ab = n_b * exp(s_ab - max_b s_ab), p_ab = w_ab / sum_b w_ab
+ *     (sum in b order); visit b by p descending (ties: lower b first),
+ *     accumulating p; keep b until the running sum reaches top_p; top_p >= 1
+ *     keeps every non-empty b.
  * Empty query clusters select nothing.  The kept set is written in ascending b
  * to sel_idx[a * kk_stride ...], its size to sel_cnt[a].                      */
 typedef struct { double p; int b; } orc_pb;
@@ -315,9 +353,40 @@ static int orc_cmp_pb(const void *x, const void *y)
     return (a->b > b->b) - (a->b < b->b);
 }
 
-void orc_select(int d, int kq, const float *q_cent, const float *q_mean_norm, const int32_t *q_count,
-                int kk, const float *k_cent, const int32_t *k_count, double top_p,
-                int kk_stride, int32_t *sel_idx, int32_t *sel_cnt)
+/* s_ab of one (query cluster, key cluster) pair, as defined for orc_select2. */
+static double orc_sel_score(int score_mode, int d, double scale, const float *mu, double rbar, const float *c,
+                        const float *M, const float *mn)
+{
+    if (score_mode == 1) {
+        double acc = 0.0;
+        for (int t = 0; t < d; t++) {
+            const double qb = rbar * (double)mu[t];
+            const double hi = qb * (double)M[t], lo = qb * (double)mn[t];
+            acc = acc + (hi > lo ? hi : lo);
+        }
+        return acc * scale;
+    }
+    double dot = 0.0;
+    for (int t = 0; t < d; t++) dot = dot + (double)mu[t] * (double)c[t];
+    return (rbar * dot) * scale;
+}
+
+/* Every s_ab into scores[a * kk + b] (for the pins). */
+void orc_scores(int score_mode, int d, int kq, const float *q_cent, const float *q_mean_norm, int kk,
+                const float *k_cent, const float *k_max, const float *k_min, double *scores)
+{
+    const double scale = 1.0 / sqrt((double)d);
+    for (int a = 0; a < kq; a++)
+        for (int b = 0; b < kk; b++)
+            scores[(int64_t)a * kk + b] =
+                orc_sel_score(score_mode, d, scale, q_cent + (int64_t)a * d, (double)q_mean_norm[a],
+                          k_cent ? k_cent + (int64_t)b * d : 0, k_max ? k_max + (int64_t)b * d : 0,
+                          k_min ? k_min + (int64_t)b * d : 0);
+}
+
+void orc_select2(int d, int kq, const float *q_cent, const float *q_mean_norm, const int32_t *q_count,
+                 int kk, const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min,
+                 int score_mode, int top_k, double top_p, int kk_stride, int32_t *sel_idx, int32_t *sel_cnt)
 {
     double scale = 1.0 / sqrt((double)d);
 #pragma omp parallel for schedule(dynamic)
@@ -329,35 +398,45 @@ void orc_select(int d, int kq, const float *q_cent, const float *q_mean_norm, co
         orc_pb *pb = (orc_pb *)malloc(sizeof(orc_pb) * (size_t)(kk > 0 ? kk : 1));
         char *keep = (char *)calloc((size_t)(kk > 0 ? kk : 1), 1);
         const float *mu = q_cent + (int64_t)a * d;
+        const double rbar = (double)q_mean_norm[a];
         double m = -INFINITY;
         for (int b = 0; b < kk; b++) {
             if (k_count[b] == 0) continue;
-            const float *c = k_cent + (int64_t)b * d;
-            double dot = 0.0;
-            for (int t = 0; t < d; t++) dot = dot + (double)mu[t] * (double)c[t];
-            s[b] = ((double)q_mean_norm[a] * dot) * scale;
+            s[b] = orc_sel_score(score_mode, d, scale, mu, rbar, k_cent + (int64_t)b * d,
+                             score_mode == 1 ? k_max + (int64_t)b * d : 0, score_mode == 1 ? k_min + (int64_t)b * d : 0);
             if (s[b] > m) m = s[b];
         }
-        double W = 0.0;
         int np = 0;
-        for (int b = 0; b < kk; b++) {
-            if (k_count[b] == 0) continue;
-            double w = (double)k_count[b] * exp(s[b] - m);
-            s[b] = w;
-            W = W + w;
-        }
-        for (int b = 0; b < kk; b++) {
-            if (k_count[b] == 0) continue;
-            pb[np].p = s[b] / W;
-            pb[np].b = b;
-            np++;
-        }
-        qsort(pb, (size_t)np, sizeof(orc_pb), orc_cmp_pb);
-        double cum = 0.0;
-        for (int r = 0; r < np; r++) {
-            keep[pb[r].b] = 1;
-            cum = cum + pb[r].p;
-            if (top_p < 1.0 && cum >= top_p) break;
+        if (top_k > 0) {
+            for (int b = 0; b < kk; b++) {
+                if (k_count[b] == 0) continue;
+                pb[np].p = s[b];
+                pb[np].b = b;
+                np++;
+            }
+            qsort(pb, (size_t)np, sizeof(orc_pb), orc_cmp_pb);
+            for (int r = 0; r < np && r < top_k; r++) keep[pb[r].b] = 1;
+        } else {
+            double W = 0.0;
+            for (int b = 0; b < kk; b++) {
+                if (k_count[b] == 0) continue;
+                double w = (double)k_count[b] * exp(s[b] - m);
+                s[b] = w;
+                W = W + w;
+            }
+            for (int b = 0; b < kk; b++) {
+                if (k_count[b] == 0) continue;
+                pb[np].p = s[b] / W;
+                pb[np].b = b;
+                np++;
+            }
+            qsort(pb, (size_t)np, sizeof(orc_pb), orc_cmp_pb);
+            double cum = 0.0;
+            for (int r = 0; r < np; r++) {
+                keep[pb[r].b] = 1;
+                cum = cum + pb[r].p;
+                if (top_p < 1.0 && cum >= top_p) break;
+            }
         }
         int c = 0;
         for (int b = 0; b < kk; b++)
@@ -367,6 +446,15 @@ void orc_select(int d, int kq, const float *q_cent, const float *q_mean_norm, co
         free(pb);
         free(keep);
     }
+}
+
+/* The centroid score with the top-p rule (score_mode 0, top_k 0). */
+void orc_select(int d, int kq, const float *q_cent, const float *q_mean_norm, const int32_t *q_count,
+                int kk, const float *k_cent, const int32_t *k_count, double top_p,
+                int kk_stride, int32_t *sel_idx, int32_t *sel_cnt)
+{
+    orc_select2(d, kq, q_cent, q_mean_norm, q_count, kk, k_cent, k_count, 0, 0, 0, 0, top_p, kk_stride, sel_idx,
+                sel_cnt);
 }
 
 /* Stable counting sort of token ids by cluster id: perm lists the tokens of

@@ -398,3 +398,105 @@ def test_forward_head_dense_flag(orc):
     r = orc.forward_head(h.q, h.k, h.v, spec, rows=np.arange(0, 400, 9))
     assert r.dense == 1
     np.testing.assert_allclose(r.out_rows, _np_attention(h.q[::9], h.k, h.v), rtol=1e-10, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Quest bounds (§3.2.3 eq. (1)) and the argtopk cut (Algorithm 3 line 7)
+# --------------------------------------------------------------------------
+def test_key_bounds_are_member_extremes(orc):
+    """Per cluster and dimension: the largest / smallest member value (numpy's
+    max/min over the members), zeros for an empty cluster."""
+    rng = np.random.default_rng(21)
+    n, d, kk = 300, 16, 9
+    k = rng.standard_normal((n, d)).astype(np.float32)
+    ids = rng.integers(0, kk - 1, size=n).astype(np.int32)  # cluster kk-1 stays empty
+    kmax, kmin = orc.key_bounds(k, ids, kk)
+    for b in range(kk):
+        mem = k[ids == b]
+        if len(mem):
+            np.testing.assert_array_equal(kmax[b], mem.max(0))
+            np.testing.assert_array_equal(kmin[b], mem.min(0))
+        else:
+            assert not kmax[b].any() and not kmin[b].any()
+
+
+def test_quest_score_bounds_every_member_and_is_tight(orc):
+    """Eq. (1) is an upper bound of qbar.k over the keys k of a page, attained
+    when a page holds one key (or when every key sits at the page's corner)."""
+    rng = np.random.default_rng(22)
+    d, kq, kk = 32, 5, 7
+    q_cent = rng.standard_normal((kq, d)).astype(np.float32)
+    rbar = rng.uniform(0.5, 2.0, kq).astype(np.float32)
+    pages = [rng.standard_normal((int(rng.integers(1, 9)), d)).astype(np.float32) for _ in range(kk)]
+    pages[0] = pages[0][:1]  # a one-key page
+    kmax = np.stack([p.max(0) for p in pages])
+    kmin = np.stack([p.min(0) for p in pages])
+    s = orc.scores(q_cent, rbar, score_mode=orc.SCORE_QUEST, k_max=kmax, k_min=kmin) * np.sqrt(d)
+    for a in range(kq):
+        qbar = rbar[a].astype(np.float64) * q_cent[a].astype(np.float64)
+        for b in range(kk):
+            dots = pages[b].astype(np.float64) @ qbar
+            assert s[a, b] >= dots.max() - 1e-9 * (1 + abs(dots.max()))
+        one = pages[0][0].astype(np.float64) @ qbar
+        assert s[a, 0] == pytest.approx(one, rel=1e-12, abs=1e-12)
+    # the corner key (per-dimension choice of max or min by the sign of qbar)
+    # attains the bound exactly
+    qbar = rbar[0].astype(np.float64) * q_cent[0].astype(np.float64)
+    corner = np.where(qbar >= 0, kmax[3], kmin[3]).astype(np.float64)
+    assert s[0, 3] == pytest.approx(corner @ qbar, rel=1e-12)
+
+
+def test_quest_score_of_single_key_pages_is_the_centroid_score(orc):
+    """With one key per page (max = min = the key = its centroid) the Quest
+    bound is the centroid dot product, so both scores pick the same top-k."""
+    rng = np.random.default_rng(23)
+    d, kq, kk = 24, 6, 40
+    q_cent = rng.standard_normal((kq, d)).astype(np.float32)
+    rbar = rng.uniform(0.5, 2.0, kq).astype(np.float32)
+    c = rng.standard_normal((kk, d)).astype(np.float32)
+    s0 = orc.scores(q_cent, rbar, k_cent=c)
+    s1 = orc.scores(q_cent, rbar, k_cent=c, score_mode=orc.SCORE_QUEST, k_max=c, k_min=c)
+    np.testing.assert_allclose(s1, s0, rtol=1e-12, atol=1e-12)
+    qc, kc = np.ones(kq, np.int32), np.ones(kk, np.int32)
+    a0, n0 = orc.select2(q_cent, rbar, qc, c, kc, top_k=7)
+    a1, n1 = orc.select2(q_cent, rbar, qc, c, kc, top_k=7, score_mode=orc.SCORE_QUEST, k_max=c, k_min=c)
+    np.testing.assert_array_equal(n0, 7)
+    np.testing.assert_array_equal(a0[:, :7], a1[:, :7])
+
+
+def test_topk_hand_example(orc):
+    """argtopk by score, ties to the lower cluster id, empty clusters never
+    kept, k larger than the non-empty count keeps them all; the size weights
+    of the top-p rule play no part."""
+    mu = np.array([[1.0, 0.0]], np.float32)
+    rbar = np.array([np.sqrt(2.0)], np.float32)  # s_b = c_b[0] exactly
+    c = np.array([[3, 0], [1, 0], [2, 0], [2, 0], [9, 0]], np.float32)
+    kc = np.array([1, 100, 5, 5, 0], np.int32)   # cluster 4 (best score) is empty
+    qc = np.array([3], np.int32)
+    s = orc.scores(mu, rbar, k_cent=c)
+    np.testing.assert_allclose(s[0], [3, 1, 2, 2, 9], rtol=1e-6)
+    sel, cnt = orc.select2(mu, rbar, qc, c, kc, top_k=2)
+    assert cnt[0] == 2 and list(sel[0, :2]) == [0, 2]
+    sel, cnt = orc.select2(mu, rbar, qc, c, kc, top_k=3)
+    assert cnt[0] == 3 and list(sel[0, :3]) == [0, 2, 3]
+    sel, cnt = orc.select2(mu, rbar, qc, c, kc, top_k=50)
+    assert cnt[0] == 4 and list(sel[0, :4]) == [0, 1, 2, 3]
+
+
+def test_quest_selects_a_page_with_an_aligned_outlier(orc):
+    """A page whose centroid points away from the query but holds one key
+    aligned with it: the centroid score ranks it last, the Quest bound first."""
+    d = 4
+    mu = np.array([[1.0, 0.0, 0.0, 0.0]], np.float32)
+    rbar = np.array([1.0], np.float32)
+    far = np.array([[-1, 0, 0, 0], [-1, 0, 0, 0], [-1, 0, 0, 0], [5, 0, 0, 0]], np.float32)  # mean (0.5, 0, 0, 0)
+    near = np.array([[1, 0, 0, 0], [1, 0, 0, 0]], np.float32)
+    pages = [far, near]
+    c = np.stack([p.mean(0) for p in pages]).astype(np.float32)
+    kmax = np.stack([p.max(0) for p in pages])
+    kmin = np.stack([p.min(0) for p in pages])
+    kc = np.array([4, 2], np.int32)
+    qc = np.array([1], np.int32)
+    sel0, _ = orc.select2(mu, rbar, qc, c, kc, top_k=1)
+    sel1, _ = orc.select2(mu, rbar, qc, c, kc, top_k=1, score_mode=orc.SCORE_QUEST, k_max=kmax, k_min=kmin)
+    assert sel0[0, 0] == 1 and sel1[0, 0] == 0
