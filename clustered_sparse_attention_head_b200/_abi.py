@@ -19,10 +19,11 @@ AC_ERR_WORKSPACE, AC_ERR_TIMEOUT, AC_ERR_NONFINITE, AC_ERR_CAPACITY = 4, 5, 6, 7
 AC_F32, AC_BF16 = 0, 1
 AC_TAU_ABS, AC_TAU_MEAN_X, AC_TAU_MEDIAN_RADIUS_X = 0, 1, 2
 AC_FLAG_WARM_START, AC_FLAG_CHECK_FINITE, AC_FLAG_PROFILE = 1, 2, 4
+AC_SCORE_CENTROID, AC_SCORE_QUEST = 0, 1
 
 # every entry point declared in include/adacluster.h
 EXPORTS = ["ac_create", "ac_destroy", "ac_capacities", "ac_workspace_size", "ac_cluster_q", "ac_cluster_k",
-           "ac_select", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_profile_read", "ac_get_status",
+           "ac_select", "ac_key_bounds", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_profile_read", "ac_get_status",
            "ac_status_string"]
 
 
@@ -30,7 +31,7 @@ class ac_config(ctypes.Structure):
     _fields_ = [("heads", c_int), ("n", c_int), ("d", c_int), ("dtype", c_int), ("kq", c_int), ("kk", c_int),
                 ("iters", c_int), ("adaptive_q", c_int), ("adaptive_k", c_int), ("tau_rule", c_int),
                 ("tau_value", c_double), ("nmax_q", c_int), ("nmax_k", c_int), ("top_p", c_double),
-                ("flags", c_uint)]
+                ("flags", c_uint), ("score_mode", c_int), ("top_k", c_int)]
 
 
 class ac_stats(ctypes.Structure):
@@ -70,7 +71,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ac_workspace_size": ([P, POINTER(c_size_t)], c_int),
         "ac_cluster_q": ([P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_cluster_k": ([P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
-        "ac_select": ([P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
+        "ac_select": ([P, P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
+        "ac_key_bounds": ([P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_cluster_sort": ([P, P, c_int, P, P, P, P, c_size_t, P], c_int),
         "ac_cluster_sort_static": ([P, c_int, c_int, c_int, P, P, P, P], c_int),
         "ac_sparse_attn": ([P, P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),

@@ -32,12 +32,14 @@ class Config:
     nmax_k: int = 0
     top_p: float = 0.9
     flags: int = 0
+    score_mode: int = _abi.AC_SCORE_CENTROID   # or AC_SCORE_QUEST
+    top_k: int = 0                             # > 0: argtopk instead of top-p
 
     def to_c(self) -> _abi.ac_config:
         return _abi.ac_config(self.heads, self.n, self.d, _abi.AC_BF16 if self.dtype == "bf16" else _abi.AC_F32,
                               self.kq, self.kk, self.iters, int(self.adaptive_q), int(self.adaptive_k),
                               self.tau_rule, float(self.tau_value), self.nmax_q, self.nmax_k, float(self.top_p),
-                              self.flags)
+                              self.flags, int(self.score_mode), int(self.top_k))
 
     @property
     def torch_dtype(self):
@@ -122,15 +124,23 @@ class AdaCluster:
         return out
 
     def ac_select(self, q_cent, q_mean_norm, q_count, k_cent, k_count, nq=None, nk=None, dense_flag=None,
-                  stream=None):
+                  k_max=None, k_min=None, stream=None):
         H = self.cfg.heads
         sel = torch.full((H, self.kq_cap, self.kk_cap), -1, dtype=torch.int32, device=self.device)
         cnt = self._i32(H, self.kq_cap)
         ws, nb = self._args_ws()
         check("ac_select", self.lib.ac_select(
-            self._ctx, ptr(q_cent), ptr(q_mean_norm), ptr(q_count), ptr(k_cent), ptr(k_count), ptr(nq), ptr(nk),
-            ptr(dense_flag), ptr(sel), ptr(cnt), ws, nb, stream_ptr(stream)))
+            self._ctx, ptr(q_cent), ptr(q_mean_norm), ptr(q_count), ptr(k_cent), ptr(k_count), ptr(k_max),
+            ptr(k_min), ptr(nq), ptr(nk), ptr(dense_flag), ptr(sel), ptr(cnt), ws, nb, stream_ptr(stream)))
         return sel, cnt
+
+    def ac_key_bounds(self, k, k_assign, nk=None, stream=None):
+        H, D = self.cfg.heads, self.cfg.d
+        kmax, kmin = self._f32(H, self.kk_cap, D), self._f32(H, self.kk_cap, D)
+        ws, nb = self._args_ws()
+        check("ac_key_bounds", self.lib.ac_key_bounds(self._ctx, ptr(k), ptr(k_assign), ptr(nk), ptr(kmax),
+                                                      ptr(kmin), ws, nb, stream_ptr(stream)))
+        return kmax, kmin
 
     def ac_cluster_sort(self, assign, cap, ncl=None, stream=None):
         H, N = self.cfg.heads, self.cfg.n

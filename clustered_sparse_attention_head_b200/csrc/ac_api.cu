@@ -61,7 +61,7 @@ struct Ws {
     // attention
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
-    size_t chi, clo, xu, amb_cand, items_scr, runs, run_info, masks;
+    size_t chi, clo, xu, amb_cand, items_scr, runs, run_info, masks, kbmax, kbmin;
     int kpad;
     size_t total;
 };
@@ -124,6 +124,9 @@ Ws layout(const ac_ctx *c) {
     w.runs = b.take(H * (size_t)c->kq_cap * c->kk_cap * 8);
     w.run_info = b.take(H * (size_t)c->kq_cap * 8);
     w.masks = b.take(H * (size_t)c->kq_cap * attn_max_chunks(c->cfg.n, c->kk_cap) * 4);
+    const bool quest = c->cfg.score_mode == AC_SCORE_QUEST;
+    w.kbmax = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
+    w.kbmin = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
     w.total = b.off;
     return w;
 }
@@ -322,6 +325,8 @@ ac_status validate(const ac_config *g) {
     if (g->dtype != AC_F32 && g->dtype != AC_BF16) return AC_ERR_INVALID_ARG;
     if (g->kq < 1 || g->kk < 1 || g->kq > g->n || g->kk > g->n) return AC_ERR_INVALID_ARG;
     if (!(g->top_p > 0.0)) return AC_ERR_INVALID_ARG;
+    if (g->score_mode != AC_SCORE_CENTROID && g->score_mode != AC_SCORE_QUEST) return AC_ERR_INVALID_ARG;
+    if (g->top_k < 0) return AC_ERR_INVALID_ARG;
     if ((long long)g->heads * g->n > 0x7fffffffLL / 2) return AC_ERR_UNSUPPORTED;
     if (g->adaptive_q && g->nmax_q < 1) return AC_ERR_INVALID_ARG;
     if (g->adaptive_k && g->nmax_k < 1) return AC_ERR_INVALID_ARG;
@@ -329,6 +334,23 @@ ac_status validate(const ac_config *g) {
         (g->tau_rule < AC_TAU_ABS || g->tau_rule > AC_TAU_MEDIAN_RADIUS_X || !(g->tau_value >= 0.0)))
         return AC_ERR_INVALID_ARG;
     return AC_OK;
+}
+}  // namespace
+
+namespace {
+// Sort the keys by cluster (into the workspace's key permutation and offsets)
+// and take each cluster's per-dimension max / min.
+void key_bounds(ac_ctx *c, const void *k, const int32_t *ka, const int32_t *nk, float *kmax, float *kmin, void *ws,
+                cudaStream_t st) {
+    const ac_config &g = c->cfg;
+    Ws w = layout(c);
+    HeadSeg *sk = at<HeadSeg>(ws, w.segk);
+    int32_t *kperm = at<int32_t>(ws, w.kperm), *koff = at<int32_t>(ws, w.koff);
+    k_seg_from_counts(g.heads, g.n, nk, g.kk, sk, st);
+    k_sort(ka, nullptr, sk, g.heads, g.n, g.n, c->kk_cap, at<int32_t>(ws, w.rank), at<int32_t>(ws, w.hist),
+           at<int32_t>(ws, w.cnt2), koff, kperm, c->d_status, st);
+    k_cluster_bounds(k, g.dtype == AC_BF16 ? DT_BF16 : DT_F32, g.heads, g.n, g.d, kperm, koff, c->kk_cap, kmax, kmin,
+                     st);
 }
 }  // namespace
 
@@ -487,16 +509,27 @@ ac_status ac_cluster_k(ac_ctx *c, const void *k, const float *init_cent, int32_t
 }
 
 ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, const int32_t *q_count,
-                    const float *k_cent, const int32_t *k_count, const int32_t *nq, const int32_t *nk,
-                    const uint8_t *dense_flag, int32_t *sel_idx, int32_t *sel_cnt, void *ws, size_t ws_bytes,
-                    void *stream) {
+                    const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min,
+                    const int32_t *nq, const int32_t *nk, const uint8_t *dense_flag, int32_t *sel_idx,
+                    int32_t *sel_cnt, void *ws, size_t ws_bytes, void *stream) {
     if (!c || !q_cent || !q_mean_norm || !q_count || !k_cent || !k_count || !sel_idx || !sel_cnt)
         return AC_ERR_INVALID_ARG;
+    const ac_config &g = c->cfg;
+    if (g.score_mode == AC_SCORE_QUEST && (!k_max || !k_min)) return AC_ERR_INVALID_ARG;
     ac_status s = check_ws(c, ws, ws_bytes);
     if (s != AC_OK) return s;
-    const ac_config &g = c->cfg;
-    k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, c->kk_cap, nq, nk, g.kq, g.kk,
-             dense_flag, g.top_p, sel_idx, sel_cnt, (cudaStream_t)stream);
+    k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, k_max, k_min, c->kk_cap, nq, nk,
+             g.kq, g.kk, dense_flag, (int)g.score_mode, g.top_k, g.top_p, sel_idx, sel_cnt, (cudaStream_t)stream);
+    return launch_check();
+}
+
+
+ac_status ac_key_bounds(ac_ctx *c, const void *k, const int32_t *k_assign, const int32_t *nk, float *k_max,
+                        float *k_min, void *ws, size_t ws_bytes, void *stream) {
+    if (!c || !k || !k_assign || !k_max || !k_min) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    key_bounds(c, k, k_assign, nk, k_max, k_min, ws, (cudaStream_t)stream);
     return launch_check();
 }
 
@@ -568,8 +601,14 @@ ac_status ac_forward(ac_ctx *c, const void *q, const void *k, const void *v, flo
     // a head is dense when either clustering set its flag F
     uint8_t *dense = dk;
     if (g.adaptive_q) ac_or_flags(g.heads, dq, dk, st);
-    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, c->kk_cap, nq, nk, g.kq, g.kk, dense, g.top_p, sel, selc,
-             st);
+    float *kbmax = nullptr, *kbmin = nullptr;
+    if (g.score_mode == AC_SCORE_QUEST) {
+        kbmax = at<float>(ws, w.kbmax);
+        kbmin = at<float>(ws, w.kbmin);
+        key_bounds(c, k, ka, nk, kbmax, kbmin, ws, st);
+    }
+    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk, dense,
+             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st);
     if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
     s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),

@@ -1,8 +1,10 @@
-// Critical-cluster selection (AdaCluster, Algorithm 3 lines 6-7, with the
-// centroid-based significance estimate of §2.3): for a query cluster a, key
-// cluster b is scored by its centroid against a's centroid, weighted by b's
-// size, and the smallest set of key clusters holding a top_p share of the
-// estimated attention mass is kept.
+// Critical-cluster selection (AdaCluster, Algorithm 3 lines 6-7): for a query
+// cluster a, key cluster b is scored either by its centroid against a's
+// centroid (the centroid-based significance estimate of §2.3) or by Quest's
+// page bound (§3.2.3 eq. (1), in TensorQuest's form of eq. (2)).  Then either
+// the top_k best-scored clusters are kept (Algorithm 3's argtopk), or, with
+// scores weighted by b's size, the smallest set holding a top_p share of the
+// estimated attention mass.
 //
 // One CTA per (query cluster, head).  Scores, weights and the running mass are
 // double, evaluated in the order of a plain sequential loop (scores per b
@@ -15,9 +17,10 @@ namespace ac {
 
 __global__ void select_kernel(int D, const float *__restrict__ q_cent, const float *__restrict__ q_mean_norm,
                               const int32_t *__restrict__ q_count, int kq_cap, const float *__restrict__ k_cent,
-                              const int32_t *__restrict__ k_count, int kk_cap, const int32_t *__restrict__ nq,
+                              const int32_t *__restrict__ k_count, const float *__restrict__ k_max,
+                              const float *__restrict__ k_min, int kk_cap, const int32_t *__restrict__ nq,
                               const int32_t *__restrict__ nk, int kq_fixed, int kk_fixed,
-                              const uint8_t *__restrict__ dense, double top_p, int n2,
+                              const uint8_t *__restrict__ dense, int score_mode, int top_k, double top_p, int n2,
                               int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_cnt) {
     extern __shared__ __align__(16) unsigned char smraw[];
     double *sp = reinterpret_cast<double *>(smraw);          // [n2] p (sort key)
@@ -25,6 +28,7 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
     double *sw = reinterpret_cast<double *>(sb + n2);        // [kk_cap] weights
     unsigned char *keep = reinterpret_cast<unsigned char *>(sw + kk_cap);  // [kk_cap]
     __shared__ double mu[128];
+    __shared__ double qpos[128], qneg[128];
     __shared__ double red[32];
     __shared__ int ired[33];
     __shared__ double sW;
@@ -40,9 +44,17 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
     }
     const float *kc = k_cent + (size_t)h * kk_cap * D;
     const int32_t *kn = k_count + (size_t)h * kk_cap;
-    for (int t = tid; t < D; t += nt) mu[t] = (double)q_cent[((size_t)h * kq_cap + a) * D + t];
     const double rbar = (double)q_mean_norm[(size_t)h * kq_cap + a];
+    for (int t = tid; t < D; t += nt) {
+        mu[t] = (double)q_cent[((size_t)h * kq_cap + a) * D + t];
+        // TensorQuest split of the representative query qbar = rbar * mu
+        const double qb = dmul(rbar, mu[t]);
+        qpos[t] = qb > 0.0 ? qb : 0.0;
+        qneg[t] = qb < 0.0 ? qb : 0.0;
+    }
     const double scale = 1.0 / sqrt((double)D);
+    const float *kmx = k_max ? k_max + (size_t)h * kk_cap * D : nullptr;
+    const float *kmn = k_min ? k_min + (size_t)h * kk_cap * D : nullptr;
     __syncthreads();
 
     // scores and their maximum over non-empty key clusters
@@ -50,10 +62,20 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
     for (int b = tid; b < nkh; b += nt) {
         double s = -INFINITY;
         if (kn[b] > 0) {
-            const float *c = kc + (size_t)b * D;
-            double dot = 0.0;
-            for (int t = 0; t < D; t++) dot = dadd(dot, dmul(mu[t], (double)c[t]));
-            s = dmul(dmul(rbar, dot), scale);
+            if (score_mode == 1) {
+                // qbar+ . M_b + qbar- . m_b, summed per dimension: each term
+                // equals max(qbar_t M_bt, qbar_t m_bt) of eq. (1) exactly
+                const float *M = kmx + (size_t)b * D, *mn = kmn + (size_t)b * D;
+                double acc = 0.0;
+                for (int t = 0; t < D; t++)
+                    acc = dadd(acc, dadd(dmul(qpos[t], (double)M[t]), dmul(qneg[t], (double)mn[t])));
+                s = dmul(acc, scale);
+            } else {
+                const float *c = kc + (size_t)b * D;
+                double dot = 0.0;
+                for (int t = 0; t < D; t++) dot = dadd(dot, dmul(mu[t], (double)c[t]));
+                s = dmul(dmul(rbar, dot), scale);
+            }
             m = fmax(m, s);
         }
         sw[b] = s;
@@ -68,25 +90,34 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
     }
     __syncthreads();
     m = red[0];
-    for (int b = tid; b < nkh; b += nt) {
-        if (kn[b] > 0) sw[b] = dmul((double)kn[b], exp(dsub(sw[b], m)));
-    }
-    __syncthreads();
-    if (tid == 0) {
-        double W = 0.0;
-        for (int b = 0; b < nkh; b++)
-            if (kn[b] > 0) W = dadd(W, sw[b]);
-        sW = W;
-    }
-    __syncthreads();
-    const double W = sW;
-    for (int i = tid; i < n2; i += nt) {
-        if (i < nkh && kn[i] > 0) {
-            sp[i] = ddiv(sw[i], W);
-            sb[i] = i;
-        } else {
-            sp[i] = -1.0;
-            sb[i] = 0x7fffffff;
+    if (top_k > 0) {
+        // argtopk: sort by the score itself
+        for (int i = tid; i < n2; i += nt) {
+            const bool live = i < nkh && kn[i] > 0;
+            sp[i] = live ? sw[i] : -INFINITY;
+            sb[i] = live ? i : 0x7fffffff;
+        }
+    } else {
+        for (int b = tid; b < nkh; b += nt) {
+            if (kn[b] > 0) sw[b] = dmul((double)kn[b], exp(dsub(sw[b], m)));
+        }
+        __syncthreads();
+        if (tid == 0) {
+            double W = 0.0;
+            for (int b = 0; b < nkh; b++)
+                if (kn[b] > 0) W = dadd(W, sw[b]);
+            sW = W;
+        }
+        __syncthreads();
+        const double W = sW;
+        for (int i = tid; i < n2; i += nt) {
+            if (i < nkh && kn[i] > 0) {
+                sp[i] = ddiv(sw[i], W);
+                sb[i] = i;
+            } else {
+                sp[i] = -1.0;
+                sb[i] = 0x7fffffff;
+            }
         }
     }
     for (int b = tid; b < kk_cap; b += nt) keep[b] = 0;
@@ -114,7 +145,9 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
         double cum = 0.0;
         for (int r = 0; r < n2; r++) {
             if (sb[r] == 0x7fffffff) break;
+            if (top_k > 0 && r >= top_k) break;
             keep[sb[r]] = 1;
+            if (top_k > 0) continue;
             cum = dadd(cum, sp[r]);
             if (top_p < 1.0 && cum >= top_p) break;
         }
@@ -145,9 +178,9 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
 }
 
 void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const int32_t *q_count, int kq_cap,
-              const float *k_cent, const int32_t *k_count, int kk_cap, const int32_t *nq, const int32_t *nk,
-              int kq_fixed, int kk_fixed, const uint8_t *dense, double top_p, int32_t *sel_idx, int32_t *sel_cnt,
-              cudaStream_t st) {
+              const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min, int kk_cap,
+              const int32_t *nq, const int32_t *nk, int kq_fixed, int kk_fixed, const uint8_t *dense, int score_mode,
+              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st) {
     int n2 = 1;
     while (n2 < kk_cap) n2 <<= 1;
     size_t smem = (size_t)n2 * (sizeof(double) + sizeof(int)) + (size_t)kk_cap * (sizeof(double) + 1);
@@ -157,8 +190,42 @@ void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const
         smem_set = smem;
     }
     dim3 g(kq_cap, H);
-    select_kernel<<<g, 256, smem, st>>>(D, q_cent, q_mean_norm, q_count, kq_cap, k_cent, k_count, kk_cap, nq, nk,
-                                        kq_fixed, kk_fixed, dense, top_p, n2, sel_idx, sel_cnt); note_launch();
+    select_kernel<<<g, 256, smem, st>>>(D, q_cent, q_mean_norm, q_count, kq_cap, k_cent, k_count, k_max, k_min,
+                                        kk_cap, nq, nk, kq_fixed, kk_fixed, dense, score_mode, top_k, top_p, n2,
+                                        sel_idx, sel_cnt);
+    note_launch();
+}
+
+// Quest page bounds: one CTA per (cluster, head), one thread per dimension,
+// walking the cluster's members in the cluster-sorted order (coalesced rows).
+template <typename T>
+__global__ void cluster_bounds_kernel(const T *__restrict__ x, int N, int D, const int32_t *__restrict__ perm,
+                                      const int32_t *__restrict__ off, int cap, float *__restrict__ xmax,
+                                      float *__restrict__ xmin) {
+    const int h = blockIdx.y, b = blockIdx.x;
+    const int32_t *o = off + (size_t)h * (cap + 1);
+    const int i0 = o[b], i1 = o[b + 1];
+    for (int t = threadIdx.x; t < D; t += blockDim.x) {
+        float mx = 0.f, mn = 0.f;
+        for (int i = i0; i < i1; i++) {
+            const float v = to_f(x[((size_t)h * N + perm[(size_t)h * N + i]) * D + t]);
+            mx = i == i0 ? v : fmaxf(mx, v);
+            mn = i == i0 ? v : fminf(mn, v);
+        }
+        xmax[((size_t)h * cap + b) * D + t] = mx;
+        xmin[((size_t)h * cap + b) * D + t] = mn;
+    }
+}
+
+void k_cluster_bounds(const void *x, int dtype, int H, int N, int D, const int32_t *perm, const int32_t *off,
+                      int cap, float *xmax, float *xmin, cudaStream_t st) {
+    dim3 g(cap, H);
+    if (dtype == DT_BF16)
+        cluster_bounds_kernel<__nv_bfloat16><<<g, D, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), N, D, perm, off,
+                                                             cap, xmax, xmin);
+    else
+        cluster_bounds_kernel<float><<<g, D, 0, st>>>(static_cast<const float *>(x), N, D, perm, off, cap, xmax, xmin);
+    note_launch();
 }
 
 }  // namespace ac

@@ -72,6 +72,17 @@ typedef enum { AC_F32 = 0, AC_BF16 = 1 } ac_dtype;
  * first-stage clusters, of the mean member-to-centre distance.              */
 typedef enum { AC_TAU_ABS = 0, AC_TAU_MEAN_X = 1, AC_TAU_MEDIAN_RADIUS_X = 2 } ac_tau_rule;
 
+/* How key clusters are scored for selection (ac_select, ac_forward).
+ * CENTROID: s_ab = mean_norm_a * (mu_a . c_b) / sqrt(d), the centroid-centroid
+ *   estimate of §2.3 (the default).
+ * QUEST: the page bound of §3.2.3 eq. (1) for the representative query
+ *   qbar = mean_norm_a * mu_a against key cluster b,
+ *   s_ab = sum_t max(qbar_t M_bt, qbar_t m_bt) / sqrt(d),
+ *   with M_b / m_b the per-dimension max / min of the keys of b (ac_key_bounds);
+ *   evaluated as TensorQuest's eq. (2), qbar+ . M_b + qbar- . m_b with
+ *   qbar+ = max(qbar, 0) and qbar- = min(qbar, 0), which gives the same value. */
+typedef enum { AC_SCORE_CENTROID = 0, AC_SCORE_QUEST = 1 } ac_score_mode;
+
 /* ac_config.flags */
 #define AC_FLAG_WARM_START 1u    /* ac_forward: seed k-means from q_cent_io/k_cent_io */
 #define AC_FLAG_CHECK_FINITE 2u  /* scan inputs for NaN/Inf (AC_ERR_NONFINITE)        */
@@ -90,6 +101,9 @@ typedef struct {
     int nmax_q, nmax_k;     /* Algorithm 1's N_max for queries / keys                  */
     double top_p;           /* (0, 1]; >= 1 keeps every non-empty key cluster          */
     unsigned flags;
+    ac_score_mode score_mode;  /* selection score (zero-initialised: CENTROID)          */
+    int top_k;              /* > 0: keep the top_k best-scored key clusters (Algorithm 3
+                               line 7, argtopk) instead of the top-p prefix            */
 } ac_config;
 
 /* Per-call statistics filled by ac_forward when `stats` is non-NULL (the call
@@ -147,17 +161,28 @@ AC_API ac_status ac_cluster_k(ac_ctx *ctx, const void *k, const float *init_cent
                        void *ws, size_t ws_bytes, void *stream);
 
 /* Critical-cluster selection.  For each non-empty query cluster a of a head
- * whose dense_flag is 0:
- *   s_ab = mean_norm_a * (mu_a . c_b) / sqrt(d)  over non-empty key clusters b,
- *   p_ab = count_b exp(s_ab - max_b s_ab) / sum_b (...),
- * then key clusters are taken in decreasing p (ties: lower b) until the taken
- * mass reaches top_p.  sel_idx lists them in ascending id.  Empty query
- * clusters and dense heads get sel_cnt = 0.  nq/nk/dense_flag may be NULL
- * (then kq/kk and 0 are used).                                              */
+ * whose dense_flag is 0, every non-empty key cluster b gets the score s_ab of
+ * config.score_mode (see ac_score_mode).  Then
+ *   top_k > 0: the top_k key clusters of largest s_ab are kept (ties: lower b);
+ *   else: p_ab = count_b exp(s_ab - max_b s_ab) / sum_b (...), and key clusters
+ *     are taken in decreasing p (ties: lower b) until the taken mass reaches top_p.
+ * sel_idx lists the kept clusters in ascending id.  Empty query clusters and
+ * dense heads get sel_cnt = 0.  nq/nk/dense_flag may be NULL (then kq/kk and 0
+ * are used).  k_max/k_min [H, kk_cap, d] (from ac_key_bounds) are read only,
+ * and required only, with AC_SCORE_QUEST.                                    */
 AC_API ac_status ac_select(ac_ctx *ctx, const float *q_cent, const float *q_mean_norm,
                     const int32_t *q_count, const float *k_cent, const int32_t *k_count,
+                    const float *k_max, const float *k_min,
                     const int32_t *nq, const int32_t *nk, const uint8_t *dense_flag,
                     int32_t *sel_idx, int32_t *sel_cnt, void *ws, size_t ws_bytes, void *stream);
+
+/* Quest page bounds of the key clusters (§3.2.3 eq. (1)): k_max / k_min
+ * [H, kk_cap, d] receive, per cluster and dimension, the largest / smallest
+ * key value over the cluster's members (0 for clusters without members).
+ * k [H, N, d] in the configured dtype, k_assign [H, N]; nk may be NULL (then kk).
+ * The values are exact (a max / min of the inputs, widened to fp32).         */
+AC_API ac_status ac_key_bounds(ac_ctx *ctx, const void *k, const int32_t *k_assign, const int32_t *nk,
+                               float *k_max, float *k_min, void *ws, size_t ws_bytes, void *stream);
 
 /* Stable counting sort of token ids by cluster id (per head): perm [H, N]
  * lists tokens of cluster 0 in increasing token order, then cluster 1, ...;
@@ -204,7 +229,7 @@ AC_API ac_status ac_sparse_attn(ac_ctx *ctx, const void *q, const void *k, const
                          size_t ws_bytes, void *stream);
 
 /* The whole of Algorithm 3 for every head: ac_cluster_q, ac_cluster_k,
- * ac_select, ac_sparse_attn.  q_cent_io / k_cent_io ([H, cap, d], nullable):
+ * (ac_key_bounds with AC_SCORE_QUEST), ac_select, ac_sparse_attn.  q_cent_io / k_cent_io ([H, cap, d], nullable):
  * with AC_FLAG_WARM_START they seed k-means (§3.2.2 "Efficient
  * initialization"); when non-NULL they receive the final centroids.
  * Adaptive clustering reads one int per head back to the host per stage; the

@@ -285,3 +285,77 @@ def test_forward_adaptive_dense_head(orc):
     for h in range(w.heads):
         ref = orc.attention_rows(q[h], k[h], v[h], None, None, 0, None, None, 1, rows)
         attn_close(got[h][rows], ref, f"adaptive-dense/h{h}")
+
+
+# --------------------------------------------------------------------------
+# Quest page bounds, the Quest score and the argtopk cut
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["f32-d64", "bf16-d128-ragged"])
+def test_key_bounds_bit_exact(orc, name):
+    """Per key cluster and dimension max / min of the keys: exact."""
+    w = _case(name)
+    q, k, v = stack_heads(w)
+    cl = _oracle_clusters(orc, w, q, k)
+    ctx = _ctx(w)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(np.stack(a))).cuda()
+    kmax, kmin = ctx.ac_key_bounds(to_dev(k, w.dtype), t([c[2].assign for c in cl]))
+    torch.cuda.synchronize()
+    assert ctx.get_status() == 0
+    for h, (_, _, rk) in enumerate(cl):
+        emax, emin = orc.key_bounds(k[h], rk.assign, w.kk)
+        np.testing.assert_array_equal(kmax[h, :w.kk].cpu().numpy(), emax)
+        np.testing.assert_array_equal(kmin[h, :w.kk].cpu().numpy(), emin)
+
+
+SELECT_MODES = [
+    # (score mode, top_k, top_p)
+    (1, 0, 0.9),     # Quest score, top-p
+    (1, 8, 0.9),     # Quest score, argtopk
+    (0, 8, 0.9),     # centroid score, argtopk
+    (1, 10000, 0.9), # argtopk with k above every cluster count
+]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("mode,top_k,top_p", SELECT_MODES)
+def test_select_modes_from_oracle_clusters(orc, name, mode, top_k, top_p):
+    """Selected sets bit-exact against the oracle for the Quest score (as
+    TensorQuest's eq. (2) on the GPU, eq. (1) in the oracle) and argtopk."""
+    w = _case(name)
+    q, k, v = stack_heads(w)
+    cl = _oracle_clusters(orc, w, q, k)
+    ctx = _ctx(w, score_mode=mode, top_k=top_k, top_p=top_p)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(np.stack(a))).cuda()
+    bounds = [orc.key_bounds(k[h], rk.assign, w.kk) for h, (_, _, rk) in enumerate(cl)]
+    sel, cnt = ctx.ac_select(t([c[0].cent for c in cl]), t([c[1] for c in cl]), t([c[0].count for c in cl]),
+                             t([c[2].cent for c in cl]), t([c[2].count for c in cl]),
+                             k_max=t([b[0] for b in bounds]), k_min=t([b[1] for b in bounds]))
+    torch.cuda.synchronize()
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for h, (rq, qmn, rk) in enumerate(cl):
+        s, c = orc.select2(rq.cent, qmn, rq.count, rk.cent, rk.count, top_p, mode, top_k, bounds[h][0], bounds[h][1])
+        np.testing.assert_array_equal(cnt[h], c)
+        for a in range(w.kq):
+            np.testing.assert_array_equal(sel[h, a, :c[a]], s[a, :c[a]])
+        if top_k:
+            assert (c <= top_k).all()
+
+
+def test_forward_quest_topk_end_to_end(orc):
+    """ac_forward with the Quest score and argtopk (Algorithm 3 as the pages
+    write it, with cluster-level pages) against the oracle's Algorithm 3."""
+    w = W.small(W.WORKLOADS["wan21-n75600-h40-d128"], 2777, heads=2, seed=6, kq=23, kk=41)
+    q, k, v = stack_heads(w)
+    ctx = _ctx(w, score_mode=1, top_k=12)
+    out, st = ctx.ac_forward(to_dev(q, w.dtype), to_dev(k, w.dtype), to_dev(v, w.dtype), stats=True)
+    torch.cuda.synchronize()
+    assert ctx.get_status() == 0
+    spec = orc.HeadSpec(kq=w.kq, kk=w.kk, iters=w.iters, top_p=w.top_p, score_mode=1, top_k=12)
+    pairs = 0
+    got = out.float().cpu().numpy()
+    for h in range(w.heads):
+        r = orc.forward_head(q[h], k[h], v[h], spec)
+        assert (r.sel_cnt <= 12).all()
+        attn_close(got[h], r.out_rows, f"forward/quest-top12/h{h}")
+        pairs += orc.pairs(r.q.count, r.k.count, r.sel_idx, r.sel_cnt)
+    assert st["pairs"] == pairs
