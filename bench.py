@@ -315,6 +315,24 @@ def main():
         dms = d0.elapsed_time(d1) / 3
         dense = {"impl": "torch.nn.functional.scaled_dot_product_attention", "ms": dms,
                  "tflops": w.dense_flops() / (dms * 1e-3) / 1e12, "speedup_of_clustered_call": dms / ms}
+        # the library's own dense path (Algorithm 3 line 4): every head flagged
+        # dense, so the attention kernel takes all N keys of each head
+        cq, ck = ac.ac_cluster_q(q), ac.ac_cluster_k(k)
+        dflag = torch.ones(w.heads, dtype=torch.uint8, device=dev)
+        sel0 = torch.zeros(w.heads, ac.kq_cap, ac.kk_cap, dtype=torch.int32, device=dev)
+        cnt0 = torch.zeros(w.heads, ac.kq_cap, dtype=torch.int32, device=dev)
+        args = (q, k, v, cq["assign"], ck["assign"], sel0, cnt0)
+        for _ in range(2):
+            ac.ac_sparse_attn(*args, dense_flag=dflag, out=out)
+        torch.cuda.synchronize(dev)
+        d0.record(stream)
+        for _ in range(3):
+            ac.ac_sparse_attn(*args, dense_flag=dflag, out=out)
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        oms = d0.elapsed_time(d1) / 3
+        dense["own_dense"] = {"impl": "ac_sparse_attn with every head dense (gathered copy + attn2_kernel)",
+                              "ms": oms, "tflops": w.dense_flops() / (oms * 1e-3) / 1e12}
 
     peaks = {}
     try:
