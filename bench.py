@@ -30,6 +30,9 @@ from clustered_sparse_attention_head_b200 import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "wan21-n75600-h40-d128"
 METRIC = "clustered sparse-attn calls/s & achieved TFLOPS at 75.6K tokens vs dense attn"
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch (ncu) on
+# the default workload cut to 8 heads; None when the kernel changed since
+ATTN_TRAFFIC_8H = None
 
 
 def parse():
@@ -331,7 +334,7 @@ def main():
         d1.record(stream)
         torch.cuda.synchronize(dev)
         oms = d0.elapsed_time(d1) / 3
-        dense["own_dense"] = {"impl": "ac_sparse_attn with every head dense (gathered copy + attn2_kernel)",
+        dense["own_dense"] = {"impl": "ac_sparse_attn with every head dense (gathered copy + attn3_kernel)",
                               "ms": oms, "tflops": w.dense_flops() / (oms * 1e-3) / 1e12}
 
     peaks = {}
@@ -342,12 +345,12 @@ def main():
     peak = peaks.get("bf16_tflops_sustained") or 1390.6
     peak_src = "measured (MEASURED_PEAKS.json bf16_tflops_sustained)" if peaks else "fallback"
     # DRAM bytes of one attention launch, from an ncu capture of this kernel
-    # on the Wan-shaped workload cut to 8 heads (2.571 GB read + 0.146 GB
-    # written), scaled by heads; only for that workload and kernel version
+    # version on the Wan-shaped workload cut to 8 heads, scaled by heads; only
+    # for that workload (None until such a capture exists)
     traffic = None
-    if w.name == DEFAULT_WORKLOAD and w.top_p == 0.9:
-        traffic = 2.717e9 * w.heads / 8
-    roof = {"kernel": "attn2_kernel (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": tflops_attn,
+    if w.name == DEFAULT_WORKLOAD and w.top_p == 0.9 and ATTN_TRAFFIC_8H:
+        traffic = ATTN_TRAFFIC_8H * w.heads / 8
+    roof = {"kernel": "attn3_kernel (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": tflops_attn,
             "peak": peak, "unit": "TFLOP/s", "frac": tflops_attn / peak, "traffic": traffic,
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, 8-head capture scaled by heads"
             if traffic else None,

@@ -123,7 +123,7 @@ Ws layout(const ac_ctx *c) {
     w.items_scr = b.take(items_scratch_elems((int)H, c->kq_cap) * 4 + 16);
     w.runs = b.take(H * (size_t)c->kq_cap * c->kk_cap * 8);
     w.run_info = b.take(H * (size_t)c->kq_cap * 8);
-    w.masks = b.take(H * (size_t)c->kq_cap * attn_max_chunks(c->cfg.n, c->kk_cap) * 4);
+    w.masks = b.take(H * (size_t)c->kq_cap * attn_max_chunks(c->cfg.n, c->kk_cap, ATTN3_CHUNK) * (ATTN3_CHUNK / 64) * 4);
     const bool quest = c->cfg.score_mode == AC_SCORE_QUEST;
     w.kbmax = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
     w.kbmin = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
@@ -300,16 +300,16 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     k_build_items(H, N, two_tiles ? 256 : 128, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items,
                   nitems, pairs_dev, at<int32_t>(ws, w.items_scr), st);
     int2 *runs = at<int2>(ws, w.runs), *run_info = at<int2>(ws, w.run_info);
-    k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN2_CHUNK, runs, run_info, st);
-    const int max_chunks = attn_max_chunks(N, c->kk_cap);
+    k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN3_CHUNK, runs, run_info, st);
+    const int max_chunks = attn_max_chunks(N, c->kk_cap, ATTN3_CHUNK);
     uint32_t *masks = at<uint32_t>(ws, w.masks);
     if (two_tiles) k_chunk_masks(H, c->kq_cap, c->kk_cap, max_chunks, runs, run_info, masks, st);
     if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
     int rc;
     if (two_tiles)
-        rc = k_attention2(D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, masks, max_chunks, items,
-                          nitems,
-                          attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
+        rc = k_attention3(D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, masks, max_chunks, items,
+                          nitems, attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn,
+                          st);
     else
         rc = k_attention(DT_F32, D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, items, nitems,
                          attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);

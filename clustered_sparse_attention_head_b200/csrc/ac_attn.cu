@@ -566,7 +566,8 @@ __global__ void items_base_kernel(int H, const int32_t *__restrict__ head_tiles,
         base += head_tiles[h];
         pr += head_pairs[h];
     }
-    *n_items = base;
+    n_items[0] = base;
+    n_items[1] = 0;  // work counter of the dynamically scheduled attention kernel
     if (pairs) *pairs = (int64_t)pr;
 }
 
@@ -700,8 +701,9 @@ void k_key_runs(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_
 }
 
 // Chunk masks of every (head, query cluster): for chunk c of the key stream
-// (chunk_rows keys as KeyStream packs the runs) the number of valid rows in
-// each of its 8-row groups, 4 bits per group (chunk_rows = 64: 8 groups).  Run
+// (CH keys as KeyStream packs the runs) the number of valid rows in each of
+// its 8-row groups, 4 bits per group, eight groups per 32-bit word (CH / 64
+// words per chunk, group g in word g / 8).  Run
 // r occupies stream positions [S_r, S_r + round8(len_r)) with S_r the prefix
 // sum of the rounded lengths, and its first len_r positions hold keys (a run
 // split at a chunk boundary is split at a multiple of 8, so this holds for
@@ -709,8 +711,10 @@ void k_key_runs(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_
 // each thread fills chunks with a binary search per group.
 constexpr int kMaskMaxRuns = 8192;
 
+template <int CH>
 __global__ void chunk_masks_kernel(int kq_cap, int kk_cap, int max_chunks, const int2 *__restrict__ runs,
                                    const int2 *__restrict__ info, uint32_t *__restrict__ masks) {
+    constexpr int W = CH / 64;
     __shared__ int s_start[kMaskMaxRuns];
     __shared__ int wsum[32];
     const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
@@ -749,12 +753,12 @@ __global__ void chunk_masks_kernel(int kq_cap, int kk_cap, int max_chunks, const
         carry += wsum[nt / 32 - 1];
         __syncthreads();
     }
-    uint32_t *out = masks + qa * max_chunks;
-    for (int c = tid; c < nch; c += nt) {
+    uint32_t *out = masks + qa * max_chunks * W;
+    for (int cw = tid; cw < nch * W; cw += nt) {
         uint32_t gm = 0;
 #pragma unroll 1
         for (int g = 0; g < 8; g++) {
-            const int pos = c * 64 + 8 * g;
+            const int pos = cw * 64 + 8 * g;
             // last run with S_r <= pos
             int lo = 0, hi = nr - 1, r = -1;
             while (lo <= hi) {
@@ -768,15 +772,15 @@ __global__ void chunk_masks_kernel(int kq_cap, int kk_cap, int max_chunks, const
                 gm |= (uint32_t)(left <= 0 ? 0 : (left >= 8 ? 8 : left)) << (4 * g);
             }
         }
-        out[c] = gm;
+        out[cw] = gm;
     }
 }
 
-int attn_max_chunks(int N, int kk_cap) { return (N + 7 * kk_cap + 63) / 64 + 1; }
+int attn_max_chunks(int N, int kk_cap, int chunk) { return (N + 7 * kk_cap + chunk - 1) / chunk + 1; }
 
 void k_chunk_masks(int H, int kq_cap, int kk_cap, int max_chunks, const int2 *runs, const int2 *info,
                    uint32_t *masks, cudaStream_t st) {
-    chunk_masks_kernel<<<dim3(kq_cap, H), 256, 0, st>>>(kq_cap, kk_cap, max_chunks, runs, info, masks);
+    chunk_masks_kernel<ATTN3_CHUNK><<<dim3(kq_cap, H), 256, 0, st>>>(kq_cap, kk_cap, max_chunks, runs, info, masks);
     note_launch();
 }
 

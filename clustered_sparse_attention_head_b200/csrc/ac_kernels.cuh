@@ -62,6 +62,7 @@ void k_cluster_bounds(const void *x, int dtype, int H, int N, int D, const int32
 struct AttnItem {
     int h, a, q_start, q_len;  // a < 0: dense head (all keys)
 };
+// n_items[0] = item count; n_items[1] = 0 (the bf16 attention kernel's work counter)
 void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
                    const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
@@ -75,18 +76,18 @@ int attn_max_items(int H, int N, int kq_cap);
 // packs them}.  Cluster ids outside [0, kk_cap) are skipped.
 void k_key_runs(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx, const int32_t *sel_cnt,
                 int chunk_rows, int2 *runs, int2 *info, cudaStream_t st);
-// Valid-row counts of every 64-key chunk (4 bits per 8-row group) of every
-// (head, query cluster) key stream: masks [H, kq_cap, max_chunks].
-int attn_max_chunks(int N, int kk_cap);
+// Valid-row counts of every chunk of ATTN3_CHUNK (128) keys (4 bits per 8-row
+// group, two 32-bit words per chunk) of every (head, query cluster) key
+// stream: masks [H, kq_cap, max_chunks, 2].
+int attn_max_chunks(int N, int kk_cap, int chunk);
 void k_chunk_masks(int H, int kq_cap, int kk_cap, int max_chunks, const int2 *runs, const int2 *info,
                    uint32_t *masks, cudaStream_t st);
-// bf16: two 128-row query tiles per CTA, 64-key chunks (ac_attn2.cu); items of up to 256 rows
-constexpr int ATTN2_CHUNK = 64;
-int k_attention2(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
+// bf16: two 128-row query tiles per CTA, 128-key chunks (ac_attn3.cu); items of up to 256 rows
+constexpr int ATTN3_CHUNK = 128;
+int k_attention3(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
                  int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const uint32_t *masks,
-                 int max_chunks, const AttnItem *items,
-                 const int32_t *n_items, int max_items, void *out, float *lse, int *status, int num_sms,
-                 void *encode_fn, cudaStream_t st);
+                 int max_chunks, const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse,
+                 int *status, int num_sms, void *encode_fn, cudaStream_t st);
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
                 const int32_t *qperm, int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info,
                 const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
