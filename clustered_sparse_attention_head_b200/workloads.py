@@ -149,6 +149,25 @@ def head_inputs(w: Workload, h: int) -> HeadInputs:
     return HeadInputs(np.ascontiguousarray(q), np.ascontiguousarray(k), np.ascontiguousarray(v), comp)
 
 
+def step_inputs(w: Workload, h: int, step: int, drift: float = 0.02) -> HeadInputs:
+    """Inputs of head h at denoising step `step`, standing in for consecutive
+    denoising steps, whose token distributions drift little.  Step 0 is
+    head_inputs(w, h); each later step adds drift * N(0, I) to the previous
+    step's q, k and v (one seeded stream per (workload seed, head, step)) and
+    rounds to bf16 again for bf16 workloads."""
+    base = head_inputs(w, h)
+    q, k, v = base.q, base.k, base.v
+    for s in range(1, step + 1):
+        r = np.random.default_rng([w.seed, h, s, 7919])
+        f = np.float32(drift)
+        q = q + f * r.standard_normal(q.shape, dtype=np.float32)
+        k = k + f * r.standard_normal(k.shape, dtype=np.float32)
+        v = v + f * r.standard_normal(v.shape, dtype=np.float32)
+        if w.dtype == "bf16":
+            q, k, v = (bf16_bits_to_f32(to_bf16_bits(a)) for a in (q, k, v))
+    return HeadInputs(np.ascontiguousarray(q), np.ascontiguousarray(k), np.ascontiguousarray(v), base.comp)
+
+
 def small(w: Workload, n: int, heads: int = 1, seed: int = 0, **over) -> Workload:
     """A reduced copy of workload w: n video tokens with iid mixture components
     and no text tokens, for tests that must finish in seconds."""

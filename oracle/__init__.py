@@ -336,7 +336,32 @@ def forward_head(q, k, v, spec: HeadSpec, rows=None):
     """Algorithm 3 for one head; attention is evaluated for `rows` (all if None)."""
     rq, qmn = cluster_q(q, spec)
     rk = cluster_k(k, spec)
-    dense = int(rq.dense or rk.dense)
+    return _select_attend(q, k, v, rq, rk, qmn, int(rq.dense or rk.dense), spec, rows)
+
+
+def forward_steps(steps, spec: HeadSpec, rows=None):
+    """One head over consecutive denoising steps (AdaCluster §3.2.2 "Efficient
+    initialization", §4.1): step 0 is forward_head (Algorithm 1 counts when the
+    spec is adaptive); every later step keeps step 0's cluster counts and dense
+    flag F and runs fixed-count k-means (spec.iters rounds) seeded with the
+    previous step's centres, then selection and attention as forward_head.
+    `steps` is a list of (q, k, v); returns one HeadResult per step."""
+    q0, k0, v0 = steps[0]
+    res = [forward_head(q0, k0, v0, spec, rows)]
+    nq, nk, dense = res[0].q.nclusters, res[0].k.nclusters, res[0].dense
+    for q, k, v in steps[1:]:
+        prev = res[-1]
+        xq, nrm = prepare(q, SPHERE)
+        rq = kmeans(xq, nq, spec.iters, SPHERE, init=prev.q.cent[:nq])
+        qmn = cluster_mean_norm(nrm, rq.assign, rq.nclusters)
+        xk, _ = prepare(k, EUCLID)
+        rk = kmeans(xk, nk, spec.iters, EUCLID, init=prev.k.cent[:nk])
+        res.append(_select_attend(q, k, v, rq, rk, qmn, dense, spec, rows))
+    return res
+
+
+def _select_attend(q, k, v, rq, rk, qmn, dense, spec: HeadSpec, rows):
+    """Algorithm 3 lines 6-9 for one head from its two clusterings."""
     if dense:
         sel = np.zeros((rq.nclusters, max(rk.nclusters, 1)), np.int32)
         cnt = np.zeros(rq.nclusters, np.int32)

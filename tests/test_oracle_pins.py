@@ -500,3 +500,112 @@ def test_quest_selects_a_page_with_an_aligned_outlier(orc):
     sel0, _ = orc.select2(mu, rbar, qc, c, kc, top_k=1)
     sel1, _ = orc.select2(mu, rbar, qc, c, kc, top_k=1, score_mode=orc.SCORE_QUEST, k_max=kmax, k_min=kmin)
     assert sel0[0, 0] == 1 and sel1[0, 0] == 0
+
+
+# --------------------------------------------------------------------------
+# Multi-step driver (§3.2.2 "Efficient initialization", §4.1): counts and F of
+# step 0 kept, k-means seeded with the previous step's centres
+# --------------------------------------------------------------------------
+def _drifting_gmm(steps, comps=6, per=40, d=16, drift=0.05, sep=12.0, seed=11):
+    """Per step (q, k, v) of `comps` well-separated components (q and k share
+    the component of a token); every step moves every point by drift * N(0, I).
+    Returns the steps and the true component of each token."""
+    rng = np.random.default_rng(seed)
+    lab = np.repeat(np.arange(comps), per)
+    mq = sep * rng.standard_normal((comps, d))
+    mk = sep * rng.standard_normal((comps, d))
+    q = mq[lab] + 0.2 * rng.standard_normal((len(lab), d))
+    k = mk[lab] + 0.2 * rng.standard_normal((len(lab), d))
+    v = rng.standard_normal((len(lab), d))
+    out = []
+    for _ in range(steps):
+        out.append((q.astype(np.float32), k.astype(np.float32), v.astype(np.float32)))
+        q = q + drift * rng.standard_normal(q.shape)
+        k = k + drift * rng.standard_normal(k.shape)
+        v = v + drift * rng.standard_normal(v.shape)
+    return out, lab
+
+
+def _same_partition(a, b):
+    """a and b split the tokens into the same groups (labels may differ)."""
+    pairs = set(zip(a.tolist(), b.tolist()))
+    return len(pairs) == len(set(a.tolist())) == len(set(b.tolist()))
+
+
+def test_steps_track_drifting_components(orc):
+    """Every step re-clusters its own inputs: the assignments stay the true
+    components while the points drift, and each key centre is the sample mean
+    of its component at that step (closed form), not step 0's centre."""
+    steps, lab = _drifting_gmm(4, drift=0.3)
+    spec = orc.HeadSpec(kq=6, kk=6, iters=5, top_p=0.9)
+    res = orc.forward_steps(steps, spec, rows=np.arange(0, len(lab), 7))
+    for s, r in enumerate(res):
+        assert _same_partition(r.q.assign, lab) and _same_partition(r.k.assign, lab), f"step {s}"
+        k = steps[s][1].astype(np.float64)
+        for c in range(6):
+            m = r.k.assign == c
+            np.testing.assert_allclose(r.k.cent[c], k[m].mean(0), rtol=1e-6, atol=1e-6)
+    assert not np.array_equal(res[0].k.cent, res[3].k.cent)
+
+
+def test_steps_fixed_point_without_drift(orc):
+    """No drift and converged centres: every later step reproduces step 0
+    exactly (assignments, centres, selection, output rows)."""
+    steps, lab = _drifting_gmm(1)
+    steps = steps * 3
+    spec = orc.HeadSpec(kq=6, kk=6, iters=6, top_p=0.8)
+    res = orc.forward_steps(steps, spec, rows=np.arange(0, len(lab), 5))
+    for r in res[1:]:
+        np.testing.assert_array_equal(r.q.assign, res[0].q.assign)
+        np.testing.assert_array_equal(r.k.assign, res[0].k.assign)
+        np.testing.assert_array_equal(r.q.cent, res[0].q.cent)
+        np.testing.assert_array_equal(r.k.cent, res[0].k.cent)
+        np.testing.assert_array_equal(r.sel_cnt, res[0].sel_cnt)
+        np.testing.assert_array_equal(r.out_rows, res[0].out_rows)
+
+
+def test_steps_keep_step0_counts(orc):
+    """Later steps keep the counts Algorithm 1 chose at step 0, even where
+    Algorithm 1 on that step's inputs would choose another count."""
+    steps, lab = _drifting_gmm(3, comps=4, per=50, drift=0.0)
+    # step 2: a fifth, far-away group appears among the tokens
+    q2, k2, v2 = (a.copy() for a in steps[2])
+    far = np.arange(0, len(lab), 4)
+    k2[far] += 60.0
+    q2[far] = -q2[far]
+    steps[2] = (q2, k2, v2)
+    spec = orc.HeadSpec(kq=4, kk=4, iters=4, top_p=0.9, adaptive_k=True, tau_rule=orc.TAU_ABS, tau_value=8.0,
+                        nmax_k=64)
+    res = orc.forward_steps(steps, spec, rows=np.arange(0, len(lab), 9))
+    xs2, _ = orc.prepare(k2, orc.EUCLID)
+    alone = orc.multistage(xs2, spec.kk, spec.iters, spec.tau_rule, spec.tau_value, spec.nmax_k, orc.EUCLID)
+    assert alone.nclusters != res[0].k.nclusters
+    assert [r.k.nclusters for r in res] == [res[0].k.nclusters] * 3
+    assert all(r.dense == res[0].dense for r in res)
+
+
+def test_steps_keep_dense_flag(orc):
+    """F set at step 0 (N_max reached) keeps every later step dense: the rows
+    are exact attention over all keys."""
+    w = W.small(W.WORKLOADS["gmm16-n2048-d64-f32"], 300)
+    steps = [(W.step_inputs(w, 0, s, drift=0.05).q, W.step_inputs(w, 0, s, drift=0.05).k,
+              W.step_inputs(w, 0, s, drift=0.05).v) for s in range(3)]
+    spec = orc.HeadSpec(kq=8, kk=16, iters=3, top_p=0.5, adaptive_k=True, tau_rule=orc.TAU_ABS,
+                        tau_value=0.0, nmax_k=16)
+    rows = np.arange(0, 300, 7)
+    res = orc.forward_steps(steps, spec, rows=rows)
+    for (q, k, v), r in zip(steps, res):
+        assert r.dense == 1
+        np.testing.assert_allclose(r.out_rows, _np_attention(q[rows], k, v), rtol=1e-10, atol=1e-12)
+
+
+def test_step_inputs_drift(orc):
+    """step_inputs: step 0 is head_inputs; step s differs from step s - 1 by
+    about drift * N(0, 1) per element (before bf16 rounding)."""
+    w = W.small(W.WORKLOADS["gmm16-n2048-d64-f32"], 256)
+    h0 = W.head_inputs(w, 0)
+    s0, s1, s2 = (W.step_inputs(w, 0, s, drift=0.1) for s in range(3))
+    np.testing.assert_array_equal(s0.q, h0.q)
+    d1, d2 = (s1.k - s0.k), (s2.k - s1.k)
+    assert abs(d1.std() - 0.1) < 0.01 and abs(d2.std() - 0.1) < 0.01
+    assert abs(np.corrcoef(d1.ravel(), d2.ravel())[0, 1]) < 0.05
