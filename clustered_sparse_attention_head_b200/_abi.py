@@ -23,8 +23,8 @@ AC_SCORE_CENTROID, AC_SCORE_QUEST = 0, 1
 
 # every entry point declared in include/adacluster.h
 EXPORTS = ["ac_create", "ac_destroy", "ac_capacities", "ac_workspace_size", "ac_cluster_q", "ac_cluster_k",
-           "ac_select", "ac_key_bounds", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_profile_read", "ac_get_status",
-           "ac_status_string"]
+           "ac_select", "ac_key_bounds", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_step_state_size", "ac_step_state_parts", "ac_forward_step",
+           "ac_profile_read", "ac_get_status", "ac_status_string"]
 
 
 class ac_config(ctypes.Structure):
@@ -37,7 +37,8 @@ class ac_config(ctypes.Structure):
 class ac_stats(ctypes.Structure):
     _fields_ = [("ms_cluster_q", c_double), ("ms_cluster_k", c_double), ("ms_select", c_double),
                 ("ms_sort", c_double), ("ms_attn", c_double), ("ms_total", c_double), ("pairs", c_int64),
-                ("dense_heads", c_int), ("max_stages_q", c_int), ("max_stages_k", c_int)]
+                ("dense_heads", c_int), ("max_stages_q", c_int), ("max_stages_k", c_int),
+                ("kmeans_rounds_q", c_int), ("kmeans_rounds_k", c_int)]
 
 
 class ac_profile(ctypes.Structure):
@@ -77,6 +78,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ac_cluster_sort_static": ([P, c_int, c_int, c_int, P, P, P, P], c_int),
         "ac_sparse_attn": ([P, P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_forward": ([P, P, P, P, P, P, P, POINTER(ac_stats), P, c_size_t, P], c_int),
+        "ac_step_state_size": ([P, POINTER(c_size_t)], c_int),
+        "ac_step_state_parts": ([P, P, P], c_int),
+        "ac_forward_step": ([P, c_int, P, P, P, P, P, POINTER(ac_stats), P, c_size_t, P], c_int),
         "ac_profile_read": ([P, POINTER(ac_profile)], c_int),
         "ac_get_status": ([P, P], c_int),
         "ac_status_string": ([c_int], ctypes.c_char_p),

@@ -175,3 +175,40 @@ class AdaCluster:
         if stats:
             return out, {f: getattr(st, f) for f, _ in _abi.ac_stats._fields_}
         return out
+
+    def step_state(self):
+        """A zeroed device buffer for ac_forward_step (counts, flags and centres
+        carried from one denoising step to the next)."""
+        n = ctypes.c_size_t(0)
+        check("ac_step_state_size", self.lib.ac_step_state_size(self._ctx, ctypes.byref(n)))
+        return torch.zeros(n.value, dtype=torch.uint8, device=self.device)
+
+    def step_state_parts(self, state):
+        """Views into a step state: nq, nk (int32 [H]), dq, dk (uint8 [H]),
+        q_cent (fp32 [H, kq_cap, d]), k_cent (fp32 [H, kk_cap, d])."""
+        parts = (ctypes.c_void_p * 6)()
+        check("ac_step_state_parts", self.lib.ac_step_state_parts(self._ctx, ptr(state), parts))
+        base = state.data_ptr()
+        H, D = self.cfg.heads, self.cfg.d
+        kq, kk = self.kq_cap, self.kk_cap
+        spec = [("nq", torch.int32, (H,)), ("nk", torch.int32, (H,)), ("dq", torch.uint8, (H,)),
+                ("dk", torch.uint8, (H,)), ("q_cent", torch.float32, (H, kq, D)), ("k_cent", torch.float32, (H, kk, D))]
+        out = {}
+        for (name, dt, shape), p in zip(spec, parts):
+            off = p - base
+            n = torch.Size(shape).numel() * torch.tensor([], dtype=dt).element_size()
+            out[name] = state[off:off + n].view(dt).view(shape)
+        return out
+
+    def ac_forward_step(self, step, q, k, v, state, out=None, stats=False, stream=None):
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        if out is None:
+            out = torch.empty(H, N, D, dtype=self.cfg.torch_dtype, device=self.device)
+        st = _abi.ac_stats() if stats else None
+        ws, nb = self._args_ws()
+        check("ac_forward_step", self.lib.ac_forward_step(
+            self._ctx, int(step), ptr(q), ptr(k), ptr(v), ptr(state), ptr(out),
+            ctypes.byref(st) if st is not None else None, ws, nb, stream_ptr(stream)))
+        if stats:
+            return out, {f: getattr(st, f) for f, _ in _abi.ac_stats._fields_}
+        return out

@@ -62,6 +62,8 @@ struct Ws {
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
     size_t chi, clo, xu, amb_cand, items_scr, runs, run_info, masks, kbmax, kbmin;
+    // early stop of fixed-count k-means: previous assignment, per-head record (q, k)
+    size_t aprev, kst;
     int kpad;
     size_t total;
 };
@@ -127,6 +129,8 @@ Ws layout(const ac_ctx *c) {
     const bool quest = c->cfg.score_mode == AC_SCORE_QUEST;
     w.kbmax = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
     w.kbmin = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
+    w.aprev = b.take(HN * 4);
+    w.kst = b.take(2 * H * 4 * 4);
     w.total = b.off;
     return w;
 }
@@ -193,16 +197,21 @@ ac_status assign_step(ac_ctx *c, const Ws &w, void *ws, const void *x, const voi
 // ------------------------------------------------------ clustering driver
 // One k-means run per head (fixed count) or Algorithm 1 (adaptive), all heads
 // batched in every launch.
+// Clustering of every head (fixed-count k-means, or Algorithm 1 when the
+// config is adaptive).  ncl_fixed / flag_fixed (device, [H], nullable): per-head
+// counts and dense flags kept from an earlier call; they select the fixed-count
+// path with those counts.  kst (device, [H, 4]): the fixed-count path's
+// convergence record (see k_conv_decide).
 ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int32_t *assign, float *cent,
                       int32_t *count, float *mean_norm, int32_t *ncl, uint8_t *flag, void *ws, cudaStream_t st,
-                      int *max_stages) {
+                      int *max_stages, const int32_t *ncl_fixed = nullptr, const uint8_t *flag_fixed = nullptr) {
     const ac_config &g = c->cfg;
     const int H = g.heads, N = g.n, D = g.d;
     const int dt = g.dtype == AC_BF16 ? DT_BF16 : DT_F32;
     const bool q = (mode == MODE_SPHERE);
     const int cap = q ? c->kq_cap : c->kk_cap;
     const int k = q ? g.kq : g.kk;
-    const bool adaptive = q ? g.adaptive_q : g.adaptive_k;
+    const bool adaptive = (q ? g.adaptive_q : g.adaptive_k) && !ncl_fixed;
     const int nmax = q ? g.nmax_q : g.nmax_k;
     Ws w = layout(c);
     double *norm = at<double>(ws, w.norm);
@@ -216,15 +225,35 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
 
     k_row_norm(x, dt, H, N, D, norm, (g.flags & AC_FLAG_CHECK_FINITE) ? 1 : 0, status, st);
     if (!adaptive) {
-        k_seg_uniform(H, N, k, seg, ncl, flag, st);
-        if (init) AC_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * H * cap * D, cudaMemcpyDeviceToDevice, st));
-        else k_init_cent(x, dt, H, N, D, nullptr, norm, seg, k, mode, cent, cap, st);
+        // per-head counts (kept from an earlier call) or the configured count
+        const int kmax = ncl_fixed ? cap : k;
+        auto set_seg = [&]() {
+            if (ncl_fixed) k_seg_from_counts(H, N, ncl_fixed, k, seg, st);
+            else k_seg_uniform(H, N, k, seg, ncl, flag, st);
+        };
+        set_seg();
+        if (ncl_fixed) {
+            AC_CUDA(cudaMemcpyAsync(ncl, ncl_fixed, sizeof(int32_t) * H, cudaMemcpyDeviceToDevice, st));
+            AC_CUDA(cudaMemcpyAsync(flag, flag_fixed, H, cudaMemcpyDeviceToDevice, st));
+        }
+        if (init && init != cent)
+            AC_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * H * cap * D, cudaMemcpyDeviceToDevice, st));
+        else if (!init)
+            k_init_cent(x, dt, H, N, D, nullptr, norm, seg, kmax, mode, cent, cap, st);
+        // Lloyd rounds; a head stops (its seg gets 0 rows) once an assignment
+        // pass repeats the previous one, which leaves every result unchanged
+        int32_t *kst = at<int32_t>(ws, w.kst) + (q ? 0 : 4 * H);
+        int32_t *prev = at<int32_t>(ws, w.aprev);
         for (int it = 0; it < g.iters; it++) {
             AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
+            k_conv_check(H, N, seg, assign, prev, kst, it == 0 ? 1 : 0, st);
+            k_conv_decide(H, seg, kst, it, st);
             k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, cnt, off, perm, status, st);
-            k_update(x, dt, H, N, D, seg, k, perm, off, cap, norm, mode, cent, st);
+            k_update(x, dt, H, N, D, seg, kmax, perm, off, cap, norm, mode, cent, st);
         }
+        // the last pass for the heads still running; then all heads again
         AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
+        if (g.iters > 0) set_seg();
         k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
         if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
         if (max_stages) *max_stages = 1;
@@ -480,6 +509,140 @@ ac_status ac_capacities(const ac_ctx *c, int *kq_cap, int *kk_cap) {
     return AC_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Where ac_forward's stages read their inputs and leave their outputs.
+struct Fwd {
+    const float *q_init = nullptr, *k_init = nullptr;  // warm-start centres (nullable)
+    float *q_cent = nullptr, *k_cent = nullptr;        // centre outputs (nullable: workspace)
+    const int32_t *nq_fixed = nullptr, *nk_fixed = nullptr;  // per-head counts kept from step 0
+    const uint8_t *dq_fixed = nullptr, *dk_fixed = nullptr;  // per-head dense flags kept from step 0
+};
+
+// Caller-owned state of the multi-step driver: {nq [H], nk [H], dq [H], dk [H],
+// q centres [H, kq_cap, d], k centres [H, kk_cap, d]}, 256-byte aligned parts.
+struct StepState {
+    int32_t *nq, *nk;
+    uint8_t *dq, *dk;
+    float *q_cent, *k_cent;
+    size_t total;
+};
+StepState step_state(const ac_ctx *c, void *base) {
+    const size_t H = c->cfg.heads, D = c->cfg.d;
+    Bump b;
+    const size_t onq = b.take(H * 4), onk = b.take(H * 4), odq = b.take(H), odk = b.take(H);
+    const size_t oqc = b.take(H * (size_t)c->kq_cap * D * 4), okc = b.take(H * (size_t)c->kk_cap * D * 4);
+    StepState ss;
+    ss.total = b.off;
+    char *p = static_cast<char *>(base);
+    ss.nq = base ? reinterpret_cast<int32_t *>(p + onq) : nullptr;
+    ss.nk = base ? reinterpret_cast<int32_t *>(p + onk) : nullptr;
+    ss.dq = base ? reinterpret_cast<uint8_t *>(p + odq) : nullptr;
+    ss.dk = base ? reinterpret_cast<uint8_t *>(p + odk) : nullptr;
+    ss.q_cent = base ? reinterpret_cast<float *>(p + oqc) : nullptr;
+    ss.k_cent = base ? reinterpret_cast<float *>(p + okc) : nullptr;
+    return ss;
+}
+
+// Max over heads of the rounds the fixed-count k-means ran (kst [H, 4]); 0 if
+// nothing was recorded.
+int max_rounds(const int32_t *kst_dev, int H) {
+    int32_t *h = (int32_t *)malloc(sizeof(int32_t) * 4 * H);
+    if (!h) return 0;
+    int m = 0;
+    if (cudaMemcpy(h, kst_dev, sizeof(int32_t) * 4 * H, cudaMemcpyDeviceToHost) == cudaSuccess)
+        for (int i = 0; i < H; i++) m = h[4 * i + 2] > m ? h[4 * i + 2] : m;
+    free(h);
+    return m;
+}
+
+// Algorithm 3 for every head: both clusterings, the selection and the sparse
+// attention, on one stream.
+ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, const Fwd &f, void *out,
+                       ac_stats *stats, void *ws, cudaStream_t st) {
+    const ac_config &g = c->cfg;
+    Ws w = layout(c);
+    float *qc = f.q_cent ? f.q_cent : at<float>(ws, w.qc);
+    float *kc = f.k_cent ? f.k_cent : at<float>(ws, w.kc);
+    int32_t *qa = at<int32_t>(ws, w.qa), *ka = at<int32_t>(ws, w.ka);
+    int32_t *qn = at<int32_t>(ws, w.qcount), *kn = at<int32_t>(ws, w.kcount);
+    float *qmn = at<float>(ws, w.qmn);
+    int32_t *nq = at<int32_t>(ws, w.nq), *nk = at<int32_t>(ws, w.nk);
+    uint8_t *dq = at<uint8_t>(ws, w.dq), *dk = at<uint8_t>(ws, w.dk);
+    int32_t *sel = at<int32_t>(ws, w.sel), *selc = at<int32_t>(ws, w.selc);
+    int32_t *kst = at<int32_t>(ws, w.kst);
+    int sq = 1, sk = 1;
+    cudaEvent_t *pe = nullptr;
+    if (g.flags & AC_FLAG_PROFILE) {
+        pe = c->prof + (size_t)(c->prof_n % PROF_RING) * PROF_EV;
+        c->prof_n++;
+        AC_CUDA(cudaEventRecord(pe[0], st));
+    }
+    if (stats) {
+        AC_CUDA(cudaMemsetAsync(kst, 0, sizeof(int32_t) * 8 * g.heads, st));
+        AC_CUDA(cudaEventRecord(c->ev[0], st));
+    }
+    ac_status s = run_cluster(c, MODE_SPHERE, q, f.q_init, qa, qc, qn, qmn, nq, dq, ws, st, &sq, f.nq_fixed, f.dq_fixed);
+    if (s != AC_OK) return s;
+    if (pe) AC_CUDA(cudaEventRecord(pe[1], st));
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[1], st));
+    s = run_cluster(c, MODE_EUCLID, k, f.k_init, ka, kc, kn, nullptr, nk, dk, ws, st, &sk, f.nk_fixed, f.dk_fixed);
+    if (s != AC_OK) return s;
+    if (pe) AC_CUDA(cudaEventRecord(pe[2], st));
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[2], st));
+    // a head is dense when either clustering set its flag F
+    uint8_t *dense = dk;
+    if (g.adaptive_q || f.dq_fixed) ac_or_flags(g.heads, dq, dk, st);
+    float *kbmax = nullptr, *kbmin = nullptr;
+    if (g.score_mode == AC_SCORE_QUEST) {
+        kbmax = at<float>(ws, w.kbmax);
+        kbmin = at<float>(ws, w.kbmin);
+        key_bounds(c, k, ka, nk, kbmax, kbmin, ws, st);
+    }
+    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk, dense,
+             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st);
+    if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
+    if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
+    s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
+                       pe ? pe + 4 : nullptr);
+    if (s != AC_OK) return s;
+    if (stats) {
+        AC_CUDA(cudaEventRecord(c->ev[4], st));
+        AC_CUDA(cudaEventSynchronize(c->ev[4]));
+        float ms[4];
+        cudaEventElapsedTime(&ms[0], c->ev[0], c->ev[1]);
+        cudaEventElapsedTime(&ms[1], c->ev[1], c->ev[2]);
+        cudaEventElapsedTime(&ms[2], c->ev[2], c->ev[3]);
+        cudaEventElapsedTime(&ms[3], c->ev[3], c->ev[4]);
+        memset(stats, 0, sizeof(*stats));
+        stats->ms_cluster_q = ms[0];
+        stats->ms_cluster_k = ms[1];
+        stats->ms_select = ms[2];
+        stats->ms_attn = ms[3];
+        stats->ms_total = ms[0] + ms[1] + ms[2] + ms[3];
+        int64_t pairs = 0;
+        AC_CUDA(cudaMemcpy(&pairs, at<int64_t>(ws, w.pairs), sizeof(pairs), cudaMemcpyDeviceToHost));
+        stats->pairs = pairs;
+        uint8_t *hd = (uint8_t *)malloc(g.heads);
+        if (hd) {
+            AC_CUDA(cudaMemcpy(hd, dense, g.heads, cudaMemcpyDeviceToHost));
+            for (int h = 0; h < g.heads; h++) stats->dense_heads += hd[h] ? 1 : 0;
+            free(hd);
+        }
+        stats->max_stages_q = sq;
+        stats->max_stages_k = sk;
+        stats->kmeans_rounds_q = max_rounds(kst, g.heads);
+        stats->kmeans_rounds_k = max_rounds(kst + 4 * g.heads, g.heads);
+    }
+    return launch_check();
+}
+
+}  // namespace
+
+extern "C" {
+
 ac_status ac_workspace_size(const ac_ctx *c, size_t *bytes) {
     if (!c || !bytes) return AC_ERR_INVALID_ARG;
     *bytes = layout(c).total;
@@ -570,76 +733,62 @@ ac_status ac_forward(ac_ctx *c, const void *q, const void *k, const void *v, flo
     if (warm && ((q_cent_io && g.adaptive_q) || (k_cent_io && g.adaptive_k))) return AC_ERR_INVALID_ARG;
     ac_status s = check_ws(c, ws, ws_bytes);
     if (s != AC_OK) return s;
+    Fwd f;
+    f.q_init = (warm && q_cent_io) ? q_cent_io : nullptr;
+    f.k_init = (warm && k_cent_io) ? k_cent_io : nullptr;
+    f.q_cent = q_cent_io;
+    f.k_cent = k_cent_io;
+    return forward_impl(c, q, k, v, f, out, stats, ws, (cudaStream_t)stream);
+}
+
+ac_status ac_step_state_size(const ac_ctx *c, size_t *bytes) {
+    if (!c || !bytes) return AC_ERR_INVALID_ARG;
+    *bytes = step_state(c, nullptr).total;
+    return AC_OK;
+}
+
+ac_status ac_step_state_parts(const ac_ctx *c, void *state, void **parts) {
+    if (!c || !state || !parts) return AC_ERR_INVALID_ARG;
+    const StepState ss = step_state(c, state);
+    parts[0] = ss.nq;
+    parts[1] = ss.nk;
+    parts[2] = ss.dq;
+    parts[3] = ss.dk;
+    parts[4] = ss.q_cent;
+    parts[5] = ss.k_cent;
+    return AC_OK;
+}
+
+ac_status ac_forward_step(ac_ctx *c, int step, const void *q, const void *k, const void *v, void *state, void *out,
+                          ac_stats *stats, void *ws, size_t ws_bytes, void *stream) {
+    if (!c || !q || !k || !v || !out || !state || step < 0) return AC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
+        return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    const StepState ss = step_state(c, state);
     cudaStream_t st = (cudaStream_t)stream;
+    Fwd f;
+    f.q_cent = ss.q_cent;
+    f.k_cent = ss.k_cent;
+    if (step > 0) {
+        // the counts and dense flags of step 0, k-means seeded with the
+        // previous step's centres (updated in place)
+        f.q_init = ss.q_cent;
+        f.k_init = ss.k_cent;
+        f.nq_fixed = ss.nq;
+        f.nk_fixed = ss.nk;
+        f.dq_fixed = ss.dq;
+        f.dk_fixed = ss.dk;
+    }
+    s = forward_impl(c, q, k, v, f, out, stats, ws, st);
+    if (s != AC_OK || step > 0) return s;
+    // step 0: keep the counts and flags Algorithm 1 (or the fixed config) chose
     Ws w = layout(c);
-    float *qc = q_cent_io ? q_cent_io : at<float>(ws, w.qc);
-    float *kc = k_cent_io ? k_cent_io : at<float>(ws, w.kc);
-    int32_t *qa = at<int32_t>(ws, w.qa), *ka = at<int32_t>(ws, w.ka);
-    int32_t *qn = at<int32_t>(ws, w.qcount), *kn = at<int32_t>(ws, w.kcount);
-    float *qmn = at<float>(ws, w.qmn);
-    int32_t *nq = at<int32_t>(ws, w.nq), *nk = at<int32_t>(ws, w.nk);
-    uint8_t *dq = at<uint8_t>(ws, w.dq), *dk = at<uint8_t>(ws, w.dk);
-    int32_t *sel = at<int32_t>(ws, w.sel), *selc = at<int32_t>(ws, w.selc);
-    int sq = 1, sk = 1;
-    cudaEvent_t *pe = nullptr;
-    if (g.flags & AC_FLAG_PROFILE) {
-        pe = c->prof + (size_t)(c->prof_n % PROF_RING) * PROF_EV;
-        c->prof_n++;
-        AC_CUDA(cudaEventRecord(pe[0], st));
-    }
-    if (stats) AC_CUDA(cudaEventRecord(c->ev[0], st));
-    s = run_cluster(c, MODE_SPHERE, q, (warm && q_cent_io) ? q_cent_io : nullptr, qa, qc, qn, qmn, nq, dq, ws, st,
-                    &sq);
-    if (s != AC_OK) return s;
-    if (pe) AC_CUDA(cudaEventRecord(pe[1], st));
-    if (stats) AC_CUDA(cudaEventRecord(c->ev[1], st));
-    s = run_cluster(c, MODE_EUCLID, k, (warm && k_cent_io) ? k_cent_io : nullptr, ka, kc, kn, nullptr, nk, dk, ws,
-                    st, &sk);
-    if (s != AC_OK) return s;
-    if (pe) AC_CUDA(cudaEventRecord(pe[2], st));
-    if (stats) AC_CUDA(cudaEventRecord(c->ev[2], st));
-    // a head is dense when either clustering set its flag F
-    uint8_t *dense = dk;
-    if (g.adaptive_q) ac_or_flags(g.heads, dq, dk, st);
-    float *kbmax = nullptr, *kbmin = nullptr;
-    if (g.score_mode == AC_SCORE_QUEST) {
-        kbmax = at<float>(ws, w.kbmax);
-        kbmin = at<float>(ws, w.kbmin);
-        key_bounds(c, k, ka, nk, kbmax, kbmin, ws, st);
-    }
-    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk, dense,
-             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st);
-    if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
-    if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
-    s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
-                       pe ? pe + 4 : nullptr);
-    if (s != AC_OK) return s;
-    if (stats) {
-        AC_CUDA(cudaEventRecord(c->ev[4], st));
-        AC_CUDA(cudaEventSynchronize(c->ev[4]));
-        float ms[4];
-        cudaEventElapsedTime(&ms[0], c->ev[0], c->ev[1]);
-        cudaEventElapsedTime(&ms[1], c->ev[1], c->ev[2]);
-        cudaEventElapsedTime(&ms[2], c->ev[2], c->ev[3]);
-        cudaEventElapsedTime(&ms[3], c->ev[3], c->ev[4]);
-        memset(stats, 0, sizeof(*stats));
-        stats->ms_cluster_q = ms[0];
-        stats->ms_cluster_k = ms[1];
-        stats->ms_select = ms[2];
-        stats->ms_attn = ms[3];
-        stats->ms_total = ms[0] + ms[1] + ms[2] + ms[3];
-        int64_t pairs = 0;
-        AC_CUDA(cudaMemcpy(&pairs, at<int64_t>(ws, w.pairs), sizeof(pairs), cudaMemcpyDeviceToHost));
-        stats->pairs = pairs;
-        uint8_t *hd = (uint8_t *)malloc(g.heads);
-        if (hd) {
-            AC_CUDA(cudaMemcpy(hd, dense, g.heads, cudaMemcpyDeviceToHost));
-            for (int h = 0; h < g.heads; h++) stats->dense_heads += hd[h] ? 1 : 0;
-            free(hd);
-        }
-        stats->max_stages_q = sq;
-        stats->max_stages_k = sk;
-    }
+    AC_CUDA(cudaMemcpyAsync(ss.nq, at<int32_t>(ws, w.nq), sizeof(int32_t) * c->cfg.heads, cudaMemcpyDeviceToDevice, st));
+    AC_CUDA(cudaMemcpyAsync(ss.nk, at<int32_t>(ws, w.nk), sizeof(int32_t) * c->cfg.heads, cudaMemcpyDeviceToDevice, st));
+    AC_CUDA(cudaMemcpyAsync(ss.dq, at<uint8_t>(ws, w.dq), c->cfg.heads, cudaMemcpyDeviceToDevice, st));
+    AC_CUDA(cudaMemcpyAsync(ss.dk, at<uint8_t>(ws, w.dk), c->cfg.heads, cudaMemcpyDeviceToDevice, st));
     return launch_check();
 }
 

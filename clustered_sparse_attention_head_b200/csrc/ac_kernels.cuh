@@ -30,6 +30,11 @@ void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg,
               const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st);
 void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const int32_t *off, int cap,
                  const double *norm, float *mean_norm, cudaStream_t st);
+// Early stop of fixed-count k-means (ac_kmeans.cu): kst [H, 4] = {stopped,
+// rows changed in the pass, rounds run, -}; a stopped head's seg gets 0 rows.
+void k_conv_check(int H, int N, const HeadSeg *seg, const int32_t *assign, int32_t *prev, int32_t *kst, int first,
+                  cudaStream_t st);
+void k_conv_decide(int H, HeadSeg *seg, int32_t *kst, int it, cudaStream_t st);
 
 // ---- ac_assign_tc.cu (bf16 inputs): tcgen05 screen; the exact pass follows
 int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const HeadSeg *seg, int nrows_max,

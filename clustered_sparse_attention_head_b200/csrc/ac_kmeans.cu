@@ -510,4 +510,56 @@ void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const in
     mean_norm_kernel<<<g, 128, 0, st>>>(N, seg, perm, off, cap, norm, mean_norm); note_launch();
 }
 
+// ------------------------------------------------------------ convergence
+// Fixed-count k-means stops per head once an assignment pass reproduces the
+// previous pass: the update of an unchanged assignment gives back the same
+// centroids, so every later pass would repeat it exactly and stopping changes
+// no result.  kst[4h + 0] = stopped, + 1 = rows changed in this pass, + 2 =
+// rounds (assignment + update) run.  A stopped head's pass segment gets 0 rows,
+// which every clustering kernel already skips.
+
+// Rows of each active head whose assignment differs from `prev`; then prev = assign.
+__global__ void conv_check_kernel(int N, const HeadSeg *__restrict__ seg, const int32_t *__restrict__ assign,
+                                  int32_t *__restrict__ prev, int32_t *__restrict__ kst, int first) {
+    const int h = blockIdx.y;
+    const int nrows = seg[h].nrows;
+    if ((int)(blockIdx.x * blockDim.x) >= nrows) return;  // whole CTA
+    const int pos = blockIdx.x * blockDim.x + threadIdx.x;
+    int diff = 0;
+    if (pos < nrows) {
+        const size_t i = (size_t)h * N + pos;
+        const int32_t a = assign[i];
+        diff = (!first && a != prev[i]) ? 1 : 0;
+        prev[i] = a;
+    }
+    const int n = __syncthreads_count(diff);
+    if (threadIdx.x == 0 && n) atomicAdd(&kst[4 * h + 1], n);
+}
+
+// After pass `it`: stop the heads whose assignment did not change.
+__global__ void conv_decide_kernel(int H, HeadSeg *__restrict__ seg, int32_t *__restrict__ kst, int it) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    if (it == 0) kst[4 * h + 0] = 0;
+    if (seg[h].nrows > 0) {
+        if (it > 0 && kst[4 * h + 1] == 0) {
+            kst[4 * h + 0] = 1;
+            seg[h].nrows = 0;
+        } else {
+            kst[4 * h + 2] = it + 1;
+        }
+    }
+    kst[4 * h + 1] = 0;
+}
+
+void k_conv_check(int H, int N, const HeadSeg *seg, const int32_t *assign, int32_t *prev, int32_t *kst, int first,
+                  cudaStream_t st) {
+    conv_check_kernel<<<dim3((N + 255) / 256, H), 256, 0, st>>>(N, seg, assign, prev, kst, first);
+    note_launch();
+}
+void k_conv_decide(int H, HeadSeg *seg, int32_t *kst, int it, cudaStream_t st) {
+    conv_decide_kernel<<<(H + 127) / 128, 128, 0, st>>>(H, seg, kst, it);
+    note_launch();
+}
+
 }  // namespace ac

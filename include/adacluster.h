@@ -113,6 +113,11 @@ typedef struct {
     int64_t pairs;          /* (query, key) pairs the attention computed, all heads   */
     int dense_heads;        /* heads that took dense attention                        */
     int max_stages_q, max_stages_k;
+    /* Rounds (assignment + update) the fixed-count k-means ran, max over heads;
+     * 0 for adaptive clustering.  A head stops before ac_config.iters rounds once
+     * an assignment pass reproduces the previous one (the result is the same as
+     * running all rounds: the update would give back the same centres).       */
+    int kmeans_rounds_q, kmeans_rounds_k;
 } ac_stats;
 
 /* Averages over the ac_forward calls recorded with AC_FLAG_PROFILE since the
@@ -237,6 +242,32 @@ AC_API ac_status ac_sparse_attn(ac_ctx *ctx, const void *q, const void *k, const
 AC_API ac_status ac_forward(ac_ctx *ctx, const void *q, const void *k, const void *v, float *q_cent_io,
                      float *k_cent_io, void *out, ac_stats *stats, void *ws, size_t ws_bytes,
                      void *stream);
+
+/* Multi-step driver over denoising steps (AdaCluster, §3.2.2 "Efficient
+ * initialization" and §4.1): the token distribution drifts little from one
+ * step to the next, so the clustering of step 0 sets each head's cluster
+ * counts (Algorithm 1 when the config is adaptive, else kq / kk) and its
+ * dense flag F, and every later step keeps those counts and flags and seeds
+ * k-means with the previous step's centres, which then needs fewer rounds
+ * (ac_stats.kmeans_rounds_*).
+ *   state: caller-owned device buffer of ac_step_state_size bytes, 16-byte
+ *          aligned, holding the per-head counts, flags and the q / k centres.
+ *          Step 0 writes all of it; step > 0 reads it and updates the centres.
+ *          Its contents are opaque; step > 0 requires a state written by an
+ *          earlier step of the same context configuration.
+ *   step:  0 for the first denoising step, > 0 afterwards.
+ * Everything else as ac_forward (no q_cent_io / k_cent_io: the centres live in
+ * the state).  Errors: AC_ERR_INVALID_ARG for NULL or misaligned buffers or
+ * step < 0; workspace errors as ac_forward. */
+AC_API ac_status ac_step_state_size(const ac_ctx *ctx, size_t *bytes);
+/* Device pointers to the parts of a step state (for inspection): parts[0] =
+ * per-head query cluster counts (int32 [H]), [1] key counts, [2] query dense
+ * flags (uint8 [H]), [3] key (combined) dense flags, [4] query centres (fp32
+ * [H, kq_cap, d]), [5] key centres (fp32 [H, kk_cap, d]).  No device access. */
+AC_API ac_status ac_step_state_parts(const ac_ctx *ctx, void *state, void **parts);
+AC_API ac_status ac_forward_step(ac_ctx *ctx, int step, const void *q, const void *k, const void *v,
+                                 void *state, void *out, ac_stats *stats, void *ws, size_t ws_bytes,
+                                 void *stream);
 
 /* Wait for the recorded events, fill *out (averages per call) and reset the
  * record.  Events are recorded on the stream each ac_forward call used. */
