@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--denoise-steps", type=int, default=0,
+                    help="also run the multi-step driver (ac_forward_step) over this many drifting steps")
+    ap.add_argument("--drift", type=float, default=0.02, help="per-element drift per denoising step")
     return ap.parse_args()
 
 
@@ -375,12 +378,44 @@ def main():
                 "gpu_launches": int(prof["launches"]) if e2e is None else None, "clocks": clocks}
         if line["gpu_launches"] is None:
             line["gpu_launches"] = launches_per_call(ac, q, k, v, out) * a.steps
+        if a.denoise_steps > 0:
+            line["denoise_steps"] = denoise_steps(ac, q, k, v, out, a.denoise_steps, a.drift, stream)
         print(json.dumps(line), flush=True)
     ac.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def denoise_steps(ac, q, k, v, out, steps, drift, stream):
+    """The multi-step driver on inputs that drift by drift * N(0, 1) per element
+    and step (seeded, drawn on the device before each step's timed call): step
+    0 clusters as configured, later steps keep its counts and warm-start
+    k-means.  Per step: call time (CUDA events) and the k-means rounds run."""
+    import torch
+    state = ac.step_state()
+    gen = torch.Generator(device=q.device)
+    gen.manual_seed(1234)
+    qs, ks, vs = q.clone(), k.clone(), v.clone()
+    rows = []
+    for s in range(steps):
+        if s > 0:
+            for t in (qs, ks, vs):
+                t.copy_((t.float() + drift * torch.randn(t.shape, generator=gen, device=t.device)).to(t.dtype))
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _, st = ac.ac_forward_step(s, qs, ks, vs, state, out=out, stats=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rows.append({"step": s, "ms": e0.elapsed_time(e1), "ms_cluster_q": st["ms_cluster_q"],
+                     "ms_cluster_k": st["ms_cluster_k"], "rounds_q": st["kmeans_rounds_q"],
+                     "rounds_k": st["kmeans_rounds_k"]})
+    status = ac.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    return {"drift": drift, "steps": rows}
 
 
 def launches_per_call(ac, q, k, v, out):
