@@ -301,6 +301,7 @@ class HeadSpec:
     nmax_k: int = 0
     score_mode: int = 0   # SCORE_CENTROID or SCORE_QUEST
     top_k: int = 0        # > 0: argtopk instead of top-p
+    text_keys: int = 0    # > 0: the last text_keys keys are always attended, not clustered
 
 
 @dataclass
@@ -326,6 +327,9 @@ def cluster_q(q, spec: HeadSpec, init=None):
 
 
 def cluster_k(k, spec: HeadSpec, init=None):
+    """Key clustering; with spec.text_keys only the keys before the text strip."""
+    if spec.text_keys:
+        k = k[:k.shape[0] - spec.text_keys]
     xs, _ = prepare(k, EUCLID)
     if spec.adaptive_k:
         return multistage(xs, spec.kk, spec.iters, spec.tau_rule, spec.tau_value, spec.nmax_k, EUCLID)
@@ -354,24 +358,35 @@ def forward_steps(steps, spec: HeadSpec, rows=None):
         xq, nrm = prepare(q, SPHERE)
         rq = kmeans(xq, nq, spec.iters, SPHERE, init=prev.q.cent[:nq])
         qmn = cluster_mean_norm(nrm, rq.assign, rq.nclusters)
-        xk, _ = prepare(k, EUCLID)
+        xk, _ = prepare(k[:k.shape[0] - spec.text_keys], EUCLID)
         rk = kmeans(xk, nk, spec.iters, EUCLID, init=prev.k.cent[:nk])
         res.append(_select_attend(q, k, v, rq, rk, qmn, dense, spec, rows))
     return res
 
 
 def _select_attend(q, k, v, rq, rk, qmn, dense, spec: HeadSpec, rows):
-    """Algorithm 3 lines 6-9 for one head from its two clusterings."""
+    """Algorithm 3 lines 6-9 for one head from its two clusterings.  With
+    spec.text_keys the text keys form one more key group (id = the number of
+    key clusters) that no score ranks and every query cluster selects."""
+    nv = rk.nclusters
+    kv = k[:k.shape[0] - spec.text_keys]
+    k_assign = rk.assign
+    if spec.text_keys:
+        k_assign = np.concatenate([rk.assign, np.full(spec.text_keys, nv, np.int32)])
     if dense:
-        sel = np.zeros((rq.nclusters, max(rk.nclusters, 1)), np.int32)
+        sel = np.zeros((rq.nclusters, max(nv, 1)), np.int32)
         cnt = np.zeros(rq.nclusters, np.int32)
     else:
         kmax = kmin = None
         if spec.score_mode == SCORE_QUEST:
-            kmax, kmin = key_bounds(k, rk.assign, rk.nclusters)
-        sel, cnt = select2(rq.cent, qmn, rq.count, rk.cent, rk.count, spec.top_p, spec.score_mode, spec.top_k,
-                           kmax, kmin)
+            kmax, kmin = key_bounds(kv, rk.assign, nv)
+        sel, cnt = select2(rq.cent, qmn, rq.count, rk.cent[:nv], rk.count, spec.top_p, spec.score_mode,
+                           spec.top_k, kmax, kmin)
+        if spec.text_keys:
+            sel = np.concatenate([sel, np.full((sel.shape[0], 1), -1, np.int32)], axis=1)
+            sel[np.arange(sel.shape[0]), cnt] = nv
+            cnt = cnt + 1
     if rows is None:
         rows = np.arange(q.shape[0], dtype=np.int32)
-    out = attention_rows(q, k, v, rq.assign, rk.assign, rk.nclusters, sel, cnt, dense, rows)
-    return HeadResult(rq, rk, qmn, sel, cnt, dense, out, np.asarray(rows, np.int32))
+    out = attention_rows(q, k, v, rq.assign, k_assign, nv + (1 if spec.text_keys else 0), sel, cnt, dense, rows)
+    return HeadResult(rq, rk, qmn, sel, cnt, dense, out, np.asarray(rows, np.int32), extra={"k_assign": k_assign})

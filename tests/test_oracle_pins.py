@@ -609,3 +609,55 @@ def test_step_inputs_drift(orc):
     d1, d2 = (s1.k - s0.k), (s2.k - s1.k)
     assert abs(d1.std() - 0.1) < 0.01 and abs(d2.std() - 0.1) < 0.01
     assert abs(np.corrcoef(d1.ravel(), d2.ravel())[0, 1]) < 0.05
+
+
+# --------------------------------------------------------------------------
+# Text keys always attended (a dense strip; SURVEY f4 variant, not in the pages)
+# --------------------------------------------------------------------------
+def _with_text(n_video=360, n_text=24, d=16, seed=21):
+    rng = np.random.default_rng(seed)
+    steps, lab = _drifting_gmm(1, comps=6, per=n_video // 6, d=d, seed=seed)
+    q, k, v = steps[0]
+    tq, tk, tv = (rng.standard_normal((n_text, d)).astype(np.float32) for _ in range(3))
+    return np.concatenate([q, tq]), np.concatenate([k, tk]), np.concatenate([v, tv]), n_text
+
+
+def test_text_keys_in_every_key_set(orc):
+    """Every query attends to the text keys plus the members of its cluster's
+    selected video key clusters: the rows equal exact attention over that set."""
+    q, k, v, T = _with_text()
+    n = q.shape[0]
+    spec = orc.HeadSpec(kq=6, kk=6, iters=5, top_p=0.3, text_keys=T)
+    rows = np.arange(0, n, 7).astype(np.int32)
+    r = orc.forward_head(q, k, v, spec, rows=rows)
+    assert r.dense == 0
+    nv = r.k.nclusters
+    for i, row in enumerate(rows):
+        a = r.q.assign[row]
+        chosen = set(r.sel_idx[a, :r.sel_cnt[a]].tolist())
+        assert nv in chosen, "the text group is always selected"
+        keys = np.concatenate([np.nonzero(np.isin(r.k.assign, sorted(chosen - {nv})))[0], np.arange(n - T, n)])
+        np.testing.assert_allclose(r.out_rows[i], _np_attention(q[row:row + 1], k[keys], v[keys])[0],
+                                   rtol=1e-10, atol=1e-12)
+
+
+def test_text_keys_not_clustered(orc):
+    """The video keys are clustered exactly as on their own; the text keys get
+    the extra group id."""
+    q, k, v, T = _with_text()
+    spec = orc.HeadSpec(kq=6, kk=6, iters=5, top_p=0.9, text_keys=T)
+    r = orc.forward_head(q, k, v, spec, rows=np.arange(0, 10, dtype=np.int32))
+    xs, _ = orc.prepare(k[:-T], orc.EUCLID)
+    alone = orc.kmeans(xs, 6, 5, orc.EUCLID)
+    np.testing.assert_array_equal(r.k.assign, alone.assign)
+    np.testing.assert_array_equal(r.extra["k_assign"][-T:], 6)
+
+
+def test_text_keys_zero_is_unchanged(orc):
+    """text_keys = 0 gives exactly Algorithm 3 without the strip."""
+    q, k, v, T = _with_text()
+    rows = np.arange(0, q.shape[0], 11).astype(np.int32)
+    a = orc.forward_head(q, k, v, orc.HeadSpec(kq=6, kk=6, iters=5, top_p=0.5), rows=rows)
+    b = orc.forward_head(q, k, v, orc.HeadSpec(kq=6, kk=6, iters=5, top_p=0.5, text_keys=0), rows=rows)
+    np.testing.assert_array_equal(a.out_rows, b.out_rows)
+    np.testing.assert_array_equal(a.sel_cnt, b.sel_cnt)
