@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--denoise-steps", type=int, default=0,
                     help="also run the multi-step driver (ac_forward_step) over this many drifting steps")
     ap.add_argument("--drift", type=float, default=0.02, help="per-element drift per denoising step")
+    ap.add_argument("--text-keys", action="store_true",
+                    help="attend every query to the workload's text keys (a dense strip), not clustered")
     return ap.parse_args()
 
 
@@ -238,6 +240,8 @@ def main():
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     cfg = Config.from_workload(w)
     cfg.flags = _abi.AC_FLAG_PROFILE
+    if a.text_keys:
+        cfg.text_keys = w.text
     ac = AdaCluster(cfg, device=dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
@@ -366,7 +370,8 @@ def main():
                 "warmup": max(a.warmup, 3), "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
                 "config": {"workload": w.name, "heads": w.heads, "n": w.n, "d": w.d, "kq": w.kq, "kk": w.kk,
-                           "iters": w.iters, "top_p": w.top_p, "parallelism": f"dp{world} (independent calls)",
+                           "iters": w.iters, "top_p": w.top_p, "text_keys": cfg.text_keys,
+                           "parallelism": f"dp{world} (independent calls)",
                            "l2": "inputs larger than L2 (774 MB per tensor), no flush"},
                 "tflops_effective_call": tflops_call, "tflops_effective_attn": tflops_attn,
                 "pairs": st["pairs"], "density": st["pairs"] / (w.heads * float(w.n) ** 2),

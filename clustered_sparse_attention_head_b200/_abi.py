@@ -31,7 +31,7 @@ class ac_config(ctypes.Structure):
     _fields_ = [("heads", c_int), ("n", c_int), ("d", c_int), ("dtype", c_int), ("kq", c_int), ("kk", c_int),
                 ("iters", c_int), ("adaptive_q", c_int), ("adaptive_k", c_int), ("tau_rule", c_int),
                 ("tau_value", c_double), ("nmax_q", c_int), ("nmax_k", c_int), ("top_p", c_double),
-                ("flags", c_uint), ("score_mode", c_int), ("top_k", c_int)]
+                ("flags", c_uint), ("score_mode", c_int), ("top_k", c_int), ("text_keys", c_int)]
 
 
 class ac_stats(ctypes.Structure):

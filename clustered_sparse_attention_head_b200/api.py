@@ -34,12 +34,13 @@ class Config:
     flags: int = 0
     score_mode: int = _abi.AC_SCORE_CENTROID   # or AC_SCORE_QUEST
     top_k: int = 0                             # > 0: argtopk instead of top-p
+    text_keys: int = 0                         # > 0: last text_keys keys always attended, not clustered
 
     def to_c(self) -> _abi.ac_config:
         return _abi.ac_config(self.heads, self.n, self.d, _abi.AC_BF16 if self.dtype == "bf16" else _abi.AC_F32,
                               self.kq, self.kk, self.iters, int(self.adaptive_q), int(self.adaptive_k),
                               self.tau_rule, float(self.tau_value), self.nmax_q, self.nmax_k, float(self.top_p),
-                              self.flags, int(self.score_mode), int(self.top_k))
+                              self.flags, int(self.score_mode), int(self.top_k), int(self.text_keys))
 
     @property
     def torch_dtype(self):

@@ -213,6 +213,9 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
     const int k = q ? g.kq : g.kk;
     const bool adaptive = (q ? g.adaptive_q : g.adaptive_k) && !ncl_fixed;
     const int nmax = q ? g.nmax_q : g.nmax_k;
+    // keys: the text strip (the last text_keys rows) is not clustered
+    const int text = q ? 0 : g.text_keys;
+    const int Nc = N - text;
     Ws w = layout(c);
     double *norm = at<double>(ws, w.norm);
     HeadSeg *seg = at<HeadSeg>(ws, w.seg);
@@ -228,8 +231,8 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         // per-head counts (kept from an earlier call) or the configured count
         const int kmax = ncl_fixed ? cap : k;
         auto set_seg = [&]() {
-            if (ncl_fixed) k_seg_from_counts(H, N, ncl_fixed, k, seg, st);
-            else k_seg_uniform(H, N, k, seg, ncl, flag, st);
+            if (ncl_fixed) k_seg_from_counts(H, Nc, ncl_fixed, k, seg, st, text > 0 ? 1 : 0);
+            else k_seg_uniform(H, Nc, k, seg, ncl, flag, st);
         };
         set_seg();
         if (ncl_fixed) {
@@ -256,6 +259,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         if (g.iters > 0) set_seg();
         k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
         if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
+        if (text > 0) k_text_group(H, N, Nc, seg, assign, count, cap, ncl, st);
         if (max_stages) *max_stages = 1;
         return launch_check();
     }
@@ -264,10 +268,10 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
     int32_t *pa = at<int32_t>(ws, w.passign);
     double *dist = at<double>(ws, w.dist);
     MsHead *ms = at<MsHead>(ws, w.ms);
-    k_ms_init(H, N, ms, U, Un, st);
+    k_ms_init(H, N, Nc, ms, U, Un, st);
     int stages = 0;
     for (int t = 0;; t++) {
-        k_ms_control(H, N, k, nmax, cap, ms, seg, c->d_info, status, st);
+        k_ms_control(H, Nc, k, nmax, cap - (text > 0 ? 1 : 0), ms, seg, c->d_info, status, st);
         AC_CUDA(cudaMemcpyAsync(c->h_info, c->d_info, 8 * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
         AC_CUDA(cudaStreamSynchronize(st));
         if (c->h_info[4]) return AC_ERR_CAPACITY;
@@ -295,10 +299,11 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         Un = tmp;
         AC_CUDA(cudaGetLastError());
     }
-    k_ms_final(H, N, ms, seg, ncl, flag, c->d_info, st);
+    k_ms_final(H, Nc, ms, seg, ncl, flag, c->d_info, st);
     AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
     k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
     if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
+    if (text > 0) k_text_group(H, N, Nc, seg, assign, count, cap, ncl, st);
     if (max_stages) *max_stages = stages;
     return launch_check();
 }
@@ -318,7 +323,7 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     AttnItem *items = at<AttnItem>(ws, w.items);
     int32_t *nitems = at<int32_t>(ws, w.nitems);
     k_seg_from_counts(H, N, nq, g.kq, sq, st);
-    k_seg_from_counts(H, N, nk, g.kk, sk, st);
+    k_seg_from_counts(H, N, nk, g.kk + (g.text_keys > 0 ? 1 : 0), sk, st);
     k_sort(qa, nullptr, sq, H, N, N, c->kq_cap, rank, hist, cnt, qoff, qperm, c->d_status, st);
     k_sort(ka, nullptr, sk, H, N, N, c->kk_cap, rank, hist, cnt, koff, kperm, c->d_status, st);
     const int rb = D * c->elt;
@@ -356,6 +361,8 @@ ac_status validate(const ac_config *g) {
     if (!(g->top_p > 0.0)) return AC_ERR_INVALID_ARG;
     if (g->score_mode != AC_SCORE_CENTROID && g->score_mode != AC_SCORE_QUEST) return AC_ERR_INVALID_ARG;
     if (g->top_k < 0) return AC_ERR_INVALID_ARG;
+    if (g->text_keys < 0 || g->text_keys >= g->n || (g->text_keys > 0 && g->kk > g->n - g->text_keys))
+        return AC_ERR_INVALID_ARG;
     if ((long long)g->heads * g->n > 0x7fffffffLL / 2) return AC_ERR_UNSUPPORTED;
     if (g->adaptive_q && g->nmax_q < 1) return AC_ERR_INVALID_ARG;
     if (g->adaptive_k && g->nmax_k < 1) return AC_ERR_INVALID_ARG;
@@ -375,7 +382,7 @@ void key_bounds(ac_ctx *c, const void *k, const int32_t *ka, const int32_t *nk, 
     Ws w = layout(c);
     HeadSeg *sk = at<HeadSeg>(ws, w.segk);
     int32_t *kperm = at<int32_t>(ws, w.kperm), *koff = at<int32_t>(ws, w.koff);
-    k_seg_from_counts(g.heads, g.n, nk, g.kk, sk, st);
+    k_seg_from_counts(g.heads, g.n, nk, g.kk + (g.text_keys > 0 ? 1 : 0), sk, st);
     k_sort(ka, nullptr, sk, g.heads, g.n, g.n, c->kk_cap, at<int32_t>(ws, w.rank), at<int32_t>(ws, w.hist),
            at<int32_t>(ws, w.cnt2), koff, kperm, c->d_status, st);
     k_cluster_bounds(k, g.dtype == AC_BF16 ? DT_BF16 : DT_F32, g.heads, g.n, g.d, kperm, koff, c->kk_cap, kmax, kmin,
@@ -409,7 +416,7 @@ ac_status ac_create(const ac_config *cfg, ac_ctx **out) {
     if (!c) return AC_ERR_INVALID_ARG;
     c->cfg = *cfg;
     c->kq_cap = cfg->adaptive_q ? cfg->nmax_q + cfg->kq : cfg->kq;
-    c->kk_cap = cfg->adaptive_k ? cfg->nmax_k + cfg->kk : cfg->kk;
+    c->kk_cap = (cfg->adaptive_k ? cfg->nmax_k + cfg->kk : cfg->kk) + (cfg->text_keys > 0 ? 1 : 0);
     c->cap_max = c->kq_cap > c->kk_cap ? c->kq_cap : c->kk_cap;
     c->elt = cfg->dtype == AC_BF16 ? 2 : 4;
     if (c->cap_max > 8192) {
@@ -601,8 +608,9 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
         kbmin = at<float>(ws, w.kbmin);
         key_bounds(c, k, ka, nk, kbmax, kbmin, ws, st);
     }
-    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk, dense,
-             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st);
+    const int tg = g.text_keys > 0 ? 1 : 0;
+    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk + tg, dense,
+             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st, tg);
     if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
     s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
@@ -682,7 +690,8 @@ ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, co
     ac_status s = check_ws(c, ws, ws_bytes);
     if (s != AC_OK) return s;
     k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, k_max, k_min, c->kk_cap, nq, nk,
-             g.kq, g.kk, dense_flag, (int)g.score_mode, g.top_k, g.top_p, sel_idx, sel_cnt, (cudaStream_t)stream);
+             g.kq, g.kk + (g.text_keys > 0 ? 1 : 0), dense_flag, (int)g.score_mode, g.top_k, g.top_p, sel_idx, sel_cnt,
+             (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0);
     return launch_check();
 }
 

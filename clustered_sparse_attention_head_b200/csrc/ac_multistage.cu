@@ -4,7 +4,8 @@
 //
 // Readings of the algorithm (the paper leaves these open):
 //  - U starts as all tokens; stage t clusters U into m_t clusters with
-//    m_0 = m0 and m_t = min(|U|, ceil(m0 |U| / N)) for t >= 1.
+//    m_0 = m0 and m_t = min(|U|, ceil(m0 |U| / N)) for t >= 1.  N is the
+//    number of tokens clustered (nrows, the first nrows of each head's N).
 //  - |C| >= N_max is tested before a stage; then F is set and the loop stops.
 //  - A token of U leaves U when its distance to its centre is < tau.
 //  - tau (MEAN_X / MEDIAN_RADIUS_X) is fixed from the first stage.
@@ -15,7 +16,7 @@ namespace ac {
 
 // Both U buffers start as the identity, so every entry is a valid token id
 // (entries past |U| are never used as members, but row gathers read them).
-__global__ void ms_init_kernel(int H, int N, MsHead *__restrict__ st, int32_t *__restrict__ U,
+__global__ void ms_init_kernel(int H, int N, int nrows, MsHead *__restrict__ st, int32_t *__restrict__ U,
                                int32_t *__restrict__ U2) {
     int h = blockIdx.y;
     int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -26,7 +27,7 @@ __global__ void ms_init_kernel(int H, int N, MsHead *__restrict__ st, int32_t *_
     if (i == 0) {
         MsHead s;
         s.nc = 0;
-        s.nu = N;
+        s.nu = nrows;
         s.stage = 0;
         s.flag = 0;
         s.mt = 0;
@@ -193,7 +194,7 @@ __global__ void ms_remove_kernel(int N, const HeadSeg *__restrict__ seg, const d
 
 // Final pass over all tokens with every centre of C; also publishes
 // nclusters and the flag F.
-__global__ void ms_final_kernel(int H, int N, const MsHead *__restrict__ st, HeadSeg *__restrict__ seg,
+__global__ void ms_final_kernel(int H, int nrows, const MsHead *__restrict__ st, HeadSeg *__restrict__ seg,
                                 int32_t *__restrict__ ncl, uint8_t *__restrict__ flag, int32_t *__restrict__ info) {
     __shared__ int mnc;
     if (threadIdx.x == 0) mnc = 0;
@@ -201,7 +202,7 @@ __global__ void ms_final_kernel(int H, int N, const MsHead *__restrict__ st, Hea
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
         MsHead s = st[h];
         HeadSeg g;
-        g.nrows = s.nc > 0 ? N : 0;
+        g.nrows = s.nc > 0 ? nrows : 0;
         g.k = s.nc;
         g.cent_off = 0;
         g.pad = 0;
@@ -228,22 +229,23 @@ __global__ void seg_uniform_kernel(int H, int nrows, int k, HeadSeg *__restrict_
     if (flag) flag[h] = 0;
 }
 
-// Per-head pass descriptors from device cluster counts (nk may be NULL).
-__global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restrict__ ncl, int kfix,
+// Per-head pass descriptors from device cluster counts (nk may be NULL), less
+// `sub` groups that the pass does not cluster (the text-key group).
+__global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restrict__ ncl, int kfix, int sub,
                                        HeadSeg *__restrict__ seg) {
     int h = blockIdx.x * blockDim.x + threadIdx.x;
     if (h >= H) return;
     HeadSeg g;
     g.nrows = nrows;
-    g.k = ncl ? ncl[h] : kfix;
+    g.k = (ncl ? ncl[h] : kfix) - sub;
     g.cent_off = 0;
     g.pad = 0;
     seg[h] = g;
 }
 
-void k_ms_init(int H, int N, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s) {
+void k_ms_init(int H, int N, int nrows, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s) {
     dim3 g((N + 255) / 256, H);
-    ms_init_kernel<<<g, 256, 0, s>>>(H, N, st, U, U2); note_launch();
+    ms_init_kernel<<<g, 256, 0, s>>>(H, N, nrows, st, U, U2); note_launch();
 }
 void k_ms_control(int H, int N, int m0, int nmax, int cap, MsHead *st, HeadSeg *seg, int32_t *info, int *status,
                   cudaStream_t s) {
@@ -265,15 +267,36 @@ void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int
                  cudaStream_t s) {
     ms_remove_kernel<<<H, 1024, 0, s>>>(N, seg, dist, U, Unext, st); note_launch();
 }
-void k_ms_final(int H, int N, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
+void k_ms_final(int H, int nrows, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
                 cudaStream_t s) {
-    ms_final_kernel<<<1, 256, 0, s>>>(H, N, st, seg, ncl, flag, info); note_launch();
+    ms_final_kernel<<<1, 256, 0, s>>>(H, nrows, st, seg, ncl, flag, info); note_launch();
 }
 void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s) {
     seg_uniform_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, k, seg, ncl, flag); note_launch();
 }
-void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s) {
-    seg_from_counts_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, ncl, kfix, seg); note_launch();
+void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s, int sub) {
+    seg_from_counts_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, ncl, kfix, sub, seg); note_launch();
+}
+
+// The text-key group after key clustering: rows [nrows, N) of every head get
+// id = the head's cluster count (seg.k of the final pass), its count is N -
+// nrows, and the head's cluster count grows by one.
+__global__ void text_group_kernel(int H, int N, int nrows, const HeadSeg *__restrict__ seg, int32_t *__restrict__ assign,
+                                  int32_t *__restrict__ count, int cap, int32_t *__restrict__ ncl) {
+    const int h = blockIdx.y;
+    const int id = seg[h].k;
+    const int i = nrows + blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < N) assign[(size_t)h * N + i] = id;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (count) count[(size_t)h * cap + id] = N - nrows;
+        ncl[h] = id + 1;
+    }
+}
+void k_text_group(int H, int N, int nrows, const HeadSeg *seg, int32_t *assign, int32_t *count, int cap,
+                  int32_t *ncl, cudaStream_t s) {
+    const int T = N - nrows;
+    text_group_kernel<<<dim3((T + 255) / 256, H), 256, 0, s>>>(H, N, nrows, seg, assign, count, cap, ncl);
+    note_launch();
 }
 
 }  // namespace ac

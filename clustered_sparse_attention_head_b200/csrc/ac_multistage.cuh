@@ -14,16 +14,21 @@ struct MsHead {
     double tau;
 };
 
-void k_ms_init(int H, int N, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s);
+// N = row stride of a head; nrows = tokens clustered (the first nrows of each head)
+void k_ms_init(int H, int N, int nrows, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s);
 void k_ms_control(int H, int N, int m0, int nmax, int cap, MsHead *st, HeadSeg *seg, int32_t *info, int *status,
                   cudaStream_t s);
 void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double *dist, const int32_t *perm,
               const int32_t *off, int cap, int kmax, MsHead *st, cudaStream_t s);
 void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int32_t *U, int32_t *Unext, MsHead *st,
                  cudaStream_t s);
-void k_ms_final(int H, int N, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
+void k_ms_final(int H, int nrows, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
                 cudaStream_t s);
 void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s);
-void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s);
+void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s, int sub = 0);
+// The text-key group (ac_config.text_keys): rows [nrows, N) get id seg.k, count
+// N - nrows, and ncl = seg.k + 1.
+void k_text_group(int H, int N, int nrows, const HeadSeg *seg, int32_t *assign, int32_t *count, int cap,
+                  int32_t *ncl, cudaStream_t s);
 
 }  // namespace ac

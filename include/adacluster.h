@@ -104,6 +104,12 @@ typedef struct {
     ac_score_mode score_mode;  /* selection score (zero-initialised: CENTROID)          */
     int top_k;              /* > 0: keep the top_k best-scored key clusters (Algorithm 3
                                line 7, argtopk) instead of the top-p prefix            */
+    int text_keys;          /* > 0: the last text_keys keys of every head (the text
+                               tokens) take no part in key clustering and form one
+                               more key group, id = the head's key cluster count,
+                               that no score ranks and every query cluster selects
+                               (a dense strip).  Not from the pages, which give text
+                               tokens no special treatment; 0 = off.  < n.         */
 } ac_config;
 
 /* Per-call statistics filled by ac_forward when `stats` is non-NULL (the call

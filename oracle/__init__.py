@@ -383,9 +383,12 @@ def _select_attend(q, k, v, rq, rk, qmn, dense, spec: HeadSpec, rows):
         sel, cnt = select2(rq.cent, qmn, rq.count, rk.cent[:nv], rk.count, spec.top_p, spec.score_mode,
                            spec.top_k, kmax, kmin)
         if spec.text_keys:
+            # every non-empty query cluster (an empty one selects nothing)
             sel = np.concatenate([sel, np.full((sel.shape[0], 1), -1, np.int32)], axis=1)
-            sel[np.arange(sel.shape[0]), cnt] = nv
-            cnt = cnt + 1
+            live = np.nonzero(np.asarray(rq.count)[:sel.shape[0]] > 0)[0]
+            sel[live, cnt[live]] = nv
+            cnt = cnt.copy()
+            cnt[live] += 1
     if rows is None:
         rows = np.arange(q.shape[0], dtype=np.int32)
     out = attention_rows(q, k, v, rq.assign, k_assign, nv + (1 if spec.text_keys else 0), sel, cnt, dense, rows)
