@@ -62,8 +62,9 @@ struct Ws {
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
     size_t chi, clo, xu, amb_cand, items_scr, runs, run_info, masks, kbmax, kbmin;
-    // early stop of fixed-count k-means: previous assignment, per-head record (q, k)
-    size_t aprev, kst;
+    // early stop of k-means: previous assignment, per-head records (q, k, Algorithm 1
+    // stages), a copy of a stage's pass descriptors
+    size_t aprev, kst, seg2;
     int kpad;
     size_t total;
 };
@@ -130,7 +131,8 @@ Ws layout(const ac_ctx *c) {
     w.kbmax = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
     w.kbmin = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
     w.aprev = b.take(HN * 4);
-    w.kst = b.take(2 * H * 4 * 4);
+    w.kst = b.take(3 * H * 4 * 4);
+    w.seg2 = b.take(H * sizeof(HeadSeg));
     w.total = b.off;
     return w;
 }
@@ -281,12 +283,22 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         k_init_cent(x, dt, H, N, D, U, norm, seg, mmt, mode, cent, cap, st);
         void *xu = at<void>(ws, w.xu);
         if (dt == DT_BF16) k_gather_rows(x, xu, U, H, N, D * c->elt, st);
+        // the stage's k-means stops per head like the fixed-count one (a
+        // repeated assignment is a fixed point); the stage's pass descriptors
+        // are kept and put back for the steps after it
+        HeadSeg *seg_keep = at<HeadSeg>(ws, w.seg2);
+        int32_t *kst = at<int32_t>(ws, w.kst) + 8 * H;
+        int32_t *prev = at<int32_t>(ws, w.aprev);
+        if (g.iters > 0) AC_CUDA(cudaMemcpyAsync(seg_keep, seg, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));
         for (int it = 0; it < g.iters; it++) {
             AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
+            k_conv_check(H, N, seg, pa, prev, kst, it == 0 ? 1 : 0, st);
+            k_conv_decide(H, seg, kst, it, st);
             k_sort(pa, U, seg, H, N, mnu, cap, rank, hist, cnt, off, perm, status, st);
             k_update(x, dt, H, N, D, seg, mmt, perm, off, cap, norm, mode, cent, st);
         }
         AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
+        if (g.iters > 0) AC_CUDA(cudaMemcpyAsync(seg, seg_keep, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));
         k_dist(x, dt, H, N, D, U, seg, mnu, cent, cap, norm, mode, pa, dist, st);
         if (t == 0) {
             if (g.tau_rule == AC_TAU_MEDIAN_RADIUS_X)
