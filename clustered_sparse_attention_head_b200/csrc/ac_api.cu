@@ -65,6 +65,8 @@ struct Ws {
     // early stop of k-means: previous assignment, per-head records (q, k, Algorithm 1
     // stages), a copy of a stage's pass descriptors
     size_t aprev, kst, seg2;
+    // selection: the key centroids transposed per head
+    size_t kct;
     int kpad;
     size_t total;
 };
@@ -133,6 +135,7 @@ Ws layout(const ac_ctx *c) {
     w.aprev = b.take(HN * 4);
     w.kst = b.take(3 * H * 4 * 4);
     w.seg2 = b.take(H * sizeof(HeadSeg));
+    w.kct = b.take(H * (size_t)c->kk_cap * D * 4);
     w.total = b.off;
     return w;
 }
@@ -622,7 +625,7 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
     }
     const int tg = g.text_keys > 0 ? 1 : 0;
     k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk + tg, dense,
-             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st, tg);
+             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st, tg, at<float>(ws, w.kct));
     if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
     s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
@@ -703,7 +706,7 @@ ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, co
     if (s != AC_OK) return s;
     k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, k_max, k_min, c->kk_cap, nq, nk,
              g.kq, g.kk + (g.text_keys > 0 ? 1 : 0), dense_flag, (int)g.score_mode, g.top_k, g.top_p, sel_idx, sel_cnt,
-             (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0);
+             (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0, at<float>(ws, layout(c).kct));
     return launch_check();
 }
 

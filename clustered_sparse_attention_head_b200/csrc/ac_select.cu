@@ -15,18 +15,39 @@
 
 namespace ac {
 
+// Key centroids transposed per head, [kk_cap, D] -> [D, kk_cap], so that the
+// selection's per-thread dot products read consecutive addresses across a warp.
+__global__ void transpose_cent_kernel(const float *__restrict__ src, int rows, int D, float *__restrict__ dst) {
+    __shared__ float tile[32][33];
+    const int h = blockIdx.z;
+    const float *s = src + (size_t)h * rows * D;
+    float *d = dst + (size_t)h * rows * D;
+    const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < D) tile[i][threadIdx.x] = s[(size_t)r * D + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < rows && c < D) d[(size_t)c * rows + r] = tile[threadIdx.x][i];
+    }
+}
+
 __global__ void select_kernel(int D, const float *__restrict__ q_cent, const float *__restrict__ q_mean_norm,
                               const int32_t *__restrict__ q_count, int kq_cap, const float *__restrict__ k_cent,
                               const int32_t *__restrict__ k_count, const float *__restrict__ k_max,
                               const float *__restrict__ k_min, int kk_cap, const int32_t *__restrict__ nq,
                               const int32_t *__restrict__ nk, int kq_fixed, int kk_fixed,
                               const uint8_t *__restrict__ dense, int score_mode, int top_k, double top_p, int n2,
-                              int text_group, int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_cnt) {
+                              int text_group, const float *__restrict__ k_cent_t, int32_t *__restrict__ sel_idx,
+                              int32_t *__restrict__ sel_cnt) {
     extern __shared__ __align__(16) unsigned char smraw[];
     double *sp = reinterpret_cast<double *>(smraw);          // [n2] p (sort key)
     int *sb = reinterpret_cast<int *>(sp + n2);             // [n2] b
     double *sw = reinterpret_cast<double *>(sb + n2);        // [kk_cap] weights
-    unsigned char *keep = reinterpret_cast<unsigned char *>(sw + kk_cap);  // [kk_cap]
+    int *skn = reinterpret_cast<int *>(sw + kk_cap);          // [kk_cap] key cluster sizes
+    unsigned char *keep = reinterpret_cast<unsigned char *>(skn + kk_cap);  // [kk_cap]
     __shared__ double mu[128];
     __shared__ double qpos[128], qneg[128];
     __shared__ double red[32];
@@ -44,7 +65,9 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
         return;
     }
     const float *kc = k_cent + (size_t)h * kk_cap * D;
-    const int32_t *kn = k_count + (size_t)h * kk_cap;
+    const float *kct = k_cent_t ? k_cent_t + (size_t)h * kk_cap * D : nullptr;  // [D, kk_cap]
+    const int *kn = skn;
+    for (int b = tid; b < kk_cap; b += nt) skn[b] = k_count[(size_t)h * kk_cap + b];
     const double rbar = (double)q_mean_norm[(size_t)h * kq_cap + a];
     for (int t = tid; t < D; t += nt) {
         mu[t] = (double)q_cent[((size_t)h * kq_cap + a) * D + t];
@@ -72,9 +95,13 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
                     acc = dadd(acc, dadd(dmul(qpos[t], (double)M[t]), dmul(qneg[t], (double)mn[t])));
                 s = dmul(acc, scale);
             } else {
-                const float *c = kc + (size_t)b * D;
                 double dot = 0.0;
-                for (int t = 0; t < D; t++) dot = dadd(dot, dmul(mu[t], (double)c[t]));
+                if (kct) {
+                    for (int t = 0; t < D; t++) dot = dadd(dot, dmul(mu[t], (double)kct[(size_t)t * kk_cap + b]));
+                } else {
+                    const float *c = kc + (size_t)b * D;
+                    for (int t = 0; t < D; t++) dot = dadd(dot, dmul(mu[t], (double)c[t]));
+                }
                 s = dmul(dmul(rbar, dot), scale);
             }
             m = fmax(m, s);
@@ -185,19 +212,28 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
 void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const int32_t *q_count, int kq_cap,
               const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min, int kk_cap,
               const int32_t *nq, const int32_t *nk, int kq_fixed, int kk_fixed, const uint8_t *dense, int score_mode,
-              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st, int text_group) {
+              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st, int text_group,
+              float *k_cent_t) {
     int n2 = 1;
     while (n2 < kk_cap) n2 <<= 1;
-    size_t smem = (size_t)n2 * (sizeof(double) + sizeof(int)) + (size_t)kk_cap * (sizeof(double) + 1);
+    size_t smem = (size_t)n2 * (sizeof(double) + sizeof(int)) + (size_t)kk_cap * (sizeof(double) + sizeof(int) + 1);
+    if (k_cent_t && score_mode == 0) {
+        transpose_cent_kernel<<<dim3((kk_cap + 31) / 32, (D + 31) / 32, H), dim3(32, 8), 0, st>>>(k_cent, kk_cap, D,
+                                                                                                   k_cent_t);
+        note_launch();
+    } else {
+        k_cent_t = nullptr;
+    }
+    // opt in whenever dynamic plus static shared memory may pass 48 KB
     static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
+    if (smem > smem_set) {
         cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         smem_set = smem;
     }
     dim3 g(kq_cap, H);
     select_kernel<<<g, 256, smem, st>>>(D, q_cent, q_mean_norm, q_count, kq_cap, k_cent, k_count, k_max, k_min,
                                         kk_cap, nq, nk, kq_fixed, kk_fixed, dense, score_mode, top_k, top_p, n2,
-                                        text_group, sel_idx, sel_cnt);
+                                        text_group, k_cent_t, sel_idx, sel_cnt);
     note_launch();
 }
 
