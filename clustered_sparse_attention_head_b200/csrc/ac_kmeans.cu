@@ -17,29 +17,37 @@ namespace ac {
 // ---------------------------------------------------------------- row norms
 // norm[h,i] = sqrt(sum_t x_t^2) (double, sequential).  With check_finite,
 // a NaN/Inf element records ST_NONFINITE.
-template <typename T>
-__global__ void row_norm_kernel(const T *__restrict__ x, int N, int D, double *__restrict__ norm, int check,
-                                int *status) {
-    // 64 rows per CTA: coalesced load into shared memory, then one thread per
-    // row sums its squares sequentially in double (the order of a plain loop).
-    __shared__ float tile[64 * 129];
-    const int h = blockIdx.y, r0 = blockIdx.x * 64;
-    const int nr = min(64, N - r0);
-    const T *xb = x + ((size_t)h * N + r0) * D;
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    row_norm_kernel(const T *__restrict__ x, int N, double *__restrict__ norm, int check, int *status) {
+    // One thread per row: 16-byte vector loads, squares summed sequentially in
+    // double in element order (the order of a plain loop).
+    constexpr int PER = 16 / sizeof(T);   // elements per vector
+    constexpr int NV = D / PER;           // vectors per row
+    constexpr int CH = NV < 8 ? NV : 8;   // vectors loaded ahead of the sum
+    const int h = blockIdx.y, r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= N) return;
+    const uint4 *row = reinterpret_cast<const uint4 *>(x + ((size_t)h * N + r) * D);
+    double ss = 0.0;
     bool bad = false;
-    for (int idx = threadIdx.x; idx < nr * D; idx += blockDim.x) {
-        const float v = to_f(xb[idx]);
-        if (check && !isfinite(v)) bad = true;
-        tile[(idx / D) * 129 + (idx % D)] = v;
+#pragma unroll
+    for (int c0 = 0; c0 < NV; c0 += CH) {
+        uint4 v[CH];
+#pragma unroll
+        for (int i = 0; i < CH; i++) v[i] = __ldg(row + c0 + i);
+#pragma unroll
+        for (int i = 0; i < CH; i++) {
+            const T *e = reinterpret_cast<const T *>(&v[i]);
+#pragma unroll
+            for (int u = 0; u < PER; u++) {
+                const float f = to_f(e[u]);
+                if (check && !isfinite(f)) bad = true;
+                ss = dadd(ss, dmul((double)f, (double)f));
+            }
+        }
     }
     if (bad) set_status(status, ST_NONFINITE);
-    __syncthreads();
-    if ((int)threadIdx.x < nr) {
-        const float *row = tile + threadIdx.x * 129;
-        double ss = 0.0;
-        for (int t = 0; t < D; t++) ss = dadd(ss, dmul((double)row[t], (double)row[t]));
-        norm[(size_t)h * N + r0 + threadIdx.x] = sqrt(ss);
-    }
+    norm[(size_t)h * N + r] = sqrt(ss);
 }
 
 // Working value of element t of token tok: x (EUCLID) or x/||x|| (SPHERE).
@@ -336,13 +344,13 @@ __global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__r
         }
         __syncthreads();
         int i = 0;
-        // members in order; 8 independent loads in flight, sums stay sequential
-        for (; i + 8 <= n; i += 8) {
-            double v[8];
+        // members in order; 16 independent loads in flight, sums stay sequential
+        for (; i + 16 <= n; i += 16) {
+            double v[16];
 #pragma unroll
-            for (int u = 0; u < 8; u++) v[u] = (double)to_f(xh[(size_t)toks[i + u] * D + t]);
+            for (int u = 0; u < 16; u++) v[u] = (double)to_f(xh[(size_t)toks[i + u] * D + t]);
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
+            for (int u = 0; u < 16; u++) {
                 const double w = (mode == MODE_SPHERE) ? (nrms[i + u] > 0.0 ? ddiv(v[u], nrms[i + u]) : 0.0) : v[u];
                 acc = dadd(acc, w);
             }
@@ -392,8 +400,10 @@ __global__ void mean_norm_kernel(int N, const HeadSeg *__restrict__ seg, const i
 template <typename T>
 static void launch_row_norm(const void *x, int H, int N, int D, double *norm, int check, int *status,
                             cudaStream_t st) {
-    dim3 g((N + 63) / 64, H);
-    row_norm_kernel<T><<<g, 256, 0, st>>>((const T *)x, N, D, norm, check, status); note_launch();
+    dim3 g((N + 255) / 256, H);
+    if (D == 64) row_norm_kernel<T, 64><<<g, 256, 0, st>>>((const T *)x, N, norm, check, status);
+    else row_norm_kernel<T, 128><<<g, 256, 0, st>>>((const T *)x, N, norm, check, status);
+    note_launch();
 }
 
 void k_row_norm(const void *x, int dtype, int H, int N, int D, double *norm, int check, int *status,
