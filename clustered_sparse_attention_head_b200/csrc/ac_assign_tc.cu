@@ -173,8 +173,9 @@ __global__ void __launch_bounds__(192, 2)
         // shared memory; the four epilogue warps share a named barrier
         float *cn_s = reinterpret_cast<float *>(sm + C::OFF_CN);
         const int kpadc = nch * C::COLS;
+        // padding columns (zero centroid rows, x.c = 0) get +inf, so they never win
         for (int i = threadIdx.x - 64; i < kpadc; i += 128)
-            cn_s[i] = (p.mode == MODE_EUCLID && i < s.k) ? p.cn2[(size_t)h * p.cap + i] : 0.f;
+            cn_s[i] = i >= s.k ? INFINITY : (p.mode == MODE_EUCLID ? p.cn2[(size_t)h * p.cap + i] : 0.f);
         asm volatile("bar.sync 1, 128;" ::: "memory");
         // four running lists (columns col = 4m + q go to list q): best score and
         // index, second best and index, third best score
@@ -205,8 +206,8 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
                         const int col = c0 + 4 * i4 + q;
-                        // EUCLID: ||c||^2 - 2 x.c; SPHERE: -(x.mu); padding columns never win
-                        const float sc = col < s.k ? fmaf(wv, __uint_as_float(r[4 * i4 + q]), cc[q]) : INFINITY;
+                        // EUCLID: ||c||^2 - 2 x.c; SPHERE: -(x.mu); padding columns: +inf
+                        const float sc = fmaf(wv, __uint_as_float(r[4 * i4 + q]), cc[q]);
                         const bool lt1 = sc < b1[q], lt2 = sc < b2[q];
                         b3[q] = fminf(b3[q], fmaxf(sc, b2[q]));
                         b2[q] = fminf(b2[q], fmaxf(sc, b1[q]));
