@@ -1,5 +1,5 @@
-"""The text-key strip (ac_config.text_keys; the survey's variant that tests the
-pages' "no special treatment" reading) through ac_forward against the oracle:
+"""The text-key strip (ac_config.text_keys; a variant, not in the pages, that
+checks their "no special treatment" of text tokens) through ac_forward against the oracle:
 the last text_keys keys are not clustered and every non-empty query cluster
 selects them.  Per head: key clusters and the dense flag exact, key centres
 within 1e-5 relative, the selected lists bit-exact (text group last), attention

@@ -612,7 +612,7 @@ def test_step_inputs_drift(orc):
 
 
 # --------------------------------------------------------------------------
-# Text keys always attended (a dense strip; SURVEY f4 variant, not in the pages)
+# Text keys always attended (a dense strip; a variant, not in the pages)
 # --------------------------------------------------------------------------
 def _with_text(n_video=360, n_text=24, d=16, seed=21):
     rng = np.random.default_rng(seed)
