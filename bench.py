@@ -358,7 +358,7 @@ def main():
         dms = d0.elapsed_time(d1) / 3
         dense = {"impl": "torch.nn.functional.scaled_dot_product_attention", "ms": dms,
                  "tflops": w.dense_flops() / (dms * 1e-3) / 1e12, "speedup_of_clustered_call": dms / ms}
-        # the library's own dense path (Algorithm 3 line 4): every head flagged
+        # the library's own dense path (Algorithm 3's dense branch): every head flagged
         # dense, so the attention kernel takes all N keys of each head
         cq, ck = ac.ac_cluster_q(q), ac.ac_cluster_k(k)
         dflag = torch.ones(w.heads, dtype=torch.uint8, device=dev)

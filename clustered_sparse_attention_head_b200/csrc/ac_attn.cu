@@ -1,5 +1,5 @@
 // Block-sparse exact softmax attention over selected key clusters (AdaCluster,
-// Algorithm 3 line 9; line 4 for dense heads) on sm_100a tensor cores.
+// Algorithm 3's sparse attention; its dense branch for dense heads) on sm_100a tensor cores.
 //
 // Inputs are gathered into cluster order (ac_sort.cu): the rows of query
 // cluster a are contiguous in Qg, the keys/values of key cluster b contiguous

@@ -1,5 +1,5 @@
 // Block-sparse exact softmax attention over selected key clusters (AdaCluster,
-// Algorithm 3 line 9; line 4 for dense heads), bf16 inputs, two query tiles
+// Algorithm 3's sparse attention; its dense branch for dense heads), bf16 inputs, two query tiles
 // per CTA, 128-key chunks.
 //
 // A work item is up to 256 query rows of one query cluster (two 128-row

@@ -1,4 +1,4 @@
-// Critical-cluster selection (AdaCluster, Algorithm 3 lines 6-7): for a query
+// Critical-cluster selection (AdaCluster, Algorithm 3's select step): for a query
 // cluster a, key cluster b is scored either by its centroid against a's
 // centroid (the centroid-based significance estimate of §2.3) or by Quest's
 // page bound (§3.2.3 eq. (1), in TensorQuest's form of eq. (2)).  Then either

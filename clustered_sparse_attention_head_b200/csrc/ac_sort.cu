@@ -1,4 +1,4 @@
-// Cluster-sort permutation and gather (Algorithm 3 line 8, "K* = K[Index]"):
+// Cluster-sort permutation and gather (Algorithm 3, "K* = K[Index]"):
 // a stable counting sort of tokens by cluster id, so every cluster's tokens are
 // contiguous and in increasing token order, then a 16-byte vectorised row
 // gather into cluster order.

@@ -102,8 +102,8 @@ typedef struct {
     double top_p;           /* (0, 1]; >= 1 keeps every non-empty key cluster          */
     unsigned flags;
     ac_score_mode score_mode;  /* selection score (zero-initialised: CENTROID)          */
-    int top_k;              /* > 0: keep the top_k best-scored key clusters (Algorithm 3
-                               line 7, argtopk) instead of the top-p prefix            */
+    int top_k;              /* > 0: keep the top_k best-scored key clusters (Algorithm 3's
+                               argtopk) instead of the top-p prefix                   */
     int text_keys;          /* > 0: the last text_keys keys of every head (the text
                                tokens) take no part in key clustering and form one
                                more key group, id = the head's key cluster count,
@@ -152,7 +152,7 @@ AC_API ac_status ac_capacities(const ac_ctx *ctx, int *kq_cap, int *kk_cap);
 /* Bytes of scratch workspace that every call below needs (one size for all). */
 AC_API ac_status ac_workspace_size(const ac_ctx *ctx, size_t *bytes);
 
-/* Query clustering (§3.1, Algorithm 3 line 1): q_hat = q/||q|| (zero stays
+/* Query clustering (§3.1, Algorithm 3): q_hat = q/||q|| (zero stays
  * zero), then spherical k-means: assign each q_hat to the centroid of largest
  * q_hat.mu (equivalently the closest unit centroid), update mu_j = s_j/||s_j||
  * with s_j the member sum (empty clusters keep their centroid); `iters`
@@ -225,8 +225,8 @@ AC_API ac_status ac_cluster_sort(ac_ctx *ctx, const int32_t *assign, int cap, co
 AC_API ac_status ac_cluster_sort_static(const int32_t *assign, int heads, int n, int cap, const int32_t *ncl,
                                         int32_t *perm, int32_t *offsets, void *stream);
 
-/* Exact softmax attention over the selected key clusters (Algorithm 3 lines
- * 8-9; line 4 for heads with dense_flag = 1):
+/* Exact softmax attention over the selected key clusters (Algorithm 3's gather
+ * and attention; its dense branch for heads with dense_flag = 1):
  *   out_i = sum_{j: assign_k(j) in S(assign_q(i))} softmax_j(q_i.k_j / sqrt(d)) v_j.
  * Tokens are gathered into cluster order internally; rows are written back in
  * token order.  A query whose selected set is empty gets zeros.  lse [H, N]

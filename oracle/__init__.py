@@ -12,7 +12,7 @@ Attention in Video Generation" (§3.3) from its steps:
   2. A_k, C_k, F <- MultiStageClustering(K, tau, N_max)  (§3.2.2, Algorithm 1;
      or plain Euclidean k-means with a fixed count, §3.2.1)
   3. F set -> dense attention; else select critical key clusters per query
-     cluster and attend over their keys only (Algorithm 3 lines 3-9).
+     cluster and attend over their keys only (Algorithm 3, after the clustering).
 
 Parity unpinned: the selection's score/weight reading (centroid-centroid score
 scaled by the cluster's mean query norm, weighted by key-cluster size, top-p
@@ -365,7 +365,7 @@ def forward_steps(steps, spec: HeadSpec, rows=None):
 
 
 def _select_attend(q, k, v, rq, rk, qmn, dense, spec: HeadSpec, rows):
-    """Algorithm 3 lines 6-9 for one head from its two clusterings.  With
+    """Algorithm 3's selection and attention for one head from its two clusterings.  With
     spec.text_keys the text keys form one more key group (id = the number of
     key clusters) that no score ranks and every query cluster selects."""
     nv = rk.nclusters

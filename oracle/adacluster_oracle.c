@@ -17,7 +17,7 @@
  * Cluster selection follows the centroid-centroid reading: score each key cluster
  * by its centroid against the query-cluster centroid, weight by cluster size,
  * keep the smallest top-p prefix (§2.3 names centroid-based significance
- * estimation; Algorithm 3 lines 6-7 is the select step it replaces).  The
+ * estimation; it stands in for the select step of Algorithm 3).  The
  * alternative score is Quest's per-page upper bound (§3.2.3, eq. (1)) of the
  * representative query against each key cluster's per-dimension max/min, and
  * the alternative cut is Algorithm 3's argtopk.
@@ -212,10 +212,10 @@ static int orc_cmp_double(const void *a, const void *b)
 }
 
 /* Algorithm 1 (MultiStageClustering), §3.2.2, with the readings:
- *  - U starts as every token (line 2's "D" is read as K).
+ *  - U starts as every token (the initialisation's "D" is read as K).
  *  - Stage t clusters U into m_t clusters: m_0 = m0, and for t >= 1
  *    m_t = min(|U|, ceil(m0 * |U| / N)) ("choose a moderate number").
- *  - The distance test of lines 11-16 runs over the tokens just clustered
+ *  - The distance test after each stage runs over the tokens just clustered
  *    (the members of U); d_i = ||x_i - c(x_i)||_2 and x_i leaves U when d_i < tau.
  *  - |C| >= N_max is tested at the top of the loop, so the last stage may
  *    overshoot N_max; F is set only by that test.
@@ -336,7 +336,7 @@ void orc_key_bounds(int64_t n, int d, const float *k, const int32_t *assign, int
  *     M_b / m_b the per-dimension maximum / minimum of the keys of b (an upper
  *     bound of qbar . k over every key k of b).
  * Then either
- *   top_k > 0 (Algorithm 3 line 7, argtopk): keep the top_k b of largest s_ab
+ *   top_k > 0 (Algorithm 3's argtopk): keep the top_k b of largest s_ab
  *     (ties: lower b first), or all of them if fewer are non-empty;
  *   else the top-p rule: w_ab = n_b * exp(s_ab - max_b s_ab), p_ab = w_ab / sum_b w_ab
  *     (sum in b order); visit b by p descending (ties: lower b first),
@@ -471,8 +471,8 @@ void orc_cluster_sort(int64_t n, const int32_t *assign, int k, int32_t *perm, in
     free(pos);
 }
 
-/* Exact softmax attention for the listed query rows (Algorithm 3 line 9, or
- * line 4 when dense != 0): row i attends to every key j whose cluster is in
+/* Exact softmax attention for the listed query rows (Algorithm 3's sparse
+ * attention, or its dense branch when dense != 0): row i attends to every key j whose cluster is in
  * the selected set of i's query cluster,
  *   o_i = sum_j exp(s_ij - m_i) v_j / sum_j exp(s_ij - m_i),  s_ij = q_i.k_j / sqrt(d).
  * A row whose selected set holds no key gets zeros.  out is [nrows, d].      */

@@ -172,7 +172,7 @@ def test_multistage_hand_trace(orc):
 
 
 def test_multistage_nmax_sets_flag(orc):
-    """Algorithm 1 lines 5-7: U is non-empty after stage 0 and |C| = 3 >= N_max = 3,
+    """Algorithm 1's N_max test: U is non-empty after stage 0 and |C| = 3 >= N_max = 3,
     so F is set and no further stage runs."""
     x = _four_groups()
     r = orc.multistage(x.astype(np.float64), 3, 10, orc.TAU_ABS, 3.0, 3, orc.EUCLID)
@@ -336,7 +336,7 @@ def test_attention_select_all_is_dense(orc):
 
 
 def test_attention_subset_is_attention_over_subset(orc):
-    """Algorithm 3 lines 8-9: attention over K* = K[Index], V* = V[Index]."""
+    """Algorithm 3's gather and attention: attention over K* = K[Index], V* = V[Index]."""
     rng = np.random.default_rng(2)
     n, d, kq, kk = 400, 16, 6, 9
     q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
@@ -390,7 +390,7 @@ def test_forward_head_top_p_one_is_dense(orc):
 
 
 def test_forward_head_dense_flag(orc):
-    """Algorithm 3 lines 3-4: F set (N_max reached) -> full attention."""
+    """Algorithm 3's dense branch: F set (N_max reached) -> full attention."""
     w = W.small(W.WORKLOADS["gmm16-n2048-d64-f32"], 400)
     h = W.head_inputs(w, 0)
     spec = orc.HeadSpec(kq=8, kk=16, iters=3, top_p=0.5, adaptive_k=True, tau_rule=orc.TAU_ABS,
@@ -401,7 +401,7 @@ def test_forward_head_dense_flag(orc):
 
 
 # --------------------------------------------------------------------------
-# Quest bounds (§3.2.3 eq. (1)) and the argtopk cut (Algorithm 3 line 7)
+# Quest bounds (§3.2.3 eq. (1)) and the argtopk cut (Algorithm 3)
 # --------------------------------------------------------------------------
 def test_key_bounds_are_member_extremes(orc):
     """Per cluster and dimension: the largest / smallest member value (numpy's
