@@ -214,7 +214,7 @@ static int orc_cmp_double(const void *a, const void *b)
 /* Algorithm 1 (MultiStageClustering), §3.2.2, with the readings:
  *  - U starts as every token (the initialisation's "D" is read as K).
  *  - Stage t clusters U into m_t clusters: m_0 = m0, and for t >= 1
- *    m_t = min(|U|, ceil(m0 * |U| / N)) ("choose a moderate number").
+ *    m_t = min(|U|, ceil(m0 * |U| / N)) (the pages only ask for a moderate count).
  *  - The distance test after each stage runs over the tokens just clustered
  *    (the members of U); d_i = ||x_i - c(x_i)||_2 and x_i leaves U when d_i < tau.
  *  - |C| >= N_max is tested at the top of the loop, so the last stage may
