@@ -170,3 +170,41 @@ def test_early_stop_matches_all_rounds(orc):
                 print(f"h{h}/{key}: near-tie in the oracle's run; not compared")
                 continue
             np.testing.assert_allclose(parts[key][h, :kc], r.cent, rtol=CENT_RTOL, atol=1e-7)
+
+
+def test_forward_steps_with_text_keys(orc):
+    """The driver with the text-key strip: the state counts the text group as
+    one more key group, later steps cluster only the video keys with step 0's
+    count and keep selecting the strip."""
+    w0, _ = CASES["bf16-d128-fixed"]
+    w = W.small(W.WORKLOADS["wan21-n75600-h40-d128"], 2400, heads=2, seed=6, kq=23, kk=41, text=96)
+    T = w.text
+    ctx = _ctx(w, text_keys=T)
+    spec = _spec(orc, w, dict(text_keys=T))
+    H, N = w.heads, w.n
+    rows = np.unique(np.concatenate([np.arange(0, N, max(1, N // 97)), [N - 1]])).astype(np.int32)
+    inp = [[W.step_inputs(w, h, s, DRIFT) for s in range(3)] for h in range(H)]
+    ref = [orc.forward_steps([(x.q, x.k, x.v) for x in inp[h]], spec, rows=rows) for h in range(H)]
+    state = ctx.step_state()
+    excused = [False] * H
+    for s in range(3):
+        q, k, v = (to_dev(np.stack([getattr(inp[h][s], a) for h in range(H)]), w.dtype) for a in "qkv")
+        out = ctx.ac_forward_step(s, q, k, v, state)
+        torch.cuda.synchronize()
+        assert ctx.get_status() == 0
+        parts = {kk: t.cpu().numpy() for kk, t in ctx.step_state_parts(state).items()}
+        got = out.float().cpu().numpy()
+        for h in range(H):
+            r = ref[h][s]
+            nv = r.k.nclusters
+            assert int(parts["nk"][h]) == nv + 1, f"step{s}/h{h}: key groups"
+            if excused[h]:
+                continue
+            if s > 0:
+                prev = ref[h][s - 1]
+                if (_kmeans_has_tie(orc, inp[h][s].q, r.q.nclusters, spec.iters, orc.SPHERE, prev.q.cent) or
+                        _kmeans_has_tie(orc, inp[h][s].k[:N - T], nv, spec.iters, orc.EUCLID, prev.k.cent)):
+                    excused[h] = True
+                    continue
+            np.testing.assert_allclose(parts["k_cent"][h, :nv], r.k.cent[:nv], rtol=CENT_RTOL, atol=1e-7)
+            attn_close(got[h][rows], r.out_rows, f"text/step{s}/h{h}/attention")
