@@ -24,7 +24,7 @@ AC_SCORE_CENTROID, AC_SCORE_QUEST = 0, 1
 # every entry point declared in include/adacluster.h
 EXPORTS = ["ac_create", "ac_destroy", "ac_capacities", "ac_workspace_size", "ac_cluster_q", "ac_cluster_k",
            "ac_select", "ac_key_bounds", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_step_state_size", "ac_step_state_parts", "ac_forward_step",
-           "ac_profile_read", "ac_get_status", "ac_status_string"]
+           "ac_profile_read", "ac_get_status", "ac_status_string", "ac_selftest_wait"]
 
 
 class ac_config(ctypes.Structure):
@@ -83,6 +83,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ac_forward_step": ([P, c_int, P, P, P, P, P, POINTER(ac_stats), P, c_size_t, P], c_int),
         "ac_profile_read": ([P, POINTER(ac_profile)], c_int),
         "ac_get_status": ([P, P], c_int),
+        "ac_selftest_wait": ([P, c_double, P], c_int),
         "ac_status_string": ([c_int], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():

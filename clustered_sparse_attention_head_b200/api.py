@@ -177,6 +177,11 @@ class AdaCluster:
             return out, {f: getattr(st, f) for f, _ in _abi.ac_stats._fields_}
         return out
 
+    def selftest_wait(self, seconds=0.2, stream=None):
+        """Runs the bounded-wait diagnostic (a wait that must expire); the next
+        get_status() returns AC_ERR_TIMEOUT."""
+        check("ac_selftest_wait", self.lib.ac_selftest_wait(self._ctx, float(seconds), stream_ptr(stream)))
+
     def step_state(self):
         """A zeroed device buffer for ac_forward_step (counts, flags and centres
         carried from one denoising step to the next)."""

@@ -17,6 +17,7 @@
 using namespace ac;
 
 void ac_or_flags(int H, const uint8_t *a, uint8_t *b, cudaStream_t st);
+void wait_selftest_launch(uint64_t limit_ns, int *status, cudaStream_t st);
 
 static std::atomic<long long> g_launches{0};
 namespace ac {
@@ -816,6 +817,12 @@ ac_status ac_forward_step(ac_ctx *c, int step, const void *q, const void *k, con
     return launch_check();
 }
 
+ac_status ac_selftest_wait(ac_ctx *c, double seconds, void *stream) {
+    if (!c || !(seconds > 0.0) || seconds > 10.0) return AC_ERR_INVALID_ARG;
+    wait_selftest_launch((uint64_t)(seconds * 1e9), c->d_status, (cudaStream_t)stream);
+    return launch_check();
+}
+
 ac_status ac_get_status(ac_ctx *c, void *stream) {
     if (!c) return AC_ERR_INVALID_ARG;
     AC_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
@@ -827,9 +834,28 @@ ac_status ac_get_status(ac_ctx *c, void *stream) {
 
 }  // extern "C"
 
+// One warp waits, through the kernels' bounded wait, on an mbarrier phase that
+// nothing completes; the wait gives up after limit_ns and records ST_TIMEOUT.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, int *status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ac::mbar_init(&bar, 1);
+        abort_flag = 0;
+        ac::fence_mbar_init();
+    }
+    __syncthreads();
+    const bool done = ac::mbar_wait_warp(&bar, 0, &abort_flag, status, limit_ns);
+    if (done && threadIdx.x == 0) ac::set_status(status, ac::ST_OK);  // unreachable: nothing arrives
+}
+
 __global__ void or_flags_kernel(int H, const uint8_t *a, uint8_t *b) {
     int h = blockIdx.x * blockDim.x + threadIdx.x;
     if (h < H) b[h] = (uint8_t)(a[h] | b[h]);
+}
+void wait_selftest_launch(uint64_t limit_ns, int *status, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, status);
+    note_launch();
 }
 void ac_or_flags(int H, const uint8_t *a, uint8_t *b, cudaStream_t st) {
     or_flags_kernel<<<(H + 127) / 128, 128, 0, st>>>(H, a, b); note_launch();

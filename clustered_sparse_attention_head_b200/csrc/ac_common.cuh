@@ -96,14 +96,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // completed phase then costs one try_wait and one vote (~17 cycles on B200);
 // a per-lane loop followed by a vote cost ~80.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                               int *status) {
+                                               int *status, uint64_t limit_ns = kWaitLimitNs) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     const uint64_t t0 = gtimer();
     for (uint32_t i = 1;; ++i) {
         if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
         if ((i & 31u) == 0) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
-            const int late = __shfl_sync(0xffffffffu, gtimer() - t0 > kWaitLimitNs ? 1 : 0, 0);
+            const int late = __shfl_sync(0xffffffffu, gtimer() - t0 > limit_ns ? 1 : 0, 0);
             if (late) {
                 if ((threadIdx.x & 31) == 0) {
                     *abort_flag = 1;

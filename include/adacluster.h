@@ -279,6 +279,13 @@ AC_API ac_status ac_forward_step(ac_ctx *ctx, int step, const void *q, const voi
  * record.  Events are recorded on the stream each ac_forward call used. */
 AC_API ac_status ac_profile_read(ac_ctx *ctx, ac_profile *out);
 
+/* Diagnostic of the failure path: one warp waits, through the bounded wait
+ * every kernel of this library uses, on a barrier phase that nothing
+ * completes.  The wait gives up after `seconds` (0 < seconds <= 10) and
+ * records AC_ERR_TIMEOUT, which the next ac_get_status returns; the context
+ * stays usable.  No fault, no hang.  AC_ERR_INVALID_ARG for a bad `seconds`. */
+AC_API ac_status ac_selftest_wait(ac_ctx *ctx, double seconds, void *stream);
+
 /* Synchronise `stream`, return the first device-side error recorded since the
  * last call (AC_OK if none) and clear it. */
 AC_API ac_status ac_get_status(ac_ctx *ctx, void *stream);
