@@ -7,23 +7,34 @@
 // 128-row tile of X against 128-centroid chunks with tcgen05.mma (both parts
 // accumulate into one fp32 TMEM tile; bf16 x bf16 products are exact).  The
 // four epilogue warps (one row per thread) read the tile from TMEM and keep
-// each row's best score, its index and the second-best score:
-//   EUCLID: ||c||^2 - 2 x.c        SPHERE: -(x.mu)   (smaller is closer)
+// each row's three smallest scores, shifted by a per-row constant:
+//   EUCLID: ||c||^2 - 2 x.c + ||x||^2     SPHERE: ||x|| - x.mu
+// (smaller is closer).  Each score travels as a packed key, its low mantissa
+// bits replaced by the column index, so a min/max network on keys alone
+// tracks the indices too; the packing adds at most 2^(kb-22) |key| to the
+// error of a score (kb index bits).
 // Error bound of a dot product: |x.r| <= 2^-18 ||x|| ||c|| plus fp32
 // accumulation of 2d exact products, <= 2d 2^-23 ||x|| ||c||; the pass uses
 // E_dot = 2^-13 ||x|| Cmax (>= 2x that bound for d <= 128).  A row whose best
-// two scores are within 2E goes to the exact double pass (assign_exact_kernel),
-// so the final decision equals the exact one.
+// two keys are within 2E plus the packing bounds goes to the exact double
+// pass (assign_exact_kernel), so the final decision equals the exact one.
 //
 // Warp 0 issues TMA (X tile once, then C_hi/C_lo chunks), warp 1 issues the
 // MMAs into two TMEM accumulators (double buffer; whole warp, one elected
 // lane), warps 2-5 run the epilogue.  The epilogue keeps four independent
-// running top-3 lists per row (columns interleaved four ways, branch-free
-// updates) and merges them at the end: one serial list per row made the
-// kernel latency-bound.  All waits are bounded.
+// running top-3 lists per row (column pairs interleaved four ways, each pair
+// merged into a list with two 3-input mins) and merges them at the end: one
+// serial list per row made the kernel latency-bound, and separate index
+// selects made it bound by the ALU pipe.  All waits are bounded.
 #include "ac_kernels.cuh"
 
 namespace ac {
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float m;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+    return m;
+}
 
 template <int D> struct TcCfg {
     static constexpr int ROWS = 128, COLS = 128;
@@ -173,20 +184,33 @@ __global__ void __launch_bounds__(192, 2)
         // shared memory; the four epilogue warps share a named barrier
         float *cn_s = reinterpret_cast<float *>(sm + C::OFF_CN);
         const int kpadc = nch * C::COLS;
-        // padding columns (zero centroid rows, x.c = 0) get +inf, so they never win
+        // padding columns (zero centroid rows, x.c = 0) get a large finite
+        // score, so their keys stay ordered numbers that never win
         for (int i = threadIdx.x - 64; i < kpadc; i += 128)
-            cn_s[i] = i >= s.k ? INFINITY : (p.mode == MODE_EUCLID ? p.cn2[(size_t)h * p.cap + i] : 0.f);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // four running lists (columns col = 4m + q go to list q): best score and
-        // index, second best and index, third best score
-        float b1[4], b2[4], b3[4];
-        int i1[4], i2[4];
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            b1[q] = b2[q] = b3[q] = INFINITY;
-            i1[q] = 0;
-            i2[q] = -1;
+            cn_s[i] = i >= s.k ? 1e30f : (p.mode == MODE_EUCLID ? p.cn2[(size_t)h * p.cap + i] : 0.f);
+        // this thread's row: ||x|| (rounded up) and the per-row shift
+        // sigma = ||x||^2 (EUCLID) or ||x|| (SPHERE), which turns the scores
+        // into ||x - c||^2 resp. ||x|| (1 - cos), small for the nearest centroids
+        const int pos = r0 + row;
+        const bool live = pos < s.nrows;
+        float xn = 0.f;
+        if (live) {
+            const int tok = p.rows ? p.rows[(size_t)h * p.N + pos] : pos;
+            xn = (float)(p.norm[(size_t)h * p.N + tok] * (1.0 + 1e-6));
         }
+        const float sigma = (p.mode == MODE_EUCLID) ? xn * xn : xn;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // Packed keys: the shifted score with its low kb mantissa bits replaced
+        // by the column index (kb = bits of the largest column).  min/max of
+        // keys then carries the index along, and a key differs from its score
+        // by less than 2^(kb-23) of its magnitude.  Four running top-3 lists of
+        // keys (column pairs 2m, 2m+1 go to list m mod 4), updated a pair at a
+        // time by merging the sorted pair into the sorted triple.
+        const int kb = 32 - __clz(kpadc - 1);
+        const uint32_t imask = (1u << kb) - 1u;
+        float b1[4], b2[4], b3[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) b1[q] = b2[q] = b3[q] = INFINITY;
         const float wv = (p.mode == MODE_EUCLID) ? -2.f : -1.f;
         bool ok = true;
         for (int j = 0; j < nch; j++) {
@@ -198,68 +222,63 @@ __global__ void __launch_bounds__(192, 2)
                 uint32_t r[32];
                 tmem_ld32(tmem + lane_addr + b * C::COLS + pc * 32, r);
                 const int c0 = j * C::COLS + pc * 32;
+                // 2^23 + c0: adding the in-group offset gives a float whose low
+                // mantissa bits are the column index
+                const float cbase = __uint_as_float(0x4B000000u + (uint32_t)c0);
                 const float4 *cn4 = reinterpret_cast<const float4 *>(cn_s + c0);
 #pragma unroll
-                for (int i4 = 0; i4 < 8; i4++) {
-                    const float4 cv = cn4[i4];
-                    const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+                for (int i8 = 0; i8 < 4; i8++) {
+                    const float4 ca = cn4[2 * i8], cb = cn4[2 * i8 + 1];
+                    const float cc[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                    float key[8];
+#pragma unroll
+                    for (int e = 0; e < 8; e++) {
+                        // EUCLID: ||c||^2 - 2 x.c + ||x||^2; SPHERE: ||x|| - x.mu
+                        const float d = __fadd_rn(fmaf(wv, __uint_as_float(r[8 * i8 + e]), cc[e]), sigma);
+                        const float ci = __fadd_rn(cbase, (float)(8 * i8 + e));
+                        key[e] = __uint_as_float((__float_as_uint(d) & ~imask) | (__float_as_uint(ci) & imask));
+                    }
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
-                        const int col = c0 + 4 * i4 + q;
-                        // EUCLID: ||c||^2 - 2 x.c; SPHERE: -(x.mu); padding columns: +inf
-                        const float sc = fmaf(wv, __uint_as_float(r[4 * i4 + q]), cc[q]);
-                        const bool lt1 = sc < b1[q], lt2 = sc < b2[q];
-                        b3[q] = fminf(b3[q], fmaxf(sc, b2[q]));
-                        b2[q] = fminf(b2[q], fmaxf(sc, b1[q]));
-                        i2[q] = lt1 ? i1[q] : (lt2 ? col : i2[q]);
-                        i1[q] = lt1 ? col : i1[q];
-                        b1[q] = fminf(b1[q], sc);
+                        const float lo = fminf(key[2 * q], key[2 * q + 1]);
+                        const float hi = fmaxf(key[2 * q], key[2 * q + 1]);
+                        const float m11 = fmaxf(b1[q], lo), m21 = fmaxf(b2[q], lo), m12 = fmaxf(b1[q], hi);
+                        b3[q] = fmin3(b3[q], m21, m12);
+                        b2[q] = fmin3(b2[q], m11, hi);
+                        b1[q] = fminf(b1[q], lo);
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(d_empty + b);
         }
-        // merge lists 1-3 into list 0 (ties: the lower column index wins)
+        // merge lists 1-3 into list 0 (keys are distinct, so no ties)
         float B1 = b1[0], B2 = b2[0], B3 = b3[0];
-        int I1 = i1[0], I2 = i2[0];
 #pragma unroll
         for (int q = 1; q < 4; q++) {
-            const float cs[3] = {b1[q], b2[q], b3[q]};
-            const int ci[3] = {i1[q], i2[q], 0x7fffffff};
-#pragma unroll
-            for (int e = 0; e < 3; e++) {
-                const float sc = cs[e];
-                const int col = ci[e];
-                const bool lt1 = sc < B1 || (sc == B1 && col < I1);
-                const bool lt2 = sc < B2 || (sc == B2 && col < I2);
-                B3 = fminf(B3, lt2 ? B2 : sc);
-                if (lt1) {
-                    B2 = B1;
-                    I2 = I1;
-                    B1 = sc;
-                    I1 = col;
-                } else if (lt2) {
-                    B2 = sc;
-                    I2 = col;
-                }
-            }
+            const float a1 = B1, a2 = B2, a3 = B3;
+            B1 = fminf(a1, b1[q]);
+            B2 = fmin3(a2, b2[q], fmaxf(a1, b1[q]));
+            B3 = fminf(fmin3(a3, b3[q], fmaxf(a2, b1[q])), fmaxf(a1, b2[q]));
         }
-        const float b1v = B1, b2v = B2, b3v = B3;
-        const int i1v = I1, i2v = I2;
-        const int pos = r0 + row;
-        if (ok && pos < s.nrows) {
-            const int tok = p.rows ? p.rows[(size_t)h * p.N + pos] : pos;
-            const float xn = (float)(p.norm[(size_t)h * p.N + tok] * (1.0 + 1e-6));
+        const int i1v = (int)(__float_as_uint(B1) & imask), i2v = (int)(__float_as_uint(B2) & imask);
+        if (ok && live) {
             const float cm = p.cmax[h];
             const float edot = 1.220703125e-4f * xn * cm;  // 2^-13 ||x|| Cmax
             const float E = (p.mode == MODE_EUCLID) ? 2.f * edot + 2.384185791e-7f * (cm * cm + 2.f * xn * cm) : edot;
-            if (s.k > 1 && !(b2v - b1v > 2.f * E)) {
-                // Every centroid other than i1 and i2 scores >= b3; if b3 > b1 + 2E
-                // none of them can be the exact winner, so only the two are re-scored.
+            // a key is within 2^(kb-23) |key| (1 + tiny) of the shifted fp32
+            // score, and the shift itself rounds to 2^-24 of it: 2^(kb-22)
+            // bounds both.  The bound on exact - key grows with the key, so the
+            // second key is the binding competitor of the first.
+            const float rho = __uint_as_float((uint32_t)(127 + kb - 22) << 23);
+            const bool decided = B2 - B1 > 2.f * E + rho * (fabsf(B1) + fabsf(B2));
+            if (s.k > 1 && !decided) {
+                // Every centroid other than i1 and i2 has a key >= B3; if even
+                // B3 is out of reach of B1, only the two are re-scored.
+                const bool two = B3 - B1 > 2.f * E + rho * (fabsf(B1) + fabsf(B3));
                 const int slot = atomicAdd(&p.amb_count[h], 1);
                 p.amb_list[(size_t)h * p.N + slot] = pos;
-                p.amb_cand[(size_t)h * p.N + slot] = (b3v - b1v > 2.f * E) ? make_int2(i1v, i2v) : make_int2(-1, -1);
+                p.amb_cand[(size_t)h * p.N + slot] = two ? make_int2(i1v, i2v) : make_int2(-1, -1);
             } else {
                 p.assign[(size_t)h * p.N + pos] = i1v;
             }
