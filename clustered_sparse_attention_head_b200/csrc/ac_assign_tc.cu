@@ -15,9 +15,10 @@
 // error of a score (kb index bits).
 // Error bound of a dot product: |x.r| <= 2^-18 ||x|| ||c|| plus fp32
 // accumulation of 2d exact products, <= 2d 2^-23 ||x|| ||c||; the pass uses
-// E_dot = 2^-13 ||x|| Cmax (>= 2x that bound for d <= 128).  A row whose best
-// two keys are within 2E plus the packing bounds goes to the exact double
-// pass (assign_exact_kernel), so the final decision equals the exact one.
+// E_dot = 2^-13 ||x|| Cmax (>= 2x that bound for d <= 128), plus an absolute
+// 2^-100 for fp32 underflow.  A row whose best two keys are within 2E plus the
+// packing bounds goes to the exact double pass (assign_exact_kernel), so the
+// final decision equals the exact one.
 //
 // Warp 0 issues TMA (X tile once, then C_hi/C_lo chunks), warp 1 issues the
 // MMAs into two TMEM accumulators (double buffer; whole warp, one elected
@@ -265,7 +266,10 @@ __global__ void __launch_bounds__(192, 2)
         if (ok && live) {
             const float cm = p.cmax[h];
             const float edot = 1.220703125e-4f * xn * cm;  // 2^-13 ||x|| Cmax
-            const float E = (p.mode == MODE_EUCLID) ? 2.f * edot + 2.384185791e-7f * (cm * cm + 2.f * xn * cm) : edot;
+            // + 2^-100: absolute slack for fp32 underflow (subnormal products and
+            // sums in the MMA, subnormal keys), where relative bounds fail
+            const float E = ((p.mode == MODE_EUCLID) ? 2.f * edot + 2.384185791e-7f * (cm * cm + 2.f * xn * cm) : edot) +
+                            0x1p-100f;
             // a key is within 2^(kb-23) |key| (1 + tiny) of the shifted fp32
             // score, and the shift itself rounds to 2^-24 of it: 2^(kb-22)
             // bounds both.  The bound on exact - key grows with the key, so the

@@ -107,9 +107,9 @@ __global__ void cent_prep_kernel(const float *__restrict__ cent, int cap, int D,
 //   of x_hat.mu equals that of x.mu since ||x|| > 0; zero rows tie everywhere).
 // Each score is within E of its exact value, E = (D+8) 2^-23 (2||x|| Cmax +
 // Cmax^2) for EUCLID and (D+8) 2^-23 ||x|| Cmax for SPHERE (twice the standard
-// bound for a length-D fp32 dot product, plus the final combination).  A row
-// whose best two scores are more than 2E apart has a certain winner; the
-// others go to the exact pass.
+// bound for a length-D fp32 dot product, plus the final combination), plus an
+// absolute 2^-100 for underflow.  A row whose best two scores are more than 2E
+// apart has a certain winner; the others go to the exact pass.
 constexpr int SCR_ROWS = 128, SCR_COLS = 64, SCR_XS = SCR_ROWS + 4, SCR_CS = SCR_COLS + 4;
 
 template <typename T, int D>
@@ -223,8 +223,10 @@ __global__ void __launch_bounds__(256) assign_screen_kernel(
             }
             float xn = xn_row;
             float cm = cmax[h];
-            float E = (float)(D + 8) * 1.1920929e-7f *
-                      ((mode == MODE_EUCLID) ? (2.f * xn * cm + cm * cm) : (xn * cm));
+            // + 2^-100: absolute slack for subnormal products, where the
+            // relative bound fails
+            float E = (float)(D + 8) * 1.1920929e-7f * ((mode == MODE_EUCLID) ? (2.f * xn * cm + cm * cm) : (xn * cm)) +
+                      0x1p-100f;
             if (s.k > 1 && !(B2 - B1 > 2.f * E)) {
                 int slot = atomicAdd(&amb_count[h], 1);
                 amb_list[(size_t)h * N + slot] = pos;
