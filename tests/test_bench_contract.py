@@ -1,0 +1,54 @@
+"""bench.py's output contract, checked on the host.
+
+The reference arm (the CPU oracle timed on a bounded sample) runs without a
+GPU, so its JSON line is checked here in full; the GPU arm must fail loudly
+when no CUDA device is present (there is no CPU fallback)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SMALL = "gmm16-n2048-d64-f32"
+
+
+def _run(args, env=None, timeout=300):
+    e = dict(os.environ)
+    e.update(env or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                          cwd=ROOT, env=e, timeout=timeout)
+
+
+def test_reference_arm_prints_one_complete_line():
+    r = _run(["--impl", "reference", "--workload", SMALL, "--steps", "2", "--warmup", "1"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["unit"] == "calls/s" and j["higher_is_better"] is True
+    assert j["steps"] == 2 and j["warmup"] == 1 and j["value"] > 0
+    assert abs(j["ms_per_step"] - 1e3 / j["value"]) < 1e-6 * j["ms_per_step"]
+    assert j["config"]["workload"] == SMALL
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
+    assert j["e2e"] == {"value": j["value"], "unit": "calls/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run(["--impl", "reference", "--workload", SMALL, "--steps", "1", "--warmup", "0"],
+             env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0 and not r.stdout.strip()
+
+
+def test_gpu_arm_fails_loudly_without_a_device():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    r = _run(["--workload", SMALL, "--steps", "1", "--warmup", "0", "--no-cpu-baseline"])
+    assert r.returncode != 0
+    assert not any(ln.startswith("{") for ln in r.stdout.splitlines())
