@@ -270,13 +270,17 @@ __global__ void __launch_bounds__(256) assign_exact_kernel(
             const int j = cand.x >= 0 ? (q == 0 ? cand.x : cand.y) : q;
             const float *c = ch + (size_t)j * D;
             double acc = 0.0;
+            // partial unrolling: a fully unrolled loop hoists all D loads into
+            // registers and spills; the summation order is unchanged
             if (mode == MODE_EUCLID) {
+#pragma unroll 16
                 for (int t = 0; t < D; t++) {
                     double df = dsub(xs[warp][t], (double)c[t]);
                     acc = dadd(acc, dmul(df, df));
                 }
                 if (acc < best) { best = acc; bj = j; }
             } else {
+#pragma unroll 16
                 for (int t = 0; t < D; t++) acc = dadd(acc, dmul(xs[warp][t], (double)c[t]));
                 if (acc > best) { best = acc; bj = j; }
             }
