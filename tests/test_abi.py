@@ -79,3 +79,45 @@ def test_no_unresolved_internal_symbols(lib):
     """Every internal launcher the entry points call is defined in the library."""
     out = subprocess.run(["nm", "-D", "--undefined-only", lib._name], capture_output=True, text=True).stdout
     assert not [l for l in out.splitlines() if "_ZN2ac" in l], out
+
+
+def _cfg(**over):
+    from clustered_sparse_attention_head_b200 import _abi
+    base = dict(heads=2, n=1000, d=128, dtype=_abi.AC_BF16, kq=10, kk=20, iters=3, adaptive_q=0, adaptive_k=0,
+                tau_rule=_abi.AC_TAU_ABS, tau_value=0.0, nmax_q=0, nmax_k=0, top_p=0.9, flags=0,
+                score_mode=_abi.AC_SCORE_CENTROID, top_k=0, text_keys=0)
+    base.update(over)
+    return _abi.ac_config(**base)
+
+
+@pytest.mark.parametrize("over, code", [
+    (dict(heads=0), "AC_ERR_INVALID_ARG"),
+    (dict(n=0), "AC_ERR_INVALID_ARG"),
+    (dict(iters=-1), "AC_ERR_INVALID_ARG"),
+    (dict(d=32), "AC_ERR_UNSUPPORTED"),
+    (dict(dtype=7), "AC_ERR_INVALID_ARG"),
+    (dict(kq=1001), "AC_ERR_INVALID_ARG"),
+    (dict(kk=1001), "AC_ERR_INVALID_ARG"),
+    (dict(kk=0), "AC_ERR_INVALID_ARG"),
+    (dict(top_p=-0.5), "AC_ERR_INVALID_ARG"),
+    (dict(top_p=float("nan")), "AC_ERR_INVALID_ARG"),
+    (dict(score_mode=9), "AC_ERR_INVALID_ARG"),
+    (dict(top_k=-1), "AC_ERR_INVALID_ARG"),
+    (dict(text_keys=-1), "AC_ERR_INVALID_ARG"),
+    (dict(text_keys=1000), "AC_ERR_INVALID_ARG"),
+    (dict(text_keys=990), "AC_ERR_INVALID_ARG"),          # 10 video keys left for kk = 20 clusters
+    (dict(heads=2 ** 20, n=2 ** 11), "AC_ERR_UNSUPPORTED"),  # H * N beyond the int32 index range
+    (dict(adaptive_q=1, nmax_q=0), "AC_ERR_INVALID_ARG"),
+    (dict(adaptive_k=1, nmax_k=40, tau_rule=5), "AC_ERR_INVALID_ARG"),
+    (dict(adaptive_k=1, nmax_k=40, tau_value=-1.0), "AC_ERR_INVALID_ARG"),
+    (dict(adaptive_k=1, nmax_k=40, tau_value=float("nan")), "AC_ERR_INVALID_ARG"),
+])
+def test_every_config_check(lib, over, code):
+    """Each argument check of ac_create rejects its case on the host, before
+    any device call, and leaves the output handle empty."""
+    from clustered_sparse_attention_head_b200 import _abi
+    L = _abi.load()
+    ctx = ctypes.c_void_p()
+    cfg = _cfg(**over)
+    assert L.ac_create(ctypes.byref(cfg), ctypes.byref(ctx)) == getattr(_abi, code)
+    assert not ctx.value
