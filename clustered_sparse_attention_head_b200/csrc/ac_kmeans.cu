@@ -329,8 +329,8 @@ __global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__r
                               const double *__restrict__ norm, int mode, float *__restrict__ cent) {
     __shared__ double ssum[D];
     __shared__ double snr;
-    __shared__ int toks[256];
-    __shared__ double nrms[256];
+    __shared__ int toks[512];
+    __shared__ double nrms[512];
     int h = blockIdx.y, j = blockIdx.x, t = threadIdx.x;
     HeadSeg s = seg[h];
     if (s.nrows <= 0 || j >= s.k) return;
@@ -340,8 +340,8 @@ __global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__r
     const int32_t *ph = perm + (size_t)h * N;
     const T *xh = x + (size_t)h * N * D;
     double acc = 0.0;
-    for (int r0 = b; r0 < e; r0 += 256) {
-        const int n = min(256, e - r0);
+    for (int r0 = b; r0 < e; r0 += 512) {
+        const int n = min(512, e - r0);
         __syncthreads();
         for (int i = t; i < n; i += D) {
             const int tk = ph[r0 + i];
