@@ -159,7 +159,7 @@ AC_API ac_status ac_workspace_size(const ac_ctx *ctx, size_t *bytes);
  * rounds, then a final assignment.  With adaptive_q, Algorithm 1 runs on q_hat
  * with the chordal distance.  Initial centroids: init_cent [H, kq, d] if non-NULL,
  * else q_hat of tokens floor(j*N/kq).  Outputs assign, cent, count, mean_norm,
- * nclusters, dense_flag (any may not be NULL).                              */
+ * nclusters, dense_flag (none of them may be NULL).                       */
 AC_API ac_status ac_cluster_q(ac_ctx *ctx, const void *q, const float *init_cent, int32_t *assign,
                        float *cent, int32_t *count, float *mean_norm, int32_t *nclusters,
                        uint8_t *dense_flag, void *ws, size_t ws_bytes, void *stream);
