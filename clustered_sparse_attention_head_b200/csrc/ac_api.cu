@@ -284,6 +284,12 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         if (c->h_info[0] == 0) break;
         const int mnu = c->h_info[1], mmt = c->h_info[2];
         stages = t + 1;
+        // A stage whose every active head has one cluster (mmt = 1) is
+        // complete after one round: all its rows are assigned to cluster 0, so
+        // the first update already gives the centre every later round repeats
+        // bit for bit.  Running one round instead of iters skips the repeats'
+        // launches (most stages of a long Algorithm-1 run are such stages).
+        const int iters_t = mmt == 1 ? (g.iters < 1 ? g.iters : 1) : g.iters;
         k_init_cent(x, dt, H, N, D, U, norm, seg, mmt, mode, cent, cap, st);
         void *xu = at<void>(ws, w.xu);
         if (dt == DT_BF16) k_gather_rows(x, xu, U, H, N, D * c->elt, st);
@@ -293,8 +299,8 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         HeadSeg *seg_keep = at<HeadSeg>(ws, w.seg2);
         int32_t *kst = at<int32_t>(ws, w.kst) + 8 * H;
         int32_t *prev = at<int32_t>(ws, w.aprev);
-        if (g.iters > 0) AC_CUDA(cudaMemcpyAsync(seg_keep, seg, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));
-        for (int it = 0; it < g.iters; it++) {
+        if (iters_t > 0) AC_CUDA(cudaMemcpyAsync(seg_keep, seg, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));
+        for (int it = 0; it < iters_t; it++) {
             AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
             k_conv_check(H, N, seg, pa, prev, kst, it == 0 ? 1 : 0, st);
             k_conv_decide(H, seg, kst, it, st);
@@ -302,7 +308,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
             k_update(x, dt, H, N, D, seg, mmt, perm, off, cap, norm, mode, cent, st);
         }
         AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
-        if (g.iters > 0) AC_CUDA(cudaMemcpyAsync(seg, seg_keep, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));
+        if (iters_t > 0) AC_CUDA(cudaMemcpyAsync(seg, seg_keep, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));
         k_dist(x, dt, H, N, D, U, seg, mnu, cent, cap, norm, mode, pa, dist, st);
         if (t == 0) {
             if (g.tau_rule == AC_TAU_MEDIAN_RADIUS_X)
