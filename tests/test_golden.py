@@ -26,7 +26,8 @@ def _load(name):
 def test_every_fixture_is_used():
     names = sorted(os.path.basename(p) for p in glob.glob(os.path.join(GOLDEN, "*.json")))
     assert names == sorted(["attention_two_keys.json", "kmeans_euclid_1d.json", "kmeans_sphere_2d.json",
-                            "multistage_four_groups.json", "select_size_and_score.json"])
+                            "multistage_four_groups.json", "multistage_strict_tau.json",
+                            "select_size_and_score.json"])
 
 
 @pytest.mark.parametrize("name", ["kmeans_euclid_1d.json", "kmeans_sphere_2d.json"])
@@ -49,6 +50,12 @@ def test_kmeans_worked_example(orc, name):
         assert abs(r.trace[-1] - e["objective"]) <= tol["abs"]
     if "mean_norm" in e:
         np.testing.assert_allclose(orc.cluster_mean_norm(nrm, r.assign, g["k"]), e["mean_norm"], atol=tol["abs"])
+    if "expected_iters0" in g:
+        r0 = orc.kmeans(xs, g["k"], 0, mode)
+        e0 = g["expected_iters0"]
+        np.testing.assert_array_equal(r0.assign, e0["assign"])
+        np.testing.assert_array_equal(r0.count, e0["count"])
+        np.testing.assert_allclose(r0.cent, e0["cent"], atol=tol["abs"])
 
 
 def test_attention_worked_example(orc):
@@ -91,3 +98,12 @@ def test_multistage_worked_example(orc):
     n = len(x)
     assert r.assign[n - 2] == r.assign[n - 1] == e["pair_cluster"]
     np.testing.assert_allclose(r.cent[e["pair_cluster"]], e["pair_centre"], atol=g["tolerance"]["abs"])
+
+
+def test_multistage_strict_threshold(orc):
+    g = _load("multistage_strict_tau.json")
+    x = np.array(g["x"], np.float64)
+    r = orc.multistage(x, g["m0"], g["iters"], orc.TAU_ABS, g["tau_abs"], g["nmax"], orc.EUCLID)
+    e = g["expected"]
+    assert (r.nclusters, r.dense, r.nstages) == (e["nclusters"], e["dense"], e["nstages"])
+    np.testing.assert_array_equal(r.cent[:r.nclusters], e["cent"])

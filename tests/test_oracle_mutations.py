@@ -1,0 +1,73 @@
+"""Planted mistakes in the oracle must fail its pins.
+
+Each case copies the oracle and its pin tests to a scratch directory, plants
+one plausible mistake in the C source, and runs the pins (tests/test_oracle_pins.py
+and the worked examples of tests/golden/) against it.  The run must fail: the
+pins are meant to catch a dropped term, a wrong tie rule, a wrong index or
+threshold, a missing normalisation or scale anywhere in the oracle."""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = [
+    ("assign ties to the highest id",
+     "if (mode == ORC_EUCLID ? (s < bs) : (s > bs))", "if (mode == ORC_EUCLID ? (s <= bs) : (s >= bs))"),
+    ("no query normalisation",
+     "xs[i * d + t] = (nr > 0.0) ? (double)xi[t] / nr : 0.0;", "xs[i * d + t] = (double)xi[t];"),
+    ("mean divides by count + 1",
+     "(float)(s[t] / (double)cnt[j])", "(float)(s[t] / (double)(cnt[j] + 1))"),
+    ("spherical update not normalised",
+     "cent[(int64_t)j * d + t] = (float)(s[t] / nr2);", "cent[(int64_t)j * d + t] = (float)(s[t]);"),
+    ("empty cluster zeroed",
+     "if (cnt[j] == 0) continue;",
+     "if (cnt[j] == 0) { for (int t = 0; t < d; t++) cent[(int64_t)j * d + t] = 0.0f; continue; }"),
+    ("initial centroid row shifted by one",
+     "int64_t r = ((int64_t)j * nr) / k;", "int64_t r = (((int64_t)j * nr) / k + 1) % nr;"),
+    ("threshold test not strict",
+     "if (!(dl[r] < tau)) U[keep++] = U[r];", "if (!(dl[r] <= tau)) U[keep++] = U[r];"),
+    ("MEAN_X rule uses the sum", "tau = tau_value * (s / (double)nu);", "tau = tau_value * s;"),
+    ("upper median radius", "tau = tau_value * rs[(m - 1) / 2];", "tau = tau_value * rs[m / 2];"),
+    ("squared distance", "        acc = acc + df * df;\n    }\n    return sqrt(acc);",
+     "        acc = acc + df * df;\n    }\n    return acc;"),
+    ("stage size m0 at every stage", "        if (t == 0) mt = m0;\n        else {", "        if (1) mt = m0;\n        else {"),
+    ("no N_max test", "        if (nc >= nmax) { F = 1; break; }\n", ""),
+    ("no final reassignment",
+     "        orc_assign(mode, n, NULL, d, xs, nc, cent, 0, assign, dist);\n        for (int j = 0; j < nc; j++) count[j] = 0;",
+     "        for (int64_t i = 0; i < n; i++) assign[i] = 0;\n        for (int j = 0; j < nc; j++) count[j] = 0;"),
+    ("selection score without the mean query norm", "return (rbar * dot) * scale;", "return dot * scale;"),
+    ("selection weights without the cluster sizes",
+     "double w = (double)k_count[b] * exp(s[b] - m);", "double w = exp(s[b] - m);"),
+    ("top-p cut strict", "if (top_p < 1.0 && cum >= top_p) break;", "if (top_p < 1.0 && cum > top_p) break;"),
+    ("attention scale 1/d", "        double *o = out + r * d;", "        double *o = out + r * d; scale = 1.0 / (double)d;"),
+]
+
+
+def _copy(dst):
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"),
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    shutil.copytree(os.path.join(ROOT, "clustered_sparse_attention_head_b200"),
+                    os.path.join(dst, "clustered_sparse_attention_head_b200"),
+                    ignore=shutil.ignore_patterns("*.so", "_build", "csrc", "__pycache__"))
+    os.makedirs(os.path.join(dst, "tests"))
+    for f in ("conftest.py", "test_oracle_pins.py", "test_golden.py"):
+        shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(dst, "tests", f))
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(dst, "tests", "golden"))
+
+
+@pytest.mark.parametrize("name, old, new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_fails_a_pin(tmp_path, name, old, new):
+    _copy(str(tmp_path))
+    src = tmp_path / "oracle" / "adacluster_oracle.c"
+    s = src.read_text()
+    assert s.count(old) == 1, f"the mistake's site is no longer unique: {name}"
+    src.write_text(s.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_oracle_pins.py", "tests/test_golden.py"],
+                       cwd=str(tmp_path), capture_output=True, text=True, timeout=600)
+    assert r.returncode not in (0, 5), f"no pin failed with '{name}' planted"
+    assert "FAILED" in r.stdout, f"'{name}': the pins did not fail cleanly:\n{r.stdout[-1500:]}\n{r.stderr[-800:]}"
