@@ -1,7 +1,8 @@
 """Planted mistakes in the oracle must fail its pins.
 
 Each case copies the oracle and its pin tests to a scratch directory, plants
-one plausible mistake in the C source, and runs the pins (tests/test_oracle_pins.py
+one plausible mistake in its C source or its Python composition of the
+steps, and runs the pins (tests/test_oracle_pins.py
 and the worked examples of tests/golden/) against it.  The run must fail: the
 pins are meant to catch a dropped term, a wrong tie rule, a wrong index or
 threshold, a missing normalisation or scale anywhere in the oracle."""
@@ -44,6 +45,19 @@ MUTATIONS = [
      "double w = (double)k_count[b] * exp(s[b] - m);", "double w = exp(s[b] - m);"),
     ("top-p cut strict", "if (top_p < 1.0 && cum >= top_p) break;", "if (top_p < 1.0 && cum > top_p) break;"),
     ("attention scale 1/d", "        double *o = out + r * d;", "        double *o = out + r * d; scale = 1.0 / (double)d;"),
+    ("Quest score keeps only the max-bound term", "acc = acc + (hi > lo ? hi : lo);", "acc = acc + hi;"),
+    ("key lower bound takes the max", "if (x[t] < m[t]) m[t] = x[t];", "if (x[t] > m[t]) m[t] = x[t];"),
+    ("cluster sort not stable", "for (int64_t i = 0; i < n; i++) perm[pos[assign[i]]++] = (int32_t)i;",
+     "for (int64_t i = n - 1; i >= 0; i--) perm[pos[assign[i]]++] = (int32_t)i;"),
+    ("selection ties to the higher id", "return (a->b > b->b) - (a->b < b->b);", "return (a->b < b->b) - (a->b > b->b);"),
+    ("argtopk keeps one too many", "for (int r = 0; r < np && r < top_k; r++) keep[pb[r].b] = 1;",
+     "for (int r = 0; r < np && r <= top_k; r++) keep[pb[r].b] = 1;"),
+    ("later steps not warm-started", "rq = kmeans(xq, nq, spec.iters, SPHERE, init=prev.q.cent[:nq])",
+     "rq = kmeans(xq, nq, spec.iters, SPHERE, init=None)", "__init__.py"),
+    ("text keys clustered", "    if spec.text_keys:\n        k = k[:k.shape[0] - spec.text_keys]\n", "", "__init__.py"),
+    ("text group also for empty query clusters",
+     "live = np.nonzero(np.asarray(rq.count)[:sel.shape[0]] > 0)[0]", "live = np.arange(sel.shape[0])",
+     "__init__.py"),
 ]
 
 
@@ -59,10 +73,12 @@ def _copy(dst):
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(dst, "tests", "golden"))
 
 
-@pytest.mark.parametrize("name, old, new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_planted_mistake_fails_a_pin(tmp_path, name, old, new):
+@pytest.mark.parametrize("mut", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_fails_a_pin(tmp_path, mut):
+    name, old, new = mut[:3]
+    fname = mut[3] if len(mut) > 3 else "adacluster_oracle.c"
     _copy(str(tmp_path))
-    src = tmp_path / "oracle" / "adacluster_oracle.c"
+    src = tmp_path / "oracle" / fname
     s = src.read_text()
     assert s.count(old) == 1, f"the mistake's site is no longer unique: {name}"
     src.write_text(s.replace(old, new))

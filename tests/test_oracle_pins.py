@@ -661,3 +661,39 @@ def test_text_keys_zero_is_unchanged(orc):
     b = orc.forward_head(q, k, v, orc.HeadSpec(kq=6, kk=6, iters=5, top_p=0.5, text_keys=0), rows=rows)
     np.testing.assert_array_equal(a.out_rows, b.out_rows)
     np.testing.assert_array_equal(a.sel_cnt, b.sel_cnt)
+
+
+def test_steps_zero_rounds_keep_the_previous_centres(orc):
+    """With zero k-means rounds a later step's centres are exactly its seeds,
+    the previous step's centres (§3.2.2 "Efficient initialization"), not rows
+    of its own inputs."""
+    steps, lab = _drifting_gmm(3, drift=0.3)
+    spec = orc.HeadSpec(kq=6, kk=6, iters=0, top_p=0.9)
+    res = orc.forward_steps(steps, spec, rows=np.arange(0, len(lab), 9))
+    for r in res[1:]:
+        np.testing.assert_array_equal(r.q.cent, res[0].q.cent)
+        np.testing.assert_array_equal(r.k.cent, res[0].k.cent)
+    # step 0's own seeds are rows of step 0 (strided), which the drift moves
+    xq, _ = orc.prepare(steps[1][0], orc.SPHERE)
+    assert not np.array_equal(res[1].q.cent, orc.init_centroids(xq, 6))
+
+
+def test_text_group_skips_empty_query_clusters(orc):
+    """An empty query cluster selects nothing, not even the text group: with
+    four copies each of two query vectors and kq = 4, the strided seeds are
+    a, a, b, b, every row goes to the lowest tied id, and clusters 1 and 3
+    stay empty."""
+    rng = np.random.default_rng(5)
+    d, T = 8, 3
+    a, b = rng.standard_normal((2, d)).astype(np.float32)
+    q = np.stack([a] * 4 + [b] * 4 + [rng.standard_normal(d).astype(np.float32) for _ in range(T)])
+    q[8:] = np.stack([a] * T)   # text-position queries also copy a
+    k = rng.standard_normal((8 + T, d)).astype(np.float32)
+    v = rng.standard_normal((8 + T, d)).astype(np.float32)
+    spec = orc.HeadSpec(kq=4, kk=2, iters=3, top_p=0.5, text_keys=T)
+    r = orc.forward_head(q, k, v, spec)
+    assert list(r.q.count) == [7, 0, 4, 0]
+    nv = r.k.nclusters
+    assert r.sel_cnt[1] == 0 and r.sel_cnt[3] == 0
+    for c in (0, 2):
+        assert nv in r.sel_idx[c, :r.sel_cnt[c]].tolist()
