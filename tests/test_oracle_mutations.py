@@ -14,6 +14,9 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+# scratch runs in parallel, each oracle with a share of the cores
+WORKERS = max(1, min(8, (os.cpu_count() or 2) // 2))
+THREADS = max(1, (os.cpu_count() or 2) // WORKERS)
 
 MUTATIONS = [
     ("assign ties to the highest id",
@@ -73,17 +76,36 @@ def _copy(dst):
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(dst, "tests", "golden"))
 
 
-@pytest.mark.parametrize("mut", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_planted_mistake_fails_a_pin(tmp_path, mut):
+def _run(base, i, mut):
     name, old, new = mut[:3]
     fname = mut[3] if len(mut) > 3 else "adacluster_oracle.c"
-    _copy(str(tmp_path))
-    src = tmp_path / "oracle" / fname
-    s = src.read_text()
-    assert s.count(old) == 1, f"the mistake's site is no longer unique: {name}"
-    src.write_text(s.replace(old, new))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        "tests/test_oracle_pins.py", "tests/test_golden.py"],
-                       cwd=str(tmp_path), capture_output=True, text=True, timeout=600)
+    dst = os.path.join(base, f"m{i}")
+    _copy(dst)
+    src = os.path.join(dst, "oracle", fname)
+    s = open(src).read()
+    if s.count(old) != 1:
+        return None
+    open(src, "w").write(s.replace(old, new))
+    env = dict(os.environ, OMP_NUM_THREADS=str(THREADS))
+    return subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                           "tests/test_oracle_pins.py", "tests/test_golden.py"],
+                          cwd=dst, capture_output=True, text=True, timeout=600, env=env)
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    """Every planted mistake, run in parallel (one scratch copy each)."""
+    from concurrent.futures import ThreadPoolExecutor
+    base = str(tmp_path_factory.mktemp("mutations"))
+    with ThreadPoolExecutor(WORKERS) as ex:
+        futs = [ex.submit(_run, base, i, m) for i, m in enumerate(MUTATIONS)]
+        return [f.result() for f in futs]
+
+
+@pytest.mark.parametrize("i", range(len(MUTATIONS)), ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_fails_a_pin(outcomes, i):
+    name = MUTATIONS[i][0]
+    r = outcomes[i]
+    assert r is not None, f"the mistake's site is no longer unique: {name}"
     assert r.returncode not in (0, 5), f"no pin failed with '{name}' planted"
     assert "FAILED" in r.stdout, f"'{name}': the pins did not fail cleanly:\n{r.stdout[-1500:]}\n{r.stderr[-800:]}"
