@@ -58,6 +58,14 @@ MUTATIONS = [
     ("later steps not warm-started", "rq = kmeans(xq, nq, spec.iters, SPHERE, init=prev.q.cent[:nq])",
      "rq = kmeans(xq, nq, spec.iters, SPHERE, init=None)", "__init__.py"),
     ("text keys clustered", "    if spec.text_keys:\n        k = k[:k.shape[0] - spec.text_keys]\n", "", "__init__.py"),
+    ("mean query norm is the sum", "mean_norm[j] = c[j] ? (float)(s[j] / (double)c[j]) : 0.0f;",
+     "mean_norm[j] = c[j] ? (float)(s[j]) : 0.0f;"),
+    ("sparse attention over every key",
+     "for (int c = 0; c < sel_cnt[a]; c++) allow[sel_idx[(int64_t)a * kk_stride + c]] = 1;",
+     "for (int c = 0; c < kk; c++) allow[c] = 1;"),
+    ("no final k-means assignment",
+     "    double o = orc_assign(mode, nr, rows, d, xs, k, cent, 0, assign, dist);\n    if (obj_trace) obj_trace[2 * iters] = o;",
+     "    double o = 0.0;\n    if (obj_trace) obj_trace[2 * iters] = o;"),
     ("text group also for empty query clusters",
      "live = np.nonzero(np.asarray(rq.count)[:sel.shape[0]] > 0)[0]", "live = np.arange(sel.shape[0])",
      "__init__.py"),
