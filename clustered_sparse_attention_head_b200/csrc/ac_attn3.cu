@@ -24,6 +24,13 @@
 // the softmax masks the columns past its end (P = 0 there) and the V ring is
 // zeroed once at the start, so the stale V rows behind them are finite.
 //
+// A persistent grid of one CTA per SM takes items dynamically: the TMA warp
+// draws the next item index from a global counter and publishes it in a small
+// shared-memory ring that every other role reads in the same order.  An item
+// of at most 128 query rows splits its key stream between the two tiles (even
+// and odd chunks, see plan_item) and merges the two partial softmax results in
+// the epilogue.
+//
 // The softmax splits its exponentials between the special-function unit
 // (ex2.approx) and the FMA pipe (2^x = 2^n 2^f, n = rint(x), f in [-1/2, 1/2],
 // 2^f by a cubic; Cody and Waite's argument reduction with a polynomial of
