@@ -697,3 +697,24 @@ def test_text_group_skips_empty_query_clusters(orc):
     assert r.sel_cnt[1] == 0 and r.sel_cnt[3] == 0
     for c in (0, 2):
         assert nv in r.sel_idx[c, :r.sel_cnt[c]].tolist()
+
+
+@pytest.mark.parametrize("mode", ["euclid", "sphere"])
+@pytest.mark.parametrize("rule, val", [("abs", 0.9), ("mean", 0.8), ("median", 0.8)])
+def test_single_cluster_stages_are_complete_after_one_round(orc, mode, rule, val):
+    """With m0 = 1 every stage of Algorithm 1 has one cluster.  Such a stage's
+    k-means puts every row in cluster 0, so its first update gives the centre
+    that every later round repeats: one round and ten give identical results
+    (the fact the GPU path uses to run such stages for one round)."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((300, 3)) * np.array([1.0, 0.5, 0.25])).astype(np.float32)
+    m = orc.EUCLID if mode == "euclid" else orc.SPHERE
+    xs, _ = orc.prepare(x, m)
+    r = {"abs": orc.TAU_ABS, "mean": orc.TAU_MEAN_X, "median": orc.TAU_MEDIAN_RADIUS_X}[rule]
+    a = orc.multistage(xs, 1, 1, r, val, 60, m)
+    b = orc.multistage(xs, 1, 10, r, val, 60, m)
+    assert a.nstages > 5, "the case should run many stages"
+    assert (a.nclusters, a.dense, a.nstages, a.tau) == (b.nclusters, b.dense, b.nstages, b.tau)
+    np.testing.assert_array_equal(a.assign, b.assign)
+    np.testing.assert_array_equal(a.count[:a.nclusters], b.count[:b.nclusters])
+    np.testing.assert_array_equal(a.cent[:a.nclusters], b.cent[:b.nclusters])
