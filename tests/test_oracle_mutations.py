@@ -66,6 +66,10 @@ MUTATIONS = [
     ("no final k-means assignment",
      "    double o = orc_assign(mode, nr, rows, d, xs, k, cent, 0, assign, dist);\n    if (obj_trace) obj_trace[2 * iters] = o;",
      "    double o = 0.0;\n    if (obj_trace) obj_trace[2 * iters] = o;"),
+    ("pair count with query and key sizes swapped",
+     "keys += k_count[sel_idx[(int64_t)a * kk_stride + c]];", "keys += q_count[sel_idx[(int64_t)a * kk_stride + c] % kq];"),
+    ("pair count of the last query cluster dropped", "for (int a = 0; a < kq; a++) {\n        int64_t keys = 0;",
+     "for (int a = 0; a < kq - 1; a++) {\n        int64_t keys = 0;"),
     ("text group also for empty query clusters",
      "live = np.nonzero(np.asarray(rq.count)[:sel.shape[0]] > 0)[0]", "live = np.arange(sel.shape[0])",
      "__init__.py"),

@@ -718,3 +718,46 @@ def test_single_cluster_stages_are_complete_after_one_round(orc, mode, rule, val
     np.testing.assert_array_equal(a.assign, b.assign)
     np.testing.assert_array_equal(a.count[:a.nclusters], b.count[:b.nclusters])
     np.testing.assert_array_equal(a.cent[:a.nclusters], b.cent[:b.nclusters])
+
+
+# ------------------------------------------------------------ pair count
+def test_pairs_hand_count(orc):
+    """The pair count of §3.3 (each query of cluster a meets every key of each
+    selected cluster b), counted by hand on an asymmetric case: 3 query clusters
+    of 5, 0 and 2 queries, 4 key clusters of 3, 7, 0 and 11 keys; cluster 0
+    selects {1, 3} (18 keys), the empty cluster 1 nothing, cluster 2 {0, 2}
+    (3 keys).  5 * 18 + 0 + 2 * 3 = 96.  The sizes are unequal on the two
+    sides, so a count that read one side's sizes for the other would differ."""
+    q_count = np.array([5, 0, 2], np.int32)
+    k_count = np.array([3, 7, 0, 11], np.int32)
+    sel = np.full((3, 4), -1, np.int32)
+    sel[0, :2] = [1, 3]
+    sel[2, :2] = [0, 2]
+    sel_cnt = np.array([2, 0, 2], np.int32)
+    assert orc.pairs(q_count, k_count, sel, sel_cnt) == 96
+    # a partial selection of a single cluster: 2 queries x 7 keys
+    sel2 = np.full((3, 4), -1, np.int32)
+    sel2[2, 0] = 1
+    assert orc.pairs(q_count, k_count, sel2, np.array([0, 0, 1], np.int32)) == 14
+
+
+def test_pairs_brute_force_over_tokens(orc):
+    """Brute force over token pairs: count (i, j) with the key's cluster in the
+    query's selected set, from random assignments with empty clusters and
+    unequal query and key counts."""
+    rng = np.random.default_rng(5)
+    nq_tok, nk_tok, kq, kk = 57, 131, 6, 9
+    qa = rng.integers(0, kq - 1, nq_tok)  # cluster kq-1 stays empty
+    ka = rng.integers(1, kk, nk_tok)      # cluster 0 stays empty
+    sel = np.full((kq, kk), -1, np.int32)
+    sel_cnt = np.zeros(kq, np.int32)
+    sets = []
+    for a in range(kq):
+        s = np.sort(rng.choice(kk, rng.integers(0, kk + 1), replace=False)).astype(np.int32)
+        sel[a, :len(s)] = s
+        sel_cnt[a] = len(s)
+        sets.append(set(s.tolist()))
+    brute = sum(1 for i in range(nq_tok) for j in range(nk_tok) if int(ka[j]) in sets[int(qa[i])])
+    q_count = np.bincount(qa, minlength=kq).astype(np.int32)
+    k_count = np.bincount(ka, minlength=kk).astype(np.int32)
+    assert orc.pairs(q_count, k_count, sel, sel_cnt) == brute
