@@ -237,7 +237,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         // per-head counts (kept from an earlier call) or the configured count
         const int kmax = ncl_fixed ? cap : k;
         auto set_seg = [&]() {
-            if (ncl_fixed) k_seg_from_counts(H, Nc, ncl_fixed, k, seg, st, text > 0 ? 1 : 0);
+            if (ncl_fixed) k_seg_from_counts(H, Nc, ncl_fixed, k, cap, seg, status, st, text > 0 ? 1 : 0);
             else k_seg_uniform(H, Nc, k, seg, ncl, flag, st);
         };
         set_seg();
@@ -344,8 +344,8 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     void *qg = at<void>(ws, w.qg), *kg = at<void>(ws, w.kg), *vg = at<void>(ws, w.vg);
     AttnItem *items = at<AttnItem>(ws, w.items);
     int32_t *nitems = at<int32_t>(ws, w.nitems);
-    k_seg_from_counts(H, N, nq, g.kq, sq, st);
-    k_seg_from_counts(H, N, nk, g.kk + (g.text_keys > 0 ? 1 : 0), sk, st);
+    k_seg_from_counts(H, N, nq, g.kq, c->kq_cap, sq, c->d_status, st);
+    k_seg_from_counts(H, N, nk, g.kk + (g.text_keys > 0 ? 1 : 0), c->kk_cap, sk, c->d_status, st);
     k_sort(qa, nullptr, sq, H, N, N, c->kq_cap, rank, hist, cnt, qoff, qperm, c->d_status, st);
     k_sort(ka, nullptr, sk, H, N, N, c->kk_cap, rank, hist, cnt, koff, kperm, c->d_status, st);
     const int rb = D * c->elt;
@@ -354,7 +354,7 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     k_gather_rows(v, vg, kperm, H, N, rb, st);
     const bool two_tiles = (g.dtype == AC_BF16);  // bf16: two query tiles per CTA (items of 256 rows)
     k_build_items(H, N, two_tiles ? 256 : 128, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items,
-                  nitems, pairs_dev, at<int32_t>(ws, w.items_scr), st);
+                  nitems, pairs_dev, at<int32_t>(ws, w.items_scr), c->d_status, st);
     int2 *runs = at<int2>(ws, w.runs), *run_info = at<int2>(ws, w.run_info);
     k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN3_CHUNK, runs, run_info, st);
     const int max_chunks = attn_max_chunks(N, c->kk_cap, ATTN3_CHUNK);
@@ -404,7 +404,7 @@ void key_bounds(ac_ctx *c, const void *k, const int32_t *ka, const int32_t *nk, 
     Ws w = layout(c);
     HeadSeg *sk = at<HeadSeg>(ws, w.segk);
     int32_t *kperm = at<int32_t>(ws, w.kperm), *koff = at<int32_t>(ws, w.koff);
-    k_seg_from_counts(g.heads, g.n, nk, g.kk + (g.text_keys > 0 ? 1 : 0), sk, st);
+    k_seg_from_counts(g.heads, g.n, nk, g.kk + (g.text_keys > 0 ? 1 : 0), c->kk_cap, sk, c->d_status, st);
     k_sort(ka, nullptr, sk, g.heads, g.n, g.n, c->kk_cap, at<int32_t>(ws, w.rank), at<int32_t>(ws, w.hist),
            at<int32_t>(ws, w.cnt2), koff, kperm, c->d_status, st);
     k_cluster_bounds(k, g.dtype == AC_BF16 ? DT_BF16 : DT_F32, g.heads, g.n, g.d, kperm, koff, c->kk_cap, kmax, kmin,
@@ -632,7 +632,7 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
     }
     const int tg = g.text_keys > 0 ? 1 : 0;
     k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk + tg, dense,
-             (int)g.score_mode, g.top_k, g.top_p, sel, selc, st, tg, at<float>(ws, w.kct));
+             (int)g.score_mode, g.top_k, g.top_p, sel, selc, c->d_status, st, tg, at<float>(ws, w.kct));
     if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
     s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
@@ -713,7 +713,7 @@ ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, co
     if (s != AC_OK) return s;
     k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, k_max, k_min, c->kk_cap, nq, nk,
              g.kq, g.kk + (g.text_keys > 0 ? 1 : 0), dense_flag, (int)g.score_mode, g.top_k, g.top_p, sel_idx, sel_cnt,
-             (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0, at<float>(ws, layout(c).kct));
+             c->d_status, (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0, at<float>(ws, layout(c).kct));
     return launch_check();
 }
 
@@ -736,7 +736,7 @@ ac_status ac_cluster_sort(ac_ctx *c, const int32_t *assign, int cap, const int32
     Ws w = layout(c);
     cudaStream_t st = (cudaStream_t)stream;
     HeadSeg *seg = at<HeadSeg>(ws, w.seg);
-    k_seg_from_counts(g.heads, g.n, ncl, cap, seg, st);
+    k_seg_from_counts(g.heads, g.n, ncl, cap, cap, seg, c->d_status, st);
     k_sort(assign, nullptr, seg, g.heads, g.n, g.n, cap, at<int32_t>(ws, w.rank), at<int32_t>(ws, w.hist),
            at<int32_t>(ws, w.cnt), offsets, perm, c->d_status, st);
     return launch_check();

@@ -275,11 +275,14 @@ __global__ void __launch_bounds__(192, 2)
             // bounds both.  The bound on exact - key grows with the key, so the
             // second key is the binding competitor of the first.
             const float rho = __uint_as_float((uint32_t)(127 + kb - 22) << 23);
-            const bool decided = B2 - B1 > 2.f * E + rho * (fabsf(B1) + fabsf(B2));
+            // A winner outside the pass's clusters (a padding column, which
+            // only wins when every real score is NaN, infinite or above the
+            // padding score) is never decided here: the exact pass rescans.
+            const bool decided = B2 - B1 > 2.f * E + rho * (fabsf(B1) + fabsf(B2)) && i1v < s.k;
             if (s.k > 1 && !decided) {
                 // Every centroid other than i1 and i2 has a key >= B3; if even
                 // B3 is out of reach of B1, only the two are re-scored.
-                const bool two = B3 - B1 > 2.f * E + rho * (fabsf(B1) + fabsf(B3));
+                const bool two = B3 - B1 > 2.f * E + rho * (fabsf(B1) + fabsf(B3)) && i1v < s.k && i2v < s.k;
                 const int slot = atomicAdd(&p.amb_count[h], 1);
                 p.amb_list[(size_t)h * p.N + slot] = pos;
                 p.amb_cand[(size_t)h * p.N + slot] = two ? make_int2(i1v, i2v) : make_int2(-1, -1);
@@ -374,11 +377,8 @@ static int launch_tc(const void *xc, int H, int N, const int32_t *rows, const He
         bf16_map(enc, &ml, clo, H * kpad, D, C::COLS))
         return -1;
     if (kpad > 8192) return -1;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem_bytes(8192));
-        attr = true;
-    }
+    // the attribute belongs to the current device: set it on every call
+    cudaFuncSetAttribute(assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem_bytes(8192));
     TcParams p;
     p.N = N;
     p.cap = cap;

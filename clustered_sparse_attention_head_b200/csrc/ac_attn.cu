@@ -494,13 +494,15 @@ __global__ void items_count_kernel(int N, int rpi, int kq_cap, int kk_cap, const
                                    const int32_t *__restrict__ nq, const uint8_t *__restrict__ dense, int kq_fixed,
                                    const int32_t *__restrict__ koff, const int32_t *__restrict__ sel_idx,
                                    const int32_t *__restrict__ sel_cnt, int32_t *__restrict__ tile_off,
-                                   int32_t *__restrict__ head_tiles, unsigned long long *__restrict__ head_pairs) {
+                                   int32_t *__restrict__ head_tiles, unsigned long long *__restrict__ head_pairs,
+                                   int *status) {
     __shared__ int wsum[32];
     __shared__ int carry;
     __shared__ unsigned long long pacc;
     const int h = blockIdx.x, tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, w = tid >> 5;
     const bool dn = dense && dense[h];
-    const int nqh = dn ? 1 : (nq ? nq[h] : kq_fixed);
+    // counts from caller memory are clamped to the capacities (ST_INVALID if not within)
+    const int nqh = dn ? 1 : (nq ? clamp_count(nq[h], kq_cap, tid == 0 ? status : nullptr) : kq_fixed);
     const int32_t *qo = qoff + (size_t)h * (kq_cap + 1);
     const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
     int32_t *to = tile_off + (size_t)h * (kq_cap + 1);
@@ -518,7 +520,7 @@ __global__ void items_count_kernel(int N, int rpi, int kq_cap, int kk_cap, const
             } else if (qn > 0) {
                 long long keys = 0;
                 const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
-                const int ns = sel_cnt[(size_t)h * kq_cap + a];
+                const int ns = clamp_count(sel_cnt[(size_t)h * kq_cap + a], kk_cap, status);
                 for (int c = 0; c < ns; c++) {
                     const int b = sl[c];
                     if (b >= 0 && b < kk_cap) keys += ko[b + 1] - ko[b];
@@ -577,7 +579,7 @@ __global__ void items_write_kernel(int N, int rpi, int kq_cap, const int32_t *__
     const int h = blockIdx.y;
     const int a = blockIdx.x * blockDim.x + threadIdx.x;
     const bool dn = dense && dense[h];
-    const int nqh = dn ? 1 : (nq ? nq[h] : kq_fixed);
+    const int nqh = dn ? 1 : (nq ? clamp_count(nq[h], kq_cap, nullptr) : kq_fixed);
     if (a >= nqh) return;
     const int32_t *qo = qoff + (size_t)h * (kq_cap + 1);
     const int qs = dn ? 0 : qo[a];
@@ -789,14 +791,14 @@ int attn_max_items(int H, int N, int kq_cap) { return H * ((N + 127) / 128 + kq_
 void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
                    const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
-                   cudaStream_t st) {
+                   int *status, cudaStream_t st) {
     int32_t *tile_off = scratch;                                      // [H, kq_cap + 1]
     int32_t *head_tiles = tile_off + (size_t)H * (kq_cap + 1);         // [H]
     int32_t *head_base = head_tiles + H;                               // [H]
     unsigned long long *head_pairs =
         reinterpret_cast<unsigned long long *>(head_base + H + ((2 * H + (size_t)H * (kq_cap + 1)) & 1));  // [H]
     items_count_kernel<<<H, 512, 0, st>>>(N, rows_per_item, kq_cap, kk_cap, qoff, nq, dense, kq_fixed, koff, sel_idx, sel_cnt,
-                                          tile_off, head_tiles, head_pairs);
+                                          tile_off, head_tiles, head_pairs, status);
     note_launch();
     items_base_kernel<<<1, 32, 0, st>>>(H, head_tiles, head_pairs, head_base, n_items, pairs);
     note_launch();
@@ -835,11 +837,8 @@ static int launch_attn(const void *qg, const void *kg, const void *vg, const Att
         make_map(enc, &mv, vg, C::ELT, rows, D, C::BOX,
                  C::ELT == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
         return -1;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(attn_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        attr = true;
-    }
+    // the attribute belongs to the current device: set it on every call
+    cudaFuncSetAttribute(attn_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int grid = max_items < num_sms ? max_items : num_sms;
     if (grid < 1) grid = 1;
     attn_kernel<T, D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p); note_launch();

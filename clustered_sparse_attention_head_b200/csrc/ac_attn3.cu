@@ -890,16 +890,13 @@ static int launch3(const void *qg, const void *kg, const void *vg, const A3Param
     const int rows = p.H * p.N;
     if (bf16_map3(enc, &mq, qg, rows, D, 128) || kv_maps3(enc, &mk, kg, rows, D) || kv_maps3(enc, &mv, vg, rows, D))
         return -1;
-    static int checked = 0;  // 1 = ok, -1 = refused
-    if (checked == 0) {
-        // the register split assumes the launch budget ptxas gave the kernel;
-        // a larger split would make setmaxnreg.inc wait forever, so refuse
-        cudaFuncAttributes fa;
-        checked = (cudaFuncGetAttributes(&fa, attn3_kernel<D>) == cudaSuccess && fa.numRegs == C::REGS_LAUNCH) ? 1 : -1;
-        if (checked == 1)
-            cudaFuncSetAttribute(attn3_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    }
-    if (checked != 1) return -1;
+    // the register split assumes the launch budget ptxas gave the kernel; a
+    // larger split would make setmaxnreg.inc wait forever, so refuse.  The
+    // shared-memory attribute belongs to the current device: set on every call.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn3_kernel<D>) != cudaSuccess || fa.numRegs != C::REGS_LAUNCH) return -1;
+    if (cudaFuncSetAttribute(attn3_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return -1;
     int grid = max_items < num_sms ? max_items : num_sms;
     if (grid < 1) grid = 1;
     attn3_kernel<D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);

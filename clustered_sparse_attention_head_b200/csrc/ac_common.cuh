@@ -8,9 +8,19 @@
 namespace ac {
 
 // ----------------------------------------------------------------- status
-enum DevStatus : int { ST_OK = 0, ST_TIMEOUT = 5, ST_NONFINITE = 6, ST_CAPACITY = 7 };
+enum DevStatus : int { ST_OK = 0, ST_INVALID = 1, ST_TIMEOUT = 5, ST_NONFINITE = 6, ST_CAPACITY = 7 };
 
 __device__ __forceinline__ void set_status(int *st, int code) { atomicCAS(st, 0, code); }
+
+// A per-head count read from caller memory (clusters in use, selected
+// clusters), clamped to [0, cap] so that no kernel indexes past a
+// capacity-sized buffer.  A value outside the range records ST_INVALID
+// (status may be NULL).
+__device__ __forceinline__ int clamp_count(int v, int cap, int *status) {
+    if (v >= 0 && v <= cap) return v;
+    if (status) set_status(status, ST_INVALID);
+    return v < 0 ? 0 : cap;
+}
 
 // Per-head description of one clustering pass (Algorithm 1 runs passes over a
 // subset U of the tokens with a stage-dependent cluster count).

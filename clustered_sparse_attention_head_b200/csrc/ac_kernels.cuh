@@ -57,7 +57,8 @@ struct MsState;  // device-side Algorithm 1 state, see ac_multistage.cu
 void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const int32_t *q_count, int kq_cap,
               const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min, int kk_cap,
               const int32_t *nq, const int32_t *nk, int kq_fixed, int kk_fixed, const uint8_t *dense, int score_mode,
-              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st, int text_group = 0,
+              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, int *status, cudaStream_t st,
+              int text_group = 0,
               float *k_cent_t = nullptr);  // k_cent_t: [H, D, kk_cap] scratch for the transposed centroids
 // Per-cluster, per-dimension max / min of x over the members listed by a
 // cluster sort (perm, off [H, cap + 1]); 0 for empty clusters.
@@ -72,7 +73,7 @@ struct AttnItem {
 void k_build_items(int H, int N, int rows_per_item, int kq_cap, int kk_cap, const int32_t *qoff, const int32_t *nq,
                    const uint8_t *dense, int kq_fixed, const int32_t *koff, const int32_t *sel_idx,
                    const int32_t *sel_cnt, AttnItem *items, int32_t *n_items, int64_t *pairs, int32_t *scratch,
-                   cudaStream_t st);
+                   int *status, cudaStream_t st);
 size_t items_scratch_elems(int H, int kq_cap);
 int attn_max_items(int H, int N, int kq_cap);
 // Key runs of every (head, query cluster) (ac_attn.cu): the selected key

@@ -263,8 +263,10 @@ __global__ void __launch_bounds__(256) assign_exact_kernel(
         __syncwarp();
         double best = (mode == MODE_EUCLID) ? INFINITY : -INFINITY;
         int bj = 0x7fffffff;
-        // shortlisted rows: only the two candidates the screen left open
-        const int2 cand = amb_cand ? amb_cand[(size_t)h * N + a] : make_int2(-1, -1);
+        // shortlisted rows: only the two candidates the screen left open (a
+        // candidate outside [0, k) means a full scan)
+        int2 cand = amb_cand ? amb_cand[(size_t)h * N + a] : make_int2(-1, -1);
+        if (cand.x >= s.k || cand.y >= s.k || cand.y < 0) cand = make_int2(-1, -1);
         const int jcount = cand.x >= 0 ? 2 : s.k;
         for (int q = lane; q < jcount; q += 32) {
             const int j = cand.x >= 0 ? (q == 0 ? cand.x : cand.y) : q;
@@ -291,6 +293,9 @@ __global__ void __launch_bounds__(256) assign_exact_kernel(
             bool better = (mode == MODE_EUCLID) ? (ob < best) : (ob > best);
             if (better || (ob == best && oj < bj)) { best = ob; bj = oj; }
         }
+        // no score compared as better than the start (every score NaN): the
+        // lowest candidate, so the id is always one of the pass's clusters
+        if (bj == 0x7fffffff) bj = cand.x >= 0 ? min(cand.x, cand.y) : 0;
         if (lane == 0) assign[(size_t)h * N + pos] = bj;
     }
 }
@@ -309,7 +314,10 @@ __global__ void dist_kernel(const T *__restrict__ x, int N, const int32_t *__res
     int tok = rows ? rows[(size_t)h * N + pos] : pos;
     const T *xi = x + ((size_t)h * N + tok) * D;
     double nrm = norm[(size_t)h * N + tok];
-    const float *c = cent + ((size_t)h * cap + s.cent_off + assign[(size_t)h * N + pos]) * D;
+    // ids are in [0, k) by construction; clamped so that no id can read
+    // outside the centroid block
+    const int a = min(max(assign[(size_t)h * N + pos], 0), max(s.k - 1, 0));
+    const float *c = cent + ((size_t)h * cap + s.cent_off + a) * D;
     double acc = 0.0;
     for (int t = 0; t < D; t++) {
         double df = dsub(work_val(xi, t, mode, nrm), (double)c[t]);
@@ -434,11 +442,8 @@ static void launch_assign(const void *x, int H, int N, const int32_t *rows, cons
                           const float *cent, int cap, const float *cn2, const float *cmax, const double *norm,
                           int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, cudaStream_t st) {
     size_t smem = (size_t)D * (SCR_XS + SCR_CS) * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaFuncSetAttribute(assign_screen_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        attr_set = true;
-    }
+    // the attribute belongs to the current device: set it on every call
+    cudaFuncSetAttribute(assign_screen_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 g((nrows_max + SCR_ROWS - 1) / SCR_ROWS, H);
     assign_screen_kernel<T, D><<<g, 256, smem, st>>>((const T *)x, N, rows, seg, cent, cap, cn2, cmax, mode, assign,
                                                       amb_list, amb_count); note_launch();

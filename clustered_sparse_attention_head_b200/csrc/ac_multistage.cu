@@ -230,14 +230,16 @@ __global__ void seg_uniform_kernel(int H, int nrows, int k, HeadSeg *__restrict_
 }
 
 // Per-head pass descriptors from device cluster counts (nk may be NULL), less
-// `sub` groups that the pass does not cluster (the text-key group).
-__global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restrict__ ncl, int kfix, int sub,
-                                       HeadSeg *__restrict__ seg) {
+// `sub` groups that the pass does not cluster (the text-key group).  A count
+// outside [0, cap] (caller memory) is clamped and records ST_INVALID: the
+// sort and every pass over the descriptors size their tables by cap.
+__global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restrict__ ncl, int kfix, int sub, int cap,
+                                       HeadSeg *__restrict__ seg, int *status) {
     int h = blockIdx.x * blockDim.x + threadIdx.x;
     if (h >= H) return;
     HeadSeg g;
     g.nrows = nrows;
-    g.k = (ncl ? ncl[h] : kfix) - sub;
+    g.k = clamp_count((ncl ? ncl[h] : kfix) - sub, cap - sub, status);
     g.cent_off = 0;
     g.pad = 0;
     seg[h] = g;
@@ -256,11 +258,8 @@ void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double
     int n2 = 1;
     while (n2 < kmax) n2 <<= 1;
     size_t smem = (size_t)n2 * sizeof(double);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-        cudaFuncSetAttribute(ms_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        smem_set = smem;
-    }
+    // the attribute belongs to the current device: set it on every call that needs it
+    if (smem > 48 * 1024) cudaFuncSetAttribute(ms_tau_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     ms_tau_kernel<<<H, 256, smem, s>>>(N, rule, x, seg, dist, perm, off, cap, st); note_launch();
 }
 void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int32_t *U, int32_t *Unext, MsHead *st,
@@ -274,8 +273,9 @@ void k_ms_final(int H, int nrows, const MsHead *st, HeadSeg *seg, int32_t *ncl, 
 void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s) {
     seg_uniform_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, k, seg, ncl, flag); note_launch();
 }
-void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s, int sub) {
-    seg_from_counts_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, ncl, kfix, sub, seg); note_launch();
+void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, int cap, HeadSeg *seg, int *status,
+                       cudaStream_t s, int sub) {
+    seg_from_counts_kernel<<<(H + 127) / 128, 128, 0, s>>>(H, nrows, ncl, kfix, sub, cap, seg, status); note_launch();
 }
 
 // The text-key group after key clustering: rows [nrows, N) of every head get

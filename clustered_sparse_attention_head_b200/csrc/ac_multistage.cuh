@@ -25,7 +25,10 @@ void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int
 void k_ms_final(int H, int nrows, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
                 cudaStream_t s);
 void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s);
-void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, HeadSeg *seg, cudaStream_t s, int sub = 0);
+// Pass descriptors from per-head counts ncl (NULL: kfix for every head) less
+// sub; counts outside [0, cap] are clamped and record ST_INVALID in status.
+void k_seg_from_counts(int H, int nrows, const int32_t *ncl, int kfix, int cap, HeadSeg *seg, int *status,
+                       cudaStream_t s, int sub = 0);
 // The text-key group (ac_config.text_keys): rows [nrows, N) get id seg.k, count
 // N - nrows, and ncl = seg.k + 1.
 void k_text_group(int H, int N, int nrows, const HeadSeg *seg, int32_t *assign, int32_t *count, int cap,

@@ -41,7 +41,7 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
                               const int32_t *__restrict__ nk, int kq_fixed, int kk_fixed,
                               const uint8_t *__restrict__ dense, int score_mode, int top_k, double top_p, int n2,
                               int text_group, const float *__restrict__ k_cent_t, int32_t *__restrict__ sel_idx,
-                              int32_t *__restrict__ sel_cnt) {
+                              int32_t *__restrict__ sel_cnt, int *status) {
     extern __shared__ __align__(16) unsigned char smraw[];
     double *sp = reinterpret_cast<double *>(smraw);          // [n2] p (sort key)
     int *sb = reinterpret_cast<int *>(sp + n2);             // [n2] b
@@ -55,9 +55,12 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
     __shared__ double sW;
 
     const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
-    const int nqh = nq ? nq[h] : kq_fixed;
+    // counts from caller memory are clamped to the capacities (ST_INVALID if not within)
+    const int nqh = nq ? clamp_count(nq[h], kq_cap, a == 0 && tid == 0 ? status : nullptr) : kq_fixed;
     // with a text-key group, the last key id is that group: never scored, always kept
-    const int nkh = (nk ? nk[h] : kk_fixed) - text_group;
+    const int nkh =
+        nk ? clamp_count(nk[h] - text_group, kk_cap - text_group, a == 0 && tid == 0 ? status : nullptr)
+           : kk_fixed - text_group;
     int32_t *out = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
     if (a >= kq_cap) return;
     if (a >= nqh || (dense && dense[h]) || q_count[(size_t)h * kq_cap + a] == 0) {
@@ -212,8 +215,8 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
 void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const int32_t *q_count, int kq_cap,
               const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min, int kk_cap,
               const int32_t *nq, const int32_t *nk, int kq_fixed, int kk_fixed, const uint8_t *dense, int score_mode,
-              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, cudaStream_t st, int text_group,
-              float *k_cent_t) {
+              int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, int *status, cudaStream_t st,
+              int text_group, float *k_cent_t) {
     int n2 = 1;
     while (n2 < kk_cap) n2 <<= 1;
     size_t smem = (size_t)n2 * (sizeof(double) + sizeof(int)) + (size_t)kk_cap * (sizeof(double) + sizeof(int) + 1);
@@ -224,16 +227,13 @@ void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const
     } else {
         k_cent_t = nullptr;
     }
-    // opt in whenever dynamic plus static shared memory may pass 48 KB
-    static size_t smem_set = 0;
-    if (smem > smem_set) {
-        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        smem_set = smem;
-    }
+    // opt in whenever dynamic plus static shared memory may pass 48 KB (the
+    // attribute belongs to the current device, so it is set on every call)
+    if (smem > 32 * 1024) cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 g(kq_cap, H);
     select_kernel<<<g, 256, smem, st>>>(D, q_cent, q_mean_norm, q_count, kq_cap, k_cent, k_count, k_max, k_min,
                                         kk_cap, nq, nk, kq_fixed, kk_fixed, dense, score_mode, top_k, top_p, n2,
-                                        text_group, k_cent_t, sel_idx, sel_cnt);
+                                        text_group, k_cent_t, sel_idx, sel_cnt, status);
     note_launch();
 }
 

@@ -155,11 +155,8 @@ void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, 
     int ntiles_max = (N + SORT_TILE - 1) / SORT_TILE;
     int nt = (nrows_max + SORT_TILE - 1) / SORT_TILE;
     size_t smem = (size_t)4 * cap * sizeof(int32_t);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-        cudaFuncSetAttribute(rank_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        smem_set = smem;
-    }
+    // the attribute belongs to the current device: set it on every call that needs it
+    if (smem > 48 * 1024) cudaFuncSetAttribute(rank_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (nt > 0) {
         dim3 g1(nt, H);
         rank_hist_kernel<<<g1, 128, smem, st>>>(ids, seg, N, cap, ntiles_max, rank, hist, status); note_launch();

@@ -34,6 +34,11 @@
  *      sel_cnt        [H, kq_cap] int32 number of selected key clusters
  *    with cap = kq_cap for queries and kk_cap for keys (ac_capacities()).
  *  - Cluster ids are int32; ties in every argmin/argmax go to the lowest id.
+ *  - Per-head counts that a call reads from device memory (nq, nk, ncl,
+ *    sel_cnt) must lie in [0, capacity] (kq_cap, kk_cap, cap).  A value
+ *    outside is clamped to that range so that no kernel indexes past a
+ *    capacity-sized buffer, and AC_ERR_INVALID_ARG is recorded in the status
+ *    word (ac_get_status).  Cluster ids outside [0, count) are skipped.
  *  - Concurrent calls on one context must not overlap on the GPU: the context's
  *    status word and the workspace are shared by the calls that use them.
  */
@@ -217,10 +222,18 @@ AC_API ac_status ac_cluster_sort(ac_ctx *ctx, const int32_t *assign, int cap, co
  *  - The first call on each device looks up that device's address of the
  *    array (cudaGetSymbolAddress, with the device current); make that first
  *    call before any stream capture.
+ *  - The device address of the array is looked up again whenever the
+ *    device's current context changes (after cudaDeviceReset, for example).
  *  - All calls share the one array, which keeps the last call's contents;
  *    calls that overlap on the GPU (different streams without ordering) race,
  *    so order them.
- *  - ids outside [0, ncl[h]) are skipped and leave their perm slots unwritten.
+ *  - ncl[h] must lie in [0, cap]; a larger (or negative) count is clamped to
+ *    cap (or 0).  There is no context, so this is not reported.
+ *  - ids outside [0, ncl[h]) are skipped: the sort covers only the valid ids
+ *    (offsets[cap] = their number) and the perm slots past them are left
+ *    unwritten.
+ *  - A pending launch error of earlier work on the calling thread is cleared
+ *    on entry (cudaGetLastError), so the return value describes this call.
  * Returns AC_ERR_INVALID_ARG for NULL pointers or non-positive sizes.         */
 AC_API ac_status ac_cluster_sort_static(const int32_t *assign, int heads, int n, int cap, const int32_t *ncl,
                                         int32_t *perm, int32_t *offsets, void *stream);
