@@ -4,7 +4,10 @@ the CPU oracle.
 
 The GPU processes all heads in one call.  The oracle recomputes Algorithm 3
 from the same seeded inputs for two sampled heads per workload (the first and
-the last; four for the small CogVideoX-shaped one), and for those heads:
+the last; four for the small CogVideoX-shaped one), plus, on the adaptive
+workloads, the first head that takes the sparse branch (dense flag F = 0), so
+that Algorithm 1's sparse branch is compared at full size too (the oracle
+checks that head's F like every other).  For those heads:
   - query and key clustering: number of clusters, the F flag, counts and every
     assignment bit-exact (a mismatch is excused only at a near-tie, as in the
     small-case tests); centroids within 1e-5 relative;
@@ -122,7 +125,12 @@ def test_full_size_forward(orc, name):
     assert bool(torch.isfinite(out.float()).all())
 
     # the oracle, from scratch, on the sampled heads
-    heads = SAMPLED[name]
+    heads = list(SAMPLED[name])
+    if w.adaptive_q or w.adaptive_k:
+        sparse = [h for h in range(w.heads) if not dense[h] and h not in heads]
+        if sparse:
+            heads.append(sparse[0])
+        print(f"{name}: oracle heads {heads} ({int(dense.sum())} of {w.heads} heads dense on the GPU)")
     rows = np.unique(np.concatenate([np.linspace(0, w.n - 1, 256).astype(np.int32), [w.n - 1]])).astype(np.int32)
     spec = _spec(orc, w)
     with ThreadPoolExecutor(max_workers=len(heads)) as ex:

@@ -4,9 +4,13 @@ fixed-count k-means.
 
 Per step and head: cluster counts and dense flag F exact; query and key
 centres within 1e-5 relative; attention rows within max-abs 2e-2 / mean-abs
-2e-3.  A head is excused from a step on only when the oracle's own k-means of
-that step meets a near-tie (two best scores within 1e-6 relative): the GPU
-may then take the other, equally valid branch."""
+2e-3.  Every head is compared at every step.  Only a head that fails the
+comparison can be excused, and only when the oracle's own k-means of that
+step meets a near-tie (two best scores within 1e-6 relative) on some rows:
+the GPU may then take the other, equally valid branch there, which moves the
+two clusters' centres and everything after.  Such a head is compared again
+at the next step only through what does not depend on that branch (counts and
+F); the excused heads and their near-tie rows are printed."""
 import numpy as np
 import pytest
 
@@ -58,8 +62,8 @@ def _spec(orc, w, over):
     return orc.HeadSpec(**g)
 
 
-def _near_tie(xs, cent, mode, orc):
-    """Any row whose two best scores against `cent` are within TIE_REL."""
+def _near_tie_rows(xs, cent, mode, orc):
+    """Rows whose two best scores against `cent` are within TIE_REL."""
     x = np.asarray(xs, np.float64)
     c = np.asarray(cent, np.float64)
     if mode == orc.EUCLID:
@@ -68,20 +72,39 @@ def _near_tie(xs, cent, mode, orc):
         s = x @ c.T
     top = np.sort(s, axis=1)[:, -2:]
     den = np.maximum(np.abs(top).max(1), 1e-300)
-    return bool(((top[:, 1] - top[:, 0]) / den < TIE_REL).any())
+    return set(np.nonzero((top[:, 1] - top[:, 0]) / den < TIE_REL)[0].tolist())
+
+
+def _kmeans_tie_rows(orc, x, k, iters, mode, init):
+    """Replays fixed-count k-means with the oracle's steps; returns the rows
+    that meet a near-tie in any of its assignment passes."""
+    xs, _ = orc.prepare(x, mode)
+    cent = np.asarray(init, np.float32)[:k].copy()
+    rows = set()
+    for _ in range(iters):
+        rows |= _near_tie_rows(xs, cent, mode, orc)
+        ids, _, _ = orc.assign(xs, cent, mode)
+        cent, _ = orc.update(xs, ids, cent, mode)
+    return rows | _near_tie_rows(xs, cent, mode, orc)
 
 
 def _kmeans_has_tie(orc, x, k, iters, mode, init):
-    """Replays fixed-count k-means with the oracle's steps and reports a near-tie
-    in any of its assignment passes."""
-    xs, _ = orc.prepare(x, mode)
-    cent = np.asarray(init, np.float32)[:k].copy()
-    for _ in range(iters):
-        if _near_tie(xs, cent, mode, orc):
-            return True
-        ids, _, _ = orc.assign(xs, cent, mode)
-        cent, _ = orc.update(xs, ids, cent, mode)
-    return _near_tie(xs, cent, mode, orc)
+    return bool(_kmeans_tie_rows(orc, x, k, iters, mode, init))
+
+
+def _compare_or_excuse(what, check, tie_rows, excused):
+    """Runs `check`; a failure is excused only when the oracle's k-means of the
+    step met near-ties (tie_rows() lists them), and is recorded in `excused`."""
+    try:
+        check()
+        return True
+    except AssertionError:
+        rows = tie_rows()
+        if not rows:
+            raise
+        excused.append((what, len(rows)))
+        print(f"{what}: differs after {len(rows)} near-tie rows in the oracle's k-means; excused")
+        return False
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -94,7 +117,8 @@ def test_forward_steps_parity(orc, name):
     inp = [[W.step_inputs(w, h, s, DRIFT) for s in range(NSTEPS)] for h in range(H)]
     ref = [orc.forward_steps([(x.q, x.k, x.v) for x in inp[h]], spec, rows=rows) for h in range(H)]
     state = ctx.step_state()
-    excused = [False] * H
+    diverged = [False] * H   # an excused branch earlier: centres follow the GPU's own branch
+    excused = []
     for s in range(NSTEPS):
         q, k, v = (to_dev(np.stack([getattr(inp[h][s], a) for h in range(H)]), w.dtype) for a in "qkv")
         out, st = ctx.ac_forward_step(s, q, k, v, state, stats=True)
@@ -106,8 +130,7 @@ def test_forward_steps_parity(orc, name):
               f"dense heads {st['dense_heads']}")
         for h in range(H):
             r = ref[h][s]
-            if excused[h]:
-                continue
+            # counts and F are fixed at step 0 and do not depend on later branches
             nq, nk = int(parts["nq"][h]), int(parts["nk"][h])
             assert nq == r.q.nclusters and nk == r.k.nclusters, f"{name}/step{s}/h{h}: counts"
             assert int(parts["dq"][h] | parts["dk"][h]) == r.dense, f"{name}/step{s}/h{h}: F"
@@ -115,17 +138,25 @@ def test_forward_steps_parity(orc, name):
                 # dense attention does not depend on the clusters
                 attn_close(got[h][rows], r.out_rows, f"{name}/step{s}/h{h}/attention (dense)")
                 continue
-            if s > 0:
+            if diverged[h]:
+                continue
+
+            def check():
+                np.testing.assert_allclose(parts["q_cent"][h, :nq], r.q.cent[:nq], rtol=CENT_RTOL, atol=1e-7)
+                np.testing.assert_allclose(parts["k_cent"][h, :nk], r.k.cent[:nk], rtol=CENT_RTOL, atol=1e-7)
+                attn_close(got[h][rows], r.out_rows, f"{name}/step{s}/h{h}/attention")
+
+            def tie_rows():
+                if s == 0:
+                    return set()
                 prev = ref[h][s - 1]
-                tie = (_kmeans_has_tie(orc, inp[h][s].q, r.q.nclusters, spec.iters, orc.SPHERE, prev.q.cent) or
-                       _kmeans_has_tie(orc, inp[h][s].k, r.k.nclusters, spec.iters, orc.EUCLID, prev.k.cent))
-                if tie:
-                    print(f"{name}/h{h}: near-tie in the oracle's k-means at step {s}; excused from here on")
-                    excused[h] = True
-                    continue
-            np.testing.assert_allclose(parts["q_cent"][h, :nq], r.q.cent[:nq], rtol=CENT_RTOL, atol=1e-7)
-            np.testing.assert_allclose(parts["k_cent"][h, :nk], r.k.cent[:nk], rtol=CENT_RTOL, atol=1e-7)
-            attn_close(got[h][rows], r.out_rows, f"{name}/step{s}/h{h}/attention")
+                return (_kmeans_tie_rows(orc, inp[h][s].q, r.q.nclusters, spec.iters, orc.SPHERE, prev.q.cent) |
+                        _kmeans_tie_rows(orc, inp[h][s].k, r.k.nclusters, spec.iters, orc.EUCLID, prev.k.cent))
+
+            if not _compare_or_excuse(f"{name}/step{s}/h{h}", check, tie_rows, excused):
+                diverged[h] = True
+    print(f"{name}: {len(excused)} head-steps excused ({sum(n for _, n in excused)} near-tie rows) "
+          f"of {H * NSTEPS}")
 
 
 def test_warm_steps_need_fewer_rounds(orc):
@@ -186,7 +217,8 @@ def test_forward_steps_with_text_keys(orc):
     inp = [[W.step_inputs(w, h, s, DRIFT) for s in range(3)] for h in range(H)]
     ref = [orc.forward_steps([(x.q, x.k, x.v) for x in inp[h]], spec, rows=rows) for h in range(H)]
     state = ctx.step_state()
-    excused = [False] * H
+    diverged = [False] * H
+    excused = []
     for s in range(3):
         q, k, v = (to_dev(np.stack([getattr(inp[h][s], a) for h in range(H)]), w.dtype) for a in "qkv")
         out = ctx.ac_forward_step(s, q, k, v, state)
@@ -198,13 +230,20 @@ def test_forward_steps_with_text_keys(orc):
             r = ref[h][s]
             nv = r.k.nclusters
             assert int(parts["nk"][h]) == nv + 1, f"step{s}/h{h}: key groups"
-            if excused[h]:
+            if diverged[h]:
                 continue
-            if s > 0:
+
+            def check():
+                np.testing.assert_allclose(parts["k_cent"][h, :nv], r.k.cent[:nv], rtol=CENT_RTOL, atol=1e-7)
+                attn_close(got[h][rows], r.out_rows, f"text/step{s}/h{h}/attention")
+
+            def tie_rows():
+                if s == 0:
+                    return set()
                 prev = ref[h][s - 1]
-                if (_kmeans_has_tie(orc, inp[h][s].q, r.q.nclusters, spec.iters, orc.SPHERE, prev.q.cent) or
-                        _kmeans_has_tie(orc, inp[h][s].k[:N - T], nv, spec.iters, orc.EUCLID, prev.k.cent)):
-                    excused[h] = True
-                    continue
-            np.testing.assert_allclose(parts["k_cent"][h, :nv], r.k.cent[:nv], rtol=CENT_RTOL, atol=1e-7)
-            attn_close(got[h][rows], r.out_rows, f"text/step{s}/h{h}/attention")
+                return (_kmeans_tie_rows(orc, inp[h][s].q, r.q.nclusters, spec.iters, orc.SPHERE, prev.q.cent) |
+                        _kmeans_tie_rows(orc, inp[h][s].k[:N - T], nv, spec.iters, orc.EUCLID, prev.k.cent))
+
+            if not _compare_or_excuse(f"text/step{s}/h{h}", check, tie_rows, excused):
+                diverged[h] = True
+    print(f"text: {len(excused)} head-steps excused ({sum(n for _, n in excused)} near-tie rows) of {H * 3}")
