@@ -6,10 +6,13 @@ clustering, critical-cluster selection, cluster sort + gather, block-sparse
 attention) on the Wan-2.1-shaped workload: 40 heads x 75,600 tokens x d=128,
 bf16, 250 query / 500 key clusters, 10 k-means iterations, top-p 0.9.
 
-Prints one JSON line (rank 0).  --impl reference times the CPU oracle on a
-bounded sample of the same workload instead.  Under torchrun every rank runs
-its own independent call (heads and calls share nothing), so scaling is weak
-and value = calls over all ranks / max-over-ranks time.
+Prints one JSON line (rank 0).  Besides the headline workload the line carries
+`per_config` (every workload of the suite: ms per call, stages, roofline and
+the SDPA comparator) and `top_p_sweep` (the headline workload at top-p 0.8,
+0.9 and 0.95).  --impl reference times the CPU oracle on bounded samples of the
+same workload instead.  Under torchrun every rank runs its own independent
+call (heads and calls share nothing), so scaling is weak and value = calls over
+all ranks / max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -34,6 +37,12 @@ METRIC = "clustered sparse-attn calls/s & achieved TFLOPS at 75.6K tokens vs den
 # the default workload cut to 8 heads (0.522 GB + 0.141 GB); None whenever the
 # kernel changes, until it is captured again
 ATTN_TRAFFIC_8H = 0.6628e9
+L2_BYTES = 126 * 2 ** 20
+# the CPU oracle's bounded sample: one head clustered and selected in full,
+# attention for SAMPLE_ROWS query rows; heads 0..SAMPLE_HEADS-1 in turn
+SAMPLE_ROWS = 128
+SAMPLE_HEADS = 4
+TOP_P_SWEEP = (0.8, 0.9, 0.95)
 
 
 def parse():
@@ -48,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload and top-p sweep keys")
+    ap.add_argument("--per-config-calls", type=int, default=3, help="timed calls per workload in per_config")
     ap.add_argument("--denoise-steps", type=int, default=0,
                     help="also run the multi-step driver (ac_forward_step) over this many drifting steps")
     ap.add_argument("--drift", type=float, default=0.02, help="per-element drift per denoising step")
@@ -136,9 +147,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ cpu baseline
-def oracle_sample(w, hi, rows_sample: int):
+def oracle_sample(w, hi, rows_sample: int = SAMPLE_ROWS):
     """Time the oracle on one head: full Q and K clustering and selection, and
-    attention for `rows_sample` query rows; extrapolate to one whole call."""
+    attention for `rows_sample` query rows.  Returns (seconds one whole call
+    would take at this rate: x heads, x n / rows_sample rows; wall seconds)."""
     import oracle
     oracle.build()
     spec = oracle.HeadSpec(kq=w.kq, kk=w.kk, iters=w.iters, top_p=w.top_p, adaptive_q=w.adaptive_q,
@@ -165,39 +177,64 @@ def omp_threads():
     return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
 
 
-def cpu_baseline_obj(w, his, rows_sample=128):
-    """The oracle on a bounded sample: the given heads (about 3 s each on 16
-    host cores for the 75.6K workload), averaged and extrapolated to a call."""
-    per, walls = zip(*(oracle_sample(w, hi, rows_sample) for hi in his))
+def sample_text(w, heads_used, walls):
+    return (f"per sample: one head (heads 0-{heads_used - 1} of {w.heads} in turn) with Q and K clustering and "
+            f"selection in full and attention for {SAMPLE_ROWS} of {w.n} query rows; the mean extrapolated "
+            f"x{w.heads} heads and x{w.n}/{SAMPLE_ROWS} rows to one call; {len(walls)} samples, "
+            f"{sum(walls):.1f} s wall time measured")
+
+
+def cpu_baseline_obj(w, his):
+    """The oracle on bounded samples of the workload (the same samples as the
+    reference arm's steps), extrapolated to calls/s."""
+    per, walls = zip(*(oracle_sample(w, hi) for hi in his))
     per_call = statistics.mean(per)
     return {"value": 1.0 / per_call, "unit": "calls/s", "cores": omp_threads(), "kind": "oracle",
-            "sample": (f"heads 0-{len(his) - 1} of {w.heads}: Q and K clustering and selection in full, attention "
-                       f"for {rows_sample} of {w.n} query rows each; mean per head extrapolated x{w.heads} heads and "
-                       f"x{w.n}/{rows_sample} rows ({sum(walls):.1f} s wall time measured)")}
+            "extrapolated": True, "samples_timed": len(walls), "wall_s": sum(walls),
+            "scale_per_sample": w.heads * w.n / SAMPLE_ROWS,
+            "sample": sample_text(w, len(his), walls)}
+
+
+def config_of(w, world, text_keys=0):
+    """The `config` object of the JSON line, the same for both arms."""
+    tb = tensor_bytes(w)
+    l2 = (f"inputs larger than L2 ({tb / 1e6:.0f} MB per tensor), no flush" if tb > L2_BYTES else
+          f"L2 flushed between timed calls (a {2 * L2_BYTES >> 20} MiB write; {tb / 1e6:.1f} MB per tensor)")
+    return {"workload": w.name, "heads": w.heads, "n": w.n, "d": w.d, "kq": w.kq, "kk": w.kk, "iters": w.iters,
+            "top_p": w.top_p, "text_keys": text_keys, "parallelism": f"dp{world} (independent calls)", "l2": l2}
+
+
+def tensor_bytes(w):
+    return w.heads * w.n * w.d * (2 if w.dtype == "bf16" else 4)
 
 
 # -------------------------------------------------------------- reference
 def run_reference(a, w):
+    """The CPU oracle as the reference arm.  A step is one bounded sample (one
+    head, SAMPLE_ROWS attention rows), so steps x ms_per_step is the measured
+    wall time; value is the samples' mean extrapolated to whole calls."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    hi = W.head_inputs(w, 0)
-    rows = 64
-    times = []
+    his = [W.head_inputs(w, h) for h in range(min(SAMPLE_HEADS, w.heads))]
+    per, walls = [], []
     for i in range(a.warmup + a.steps):
-        per_call, _ = oracle_sample(w, hi, rows)
+        per_call, wall = oracle_sample(w, his[i % len(his)])
         if i >= a.warmup:
-            times.append(per_call)
-    per_call = statistics.mean(times)
-    v = 1.0 / per_call
+            per.append(per_call)
+            walls.append(wall)
+    v = 1.0 / statistics.mean(per)
+    ms_step = 1e3 * statistics.mean(walls)
     line = {"metric": METRIC, "value": v, "unit": "calls/s", "n_gpus": 0, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": per_call * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "heads": w.heads, "n": w.n, "d": w.d, "kq": w.kq, "kk": w.kk,
-                       "iters": w.iters, "top_p": w.top_p},
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference", "config": config_of(w, 1),
+            "extrapolated": True,
+            "step": f"one bounded sample ({SAMPLE_ROWS} attention rows of one head); value extrapolates the samples "
+                    f"to whole calls (x{w.heads * w.n / SAMPLE_ROWS:.0f} per sample)",
             "cpu_baseline": {"value": v, "unit": "calls/s", "cores": omp_threads(), "kind": "oracle",
-                             "sample": f"per step: head 0 clustered and selected in full, attention for {rows} of "
-                                       f"{w.n} rows, extrapolated to {w.heads} heads x {w.n} rows"},
+                             "extrapolated": True, "samples_timed": len(walls), "wall_s": sum(walls),
+                             "scale_per_sample": w.heads * w.n / SAMPLE_ROWS,
+                             "sample": sample_text(w, len(his), walls)},
             "e2e": {"value": v, "unit": "calls/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -220,7 +257,7 @@ def main():
     hs = gen_inputs(w)
     cpu_base = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu_base = cpu_baseline_obj(w, hs[:min(4, len(hs))])
+        cpu_base = cpu_baseline_obj(w, hs[:min(SAMPLE_HEADS, len(hs))])
 
     import torch
     torch.cuda.set_device(local)
@@ -261,18 +298,15 @@ def main():
         raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
     ac.profile_read()
 
-    # timed region: inputs (774 MB per tensor) exceed the 126 MB L2, so no flush
+    # timed region: inputs larger than L2 need no flush; smaller ones get an L2
+    # flush before every call, outside the events that time the call
     sampler = ClockSampler(local)
+    flush = None if tensor_bytes(w) > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     barrier()
     sampler.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(a.steps):
-        ac.ac_forward(q, k, v, out=out)
-    e1.record(stream)
+    ms = time_calls(lambda: ac.ac_forward(q, k, v, out=out), a.steps, stream, flush)
     barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1) / a.steps
     prof = ac.profile_read()
     status = ac.get_status()
     if status != 0:
@@ -344,18 +378,7 @@ def main():
     # dense comparator: torch SDPA at the same shape (40 heads x 75.6K x 128)
     dense = None
     if not a.no_dense and rank == 0:
-        import torch.nn.functional as F
-        qd, kd, vd = (t.unsqueeze(0) for t in (q, k, v))
-        for _ in range(2):
-            F.scaled_dot_product_attention(qd, kd, vd)
-        torch.cuda.synchronize(dev)
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for _ in range(3):
-            F.scaled_dot_product_attention(qd, kd, vd)
-        d1.record(stream)
-        torch.cuda.synchronize(dev)
-        dms = d0.elapsed_time(d1) / 3
+        dms = sdpa_ms(q, k, v, stream, flush)
         dense = {"impl": "torch.nn.functional.scaled_dot_product_attention", "ms": dms,
                  "tflops": w.dense_flops() / (dms * 1e-3) / 1e12, "speedup_of_clustered_call": dms / ms}
         # the library's own dense path (Algorithm 3's dense branch): every head flagged
@@ -365,17 +388,17 @@ def main():
         sel0 = torch.zeros(w.heads, ac.kq_cap, ac.kk_cap, dtype=torch.int32, device=dev)
         cnt0 = torch.zeros(w.heads, ac.kq_cap, dtype=torch.int32, device=dev)
         args = (q, k, v, cq["assign"], ck["assign"], sel0, cnt0)
-        for _ in range(2):
-            ac.ac_sparse_attn(*args, dense_flag=dflag, out=out)
-        torch.cuda.synchronize(dev)
-        d0.record(stream)
-        for _ in range(3):
-            ac.ac_sparse_attn(*args, dense_flag=dflag, out=out)
-        d1.record(stream)
-        torch.cuda.synchronize(dev)
-        oms = d0.elapsed_time(d1) / 3
+        ac.ac_sparse_attn(*args, dense_flag=dflag, out=out)
+        oms = time_calls(lambda: ac.ac_sparse_attn(*args, dense_flag=dflag, out=out), 3, stream, flush)
+        del cq, ck, sel0, cnt0, args
         dense["own_dense"] = {"impl": "ac_sparse_attn with every head dense (gathered copy + attn3_kernel)",
                               "ms": oms, "tflops": w.dense_flops() / (oms * 1e-3) / 1e12}
+
+    launches_timed = int(prof["launches"]) if e2e is None else launches_per_call(ac, q, k, v, out) * a.steps
+    denoise = None
+    if rank == 0 and a.denoise_steps > 0:
+        denoise = denoise_steps(ac, q, k, v, out, a.denoise_steps, a.drift, stream)
+    qs = ks = vs = outs = None
 
     peaks = {}
     try:
@@ -397,14 +420,21 @@ def main():
             "peak_source": peak_src, "ms_per_launch": attn_ms,
             "flops_per_launch": flops, "flops_rule": "4 * d * computed (query, key) pairs"}
 
+    extra = {}
+    if rank == 0 and not a.no_per_config and world == 1:
+        # every workload gets its own context
+        extra["top_p_sweep"] = top_p_sweep(w, q, k, v, out, dev, stream, a.per_config_calls, peak,
+                                           dense["ms"] if dense else None)
+        del q, k, v, out
+        ac.close()
+        torch.cuda.empty_cache()
+        extra["per_config"] = per_config(dev, stream, a.per_config_calls, peak)
+
     if rank == 0:
         line = {"metric": METRIC, "value": calls_per_s, "unit": "calls/s", "n_gpus": world, "steps": a.steps,
                 "warmup": max(a.warmup, 3), "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-                "config": {"workload": w.name, "heads": w.heads, "n": w.n, "d": w.d, "kq": w.kq, "kk": w.kk,
-                           "iters": w.iters, "top_p": w.top_p, "text_keys": cfg.text_keys,
-                           "parallelism": f"dp{world} (independent calls)",
-                           "l2": "inputs larger than L2 (774 MB per tensor), no flush"},
+                "config": config_of(w, world, cfg.text_keys),
                 "tflops_effective_call": tflops_call, "tflops_effective_attn": tflops_attn,
                 "pairs": st["pairs"], "density": st["pairs"] / (w.heads * float(w.n) ** 2),
                 "dense_heads": st["dense_heads"],
@@ -412,17 +442,121 @@ def main():
                                                      "ms_attn_kernel", "ms_total")},
                 "roofline": roof, "dense_attention": dense,
                 "cpu_baseline": cpu_base, "e2e": e2e,
-                "gpu_launches": int(prof["launches"]) if e2e is None else None, "clocks": clocks}
-        if line["gpu_launches"] is None:
-            line["gpu_launches"] = launches_per_call(ac, q, k, v, out) * a.steps
-        if a.denoise_steps > 0:
-            line["denoise_steps"] = denoise_steps(ac, q, k, v, out, a.denoise_steps, a.drift, stream)
+                "gpu_launches": launches_timed, "clocks": clocks}
+        line.update(extra)
+        if denoise is not None:
+            line["denoise_steps"] = denoise
         print(json.dumps(line), flush=True)
     ac.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def time_calls(fn, n, stream, flush=None):
+    """Mean ms of n calls of fn, CUDA events on the launching stream.  With a
+    flush buffer, L2 is overwritten before every call, outside the timing."""
+    import torch
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / n
+    evs = []
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        evs.append((e0, e1))
+    evs[-1][1].synchronize()
+    return sum(x.elapsed_time(y) for x, y in evs) / n
+
+
+def sdpa_ms(q, k, v, stream, flush, calls=3):
+    import torch.nn.functional as F
+    qd, kd, vd = (t.unsqueeze(0) for t in (q, k, v))
+    F.scaled_dot_product_attention(qd, kd, vd)
+    return time_calls(lambda: F.scaled_dot_product_attention(qd, kd, vd), calls, stream, flush)
+
+
+def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0):
+    """One workload through ac_forward: ms per call (CUDA events, L2 flushed
+    first when an input tensor fits in L2), the stage breakdown, computed pairs
+    and the attention kernel's rate against the peak."""
+    import torch
+    from clustered_sparse_attention_head_b200 import _abi
+    from clustered_sparse_attention_head_b200.api import AdaCluster, Config
+    cfg = Config.from_workload(w)
+    cfg.flags = _abi.AC_FLAG_PROFILE
+    cfg.text_keys = text_keys
+    ac = AdaCluster(cfg, device=dev)
+    flush = None if tensor_bytes(w) > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    ac.ac_forward(q, k, v, out=out)
+    _, st = ac.ac_forward(q, k, v, out=out, stats=True)
+    if ac.get_status() != 0:
+        raise RuntimeError(f"{w.name}: device status {ac.get_status()}")
+    ac.profile_read()
+    ms = time_calls(lambda: ac.ac_forward(q, k, v, out=out), calls, stream, flush)
+    prof = ac.profile_read()
+    status = ac.get_status()
+    ac.close()
+    if status != 0:
+        raise RuntimeError(f"{w.name}: device status {status}")
+    flops = 4.0 * w.d * st["pairs"]
+    attn = prof["ms_attn_kernel"]
+    r = {"ms_per_call": ms, "calls_per_s": 1e3 / ms, "pairs": st["pairs"],
+         "density": st["pairs"] / (w.heads * float(w.n) ** 2), "dense_heads": st["dense_heads"],
+         "stages_q": st["max_stages_q"], "stages_k": st["max_stages_k"],
+         "stage_ms": {k2: prof[k2] for k2 in ("ms_cluster_q", "ms_cluster_k", "ms_select", "ms_prep",
+                                              "ms_attn_kernel", "ms_total")},
+         "launches_per_call": int(prof["launches"]) // max(calls, 1),
+         "tflops_effective_call": flops / (ms * 1e-3) / 1e12,
+         "tflops_effective_attn": flops / (attn * 1e-3) / 1e12 if attn > 0 else None,
+         "roofline_frac_attn": flops / (attn * 1e-3) / 1e12 / peak if attn > 0 else None,
+         "l2": config_of(w, 1)["l2"]}
+    return r, flush
+
+
+def top_p_sweep(w, q, k, v, out, dev, stream, calls, peak, sdpa):
+    """The headline workload at each top-p of TOP_P_SWEEP (same inputs)."""
+    from dataclasses import replace
+    rows = []
+    for tp in TOP_P_SWEEP:
+        r, _ = measure(replace(w, top_p=tp), q, k, v, out, dev, stream, calls, peak)
+        r["top_p"] = tp
+        if sdpa:
+            r["sdpa_ms"] = sdpa
+            r["speedup_vs_sdpa"] = sdpa / r["ms_per_call"]
+        rows.append(r)
+    return rows
+
+
+def per_config(dev, stream, calls, peak):
+    """Every workload of the suite at full size, with the SDPA comparator."""
+    import torch
+    res = {}
+    for name in W.ORDER:
+        w = W.WORKLOADS[name]
+        hs = gen_inputs(w)
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        q, k, v = (torch.from_numpy(np.stack([getattr(h, a) for h in hs])).to(dev).to(tdt) for a in "qkv")
+        del hs
+        out = torch.empty_like(q)
+        r, flush = measure(w, q, k, v, out, dev, stream, calls, peak)
+        d = sdpa_ms(q, k, v, stream, flush)
+        r["sdpa_ms"] = d
+        r["sdpa_tflops"] = w.dense_flops() / (d * 1e-3) / 1e12
+        r["speedup_vs_sdpa"] = d / r["ms_per_call"]
+        res[name] = r
+        del q, k, v, out, flush
+        torch.cuda.empty_cache()
+    return res
 
 
 def denoise_steps(ac, q, k, v, out, steps, drift, stream):

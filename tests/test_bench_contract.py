@@ -32,9 +32,17 @@ def test_reference_arm_prints_one_complete_line():
         assert key in j, key
     assert j["impl"] == "reference" and j["unit"] == "calls/s" and j["higher_is_better"] is True
     assert j["steps"] == 2 and j["warmup"] == 1 and j["value"] > 0
-    assert abs(j["ms_per_step"] - 1e3 / j["value"]) < 1e-6 * j["ms_per_step"]
-    assert j["config"]["workload"] == SMALL
+    # a step is one bounded sample: steps x ms_per_step is the measured wall
+    # time, and value extrapolates the samples to whole calls
+    assert j["extrapolated"] is True
     cb = j["cpu_baseline"]
+    assert cb["samples_timed"] == 2 and abs(cb["wall_s"] - 2 * j["ms_per_step"] / 1e3) < 1e-6 * cb["wall_s"]
+    assert cb["scale_per_sample"] > 1
+    assert j["config"]["workload"] == SMALL
+    import bench
+    from clustered_sparse_attention_head_b200 import workloads as W
+    assert j["config"] == bench.config_of(W.WORKLOADS[SMALL], 1), "the reference config must equal the GPU arm's"
+    assert "flushed" in j["config"]["l2"], "a workload smaller than L2 is timed with an L2 flush"
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
     assert j["e2e"] == {"value": j["value"], "unit": "calls/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
@@ -43,6 +51,14 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run(["--impl", "reference", "--workload", SMALL, "--steps", "1", "--warmup", "0"],
              env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0 and not r.stdout.strip()
+
+
+def test_l2_policy_follows_the_tensor_size():
+    import bench
+    from clustered_sparse_attention_head_b200 import workloads as W
+    big = bench.config_of(W.WORKLOADS["wan21-n75600-h40-d128"], 1)["l2"]
+    assert big.startswith("inputs larger than L2 (774 MB per tensor)")
+    assert "flushed" in bench.config_of(W.WORKLOADS["cogvideox2b-n17776-h30-d64"], 1)["l2"]
 
 
 def test_gpu_arm_fails_loudly_without_a_device():
