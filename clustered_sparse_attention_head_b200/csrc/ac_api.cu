@@ -2,6 +2,7 @@
 // orchestration of AdaCluster's Algorithm 3 ("AdaCluster: Adaptive Query-Key
 // Clustering for Sparse Attention in Video Generation", §3.3).  All compute
 // runs in the kernels of this directory; this file only launches them.
+#include <algorithm>
 #include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -68,6 +69,9 @@ struct Ws {
     size_t aprev, kst, seg2;
     // selection: the key centroids transposed per head
     size_t kct;
+    // Algorithm 1's single-cluster stages on chip: working vectors [H, wrows, d] (double)
+    size_t wc;
+    int wrows;
     int kpad;
     size_t total;
 };
@@ -137,6 +141,11 @@ Ws layout(const ac_ctx *c) {
     w.kst = b.take(3 * H * 4 * 4);
     w.seg2 = b.take(H * sizeof(HeadSeg));
     w.kct = b.take(H * (size_t)c->kk_cap * D * 4);
+    // a stage with m_t = ceil(m0 |U| / N) = 1 has |U| <= N / m0
+    w.wrows = 0;
+    if (g.adaptive_q) w.wrows = (int)(N / g.kq + 1);
+    if (g.adaptive_k) w.wrows = std::max(w.wrows, (int)(N / g.kk + 1));
+    w.wc = b.take(H * (size_t)w.wrows * D * 8);
     w.total = b.off;
     return w;
 }
@@ -275,7 +284,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
     double *dist = at<double>(ws, w.dist);
     MsHead *ms = at<MsHead>(ws, w.ms);
     k_ms_init(H, N, Nc, ms, U, Un, st);
-    int stages = 0;
+    bool on_chip = false;
     for (int t = 0;; t++) {
         k_ms_control(H, Nc, k, nmax, cap - (text > 0 ? 1 : 0), ms, seg, c->d_info, status, st);
         AC_CUDA(cudaMemcpyAsync(c->h_info, c->d_info, 8 * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
@@ -283,7 +292,16 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         if (c->h_info[4]) return AC_ERR_CAPACITY;
         if (c->h_info[0] == 0) break;
         const int mnu = c->h_info[1], mmt = c->h_info[2];
-        stages = t + 1;
+        // From the first stage after tau is fixed on, once every active head
+        // has m_t = 1, all their remaining stages are single-cluster stages:
+        // one kernel runs them all on chip (one CTA per head), without a host
+        // round trip per stage.  The next control pass finds every head done.
+        if (t >= 1 && mmt == 1 && !on_chip && w.wrows > 0) {
+            k_ms_single(x, dt, H, N, D, Nc, k, nmax, cap - (text > 0 ? 1 : 0), g.iters, norm, mode, U, Un,
+                        at<double>(ws, w.wc), w.wrows, ms, cent, cap, status, st);
+            on_chip = true;
+            continue;
+        }
         // A stage whose every active head has one cluster (mmt = 1) is
         // complete after one round: all its rows are assigned to cluster 0, so
         // the first update already gives the centre every later round repeats
@@ -322,11 +340,16 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         AC_CUDA(cudaGetLastError());
     }
     k_ms_final(H, Nc, ms, seg, ncl, flag, c->d_info, st);
+    if (max_stages) {
+        // stages run by the host loop and on chip: max over heads (info[6])
+        AC_CUDA(cudaMemcpyAsync(c->h_info, c->d_info, 8 * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+        AC_CUDA(cudaStreamSynchronize(st));
+        *max_stages = c->h_info[6];
+    }
     AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
     k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
     if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
     if (text > 0) k_text_group(H, N, Nc, seg, assign, count, cap, ncl, st);
-    if (max_stages) *max_stages = stages;
     return launch_check();
 }
 
@@ -613,11 +636,13 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
         AC_CUDA(cudaMemsetAsync(kst, 0, sizeof(int32_t) * 8 * g.heads, st));
         AC_CUDA(cudaEventRecord(c->ev[0], st));
     }
-    ac_status s = run_cluster(c, MODE_SPHERE, q, f.q_init, qa, qc, qn, qmn, nq, dq, ws, st, &sq, f.nq_fixed, f.dq_fixed);
+    ac_status s = run_cluster(c, MODE_SPHERE, q, f.q_init, qa, qc, qn, qmn, nq, dq, ws, st, stats ? &sq : nullptr,
+                              f.nq_fixed, f.dq_fixed);
     if (s != AC_OK) return s;
     if (pe) AC_CUDA(cudaEventRecord(pe[1], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[1], st));
-    s = run_cluster(c, MODE_EUCLID, k, f.k_init, ka, kc, kn, nullptr, nk, dk, ws, st, &sk, f.nk_fixed, f.dk_fixed);
+    s = run_cluster(c, MODE_EUCLID, k, f.k_init, ka, kc, kn, nullptr, nk, dk, ws, st, stats ? &sk : nullptr,
+                    f.nk_fixed, f.dk_fixed);
     if (s != AC_OK) return s;
     if (pe) AC_CUDA(cudaEventRecord(pe[2], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[2], st));

@@ -8,6 +8,15 @@ enum { MODE_EUCLID = 0, MODE_SPHERE = 1 };
 enum { DT_F32 = 0, DT_BF16 = 1 };
 constexpr int SORT_TILE = 1024;  // positions per rank/histogram tile (one CTA of 4 warps)
 
+// Working value of element t of a row: x (EUCLID) or x/||x|| (SPHERE), in
+// double (nrm = ||x|| in double; a zero row stays zero).
+template <typename T>
+__device__ __forceinline__ double work_val(const T *xi, int t, int mode, double nrm) {
+    double v = (double)to_f(xi[t]);
+    if (mode == MODE_SPHERE) return nrm > 0.0 ? ddiv(v, nrm) : 0.0;
+    return v;
+}
+
 // Host-side count of kernels this library has launched (profiling).
 void note_launch();
 long long launches_total();

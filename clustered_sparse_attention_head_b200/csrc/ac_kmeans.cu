@@ -50,13 +50,6 @@ __global__ void __launch_bounds__(256)
     norm[(size_t)h * N + r] = sqrt(ss);
 }
 
-// Working value of element t of token tok: x (EUCLID) or x/||x|| (SPHERE).
-template <typename T>
-__device__ __forceinline__ double work_val(const T *xi, int t, int mode, double nrm) {
-    double v = (double)to_f(xi[t]);
-    if (mode == MODE_SPHERE) return nrm > 0.0 ? ddiv(v, nrm) : 0.0;
-    return v;
-}
 
 // ------------------------------------------------------------------- init
 // Centroid j of the pass = working vector of listed row floor(j * nrows / k).
@@ -390,6 +383,127 @@ __global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__r
     if (snr > 0.0) c[t] = (float)ddiv(acc, snr);
 }
 
+// Same result as update_kernel, with the member rows staged through shared
+// memory.  The rows of cluster j are perm[off[j] .. off[j+1]) (token order);
+// chunks of R rows are copied by cp.async as 16-byte pieces (every thread
+// copies pieces of several rows, so a CTA keeps up to two chunks in flight
+// while it sums a third), and thread t adds element t of the chunk's rows in
+// order, in double.  On the sphere the working value x/||x|| is the correctly
+// rounded quotient, computed from y = RN(1/||x||) (one per row) with
+// Markstein's correction (q = RN(x y), r = x - ||x|| q exactly by FMA,
+// RN(q + r y) = RN(x / ||x||); Markstein 1990, see Muller et al., Handbook of
+// Floating-Point Arithmetic, on division by FMA), the value plain division
+// gives.
+namespace {
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int NPEND> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(NPEND) : "memory");
+}
+}  // namespace
+
+constexpr int UPD_THREADS = 128, UPD_STAGES = 3, UPD_CHUNK_BYTES = 16384;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restrict__ x, int N,
+                                                             const HeadSeg *__restrict__ seg,
+                                                             const int32_t *__restrict__ perm,
+                                                             const int32_t *__restrict__ off, int cap,
+                                                             const double *__restrict__ norm, int mode,
+                                                             float *__restrict__ cent) {
+    constexpr int ROW_BYTES = D * (int)sizeof(T);
+    constexpr int R = UPD_CHUNK_BYTES / ROW_BYTES;   // rows per chunk
+    constexpr int PIECES = ROW_BYTES / 16;           // 16-byte pieces per row
+    extern __shared__ __align__(16) unsigned char upd_smem[];
+    T *rows = reinterpret_cast<T *>(upd_smem);                                           // [S][R][D]
+    double *nrm = reinterpret_cast<double *>(upd_smem + UPD_STAGES * UPD_CHUNK_BYTES);  // [S][R]
+    double *rcp = nrm + UPD_STAGES * R;                                                  // [S][R]
+    __shared__ double ssum[D];
+    __shared__ double snr;
+    const int h = blockIdx.y, j = blockIdx.x, tid = threadIdx.x;
+    const HeadSeg s = seg[h];
+    if (s.nrows <= 0 || j >= s.k) return;
+    const int32_t *o = off + (size_t)h * (cap + 1);
+    const int b = o[j], e = o[j + 1];
+    if (e <= b) return;
+    const int n = e - b, nchunks = (n + R - 1) / R;
+    const int32_t *ph = perm + (size_t)h * N + b;
+    const T *xh = x + (size_t)h * N * D;
+    const double *nh = norm + (size_t)h * N;
+    const bool sphere = mode == MODE_SPHERE;
+    // copy chunk c into stage c % S (one commit group per chunk, also when empty)
+    auto issue = [&](int c) {
+        if (c < nchunks) {
+            const int r0 = c * R, nr = min(R, n - r0), st = c % UPD_STAGES;
+            unsigned char *dst = reinterpret_cast<unsigned char *>(rows) + (size_t)st * UPD_CHUNK_BYTES;
+            for (int pc = tid; pc < nr * PIECES; pc += UPD_THREADS) {
+                const int r = pc / PIECES, q = pc - r * PIECES;
+                const int tok = ph[r0 + r];
+                cp_async16(dst + r * ROW_BYTES + q * 16,
+                           reinterpret_cast<const unsigned char *>(xh + (size_t)tok * D) + q * 16);
+            }
+            if (sphere)
+                for (int r = tid; r < nr; r += UPD_THREADS) cp_async8(nrm + st * R + r, nh + ph[r0 + r]);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int c = 0; c < UPD_STAGES - 1; c++) issue(c);
+    double acc = 0.0;
+    for (int c = 0; c < nchunks; c++) {
+        cp_async_wait<UPD_STAGES - 2>();
+        __syncthreads();  // chunk c has landed for every thread; stage (c - 1) % S is free
+        const int st = c % UPD_STAGES, nr = min(R, n - c * R);
+        if (sphere) {
+            for (int r = tid; r < nr; r += UPD_THREADS) {
+                const double v = nrm[st * R + r];
+                rcp[st * R + r] = v > 0.0 ? __drcp_rn(v) : 0.0;
+            }
+            __syncthreads();
+        }
+        issue(c + UPD_STAGES - 1);
+        if (tid < D) {
+            const T *rs = rows + (size_t)st * R * D + tid;
+            if (sphere) {
+                const double *nr_s = nrm + st * R, *rc_s = rcp + st * R;
+                for (int r = 0; r < nr; r++) {
+                    const double v = (double)to_f(rs[r * D]);
+                    const double bn = nr_s[r], y = rc_s[r];
+                    double q = 0.0;
+                    if (bn > 0.0) {
+                        const double q0 = dmul(v, y);
+                        const double rr = __fma_rn(-bn, q0, v);
+                        q = __fma_rn(rr, y, q0);
+                    }
+                    acc = dadd(acc, q);
+                }
+            } else {
+                for (int r = 0; r < nr; r++) acc = dadd(acc, (double)to_f(rs[r * D]));
+            }
+        }
+    }
+    cp_async_wait<0>();
+    float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
+    if (!sphere) {
+        if (tid < D) c[tid] = (float)ddiv(acc, (double)n);
+        return;
+    }
+    if (tid < D) ssum[tid] = acc;
+    __syncthreads();
+    if (tid == 0) {
+        double ss = 0.0;
+        for (int u = 0; u < D; u++) ss = dadd(ss, dmul(ssum[u], ssum[u]));
+        snr = sqrt(ss);
+    }
+    __syncthreads();
+    if (tid < D && snr > 0.0) c[tid] = (float)ddiv(acc, snr);
+}
+
 // Mean ||q|| over the members of each cluster (sequential double sum in
 // token order); 0 for empty clusters.
 __global__ void mean_norm_kernel(int N, const HeadSeg *__restrict__ seg, const int32_t *__restrict__ perm,
@@ -512,8 +626,14 @@ void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, 
 void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg, int kmax, const int32_t *perm,
               const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st) {
     dim3 g(kmax, H);
-#define AC_UPD(T, DD) \
-    update_kernel<T, DD><<<g, DD, 0, st>>>((const T *)x, N, seg, perm, off, cap, norm, mode, cent)
+    // staged rows (16 KB chunks, three stages) plus the rows' norms and reciprocals
+#define AC_UPD(T, DD)                                                                                             \
+    do {                                                                                                          \
+        constexpr int R_ = UPD_CHUNK_BYTES / (DD * (int)sizeof(T));                                               \
+        constexpr int SM_ = UPD_STAGES * (UPD_CHUNK_BYTES + 2 * R_ * 8);                                          \
+        cudaFuncSetAttribute(update2_kernel<T, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM_);             \
+        update2_kernel<T, DD><<<g, UPD_THREADS, SM_, st>>>((const T *)x, N, seg, perm, off, cap, norm, mode, cent); \
+    } while (0)
     if (dtype == DT_BF16) {
         if (D == 64) AC_UPD(__nv_bfloat16, 64);
         else AC_UPD(__nv_bfloat16, 128);

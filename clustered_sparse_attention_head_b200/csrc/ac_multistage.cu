@@ -196,8 +196,11 @@ __global__ void ms_remove_kernel(int N, const HeadSeg *__restrict__ seg, const d
 // nclusters and the flag F.
 __global__ void ms_final_kernel(int H, int nrows, const MsHead *__restrict__ st, HeadSeg *__restrict__ seg,
                                 int32_t *__restrict__ ncl, uint8_t *__restrict__ flag, int32_t *__restrict__ info) {
-    __shared__ int mnc;
-    if (threadIdx.x == 0) mnc = 0;
+    __shared__ int mnc, mst;
+    if (threadIdx.x == 0) {
+        mnc = 0;
+        mst = 0;
+    }
     __syncthreads();
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
         MsHead s = st[h];
@@ -210,9 +213,13 @@ __global__ void ms_final_kernel(int H, int nrows, const MsHead *__restrict__ st,
         if (ncl) ncl[h] = s.nc;
         if (flag) flag[h] = (uint8_t)s.flag;
         atomicMax(&mnc, s.nc);
+        atomicMax(&mst, s.stage);
     }
     __syncthreads();
-    if (threadIdx.x == 0) info[5] = mnc;
+    if (threadIdx.x == 0) {
+        info[5] = mnc;
+        info[6] = mst;
+    }
 }
 
 __global__ void seg_uniform_kernel(int H, int nrows, int k, HeadSeg *__restrict__ seg, int32_t *__restrict__ ncl,
@@ -243,6 +250,165 @@ __global__ void seg_from_counts_kernel(int H, int nrows, const int32_t *__restri
     g.cent_off = 0;
     g.pad = 0;
     seg[h] = g;
+}
+
+// ---------------------------------------------------------------------------
+// Single-cluster stages on chip.  Once a head's stage size m_t is 1 it stays 1
+// (m_t = min(|U|, ceil(m0 |U| / N)) cannot grow while |U| shrinks), so every
+// remaining stage of the head clusters U into one cluster.  Such a stage is
+// complete after one k-means round: every row goes to cluster 0, so the first
+// update gives the centre every later round repeats.  One CTA per head runs all
+// of the head's remaining stages back to back, with the arithmetic and order
+// of the host-driven stage:
+//   init   c = working vector of U's first row (kept if iters = 0, or on the
+//          sphere when the member sum is zero);
+//   update s_t = sum over U in list (token) order of w_i[t], in double;
+//          EUCLID c_t = s_t / |U|; SPHERE c_t = s_t / sqrt(sum_t s_t^2);
+//   d_i    = sqrt(sum over t in order of (w_i[t] - c_t)^2) with c as stored (fp32);
+//   U     <- the rows with !(d_i < tau), order kept; |C| += 1.
+// The control of every stage is ms_control_kernel's: |U| = 0 ends the head,
+// |C| >= N_max sets F and ends it, |C| + 1 > capacity records ST_CAPACITY.
+// The working vectors of the rows in U when the kernel starts are computed once
+// into wc (double, [H, wrows, D], row = position in that first list), and U is
+// replaced by positions into wc as the stages shrink it.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) ms_single_kernel(const T *__restrict__ x, int N, int nrows, int m0, int nmax,
+                                                        int cap_c, int iters, const double *__restrict__ norm,
+                                                        int mode, int32_t *__restrict__ Ua, int32_t *__restrict__ Ub,
+                                                        double *__restrict__ wc, int wrows, MsHead *__restrict__ st,
+                                                        float *__restrict__ cent, int cap, int *status) {
+    __shared__ double ssum[D];
+    __shared__ float cs[D];
+    __shared__ double snr;
+    __shared__ int wsum[8];
+    __shared__ int base;
+    const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    MsHead s = st[h];  // every thread keeps the same copy; thread 0 writes it back
+    if (s.done || s.nu <= 0) return;
+    if (s.nu > wrows) {  // cannot happen when m_t = 1 (|U| <= N / m0); left to the host loop
+        return;
+    }
+    int32_t *U = Ua + (size_t)h * N, *P = Ub + (size_t)h * N;
+    const T *xh = x + (size_t)h * N * D;
+    const double *nh = norm + (size_t)h * N;
+    double *wh = wc + (size_t)h * wrows * D;
+    // working vectors of U, in list order; positions replace tokens from here on
+    for (int e = tid; e < s.nu * D; e += blockDim.x) {
+        const int r = e / D, t = e - r * D;
+        const int tok = U[r];
+        wh[e] = work_val(xh + (size_t)tok * D, t, mode, nh[tok]);
+    }
+    for (int r = tid; r < s.nu; r += blockDim.x) P[r] = r;
+    int32_t *Pn = U;  // the other buffer
+    __syncthreads();
+    for (;;) {
+        // ---- control (every thread takes the same decision)
+        if (s.nu <= 0) { s.done = 1; break; }
+        if (s.nc >= nmax) { s.flag = 1; s.done = 1; break; }
+        const long long num = (long long)m0 * s.nu;
+        int mt = (int)((num + nrows - 1) / nrows);
+        if (mt > s.nu) mt = s.nu;
+        if (mt != 1) break;  // not a single-cluster stage: back to the host loop
+        if (s.nc + 1 > cap_c) {
+            if (tid == 0) set_status(status, ST_CAPACITY);
+            s.done = 1;
+            break;
+        }
+        // ---- centre: init, then (iters >= 1) the update over U in list order
+        const int p0 = P[0];
+        if (tid < D) {
+            cs[tid] = (float)wh[(size_t)p0 * D + tid];
+            if (iters > 0) {
+                double acc = 0.0;
+                int i = 0;
+                for (; i + 8 <= s.nu; i += 8) {
+                    double v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; u++) v[u] = wh[(size_t)P[i + u] * D + tid];
+#pragma unroll
+                    for (int u = 0; u < 8; u++) acc = dadd(acc, v[u]);
+                }
+                for (; i < s.nu; i++) acc = dadd(acc, wh[(size_t)P[i] * D + tid]);
+                ssum[tid] = acc;
+            }
+        }
+        __syncthreads();
+        if (iters > 0) {
+            if (mode == MODE_EUCLID) {
+                if (tid < D) cs[tid] = (float)ddiv(ssum[tid], (double)s.nu);
+            } else {
+                if (tid == 0) {
+                    double ss = 0.0;
+                    for (int u = 0; u < D; u++) ss = dadd(ss, dmul(ssum[u], ssum[u]));
+                    snr = sqrt(ss);
+                }
+                __syncthreads();
+                if (tid < D && snr > 0.0) cs[tid] = (float)ddiv(ssum[tid], snr);
+            }
+        }
+        __syncthreads();
+        if (tid < D) cent[((size_t)h * cap + s.nc) * D + tid] = cs[tid];
+        // ---- distances to the centre and ordered compaction of the rows kept
+        if (tid == 0) base = 0;
+        __syncthreads();
+        for (int q0 = 0; q0 < s.nu; q0 += blockDim.x) {
+            const int i = q0 + tid;
+            int keep = 0, pi = 0;
+            if (i < s.nu) {
+                pi = P[i];
+                const double2 *row = reinterpret_cast<const double2 *>(wh + (size_t)pi * D);
+                double acc = 0.0;
+#pragma unroll 4
+                for (int t2 = 0; t2 < D / 2; t2++) {
+                    const double2 v = row[t2];
+                    const double d0 = dsub(v.x, (double)cs[2 * t2]);
+                    acc = dadd(acc, dmul(d0, d0));
+                    const double d1 = dsub(v.y, (double)cs[2 * t2 + 1]);
+                    acc = dadd(acc, dmul(d1, d1));
+                }
+                keep = !(sqrt(acc) < s.tau);
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0) wsum[w] = __popc(bal);
+            __syncthreads();
+            int before = base;
+            for (int u = 0; u < w; u++) before += wsum[u];
+            if (keep) Pn[before + __popc(bal & ((1u << lane) - 1u))] = pi;
+            __syncthreads();
+            if (tid == 0) {
+                int tt = 0;
+                for (int u = 0; u < (int)(blockDim.x >> 5); u++) tt += wsum[u];
+                base += tt;
+            }
+            __syncthreads();
+        }
+        s.nu = base;
+        s.nc += 1;
+        s.stage += 1;
+        int32_t *tmp = P;
+        P = Pn;
+        Pn = tmp;
+        __syncthreads();  // this stage's reads of base and P are done before the next stage writes them
+    }
+    if (tid == 0) st[h] = s;
+}
+
+int k_ms_single(const void *x, int dtype, int H, int N, int D, int nrows, int m0, int nmax, int cap_c, int iters,
+                const double *norm, int mode, int32_t *U, int32_t *U2, double *wc, int wrows, MsHead *st,
+                float *cent, int cap, int *status, cudaStream_t s) {
+#define AC_MS_SINGLE(T, DD)                                                                                     \
+    ms_single_kernel<T, DD><<<H, 256, 0, s>>>(static_cast<const T *>(x), N, nrows, m0, nmax, cap_c, iters, norm, \
+                                              mode, U, U2, wc, wrows, st, cent, cap, status)
+    if (dtype == DT_BF16) {
+        if (D == 64) AC_MS_SINGLE(__nv_bfloat16, 64);
+        else AC_MS_SINGLE(__nv_bfloat16, 128);
+    } else {
+        if (D == 64) AC_MS_SINGLE(float, 64);
+        else AC_MS_SINGLE(float, 128);
+    }
+#undef AC_MS_SINGLE
+    note_launch();
+    return 0;
 }
 
 void k_ms_init(int H, int N, int nrows, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s) {

@@ -22,6 +22,12 @@ void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double
               const int32_t *off, int cap, int kmax, MsHead *st, cudaStream_t s);
 void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int32_t *U, int32_t *Unext, MsHead *st,
                  cudaStream_t s);
+// Every remaining single-cluster stage of each head on chip (one CTA per
+// head); wc: [H, wrows, D] doubles of scratch, wrows >= the largest |U| with
+// m_t = 1 (N / m0).  A head whose |U| exceeds wrows is left to the host loop.
+int k_ms_single(const void *x, int dtype, int H, int N, int D, int nrows, int m0, int nmax, int cap_c, int iters,
+                const double *norm, int mode, int32_t *U, int32_t *U2, double *wc, int wrows, MsHead *st,
+                float *cent, int cap, int *status, cudaStream_t s);
 void k_ms_final(int H, int nrows, const MsHead *st, HeadSeg *seg, int32_t *ncl, uint8_t *flag, int32_t *info,
                 cudaStream_t s);
 void k_seg_uniform(int H, int nrows, int k, HeadSeg *seg, int32_t *ncl, uint8_t *flag, cudaStream_t s);

@@ -99,7 +99,7 @@ def test_static_sort_large_cap_matches_workspace_sort():
     from clustered_sparse_attention_head_b200.api import AdaCluster, Config
     build()
     lib = _abi.load()
-    heads, n, cap = 2, 3001, 4096
+    heads, n, cap = 2, 4099, 4096  # a context needs n >= its cluster count
     ncl = np.array([4096, 3000], np.int32)
     ref_ctx = AdaCluster(Config(heads=heads, n=n, d=64, kq=cap, kk=cap))
     ncl_t = torch.from_numpy(ncl).cuda()
