@@ -236,6 +236,29 @@ def select2(q_cent, q_mean_norm, q_count, k_cent, k_count, top_p=0.9, score_mode
     return sel, cnt
 
 
+def select_per_query(q_rows, k_cent, k_count, top_p=0.9, score_mode=SCORE_CENTROID, top_k=0, k_max=None,
+                     k_min=None):
+    """Per-query selection (AdaCluster §3.3, Algorithm 3: the score matrix S has
+    one row per query token and argtopk runs along each row).  Each query row is
+    scored as its own one-member cluster: its representative is the query itself
+    (centroid = q, mean norm 1), so s_ib = q_i . c_b / sqrt(d) (CENTROID) or the
+    Quest bound of q_i against cluster b (QUEST), and the cut is select2's.
+    Returns (sel_idx, sel_cnt) with one row per query row."""
+    q_rows = _f32(q_rows)
+    n = q_rows.shape[0]
+    return select2(q_rows, np.ones(n, np.float32), np.ones(n, np.int32), k_cent, k_count, top_p, score_mode, top_k,
+                   k_max, k_min)
+
+
+def attend_per_query(q, k, v, k_assign, kk, sel_rows, cnt_rows, rows):
+    """Attention of each listed query row over the keys of its own selected
+    clusters (row i of sel_rows / cnt_rows belongs to rows[i])."""
+    rows = _i32(rows)
+    qa = np.zeros(q.shape[0], np.int32)
+    qa[rows] = np.arange(len(rows), dtype=np.int32)
+    return attention_rows(q, k, v, qa, k_assign, kk, sel_rows, cnt_rows, 0, rows)
+
+
 def scores(q_cent, q_mean_norm, k_cent=None, score_mode=SCORE_CENTROID, k_max=None, k_min=None):
     """The selection score s_ab of every (query cluster, key cluster) pair."""
     q_cent = _f32(q_cent)
@@ -302,6 +325,7 @@ class HeadSpec:
     score_mode: int = 0   # SCORE_CENTROID or SCORE_QUEST
     top_k: int = 0        # > 0: argtopk instead of top-p
     text_keys: int = 0    # > 0: the last text_keys keys are always attended, not clustered
+    per_query: bool = False  # selection per query row (Algorithm 3's argtopk along S's rows)
 
 
 @dataclass
@@ -391,5 +415,21 @@ def _select_attend(q, k, v, rq, rk, qmn, dense, spec: HeadSpec, rows):
             cnt[live] += 1
     if rows is None:
         rows = np.arange(q.shape[0], dtype=np.int32)
+    if spec.per_query and not dense:
+        # every evaluated row selects for itself; the per-cluster selection above
+        # is kept in the result for reference
+        kmax = kmin = None
+        if spec.score_mode == SCORE_QUEST:
+            kmax, kmin = key_bounds(kv, rk.assign, nv)
+        rows = np.asarray(rows, np.int32)
+        sq, cq = select_per_query(q[rows], rk.cent[:nv], rk.count, spec.top_p, spec.score_mode, spec.top_k, kmax,
+                                  kmin)
+        if spec.text_keys:
+            sq = np.concatenate([sq, np.full((sq.shape[0], 1), -1, np.int32)], axis=1)
+            sq[np.arange(len(rows)), cq] = nv
+            cq = cq + 1
+        out = attend_per_query(q, k, v, k_assign, nv + (1 if spec.text_keys else 0), sq, cq, rows)
+        return HeadResult(rq, rk, qmn, sel, cnt, dense, out, rows,
+                          extra={"k_assign": k_assign, "sel_rows": sq, "cnt_rows": cq})
     out = attention_rows(q, k, v, rq.assign, k_assign, nv + (1 if spec.text_keys else 0), sel, cnt, dense, rows)
     return HeadResult(rq, rk, qmn, sel, cnt, dense, out, np.asarray(rows, np.int32), extra={"k_assign": k_assign})

@@ -70,6 +70,13 @@ MUTATIONS = [
      "keys += k_count[sel_idx[(int64_t)a * kk_stride + c]];", "keys += q_count[sel_idx[(int64_t)a * kk_stride + c] % kq];"),
     ("pair count of the last query cluster dropped", "for (int a = 0; a < kq; a++) {\n        int64_t keys = 0;",
      "for (int a = 0; a < kq - 1; a++) {\n        int64_t keys = 0;"),
+    ("per-query score of the normalised query", "    q_rows = _f32(q_rows)\n    n = q_rows.shape[0]",
+     "    q_rows = _f32(q_rows / np.linalg.norm(q_rows, axis=1, keepdims=True))\n    n = q_rows.shape[0]",
+     "__init__.py"),
+    ("per-query rows attend with their cluster's selection",
+     "out = attend_per_query(q, k, v, k_assign, nv + (1 if spec.text_keys else 0), sq, cq, rows)",
+     "out = attention_rows(q, k, v, rq.assign, k_assign, nv + (1 if spec.text_keys else 0), sel, cnt, dense, rows)",
+     "__init__.py"),
     ("text group also for empty query clusters",
      "live = np.nonzero(np.asarray(rq.count)[:sel.shape[0]] > 0)[0]", "live = np.arange(sel.shape[0])",
      "__init__.py"),

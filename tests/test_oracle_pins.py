@@ -761,3 +761,112 @@ def test_pairs_brute_force_over_tokens(orc):
     q_count = np.bincount(qa, minlength=kq).astype(np.int32)
     k_count = np.bincount(ka, minlength=kk).astype(np.int32)
     assert orc.pairs(q_count, k_count, sel, sel_cnt) == brute
+
+
+# ------------------------------------------------- per-query selection (f2)
+def _np_attention_row(q, k, v, allowed):
+    s = (k[allowed].astype(np.float64) @ q.astype(np.float64)) / math.sqrt(q.shape[0])
+    w = np.exp(s - s.max())
+    return (w[:, None] * v[allowed].astype(np.float64)).sum(0) / w.sum()
+
+
+def test_per_query_hand_example(orc):
+    """Algorithm 3 selects along each row of S (one row per query): two queries
+    of one query cluster that point at different key clusters each keep their
+    own best cluster under argtopk with top_k = 1, and attend to its keys only;
+    the per-cluster selection would give both the same cluster."""
+    k = np.array([[3, 0], [2.5, 0.5], [0, 3], [0.5, 2.5]], np.float32)
+    v = np.array([[1, 0], [2, 0], [0, 1], [0, 2]], np.float32)
+    ka = np.array([0, 0, 1, 1], np.int32)
+    cent = np.array([[2.75, 0.25], [0.25, 2.75]], np.float32)
+    # one token count for queries and keys (rows 2 and 3 are not evaluated)
+    q = np.array([[4, 0.1], [0.1, 4], [1, 1], [1, -1]], np.float32)
+    sel, cnt = orc.select_per_query(q[:2], cent, np.array([2, 2], np.int32), top_k=1)
+    assert cnt.tolist() == [1, 1] and sel[0, 0] == 0 and sel[1, 0] == 1
+    out = orc.attend_per_query(q, k, v, ka, 2, sel, cnt, np.array([0, 1], np.int32))
+    np.testing.assert_allclose(out[0], _np_attention_row(q[0], k, v, ka == 0), rtol=1e-12)
+    np.testing.assert_allclose(out[1], _np_attention_row(q[1], k, v, ka == 1), rtol=1e-12)
+    # as one cluster (representative = the mean of the two queries) both rows share one set
+    qc = q[:2].mean(0, keepdims=True) / np.linalg.norm(q[:2].mean(0))
+    sel_c, cnt_c = orc.select2(qc.astype(np.float32), np.array([np.linalg.norm(q[:2], axis=1).mean()], np.float32),
+                               np.array([2], np.int32), cent, np.array([2, 2], np.int32), top_k=1)
+    assert cnt_c.tolist() == [1]
+
+
+def test_per_query_argtopk_matches_numpy_ranking(orc):
+    """argtopk per row equals numpy's ranking of q . c_b (separated random data,
+    no near-ties), empty clusters never kept; QUEST scores the Quest bound of
+    the query itself."""
+    rng = np.random.default_rng(12)
+    d, kk, n = 16, 23, 40
+    cent = rng.standard_normal((kk, d)).astype(np.float32)
+    cnt = rng.integers(1, 9, kk).astype(np.int32)
+    cnt[[4, 17]] = 0
+    q = rng.standard_normal((n, d)).astype(np.float32)
+    sel, c = orc.select_per_query(q, cent, cnt, top_k=5)
+    s = q.astype(np.float64) @ cent.astype(np.float64).T
+    s[:, cnt == 0] = -np.inf
+    for i in range(n):
+        want = np.sort(np.argsort(-s[i], kind="stable")[:5])
+        assert c[i] == 5 and sel[i, :5].tolist() == want.tolist()
+    kmax = cent + np.abs(rng.standard_normal((kk, d))).astype(np.float32)
+    kmin = cent - np.abs(rng.standard_normal((kk, d))).astype(np.float32)
+    sel, c = orc.select_per_query(q, cent, cnt, score_mode=orc.SCORE_QUEST, top_k=3, k_max=kmax, k_min=kmin)
+    qd = q.astype(np.float64)[:, None, :]
+    sq = np.maximum(qd * kmax[None].astype(np.float64), qd * kmin[None].astype(np.float64)).sum(2)
+    sq[:, cnt == 0] = -np.inf
+    for i in range(n):
+        assert sel[i, :3].tolist() == np.sort(np.argsort(-sq[i], kind="stable")[:3]).tolist()
+
+
+def test_per_query_top_p_matches_numpy_cut(orc):
+    """The top-p cut per query row: weights n_b exp(q . c_b / sqrt(d)), shares
+    in decreasing order (ties to the lower b), shortest prefix reaching top_p;
+    the query is not normalised (its scale sets the softmax temperature)."""
+    rng = np.random.default_rng(3)
+    d, kk, n = 8, 12, 30
+    cent = rng.standard_normal((kk, d)).astype(np.float32)
+    cnt = rng.integers(1, 20, kk).astype(np.int32)
+    q = (3.0 * rng.standard_normal((n, d))).astype(np.float32)
+    for tp in (0.5, 0.9):
+        sel, c = orc.select_per_query(q, cent, cnt, top_p=tp)
+        s = (q.astype(np.float64) @ cent.astype(np.float64).T) / math.sqrt(d)
+        for i in range(n):
+            w = cnt * np.exp(s[i] - s[i].max())
+            pr = w / w.sum()
+            order = np.argsort(-pr, kind="stable")
+            k = int(np.searchsorted(np.cumsum(pr[order]), tp) + 1)
+            assert sel[i, :c[i]].tolist() == np.sort(order[:k]).tolist(), (tp, i)
+
+
+def test_per_query_select_all_is_dense(orc):
+    """top_k at least the number of key clusters: every row attends to every key."""
+    rng = np.random.default_rng(8)
+    n, d = 60, 8
+    q, k, v = (rng.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    spec = orc.HeadSpec(kq=4, kk=5, iters=3, top_k=5, per_query=True)
+    r = orc.forward_head(q, k, v, spec, rows=np.arange(0, n, 7, dtype=np.int32))
+    for i, row in enumerate(r.rows):
+        np.testing.assert_allclose(r.out_rows[i], _np_attention_row(q[row], k, v, np.ones(n, bool)), rtol=1e-10)
+
+
+def test_per_query_forward_rows_use_their_own_sets(orc):
+    """forward_head with per-query argtopk (top_k = 2): each evaluated row
+    attends exactly to the keys of the two key clusters whose centroids score
+    highest against the row itself (numpy ranking of q . c over the oracle's
+    key clustering), which differs from its query cluster's set on some rows."""
+    w = W.small(W.WORKLOADS["wan21-n75600-h40-d128"], 600, heads=1, seed=4, kq=3, kk=9, outlier_frac=0.0)
+    x = W.head_inputs(w, 0)
+    spec = orc.HeadSpec(kq=3, kk=9, iters=4, top_k=2, per_query=True)
+    rows = np.arange(0, 600, 11, dtype=np.int32)
+    r = orc.forward_head(x.q, x.k, x.v, spec, rows=rows)
+    s = x.q[rows].astype(np.float64) @ r.k.cent.astype(np.float64).T
+    s[:, np.asarray(r.k.count) == 0] = -np.inf
+    differs = 0
+    for i, row in enumerate(rows):
+        top = np.argsort(-s[i], kind="stable")[:2]
+        allowed = np.isin(r.extra["k_assign"], top)
+        np.testing.assert_allclose(r.out_rows[i], _np_attention_row(x.q[row], x.k, x.v, allowed), rtol=1e-9, atol=1e-12)
+        a = int(r.q.assign[row])
+        differs += set(top.tolist()) != set(r.sel_idx[a, :r.sel_cnt[a]].tolist())
+    assert differs > 0, "the per-query sets should differ from the per-cluster ones somewhere"
