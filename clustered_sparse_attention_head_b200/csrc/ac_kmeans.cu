@@ -407,7 +407,8 @@ template <int NPEND> __device__ __forceinline__ void cp_async_wait() {
 }
 }  // namespace
 
-constexpr int UPD_THREADS = 128, UPD_STAGES = 3, UPD_CHUNK_BYTES = 16384;
+// 8 KB chunks, three stages: about 25 KB of shared memory, eight CTAs (clusters) per SM
+constexpr int UPD_THREADS = 128, UPD_STAGES = 3, UPD_CHUNK_BYTES = 8192;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restrict__ x, int N,
@@ -471,6 +472,7 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
             const T *rs = rows + (size_t)st * R * D + tid;
             if (sphere) {
                 const double *nr_s = nrm + st * R, *rc_s = rcp + st * R;
+#pragma unroll 8
                 for (int r = 0; r < nr; r++) {
                     const double v = (double)to_f(rs[r * D]);
                     const double bn = nr_s[r], y = rc_s[r];
@@ -483,6 +485,7 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
                     acc = dadd(acc, q);
                 }
             } else {
+#pragma unroll 8
                 for (int r = 0; r < nr; r++) acc = dadd(acc, (double)to_f(rs[r * D]));
             }
         }

@@ -81,7 +81,20 @@ __global__ void scan_tiles_kernel(const HeadSeg *__restrict__ seg, int cap, int 
     if (j < s.k && s.nrows > 0) {
         int nt = (s.nrows + SORT_TILE - 1) / SORT_TILE;
         int32_t *p = hist + (size_t)h * ntiles_max * cap + j;
-        for (int t = 0; t < nt; t++) {
+        // eight tiles' counts loaded before they are scanned, so the loads do
+        // not wait on one another
+        int t = 0;
+        for (; t + 8 <= nt; t += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) v[u] = p[(size_t)(t + u) * cap];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                p[(size_t)(t + u) * cap] = run;
+                run += v[u];
+            }
+        }
+        for (; t < nt; t++) {
             int v = p[(size_t)t * cap];
             p[(size_t)t * cap] = run;
             run += v;
