@@ -23,7 +23,7 @@ AC_SCORE_CENTROID, AC_SCORE_QUEST = 0, 1
 
 # every entry point declared in include/adacluster.h
 EXPORTS = ["ac_create", "ac_destroy", "ac_capacities", "ac_workspace_size", "ac_cluster_q", "ac_cluster_k",
-           "ac_select", "ac_key_bounds", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_step_state_size", "ac_step_state_parts", "ac_forward_step",
+           "ac_select", "ac_select_rows", "ac_sparse_attn_rows", "ac_key_bounds", "ac_cluster_sort", "ac_cluster_sort_static", "ac_sparse_attn", "ac_forward", "ac_step_state_size", "ac_step_state_parts", "ac_forward_step",
            "ac_profile_read", "ac_get_status", "ac_status_string", "ac_selftest_wait"]
 
 
@@ -31,14 +31,15 @@ class ac_config(ctypes.Structure):
     _fields_ = [("heads", c_int), ("n", c_int), ("d", c_int), ("dtype", c_int), ("kq", c_int), ("kk", c_int),
                 ("iters", c_int), ("adaptive_q", c_int), ("adaptive_k", c_int), ("tau_rule", c_int),
                 ("tau_value", c_double), ("nmax_q", c_int), ("nmax_k", c_int), ("top_p", c_double),
-                ("flags", c_uint), ("score_mode", c_int), ("top_k", c_int), ("text_keys", c_int)]
+                ("flags", c_uint), ("score_mode", c_int), ("top_k", c_int), ("text_keys", c_int),
+                ("per_query", c_int)]
 
 
 class ac_stats(ctypes.Structure):
     _fields_ = [("ms_cluster_q", c_double), ("ms_cluster_k", c_double), ("ms_select", c_double),
                 ("ms_sort", c_double), ("ms_attn", c_double), ("ms_total", c_double), ("pairs", c_int64),
                 ("dense_heads", c_int), ("max_stages_q", c_int), ("max_stages_k", c_int),
-                ("kmeans_rounds_q", c_int), ("kmeans_rounds_k", c_int)]
+                ("kmeans_rounds_q", c_int), ("kmeans_rounds_k", c_int), ("pairs_computed", c_int64)]
 
 
 class ac_profile(ctypes.Structure):
@@ -74,6 +75,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ac_cluster_k": ([P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_select": ([P, P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_key_bounds": ([P, P, P, P, P, P, P, c_size_t, P], c_int),
+        "ac_select_rows": ([P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
+        "ac_sparse_attn_rows": ([P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),
         "ac_cluster_sort": ([P, P, c_int, P, P, P, P, c_size_t, P], c_int),
         "ac_cluster_sort_static": ([P, c_int, c_int, c_int, P, P, P, P], c_int),
         "ac_sparse_attn": ([P, P, P, P, P, P, P, P, P, P, P, P, P, P, c_size_t, P], c_int),

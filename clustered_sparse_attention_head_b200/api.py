@@ -35,12 +35,14 @@ class Config:
     score_mode: int = _abi.AC_SCORE_CENTROID   # or AC_SCORE_QUEST
     top_k: int = 0                             # > 0: argtopk instead of top-p
     text_keys: int = 0                         # > 0: last text_keys keys always attended, not clustered
+    per_query: bool = False                    # selection per query row (argtopk along each row of S)
 
     def to_c(self) -> _abi.ac_config:
         return _abi.ac_config(self.heads, self.n, self.d, _abi.AC_BF16 if self.dtype == "bf16" else _abi.AC_F32,
                               self.kq, self.kk, self.iters, int(self.adaptive_q), int(self.adaptive_k),
                               self.tau_rule, float(self.tau_value), self.nmax_q, self.nmax_k, float(self.top_p),
-                              self.flags, int(self.score_mode), int(self.top_k), int(self.text_keys))
+                              self.flags, int(self.score_mode), int(self.top_k), int(self.text_keys),
+                              int(self.per_query))
 
     @property
     def torch_dtype(self):
@@ -142,6 +144,30 @@ class AdaCluster:
         check("ac_key_bounds", self.lib.ac_key_bounds(self._ctx, ptr(k), ptr(k_assign), ptr(nk), ptr(kmax),
                                                       ptr(kmin), ws, nb, stream_ptr(stream)))
         return kmax, kmin
+
+    def ac_select_rows(self, q, k_count, k_cent=None, nk=None, dense_flag=None, k_max=None, k_min=None,
+                       stream=None):
+        """Per-query selection: each query row's top_k key clusters as a bit
+        set [H, N, W] (int32 words, W = ceil(kk_cap / 32))."""
+        H, N = self.cfg.heads, self.cfg.n
+        bits = torch.zeros(H, N, (self.kk_cap + 31) // 32, dtype=torch.int32, device=self.device)
+        ws, nb = self._args_ws()
+        check("ac_select_rows", self.lib.ac_select_rows(
+            self._ctx, ptr(q), ptr(k_cent), ptr(k_count), ptr(k_max), ptr(k_min), ptr(nk), ptr(dense_flag),
+            ptr(bits), ws, nb, stream_ptr(stream)))
+        return bits
+
+    def ac_sparse_attn_rows(self, q, k, v, q_assign, k_assign, row_bits, nq=None, nk=None, dense_flag=None,
+                            lse=False, out=None, stream=None):
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        if out is None:
+            out = torch.empty(H, N, D, dtype=self.cfg.torch_dtype, device=self.device)
+        lse_t = self._f32(H, N) if lse else None
+        ws, nb = self._args_ws()
+        check("ac_sparse_attn_rows", self.lib.ac_sparse_attn_rows(
+            self._ctx, ptr(q), ptr(k), ptr(v), ptr(q_assign), ptr(k_assign), ptr(row_bits), ptr(nq), ptr(nk),
+            ptr(dense_flag), ptr(out), ptr(lse_t), ws, nb, stream_ptr(stream)))
+        return (out, lse_t) if lse else out
 
     def ac_cluster_sort(self, assign, cap, ncl=None, stream=None):
         H, N = self.cfg.heads, self.cfg.n

@@ -72,6 +72,12 @@ struct Ws {
     // Algorithm 1's single-cluster stages on chip: working vectors [H, wrows, d] (double)
     size_t wc;
     int wrows;
+    // Algorithm 1's final reassignment over the distinct centres: [H, cap, d], ids [H, cap], descriptors
+    size_t cu, cmap, segu;
+    // per-query selection: row bit sets [H, N, W], score batch [H, pq_batch, kk_cap] (double),
+    // row masks [H, max_chunks, N] (uint16), per-head pairs [H]
+    size_t rbits, pqs, rowmask, hpairs;
+    int W, pq_batch;
     int kpad;
     size_t total;
 };
@@ -146,6 +152,17 @@ Ws layout(const ac_ctx *c) {
     if (g.adaptive_q) w.wrows = (int)(N / g.kq + 1);
     if (g.adaptive_k) w.wrows = std::max(w.wrows, (int)(N / g.kk + 1));
     w.wc = b.take(H * (size_t)w.wrows * D * 8);
+    const bool adaptive = g.adaptive_q || g.adaptive_k;
+    w.cu = b.take(adaptive ? H * capm * D * 4 : 0);
+    w.cmap = b.take(adaptive ? H * capm * 4 : 0);
+    w.segu = b.take(adaptive ? H * sizeof(HeadSeg) : 0);
+    const bool pq = g.per_query != 0;
+    w.W = (c->kk_cap + 31) / 32;
+    w.pq_batch = pq ? (int)pq_score_batch_rows((int)H, (int)N, c->kk_cap) : 0;
+    w.rbits = b.take(pq ? HN * w.W * 4 : 0);
+    w.pqs = b.take(pq ? H * (size_t)w.pq_batch * c->kk_cap * 8 : 0);
+    w.rowmask = b.take(pq ? H * (size_t)attn_max_chunks(c->cfg.n, c->kk_cap, ATTN3_CHUNK) * N * 2 : 0);
+    w.hpairs = b.take(pq ? H * 8 : 0);
     w.total = b.off;
     return w;
 }
@@ -290,6 +307,8 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         AC_CUDA(cudaMemcpyAsync(c->h_info, c->d_info, 8 * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
         AC_CUDA(cudaStreamSynchronize(st));
         if (c->h_info[4]) return AC_ERR_CAPACITY;
+        // heads whose last stage removed nothing skip their repeats: copy the centres
+        if (c->h_info[7] > 0) k_ms_repeat(H, D, ms, cent, cap, st);
         if (c->h_info[0] == 0) break;
         const int mnu = c->h_info[1], mmt = c->h_info[2];
         // From the first stage after tau is fixed on, once every active head
@@ -346,17 +365,31 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
         AC_CUDA(cudaStreamSynchronize(st));
         *max_stages = c->h_info[6];
     }
-    AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
+    // Final reassignment of every token to the closest centre of C (ties to the
+    // lowest id).  Stages that repeat leave identical centres in C; the pass runs
+    // over the distinct ones (the first of identical centres, in id order) and
+    // maps the ids back, which is the same assignment at a fraction of the work.
+    {
+        float *cu = at<float>(ws, w.cu);
+        int32_t *cmap = at<int32_t>(ws, w.cmap);
+        HeadSeg *segu = at<HeadSeg>(ws, w.segu);
+        k_dedup_cent(H, D, seg, cent, cap, cu, cmap, segu, st);
+        AC_TRY(assign_step(c, w, ws, x, x, nullptr, segu, N, cu, cap, mode, assign, st));
+        k_map_ids(H, N, seg, cmap, cap, assign, st);
+    }
     k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, count, off, perm, status, st);
     if (mean_norm) k_mean_norm(H, N, seg, perm, off, cap, norm, mean_norm, st);
     if (text > 0) k_text_group(H, N, Nc, seg, assign, count, cap, ncl, st);
     return launch_check();
 }
 
+// row_bits (device, [H, N, W], nullable): per-query selection.  Each query row
+// attends only to the key clusters of its own bit set; the work list takes the
+// union of the sets of each query cluster (sel / selc are then ignored).
 ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v, const int32_t *qa,
                          const int32_t *ka, const int32_t *sel, const int32_t *selc, const int32_t *nq,
                          const int32_t *nk, const uint8_t *dense, void *out, float *lse, void *ws, cudaStream_t st,
-                         int64_t *pairs_dev, cudaEvent_t *ev_kernel = nullptr) {
+                         int64_t *pairs_dev, cudaEvent_t *ev_kernel = nullptr, const uint32_t *row_bits = nullptr) {
     const ac_config &g = c->cfg;
     const int H = g.heads, N = g.n, D = g.d;
     Ws w = layout(c);
@@ -376,19 +409,34 @@ ac_status do_sparse_attn(ac_ctx *c, const void *q, const void *k, const void *v,
     k_gather_rows(k, kg, kperm, H, N, rb, st);
     k_gather_rows(v, vg, kperm, H, N, rb, st);
     const bool two_tiles = (g.dtype == AC_BF16);  // bf16: two query tiles per CTA (items of 256 rows)
+    if (row_bits) {
+        // the union of each query cluster's row sets is the cluster's key stream
+        sel = at<int32_t>(ws, w.sel);
+        selc = at<int32_t>(ws, w.selc);
+        k_select_union(H, N, row_bits, w.W, qperm, qoff, c->kq_cap, nq, g.kq, dense, c->kk_cap,
+                       const_cast<int32_t *>(sel), const_cast<int32_t *>(selc), st);
+    }
     k_build_items(H, N, two_tiles ? 256 : 128, c->kq_cap, c->kk_cap, qoff, nq, dense, g.kq, koff, sel, selc, items,
                   nitems, pairs_dev, at<int32_t>(ws, w.items_scr), c->d_status, st);
     int2 *runs = at<int2>(ws, w.runs), *run_info = at<int2>(ws, w.run_info);
-    k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN3_CHUNK, runs, run_info, st);
+    if (row_bits) k_key_runs_single(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN3_CHUNK, runs, run_info, st);
+    else k_key_runs(H, c->kq_cap, c->kk_cap, koff, sel, selc, ATTN3_CHUNK, runs, run_info, st);
     const int max_chunks = attn_max_chunks(N, c->kk_cap, ATTN3_CHUNK);
     uint32_t *masks = at<uint32_t>(ws, w.masks);
     if (two_tiles) k_chunk_masks(H, c->kq_cap, c->kk_cap, max_chunks, runs, run_info, masks, st);
+    uint16_t *rowmask = nullptr;
+    if (row_bits) {
+        rowmask = at<uint16_t>(ws, w.rowmask);
+        if (k_rowmask(H, N, c->kq_cap, c->kk_cap, max_chunks, koff, runs, run_info, qperm, qoff, row_bits, w.W,
+                      rowmask, st) != 0)
+            return AC_ERR_UNSUPPORTED;
+    }
     if (ev_kernel) cudaEventRecord(ev_kernel[0], st);
     int rc;
     if (two_tiles)
         rc = k_attention3(D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, masks, max_chunks, items,
                           nitems, attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn,
-                          st);
+                          st, rowmask);
     else
         rc = k_attention(DT_F32, D, H, N, qg, kg, vg, qperm, c->kk_cap, c->kq_cap, runs, run_info, items, nitems,
                          attn_max_items(H, N, c->kq_cap), out, lse, c->d_status, c->num_sms, c->encode_fn, st);
@@ -409,6 +457,9 @@ ac_status validate(const ac_config *g) {
     if (g->text_keys < 0 || g->text_keys >= g->n || (g->text_keys > 0 && g->kk > g->n - g->text_keys))
         return AC_ERR_INVALID_ARG;
     if ((long long)g->heads * g->n > 0x7fffffffLL / 2) return AC_ERR_UNSUPPORTED;
+    if (g->per_query != 0 && g->per_query != 1) return AC_ERR_INVALID_ARG;
+    // per-query selection: argtopk (Algorithm 3's form) on the bf16 path
+    if (g->per_query && (g->top_k <= 0 || g->dtype != AC_BF16)) return AC_ERR_UNSUPPORTED;
     if (g->adaptive_q && g->nmax_q < 1) return AC_ERR_INVALID_ARG;
     if (g->adaptive_k && g->nmax_k < 1) return AC_ERR_INVALID_ARG;
     if ((g->adaptive_q || g->adaptive_k) &&
@@ -656,12 +707,21 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
         key_bounds(c, k, ka, nk, kbmax, kbmin, ws, st);
     }
     const int tg = g.text_keys > 0 ? 1 : 0;
-    k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk + tg, dense,
-             (int)g.score_mode, g.top_k, g.top_p, sel, selc, c->d_status, st, tg, at<float>(ws, w.kct));
+    uint32_t *rbits = nullptr;
+    if (g.per_query) {
+        // Algorithm 3's argtopk along each row of S: every query row's own set
+        rbits = at<uint32_t>(ws, w.rbits);
+        k_select_rows(q, DT_BF16, g.heads, g.n, g.d, kc, kbmax, kbmin, kn, c->kk_cap, nk, g.kk + tg, tg, dense,
+                      (int)g.score_mode, g.top_k, rbits, w.W, at<double>(ws, w.pqs), w.pq_batch,
+                      at<unsigned long long>(ws, w.hpairs), st);
+    } else {
+        k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk + tg, dense,
+                 (int)g.score_mode, g.top_k, g.top_p, sel, selc, c->d_status, st, tg, at<float>(ws, w.kct));
+    }
     if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
     s = do_sparse_attn(c, q, k, v, qa, ka, sel, selc, nq, nk, dense, out, nullptr, ws, st, at<int64_t>(ws, w.pairs),
-                       pe ? pe + 4 : nullptr);
+                       pe ? pe + 4 : nullptr, rbits);
     if (s != AC_OK) return s;
     if (stats) {
         AC_CUDA(cudaEventRecord(c->ev[4], st));
@@ -680,12 +740,24 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
         int64_t pairs = 0;
         AC_CUDA(cudaMemcpy(&pairs, at<int64_t>(ws, w.pairs), sizeof(pairs), cudaMemcpyDeviceToHost));
         stats->pairs = pairs;
+        stats->pairs_computed = pairs;
         uint8_t *hd = (uint8_t *)malloc(g.heads);
-        if (hd) {
+        unsigned long long *hp = (unsigned long long *)malloc(sizeof(unsigned long long) * g.heads);
+        if (hd && hp) {
             AC_CUDA(cudaMemcpy(hd, dense, g.heads, cudaMemcpyDeviceToHost));
             for (int h = 0; h < g.heads; h++) stats->dense_heads += hd[h] ? 1 : 0;
-            free(hd);
+            if (g.per_query) {
+                // the pairs the method attends: each row's own set (dense heads: N^2)
+                AC_CUDA(cudaMemcpy(hp, at<unsigned long long>(ws, w.hpairs), sizeof(unsigned long long) * g.heads,
+                                   cudaMemcpyDeviceToHost));
+                int64_t own = 0;
+                for (int h = 0; h < g.heads; h++)
+                    own += hd[h] ? (int64_t)g.n * (int64_t)g.n : (int64_t)hp[h];
+                stats->pairs = own;
+            }
         }
+        free(hd);
+        free(hp);
         stats->max_stages_q = sq;
         stats->max_stages_k = sk;
         stats->kmeans_rounds_q = max_rounds(kst, g.heads);
@@ -742,6 +814,37 @@ ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, co
     return launch_check();
 }
 
+
+ac_status ac_select_rows(ac_ctx *c, const void *q, const float *k_cent, const int32_t *k_count, const float *k_max,
+                         const float *k_min, const int32_t *nk, const uint8_t *dense_flag, uint32_t *row_bits,
+                         void *ws, size_t ws_bytes, void *stream) {
+    if (!c || !q || !k_count || !row_bits) return AC_ERR_INVALID_ARG;
+    const ac_config &g = c->cfg;
+    if (!g.per_query) return AC_ERR_UNSUPPORTED;
+    if (g.score_mode == AC_SCORE_QUEST ? (!k_max || !k_min) : !k_cent) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    Ws w = layout(c);
+    const int tg = g.text_keys > 0 ? 1 : 0;
+    k_select_rows(q, DT_BF16, g.heads, g.n, g.d, k_cent, k_max, k_min, k_count, c->kk_cap, nk, g.kk + tg, tg,
+                  dense_flag, (int)g.score_mode, g.top_k, row_bits, w.W, at<double>(ws, w.pqs), w.pq_batch,
+                  at<unsigned long long>(ws, w.hpairs), (cudaStream_t)stream);
+    return launch_check();
+}
+
+ac_status ac_sparse_attn_rows(ac_ctx *c, const void *q, const void *k, const void *v, const int32_t *q_assign,
+                              const int32_t *k_assign, const uint32_t *row_bits, const int32_t *nq, const int32_t *nk,
+                              const uint8_t *dense_flag, void *out, float *lse, void *ws, size_t ws_bytes,
+                              void *stream) {
+    if (!c || !q || !k || !v || !q_assign || !k_assign || !row_bits || !out) return AC_ERR_INVALID_ARG;
+    if (!c->cfg.per_query) return AC_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return AC_ERR_INVALID_ARG;
+    ac_status s = check_ws(c, ws, ws_bytes);
+    if (s != AC_OK) return s;
+    Ws w = layout(c);
+    return do_sparse_attn(c, q, k, v, q_assign, k_assign, nullptr, nullptr, nq, nk, dense_flag, out, lse, ws,
+                          (cudaStream_t)stream, at<int64_t>(ws, w.pairs), nullptr, row_bits);
+}
 
 ac_status ac_key_bounds(ac_ctx *c, const void *k, const int32_t *k_assign, const int32_t *nk, float *k_max,
                         float *k_min, void *ws, size_t ws_bytes, void *stream) {

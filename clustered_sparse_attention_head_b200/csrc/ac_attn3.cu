@@ -84,6 +84,9 @@ struct A3Params {
     const AttnItem *items;
     const int32_t *n_items;
     int *work;             // items handed out so far (zeroed by the work-list builder)
+    // per-query selection: [H, max_chunks, N] by the row's position in cluster
+    // order, bit g = the row keeps 8-key group g of the chunk (NULL: all rows keep all)
+    const uint16_t *rowmask;
     __nv_bfloat16 *out;
     float *lse;
     int *status;
@@ -320,6 +323,21 @@ template <int B> __device__ __forceinline__ void mask_word(uint32_t (&s)[128], u
         }
     }
 }
+// 8 bits (one per 8-key group) to 8 nibbles: 0xF where the bit is set, 0 elsewhere
+__device__ __forceinline__ uint32_t nibbles8(uint32_t b) {
+    uint32_t x = b & 0xFFu;
+    x = (x | (x << 12)) & 0x000F000Fu;
+    x = (x | (x << 6)) & 0x03030303u;
+    x = (x | (x << 3)) & 0x11111111u;
+    return x * 0xFu;
+}
+__device__ __forceinline__ uint32_t load_rowmask(const A3Params &p, int h, int chunk, int pos) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];"
+                 : "=h"(v)
+                 : "l"(p.rowmask + ((size_t)h * p.max_chunks + chunk) * p.N + pos));
+    return v;
+}
 // Scores of 8-row groups past their valid count set to -inf (masks: 4 bits a group)
 __device__ __forceinline__ void apply_mask(uint32_t (&s)[128], uint2 gm) {
     if (gm.x != kFullMask) mask_word<0>(s, gm.x);
@@ -350,7 +368,9 @@ __device__ __forceinline__ void exp_pairs(const uint32_t (&s)[128], uint32_t (&p
 
 }  // namespace
 
-template <int D>
+// ROWS: per-query selection (p.rowmask), a separate instance so that the
+// default kernel carries none of its registers.
+template <int D, bool ROWS>
 __global__ void __launch_bounds__(384, 1)
     attn3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KVMaps3 mk,
                  const __grid_constant__ KVMaps3 mv, const A3Params p) {
@@ -702,11 +722,23 @@ __global__ void __launch_bounds__(384, 1)
             // chunk's time to arrive before its value is needed
             uint2 gm_next = item_mask3(p, mrow, cbase);
             uint2 gm_next2 = nch > 1 ? item_mask3(p, mrow, cbase + cstep) : make_uint2(0u, 0u);
+            // per-query selection: the row's own groups of each chunk, also two ahead
+            const bool own = ROWS && it.a >= 0 && valid;
+            const int rpos = it.q_start + r;
+            uint32_t rm_next = own ? load_rowmask(p, it.h, cbase, rpos) : 0xFFFFu;
+            uint32_t rm_next2 = own && nch > 1 ? load_rowmask(p, it.h, cbase + cstep, rpos) : 0xFFFFu;
             float m_ref = -INFINITY, l0 = 0.f, l1 = 0.f;
             for (int j = 0; j < nch; j++) {
-                const uint2 gm = gm_next;
+                uint2 gm = gm_next;
                 gm_next = gm_next2;
                 if (j + 2 < nch) gm_next2 = item_mask3(p, mrow, cbase + cstep * (j + 2));
+                if (ROWS) {
+                    const uint32_t rm = rm_next;
+                    rm_next = rm_next2;
+                    if (own && j + 2 < nch) rm_next2 = load_rowmask(p, it.h, cbase + cstep * (j + 2), rpos);
+                    gm.x &= nibbles8(rm);
+                    gm.y &= nibbles8(rm >> 8);
+                }
                 const uint32_t c = cnt + j;
                 if (!mbar_wait_warp(s_full + t, c & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
@@ -736,10 +768,14 @@ __global__ void __launch_bounds__(384, 1)
                 float f = 1.f;
                 if (rescale) {
                     const float m_to = fmaxf(m_ref, m_new);
-                    f = ex2_approx(m_ref - m_to);
+                    // a row with no unmasked key yet keeps f = 1 (its O and l are 0)
+                    f = m_to == -INFINITY ? 1.f : ex2_approx(m_ref - m_to);
                     m_ref = m_to;
                 }
-                const uint64_t scale2 = pack2(sc, sc), neg2 = pack2(-m_ref, -m_ref);
+                // a row whose keys so far are all masked (per-query selection) has
+                // m_ref = -inf: its scores are all -inf and must give P = 0
+                const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
+                const uint64_t scale2 = pack2(sc, sc), neg2 = pack2(negm, negm);
                 // row sum in four partial sums (two packed pairs), folded into l0/l1
                 uint64_t la[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
                 uint32_t pk[32];
@@ -880,7 +916,7 @@ static int kv_maps3(EncodeTiledFn3 enc, KVMaps3 *m, const void *base, int rows, 
                : 0;
 }
 
-template <int D>
+template <int D, bool ROWS>
 static int launch3(const void *qg, const void *kg, const void *vg, const A3Params &p, int max_items, int num_sms,
                    void *encode_fn, cudaStream_t st) {
     using C = A3Cfg<D>;
@@ -894,12 +930,12 @@ static int launch3(const void *qg, const void *kg, const void *vg, const A3Param
     // larger split would make setmaxnreg.inc wait forever, so refuse.  The
     // shared-memory attribute belongs to the current device: set on every call.
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn3_kernel<D>) != cudaSuccess || fa.numRegs != C::REGS_LAUNCH) return -1;
-    if (cudaFuncSetAttribute(attn3_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, attn3_kernel<D, ROWS>) != cudaSuccess || fa.numRegs != C::REGS_LAUNCH) return -1;
+    if (cudaFuncSetAttribute(attn3_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return -1;
     int grid = max_items < num_sms ? max_items : num_sms;
     if (grid < 1) grid = 1;
-    attn3_kernel<D><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);
+    attn3_kernel<D, ROWS><<<grid, C::NTHREADS, C::SMEM, st>>>(mq, mk, mv, p);
     note_launch();
     return 0;
 }
@@ -907,7 +943,7 @@ static int launch3(const void *qg, const void *kg, const void *vg, const A3Param
 int k_attention3(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
                  int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const uint32_t *masks,
                  int max_chunks, const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse,
-                 int *status, int num_sms, void *encode_fn, cudaStream_t st) {
+                 int *status, int num_sms, void *encode_fn, cudaStream_t st, const uint16_t *rowmask) {
     A3Params p;
     p.H = H;
     p.N = N;
@@ -924,9 +960,14 @@ int k_attention3(int D, int H, int N, const void *qg, const void *kg, const void
     p.out = reinterpret_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
     p.status = status;
+    p.rowmask = rowmask;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    if (D == 64) return launch3<64>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
-    return launch3<128>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+    if (rowmask) {
+        if (D == 64) return launch3<64, true>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+        return launch3<128, true>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+    }
+    if (D == 64) return launch3<64, false>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
+    return launch3<128, false>(qg, kg, vg, p, max_items, num_sms, encode_fn, st);
 }
 
 }  // namespace ac

@@ -103,11 +103,33 @@ constexpr int ATTN3_CHUNK = 128;
 int k_attention3(int D, int H, int N, const void *qg, const void *kg, const void *vg, const int32_t *qperm,
                  int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info, const uint32_t *masks,
                  int max_chunks, const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse,
-                 int *status, int num_sms, void *encode_fn, cudaStream_t st);
+                 int *status, int num_sms, void *encode_fn, cudaStream_t st, const uint16_t *rowmask = nullptr);
 int k_attention(int dtype, int D, int H, int N, const void *qg, const void *kg, const void *vg,
                 const int32_t *qperm, int kk_cap, int kq_cap, const int2 *runs, const int2 *run_info,
                 const AttnItem *items, const int32_t *n_items, int max_items, void *out, float *lse, int *status,
                 int num_sms, void *encode_fn, cudaStream_t st);
+
+// ---- ac_perquery.cu: per-query selection (argtopk along each row of S)
+// Rows of scores per batch (all heads) that fit the scratch of about 1 GiB.
+size_t pq_score_batch_rows(int H, int N, int kk_cap);
+// bits [H, N, W]: each query row's top_k key clusters (W = ceil(kk_cap / 32));
+// head_pairs [H]: sum over rows of the selected clusters' sizes.
+int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_cent, const float *k_max,
+                  const float *k_min, const int32_t *k_count, int kk_cap, const int32_t *nk, int kk_fixed,
+                  int text_group, const uint8_t *dense, int score_mode, int top_k, uint32_t *bits, int W,
+                  double *scores, int batch, unsigned long long *head_pairs, cudaStream_t st);
+// Per query cluster: the union of its rows' sets as ascending sel_idx / sel_cnt.
+void k_select_union(int H, int N, const uint32_t *bits, int W, const int32_t *qperm, const int32_t *qoff, int kq_cap,
+                    const int32_t *nq, int kq_fixed, const uint8_t *dense, int kk_cap, int32_t *sel_idx,
+                    int32_t *sel_cnt, cudaStream_t st);
+// One key run per selected non-empty cluster (not merged).
+void k_key_runs_single(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx,
+                       const int32_t *sel_cnt, int chunk_rows, int2 *runs, int2 *info, cudaStream_t st);
+// rowmask [H, max_chunks, N]: per row (cluster order) and chunk, the 8-key groups the row keeps.
+// Returns -1 (nothing launched) when its group table would not fit in shared memory.
+int k_rowmask(int H, int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *koff, const int2 *runs,
+              const int2 *info, const int32_t *qperm, const int32_t *qoff, const uint32_t *bits, int W,
+              uint16_t *rowmask, cudaStream_t st);
 
 // The key rows of one work item as a stream of pieces: the rows of each run in
 // turn (all rows [0, dense_rows) of a dense head).  piece(room) hands out the

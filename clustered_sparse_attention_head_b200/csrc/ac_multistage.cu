@@ -32,17 +32,28 @@ __global__ void ms_init_kernel(int H, int N, int nrows, MsHead *__restrict__ st,
         s.flag = 0;
         s.mt = 0;
         s.done = 0;
+        s.same = 0;
+        s.rep_src = 0;
+        s.rep_n = 0;
+        s.pad = 0;
         s.tau = 0.0;
         st[h] = s;
     }
 }
 
 // Decide the next stage of every head; writes the pass descriptors and a
-// summary {active heads, max |U|, max m_t, max |C|, capacity error} for the host.
+// summary {active heads, max |U|, max m_t, max |C|, capacity error, -, -,
+// heads that repeat} for the host.
+//
+// A stage that removed no token is a fixed point: the next stage has the same
+// U (same order), hence the same m_t and the same starting rows, runs the same
+// k-means and removes nothing again, so every stage until |C| >= N_max
+// repeats it and F is set.  The head then skips them: its centres are copied
+// forward (k_ms_repeat), which gives what running them gives, bit for bit.
 __global__ void ms_control_kernel(int H, int N, int m0, int nmax, int cap, MsHead *__restrict__ st,
                                   HeadSeg *__restrict__ seg, int32_t *__restrict__ info, int *status) {
-    __shared__ int act, mnu, mmt, mnc, err;
-    if (threadIdx.x == 0) { act = 0; mnu = 0; mmt = 0; mnc = 0; err = 0; }
+    __shared__ int act, mnu, mmt, mnc, err, nrep;
+    if (threadIdx.x == 0) { act = 0; mnu = 0; mmt = 0; mnc = 0; err = 0; nrep = 0; }
     __syncthreads();
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
         MsHead s = st[h];
@@ -57,6 +68,22 @@ __global__ void ms_control_kernel(int H, int N, int m0, int nmax, int cap, MsHea
             } else if (s.nc >= nmax) {
                 s.flag = 1;
                 s.done = 1;
+            } else if (s.same && s.stage >= 1) {
+                const int m = s.mt;  // the repeated stage's m_t (|U| is unchanged)
+                const int r = (nmax - s.nc + m - 1) / m;
+                if (s.nc + r * m > cap) {
+                    atomicExch(&err, 1);
+                    set_status(status, ST_CAPACITY);
+                    s.done = 1;
+                } else {
+                    s.rep_src = s.nc - m;
+                    s.rep_n = r;
+                    s.nc += r * m;
+                    s.stage += r;
+                    s.flag = 1;
+                    s.done = 1;
+                    atomicAdd(&nrep, 1);
+                }
             } else {
                 int mt;
                 if (s.stage == 0) mt = m0;
@@ -91,7 +118,22 @@ __global__ void ms_control_kernel(int H, int N, int m0, int nmax, int cap, MsHea
         info[2] = mmt;
         info[3] = mnc;
         info[4] = err;
+        info[7] = nrep;
     }
+}
+
+__global__ void ms_repeat_kernel(int D, MsHead *__restrict__ st, float *__restrict__ cent, int cap) {
+    const int h = blockIdx.x;
+    const MsHead s = st[h];
+    if (s.rep_n <= 0) return;
+    const int m = s.mt;
+    const float *src = cent + ((size_t)h * cap + s.rep_src) * D;
+    for (int e = threadIdx.x; e < s.rep_n * m * D; e += blockDim.x) {
+        const int i = e / (m * D), r = e - i * (m * D);
+        cent[((size_t)h * cap + s.rep_src + (size_t)(i + 1) * m) * D + r] = src[r];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) st[h].rep_n = 0;
 }
 
 // tau of the first stage (one CTA per head; positions = tokens at stage 0).
@@ -185,6 +227,7 @@ __global__ void ms_remove_kernel(int N, const HeadSeg *__restrict__ seg, const d
     }
     if (tid == 0) {
         MsHead s = st[h];
+        s.same = base == g.nrows ? 1 : 0;
         s.nu = base;
         s.nc += s.mt;
         s.stage += 1;
@@ -382,9 +425,19 @@ __global__ void __launch_bounds__(256) ms_single_kernel(const T *__restrict__ x,
             }
             __syncthreads();
         }
+        const bool same = base == s.nu;
         s.nu = base;
         s.nc += 1;
         s.stage += 1;
+        if (same && s.nc < nmax) {
+            // no row left U: every later stage repeats this one (same U, same
+            // centre) until |C| >= N_max; their centres are this one's
+            const int r = nmax - s.nc;
+            for (int e = tid; e < r * D; e += blockDim.x)
+                cent[((size_t)h * cap + s.nc) * D + e] = cs[e % D];
+            s.nc += r;
+            s.stage += r;
+        }
         int32_t *tmp = P;
         P = Pn;
         Pn = tmp;
@@ -409,6 +462,91 @@ int k_ms_single(const void *x, int dtype, int H, int N, int D, int nrows, int m0
 #undef AC_MS_SINGLE
     note_launch();
     return 0;
+}
+
+void k_ms_repeat(int H, int D, MsHead *st, float *cent, int cap, cudaStream_t s) {
+    ms_repeat_kernel<<<H, 256, 0, s>>>(D, st, cent, cap);
+    note_launch();
+}
+
+// One CTA per head.  A centre is a duplicate when an earlier one has the same
+// bits in every element; a 32-bit hash of each centre (in shared memory)
+// screens the pairs, and equal hashes are compared element by element.
+__global__ void dedup_cent_kernel(int D, const HeadSeg *__restrict__ seg, const float *__restrict__ cent, int cap,
+                                  float *__restrict__ cu, int32_t *__restrict__ cmap, HeadSeg *__restrict__ segu) {
+    extern __shared__ uint32_t hsh[];  // [cap] hashes, then [cap] first-copy flags
+    uint32_t *first = hsh + cap;
+    __shared__ int wsum[32];
+    const int h = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const HeadSeg g = seg[h];
+    const int k = g.k;
+    const uint32_t *c = reinterpret_cast<const uint32_t *>(cent + (size_t)h * cap * D);
+    for (int j = tid; j < k; j += nt) {
+        uint32_t x = 2166136261u;
+        for (int t = 0; t < D; t++) x = (x ^ c[(size_t)j * D + t]) * 16777619u;
+        hsh[j] = x;
+    }
+    __syncthreads();
+    for (int j = tid; j < k; j += nt) {
+        uint32_t f = 1u;
+        for (int i = 0; i < j && f; i++) {
+            if (hsh[i] != hsh[j]) continue;
+            bool eq = true;
+            for (int t = 0; t < D && eq; t++) eq = c[(size_t)i * D + t] == c[(size_t)j * D + t];
+            if (eq) f = 0u;
+        }
+        first[j] = f;
+    }
+    __syncthreads();
+    // ordered compaction of the first copies (block-wide exclusive scan)
+    int base = 0;
+    for (int j0 = 0; j0 < k; j0 += nt) {
+        const int j = j0 + tid;
+        const int f = j < k ? (int)first[j] : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        const int lane = tid & 31, w = tid >> 5;
+        if (lane == 0) wsum[w] = __popc(bal);
+        __syncthreads();
+        int before = base;
+        for (int u = 0; u < w; u++) before += wsum[u];
+        if (f) {
+            const int u = before + __popc(bal & ((1u << lane) - 1u));
+            cmap[(size_t)h * cap + u] = j;
+            for (int t = 0; t < D; t++)
+                cu[((size_t)h * cap + u) * D + t] = cent[((size_t)h * cap + j) * D + t];
+        }
+        __syncthreads();
+        for (int u = 0; u < nt / 32; u++) base += wsum[u];
+        __syncthreads();
+    }
+    if (tid == 0) {
+        HeadSeg o = g;
+        o.k = base;
+        o.cent_off = 0;
+        segu[h] = o;
+    }
+}
+
+__global__ void map_ids_kernel(int N, const HeadSeg *__restrict__ seg, const int32_t *__restrict__ cmap, int cap,
+                               int32_t *__restrict__ assign) {
+    const int h = blockIdx.y;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= seg[h].nrows) return;
+    const int a = assign[(size_t)h * N + i];
+    if (a >= 0 && a < cap) assign[(size_t)h * N + i] = cmap[(size_t)h * cap + a];
+}
+
+void k_dedup_cent(int H, int D, const HeadSeg *seg, const float *cent, int cap, float *cu, int32_t *cmap,
+                  HeadSeg *segu, cudaStream_t s) {
+    const size_t smem = (size_t)2 * cap * sizeof(uint32_t);
+    if (smem > 48 * 1024) cudaFuncSetAttribute(dedup_cent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dedup_cent_kernel<<<H, 256, smem, s>>>(D, seg, cent, cap, cu, cmap, segu);
+    note_launch();
+}
+
+void k_map_ids(int H, int N, const HeadSeg *seg, const int32_t *cmap, int cap, int32_t *assign, cudaStream_t s) {
+    map_ids_kernel<<<dim3((N + 255) / 256, H), 256, 0, s>>>(N, seg, cmap, cap, assign);
+    note_launch();
 }
 
 void k_ms_init(int H, int N, int nrows, MsHead *st, int32_t *U, int32_t *U2, cudaStream_t s) {

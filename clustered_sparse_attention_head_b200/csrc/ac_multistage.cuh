@@ -11,6 +11,9 @@ struct MsHead {
     int flag;    // F
     int mt;      // m_t of the stage in progress
     int done;
+    int same;    // the last stage removed no token (every later stage repeats it)
+    int rep_src, rep_n;  // repeat to copy: centres [rep_src, rep_src + mt) rep_n more times
+    int pad;
     double tau;
 };
 
@@ -22,6 +25,16 @@ void k_ms_tau(int H, int N, int rule, double x, const HeadSeg *seg, const double
               const int32_t *off, int cap, int kmax, MsHead *st, cudaStream_t s);
 void k_ms_remove(int H, int N, const HeadSeg *seg, const double *dist, const int32_t *U, int32_t *Unext, MsHead *st,
                  cudaStream_t s);
+// Copies the centres of a repeated stage (MsHead.rep_*) and clears the request.
+void k_ms_repeat(int H, int D, MsHead *st, float *cent, int cap, cudaStream_t s);
+// The distinct centres of each head's final set, in id order: cu [H, cap, D]
+// (ku of them), cmap [H, cap] their ids, segu the pass descriptors over cu.
+// Ties in the final reassignment go to the lowest id, which is always the first
+// of identical centres, so assigning over cu and mapping back through cmap gives
+// the assignment over the whole set.
+void k_dedup_cent(int H, int D, const HeadSeg *seg, const float *cent, int cap, float *cu, int32_t *cmap,
+                  HeadSeg *segu, cudaStream_t s);
+void k_map_ids(int H, int N, const HeadSeg *seg, const int32_t *cmap, int cap, int32_t *assign, cudaStream_t s);
 // Every remaining single-cluster stage of each head on chip (one CTA per
 // head); wc: [H, wrows, D] doubles of scratch, wrows >= the largest |U| with
 // m_t = 1 (N / m0).  A head whose |U| exceeds wrows is left to the host loop.

@@ -1,0 +1,413 @@
+// Per-query selection (AdaCluster §3.3, Algorithm 3: the score matrix S has one
+// row per query token, Index <- argtopk(S, topk) along each row), and the
+// tables that let the block-sparse attention kernel honour each row's own set.
+//
+//  1. pq_scores_kernel: s_ib for every query row i and key cluster b, in double
+//     with the oracle's summation order (one thread per score, elements in
+//     order): CENTROID s = (q_i . c_b) / sqrt(d); QUEST s = sum_t
+//     max(q_t M_bt, q_t m_bt) / sqrt(d) (the query is its own representative).
+//  2. pq_topk_kernel: one warp per row keeps the top_k non-empty clusters of
+//     largest s (ties to the lower id) as a bit set [H, N, W] (W = kk_cap / 32
+//     words); the text-key group, if any, is always set.  It also sums the
+//     row's pairs (sum of the selected clusters' sizes).
+//  3. pq_union_kernel: per query cluster, the union of its rows' sets, as the
+//     ascending sel_idx / sel_cnt lists the work list and key runs take.
+//  4. key_runs_single_kernel: one key run per selected non-empty cluster (not
+//     merged), so every 8-key group of a chunk belongs to one cluster.
+//  5. pq_rowmask_kernel: per row and chunk a 16-bit mask, bit g = the row's
+//     set holds the cluster of 8-key group g ([H, max_chunks, N] by the
+//     row's position in cluster order); the attention kernel masks the groups
+//     whose bit is clear.
+#include "ac_kernels.cuh"
+
+namespace ac {
+
+constexpr int PQ_ROWS = 32, PQ_COLS = 32;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) pq_scores_kernel(const T *__restrict__ q, int N, int r0, int nb,
+                                                        const float *__restrict__ k_cent,
+                                                        const float *__restrict__ k_max,
+                                                        const float *__restrict__ k_min, int kk_cap,
+                                                        const int32_t *__restrict__ nk, int kk_fixed, int text_group,
+                                                        int score_mode, double *__restrict__ scores) {
+    constexpr int LD = D + 1;  // padded rows: the 32 rows of a tile sit in 32 banks
+    extern __shared__ float pqs[];
+    float *qs = pqs;                     // [PQ_ROWS][LD]
+    float *cs = qs + PQ_ROWS * LD;       // [PQ_COLS][LD] (centroid or M)
+    float *ms = cs + PQ_COLS * LD;       // [PQ_COLS][LD] (m, Quest only)
+    const int h = blockIdx.z, tid = threadIdx.x;
+    const int nkh = (nk ? min(max(nk[h], 0), kk_cap) : kk_fixed) - text_group;
+    const int b0 = blockIdx.y * PQ_COLS, i0 = blockIdx.x * PQ_ROWS;
+    if (b0 >= nkh) return;
+    for (int e = tid; e < PQ_ROWS * D; e += 128) {
+        const int r = e / D, t = e - r * D;
+        const int i = r0 + i0 + r;
+        qs[r * LD + t] = (i0 + r < nb && i < N) ? to_f(q[((size_t)h * N + i) * D + t]) : 0.f;
+    }
+    for (int e = tid; e < PQ_COLS * D; e += 128) {
+        const int c = e / D, t = e - c * D;
+        const int b = b0 + c;
+        const size_t o = ((size_t)h * kk_cap + b) * D + t;
+        if (score_mode == 1) {
+            cs[c * LD + t] = b < nkh ? k_max[o] : 0.f;
+            ms[c * LD + t] = b < nkh ? k_min[o] : 0.f;
+        } else {
+            cs[c * LD + t] = b < nkh ? k_cent[o] : 0.f;
+        }
+    }
+    __syncthreads();
+    const int tx = tid & 7, ty = tid >> 3;  // 4 clusters x 2 rows per thread
+    double acc[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) acc[i][j] = 0.0;
+    if (score_mode == 1) {
+        for (int t = 0; t < D; t++) {
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const double qb = (double)qs[(2 * ty + i) * LD + t];
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const double hi = dmul(qb, (double)cs[(4 * tx + j) * LD + t]);
+                    const double lo = dmul(qb, (double)ms[(4 * tx + j) * LD + t]);
+                    acc[i][j] = dadd(acc[i][j], hi > lo ? hi : lo);
+                }
+            }
+        }
+    } else {
+        for (int t = 0; t < D; t++) {
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const double qv = (double)qs[(2 * ty + i) * LD + t];
+#pragma unroll
+                for (int j = 0; j < 4; j++) acc[i][j] = dadd(acc[i][j], dmul(qv, (double)cs[(4 * tx + j) * LD + t]));
+            }
+        }
+    }
+    const double scale = 1.0 / sqrt((double)D);
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        const int r = i0 + 2 * ty + i;
+        if (r >= nb || r0 + r >= N) continue;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int b = b0 + 4 * tx + j;
+            if (b < nkh) scores[((size_t)h * nb + r) * kk_cap + b] = dmul(acc[i][j], scale);
+        }
+    }
+}
+
+// One warp per query row: top_k rounds of a warp-wide argmax over the row's
+// scores (staged in shared memory), ties to the lower id, empty clusters and
+// clusters already taken skipped.  Up to four warps (rows) per block, fewer
+// when kk_cap is large.
+constexpr int PQ_WARPS = 4;
+__global__ void __launch_bounds__(PQ_WARPS * 32) pq_topk_kernel(const double *__restrict__ scores, int N, int r0,
+                                                               int nb, const int32_t *__restrict__ k_count, int kk_cap,
+                                                               const int32_t *__restrict__ nk, int kk_fixed,
+                                                               int text_group, const uint8_t *__restrict__ dense,
+                                                               int top_k, int W, uint32_t *__restrict__ bits,
+                                                               unsigned long long *__restrict__ head_pairs) {
+    extern __shared__ unsigned char pqt[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    double *sc = reinterpret_cast<double *>(pqt) + (size_t)warp * kk_cap;               // [warps][kk_cap]
+    uint32_t *bw = reinterpret_cast<uint32_t *>(reinterpret_cast<double *>(pqt) + (size_t)nw * kk_cap) +
+                   (size_t)warp * W;                                                      // [warps][W]
+    const int h = blockIdx.y;
+    const int r = blockIdx.x * nw + warp;
+    if (r >= nb || r0 + r >= N) return;  // whole warp
+    const int nkh_all = nk ? min(max(nk[h], 0), kk_cap) : kk_fixed;
+    const int nkh = nkh_all - text_group;
+    const int32_t *kc = k_count + (size_t)h * kk_cap;
+    for (int w = lane; w < W; w += 32) bw[w] = 0u;
+    const bool dn = dense && dense[h];
+    unsigned long long pairs = 0ull;
+    if (!dn) {
+        const double *srow = scores + ((size_t)h * nb + r) * kk_cap;
+        for (int b = lane; b < nkh; b += 32) sc[b] = kc[b] > 0 ? srow[b] : -INFINITY;
+        __syncwarp();
+        // taken clusters get NaN, which no comparison below accepts
+        for (int round = 0; round < top_k; round++) {
+            double best = -INFINITY;
+            int bb = 0x7fffffff;
+            for (int b = lane; b < nkh; b += 32) {
+                const double v = sc[b];
+                if (kc[b] > 0 && (v > best || (v == best && b < bb))) {
+                    best = v;
+                    bb = b;
+                }
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+                const int oj = __shfl_xor_sync(0xffffffffu, bb, o);
+                if (ob > best || (ob == best && oj < bb)) {
+                    best = ob;
+                    bb = oj;
+                }
+            }
+            if (bb == 0x7fffffff) break;  // no non-empty cluster left
+            if (lane == 0) {
+                sc[bb] = __longlong_as_double(0x7ff8000000000000ll);
+                bw[bb >> 5] |= 1u << (bb & 31);
+                pairs += (unsigned long long)kc[bb];
+            }
+            __syncwarp();
+        }
+        if (text_group && lane == 0) {
+            const int tg = nkh;  // the text-key group's id
+            bw[tg >> 5] |= 1u << (tg & 31);
+            pairs += (unsigned long long)kc[tg];
+        }
+    }
+    __syncwarp();
+    uint32_t *out = bits + ((size_t)h * N + r0 + r) * W;
+    for (int w = lane; w < W; w += 32) out[w] = bw[w];
+    if (lane == 0 && pairs) atomicAdd(head_pairs + h, pairs);
+}
+
+// Union of the rows' sets of query cluster a (members listed by the query
+// cluster sort), as an ascending list.  One CTA per (cluster, head).
+__global__ void pq_union_kernel(int N, const uint32_t *__restrict__ bits, int W, const int32_t *__restrict__ qperm,
+                                const int32_t *__restrict__ qoff, int kq_cap, const int32_t *__restrict__ nq,
+                                int kq_fixed, const uint8_t *__restrict__ dense, int kk_cap,
+                                int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_cnt) {
+    extern __shared__ uint32_t uw[];  // [W]
+    __shared__ int wsum[32];
+    const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const int nqh = nq ? min(max(nq[h], 0), kq_cap) : kq_fixed;
+    const int32_t *o = qoff + (size_t)h * (kq_cap + 1);
+    if (a >= nqh || (dense && dense[h]) || o[a + 1] <= o[a]) {
+        if (tid == 0) sel_cnt[(size_t)h * kq_cap + a] = 0;
+        return;
+    }
+    for (int w = tid; w < W; w += nt) {
+        uint32_t x = 0u;
+        for (int p = o[a]; p < o[a + 1]; p++) x |= bits[((size_t)h * N + qperm[(size_t)h * N + p]) * W + w];
+        uw[w] = x;
+    }
+    __syncthreads();
+    // ascending list of the set bits (block-wide exclusive scan of the word counts)
+    int base = 0;
+    int32_t *out = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
+    for (int w0 = 0; w0 < W; w0 += nt) {
+        const int w = w0 + tid;
+        const int c = w < W ? __popc(uw[w]) : 0;
+        int x = c;
+        const int lane = tid & 31, wi = tid >> 5;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        if (lane == 31) wsum[wi] = x;
+        __syncthreads();
+        int before = base + x - c;
+        for (int u = 0; u < wi; u++) before += wsum[u];
+        if (w < W) {
+            uint32_t m = uw[w];
+            while (m) {
+                const int b = w * 32 + __ffs(m) - 1;
+                m &= m - 1u;
+                if (b < kk_cap) out[before++] = b;
+            }
+        }
+        __syncthreads();
+        for (int u = 0; u < nt / 32; u++) base += wsum[u];
+        __syncthreads();
+    }
+    if (tid == 0) sel_cnt[(size_t)h * kq_cap + a] = min(base, kk_cap);
+}
+
+// One key run per selected non-empty cluster, ascending (the runs are not
+// merged); info = {runs, chunks of chunk_rows rows}.  One thread per (head,
+// query cluster) walks its list.
+__global__ void key_runs_single_kernel(int H, int kq_cap, int kk_cap, const int32_t *__restrict__ koff,
+                                       const int32_t *__restrict__ sel_idx, const int32_t *__restrict__ sel_cnt,
+                                       int chunk_rows, int2 *__restrict__ runs, int2 *__restrict__ info) {
+    const int g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= H * kq_cap) return;
+    const int h = g / kq_cap, a = g - h * kq_cap;
+    const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
+    const int32_t *sl = sel_idx + ((size_t)h * kq_cap + a) * kk_cap;
+    const int n = min(max(sel_cnt[(size_t)h * kq_cap + a], 0), kk_cap);
+    int2 *out = runs + ((size_t)h * kq_cap + a) * kk_cap;
+    int nr = 0;
+    unsigned long long slot_rows = 0ull;
+    for (int c = 0; c < n; c++) {
+        const int b = sl[c];
+        if (b < 0 || b >= kk_cap) continue;
+        const int r0 = ko[b], r1 = ko[b + 1];
+        if (r1 <= r0) continue;
+        out[nr++] = make_int2(r0, r1);
+        slot_rows += (unsigned long long)((r1 - r0 + 7) & ~7);
+    }
+    info[(size_t)h * kq_cap + a] =
+        make_int2(nr, (int)((slot_rows + (unsigned long long)chunk_rows - 1) / (unsigned long long)chunk_rows));
+}
+
+// Per row of query cluster a and chunk j of its key stream: bit g set when
+// the row's own set holds the cluster of 8-key group g.  The groups' clusters
+// come from the runs' slot layout (every run's rows from its slot start, its
+// last group padded), as the key stream packs them.
+constexpr int PQ_MAX_RUNS = 8192;
+__global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *__restrict__ koff,
+                                  const int2 *__restrict__ runs, const int2 *__restrict__ info,
+                                  const int32_t *__restrict__ qperm, const int32_t *__restrict__ qoff,
+                                  const uint32_t *__restrict__ bits, int W, uint16_t *__restrict__ rowmask) {
+    extern __shared__ int pqr[];
+    int *s_start = pqr;                  // [nr] slot start of each run
+    int *gcl = pqr + PQ_MAX_RUNS;        // [nch * 16] cluster of each group (-1: padding)
+    __shared__ int wsum[32];
+    const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const size_t qa = (size_t)h * kq_cap + a;
+    const int2 inf = info[qa];
+    const int nr = min(inf.x, PQ_MAX_RUNS), nch = min(inf.y, max_chunks);
+    const int32_t *o = qoff + (size_t)h * (kq_cap + 1);
+    if (nch <= 0 || o[a + 1] <= o[a]) return;
+    const int2 *rr = runs + qa * kk_cap;
+    const int32_t *ko = koff + (size_t)h * (kk_cap + 1);
+    int carry = 0;
+    for (int b0 = 0; b0 < nr; b0 += nt) {
+        const int r = b0 + tid;
+        int len = 0;
+        if (r < nr) {
+            const int2 v = rr[r];
+            len = (v.y - v.x + 7) & ~7;
+        }
+        int x = len;
+        const int lane = tid & 31, w = tid >> 5;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
+        __syncthreads();
+        int before = carry + x - len;
+        for (int u = 0; u < w; u++) before += wsum[u];
+        if (r < nr) s_start[r] = before;
+        __syncthreads();
+        for (int u = 0; u < nt / 32; u++) carry += wsum[u];
+        __syncthreads();
+    }
+    for (int gi = tid; gi < nch * 16; gi += nt) {
+        const int pos = gi * 8;
+        int lo = 0, hi = nr - 1, r = -1;
+        while (lo <= hi) {
+            const int mid = (lo + hi) >> 1;
+            if (s_start[mid] <= pos) { r = mid; lo = mid + 1; }
+            else hi = mid - 1;
+        }
+        int cl = -1;
+        if (r >= 0) {
+            const int2 v = rr[r];
+            const int key = v.x + (pos - s_start[r]);
+            if (key < v.y) {
+                // the cluster whose rows hold `key`: last b with koff[b] <= key
+                int l2 = 0, h2 = kk_cap - 1, b = 0;
+                while (l2 <= h2) {
+                    const int mid = (l2 + h2) >> 1;
+                    if (ko[mid] <= key) { b = mid; l2 = mid + 1; }
+                    else h2 = mid - 1;
+                }
+                cl = b;
+            }
+        }
+        gcl[gi] = cl;
+    }
+    __syncthreads();
+    for (int p = o[a] + tid; p < o[a + 1]; p += nt) {
+        const uint32_t *rb = bits + ((size_t)h * N + qperm[(size_t)h * N + p]) * W;
+        for (int j = 0; j < nch; j++) {
+            uint32_t m = 0u;
+#pragma unroll
+            for (int g = 0; g < 16; g++) {
+                const int cl = gcl[j * 16 + g];
+                if (cl >= 0 && ((rb[cl >> 5] >> (cl & 31)) & 1u)) m |= 1u << g;
+            }
+            rowmask[((size_t)h * max_chunks + j) * N + p] = (uint16_t)m;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+size_t pq_score_batch_rows(int H, int N, int kk_cap) {
+    // scores of a batch of rows for all heads in about 1 GiB
+    size_t per_row = (size_t)H * kk_cap * sizeof(double);
+    size_t b = ((size_t)1 << 30) / (per_row ? per_row : 1);
+    b = b < 1024 ? 1024 : b;
+    return b < (size_t)N ? b : (size_t)N;
+}
+
+int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_cent, const float *k_max,
+                  const float *k_min, const int32_t *k_count, int kk_cap, const int32_t *nk, int kk_fixed,
+                  int text_group, const uint8_t *dense, int score_mode, int top_k, uint32_t *bits, int W,
+                  double *scores, int batch, unsigned long long *head_pairs, cudaStream_t st) {
+    const int nkmax = nk ? kk_cap : kk_fixed;
+    const int LD = D + 1;
+    const size_t smem_s = (size_t)(PQ_ROWS + 2 * PQ_COLS) * LD * sizeof(float);
+    const size_t per_warp = (size_t)kk_cap * sizeof(double) + (size_t)W * sizeof(uint32_t);
+    int nwarps = (int)((size_t)(200 * 1024) / per_warp);
+    nwarps = nwarps < 1 ? 1 : (nwarps > PQ_WARPS ? PQ_WARPS : nwarps);
+    const size_t smem_t = (size_t)nwarps * per_warp;
+    cudaMemsetAsync(head_pairs, 0, sizeof(unsigned long long) * H, st);
+    for (int r0 = 0; r0 < N; r0 += batch) {
+        const int nb = N - r0 < batch ? N - r0 : batch;
+        dim3 g1((nb + PQ_ROWS - 1) / PQ_ROWS, (nkmax + PQ_COLS - 1) / PQ_COLS, H);
+#define AC_PQS(T, DD)                                                                                              \
+    do {                                                                                                           \
+        if (smem_s > 48 * 1024)                                                                                    \
+            cudaFuncSetAttribute(pq_scores_kernel<T, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s); \
+        pq_scores_kernel<T, DD><<<g1, 128, smem_s, st>>>(static_cast<const T *>(q), N, r0, nb, k_cent, k_max, k_min, \
+                                                         kk_cap, nk, kk_fixed, text_group, score_mode, scores);     \
+    } while (0)
+        if (dtype == DT_BF16) {
+            if (D == 64) AC_PQS(__nv_bfloat16, 64);
+            else AC_PQS(__nv_bfloat16, 128);
+        } else {
+            if (D == 64) AC_PQS(float, 64);
+            else AC_PQS(float, 128);
+        }
+#undef AC_PQS
+        note_launch();
+        if (smem_t > 48 * 1024)
+            cudaFuncSetAttribute(pq_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
+        dim3 g2((nb + nwarps - 1) / nwarps, H);
+        pq_topk_kernel<<<g2, nwarps * 32, smem_t, st>>>(scores, N, r0, nb, k_count, kk_cap, nk, kk_fixed,
+                                                          text_group, dense, top_k, W, bits, head_pairs);
+        note_launch();
+    }
+    return 0;
+}
+
+void k_select_union(int H, int N, const uint32_t *bits, int W, const int32_t *qperm, const int32_t *qoff, int kq_cap,
+                    const int32_t *nq, int kq_fixed, const uint8_t *dense, int kk_cap, int32_t *sel_idx,
+                    int32_t *sel_cnt, cudaStream_t st) {
+    const size_t smem = (size_t)W * sizeof(uint32_t);
+    if (smem > 48 * 1024) cudaFuncSetAttribute(pq_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    pq_union_kernel<<<dim3(kq_cap, H), 256, smem, st>>>(N, bits, W, qperm, qoff, kq_cap, nq, kq_fixed, dense, kk_cap,
+                                                        sel_idx, sel_cnt);
+    note_launch();
+}
+
+void k_key_runs_single(int H, int kq_cap, int kk_cap, const int32_t *koff, const int32_t *sel_idx,
+                       const int32_t *sel_cnt, int chunk_rows, int2 *runs, int2 *info, cudaStream_t st) {
+    const int n = H * kq_cap;
+    key_runs_single_kernel<<<(n + 127) / 128, 128, 0, st>>>(H, kq_cap, kk_cap, koff, sel_idx, sel_cnt, chunk_rows,
+                                                            runs, info);
+    note_launch();
+}
+
+int k_rowmask(int H, int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *koff, const int2 *runs,
+              const int2 *info, const int32_t *qperm, const int32_t *qoff, const uint32_t *bits, int W,
+              uint16_t *rowmask, cudaStream_t st) {
+    const size_t smem = (size_t)(PQ_MAX_RUNS + (size_t)max_chunks * 16) * sizeof(int);
+    if (smem > 227 * 1024) return -1;  // the group table of the longest key stream does not fit
+    cudaFuncSetAttribute(pq_rowmask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    pq_rowmask_kernel<<<dim3(kq_cap, H), 256, smem, st>>>(N, kq_cap, kk_cap, max_chunks, koff, runs, info, qperm,
+                                                          qoff, bits, W, rowmask);
+    note_launch();
+    return 0;
+}
+
+}  // namespace ac

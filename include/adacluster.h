@@ -115,6 +115,11 @@ typedef struct {
                                that no score ranks and every query cluster selects
                                (a dense strip).  Not from the pages, which give text
                                tokens no special treatment; 0 = off.  < n.         */
+    int per_query;          /* 1: selection per query row, as Algorithm 3 writes it
+                               (S has one row per query token; argtopk along each
+                               row): each query attends to the keys of its own
+                               top_k key clusters.  Requires top_k > 0 and bf16
+                               (else AC_ERR_UNSUPPORTED); 0 = per query cluster.   */
 } ac_config;
 
 /* Per-call statistics filled by ac_forward when `stats` is non-NULL (the call
@@ -129,6 +134,10 @@ typedef struct {
      * an assignment pass reproduces the previous one (the result is the same as
      * running all rounds: the update would give back the same centres).       */
     int kmeans_rounds_q, kmeans_rounds_k;
+    /* Pairs the attention kernel computed.  Equal to `pairs` with per-cluster
+     * selection; with per_query, `pairs` counts each row's own set and this the
+     * union per query cluster (rows mask the rest).                          */
+    int64_t pairs_computed;
 } ac_stats;
 
 /* Averages over the ac_forward calls recorded with AC_FLAG_PROFILE since the
@@ -192,6 +201,35 @@ AC_API ac_status ac_select(ac_ctx *ctx, const float *q_cent, const float *q_mean
                     const int32_t *nq, const int32_t *nk, const uint8_t *dense_flag,
                     int32_t *sel_idx, int32_t *sel_cnt, void *ws, size_t ws_bytes, void *stream);
 
+/* Per-query selection (config.per_query = 1; §3.3, Algorithm 3: the score
+ * matrix S has one row per query token and Index <- argtopk(S, topk) runs along
+ * each row).  For every query row i of every head whose dense_flag is 0 (NULL:
+ * none is), each non-empty key cluster b gets
+ *   CENTROID: s_ib = (q_i . c_b) / sqrt(d)
+ *   QUEST:    s_ib = sum_t max(q_it M_bt, q_it m_bt) / sqrt(d)   (k_max, k_min)
+ * (the query is its own representative), and the top_k of largest s_ib (ties:
+ * lower b) are kept; with text_keys, the text group (id = the head's key cluster
+ * count) is always kept.  row_bits [H, N, W] (W = ceil(kk_cap / 32) words,
+ * bit b of word b / 32) receives each row's set; rows of dense heads get none.
+ * k_cent [H, kk_cap, d] (CENTROID), k_count [H, kk_cap], nk [H] (NULL: kk).
+ * Scores are double, in the order of a plain loop over the d elements, so the
+ * sets are exact.  AC_ERR_UNSUPPORTED unless config.per_query.              */
+AC_API ac_status ac_select_rows(ac_ctx *ctx, const void *q, const float *k_cent, const int32_t *k_count,
+                                const float *k_max, const float *k_min, const int32_t *nk,
+                                const uint8_t *dense_flag, uint32_t *row_bits, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* Sparse attention with per-query selection: query row i attends to the keys
+ * of the clusters in its own set row_bits[h, i] (from ac_select_rows):
+ *   out_i = sum_{j: assign_k(j) in S_i} softmax_j(q_i.k_j / sqrt(d)) v_j.
+ * The kernel runs, per query cluster, over the union of its rows' sets and
+ * masks each row to its own clusters.  Everything else as ac_sparse_attn.
+ * AC_ERR_UNSUPPORTED unless config.per_query.                              */
+AC_API ac_status ac_sparse_attn_rows(ac_ctx *ctx, const void *q, const void *k, const void *v,
+                                     const int32_t *q_assign, const int32_t *k_assign, const uint32_t *row_bits,
+                                     const int32_t *nq, const int32_t *nk, const uint8_t *dense_flag, void *out,
+                                     float *lse, void *ws, size_t ws_bytes, void *stream);
+
 /* Quest page bounds of the key clusters (§3.2.3 eq. (1)): k_max / k_min
  * [H, kk_cap, d] receive, per cluster and dimension, the largest / smallest
  * key value over the cluster's members (0 for clusters without members).
@@ -253,7 +291,8 @@ AC_API ac_status ac_sparse_attn(ac_ctx *ctx, const void *q, const void *k, const
                          size_t ws_bytes, void *stream);
 
 /* The whole of Algorithm 3 for every head: ac_cluster_q, ac_cluster_k,
- * (ac_key_bounds with AC_SCORE_QUEST), ac_select, ac_sparse_attn.  q_cent_io / k_cent_io ([H, cap, d], nullable):
+ * (ac_key_bounds with AC_SCORE_QUEST), ac_select, ac_sparse_attn (with
+ * per_query: ac_select_rows, ac_sparse_attn_rows).  q_cent_io / k_cent_io ([H, cap, d], nullable):
  * with AC_FLAG_WARM_START they seed k-means (§3.2.2 "Efficient
  * initialization"); when non-NULL they receive the final centroids.
  * Adaptive clustering reads one int per head back to the host per stage; the
