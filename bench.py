@@ -34,9 +34,9 @@ from clustered_sparse_attention_head_b200 import workloads as W  # noqa: E402
 DEFAULT_WORKLOAD = "wan21-n75600-h40-d128"
 METRIC = "clustered sparse-attn calls/s & achieved TFLOPS at 75.6K tokens vs dense attn"
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention launch (ncu) on
-# the default workload cut to 8 heads (0.522 GB + 0.141 GB); None whenever the
-# kernel changes, until it is captured again
-ATTN_TRAFFIC_8H = 0.6628e9
+# the default workload cut to 8 heads; None whenever the kernel changes, until
+# it is captured again
+ATTN_TRAFFIC_8H = None
 L2_BYTES = 126 * 2 ** 20
 # the CPU oracle's bounded sample: one head clustered and selected in full,
 # attention for SAMPLE_ROWS query rows; heads 0..SAMPLE_HEADS-1 in turn
@@ -425,6 +425,7 @@ def main():
         # every workload gets its own context
         extra["top_p_sweep"] = top_p_sweep(w, q, k, v, out, dev, stream, a.per_config_calls, peak,
                                            dense["ms"] if dense else None)
+        extra["select_modes"] = select_modes(w, q, k, v, out, dev, stream, a.per_config_calls, peak)
         del q, k, v, out
         ac.close()
         torch.cuda.empty_cache()
@@ -485,7 +486,7 @@ def sdpa_ms(q, k, v, stream, flush, calls=3):
     return time_calls(lambda: F.scaled_dot_product_attention(qd, kd, vd), calls, stream, flush)
 
 
-def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0):
+def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0, over=None):
     """One workload through ac_forward: ms per call (CUDA events, L2 flushed
     first when an input tensor fits in L2), the stage breakdown, computed pairs
     and the attention kernel's rate against the peak."""
@@ -495,6 +496,8 @@ def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0):
     cfg = Config.from_workload(w)
     cfg.flags = _abi.AC_FLAG_PROFILE
     cfg.text_keys = text_keys
+    for key, val in (over or {}).items():
+        setattr(cfg, key, val)
     ac = AdaCluster(cfg, device=dev)
     flush = None if tensor_bytes(w) > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     ac.ac_forward(q, k, v, out=out)
@@ -510,7 +513,7 @@ def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0):
         raise RuntimeError(f"{w.name}: device status {status}")
     flops = 4.0 * w.d * st["pairs"]
     attn = prof["ms_attn_kernel"]
-    r = {"ms_per_call": ms, "calls_per_s": 1e3 / ms, "pairs": st["pairs"],
+    r = {"ms_per_call": ms, "calls_per_s": 1e3 / ms, "pairs": st["pairs"], "pairs_computed": st["pairs_computed"],
          "density": st["pairs"] / (w.heads * float(w.n) ** 2), "dense_heads": st["dense_heads"],
          "stages_q": st["max_stages_q"], "stages_k": st["max_stages_k"],
          "stage_ms": {k2: prof[k2] for k2 in ("ms_cluster_q", "ms_cluster_k", "ms_select", "ms_prep",
@@ -535,6 +538,24 @@ def top_p_sweep(w, q, k, v, out, dev, stream, calls, peak, sdpa):
             r["speedup_vs_sdpa"] = sdpa / r["ms_per_call"]
         rows.append(r)
     return rows
+
+
+SELECT_MODES = {
+    "quest_top_p": dict(score_mode=1),
+    "centroid_top_k64": dict(top_k=64),
+    "per_query_top_k64": dict(top_k=64, per_query=True),
+}
+
+
+def select_modes(w, q, k, v, out, dev, stream, calls, peak):
+    """The selection options on the headline workload: the Quest score with the
+    top-p cut, argtopk per query cluster, argtopk per query row."""
+    res = {}
+    for name, over in SELECT_MODES.items():
+        r, _ = measure(w, q, k, v, out, dev, stream, calls, peak, over=over)
+        r["options"] = over
+        res[name] = r
+    return res
 
 
 def per_config(dev, stream, calls, peak):
