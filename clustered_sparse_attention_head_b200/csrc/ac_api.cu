@@ -63,7 +63,7 @@ struct Ws {
     // attention
     size_t qperm, kperm, qoff, koff, qg, kg, vg, items, nitems, pairs, cnt2, segq, segk;
     // tensor-core screen: split centroids and per-stage gathered rows
-    size_t chi, clo, xu, amb_cand, items_scr, runs, run_info, masks, kbmax, kbmin;
+    size_t chi, clo, cnp, xu, amb_cand, items_scr, runs, run_info, masks, kbmax, kbmin;
     // early stop of k-means: previous assignment, per-head records (q, k, Algorithm 1
     // stages), a copy of a stage's pass descriptors
     size_t aprev, kst, seg2;
@@ -134,6 +134,7 @@ Ws layout(const ac_ctx *c) {
     w.kpad = (int)((capm + 127) / 128 * 128);
     w.chi = b.take(H * (size_t)w.kpad * D * 2);
     w.clo = b.take(H * (size_t)w.kpad * D * 2);
+    w.cnp = b.take(H * (size_t)w.kpad * 4);
     w.xu = b.take(HN * D * c->elt);
     w.amb_cand = b.take(HN * 8);
     w.items_scr = b.take(items_scratch_elems((int)H, c->kq_cap) * 4 + 16);
@@ -210,7 +211,7 @@ ac_status assign_step(ac_ctx *c, const Ws &w, void *ws, const void *x, const voi
         AC_CUDA(cudaMemsetAsync(ambc, 0, sizeof(int32_t) * H, st));
         if (k_assign_tc(xc, H, N, D, rows, seg, nrows_max, cent, cap, w.kpad, at<void>(ws, w.chi),
                         at<void>(ws, w.clo), cn2, cmax, norm, mode, assign, amb, ambc, at<int2>(ws, w.amb_cand),
-                        c->d_status, c->encode_fn, st) != 0)
+                        c->d_status, c->encode_fn, at<float>(ws, w.cnp), c->num_sms, st) != 0)
             return AC_ERR_CUDA;
         k_assign_exact(x, DT_BF16, H, N, D, rows, seg, cent, cap, norm, mode, amb, ambc, at<int2>(ws, w.amb_cand),
                        assign, st);

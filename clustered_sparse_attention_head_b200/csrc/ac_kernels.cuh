@@ -46,10 +46,12 @@ void k_conv_check(int H, int N, const HeadSeg *seg, const int32_t *assign, int32
 void k_conv_decide(int H, HeadSeg *seg, int32_t *kst, int it, cudaStream_t st);
 
 // ---- ac_assign_tc.cu (bf16 inputs): tcgen05 screen; the exact pass follows
+// cnp [H, kpad] (nullable: the per-tile kernel): the per-column score shift
+// of the persistent kernel, which runs one CTA per SM (num_sms).
 int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const HeadSeg *seg, int nrows_max,
                 const float *cent, int cap, int kpad, void *chi, void *clo, float *cn2, float *cmax,
                 const double *norm, int mode, int32_t *assign, int32_t *amb_list, int32_t *amb_count, int2 *amb_cand,
-                int *status, void *encode_fn, cudaStream_t st);
+                int *status, void *encode_fn, float *cnp, int num_sms, cudaStream_t st);
 
 // ---- ac_sort.cu
 // Stable counting sort of positions 0..seg.nrows-1 by id (< seg.k): perm gets
