@@ -36,7 +36,7 @@ METRIC = "clustered sparse-attn calls/s & achieved TFLOPS at 75.6K tokens vs den
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention launch (ncu) on
 # the default workload cut to 8 heads; None whenever the kernel changes, until
 # it is captured again
-ATTN_TRAFFIC_8H = None
+ATTN_TRAFFIC_8H = 0.655e9
 L2_BYTES = 126 * 2 ** 20
 # the CPU oracle's bounded sample: one head clustered and selected in full,
 # attention for SAMPLE_ROWS query rows; heads 0..SAMPLE_HEADS-1 in turn

@@ -67,8 +67,8 @@ struct Ws {
     // early stop of k-means: previous assignment, per-head records (q, k, Algorithm 1
     // stages), a copy of a stage's pass descriptors
     size_t aprev, kst, seg2;
-    // selection: the key centroids transposed per head
-    size_t kct;
+    // selection: the key centroids (or Quest maxima) transposed per head, the Quest minima transposed
+    size_t kct, kmt;
     // Algorithm 1's single-cluster stages on chip: working vectors [H, wrows, d] (double)
     size_t wc;
     int wrows;
@@ -148,6 +148,7 @@ Ws layout(const ac_ctx *c) {
     w.kst = b.take(3 * H * 4 * 4);
     w.seg2 = b.take(H * sizeof(HeadSeg));
     w.kct = b.take(H * (size_t)c->kk_cap * D * 4);
+    w.kmt = b.take(quest ? H * (size_t)c->kk_cap * D * 4 : 0);
     // a stage with m_t = ceil(m0 |U| / N) = 1 has |U| <= N / m0
     w.wrows = 0;
     if (g.adaptive_q) w.wrows = (int)(N / g.kq + 1);
@@ -717,7 +718,8 @@ ac_status forward_impl(ac_ctx *c, const void *q, const void *k, const void *v, c
                       at<unsigned long long>(ws, w.hpairs), st);
     } else {
         k_select(g.heads, g.d, qc, qmn, qn, c->kq_cap, kc, kn, kbmax, kbmin, c->kk_cap, nq, nk, g.kq, g.kk + tg, dense,
-                 (int)g.score_mode, g.top_k, g.top_p, sel, selc, c->d_status, st, tg, at<float>(ws, w.kct));
+                 (int)g.score_mode, g.top_k, g.top_p, sel, selc, c->d_status, st, tg, at<float>(ws, w.kct),
+                 g.score_mode == AC_SCORE_QUEST ? at<float>(ws, w.kmt) : nullptr);
     }
     if (pe) AC_CUDA(cudaEventRecord(pe[3], st));
     if (stats) AC_CUDA(cudaEventRecord(c->ev[3], st));
@@ -811,7 +813,8 @@ ac_status ac_select(ac_ctx *c, const float *q_cent, const float *q_mean_norm, co
     if (s != AC_OK) return s;
     k_select(g.heads, g.d, q_cent, q_mean_norm, q_count, c->kq_cap, k_cent, k_count, k_max, k_min, c->kk_cap, nq, nk,
              g.kq, g.kk + (g.text_keys > 0 ? 1 : 0), dense_flag, (int)g.score_mode, g.top_k, g.top_p, sel_idx, sel_cnt,
-             c->d_status, (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0, at<float>(ws, layout(c).kct));
+             c->d_status, (cudaStream_t)stream, g.text_keys > 0 ? 1 : 0, at<float>(ws, layout(c).kct),
+             g.score_mode == AC_SCORE_QUEST ? at<float>(ws, layout(c).kmt) : nullptr);
     return launch_check();
 }
 

@@ -70,7 +70,8 @@ void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const
               const int32_t *nq, const int32_t *nk, int kq_fixed, int kk_fixed, const uint8_t *dense, int score_mode,
               int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, int *status, cudaStream_t st,
               int text_group = 0,
-              float *k_cent_t = nullptr);  // k_cent_t: [H, D, kk_cap] scratch for the transposed centroids
+              float *k_cent_t = nullptr,   // [H, D, kk_cap] scratch: transposed centroids (or Quest maxima)
+              float *k_min_t = nullptr);   // [H, D, kk_cap] scratch: transposed Quest minima
 // Per-cluster, per-dimension max / min of x over the members listed by a
 // cluster sort (perm, off [H, cap + 1]); 0 for empty clusters.
 void k_cluster_bounds(const void *x, int dtype, int H, int N, int D, const int32_t *perm, const int32_t *off,

@@ -40,8 +40,8 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
                               const float *__restrict__ k_min, int kk_cap, const int32_t *__restrict__ nq,
                               const int32_t *__restrict__ nk, int kq_fixed, int kk_fixed,
                               const uint8_t *__restrict__ dense, int score_mode, int top_k, double top_p, int n2,
-                              int text_group, const float *__restrict__ k_cent_t, int32_t *__restrict__ sel_idx,
-                              int32_t *__restrict__ sel_cnt, int *status) {
+                              int text_group, const float *__restrict__ k_cent_t, const float *__restrict__ k_min_t,
+                              int32_t *__restrict__ sel_idx, int32_t *__restrict__ sel_cnt, int *status) {
     extern __shared__ __align__(16) unsigned char smraw[];
     double *sp = reinterpret_cast<double *>(smraw);          // [n2] p (sort key)
     int *sb = reinterpret_cast<int *>(sp + n2);             // [n2] b
@@ -92,10 +92,18 @@ __global__ void select_kernel(int D, const float *__restrict__ q_cent, const flo
             if (score_mode == 1) {
                 // qbar+ . M_b + qbar- . m_b, summed per dimension: each term
                 // equals max(qbar_t M_bt, qbar_t m_bt) of eq. (1) exactly
-                const float *M = kmx + (size_t)b * D, *mn = kmn + (size_t)b * D;
                 double acc = 0.0;
-                for (int t = 0; t < D; t++)
-                    acc = dadd(acc, dadd(dmul(qpos[t], (double)M[t]), dmul(qneg[t], (double)mn[t])));
+                if (kct && k_min_t) {
+                    // transposed bounds: a warp reads consecutive clusters
+                    const float *Mt = kct, *mt = k_min_t + (size_t)h * kk_cap * D;
+                    for (int t = 0; t < D; t++)
+                        acc = dadd(acc, dadd(dmul(qpos[t], (double)Mt[(size_t)t * kk_cap + b]),
+                                             dmul(qneg[t], (double)mt[(size_t)t * kk_cap + b])));
+                } else {
+                    const float *M = kmx + (size_t)b * D, *mn = kmn + (size_t)b * D;
+                    for (int t = 0; t < D; t++)
+                        acc = dadd(acc, dadd(dmul(qpos[t], (double)M[t]), dmul(qneg[t], (double)mn[t])));
+                }
                 s = dmul(acc, scale);
             } else {
                 double dot = 0.0;
@@ -216,16 +224,24 @@ void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const
               const float *k_cent, const int32_t *k_count, const float *k_max, const float *k_min, int kk_cap,
               const int32_t *nq, const int32_t *nk, int kq_fixed, int kk_fixed, const uint8_t *dense, int score_mode,
               int top_k, double top_p, int32_t *sel_idx, int32_t *sel_cnt, int *status, cudaStream_t st,
-              int text_group, float *k_cent_t) {
+              int text_group, float *k_cent_t, float *k_min_t) {
     int n2 = 1;
     while (n2 < kk_cap) n2 <<= 1;
     size_t smem = (size_t)n2 * (sizeof(double) + sizeof(int)) + (size_t)kk_cap * (sizeof(double) + sizeof(int) + 1);
+    const dim3 tg((kk_cap + 31) / 32, (D + 31) / 32, H), tb(32, 8);
     if (k_cent_t && score_mode == 0) {
-        transpose_cent_kernel<<<dim3((kk_cap + 31) / 32, (D + 31) / 32, H), dim3(32, 8), 0, st>>>(k_cent, kk_cap, D,
-                                                                                                   k_cent_t);
+        transpose_cent_kernel<<<tg, tb, 0, st>>>(k_cent, kk_cap, D, k_cent_t);
+        note_launch();
+        k_min_t = nullptr;
+    } else if (k_cent_t && k_min_t && score_mode == 1) {
+        // the Quest bounds, transposed the same way (k_cent_t holds M^T)
+        transpose_cent_kernel<<<tg, tb, 0, st>>>(k_max, kk_cap, D, k_cent_t);
+        transpose_cent_kernel<<<tg, tb, 0, st>>>(k_min, kk_cap, D, k_min_t);
+        note_launch();
         note_launch();
     } else {
         k_cent_t = nullptr;
+        k_min_t = nullptr;
     }
     // opt in whenever dynamic plus static shared memory may pass 48 KB (the
     // attribute belongs to the current device, so it is set on every call)
@@ -233,7 +249,7 @@ void k_select(int H, int D, const float *q_cent, const float *q_mean_norm, const
     dim3 g(kq_cap, H);
     select_kernel<<<g, 256, smem, st>>>(D, q_cent, q_mean_norm, q_count, kq_cap, k_cent, k_count, k_max, k_min,
                                         kk_cap, nq, nk, kq_fixed, kk_fixed, dense, score_mode, top_k, top_p, n2,
-                                        text_group, k_cent_t, sel_idx, sel_cnt, status);
+                                        text_group, k_cent_t, k_min_t, sel_idx, sel_cnt, status);
     note_launch();
 }
 
