@@ -320,80 +320,21 @@ __global__ void dist_kernel(const T *__restrict__ x, int N, const int32_t *__res
 }
 
 // ----------------------------------------------------------------- update
-// Cluster j of head h (grid x = j, y = h; blockDim = D): members are
-// perm[off[j] .. off[j+1]) in token order; thread t sums element t of their
-// working vectors in double in that order.  EUCLID: c = sum / count.
-// SPHERE: mu = sum / ||sum||.  Empty clusters (or a zero sum) keep their centroid.
-template <typename T, int D>
-__global__ void update_kernel(const T *__restrict__ x, int N, const HeadSeg *__restrict__ seg,
-                              const int32_t *__restrict__ perm, const int32_t *__restrict__ off, int cap,
-                              const double *__restrict__ norm, int mode, float *__restrict__ cent) {
-    __shared__ double ssum[D];
-    __shared__ double snr;
-    __shared__ int toks[512];
-    __shared__ double nrms[512];
-    int h = blockIdx.y, j = blockIdx.x, t = threadIdx.x;
-    HeadSeg s = seg[h];
-    if (s.nrows <= 0 || j >= s.k) return;
-    const int32_t *o = off + (size_t)h * (cap + 1);
-    const int b = o[j], e = o[j + 1];
-    if (e <= b) return;
-    const int32_t *ph = perm + (size_t)h * N;
-    const T *xh = x + (size_t)h * N * D;
-    double acc = 0.0;
-    for (int r0 = b; r0 < e; r0 += 512) {
-        const int n = min(512, e - r0);
-        __syncthreads();
-        for (int i = t; i < n; i += D) {
-            const int tk = ph[r0 + i];
-            toks[i] = tk;
-            nrms[i] = (mode == MODE_SPHERE) ? norm[(size_t)h * N + tk] : 1.0;
-        }
-        __syncthreads();
-        int i = 0;
-        // members in order; 16 independent loads in flight, sums stay sequential
-        for (; i + 16 <= n; i += 16) {
-            double v[16];
-#pragma unroll
-            for (int u = 0; u < 16; u++) v[u] = (double)to_f(xh[(size_t)toks[i + u] * D + t]);
-#pragma unroll
-            for (int u = 0; u < 16; u++) {
-                const double w = (mode == MODE_SPHERE) ? (nrms[i + u] > 0.0 ? ddiv(v[u], nrms[i + u]) : 0.0) : v[u];
-                acc = dadd(acc, w);
-            }
-        }
-        for (; i < n; i++) {
-            const double v = (double)to_f(xh[(size_t)toks[i] * D + t]);
-            acc = dadd(acc, (mode == MODE_SPHERE) ? (nrms[i] > 0.0 ? ddiv(v, nrms[i]) : 0.0) : v);
-        }
-    }
-    float *c = cent + ((size_t)h * cap + s.cent_off + j) * D;
-    if (mode == MODE_EUCLID) {
-        c[t] = (float)ddiv(acc, (double)(e - b));
-        return;
-    }
-    ssum[t] = acc;
-    __syncthreads();
-    if (t == 0) {
-        double ss = 0.0;
-        for (int u = 0; u < D; u++) ss = dadd(ss, dmul(ssum[u], ssum[u]));
-        snr = sqrt(ss);
-    }
-    __syncthreads();
-    if (snr > 0.0) c[t] = (float)ddiv(acc, snr);
-}
-
-// Same result as update_kernel, with the member rows staged through shared
-// memory.  The rows of cluster j are perm[off[j] .. off[j+1]) (token order);
-// chunks of R rows are copied by cp.async as 16-byte pieces (every thread
-// copies pieces of several rows, so a CTA keeps up to two chunks in flight
-// while it sums a third), and thread t adds element t of the chunk's rows in
-// order, in double.  On the sphere the working value x/||x|| is the correctly
-// rounded quotient, computed from y = RN(1/||x||) (one per row) with
-// Markstein's correction (q = RN(x y), r = x - ||x|| q exactly by FMA,
-// RN(q + r y) = RN(x / ||x||); Markstein 1990, see Muller et al., Handbook of
-// Floating-Point Arithmetic, on division by FMA), the value plain division
-// gives.
+// Cluster j of head h (grid x = j, y = h): members are perm[off[j] .. off[j+1])
+// in token order; element t of their working vectors is summed in double in
+// that order.  EUCLID: c = sum / count.  SPHERE: mu = sum / ||sum||.  Empty
+// clusters (or a zero sum) keep their centroid.
+//
+// The member rows are staged through shared memory: chunks of R rows are
+// copied by cp.async as 16-byte pieces (every thread copies four pieces, so a
+// CTA keeps two chunks in flight while it sums a third), and thread t adds
+// element t of the chunk's rows in order.  The token ids of a chunk are read
+// one chunk before its copy is issued, so the copy never waits for them.  On
+// the sphere the working value x/||x|| is the correctly rounded quotient,
+// computed from y = RN(1/||x||) (one per row) with Markstein's correction
+// (q = RN(x y), r = x - ||x|| q exactly by FMA, RN(q + r y) = RN(x / ||x||);
+// Markstein 1990, see Muller et al., Handbook of Floating-Point Arithmetic,
+// on division by FMA), the value plain division gives.
 namespace {
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -409,6 +350,7 @@ template <int NPEND> __device__ __forceinline__ void cp_async_wait() {
 
 // 8 KB chunks, three stages: about 25 KB of shared memory, eight CTAs (clusters) per SM
 constexpr int UPD_THREADS = 128, UPD_STAGES = 3, UPD_CHUNK_BYTES = 8192;
+constexpr int UPD_PIECES_PER_THREAD = UPD_CHUNK_BYTES / 16 / UPD_THREADS;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restrict__ x, int N,
@@ -420,6 +362,8 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
     constexpr int ROW_BYTES = D * (int)sizeof(T);
     constexpr int R = UPD_CHUNK_BYTES / ROW_BYTES;   // rows per chunk
     constexpr int PIECES = ROW_BYTES / 16;           // 16-byte pieces per row
+    static_assert(R * PIECES == UPD_PIECES_PER_THREAD * UPD_THREADS, "four pieces per thread");
+    static_assert(R <= UPD_THREADS && D <= UPD_THREADS, "one thread per row / element");
     extern __shared__ __align__(16) unsigned char upd_smem[];
     T *rows = reinterpret_cast<T *>(upd_smem);                                           // [S][R][D]
     double *nrm = reinterpret_cast<double *>(upd_smem + UPD_STAGES * UPD_CHUNK_BYTES);  // [S][R]
@@ -437,37 +381,52 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
     const T *xh = x + (size_t)h * N * D;
     const double *nh = norm + (size_t)h * N;
     const bool sphere = mode == MODE_SPHERE;
-    // copy chunk c into stage c % S (one commit group per chunk, also when empty)
-    auto issue = [&](int c) {
-        if (c < nchunks) {
-            const int r0 = c * R, nr = min(R, n - r0), st = c % UPD_STAGES;
-            unsigned char *dst = reinterpret_cast<unsigned char *>(rows) + (size_t)st * UPD_CHUNK_BYTES;
-            for (int pc = tid; pc < nr * PIECES; pc += UPD_THREADS) {
-                const int r = pc / PIECES, q = pc - r * PIECES;
-                const int tok = ph[r0 + r];
-                cp_async16(dst + r * ROW_BYTES + q * 16,
-                           reinterpret_cast<const unsigned char *>(xh + (size_t)tok * D) + q * 16);
-            }
-            if (sphere)
-                for (int r = tid; r < nr; r += UPD_THREADS) cp_async8(nrm + st * R + r, nh + ph[r0 + r]);
+    // token ids of this thread's pieces of the next chunk to copy (and, on the
+    // sphere, of row tid, whose norm it copies); -1 past the chunk's end
+    int tk[UPD_PIECES_PER_THREAD], tkn = -1;
+    auto load_tokens = [&](int c) {
+        const int r0 = c * R, nr = c < nchunks ? min(R, n - r0) : 0;
+#pragma unroll
+        for (int k = 0; k < UPD_PIECES_PER_THREAD; k++) {
+            const int r = (tid + k * UPD_THREADS) / PIECES;
+            tk[k] = r < nr ? ph[r0 + r] : -1;
         }
+        tkn = (sphere && tid < nr) ? ph[r0 + tid] : -1;
+    };
+    // copy chunk c (tokens in tk) into stage c % S: one commit group per chunk, also when empty
+    auto issue = [&](int c) {
+        unsigned char *dst = reinterpret_cast<unsigned char *>(rows) + (size_t)(c % UPD_STAGES) * UPD_CHUNK_BYTES;
+#pragma unroll
+        for (int k = 0; k < UPD_PIECES_PER_THREAD; k++) {
+            const int pc = tid + k * UPD_THREADS, r = pc / PIECES, q = pc - r * PIECES;
+            if (tk[k] >= 0)
+                cp_async16(dst + r * ROW_BYTES + q * 16,
+                           reinterpret_cast<const unsigned char *>(xh + (size_t)tk[k] * D) + q * 16);
+        }
+        if (tkn >= 0) cp_async8(nrm + (c % UPD_STAGES) * R + tid, nh + tkn);
         cp_async_commit();
     };
 #pragma unroll
-    for (int c = 0; c < UPD_STAGES - 1; c++) issue(c);
+    for (int c = 0; c < UPD_STAGES - 1; c++) {
+        load_tokens(c);
+        issue(c);
+    }
+    load_tokens(UPD_STAGES - 1);
     double acc = 0.0;
     for (int c = 0; c < nchunks; c++) {
         cp_async_wait<UPD_STAGES - 2>();
         __syncthreads();  // chunk c has landed for every thread; stage (c - 1) % S is free
         const int st = c % UPD_STAGES, nr = min(R, n - c * R);
         if (sphere) {
-            for (int r = tid; r < nr; r += UPD_THREADS) {
-                const double v = nrm[st * R + r];
-                rcp[st * R + r] = v > 0.0 ? __drcp_rn(v) : 0.0;
+            // y = RN(1/||x||) once per row; 0 marks a zero row (its quotients are 0)
+            if (tid < nr) {
+                const double v = nrm[st * R + tid];
+                rcp[st * R + tid] = v > 0.0 ? __drcp_rn(v) : 0.0;
             }
             __syncthreads();
         }
         issue(c + UPD_STAGES - 1);
+        load_tokens(c + UPD_STAGES);
         if (tid < D) {
             const T *rs = rows + (size_t)st * R * D + tid;
             if (sphere) {
@@ -476,13 +435,10 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
                 for (int r = 0; r < nr; r++) {
                     const double v = (double)to_f(rs[r * D]);
                     const double bn = nr_s[r], y = rc_s[r];
-                    double q = 0.0;
-                    if (bn > 0.0) {
-                        const double q0 = dmul(v, y);
-                        const double rr = __fma_rn(-bn, q0, v);
-                        q = __fma_rn(rr, y, q0);
-                    }
-                    acc = dadd(acc, q);
+                    const double q0 = dmul(v, y);
+                    const double rr = __fma_rn(-bn, q0, v);
+                    const double q = __fma_rn(rr, y, q0);
+                    acc = dadd(acc, bn > 0.0 ? q : 0.0);
                 }
             } else {
 #pragma unroll 8
@@ -629,7 +585,7 @@ void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, 
 void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg, int kmax, const int32_t *perm,
               const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st) {
     dim3 g(kmax, H);
-    // staged rows (16 KB chunks, three stages) plus the rows' norms and reciprocals
+    // staged rows (8 KB chunks, three stages) plus the rows' norms and reciprocals
 #define AC_UPD(T, DD)                                                                                             \
     do {                                                                                                          \
         constexpr int R_ = UPD_CHUNK_BYTES / (DD * (int)sizeof(T));                                               \
