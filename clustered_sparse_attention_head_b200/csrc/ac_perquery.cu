@@ -3,8 +3,8 @@
 // tables that let the block-sparse attention kernel honour each row's own set.
 //
 //  1. pq_scores_kernel: s_ib for every query row i and key cluster b, in double
-//     with the oracle's summation order (one thread per score, elements in
-//     order): CENTROID s = (q_i . c_b) / sqrt(d); QUEST s = sum_t
+//     with the oracle's summation order (each thread 4 x 4 scores, elements
+//     in order): CENTROID s = (q_i . c_b) / sqrt(d); QUEST s = sum_t
 //     max(q_t M_bt, q_t m_bt) / sqrt(d) (the query is its own representative).
 //  2. pq_topk_kernel: one warp per row keeps the top_k non-empty clusters of
 //     largest s (ties to the lower id) as a bit set [H, N, W] (W = kk_cap / 32
@@ -22,74 +22,86 @@
 
 namespace ac {
 
-constexpr int PQ_ROWS = 32, PQ_COLS = 32;
+// Score tiles of 64 rows x 64 clusters per 256-thread CTA, each thread 4 x 4;
+// operands staged in shared memory as doubles, element-major (so a thread's
+// four rows or four clusters of one element are two 16-byte loads), rows of
+// PQ_LD doubles
+constexpr int PQ_ROWS = 64, PQ_COLS = 64, PQ_LD = 66;
 
 template <typename T, int D>
-__global__ void __launch_bounds__(128) pq_scores_kernel(const T *__restrict__ q, int N, int r0, int nb,
+__global__ void __launch_bounds__(256) pq_scores_kernel(const T *__restrict__ q, int N, int r0, int nb,
                                                         const float *__restrict__ k_cent,
                                                         const float *__restrict__ k_max,
                                                         const float *__restrict__ k_min, int kk_cap,
                                                         const int32_t *__restrict__ nk, int kk_fixed, int text_group,
                                                         int score_mode, double *__restrict__ scores) {
-    constexpr int LD = D + 1;  // padded rows: the 32 rows of a tile sit in 32 banks
-    extern __shared__ float pqs[];
-    float *qs = pqs;                     // [PQ_ROWS][LD]
-    float *cs = qs + PQ_ROWS * LD;       // [PQ_COLS][LD] (centroid or M)
-    float *ms = cs + PQ_COLS * LD;       // [PQ_COLS][LD] (m, Quest only)
+    extern __shared__ double pqs[];
+    double *qs = pqs;                 // [D][PQ_LD]: element t of row r at qs[t * PQ_LD + r]
+    double *cs = qs + D * PQ_LD;      // [D][PQ_LD]: centroid (or M) element t of cluster c
+    double *ms = cs + D * PQ_LD;      // [D][PQ_LD]: m (Quest only)
     const int h = blockIdx.z, tid = threadIdx.x;
     const int nkh = (nk ? min(max(nk[h], 0), kk_cap) : kk_fixed) - text_group;
     const int b0 = blockIdx.y * PQ_COLS, i0 = blockIdx.x * PQ_ROWS;
     if (b0 >= nkh) return;
-    for (int e = tid; e < PQ_ROWS * D; e += 128) {
+    for (int e = tid; e < PQ_ROWS * D; e += 256) {
         const int r = e / D, t = e - r * D;
         const int i = r0 + i0 + r;
-        qs[r * LD + t] = (i0 + r < nb && i < N) ? to_f(q[((size_t)h * N + i) * D + t]) : 0.f;
+        qs[t * PQ_LD + r] = (i0 + r < nb && i < N) ? (double)to_f(q[((size_t)h * N + i) * D + t]) : 0.0;
     }
-    for (int e = tid; e < PQ_COLS * D; e += 128) {
+    for (int e = tid; e < PQ_COLS * D; e += 256) {
         const int c = e / D, t = e - c * D;
         const int b = b0 + c;
         const size_t o = ((size_t)h * kk_cap + b) * D + t;
         if (score_mode == 1) {
-            cs[c * LD + t] = b < nkh ? k_max[o] : 0.f;
-            ms[c * LD + t] = b < nkh ? k_min[o] : 0.f;
+            cs[t * PQ_LD + c] = b < nkh ? (double)k_max[o] : 0.0;
+            ms[t * PQ_LD + c] = b < nkh ? (double)k_min[o] : 0.0;
         } else {
-            cs[c * LD + t] = b < nkh ? k_cent[o] : 0.f;
+            cs[t * PQ_LD + c] = b < nkh ? (double)k_cent[o] : 0.0;
         }
     }
     __syncthreads();
-    const int tx = tid & 7, ty = tid >> 3;  // 4 clusters x 2 rows per thread
-    double acc[2][4];
+    const int tx = tid & 15, ty = tid >> 4;  // clusters 4 tx .. 4 tx + 3, rows 4 ty .. 4 ty + 3
+    double acc[4][4];
 #pragma unroll
-    for (int i = 0; i < 2; i++)
+    for (int i = 0; i < 4; i++)
 #pragma unroll
         for (int j = 0; j < 4; j++) acc[i][j] = 0.0;
     if (score_mode == 1) {
         for (int t = 0; t < D; t++) {
+            const double2 qa = *reinterpret_cast<const double2 *>(qs + t * PQ_LD + 4 * ty);
+            const double2 qb = *reinterpret_cast<const double2 *>(qs + t * PQ_LD + 4 * ty + 2);
+            const double2 ca = *reinterpret_cast<const double2 *>(cs + t * PQ_LD + 4 * tx);
+            const double2 cb = *reinterpret_cast<const double2 *>(cs + t * PQ_LD + 4 * tx + 2);
+            const double2 ma = *reinterpret_cast<const double2 *>(ms + t * PQ_LD + 4 * tx);
+            const double2 mb = *reinterpret_cast<const double2 *>(ms + t * PQ_LD + 4 * tx + 2);
+            const double qv[4] = {qa.x, qa.y, qb.x, qb.y}, cv[4] = {ca.x, ca.y, cb.x, cb.y},
+                         mv[4] = {ma.x, ma.y, mb.x, mb.y};
 #pragma unroll
-            for (int i = 0; i < 2; i++) {
-                const double qb = (double)qs[(2 * ty + i) * LD + t];
+            for (int i = 0; i < 4; i++)
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
-                    const double hi = dmul(qb, (double)cs[(4 * tx + j) * LD + t]);
-                    const double lo = dmul(qb, (double)ms[(4 * tx + j) * LD + t]);
+                    const double hi = dmul(qv[i], cv[j]);
+                    const double lo = dmul(qv[i], mv[j]);
                     acc[i][j] = dadd(acc[i][j], hi > lo ? hi : lo);
                 }
-            }
         }
     } else {
         for (int t = 0; t < D; t++) {
+            const double2 qa = *reinterpret_cast<const double2 *>(qs + t * PQ_LD + 4 * ty);
+            const double2 qb = *reinterpret_cast<const double2 *>(qs + t * PQ_LD + 4 * ty + 2);
+            const double2 ca = *reinterpret_cast<const double2 *>(cs + t * PQ_LD + 4 * tx);
+            const double2 cb = *reinterpret_cast<const double2 *>(cs + t * PQ_LD + 4 * tx + 2);
+            const double qv[4] = {qa.x, qa.y, qb.x, qb.y}, cv[4] = {ca.x, ca.y, cb.x, cb.y};
 #pragma unroll
-            for (int i = 0; i < 2; i++) {
-                const double qv = (double)qs[(2 * ty + i) * LD + t];
+            for (int i = 0; i < 4; i++)
 #pragma unroll
-                for (int j = 0; j < 4; j++) acc[i][j] = dadd(acc[i][j], dmul(qv, (double)cs[(4 * tx + j) * LD + t]));
-            }
+                for (int j = 0; j < 4; j++) acc[i][j] = dadd(acc[i][j], dmul(qv[i], cv[j]));
         }
     }
     const double scale = 1.0 / sqrt((double)D);
 #pragma unroll
-    for (int i = 0; i < 2; i++) {
-        const int r = i0 + 2 * ty + i;
+    for (int i = 0; i < 4; i++) {
+        const int r = i0 + 4 * ty + i;
         if (r >= nb || r0 + r >= N) continue;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
@@ -316,14 +328,34 @@ __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks,
         gcl[gi] = cl;
     }
     __syncthreads();
+    // compress each chunk's 16 groups, in place, into (cluster << 16 | groups)
+    // entries, one per run of groups of one cluster (usually one or two)
+    int *nent = gcl + max_chunks * 16;  // [nch]
+    for (int j = tid; j < nch; j += nt) {
+        int ne = 0, cur = -1;
+        uint32_t gm = 0u;
+        for (int g = 0; g < 16; g++) {
+            const int cl = gcl[j * 16 + g];
+            if (cl != cur) {
+                if (cur >= 0) gcl[j * 16 + ne++] = (int)(((uint32_t)cur << 16) | gm);
+                cur = cl;
+                gm = 0u;
+            }
+            if (cl >= 0) gm |= 1u << g;
+        }
+        if (cur >= 0) gcl[j * 16 + ne++] = (int)(((uint32_t)cur << 16) | gm);
+        nent[j] = ne;
+    }
+    __syncthreads();
     for (int p = o[a] + tid; p < o[a + 1]; p += nt) {
         const uint32_t *rb = bits + ((size_t)h * N + qperm[(size_t)h * N + p]) * W;
         for (int j = 0; j < nch; j++) {
             uint32_t m = 0u;
-#pragma unroll
-            for (int g = 0; g < 16; g++) {
-                const int cl = gcl[j * 16 + g];
-                if (cl >= 0 && ((rb[cl >> 5] >> (cl & 31)) & 1u)) m |= 1u << g;
+            const int ne = nent[j];
+            for (int e = 0; e < ne; e++) {
+                const uint32_t v = (uint32_t)gcl[j * 16 + e];
+                const uint32_t cl = v >> 16;
+                if ((rb[cl >> 5] >> (cl & 31)) & 1u) m |= v & 0xFFFFu;
             }
             rowmask[((size_t)h * max_chunks + j) * N + p] = (uint16_t)m;
         }
@@ -344,8 +376,7 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
                   int text_group, const uint8_t *dense, int score_mode, int top_k, uint32_t *bits, int W,
                   double *scores, int batch, unsigned long long *head_pairs, cudaStream_t st) {
     const int nkmax = nk ? kk_cap : kk_fixed;
-    const int LD = D + 1;
-    const size_t smem_s = (size_t)(PQ_ROWS + 2 * PQ_COLS) * LD * sizeof(float);
+    const size_t smem_s = (size_t)(score_mode == 1 ? 3 : 2) * D * PQ_LD * sizeof(double);
     const size_t per_warp = (size_t)kk_cap * sizeof(double) + (size_t)W * sizeof(uint32_t);
     int nwarps = (int)((size_t)(200 * 1024) / per_warp);
     nwarps = nwarps < 1 ? 1 : (nwarps > PQ_WARPS ? PQ_WARPS : nwarps);
@@ -358,7 +389,7 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
     do {                                                                                                           \
         if (smem_s > 48 * 1024)                                                                                    \
             cudaFuncSetAttribute(pq_scores_kernel<T, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s); \
-        pq_scores_kernel<T, DD><<<g1, 128, smem_s, st>>>(static_cast<const T *>(q), N, r0, nb, k_cent, k_max, k_min, \
+        pq_scores_kernel<T, DD><<<g1, 256, smem_s, st>>>(static_cast<const T *>(q), N, r0, nb, k_cent, k_max, k_min, \
                                                          kk_cap, nk, kk_fixed, text_group, score_mode, scores);     \
     } while (0)
         if (dtype == DT_BF16) {
@@ -401,7 +432,7 @@ void k_key_runs_single(int H, int kq_cap, int kk_cap, const int32_t *koff, const
 int k_rowmask(int H, int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *koff, const int2 *runs,
               const int2 *info, const int32_t *qperm, const int32_t *qoff, const uint32_t *bits, int W,
               uint16_t *rowmask, cudaStream_t st) {
-    const size_t smem = (size_t)(PQ_MAX_RUNS + (size_t)max_chunks * 16) * sizeof(int);
+    const size_t smem = (size_t)(PQ_MAX_RUNS + (size_t)max_chunks * 17) * sizeof(int);
     if (smem > 227 * 1024) return -1;  // the group table of the longest key stream does not fit
     cudaFuncSetAttribute(pq_rowmask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     pq_rowmask_kernel<<<dim3(kq_cap, H), 256, smem, st>>>(N, kq_cap, kk_cap, max_chunks, koff, runs, info, qperm,
