@@ -111,11 +111,22 @@ __global__ void __launch_bounds__(256) pq_scores_kernel(const T *__restrict__ q,
     }
 }
 
-// One warp per query row: top_k rounds of a warp-wide argmax over the row's
-// scores (staged in shared memory), ties to the lower id, empty clusters and
-// clusters already taken skipped.  Up to four warps (rows) per block, fewer
-// when kk_cap is large.
-constexpr int PQ_WARPS = 4;
+// One warp per query row keeps the top_k non-empty clusters of largest score,
+// ties to the lower id.  Up to 512 clusters: lane l holds clusters l + 32 i
+// (i < 16), sorts them once (a bitonic network in registers, by score
+// descending then id ascending; empty clusters and NaN scores last), and
+// top_k rounds merge the 32 sorted lists (a warp-wide argmax over the lists'
+// heads; the winning lane shifts its list up by one).  More clusters: top_k rounds of a
+// warp-wide argmax over the row's scores staged in shared memory, clusters
+// already taken skipped.  Up to four warps (rows) per block, fewer when
+// kk_cap is large.
+constexpr int PQ_WARPS = 4, PQ_SORTED = 512;
+// bytes of a warp's score region
+__host__ __device__ constexpr size_t pq_topk_region(int kk_cap) { return (size_t)kk_cap * 8; }
+// x before y in the selection order: larger score, then lower id
+__device__ __forceinline__ bool pq_before(double xv, int xi, double yv, int yi) {
+    return xv > yv || (xv == yv && xi < yi);
+}
 __global__ void __launch_bounds__(PQ_WARPS * 32) pq_topk_kernel(const double *__restrict__ scores, int N, int r0,
                                                                int nb, const int32_t *__restrict__ k_count, int kk_cap,
                                                                const int32_t *__restrict__ nk, int kk_fixed,
@@ -124,9 +135,9 @@ __global__ void __launch_bounds__(PQ_WARPS * 32) pq_topk_kernel(const double *__
                                                                unsigned long long *__restrict__ head_pairs) {
     extern __shared__ unsigned char pqt[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    double *sc = reinterpret_cast<double *>(pqt) + (size_t)warp * kk_cap;               // [warps][kk_cap]
-    uint32_t *bw = reinterpret_cast<uint32_t *>(reinterpret_cast<double *>(pqt) + (size_t)nw * kk_cap) +
-                   (size_t)warp * W;                                                      // [warps][W]
+    const size_t region = pq_topk_region(kk_cap);
+    double *sc = reinterpret_cast<double *>(pqt + (size_t)warp * region);  // [warps][region]
+    uint32_t *bw = reinterpret_cast<uint32_t *>(pqt + (size_t)nw * region) + (size_t)warp * W;  // [warps][W]
     const int h = blockIdx.y;
     const int r = blockIdx.x * nw + warp;
     if (r >= nb || r0 + r >= N) return;  // whole warp
@@ -136,17 +147,93 @@ __global__ void __launch_bounds__(PQ_WARPS * 32) pq_topk_kernel(const double *__
     for (int w = lane; w < W; w += 32) bw[w] = 0u;
     const bool dn = dense && dense[h];
     unsigned long long pairs = 0ull;
-    if (!dn) {
+    if (!dn && nkh <= PQ_SORTED) {
         const double *srow = scores + ((size_t)h * nb + r) * kk_cap;
-        for (int b = lane; b < nkh; b += 32) sc[b] = kc[b] > 0 ? srow[b] : -INFINITY;
+        double v[16];
+        int ix[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const int b = lane + 32 * i;
+            double x = -INFINITY;
+            int id = 0x7fffffff;  // empty cluster or NaN score: after every selectable one
+            if (b < nkh && kc[b] > 0) {
+                const double sv = srow[b];
+                if (sv == sv) {
+                    x = sv;
+                    id = b;
+                }
+            }
+            v[i] = x;
+            ix[i] = id;
+        }
+        // bitonic sort into selection order (pq_before)
+#pragma unroll
+        for (int k = 2; k <= 16; k <<= 1)
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+                for (int i = 0; i < 16; i++) {
+                    const int l = i ^ j;
+                    if (l > i) {
+                        const bool sw = (i & k) == 0 ? pq_before(v[l], ix[l], v[i], ix[i])
+                                                     : pq_before(v[i], ix[i], v[l], ix[l]);
+                        if (sw) {
+                            const double tv = v[i];
+                            v[i] = v[l];
+                            v[l] = tv;
+                            const int ti = ix[i];
+                            ix[i] = ix[l];
+                            ix[l] = ti;
+                        }
+                    }
+                }
+        __syncwarp();  // the bit set's zeroing (other lanes) before lane 0 sets bits
+        for (int round = 0; round < top_k; round++) {
+            double bv = v[0];
+            int bi = ix[0];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (pq_before(ov, oi, bv, bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if (bi == 0x7fffffff) break;  // no non-empty cluster left
+            if (lane == 0) {
+                bw[bi >> 5] |= 1u << (bi & 31);
+                pairs += (unsigned long long)kc[bi];
+            }
+            // the lane whose head was taken moves its list up by one
+            if (ix[0] == bi) {
+#pragma unroll
+                for (int i = 0; i < 15; i++) {
+                    v[i] = v[i + 1];
+                    ix[i] = ix[i + 1];
+                }
+                v[15] = -INFINITY;
+                ix[15] = 0x7fffffff;
+            }
+        }
         __syncwarp();
-        // taken clusters get NaN, which no comparison below accepts
+        if (text_group && lane == 0) {
+            const int tg = nkh;  // the text-key group's id
+            bw[tg >> 5] |= 1u << (tg & 31);
+            pairs += (unsigned long long)kc[tg];
+        }
+    } else if (!dn) {
+        const double *srow = scores + ((size_t)h * nb + r) * kk_cap;
+        // empty clusters and (below) taken ones hold NaN, which no comparison accepts
+        const double qnan = __longlong_as_double(0x7ff8000000000000ll);
+        for (int b = lane; b < nkh; b += 32) sc[b] = kc[b] > 0 ? srow[b] : qnan;
+        __syncwarp();
         for (int round = 0; round < top_k; round++) {
             double best = -INFINITY;
             int bb = 0x7fffffff;
             for (int b = lane; b < nkh; b += 32) {
                 const double v = sc[b];
-                if (kc[b] > 0 && (v > best || (v == best && b < bb))) {
+                if (v > best || (v == best && b < bb)) {
                     best = v;
                     bb = b;
                 }
@@ -161,7 +248,7 @@ __global__ void __launch_bounds__(PQ_WARPS * 32) pq_topk_kernel(const double *__
             }
             if (bb == 0x7fffffff) break;  // no non-empty cluster left
             if (lane == 0) {
-                sc[bb] = __longlong_as_double(0x7ff8000000000000ll);
+                sc[bb] = qnan;
                 bw[bb >> 5] |= 1u << (bb & 31);
                 pairs += (unsigned long long)kc[bb];
             }
@@ -377,7 +464,7 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
                   double *scores, int batch, unsigned long long *head_pairs, cudaStream_t st) {
     const int nkmax = nk ? kk_cap : kk_fixed;
     const size_t smem_s = (size_t)(score_mode == 1 ? 3 : 2) * D * PQ_LD * sizeof(double);
-    const size_t per_warp = (size_t)kk_cap * sizeof(double) + (size_t)W * sizeof(uint32_t);
+    const size_t per_warp = pq_topk_region(kk_cap) + (size_t)W * sizeof(uint32_t);
     int nwarps = (int)((size_t)(200 * 1024) / per_warp);
     nwarps = nwarps < 1 ? 1 : (nwarps > PQ_WARPS ? PQ_WARPS : nwarps);
     const size_t smem_t = (size_t)nwarps * per_warp;
