@@ -106,6 +106,51 @@ def test_select_rows_and_attention_from_oracle_clusters(orc, name):
         attn_close(got[h], ref, f"{name}/h{h}/attention")
 
 
+# hand-made key clusters for the per-row argtopk: duplicated centroids (exact
+# score ties, broken towards the lower id), empty clusters (never chosen, also
+# when they duplicate a chosen one), and cluster counts on both sides of 512
+# (one sorted list of 16 per lane up to 512 clusters, the scan beyond)
+TIE_CASES = {
+    "ties-kk40": (300, 40, 6),
+    "ties-kk512": (600, 512, 5),
+    "ties-kk600": (700, 600, 9),
+}
+
+
+@pytest.mark.parametrize("name", list(TIE_CASES))
+def test_select_rows_ties_and_empty_clusters(orc, name):
+    n, kk, top_k = TIE_CASES[name]
+    w = W.small(W.WORKLOADS["wan21-n75600-h40-d128"], n, heads=1, seed=9, kq=4, kk=kk)
+    ctx = _ctx(w, dict(score_mode=0, top_k=top_k))
+    D = w.d
+    q, _, _ = stack_heads(w)
+    rng = np.random.default_rng(11)
+    cent = (0.3 * rng.standard_normal((kk, D))).astype(np.float32)
+    for a, b in ((5, 17), (20, 33), (3, 8), (1, kk - 1)):
+        cent[b] = cent[a]
+    count = rng.integers(1, 50, kk).astype(np.int32)
+    count[[2, 11, 30, 33]] = 0
+    kk_cap = ctx.kk_cap
+    Wd = (kk_cap + 31) // 32
+    k_cent = np.zeros((1, kk_cap, D), np.float32)
+    k_count = np.zeros((1, kk_cap), np.int32)
+    k_cent[0, :kk], k_count[0, :kk] = cent, count
+    sel, cnt = orc.select_per_query(q[0], cent, count, w.top_p, 0, top_k, None, None)
+    want = _bits(sel, cnt, Wd)
+    bits = ctx.ac_select_rows(to_dev(q, w.dtype), torch.from_numpy(k_count).cuda(),
+                              k_cent=torch.from_numpy(k_cent).cuda())
+    torch.cuda.synchronize()
+    assert ctx.get_status() == 0
+    got = bits.cpu().numpy().view(np.uint32)[0]
+    bad = np.nonzero((got != want).any(axis=1))[0]
+    assert len(bad) == 0, f"{name}: {len(bad)} rows with a different set, e.g. rows {bad[:5].tolist()}"
+    # the duplicated pairs tie exactly: wherever the higher id is chosen, so is the lower
+    for a, b in ((5, 17), (3, 8), (1, kk - 1)):
+        hi_on = ((got[:, b >> 5] >> np.uint32(b & 31)) & 1).astype(bool)
+        lo_on = ((got[:, a >> 5] >> np.uint32(a & 31)) & 1).astype(bool)
+        assert not np.any(hi_on & ~lo_on), f"{name}: tie between {a} and {b} broken upwards"
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_forward_per_query_end_to_end(orc, name):
     w, over = CASES[name]
