@@ -58,6 +58,8 @@ struct Bump {
 struct Ws {
     // clustering scratch
     size_t norm, U0, U1, passign, dist, rank, hist, cnt, off, perm, amb, ambc, cn2, cmax, seg, ms;
+    // the k-means rounds' clusters largest first (update launch order)
+    size_t uorder;
     // ac_forward internals
     size_t qa, ka, qc, kc, qcount, kcount, qmn, nq, nk, dq, dk, sel, selc;
     // attention
@@ -98,6 +100,7 @@ Ws layout(const ac_ctx *c) {
     w.hist = b.take(sort_hist_elems((int)H, (int)N, (int)capm) * 4);
     w.cnt = b.take(H * capm * 4);
     w.off = b.take(H * (capm + 1) * 4);
+    w.uorder = b.take(H * capm * 4);
     w.perm = b.take(HN * 4);
     w.amb = b.take(HN * 4);
     w.ambc = b.take(H * 4);
@@ -256,6 +259,7 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
     int32_t *perm = at<int32_t>(ws, w.perm), *off = at<int32_t>(ws, w.off);
     int32_t *rank = at<int32_t>(ws, w.rank), *hist = at<int32_t>(ws, w.hist);
     int32_t *cnt = at<int32_t>(ws, w.cnt);
+    int32_t *uorder = at<int32_t>(ws, w.uorder);
     float *cn2 = at<float>(ws, w.cn2), *cmax = at<float>(ws, w.cmax);
     int32_t *amb = at<int32_t>(ws, w.amb), *ambc = at<int32_t>(ws, w.ambc);
     int *status = c->d_status;
@@ -285,8 +289,8 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
             AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
             k_conv_check(H, N, seg, assign, prev, kst, it == 0 ? 1 : 0, st);
             k_conv_decide(H, seg, kst, it, st);
-            k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, cnt, off, perm, status, st);
-            k_update(x, dt, H, N, D, seg, kmax, perm, off, cap, norm, mode, cent, st);
+            k_sort(assign, nullptr, seg, H, N, N, cap, rank, hist, cnt, off, perm, status, st, uorder);
+            k_update(x, dt, H, N, D, seg, kmax, perm, off, cap, norm, mode, cent, st, uorder);
         }
         // the last pass for the heads still running; then all heads again
         AC_TRY(assign_step(c, w, ws, x, x, nullptr, seg, N, cent, cap, mode, assign, st));
@@ -343,8 +347,8 @@ ac_status run_cluster(ac_ctx *c, int mode, const void *x, const float *init, int
             AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
             k_conv_check(H, N, seg, pa, prev, kst, it == 0 ? 1 : 0, st);
             k_conv_decide(H, seg, kst, it, st);
-            k_sort(pa, U, seg, H, N, mnu, cap, rank, hist, cnt, off, perm, status, st);
-            k_update(x, dt, H, N, D, seg, mmt, perm, off, cap, norm, mode, cent, st);
+            k_sort(pa, U, seg, H, N, mnu, cap, rank, hist, cnt, off, perm, status, st, uorder);
+            k_update(x, dt, H, N, D, seg, mmt, perm, off, cap, norm, mode, cent, st, uorder);
         }
         AC_TRY(assign_step(c, w, ws, x, xu, U, seg, mnu, cent, cap, mode, pa, st));
         if (iters_t > 0) AC_CUDA(cudaMemcpyAsync(seg, seg_keep, sizeof(HeadSeg) * H, cudaMemcpyDeviceToDevice, st));

@@ -35,8 +35,10 @@ void k_assign_exact(const void *x, int dtype, int H, int N, int D, const int32_t
 void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
             int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
             double *dist, cudaStream_t st);
+// order (optional, from k_sort): the clusters are taken largest first
 void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg, int kmax, const int32_t *perm,
-              const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st);
+              const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st,
+              const int32_t *order = nullptr);
 void k_mean_norm(int H, int N, const HeadSeg *seg, const int32_t *perm, const int32_t *off, int cap,
                  const double *norm, float *mean_norm, cudaStream_t st);
 // Early stop of fixed-count k-means (ac_kmeans.cu): kst [H, 4] = {stopped,
@@ -55,9 +57,11 @@ int k_assign_tc(const void *xc, int H, int N, int D, const int32_t *rows, const 
 
 // ---- ac_sort.cu
 // Stable counting sort of positions 0..seg.nrows-1 by id (< seg.k): perm gets
-// rows[pos] (or pos), off [H, cap+1] the cluster offsets, cnt [H, cap] the sizes.
+// rows[pos] (or pos), off [H, cap+1] the cluster offsets, cnt [H, cap] the sizes;
+// order [H, cap] (optional) the non-empty clusters by size class, largest first, then -1.
 void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, int N, int nrows_max, int cap,
-            int32_t *rank, int32_t *hist, int32_t *cnt, int32_t *off, int32_t *perm, int *status, cudaStream_t st);
+            int32_t *rank, int32_t *hist, int32_t *cnt, int32_t *off, int32_t *perm, int *status, cudaStream_t st,
+            int32_t *order = nullptr);
 size_t sort_hist_elems(int H, int N, int cap);
 void k_gather_rows(const void *src, void *dst, const int32_t *perm, int H, int N, int row_bytes, cudaStream_t st);
 

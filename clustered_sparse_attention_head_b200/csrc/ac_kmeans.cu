@@ -358,7 +358,8 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
                                                              const int32_t *__restrict__ perm,
                                                              const int32_t *__restrict__ off, int cap,
                                                              const double *__restrict__ norm, int mode,
-                                                             float *__restrict__ cent) {
+                                                             float *__restrict__ cent,
+                                                             const int32_t *__restrict__ order) {
     constexpr int ROW_BYTES = D * (int)sizeof(T);
     constexpr int R = UPD_CHUNK_BYTES / ROW_BYTES;   // rows per chunk
     constexpr int PIECES = ROW_BYTES / 16;           // 16-byte pieces per row
@@ -370,9 +371,11 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
     double *rcp = nrm + UPD_STAGES * R;                                                  // [S][R]
     __shared__ double ssum[D];
     __shared__ double snr;
-    const int h = blockIdx.y, j = blockIdx.x, tid = threadIdx.x;
+    // grid (head, rank): with an order the rank-th largest cluster of the head
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const int j = order ? order[(size_t)h * cap + blockIdx.y] : (int)blockIdx.y;
     const HeadSeg s = seg[h];
-    if (s.nrows <= 0 || j >= s.k) return;
+    if (s.nrows <= 0 || j < 0 || j >= s.k) return;
     const int32_t *o = off + (size_t)h * (cap + 1);
     const int b = o[j], e = o[j + 1];
     if (e <= b) return;
@@ -583,15 +586,17 @@ void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, 
 }
 
 void k_update(const void *x, int dtype, int H, int N, int D, const HeadSeg *seg, int kmax, const int32_t *perm,
-              const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st) {
-    dim3 g(kmax, H);
+              const int32_t *off, int cap, const double *norm, int mode, float *cent, cudaStream_t st,
+              const int32_t *order) {
+    // blocks start in launch order, x fastest: every head's rank-0 cluster, then rank 1, ...
+    dim3 g(H, kmax);
     // staged rows (8 KB chunks, three stages) plus the rows' norms and reciprocals
 #define AC_UPD(T, DD)                                                                                             \
     do {                                                                                                          \
         constexpr int R_ = UPD_CHUNK_BYTES / (DD * (int)sizeof(T));                                               \
         constexpr int SM_ = UPD_STAGES * (UPD_CHUNK_BYTES + 2 * R_ * 8);                                          \
         cudaFuncSetAttribute(update2_kernel<T, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM_);             \
-        update2_kernel<T, DD><<<g, UPD_THREADS, SM_, st>>>((const T *)x, N, seg, perm, off, cap, norm, mode, cent); \
+        update2_kernel<T, DD><<<g, UPD_THREADS, SM_, st>>>((const T *)x, N, seg, perm, off, cap, norm, mode, cent, order); \
     } while (0)
     if (dtype == DT_BF16) {
         if (D == 64) AC_UPD(__nv_bfloat16, 64);

@@ -103,8 +103,20 @@ __global__ void scan_tiles_kernel(const HeadSeg *__restrict__ seg, int cap, int 
     cnt[(size_t)h * cap + j] = run;
 }
 
-// Per head: exclusive scan of cluster sizes -> offsets [cap + 1].
-__global__ void scan_clusters_kernel(const int32_t *__restrict__ cnt, int cap, int32_t *__restrict__ off) {
+// Size class of a non-empty cluster: 4 per octave (the exponent and the two
+// bits below the leading one), 0..127
+__device__ __forceinline__ int size_class(int v) {
+    const int e = 31 - __clz(v);
+    const int m = e >= 2 ? ((v >> (e - 2)) & 3) : 0;
+    return min(4 * e + m, 127);
+}
+
+// Per head: exclusive scan of cluster sizes -> offsets [cap + 1].  With
+// `order`, also the non-empty clusters by size class, largest first (-1 after
+// them): a kernel with one CTA per cluster launched over (head, rank) then
+// starts every head's largest clusters first.
+__global__ void scan_clusters_kernel(const int32_t *__restrict__ cnt, int cap, int32_t *__restrict__ off,
+                                     int32_t *__restrict__ order) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     int h = blockIdx.x;
@@ -140,6 +152,28 @@ __global__ void scan_clusters_kernel(const int32_t *__restrict__ cnt, int cap, i
         __syncthreads();
     }
     if (threadIdx.x == 0) o[cap] = carry;
+    if (!order) return;
+    __shared__ int32_t cls[128];
+    __shared__ int32_t nonempty;
+    int32_t *ord = order + (size_t)h * cap;
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) cls[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < cap; j += blockDim.x)
+        if (c[j] > 0) atomicAdd(&cls[size_class(c[j])], 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int i = 127; i >= 0; i--) {
+            const int t = cls[i];
+            cls[i] = run;
+            run += t;
+        }
+        nonempty = run;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < cap; j += blockDim.x)
+        if (c[j] > 0) ord[atomicAdd(&cls[size_class(c[j])], 1)] = j;
+    for (int p = nonempty + threadIdx.x; p < cap; p += blockDim.x) ord[p] = -1;
 }
 
 __global__ void scatter_kernel(const int32_t *__restrict__ ids, const int32_t *__restrict__ rows,
@@ -164,7 +198,8 @@ size_t sort_hist_elems(int H, int N, int cap) {
 }
 
 void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, int N, int nrows_max, int cap,
-            int32_t *rank, int32_t *hist, int32_t *cnt, int32_t *off, int32_t *perm, int *status, cudaStream_t st) {
+            int32_t *rank, int32_t *hist, int32_t *cnt, int32_t *off, int32_t *perm, int *status, cudaStream_t st,
+            int32_t *order) {
     int ntiles_max = (N + SORT_TILE - 1) / SORT_TILE;
     int nt = (nrows_max + SORT_TILE - 1) / SORT_TILE;
     size_t smem = (size_t)4 * cap * sizeof(int32_t);
@@ -176,7 +211,7 @@ void k_sort(const int32_t *ids, const int32_t *rows, const HeadSeg *seg, int H, 
     }
     dim3 g2((cap + 127) / 128, H);
     scan_tiles_kernel<<<g2, 128, 0, st>>>(seg, cap, ntiles_max, hist, cnt); note_launch();
-    scan_clusters_kernel<<<H, 1024, 0, st>>>(cnt, cap, off); note_launch();
+    scan_clusters_kernel<<<H, 1024, 0, st>>>(cnt, cap, off, order); note_launch();
     if (nrows_max > 0) {
         dim3 g3((nrows_max + 255) / 256, H);
         scatter_kernel<<<g3, 256, 0, st>>>(ids, rows, seg, N, cap, ntiles_max, rank, hist, off, perm); note_launch();
