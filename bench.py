@@ -421,6 +421,12 @@ def main():
             "flops_per_launch": flops, "flops_rule": "4 * d * computed (query, key) pairs"}
 
     extra = {}
+    if rank == 0 and not a.no_per_config and world == 1 and cfg.text_keys == 0:
+        # the same call replayed from a CUDA graph (fixed counts only)
+        gms = graph_ms(w, q, k, v, out, dev, stream, 3, flush)
+        if gms is not None:
+            extra["graph"] = {"ms_per_call": gms, "calls_per_s": 1e3 / gms,
+                              "how": "AdaCluster.capture_forward: one captured ac_forward replayed on the same buffers"}
     if rank == 0 and not a.no_per_config and world == 1:
         # every workload gets its own context
         extra["top_p_sweep"] = top_p_sweep(w, q, k, v, out, dev, stream, a.per_config_calls, peak,
@@ -486,7 +492,25 @@ def sdpa_ms(q, k, v, stream, flush, calls=3):
     return time_calls(lambda: F.scaled_dot_product_attention(qd, kd, vd), calls, stream, flush)
 
 
-def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0, over=None):
+def graph_ms(w, q, k, v, out, dev, stream, calls, flush):
+    """ms per call of the same ac_forward replayed from a CUDA graph
+    (AdaCluster.capture_forward: the call's launches issued at once), or None
+    for adaptive counts, whose call reads each Algorithm-1 stage on the host."""
+    if w.adaptive_q or w.adaptive_k:
+        return None
+    from clustered_sparse_attention_head_b200.api import AdaCluster, Config
+    ac = AdaCluster(Config.from_workload(w), device=dev)
+    graph, _ = ac.capture_forward(q, k, v, out=out)
+    ms = time_calls(graph.replay, calls, stream, flush)
+    status = ac.get_status()
+    del graph
+    ac.close()
+    if status != 0:
+        raise RuntimeError(f"{w.name}: device status {status} (graph replay)")
+    return ms
+
+
+def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0, over=None, graph=False):
     """One workload through ac_forward: ms per call (CUDA events, L2 flushed
     first when an input tensor fits in L2), the stage breakdown, computed pairs
     and the attention kernel's rate against the peak."""
@@ -523,6 +547,11 @@ def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0, over=None):
          "tflops_effective_attn": flops / (attn * 1e-3) / 1e12 if attn > 0 else None,
          "roofline_frac_attn": flops / (attn * 1e-3) / 1e12 / peak if attn > 0 else None,
          "l2": config_of(w, 1)["l2"]}
+    if graph and not over and not text_keys:
+        gms = graph_ms(w, q, k, v, out, dev, stream, calls, flush)
+        if gms is not None:
+            r["graph_ms_per_call"] = gms
+            r["graph_calls_per_s"] = 1e3 / gms
     return r, flush
 
 
@@ -569,7 +598,7 @@ def per_config(dev, stream, calls, peak):
         q, k, v = (torch.from_numpy(np.stack([getattr(h, a) for h in hs])).to(dev).to(tdt) for a in "qkv")
         del hs
         out = torch.empty_like(q)
-        r, flush = measure(w, q, k, v, out, dev, stream, calls, peak)
+        r, flush = measure(w, q, k, v, out, dev, stream, calls, peak, graph=True)
         d = sdpa_ms(q, k, v, stream, flush)
         r["sdpa_ms"] = d
         r["sdpa_tflops"] = w.dense_flops() / (d * 1e-3) / 1e12

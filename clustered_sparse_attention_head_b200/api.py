@@ -203,6 +203,33 @@ class AdaCluster:
             return out, {f: getattr(st, f) for f, _ in _abi.ac_stats._fields_}
         return out
 
+    def capture_forward(self, q, k, v, out=None):
+        """One ac_forward call (q, k, v -> out) captured into a CUDA graph, for
+        loops that call it again and again on the same buffers: replaying the
+        graph issues the call's ~250 kernel launches at once, which is what
+        small workloads are bound by.  Returns (graph, out); graph.replay()
+        recomputes out from the buffers' current contents.  The launches keep
+        the buffers' addresses, so new inputs are copied into q, k and v.  Only
+        for fixed cluster counts: Algorithm 1 (adaptive_q / adaptive_k) reads
+        each stage's counts on the host, and neither stats nor profiling can
+        run inside a graph."""
+        if self.cfg.adaptive_q or self.cfg.adaptive_k:
+            raise ValueError("capture_forward: Algorithm 1 (adaptive counts) synchronises with the host per stage")
+        if self.cfg.flags & _abi.AC_FLAG_PROFILE:
+            raise ValueError("capture_forward: profiling records host-side timings")
+        H, N, D = self.cfg.heads, self.cfg.n, self.cfg.d
+        if out is None:
+            out = torch.empty(H, N, D, dtype=self.cfg.torch_dtype, device=self.device)
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            self.ac_forward(q, k, v, out=out)  # first-call work (attributes, tensor maps) outside the graph
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.ac_forward(q, k, v, out=out)
+        return graph, out
+
     def selftest_wait(self, seconds=0.2, stream=None):
         """Runs the bounded-wait diagnostic (a wait that must expire); the next
         get_status() returns AC_ERR_TIMEOUT."""
