@@ -275,6 +275,14 @@ def main():
     v_h = torch.from_numpy(np.stack([h.v for h in hs])).to(tdt)
     del hs
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    # two contexts: `ac_t` with the default flags is the one timed (the library
+    # replays its cached CUDA graph of the call when a call repeats the buffers);
+    # `ac` records per-stage events, which keeps it launch by launch, and gives
+    # the stage breakdown, the statistics and a launch-by-launch timing
+    cfg = Config.from_workload(w)
+    if a.text_keys:
+        cfg.text_keys = w.text
+    ac_t = AdaCluster(cfg, device=dev)
     cfg = Config.from_workload(w)
     cfg.flags = _abi.AC_FLAG_PROFILE
     if a.text_keys:
@@ -289,14 +297,17 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # warm-up, then one call with statistics (pairs, dense heads)
+    # warm-up (both contexts), then one call with statistics (pairs, dense heads)
     for _ in range(max(a.warmup, 3) - 1):
+        ac_t.ac_forward(q, k, v, out=out)
         ac.ac_forward(q, k, v, out=out)
     _, st = ac.ac_forward(q, k, v, out=out, stats=True)
-    status = ac.get_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
+    for c_ in (ac, ac_t):
+        status = c_.get_status()
+        if status != 0:
+            raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
     ac.profile_read()
+    ac_t.profile_read()
 
     # timed region: inputs larger than L2 need no flush; smaller ones get an L2
     # flush before every call, outside the events that time the call
@@ -304,9 +315,16 @@ def main():
     flush = None if tensor_bytes(w) > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     barrier()
     sampler.start()
-    ms = time_calls(lambda: ac.ac_forward(q, k, v, out=out), a.steps, stream, flush)
+    ms = time_calls(lambda: ac_t.ac_forward(q, k, v, out=out), a.steps, stream, flush)
     barrier()
     clocks = sampler.stop()
+    prof_t = ac_t.profile_read()
+    status = ac_t.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {_abi.status_string(status)}")
+    # the same calls launch by launch, with per-stage events
+    ms_lbl = time_calls(lambda: ac.ac_forward(q, k, v, out=out), a.steps, stream, flush)
+    t_lbl = max_over_ranks(ms_lbl, world, dev)
     prof = ac.profile_read()
     status = ac.get_status()
     if status != 0:
@@ -346,7 +364,7 @@ def main():
                 stream.wait_event(in_ready[b])
                 if i >= 2:
                     stream.wait_event(out_free[b])
-                ac.ac_forward(qs[b], ks[b], vs[b], out=outs[b], stream=stream)
+                ac_t.ac_forward(qs[b], ks[b], vs[b], out=outs[b], stream=stream)
                 in_free[b].record(stream)
                 out_ready[b].record(stream)
                 with torch.cuda.stream(d2h):
@@ -355,7 +373,7 @@ def main():
                     out_free[b].record(d2h)
             stream.wait_stream(d2h)
 
-        run_steps(2)
+        run_steps(4)  # each buffer set twice: both graphs captured before the timed steps
         torch.cuda.synchronize(dev)
         barrier()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -394,7 +412,7 @@ def main():
         dense["own_dense"] = {"impl": "ac_sparse_attn with every head dense (gathered copy + attn3_kernel)",
                               "ms": oms, "tflops": w.dense_flops() / (oms * 1e-3) / 1e12}
 
-    launches_timed = int(prof["launches"]) if e2e is None else launches_per_call(ac, q, k, v, out) * a.steps
+    launches_timed = int(prof_t["launches"]) if e2e is None else launches_per_call(ac_t, q, k, v, out) * a.steps
     denoise = None
     if rank == 0 and a.denoise_steps > 0:
         denoise = denoise_steps(ac, q, k, v, out, a.denoise_steps, a.drift, stream)
@@ -421,12 +439,11 @@ def main():
             "flops_per_launch": flops, "flops_rule": "4 * d * computed (query, key) pairs"}
 
     extra = {}
-    if rank == 0 and not a.no_per_config and world == 1 and cfg.text_keys == 0:
-        # the same call replayed from a CUDA graph (fixed counts only)
-        gms = graph_ms(w, q, k, v, out, dev, stream, 3, flush)
-        if gms is not None:
-            extra["graph"] = {"ms_per_call": gms, "calls_per_s": 1e3 / gms,
-                              "how": "AdaCluster.capture_forward: one captured ac_forward replayed on the same buffers"}
+    if rank == 0:
+        extra["launch_by_launch"] = {
+            "ms_per_call": t_lbl, "calls_per_s": calls_per_second(t_lbl, world),
+            "how": "the same calls with AC_FLAG_PROFILE (per-stage events), which ac_forward never replays "
+                   "from its cached CUDA graph"}
     if rank == 0 and not a.no_per_config and world == 1:
         # every workload gets its own context
         extra["top_p_sweep"] = top_p_sweep(w, q, k, v, out, dev, stream, a.per_config_calls, peak,
@@ -434,6 +451,7 @@ def main():
         extra["select_modes"] = select_modes(w, q, k, v, out, dev, stream, a.per_config_calls, peak)
         del q, k, v, out
         ac.close()
+        ac_t.close()
         torch.cuda.empty_cache()
         extra["per_config"] = per_config(dev, stream, a.per_config_calls, peak)
 
@@ -455,6 +473,7 @@ def main():
             line["denoise_steps"] = denoise
         print(json.dumps(line), flush=True)
     ac.close()
+    ac_t.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -492,66 +511,55 @@ def sdpa_ms(q, k, v, stream, flush, calls=3):
     return time_calls(lambda: F.scaled_dot_product_attention(qd, kd, vd), calls, stream, flush)
 
 
-def graph_ms(w, q, k, v, out, dev, stream, calls, flush):
-    """ms per call of the same ac_forward replayed from a CUDA graph
-    (AdaCluster.capture_forward: the call's launches issued at once), or None
-    for adaptive counts, whose call reads each Algorithm-1 stage on the host."""
-    if w.adaptive_q or w.adaptive_k:
-        return None
-    from clustered_sparse_attention_head_b200.api import AdaCluster, Config
-    ac = AdaCluster(Config.from_workload(w), device=dev)
-    graph, _ = ac.capture_forward(q, k, v, out=out)
-    ms = time_calls(graph.replay, calls, stream, flush)
-    status = ac.get_status()
-    del graph
-    ac.close()
-    if status != 0:
-        raise RuntimeError(f"{w.name}: device status {status} (graph replay)")
-    return ms
-
-
-def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0, over=None, graph=False):
+def measure(w, q, k, v, out, dev, stream, calls, peak, text_keys=0, over=None):
     """One workload through ac_forward: ms per call (CUDA events, L2 flushed
-    first when an input tensor fits in L2), the stage breakdown, computed pairs
-    and the attention kernel's rate against the peak."""
+    first when an input tensor fits in L2) with the default flags (so a repeated
+    call replays the library's cached CUDA graph where the counts are fixed),
+    the same launch by launch with per-stage events (the stage breakdown), the
+    computed pairs and the attention kernel's rate against the peak."""
     import torch
     from clustered_sparse_attention_head_b200 import _abi
     from clustered_sparse_attention_head_b200.api import AdaCluster, Config
-    cfg = Config.from_workload(w)
-    cfg.flags = _abi.AC_FLAG_PROFILE
-    cfg.text_keys = text_keys
-    for key, val in (over or {}).items():
-        setattr(cfg, key, val)
-    ac = AdaCluster(cfg, device=dev)
+
+    def make(flags):
+        cfg = Config.from_workload(w)
+        cfg.flags = flags
+        cfg.text_keys = text_keys
+        for key, val in (over or {}).items():
+            setattr(cfg, key, val)
+        return AdaCluster(cfg, device=dev)
+    ac_t, ac = make(0), make(_abi.AC_FLAG_PROFILE)
     flush = None if tensor_bytes(w) > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(2):  # the second call on these buffers captures the library's graph
+        ac_t.ac_forward(q, k, v, out=out)
     ac.ac_forward(q, k, v, out=out)
     _, st = ac.ac_forward(q, k, v, out=out, stats=True)
-    if ac.get_status() != 0:
-        raise RuntimeError(f"{w.name}: device status {ac.get_status()}")
+    if ac.get_status() != 0 or ac_t.get_status() != 0:
+        raise RuntimeError(f"{w.name}: device status {ac.get_status()} / {ac_t.get_status()}")
     ac.profile_read()
-    ms = time_calls(lambda: ac.ac_forward(q, k, v, out=out), calls, stream, flush)
+    ac_t.profile_read()
+    ms = time_calls(lambda: ac_t.ac_forward(q, k, v, out=out), calls, stream, flush)
+    launches = ac_t.profile_read()["launches"]
+    ms_lbl = time_calls(lambda: ac.ac_forward(q, k, v, out=out), calls, stream, flush)
     prof = ac.profile_read()
-    status = ac.get_status()
+    status = max(ac.get_status(), ac_t.get_status())
     ac.close()
+    ac_t.close()
     if status != 0:
         raise RuntimeError(f"{w.name}: device status {status}")
     flops = 4.0 * w.d * st["pairs"]
     attn = prof["ms_attn_kernel"]
-    r = {"ms_per_call": ms, "calls_per_s": 1e3 / ms, "pairs": st["pairs"], "pairs_computed": st["pairs_computed"],
+    r = {"ms_per_call": ms, "calls_per_s": 1e3 / ms, "ms_per_call_launch_by_launch": ms_lbl,
+         "pairs": st["pairs"], "pairs_computed": st["pairs_computed"],
          "density": st["pairs"] / (w.heads * float(w.n) ** 2), "dense_heads": st["dense_heads"],
          "stages_q": st["max_stages_q"], "stages_k": st["max_stages_k"],
          "stage_ms": {k2: prof[k2] for k2 in ("ms_cluster_q", "ms_cluster_k", "ms_select", "ms_prep",
                                               "ms_attn_kernel", "ms_total")},
-         "launches_per_call": int(prof["launches"]) // max(calls, 1),
+         "launches_per_call": int(launches) // max(calls, 1),
          "tflops_effective_call": flops / (ms * 1e-3) / 1e12,
          "tflops_effective_attn": flops / (attn * 1e-3) / 1e12 if attn > 0 else None,
          "roofline_frac_attn": flops / (attn * 1e-3) / 1e12 / peak if attn > 0 else None,
          "l2": config_of(w, 1)["l2"]}
-    if graph and not over and not text_keys:
-        gms = graph_ms(w, q, k, v, out, dev, stream, calls, flush)
-        if gms is not None:
-            r["graph_ms_per_call"] = gms
-            r["graph_calls_per_s"] = 1e3 / gms
     return r, flush
 
 
@@ -598,7 +606,7 @@ def per_config(dev, stream, calls, peak):
         q, k, v = (torch.from_numpy(np.stack([getattr(h, a) for h in hs])).to(dev).to(tdt) for a in "qkv")
         del hs
         out = torch.empty_like(q)
-        r, flush = measure(w, q, k, v, out, dev, stream, calls, peak, graph=True)
+        r, flush = measure(w, q, k, v, out, dev, stream, calls, peak)
         d = sdpa_ms(q, k, v, stream, flush)
         r["sdpa_ms"] = d
         r["sdpa_tflops"] = w.dense_flops() / (d * 1e-3) / 1e12

@@ -18,7 +18,7 @@ AC_OK, AC_ERR_INVALID_ARG, AC_ERR_UNSUPPORTED, AC_ERR_CUDA = 0, 1, 2, 3
 AC_ERR_WORKSPACE, AC_ERR_TIMEOUT, AC_ERR_NONFINITE, AC_ERR_CAPACITY = 4, 5, 6, 7
 AC_F32, AC_BF16 = 0, 1
 AC_TAU_ABS, AC_TAU_MEAN_X, AC_TAU_MEDIAN_RADIUS_X = 0, 1, 2
-AC_FLAG_WARM_START, AC_FLAG_CHECK_FINITE, AC_FLAG_PROFILE = 1, 2, 4
+AC_FLAG_WARM_START, AC_FLAG_CHECK_FINITE, AC_FLAG_PROFILE, AC_FLAG_NO_GRAPH = 1, 2, 4, 8
 AC_SCORE_CENTROID, AC_SCORE_QUEST = 0, 1
 
 # every entry point declared in include/adacluster.h

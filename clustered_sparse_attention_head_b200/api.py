@@ -204,10 +204,11 @@ class AdaCluster:
         return out
 
     def capture_forward(self, q, k, v, out=None):
-        """One ac_forward call (q, k, v -> out) captured into a CUDA graph, for
-        loops that call it again and again on the same buffers: replaying the
-        graph issues the call's ~250 kernel launches at once, which is what
-        small workloads are bound by.  Returns (graph, out); graph.replay()
+        """One ac_forward call (q, k, v -> out) captured into a CUDA graph that
+        the caller owns (to replay it inside a larger graph of its own, say).
+        ac_forward itself already replays a cached graph of its launches when a
+        call repeats the buffers of an earlier one (include/adacluster.h), so a
+        plain loop needs none of this.  Returns (graph, out); graph.replay()
         recomputes out from the buffers' current contents.  The launches keep
         the buffers' addresses, so new inputs are copied into q, k and v.  Only
         for fixed cluster counts: Algorithm 1 (adaptive_q / adaptive_k) reads

@@ -23,6 +23,7 @@ void wait_selftest_launch(uint64_t limit_ns, int *status, cudaStream_t st);
 static std::atomic<long long> g_launches{0};
 namespace ac {
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+void note_launches(long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 long long launches_total() { return g_launches.load(std::memory_order_relaxed); }
 }  // namespace ac
 
@@ -42,6 +43,17 @@ struct ac_ctx {
     cudaEvent_t *prof;     // [PROF_RING][PROF_EV]
     long long prof_n;      // calls recorded since the last read
     long long launch_base;
+    // ac_forward's captured launch sequences, by the call's buffers
+    struct GraphSlot {
+        const void *key[7];
+        size_t ws_bytes;
+        cudaGraphExec_t exec;  // null: seen once, not captured yet
+        long long launches;
+        bool used;
+    } graphs[4];
+    int graph_next;
+    bool graph_off;  // a capture failed: run launch by launch from then on
+    cudaStream_t cap_stream;  // captures calls made on the legacy default stream, which cannot capture
 };
 
 // ------------------------------------------------------------ workspace
@@ -566,6 +578,9 @@ ac_status ac_create(const ac_config *cfg, ac_ctx **out) {
 
 void ac_destroy(ac_ctx *c) {
     if (!c) return;
+    for (auto &gs : c->graphs)
+        if (gs.exec) cudaGraphExecDestroy(gs.exec);
+    if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
     if (c->d_status) cudaFree(c->d_status);
     if (c->d_info) cudaFree(c->d_info);
     if (c->h_info) cudaFreeHost(c->h_info);
@@ -905,7 +920,71 @@ ac_status ac_forward(ac_ctx *c, const void *q, const void *k, const void *v, flo
     f.k_init = (warm && k_cent_io) ? k_cent_io : nullptr;
     f.q_cent = q_cent_io;
     f.k_cent = k_cent_io;
-    return forward_impl(c, q, k, v, f, out, stats, ws, (cudaStream_t)stream);
+    const cudaStream_t st = (cudaStream_t)stream;
+    const bool graphable = !stats && !(g.flags & (AC_FLAG_PROFILE | AC_FLAG_NO_GRAPH)) && !g.adaptive_q &&
+                           !g.adaptive_k && !c->graph_off;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (!graphable || cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+        return forward_impl(c, q, k, v, f, out, stats, ws, st);
+    // a call on the same buffers as a captured one replays it; buffers seen
+    // once before are captured now; new buffers are only noted (a call that
+    // never repeats its buffers pays no capture)
+    const void *key[7] = {q, k, v, q_cent_io, k_cent_io, out, ws};
+    ac_ctx::GraphSlot *hit = nullptr;
+    for (auto &gs : c->graphs)
+        if (gs.used && gs.ws_bytes == ws_bytes && memcmp(gs.key, key, sizeof(key)) == 0) hit = &gs;
+    if (hit && hit->exec) {
+        AC_CUDA(cudaGraphLaunch(hit->exec, st));
+        note_launches(hit->launches);
+        return AC_OK;
+    }
+    if (!hit) {
+        auto &slot = c->graphs[c->graph_next];
+        c->graph_next = (c->graph_next + 1) % 4;
+        if (slot.exec) cudaGraphExecDestroy(slot.exec);
+        memcpy(slot.key, key, sizeof(key));
+        slot.ws_bytes = ws_bytes;
+        slot.exec = nullptr;
+        slot.used = true;
+        return forward_impl(c, q, k, v, f, out, stats, ws, st);
+    }
+    // capture this call's launches (nothing runs during capture), then launch the
+    // graph on the caller's stream, which orders it like the launches it holds.
+    // The legacy default stream cannot capture: the context's own stream does.
+    cudaStream_t cap = st;
+    if (st == nullptr || st == cudaStreamLegacy) {
+        if (!c->cap_stream && cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+            cudaGetLastError();
+            c->cap_stream = nullptr;
+            c->graph_off = true;
+            return forward_impl(c, q, k, v, f, out, stats, ws, st);
+        }
+        cap = c->cap_stream;
+    }
+    const long long l0 = launches_total();
+    if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        cudaGetLastError();
+        c->graph_off = true;
+        return forward_impl(c, q, k, v, f, out, stats, ws, st);
+    }
+    const ac_status s2 = forward_impl(c, q, k, v, f, out, stats, ws, cap);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(cap, &graph);
+    const long long nl = launches_total() - l0;
+    cudaGraphExec_t exec = nullptr;
+    if (s2 == AC_OK && e == cudaSuccess && graph && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess)
+        exec = nullptr;
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    if (s2 != AC_OK) return s2;  // the argument errors a plain call returns, before any launch
+    if (!exec) {
+        c->graph_off = true;
+        return forward_impl(c, q, k, v, f, out, stats, ws, st);
+    }
+    hit->exec = exec;
+    hit->launches = nl;
+    AC_CUDA(cudaGraphLaunch(exec, st));
+    return AC_OK;
 }
 
 ac_status ac_step_state_size(const ac_ctx *c, size_t *bytes) {

@@ -93,6 +93,7 @@ typedef enum { AC_SCORE_CENTROID = 0, AC_SCORE_QUEST = 1 } ac_score_mode;
 #define AC_FLAG_CHECK_FINITE 2u  /* scan inputs for NaN/Inf (AC_ERR_NONFINITE)        */
 #define AC_FLAG_PROFILE 4u       /* ac_forward records per-stage CUDA events (no sync);
                                     read them with ac_profile_read                     */
+#define AC_FLAG_NO_GRAPH 8u      /* ac_forward: never replay its cached CUDA graphs    */
 
 typedef struct {
     int heads, n, d;        /* H, N, d (d in {64, 128}); batch is folded into heads   */
@@ -296,7 +297,15 @@ AC_API ac_status ac_sparse_attn(ac_ctx *ctx, const void *q, const void *k, const
  * with AC_FLAG_WARM_START they seed k-means (§3.2.2 "Efficient
  * initialization"); when non-NULL they receive the final centroids.
  * Adaptive clustering reads one int per head back to the host per stage; the
- * fixed-count path never synchronises unless `stats` is non-NULL.          */
+ * fixed-count path never synchronises unless `stats` is non-NULL.
+ * Graph replay: a fixed-count call without stats, AC_FLAG_PROFILE or
+ * AC_FLAG_NO_GRAPH, on a stream that is not being captured, whose q, k, v,
+ * q_cent_io, k_cent_io, out and workspace repeat those of an earlier call, is
+ * captured into a CUDA graph (the call's ~250 launches) on that second call
+ * and replayed on every later one; the replay reads the buffers' current
+ * contents.  Four buffer sets are remembered per context (ac_destroy releases
+ * their graphs).  If capture fails the call runs launch by launch and the
+ * context stops capturing.                                                */
 AC_API ac_status ac_forward(ac_ctx *ctx, const void *q, const void *k, const void *v, float *q_cent_io,
                      float *k_cent_io, void *out, ac_stats *stats, void *ws, size_t ws_bytes,
                      void *stream);

@@ -32,6 +32,16 @@ def test_header_declares_the_boundary():
         assert n in names
 
 
+def test_binding_constants_match_the_header():
+    import re
+    from clustered_sparse_attention_head_b200 import _abi
+    hdr = open(os.path.join(ROOT, "include", "adacluster.h")).read()
+    flags = dict(re.findall(r"#define (AC_FLAG_\w+) (\d+)u", hdr))
+    assert set(flags) == {n for n in dir(_abi) if n.startswith("AC_FLAG_")}
+    for name, val in flags.items():
+        assert getattr(_abi, name) == int(val), name
+
+
 def test_every_declared_symbol_is_exported(lib):
     from clustered_sparse_attention_head_b200 import _abi
     names = declared()

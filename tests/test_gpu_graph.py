@@ -1,4 +1,6 @@
-"""ac_forward replayed from a CUDA graph (AdaCluster.capture_forward) on the GPU.
+"""ac_forward replayed from CUDA graphs on the GPU: the library's own cache (a
+fixed-count call on the same buffers as an earlier one replays that call's
+captured launches) and AdaCluster.capture_forward (a graph the caller owns).
 
   * a replay gives the output of a plain ac_forward call bit for bit (bf16 and
     fp32 inputs; every kernel of the path is deterministic, the dynamic item
@@ -7,7 +9,10 @@
     the plain call's output on those values (the graph holds the buffers'
     addresses, not their contents);
   * configurations whose call reads results on the host (Algorithm 1's
-    adaptive counts, profiling) are refused."""
+    adaptive counts, profiling) are refused;
+  * the library's cache: repeated calls, calls on new contents of the same
+    buffers and calls that alternate two buffer sets give, bit for bit, what a
+    context with AC_FLAG_NO_GRAPH (every call launch by launch) gives."""
 import numpy as np
 import pytest
 
@@ -85,3 +90,53 @@ def test_capture_refuses_host_reads():
         ctx = AdaCluster(cfg)
         with pytest.raises(ValueError):
             ctx.capture_forward(q, k, v)
+
+
+def _ctx_flags(w, flags):
+    from clustered_sparse_attention_head_b200.api import AdaCluster, Config
+    cfg = Config.from_workload(w)
+    cfg.flags = flags
+    return AdaCluster(cfg)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_library_graph_cache_equals_launch_by_launch(name):
+    from dataclasses import replace
+    from clustered_sparse_attention_head_b200 import _abi
+    w = CASES[name]
+    ctx, ref = _ctx_flags(w, 0), _ctx_flags(w, _abi.AC_FLAG_NO_GRAPH)
+    sets = [_inputs(w), _inputs(replace(w, seed=w.seed + 7))]
+    outs = [torch.empty_like(sets[0][0]), torch.empty_like(sets[0][0])]
+    want = [ref.ac_forward(*sets[i]).clone() for i in range(2)]
+    for rep in range(3):  # first call captures, later ones replay; two buffer sets alternate
+        for i in range(2):
+            outs[i].zero_()
+            ctx.ac_forward(*sets[i], out=outs[i])
+            torch.cuda.synchronize()
+            assert ctx.get_status() == 0
+            assert torch.equal(outs[i], want[i]), f"{name}: call {rep}/{i} differs"
+    # new contents in the first buffer set: the replay reads them
+    q2, k2, v2 = _inputs(replace(w, seed=w.seed + 13))
+    for dst, src in zip(sets[0], (q2, k2, v2)):
+        dst.copy_(src)
+    ctx.ac_forward(*sets[0], out=outs[0])
+    want2 = ref.ac_forward(q2, k2, v2)
+    torch.cuda.synchronize()
+    assert ctx.get_status() == 0 and ref.get_status() == 0
+    assert torch.equal(outs[0], want2), f"{name}: replay on new contents differs"
+    # and the calls do replay: one graph launch costs the host far less than
+    # the call's ~250 separate launches
+    import time
+
+    def host_s(c):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(10):
+            c.ac_forward(*sets[1], out=outs[1])
+        t1 = time.perf_counter()
+        torch.cuda.synchronize()
+        return t1 - t0
+    t_graph, t_plain = host_s(ctx), host_s(ref)
+    print(f"{name}: host time per call {1e6 * t_graph / 10:.0f} us replayed, {1e6 * t_plain / 10:.0f} us launch by launch")
+    assert t_graph < 0.5 * t_plain, f"{name}: the calls were not replayed"
+
