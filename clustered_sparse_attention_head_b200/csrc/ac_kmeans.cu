@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(256) assign_exact_kernel(
     const T *__restrict__ x, int N, const int32_t *__restrict__ rows, const HeadSeg *__restrict__ seg,
     const float *__restrict__ cent, int cap, const double *__restrict__ norm, int mode,
     const int32_t *__restrict__ amb_list, const int32_t *__restrict__ amb_count, const int2 *__restrict__ amb_cand,
-    int32_t *__restrict__ assign) {
+    int32_t *__restrict__ assign, bool vec) {
     __shared__ double xs[8][D];
     int h = blockIdx.y;
     HeadSeg s = seg[h];
@@ -267,16 +267,43 @@ __global__ void __launch_bounds__(256) assign_exact_kernel(
             double acc = 0.0;
             // partial unrolling: a fully unrolled loop hoists all D loads into
             // registers and spills; the summation order is unchanged
+            // (the centroid read 16 bytes at a time when its base is 16-byte
+            // aligned: rows of D floats keep that alignment)
             if (mode == MODE_EUCLID) {
+                if (vec) {
+                    const float4 *c4 = reinterpret_cast<const float4 *>(c);
+#pragma unroll 4
+                    for (int t4 = 0; t4 < D / 4; t4++) {
+                        const float4 f = __ldg(c4 + t4);
+                        const float cf[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const double df = dsub(xs[warp][4 * t4 + e], (double)cf[e]);
+                            acc = dadd(acc, dmul(df, df));
+                        }
+                    }
+                } else {
 #pragma unroll 16
-                for (int t = 0; t < D; t++) {
-                    double df = dsub(xs[warp][t], (double)c[t]);
-                    acc = dadd(acc, dmul(df, df));
+                    for (int t = 0; t < D; t++) {
+                        double df = dsub(xs[warp][t], (double)c[t]);
+                        acc = dadd(acc, dmul(df, df));
+                    }
                 }
                 if (acc < best) { best = acc; bj = j; }
             } else {
+                if (vec) {
+                    const float4 *c4 = reinterpret_cast<const float4 *>(c);
+#pragma unroll 4
+                    for (int t4 = 0; t4 < D / 4; t4++) {
+                        const float4 f = __ldg(c4 + t4);
+                        const float cf[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                        for (int e = 0; e < 4; e++) acc = dadd(acc, dmul(xs[warp][4 * t4 + e], (double)cf[e]));
+                    }
+                } else {
 #pragma unroll 16
-                for (int t = 0; t < D; t++) acc = dadd(acc, dmul(xs[warp][t], (double)c[t]));
+                    for (int t = 0; t < D; t++) acc = dadd(acc, dmul(xs[warp][t], (double)c[t]));
+                }
                 if (acc > best) { best = acc; bj = j; }
             }
         }
@@ -299,7 +326,7 @@ template <typename T, int D>
 __global__ void dist_kernel(const T *__restrict__ x, int N, const int32_t *__restrict__ rows,
                             const HeadSeg *__restrict__ seg, const float *__restrict__ cent, int cap,
                             const double *__restrict__ norm, int mode, const int32_t *__restrict__ assign,
-                            double *__restrict__ dist) {
+                            double *__restrict__ dist, bool vec) {
     int h = blockIdx.y;
     HeadSeg s = seg[h];
     int pos = blockIdx.x * blockDim.x + threadIdx.x;
@@ -312,9 +339,38 @@ __global__ void dist_kernel(const T *__restrict__ x, int N, const int32_t *__res
     const int a = min(max(assign[(size_t)h * N + pos], 0), max(s.k - 1, 0));
     const float *c = cent + ((size_t)h * cap + s.cent_off + a) * D;
     double acc = 0.0;
-    for (int t = 0; t < D; t++) {
-        double df = dsub(work_val(xi, t, mode, nrm), (double)c[t]);
-        acc = dadd(acc, dmul(df, df));
+    if (!vec) {  // a base not 16-byte aligned: element by element
+        for (int t = 0; t < D; t++) {
+            const double df = dsub(work_val(xi, t, mode, nrm), (double)c[t]);
+            acc = dadd(acc, dmul(df, df));
+        }
+        dist[(size_t)h * N + pos] = sqrt(acc);
+        return;
+    }
+    // the row and its centroid read 16 bytes at a time (both bases 16-byte
+    // aligned, rows of 128 or 256 bytes); the squares are still summed element
+    // by element in order
+    constexpr int V = 16 / (int)sizeof(T);  // row elements per load
+    const uint4 *xv = reinterpret_cast<const uint4 *>(xi);
+    const float4 *cv = reinterpret_cast<const float4 *>(c);
+#pragma unroll 2
+    for (int u = 0; u < D / V; u++) {
+        const uint4 w = __ldg(xv + u);
+        const T *xs = reinterpret_cast<const T *>(&w);
+        float cf[V];
+#pragma unroll
+        for (int i = 0; i < V / 4; i++) {
+            const float4 f = __ldg(cv + u * (V / 4) + i);
+            cf[4 * i] = f.x;
+            cf[4 * i + 1] = f.y;
+            cf[4 * i + 2] = f.z;
+            cf[4 * i + 3] = f.w;
+        }
+#pragma unroll
+        for (int e = 0; e < V; e++) {
+            const double df = dsub(work_val(xs, e, mode, nrm), (double)cf[e]);
+            acc = dadd(acc, dmul(df, df));
+        }
     }
     dist[(size_t)h * N + pos] = sqrt(acc);
 }
@@ -524,8 +580,9 @@ static void launch_assign(const void *x, int H, int N, const int32_t *rows, cons
     assign_screen_kernel<T, D><<<g, 256, smem, st>>>((const T *)x, N, rows, seg, cent, cap, cn2, cmax, mode, assign,
                                                       amb_list, amb_count); note_launch();
     dim3 g2(64, H);
+    const bool vec = (reinterpret_cast<uintptr_t>(cent) & 15) == 0;
     assign_exact_kernel<T, D><<<g2, 256, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, amb_list,
-                                                   amb_count, nullptr, assign); note_launch();
+                                                   amb_count, nullptr, assign, vec); note_launch();
 }
 
 void k_assign(const void *x, int dtype, int H, int N, int D, const int32_t *rows, const HeadSeg *seg,
@@ -554,9 +611,10 @@ void k_assign_exact(const void *x, int dtype, int H, int N, int D, const int32_t
                     const float *cent, int cap, const double *norm, int mode, const int32_t *amb_list,
                     const int32_t *amb_count, const int2 *amb_cand, int32_t *assign, cudaStream_t st) {
     dim3 g2(64, H);
+    const bool vec = (reinterpret_cast<uintptr_t>(cent) & 15) == 0;
 #define AC_EXACT(T, DD)                                                                                          \
     assign_exact_kernel<T, DD><<<g2, 256, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, amb_list, \
-                                                    amb_count, amb_cand, assign)
+                                                    amb_count, amb_cand, assign, vec)
     if (dtype == DT_BF16) {
         if (D == 64) AC_EXACT(__nv_bfloat16, 64);
         else AC_EXACT(__nv_bfloat16, 128);
@@ -572,8 +630,9 @@ void k_dist(const void *x, int dtype, int H, int N, int D, const int32_t *rows, 
             int nrows_max, const float *cent, int cap, const double *norm, int mode, const int32_t *assign,
             double *dist, cudaStream_t st) {
     dim3 g((nrows_max + 127) / 128, H);
+    const bool vec = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(cent)) & 15) == 0;
 #define AC_DIST(T, DD) \
-    dist_kernel<T, DD><<<g, 128, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, assign, dist)
+    dist_kernel<T, DD><<<g, 128, 0, st>>>((const T *)x, N, rows, seg, cent, cap, norm, mode, assign, dist, vec)
     if (dtype == DT_BF16) {
         if (D == 64) AC_DIST(__nv_bfloat16, 64);
         else AC_DIST(__nv_bfloat16, 128);
