@@ -732,12 +732,12 @@ __global__ void __launch_bounds__(384, 1)
                 uint2 gm = gm_next;
                 gm_next = gm_next2;
                 if (j + 2 < nch) gm_next2 = item_mask3(p, mrow, cbase + cstep * (j + 2));
+                uint32_t drop = 0u;  // per-query selection: 8-key groups this row does not keep
                 if (ROWS) {
                     const uint32_t rm = rm_next;
                     rm_next = rm_next2;
                     if (own && j + 2 < nch) rm_next2 = load_rowmask(p, it.h, cbase + cstep * (j + 2), rpos);
-                    gm.x &= nibbles8(rm);
-                    gm.y &= nibbles8(rm >> 8);
+                    drop = ~rm & 0xFFFFu;
                 }
                 const uint32_t c = cnt + j;
                 if (!mbar_wait_warp(s_full + t, c & 1, abort_flag, p.status)) { ok = false; break; }
@@ -745,6 +745,17 @@ __global__ void __launch_bounds__(384, 1)
                 uint32_t s[128];
                 tmem_ld128(s_addr, s);
                 apply_mask(s, gm);
+                if (ROWS && drop) {
+                    // a row keeps about one group in seven of its tile's union:
+                    // every group is dropped by predicated selects, not visited
+                    // one by one as the chunk's few partial groups are
+#pragma unroll
+                    for (int g = 0; g < 16; g++) {
+                        const bool d = (drop >> g) & 1u;
+#pragma unroll
+                        for (int i = 0; i < 8; i++) s[8 * g + i] = d ? __float_as_uint(-INFINITY) : s[8 * g + i];
+                    }
+                }
                 // row max: four independent chains of 3-input max
                 float mq[4];
 #pragma unroll
