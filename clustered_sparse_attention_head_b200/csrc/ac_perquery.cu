@@ -6,6 +6,9 @@
 //     with the oracle's summation order (each thread 4 x 4 scores, elements
 //     in order): CENTROID s = (q_i . c_b) / sqrt(d); QUEST s = sum_t
 //     max(q_t M_bt, q_t m_bt) / sqrt(d) (the query is its own representative).
+//     A bf16 or fp32 element times an fp32 centroid element has at most 48
+//     significant bits, so its double product is exact and one fused
+//     multiply-add per element rounds exactly where a multiply then an add does.
 //  2. pq_topk_kernel: one warp per row keeps the top_k non-empty clusters of
 //     largest s (ties to the lower id) as a bit set [H, N, W] (W = kk_cap / 32
 //     words); the text-key group, if any, is always set.  It also sums the
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(256) pq_scores_kernel(const T *__restrict__ q,
 #pragma unroll
             for (int i = 0; i < 4; i++)
 #pragma unroll
-                for (int j = 0; j < 4; j++) acc[i][j] = dadd(acc[i][j], dmul(qv[i], cv[j]));
+                for (int j = 0; j < 4; j++) acc[i][j] = __fma_rn(qv[i], cv[j], acc[i][j]);
         }
     }
     const double scale = 1.0 / sqrt((double)D);
@@ -113,156 +116,166 @@ __global__ void __launch_bounds__(256) pq_scores_kernel(const T *__restrict__ q,
 
 // One warp per query row keeps the top_k non-empty clusters of largest score,
 // ties to the lower id.  Up to 512 clusters: lane l holds clusters l + 32 i
-// (i < 16), sorts them once (a bitonic network in registers, by score
-// descending then id ascending; empty clusters and NaN scores last), and
-// top_k rounds merge the 32 sorted lists (a warp-wide argmax over the lists'
-// heads; the winning lane shifts its list up by one).  More clusters: top_k rounds of a
+// (i < 16) in registers and the warp runs a quickselect for the row's top_k-th
+// cluster e* in the selection order (larger score, then lower id): a pivot is
+// drawn from the clusters still in question, every lane counts its candidates
+// at or before it, and the warp-wide count places e* before, at or after the
+// pivot.  The row keeps e* and every cluster before it; bit word i of the set
+// is a ballot of lane bits i.  Rotating the pivot's lane and register with the
+// round keeps rows whose scores follow the cluster order from splitting
+// unevenly (about ten rounds for 500 clusters).  More clusters: top_k rounds of a
 // warp-wide argmax over the row's scores staged in shared memory, clusters
-// already taken skipped.  Up to four warps (rows) per block, fewer when
-// kk_cap is large.
+// already taken skipped.  Up to four warps per block, fewer when kk_cap is
+// large; each warp takes rows in turn and adds its rows' pairs to the head's
+// total once.
 constexpr int PQ_WARPS = 4, PQ_SORTED = 512;
 // bytes of a warp's score region
 __host__ __device__ constexpr size_t pq_topk_region(int kk_cap) { return (size_t)kk_cap * 8; }
-// x before y in the selection order: larger score, then lower id
-__device__ __forceinline__ bool pq_before(double xv, int xi, double yv, int yi) {
-    return xv > yv || (xv == yv && xi < yi);
-}
-__global__ void __launch_bounds__(PQ_WARPS * 32) pq_topk_kernel(const double *__restrict__ scores, int N, int r0,
+// blocks per head of the top-k launch
+__host__ __device__ constexpr int pq_topk_blocks(int H) { return 8192 / H > 64 ? 8192 / H : 64; }
+__global__ void __launch_bounds__(PQ_WARPS * 32, 4) pq_topk_kernel(const double *__restrict__ scores, int N, int r0,
                                                                int nb, const int32_t *__restrict__ k_count, int kk_cap,
                                                                const int32_t *__restrict__ nk, int kk_fixed,
                                                                int text_group, const uint8_t *__restrict__ dense,
                                                                int top_k, int W, uint32_t *__restrict__ bits,
                                                                unsigned long long *__restrict__ head_pairs) {
     extern __shared__ unsigned char pqt[];
+    const unsigned full = 0xffffffffu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const size_t region = pq_topk_region(kk_cap);
     double *sc = reinterpret_cast<double *>(pqt + (size_t)warp * region);  // [warps][region]
     uint32_t *bw = reinterpret_cast<uint32_t *>(pqt + (size_t)nw * region) + (size_t)warp * W;  // [warps][W]
     const int h = blockIdx.y;
-    const int r = blockIdx.x * nw + warp;
-    if (r >= nb || r0 + r >= N) return;  // whole warp
     const int nkh_all = nk ? min(max(nk[h], 0), kk_cap) : kk_fixed;
     const int nkh = nkh_all - text_group;
     const int32_t *kc = k_count + (size_t)h * kk_cap;
-    for (int w = lane; w < W; w += 32) bw[w] = 0u;
     const bool dn = dense && dense[h];
-    unsigned long long pairs = 0ull;
-    if (!dn && nkh <= PQ_SORTED) {
-        const double *srow = scores + ((size_t)h * nb + r) * kk_cap;
-        double v[16];
-        int ix[16];
+    const bool regs = nkh <= PQ_SORTED;
+    // register path: the lane's clusters that hold keys
+    uint32_t km = 0u;
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            const int b = lane + 32 * i;
-            double x = -INFINITY;
-            int id = 0x7fffffff;  // empty cluster or NaN score: after every selectable one
-            if (b < nkh && kc[b] > 0) {
-                const double sv = srow[b];
-                if (sv == sv) {
-                    x = sv;
-                    id = b;
+    for (int i = 0; i < 16; i++) {
+        const int b = lane + 32 * i;
+        if (regs && b < nkh && kc[b] > 0) km |= 1u << i;
+    }
+    const unsigned long long text_pairs = text_group ? (unsigned long long)kc[nkh] : 0ull;
+    unsigned long long pairs = 0ull;  // lane 0: this warp's rows
+    for (int r = blockIdx.x * nw + warp; r < nb && r0 + r < N; r += gridDim.x * nw) {
+        uint32_t *out = bits + ((size_t)h * N + r0 + r) * W;
+        const double *srow = scores + ((size_t)h * nb + r) * kk_cap;
+        if (dn) {
+            for (int w = lane; w < W; w += 32) out[w] = 0u;
+        } else if (regs) {
+            double v[16];
+            uint32_t vm = 0u;  // bit i: cluster lane + 32 i holds keys and its score is a number
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                v[i] = 0.0;
+                if ((km >> i) & 1u) {
+                    const double sv = srow[lane + 32 * i];
+                    v[i] = sv;
+                    if (sv == sv) vm |= 1u << i;
                 }
             }
-            v[i] = x;
-            ix[i] = id;
-        }
-        // bitonic sort into selection order (pq_before)
+            const int tot = (int)__reduce_add_sync(full, (unsigned)__popc(vm));
+            uint32_t sel = vm;
+            if (tot > top_k) {
+                // C: candidates for e*; S: clusters known to be before e*, base of them
+                uint32_t C = vm, S = 0u;
+                int base = 0;
+                sel = 0u;
+                for (int it = 0; it < PQ_SORTED; it++) {  // each round drops at least the pivot from C
+                    const uint32_t lanes = __ballot_sync(full, C != 0u);
+                    const int rot = (it * 13 + r * 7) & 31;
+                    const uint32_t rl = rot ? ((lanes >> rot) | (lanes << (32 - rot))) : lanes;
+                    const int lead = (__ffs(rl) - 1 + rot) & 31;
+                    const int es = (it * 5 + r) & 15;
+                    const uint32_t rc = ((C | (C << 16)) >> es) & 0xFFFFu;
+                    const int e = (__ffs(rc) - 1 + es) & 15;
+                    double pv = 0.0;
 #pragma unroll
-        for (int k = 2; k <= 16; k <<= 1)
+                    for (int i = 0; i < 16; i++) pv = i == e ? v[i] : pv;
+                    pv = __shfl_sync(full, pv, lead);
+                    const int pid = __shfl_sync(full, lane + 32 * e, lead);
+                    uint32_t le = 0u;  // candidates at or before the pivot
 #pragma unroll
-            for (int j = k >> 1; j > 0; j >>= 1)
-#pragma unroll
-                for (int i = 0; i < 16; i++) {
-                    const int l = i ^ j;
-                    if (l > i) {
-                        const bool sw = (i & k) == 0 ? pq_before(v[l], ix[l], v[i], ix[i])
-                                                     : pq_before(v[i], ix[i], v[l], ix[l]);
-                        if (sw) {
-                            const double tv = v[i];
-                            v[i] = v[l];
-                            v[l] = tv;
-                            const int ti = ix[i];
-                            ix[i] = ix[l];
-                            ix[l] = ti;
-                        }
+                    for (int i = 0; i < 16; i++) {
+                        const bool bf = v[i] > pv || (v[i] == pv && lane + 32 * i <= pid);
+                        le |= (uint32_t)bf << i;
+                    }
+                    le &= C;
+                    const int cnt = (int)__reduce_add_sync(full, (unsigned)__popc(le));
+                    if (base + cnt == top_k) {
+                        sel = S | le;
+                        break;
+                    }
+                    if (base + cnt > top_k) {
+                        C = le;
+                        if (lane == lead) C &= ~(1u << e);
+                    } else {
+                        S |= le;
+                        base += cnt;
+                        C &= ~le;
                     }
                 }
-        __syncwarp();  // the bit set's zeroing (other lanes) before lane 0 sets bits
-        for (int round = 0; round < top_k; round++) {
-            double bv = v[0];
-            int bi = ix[0];
+            }
+            unsigned rp = 0u;
+            uint32_t myw = 0u;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (pq_before(ov, oi, bv, bi)) {
-                    bv = ov;
-                    bi = oi;
+            for (int i = 0; i < 16; i++) {
+                if ((sel >> i) & 1u) rp += (unsigned)kc[lane + 32 * i];
+                const uint32_t wd = __ballot_sync(full, (sel >> i) & 1u);
+                if (lane == i) myw = wd;
+            }
+            rp = __reduce_add_sync(full, rp);
+            for (int w = lane; w < W; w += 32) {
+                uint32_t x = w < 16 ? myw : 0u;
+                if (text_group && w == (nkh >> 5)) x |= 1u << (nkh & 31);  // the text-key group, always kept
+                out[w] = x;
+            }
+            if (lane == 0) pairs += (unsigned long long)rp + text_pairs;
+        } else {
+            for (int w = lane; w < W; w += 32) bw[w] = 0u;
+            // empty clusters and (below) taken ones hold NaN, which no comparison accepts
+            const double qnan = __longlong_as_double(0x7ff8000000000000ll);
+            for (int b = lane; b < nkh; b += 32) sc[b] = kc[b] > 0 ? srow[b] : qnan;
+            __syncwarp();
+            for (int round = 0; round < top_k; round++) {
+                double best = -INFINITY;
+                int bb = 0x7fffffff;
+                for (int b = lane; b < nkh; b += 32) {
+                    const double x = sc[b];
+                    if (x > best || (x == best && b < bb)) {
+                        best = x;
+                        bb = b;
+                    }
                 }
-            }
-            if (bi == 0x7fffffff) break;  // no non-empty cluster left
-            if (lane == 0) {
-                bw[bi >> 5] |= 1u << (bi & 31);
-                pairs += (unsigned long long)kc[bi];
-            }
-            // the lane whose head was taken moves its list up by one
-            if (ix[0] == bi) {
-#pragma unroll
-                for (int i = 0; i < 15; i++) {
-                    v[i] = v[i + 1];
-                    ix[i] = ix[i + 1];
+                for (int o = 16; o > 0; o >>= 1) {
+                    const double ob = __shfl_xor_sync(full, best, o);
+                    const int oj = __shfl_xor_sync(full, bb, o);
+                    if (ob > best || (ob == best && oj < bb)) {
+                        best = ob;
+                        bb = oj;
+                    }
                 }
-                v[15] = -INFINITY;
-                ix[15] = 0x7fffffff;
-            }
-        }
-        __syncwarp();
-        if (text_group && lane == 0) {
-            const int tg = nkh;  // the text-key group's id
-            bw[tg >> 5] |= 1u << (tg & 31);
-            pairs += (unsigned long long)kc[tg];
-        }
-    } else if (!dn) {
-        const double *srow = scores + ((size_t)h * nb + r) * kk_cap;
-        // empty clusters and (below) taken ones hold NaN, which no comparison accepts
-        const double qnan = __longlong_as_double(0x7ff8000000000000ll);
-        for (int b = lane; b < nkh; b += 32) sc[b] = kc[b] > 0 ? srow[b] : qnan;
-        __syncwarp();
-        for (int round = 0; round < top_k; round++) {
-            double best = -INFINITY;
-            int bb = 0x7fffffff;
-            for (int b = lane; b < nkh; b += 32) {
-                const double v = sc[b];
-                if (v > best || (v == best && b < bb)) {
-                    best = v;
-                    bb = b;
+                if (bb == 0x7fffffff) break;  // no non-empty cluster left
+                if (lane == 0) {
+                    sc[bb] = qnan;
+                    bw[bb >> 5] |= 1u << (bb & 31);
+                    pairs += (unsigned long long)kc[bb];
                 }
+                __syncwarp();
             }
-            for (int o = 16; o > 0; o >>= 1) {
-                const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-                const int oj = __shfl_xor_sync(0xffffffffu, bb, o);
-                if (ob > best || (ob == best && oj < bb)) {
-                    best = ob;
-                    bb = oj;
-                }
-            }
-            if (bb == 0x7fffffff) break;  // no non-empty cluster left
-            if (lane == 0) {
-                sc[bb] = qnan;
-                bw[bb >> 5] |= 1u << (bb & 31);
-                pairs += (unsigned long long)kc[bb];
+            if (text_group && lane == 0) {
+                const int tg = nkh;  // the text-key group's id
+                bw[tg >> 5] |= 1u << (tg & 31);
+                pairs += text_pairs;
             }
             __syncwarp();
-        }
-        if (text_group && lane == 0) {
-            const int tg = nkh;  // the text-key group's id
-            bw[tg >> 5] |= 1u << (tg & 31);
-            pairs += (unsigned long long)kc[tg];
+            for (int w = lane; w < W; w += 32) out[w] = bw[w];
+            __syncwarp();  // the next row's staging after every lane's reads
         }
     }
-    __syncwarp();
-    uint32_t *out = bits + ((size_t)h * N + r0 + r) * W;
-    for (int w = lane; w < W; w += 32) out[w] = bw[w];
     if (lane == 0 && pairs) atomicAdd(head_pairs + h, pairs);
 }
 
@@ -490,7 +503,8 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
         note_launch();
         if (smem_t > 48 * 1024)
             cudaFuncSetAttribute(pq_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
-        dim3 g2((nb + nwarps - 1) / nwarps, H);
+        const int need = (nb + nwarps - 1) / nwarps;
+        dim3 g2(need < pq_topk_blocks(H) ? need : pq_topk_blocks(H), H);
         pq_topk_kernel<<<g2, nwarps * 32, smem_t, st>>>(scores, N, r0, nb, k_count, kk_cap, nk, kk_fixed,
                                                           text_group, dense, top_k, W, bits, head_pairs);
         note_launch();
