@@ -114,6 +114,142 @@ __global__ void __launch_bounds__(256) pq_scores_kernel(const T *__restrict__ q,
     }
 }
 
+// Centroid scores, the same sums as pq_scores_kernel (elements in order, one
+// fused multiply-add each), tiled for the FP64 pipe: a CTA computes 128 rows x
+// 64 clusters, each thread 8 rows x 4 clusters, with the element axis staged in
+// chunks of 32 through two shared-memory stages (the next chunk's global loads
+// are in flight while the FMAs run on the current one), so two CTAs share an
+// SM.  A warp covers 4 row groups x 8 cluster groups, so each of its shared
+// loads reads at most 128 bytes.  Needs q and the centroids 16-byte aligned
+// (checked on the host; pq_scores_kernel otherwise).  fp32 queries hold twice
+// the registers in flight: one CTA per SM.
+constexpr int PQC_ROWS = 128, PQC_COLS = 64, PQC_KC = 32;
+constexpr size_t PQC_SMEM = (size_t)2 * PQC_KC * (PQC_ROWS + PQC_COLS) * sizeof(double);
+
+template <typename T> struct PqcRow;  // one thread's 16 consecutive query elements
+template <> struct PqcRow<__nv_bfloat16> {
+    uint4 a, b;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+        a = __ldg(reinterpret_cast<const uint4 *>(p));
+        b = __ldg(reinterpret_cast<const uint4 *>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ float get(int u) const {
+        const uint4 &x = u < 8 ? a : b;
+        const int v = u & 7;
+        const uint32_t w = v < 2 ? x.x : (v < 4 ? x.y : (v < 6 ? x.z : x.w));
+        return __uint_as_float((v & 1) ? (w & 0xFFFF0000u) : (w << 16));
+    }
+};
+template <> struct PqcRow<float> {
+    float4 x[4];
+    __device__ __forceinline__ void load(const float *p) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) x[i] = __ldg(reinterpret_cast<const float4 *>(p) + i);
+    }
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int i = 0; i < 4; i++) x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __device__ __forceinline__ float get(int u) const {
+        const float4 &v = x[u >> 2];
+        const int c = u & 3;
+        return c == 0 ? v.x : (c == 1 ? v.y : (c == 2 ? v.z : v.w));
+    }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) pq_scores_c_kernel(const T *__restrict__ q, int N, int r0, int nb,
+                                                            const float *__restrict__ k_cent, int kk_cap,
+                                                            const int32_t *__restrict__ nk, int kk_fixed,
+                                                            int text_group, double *__restrict__ scores) {
+    extern __shared__ double pqc[];
+    // stage s: qs = pqc + s * KC * (ROWS + COLS), [KC][ROWS]; cs follows, [KC][COLS]
+    const int h = blockIdx.z, tid = threadIdx.x;
+    const int nkh = (nk ? min(max(nk[h], 0), kk_cap) : kk_fixed) - text_group;
+    const int b0 = blockIdx.y * PQC_COLS, i0 = blockIdx.x * PQC_ROWS;
+    if (b0 >= nkh) return;
+    // staging roles: query row lr (16 elements from 16 lj), centroid lc (8 elements from 8 cj)
+    const int lr = tid & 127, lj = tid >> 7;
+    const int lc = tid & 63, cj = tid >> 6;
+    const bool row_ok = i0 + lr < nb && r0 + i0 + lr < N;
+    const bool cl_ok = b0 + lc < nkh;
+    const T *qrow = q + ((size_t)h * N + (row_ok ? r0 + i0 + lr : 0)) * D + 16 * lj;
+    const float *crow = k_cent + ((size_t)h * kk_cap + (cl_ok ? b0 + lc : 0)) * D + 8 * cj;
+    PqcRow<T> qr;
+    float4 c0, c1;
+    auto fetch = [&](int t0) {
+        if (row_ok) qr.load(qrow + t0); else qr.zero();
+        if (cl_ok) {
+            c0 = __ldg(reinterpret_cast<const float4 *>(crow + t0));
+            c1 = __ldg(reinterpret_cast<const float4 *>(crow + t0) + 1);
+        } else {
+            c0 = c1 = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto stash = [&](int s) {
+        double *qs = pqc + (size_t)s * PQC_KC * (PQC_ROWS + PQC_COLS);
+        double *cs = qs + PQC_KC * PQC_ROWS;
+#pragma unroll
+        for (int u = 0; u < 16; u++) qs[(16 * lj + u) * PQC_ROWS + lr] = (double)qr.get(u);
+        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int u = 0; u < 8; u++) cs[(8 * cj + u) * PQC_COLS + lc] = (double)cv[u];
+    };
+    // compute roles: warp w = row groups 4 (w >> 1) .. + 3, cluster groups 8 (w & 1) .. + 7
+    const int w = tid >> 5, l = tid & 31;
+    const int ty = 4 * (w >> 1) + (l >> 3), tx = 8 * (w & 1) + (l & 7);  // rows 8 ty.., clusters 4 tx..
+    double acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) acc[i][j] = 0.0;
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    constexpr int NCH = D / PQC_KC;
+#pragma unroll 1
+    for (int c = 0; c < NCH; c++) {
+        if (c + 1 < NCH) fetch((c + 1) * PQC_KC);
+        const double *qs = pqc + (size_t)(c & 1) * PQC_KC * (PQC_ROWS + PQC_COLS);
+        const double *cs = qs + PQC_KC * PQC_ROWS;
+#pragma unroll 4
+        for (int t = 0; t < PQC_KC; t++) {
+            double qv[8], cv[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const double2 x = *reinterpret_cast<const double2 *>(qs + t * PQC_ROWS + 8 * ty + 2 * i);
+                qv[2 * i] = x.x;
+                qv[2 * i + 1] = x.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                const double2 x = *reinterpret_cast<const double2 *>(cs + t * PQC_COLS + 4 * tx + 2 * j);
+                cv[2 * j] = x.x;
+                cv[2 * j + 1] = x.y;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+#pragma unroll
+                for (int j = 0; j < 4; j++) acc[i][j] = __fma_rn(qv[i], cv[j], acc[i][j]);
+        }
+        if (c + 1 < NCH) stash((c + 1) & 1);
+        __syncthreads();
+    }
+    const double scale = 1.0 / sqrt((double)D);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const int r = i0 + 8 * ty + i;
+        if (r >= nb || r0 + r >= N) continue;
+        double *srow = scores + ((size_t)h * nb + r) * kk_cap;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int b = b0 + 4 * tx + j;
+            if (b < nkh) srow[b] = dmul(acc[i][j], scale);
+        }
+    }
+}
+
 // One warp per query row keeps the top_k non-empty clusters of largest score,
 // ties to the lower id.  Up to 512 clusters: lane l holds clusters l + 32 i
 // (i < 16) in registers and the warp runs a quickselect for the row's top_k-th
@@ -482,6 +618,8 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
     nwarps = nwarps < 1 ? 1 : (nwarps > PQ_WARPS ? PQ_WARPS : nwarps);
     const size_t smem_t = (size_t)nwarps * per_warp;
     cudaMemsetAsync(head_pairs, 0, sizeof(unsigned long long) * H, st);
+    // centroid scores from 16-byte aligned operands: the chunked kernel
+    const bool tiled = score_mode == 0 && ((uintptr_t)q & 15u) == 0 && ((uintptr_t)k_cent & 15u) == 0;
     for (int r0 = 0; r0 < N; r0 += batch) {
         const int nb = N - r0 < batch ? N - r0 : batch;
         dim3 g1((nb + PQ_ROWS - 1) / PQ_ROWS, (nkmax + PQ_COLS - 1) / PQ_COLS, H);
@@ -492,7 +630,22 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
         pq_scores_kernel<T, DD><<<g1, 256, smem_s, st>>>(static_cast<const T *>(q), N, r0, nb, k_cent, k_max, k_min, \
                                                          kk_cap, nk, kk_fixed, text_group, score_mode, scores);     \
     } while (0)
-        if (dtype == DT_BF16) {
+#define AC_PQC(T, DD)                                                                                              \
+    do {                                                                                                           \
+        cudaFuncSetAttribute(pq_scores_c_kernel<T, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PQC_SMEM); \
+        pq_scores_c_kernel<T, DD><<<gc, 256, PQC_SMEM, st>>>(static_cast<const T *>(q), N, r0, nb, k_cent, kk_cap,  \
+                                                           nk, kk_fixed, text_group, scores);                      \
+    } while (0)
+        if (tiled) {
+            dim3 gc((nb + PQC_ROWS - 1) / PQC_ROWS, (nkmax + PQC_COLS - 1) / PQC_COLS, H);
+            if (dtype == DT_BF16) {
+                if (D == 64) AC_PQC(__nv_bfloat16, 64);
+                else AC_PQC(__nv_bfloat16, 128);
+            } else {
+                if (D == 64) AC_PQC(float, 64);
+                else AC_PQC(float, 128);
+            }
+        } else if (dtype == DT_BF16) {
             if (D == 64) AC_PQS(__nv_bfloat16, 64);
             else AC_PQS(__nv_bfloat16, 128);
         } else {
@@ -500,6 +653,7 @@ int k_select_rows(const void *q, int dtype, int H, int N, int D, const float *k_
             else AC_PQS(float, 128);
         }
 #undef AC_PQS
+#undef AC_PQC
         note_launch();
         if (smem_t > 48 * 1024)
             cudaFuncSetAttribute(pq_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);

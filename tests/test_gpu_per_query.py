@@ -2,7 +2,9 @@
 against the oracle's per-query path.
 
   * ac_select_rows, fed the oracle's key clusters, gives every query row the
-    oracle's set bit for bit (CENTROID and QUEST scores, ragged sizes);
+    oracle's set bit for bit (CENTROID and QUEST scores, ragged sizes; also
+    from query and centroid buffers off the 16-byte grid, which take the
+    element-wise score kernel instead of the tiled one);
   * ac_sparse_attn_rows, fed the oracle's clusters and row sets, matches the
     oracle's attention of each row over its own keys (max-abs 2e-2, mean-abs
     2e-3 on all rows);
@@ -91,6 +93,19 @@ def test_select_rows_and_attention_from_oracle_clusters(orc, name):
     got_bits = bits.cpu().numpy().view(np.uint32)
     bad = np.nonzero((got_bits != want_bits).any(axis=2))
     assert len(bad[0]) == 0, f"{name}: {len(bad[0])} rows with a different set, e.g. {list(zip(*bad))[:5]}"
+    if over["score_mode"] == 0:
+        # queries and centroids at addresses off the 16-byte grid (the element-wise score kernel)
+        def shifted(t):
+            buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+            view = buf[1:].view(t.shape)
+            view.copy_(t)
+            assert view.data_ptr() % 16 != 0
+            return view
+        bits_u = ctx.ac_select_rows(shifted(qd), dev(k_count), k_cent=shifted(dev(k_cent)))
+        torch.cuda.synchronize()
+        assert ctx.get_status() == 0
+        got_u = bits_u.cpu().numpy().view(np.uint32)
+        assert np.array_equal(got_u, want_bits), f"{name}: unaligned operands give other sets"
     # attention from the oracle's clusters and sets, every row
     rb = torch.from_numpy(want_bits.view(np.int32)).cuda()
     nq = torch.full((H,), w.kq, dtype=torch.int32, device="cuda")
@@ -109,7 +124,7 @@ def test_select_rows_and_attention_from_oracle_clusters(orc, name):
 # hand-made key clusters for the per-row argtopk: duplicated centroids (exact
 # score ties, broken towards the lower id), empty clusters (never chosen, also
 # when they duplicate a chosen one), and cluster counts on both sides of 512
-# (one sorted list of 16 per lane up to 512 clusters, the scan beyond)
+# (a register quickselect up to 512 clusters, the shared-memory scan beyond)
 TIE_CASES = {
     "ties-kk40": (300, 40, 6),
     "ties-kk512": (600, 512, 5),
