@@ -116,14 +116,14 @@ __global__ void __launch_bounds__(256) pq_scores_kernel(const T *__restrict__ q,
 
 // Centroid scores, the same sums as pq_scores_kernel (elements in order, one
 // fused multiply-add each), tiled for the FP64 pipe: a CTA computes 128 rows x
-// 64 clusters, each thread 8 rows x 4 clusters, with the element axis staged in
-// chunks of 32 through two shared-memory stages (the next chunk's global loads
-// are in flight while the FMAs run on the current one), so two CTAs share an
-// SM.  A warp covers 4 row groups x 8 cluster groups, so each of its shared
-// loads reads at most 128 bytes.  Needs q and the centroids 16-byte aligned
-// (checked on the host; pq_scores_kernel otherwise).  fp32 queries hold twice
-// the registers in flight: one CTA per SM.
-constexpr int PQC_ROWS = 128, PQC_COLS = 64, PQC_KC = 32;
+// 128 clusters, each thread 8 rows x 8 clusters, with the element axis staged
+// in chunks of 32 through two shared-memory stages (the next chunk's global
+// loads are in flight while the FMAs run on the current one).  Shared memory
+// delivers 128 bytes per cycle whatever the broadcast, so the thread tile sets
+// the ratio of shared-memory wavefronts to FMAs: (8 + 8) doubles read per 64
+// FMAs.  One CTA per SM (232 registers a thread).  Needs q and the centroids
+// 16-byte aligned (checked on the host; pq_scores_kernel otherwise).
+constexpr int PQC_ROWS = 128, PQC_COLS = 128, PQC_KC = 32;
 constexpr size_t PQC_SMEM = (size_t)2 * PQC_KC * (PQC_ROWS + PQC_COLS) * sizeof(double);
 
 template <typename T> struct PqcRow;  // one thread's 16 consecutive query elements
@@ -159,7 +159,7 @@ template <> struct PqcRow<float> {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) pq_scores_c_kernel(const T *__restrict__ q, int N, int r0, int nb,
+__global__ void __launch_bounds__(256, 1) pq_scores_c_kernel(const T *__restrict__ q, int N, int r0, int nb,
                                                             const float *__restrict__ k_cent, int kk_cap,
                                                             const int32_t *__restrict__ nk, int kk_fixed,
                                                             int text_group, double *__restrict__ scores) {
@@ -169,41 +169,37 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) pq_scores_c_kerne
     const int nkh = (nk ? min(max(nk[h], 0), kk_cap) : kk_fixed) - text_group;
     const int b0 = blockIdx.y * PQC_COLS, i0 = blockIdx.x * PQC_ROWS;
     if (b0 >= nkh) return;
-    // staging roles: query row lr (16 elements from 16 lj), centroid lc (8 elements from 8 cj)
+    // staging roles: query row lr and centroid lc, 16 elements each from 16 lj
     const int lr = tid & 127, lj = tid >> 7;
-    const int lc = tid & 63, cj = tid >> 6;
+    const int lc = tid & 127;
     const bool row_ok = i0 + lr < nb && r0 + i0 + lr < N;
     const bool cl_ok = b0 + lc < nkh;
     const T *qrow = q + ((size_t)h * N + (row_ok ? r0 + i0 + lr : 0)) * D + 16 * lj;
-    const float *crow = k_cent + ((size_t)h * kk_cap + (cl_ok ? b0 + lc : 0)) * D + 8 * cj;
+    const float *crow = k_cent + ((size_t)h * kk_cap + (cl_ok ? b0 + lc : 0)) * D + 16 * lj;
     PqcRow<T> qr;
-    float4 c0, c1;
+    PqcRow<float> cr;
     auto fetch = [&](int t0) {
         if (row_ok) qr.load(qrow + t0); else qr.zero();
-        if (cl_ok) {
-            c0 = __ldg(reinterpret_cast<const float4 *>(crow + t0));
-            c1 = __ldg(reinterpret_cast<const float4 *>(crow + t0) + 1);
-        } else {
-            c0 = c1 = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+        if (cl_ok) cr.load(crow + t0); else cr.zero();
     };
     auto stash = [&](int s) {
         double *qs = pqc + (size_t)s * PQC_KC * (PQC_ROWS + PQC_COLS);
         double *cs = qs + PQC_KC * PQC_ROWS;
 #pragma unroll
         for (int u = 0; u < 16; u++) qs[(16 * lj + u) * PQC_ROWS + lr] = (double)qr.get(u);
-        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int u = 0; u < 8; u++) cs[(8 * cj + u) * PQC_COLS + lc] = (double)cv[u];
+        for (int u = 0; u < 16; u++) cs[(16 * lj + u) * PQC_COLS + lc] = (double)cr.get(u);
     };
-    // compute roles: warp w = row groups 4 (w >> 1) .. + 3, cluster groups 8 (w & 1) .. + 7
+    // compute roles: warp w = row groups 4 (w >> 1) .. + 3, cluster groups 8 (w & 1) .. + 7;
+    // thread: rows 8 ty .. 8 ty + 7, clusters tx + 16 j (j < 8: eight threads of
+    // a quarter warp read eight consecutive doubles, no bank conflict)
     const int w = tid >> 5, l = tid & 31;
-    const int ty = 4 * (w >> 1) + (l >> 3), tx = 8 * (w & 1) + (l & 7);  // rows 8 ty.., clusters 4 tx..
-    double acc[8][4];
+    const int ty = 4 * (w >> 1) + (l >> 3), tx = 8 * (w & 1) + (l & 7);
+    double acc[8][8];
 #pragma unroll
     for (int i = 0; i < 8; i++)
 #pragma unroll
-        for (int j = 0; j < 4; j++) acc[i][j] = 0.0;
+        for (int j = 0; j < 8; j++) acc[i][j] = 0.0;
     fetch(0);
     stash(0);
     __syncthreads();
@@ -215,7 +211,7 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) pq_scores_c_kerne
         const double *cs = qs + PQC_KC * PQC_ROWS;
 #pragma unroll 4
         for (int t = 0; t < PQC_KC; t++) {
-            double qv[8], cv[4];
+            double qv[8], cv[8];
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 const double2 x = *reinterpret_cast<const double2 *>(qs + t * PQC_ROWS + 8 * ty + 2 * i);
@@ -223,15 +219,11 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) pq_scores_c_kerne
                 qv[2 * i + 1] = x.y;
             }
 #pragma unroll
-            for (int j = 0; j < 2; j++) {
-                const double2 x = *reinterpret_cast<const double2 *>(cs + t * PQC_COLS + 4 * tx + 2 * j);
-                cv[2 * j] = x.x;
-                cv[2 * j + 1] = x.y;
-            }
+            for (int j = 0; j < 8; j++) cv[j] = cs[t * PQC_COLS + tx + 16 * j];
 #pragma unroll
             for (int i = 0; i < 8; i++)
 #pragma unroll
-                for (int j = 0; j < 4; j++) acc[i][j] = __fma_rn(qv[i], cv[j], acc[i][j]);
+                for (int j = 0; j < 8; j++) acc[i][j] = __fma_rn(qv[i], cv[j], acc[i][j]);
         }
         if (c + 1 < NCH) stash((c + 1) & 1);
         __syncthreads();
@@ -243,8 +235,8 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) pq_scores_c_kerne
         if (r >= nb || r0 + r >= N) continue;
         double *srow = scores + ((size_t)h * nb + r) * kk_cap;
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int b = b0 + 4 * tx + j;
+        for (int j = 0; j < 8; j++) {
+            const int b = b0 + tx + 16 * j;
             if (b < nkh) srow[b] = dmul(acc[i][j], scale);
         }
     }
@@ -502,7 +494,8 @@ constexpr int PQ_MAX_RUNS = 8192;
 __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *__restrict__ koff,
                                   const int2 *__restrict__ runs, const int2 *__restrict__ info,
                                   const int32_t *__restrict__ qperm, const int32_t *__restrict__ qoff,
-                                  const uint32_t *__restrict__ bits, int W, uint16_t *__restrict__ rowmask) {
+                                  const uint32_t *__restrict__ bits, int W, int rows_pass,
+                                  uint16_t *__restrict__ rowmask) {
     extern __shared__ int pqr[];
     int *s_start = pqr;                  // [nr] slot start of each run
     int *gcl = pqr + PQ_MAX_RUNS;        // [nch * 16] cluster of each group (-1: padding)
@@ -582,18 +575,32 @@ __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks,
         if (cur >= 0) gcl[j * 16 + ne++] = (int)(((uint32_t)cur << 16) | gm);
         nent[j] = ne;
     }
-    __syncthreads();
-    for (int p = o[a] + tid; p < o[a + 1]; p += nt) {
-        const uint32_t *rb = bits + ((size_t)h * N + qperm[(size_t)h * N + p]) * W;
-        for (int j = 0; j < nch; j++) {
-            uint32_t m = 0u;
-            const int ne = nent[j];
-            for (int e = 0; e < ne; e++) {
-                const uint32_t v = (uint32_t)gcl[j * 16 + e];
-                const uint32_t cl = v >> 16;
-                if ((rb[cl >> 5] >> (cl & 31)) & 1u) m |= v & 0xFFFFu;
+    // rows in passes of rows_pass: their bit sets copied row by row (coalesced)
+    // into shared memory at an odd stride, so that the per-chunk tests read
+    // 32 different rows' words without bank conflicts
+    uint32_t *sb = reinterpret_cast<uint32_t *>(nent + max_chunks);  // [rows_pass][W + 1]
+    const int ld = W + 1;
+    for (int p0 = o[a]; p0 < o[a + 1]; p0 += rows_pass) {
+        const int np = min(rows_pass, o[a + 1] - p0);
+        __syncthreads();  // the previous pass's reads of sb (and, first, the entry table)
+        for (int g = tid; g < np * W; g += nt) {
+            const int rr = g / W, w = g - rr * W;
+            sb[rr * ld + w] = bits[((size_t)h * N + qperm[(size_t)h * N + p0 + rr]) * W + w];
+        }
+        __syncthreads();
+        for (int rr = tid; rr < np; rr += nt) {
+            const uint32_t *rb = sb + rr * ld;
+            const int p = p0 + rr;
+            for (int j = 0; j < nch; j++) {
+                uint32_t m = 0u;
+                const int ne = nent[j];
+                for (int e = 0; e < ne; e++) {
+                    const uint32_t v = (uint32_t)gcl[j * 16 + e];
+                    const uint32_t cl = v >> 16;
+                    if ((rb[cl >> 5] >> (cl & 31)) & 1u) m |= v & 0xFFFFu;
+                }
+                rowmask[((size_t)h * max_chunks + j) * N + p] = (uint16_t)m;
             }
-            rowmask[((size_t)h * max_chunks + j) * N + p] = (uint16_t)m;
         }
     }
 }
@@ -687,11 +694,15 @@ void k_key_runs_single(int H, int kq_cap, int kk_cap, const int32_t *koff, const
 int k_rowmask(int H, int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *koff, const int2 *runs,
               const int2 *info, const int32_t *qperm, const int32_t *qoff, const uint32_t *bits, int W,
               uint16_t *rowmask, cudaStream_t st) {
-    const size_t smem = (size_t)(PQ_MAX_RUNS + (size_t)max_chunks * 17) * sizeof(int);
-    if (smem > 227 * 1024) return -1;  // the group table of the longest key stream does not fit
+    const size_t base = (size_t)(PQ_MAX_RUNS + (size_t)max_chunks * 17) * sizeof(int);
+    const size_t limit = 227 * 1024, per_row = (size_t)(W + 1) * sizeof(uint32_t);
+    // rows per pass: the block's 256 threads, fewer when the bit sets are long
+    const int rows_pass = base + 32 * per_row > limit ? 0 : (int)std::min<size_t>(256, (limit - base) / per_row / 32 * 32);
+    if (rows_pass < 32) return -1;  // the group table of the longest key stream does not fit
+    const size_t smem = base + (size_t)rows_pass * per_row;
     cudaFuncSetAttribute(pq_rowmask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     pq_rowmask_kernel<<<dim3(kq_cap, H), 256, smem, st>>>(N, kq_cap, kk_cap, max_chunks, koff, runs, info, qperm,
-                                                          qoff, bits, W, rowmask);
+                                                          qoff, bits, W, rows_pass, rowmask);
     note_launch();
     return 0;
 }
