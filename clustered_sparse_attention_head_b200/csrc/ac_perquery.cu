@@ -489,8 +489,11 @@ __global__ void key_runs_single_kernel(int H, int kq_cap, int kk_cap, const int3
 // Per row of query cluster a and chunk j of its key stream: bit g set when
 // the row's own set holds the cluster of 8-key group g.  The groups' clusters
 // come from the runs' slot layout (every run's rows from its slot start, its
-// last group padded), as the key stream packs them.
-constexpr int PQ_MAX_RUNS = 8192;
+// last group padded), as the key stream packs them.  One run per selected
+// cluster, so at most kk_cap runs (their slot starts take kk_cap rounded up to
+// even ints of shared memory, so that the group table behind them is 8-byte
+// aligned).
+__host__ __device__ constexpr int pq_run_slots(int kk_cap) { return (kk_cap + 1) & ~1; }
 __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *__restrict__ koff,
                                   const int2 *__restrict__ runs, const int2 *__restrict__ info,
                                   const int32_t *__restrict__ qperm, const int32_t *__restrict__ qoff,
@@ -498,12 +501,12 @@ __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks,
                                   uint16_t *__restrict__ rowmask) {
     extern __shared__ int pqr[];
     int *s_start = pqr;                  // [nr] slot start of each run
-    int *gcl = pqr + PQ_MAX_RUNS;        // [nch * 16] cluster of each group (-1: padding)
+    int *gcl = pqr + pq_run_slots(kk_cap);  // [nch * 16] cluster of each group (-1: padding)
     __shared__ int wsum[32];
     const int h = blockIdx.y, a = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
     const size_t qa = (size_t)h * kq_cap + a;
     const int2 inf = info[qa];
-    const int nr = min(inf.x, PQ_MAX_RUNS), nch = min(inf.y, max_chunks);
+    const int nr = min(inf.x, kk_cap), nch = min(inf.y, max_chunks);
     const int32_t *o = qoff + (size_t)h * (kq_cap + 1);
     if (nch <= 0 || o[a + 1] <= o[a]) return;
     const int2 *rr = runs + qa * kk_cap;
@@ -558,7 +561,8 @@ __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks,
     }
     __syncthreads();
     // compress each chunk's 16 groups, in place, into (cluster << 16 | groups)
-    // entries, one per run of groups of one cluster (usually one or two)
+    // entries, one per run of groups of one cluster (usually one or two; the
+    // first two always written, zero entries select nothing)
     int *nent = gcl + max_chunks * 16;  // [nch]
     for (int j = tid; j < nch; j += nt) {
         int ne = 0, cur = -1;
@@ -574,6 +578,7 @@ __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks,
         }
         if (cur >= 0) gcl[j * 16 + ne++] = (int)(((uint32_t)cur << 16) | gm);
         nent[j] = ne;
+        for (int e = ne; e < 2; e++) gcl[j * 16 + e] = 0;
     }
     // rows in passes of rows_pass: their bit sets copied row by row (coalesced)
     // into shared memory at an odd stride, so that the per-chunk tests read
@@ -590,16 +595,15 @@ __global__ void pq_rowmask_kernel(int N, int kq_cap, int kk_cap, int max_chunks,
         __syncthreads();
         for (int rr = tid; rr < np; rr += nt) {
             const uint32_t *rb = sb + rr * ld;
-            const int p = p0 + rr;
-            for (int j = 0; j < nch; j++) {
-                uint32_t m = 0u;
+            uint16_t *dst = rowmask + (size_t)h * max_chunks * N + p0 + rr;
+            // entry v keeps its groups when the row's set holds cluster v >> 16
+            auto take = [&](uint32_t v) { return ((rb[v >> 21] >> ((v >> 16) & 31u)) & 1u) ? (v & 0xFFFFu) : 0u; };
+            for (int j = 0; j < nch; j++, dst += N) {
                 const int ne = nent[j];
-                for (int e = 0; e < ne; e++) {
-                    const uint32_t v = (uint32_t)gcl[j * 16 + e];
-                    const uint32_t cl = v >> 16;
-                    if ((rb[cl >> 5] >> (cl & 31)) & 1u) m |= v & 0xFFFFu;
-                }
-                rowmask[((size_t)h * max_chunks + j) * N + p] = (uint16_t)m;
+                const int2 v2 = *reinterpret_cast<const int2 *>(gcl + j * 16);
+                uint32_t m = take((uint32_t)v2.x) | take((uint32_t)v2.y);
+                for (int e = 2; e < ne; e++) m |= take((uint32_t)gcl[j * 16 + e]);
+                *dst = (uint16_t)m;
             }
         }
     }
@@ -694,7 +698,7 @@ void k_key_runs_single(int H, int kq_cap, int kk_cap, const int32_t *koff, const
 int k_rowmask(int H, int N, int kq_cap, int kk_cap, int max_chunks, const int32_t *koff, const int2 *runs,
               const int2 *info, const int32_t *qperm, const int32_t *qoff, const uint32_t *bits, int W,
               uint16_t *rowmask, cudaStream_t st) {
-    const size_t base = (size_t)(PQ_MAX_RUNS + (size_t)max_chunks * 17) * sizeof(int);
+    const size_t base = (size_t)(pq_run_slots(kk_cap) + (size_t)max_chunks * 17) * sizeof(int);
     const size_t limit = 227 * 1024, per_row = (size_t)(W + 1) * sizeof(uint32_t);
     // rows per pass: the block's 256 threads, fewer when the bit sets are long
     const int rows_pass = base + 32 * per_row > limit ? 0 : (int)std::min<size_t>(256, (limit - base) / per_row / 32 * 32);
