@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.ORDER)
     ap.add_argument("--top-p", type=float, default=None)
     ap.add_argument("--heads", type=int, default=None, help="fewer heads (profiling captures only)")
+    ap.add_argument("--select-mode", default=None, choices=sorted(SELECT_MODES),
+                    help="time the main call with one of the selection options instead of the top-p cut")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -279,14 +281,16 @@ def main():
     # replays its cached CUDA graph of the call when a call repeats the buffers);
     # `ac` records per-stage events, which keeps it launch by launch, and gives
     # the stage breakdown, the statistics and a launch-by-launch timing
-    cfg = Config.from_workload(w)
-    if a.text_keys:
-        cfg.text_keys = w.text
-    ac_t = AdaCluster(cfg, device=dev)
-    cfg = Config.from_workload(w)
+    def main_cfg():
+        cfg = Config.from_workload(w)
+        if a.text_keys:
+            cfg.text_keys = w.text
+        for key, val in SELECT_MODES.get(a.select_mode, {}).items():
+            setattr(cfg, key, val)
+        return cfg
+    ac_t = AdaCluster(main_cfg(), device=dev)
+    cfg = main_cfg()
     cfg.flags = _abi.AC_FLAG_PROFILE
-    if a.text_keys:
-        cfg.text_keys = w.text
     ac = AdaCluster(cfg, device=dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
@@ -429,7 +433,7 @@ def main():
     # version on the Wan-shaped workload cut to 8 heads, scaled by heads; only
     # for that workload (None until such a capture exists)
     traffic = None
-    if w.name == DEFAULT_WORKLOAD and w.top_p == 0.9 and ATTN_TRAFFIC_8H:
+    if w.name == DEFAULT_WORKLOAD and w.top_p == 0.9 and ATTN_TRAFFIC_8H and not a.select_mode:
         traffic = ATTN_TRAFFIC_8H * w.heads / 8
     roof = {"kernel": "attn3_kernel (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": tflops_attn,
             "peak": peak, "unit": "TFLOP/s", "frac": tflops_attn / peak, "traffic": traffic,
@@ -459,7 +463,8 @@ def main():
         line = {"metric": METRIC, "value": calls_per_s, "unit": "calls/s", "n_gpus": world, "steps": a.steps,
                 "warmup": max(a.warmup, 3), "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-                "config": config_of(w, world, cfg.text_keys),
+                "config": dict(config_of(w, world, cfg.text_keys),
+                               **({"select_mode": {a.select_mode: SELECT_MODES[a.select_mode]}} if a.select_mode else {})),
                 "tflops_effective_call": tflops_call, "tflops_effective_attn": tflops_attn,
                 "pairs": st["pairs"], "density": st["pairs"] / (w.heads * float(w.n) ** 2),
                 "dense_heads": st["dense_heads"],
