@@ -423,8 +423,8 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
     static_assert(R <= UPD_THREADS && D <= UPD_THREADS, "one thread per row / element");
     extern __shared__ __align__(16) unsigned char upd_smem[];
     T *rows = reinterpret_cast<T *>(upd_smem);                                           // [S][R][D]
-    double *nrm = reinterpret_cast<double *>(upd_smem + UPD_STAGES * UPD_CHUNK_BYTES);  // [S][R]
-    double *rcp = nrm + UPD_STAGES * R;                                                  // [S][R]
+    // per staged row (||x||, RN(1/||x||)), read by the summing threads as one 16-byte pair
+    double2 *nry = reinterpret_cast<double2 *>(upd_smem + UPD_STAGES * UPD_CHUNK_BYTES);  // [S][R]
     __shared__ double ssum[D];
     __shared__ double snr;
     // grid (head, rank): with an order the rank-th largest cluster of the head
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
                 cp_async16(dst + r * ROW_BYTES + q * 16,
                            reinterpret_cast<const unsigned char *>(xh + (size_t)tk[k] * D) + q * 16);
         }
-        if (tkn >= 0) cp_async8(nrm + (c % UPD_STAGES) * R + tid, nh + tkn);
+        if (tkn >= 0) cp_async8(&nry[(c % UPD_STAGES) * R + tid].x, nh + tkn);
         cp_async_commit();
     };
 #pragma unroll
@@ -477,10 +477,10 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
         __syncthreads();  // chunk c has landed for every thread; stage (c - 1) % S is free
         const int st = c % UPD_STAGES, nr = min(R, n - c * R);
         if (sphere) {
-            // y = RN(1/||x||) once per row; 0 marks a zero row (its quotients are 0)
+            // y = RN(1/||x||) once per row, 0 for a zero row
             if (tid < nr) {
-                const double v = nrm[st * R + tid];
-                rcp[st * R + tid] = v > 0.0 ? __drcp_rn(v) : 0.0;
+                const double v = nry[st * R + tid].x;
+                nry[st * R + tid].y = v > 0.0 ? __drcp_rn(v) : 0.0;
             }
             __syncthreads();
         }
@@ -489,15 +489,16 @@ __global__ void __launch_bounds__(UPD_THREADS) update2_kernel(const T *__restric
         if (tid < D) {
             const T *rs = rows + (size_t)st * R * D + tid;
             if (sphere) {
-                const double *nr_s = nrm + st * R, *rc_s = rcp + st * R;
+                const double2 *ny_s = nry + st * R;
+                // a zero row (||x|| = 0) has every element +-0 and y = 0, so q0,
+                // rr and q are all +0, which is what a zero row adds
 #pragma unroll 8
                 for (int r = 0; r < nr; r++) {
                     const double v = (double)to_f(rs[r * D]);
-                    const double bn = nr_s[r], y = rc_s[r];
-                    const double q0 = dmul(v, y);
-                    const double rr = __fma_rn(-bn, q0, v);
-                    const double q = __fma_rn(rr, y, q0);
-                    acc = dadd(acc, bn > 0.0 ? q : 0.0);
+                    const double2 ny = ny_s[r];
+                    const double q0 = dmul(v, ny.y);
+                    const double rr = __fma_rn(-ny.x, q0, v);
+                    acc = dadd(acc, __fma_rn(rr, ny.y, q0));
                 }
             } else {
 #pragma unroll 8
