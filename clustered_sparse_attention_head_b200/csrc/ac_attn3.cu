@@ -742,73 +742,83 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t c = cnt + j;
                 if (!mbar_wait_warp(s_full + t, c & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t s[128];
-                tmem_ld128(s_addr, s);
-                apply_mask(s, gm);
-                if (ROWS && drop) {
-                    // a row keeps about one group in seven of its tile's union:
-                    // every group is dropped by predicated selects, not visited
-                    // one by one as the chunk's few partial groups are
+                // A warp none of whose rows takes a key of this chunk (rows past
+                // the item's query rows, whose output is never written, and rows
+                // that keep none of the chunk's groups) would compute P = 0 with
+                // its row maxima, sums and O unchanged: it stores the zeros
+                // (after S_t(j) is complete, as P always is) and skips the rest.
+                if (__all_sync(0xffffffffu, !valid || (ROWS && drop == 0xFFFFu))) {
+                    tmem_st32_zero(s_addr);
+                    tmem_st32_zero(s_addr + 32);
+                } else {
+                    uint32_t s[128];
+                    tmem_ld128(s_addr, s);
+                    apply_mask(s, gm);
+                    if (ROWS && drop) {
+                        // a row keeps about one group in seven of its tile's union:
+                        // every group is dropped by predicated selects, not visited
+                        // one by one as the chunk's few partial groups are
 #pragma unroll
-                    for (int g = 0; g < 16; g++) {
-                        const bool d = (drop >> g) & 1u;
+                        for (int g = 0; g < 16; g++) {
+                            const bool d = (drop >> g) & 1u;
 #pragma unroll
-                        for (int i = 0; i < 8; i++) s[8 * g + i] = d ? __float_as_uint(-INFINITY) : s[8 * g + i];
+                            for (int i = 0; i < 8; i++) s[8 * g + i] = d ? __float_as_uint(-INFINITY) : s[8 * g + i];
+                        }
                     }
-                }
-                // row max: four independent chains of 3-input max
-                float mq[4];
+                    // row max: four independent chains of 3-input max
+                    float mq[4];
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    float m = fmaxf(__uint_as_float(s[32 * q]), __uint_as_float(s[32 * q + 1]));
+                    for (int q = 0; q < 4; q++) {
+                        float m = fmaxf(__uint_as_float(s[32 * q]), __uint_as_float(s[32 * q + 1]));
 #pragma unroll
-                    for (int i = 2; i < 32; i += 2)
-                        m = fmax3(m, __uint_as_float(s[32 * q + i]), __uint_as_float(s[32 * q + i + 1]));
-                    mq[q] = m;
-                }
-                const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
-                const float m_new = mx * sc;
-                if (j == 0) m_ref = m_new;
-                // Move the reference max (and rescale O_t and l by f) only when it
-                // grew by more than 2^8; warp-uniform because TMEM access is
-                // collective.  The rescale of O_t waits until P_t(j) is stored (the
-                // scores are then dead, which keeps the register peak low); it
-                // only has to precede the arrival that lets PV_t(j) go, and
-                // PV_t(j-1) is complete: S_t(j) was issued after it.
-                const bool rescale = j > 0 && __any_sync(0xffffffffu, m_new > m_ref + 8.f);
-                float f = 1.f;
-                if (rescale) {
-                    const float m_to = fmaxf(m_ref, m_new);
-                    // a row with no unmasked key yet keeps f = 1 (its O and l are 0)
-                    f = m_to == -INFINITY ? 1.f : ex2_approx(m_ref - m_to);
-                    m_ref = m_to;
-                }
-                // a row whose keys so far are all masked (per-query selection) has
-                // m_ref = -inf: its scores are all -inf and must give P = 0
-                const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
-                const uint64_t scale2 = pack2(sc, sc), neg2 = pack2(negm, negm);
-                // row sum in four partial sums (two packed pairs), folded into l0/l1
-                uint64_t la[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
-                uint32_t pk[32];
-                exp_pairs<C::EMU_PER8, 0, 32>(s, pk, scale2, neg2, la);
-                tmem_st32(s_addr, pk);
-                exp_pairs<C::EMU_PER8, 32, 32>(s, pk, scale2, neg2, la);
-                tmem_st32(s_addr + 32, pk);
-                if (rescale) {
-#pragma unroll
-                    for (int pc = 0; pc < D / 32; pc++) {
-                        uint32_t o[32];
-                        tmem_ld32(o_addr + pc * 32, o);
-#pragma unroll
-                        for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                        tmem_st32(o_addr + pc * 32, o);
+                        for (int i = 2; i < 32; i += 2)
+                            m = fmax3(m, __uint_as_float(s[32 * q + i]), __uint_as_float(s[32 * q + i + 1]));
+                        mq[q] = m;
                     }
+                    const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+                    const float m_new = mx * sc;
+                    if (j == 0) m_ref = m_new;
+                    // Move the reference max (and rescale O_t and l by f) only when it
+                    // grew by more than 2^8; warp-uniform because TMEM access is
+                    // collective.  The rescale of O_t waits until P_t(j) is stored (the
+                    // scores are then dead, which keeps the register peak low); it
+                    // only has to precede the arrival that lets PV_t(j) go, and
+                    // PV_t(j-1) is complete: S_t(j) was issued after it.
+                    const bool rescale = j > 0 && __any_sync(0xffffffffu, m_new > m_ref + 8.f);
+                    float f = 1.f;
+                    if (rescale) {
+                        const float m_to = fmaxf(m_ref, m_new);
+                        // a row with no unmasked key yet keeps f = 1 (its O and l are 0)
+                        f = m_to == -INFINITY ? 1.f : ex2_approx(m_ref - m_to);
+                        m_ref = m_to;
+                    }
+                    // a row whose keys so far are all masked (per-query selection) has
+                    // m_ref = -inf: its scores are all -inf and must give P = 0
+                    const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
+                    const uint64_t scale2 = pack2(sc, sc), neg2 = pack2(negm, negm);
+                    // row sum in four partial sums (two packed pairs), folded into l0/l1
+                    uint64_t la[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+                    uint32_t pk[32];
+                    exp_pairs<C::EMU_PER8, 0, 32>(s, pk, scale2, neg2, la);
+                    tmem_st32(s_addr, pk);
+                    exp_pairs<C::EMU_PER8, 32, 32>(s, pk, scale2, neg2, la);
+                    tmem_st32(s_addr + 32, pk);
+                    if (rescale) {
+#pragma unroll
+                        for (int pc = 0; pc < D / 32; pc++) {
+                            uint32_t o[32];
+                            tmem_ld32(o_addr + pc * 32, o);
+#pragma unroll
+                            for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                            tmem_st32(o_addr + pc * 32, o);
+                        }
+                    }
+                    float a0, a1, b0, b1;
+                    unpack2(la[0], a0, a1);
+                    unpack2(la[1], b0, b1);
+                    l0 = fmaf(l0, f, a0 + b0);
+                    l1 = fmaf(l1, f, a1 + b1);
                 }
-                float a0, a1, b0, b1;
-                unpack2(la[0], a0, a1);
-                unpack2(la[1], b0, b1);
-                l0 = fmaf(l0, f, a0 + b0);
-                l1 = fmaf(l1, f, a1 + b1);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(p_full + t);
