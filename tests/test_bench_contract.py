@@ -68,3 +68,19 @@ def test_gpu_arm_fails_loudly_without_a_device():
     r = _run(["--workload", SMALL, "--steps", "1", "--warmup", "0", "--no-cpu-baseline"])
     assert r.returncode != 0
     assert not any(ln.startswith("{") for ln in r.stdout.splitlines())
+
+
+def test_select_mode_names_config_fields():
+    """--select-mode accepts only the listed options, and every option sets
+    fields the binding's Config has (the main call's contexts take them)."""
+    import bench
+    from clustered_sparse_attention_head_b200 import workloads as W
+    from clustered_sparse_attention_head_b200.api import Config
+    r = _run(["--select-mode", "no_such_mode", "--steps", "1"])
+    assert r.returncode == 2 and "invalid choice" in r.stderr
+    cfg = Config.from_workload(W.WORKLOADS["wan21-n75600-h40-d128"])
+    assert bench.SELECT_MODES, "no selection options listed"
+    for name, over in bench.SELECT_MODES.items():
+        for key in over:
+            assert hasattr(cfg, key), f"{name}: Config has no field {key}"
+    assert bench.SELECT_MODES["per_query_top_k64"] == {"top_k": 64, "per_query": True}
