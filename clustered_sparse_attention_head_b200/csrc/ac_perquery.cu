@@ -2,17 +2,20 @@
 // row per query token, Index <- argtopk(S, topk) along each row), and the
 // tables that let the block-sparse attention kernel honour each row's own set.
 //
-//  1. pq_scores_kernel: s_ib for every query row i and key cluster b, in double
-//     with the oracle's summation order (each thread 4 x 4 scores, elements
-//     in order): CENTROID s = (q_i . c_b) / sqrt(d); QUEST s = sum_t
-//     max(q_t M_bt, q_t m_bt) / sqrt(d) (the query is its own representative).
-//     A bf16 or fp32 element times an fp32 centroid element has at most 48
-//     significant bits, so its double product is exact and one fused
-//     multiply-add per element rounds exactly where a multiply then an add does.
+//  1. pq_scores_c_kernel (CENTROID scores, 16-byte aligned operands) and
+//     pq_scores_kernel (QUEST scores, or unaligned operands): s_ib for every
+//     query row i and key cluster b, in double with the oracle's summation
+//     order (elements in order): CENTROID s = (q_i . c_b) / sqrt(d); QUEST
+//     s = sum_t max(q_t M_bt, q_t m_bt) / sqrt(d) (the query is its own
+//     representative).  A bf16 or fp32 element times an fp32 centroid element
+//     has at most 48 significant bits, so its double product is exact and one
+//     fused multiply-add per element rounds exactly where a multiply then an
+//     add does.
 //  2. pq_topk_kernel: one warp per row keeps the top_k non-empty clusters of
 //     largest s (ties to the lower id) as a bit set [H, N, W] (W = kk_cap / 32
-//     words); the text-key group, if any, is always set.  It also sums the
-//     row's pairs (sum of the selected clusters' sizes).
+//     words), by a warp quickselect up to 512 clusters; the text-key group, if
+//     any, is always set.  It also sums the row's pairs (sum of the selected
+//     clusters' sizes).
 //  3. pq_union_kernel: per query cluster, the union of its rows' sets, as the
 //     ascending sel_idx / sel_cnt lists the work list and key runs take.
 //  4. key_runs_single_kernel: one key run per selected non-empty cluster (not
