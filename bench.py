@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.ORDER)
     ap.add_argument("--top-p", type=float, default=None)
     ap.add_argument("--heads", type=int, default=None, help="fewer heads (profiling captures only)")
+    ap.add_argument("--kq", type=int, default=None, help="another query cluster count (selection timings)")
+    ap.add_argument("--kk", type=int, default=None, help="another key cluster count (selection timings)")
     ap.add_argument("--select-mode", default=None, choices=sorted(SELECT_MODES),
                     help="time the main call with one of the selection options instead of the top-p cut")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -251,6 +253,10 @@ def main():
         w = replace(w, top_p=a.top_p)
     if a.heads is not None:
         w = replace(w, heads=a.heads)
+    if a.kq is not None:
+        w = replace(w, kq=a.kq)
+    if a.kk is not None:
+        w = replace(w, kk=a.kk)
     if a.impl == "reference":
         return run_reference(a, w)
 
