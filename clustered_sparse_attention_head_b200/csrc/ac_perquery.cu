@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(256, 1) pq_scores_c_kernel(const T *__restrict
 // already taken skipped.  Up to four warps per block, fewer when kk_cap is
 // large; each warp takes rows in turn and adds its rows' pairs to the head's
 // total once.
-constexpr int PQ_WARPS = 4, PQ_SORTED = 512;
+// PQ_REG_CLUSTERS: most key clusters a row holds in its lanes' registers (16 per lane)
+constexpr int PQ_WARPS = 4, PQ_REG_CLUSTERS = 512;
 // bytes of a warp's score region
 __host__ __device__ constexpr size_t pq_topk_region(int kk_cap) { return (size_t)kk_cap * 8; }
 // blocks per head of the top-k launch
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(PQ_WARPS * 32, 4) pq_topk_kernel(const double 
     const int nkh = nkh_all - text_group;
     const int32_t *kc = k_count + (size_t)h * kk_cap;
     const bool dn = dense && dense[h];
-    const bool regs = nkh <= PQ_SORTED;
+    const bool regs = nkh <= PQ_REG_CLUSTERS;
     // register path: the lane's clusters that hold keys
     uint32_t km = 0u;
 #pragma unroll
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(PQ_WARPS * 32, 4) pq_topk_kernel(const double 
                 uint32_t C = vm, S = 0u;
                 int base = 0;
                 sel = 0u;
-                for (int it = 0; it < PQ_SORTED; it++) {  // each round drops at least the pivot from C
+                for (int it = 0; it < PQ_REG_CLUSTERS; it++) {  // each round drops at least the pivot from C
                     const uint32_t lanes = __ballot_sync(full, C != 0u);
                     const int rot = (it * 13 + r * 7) & 31;
                     const uint32_t rl = rot ? ((lanes >> rot) | (lanes << (32 - rot))) : lanes;
