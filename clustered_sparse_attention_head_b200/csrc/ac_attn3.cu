@@ -742,12 +742,14 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t c = cnt + j;
                 if (!mbar_wait_warp(s_full + t, c & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
-                // A warp none of whose rows takes a key of this chunk (rows past
-                // the item's query rows, whose output is never written, and rows
-                // that keep none of the chunk's groups) would compute P = 0 with
-                // its row maxima, sums and O unchanged: it stores the zeros
-                // (after S_t(j) is complete, as P always is) and skips the rest.
-                if (__all_sync(0xffffffffu, !valid || (ROWS && drop == 0xFFFFu))) {
+                // Per-query selection: a warp none of whose rows takes a key of
+                // this chunk (rows that keep none of the chunk's groups, and rows
+                // past the item's query rows, whose output is never written)
+                // would compute P = 0 with its row maxima, sums and O unchanged:
+                // it stores the zeros (after S_t(j) is complete, as P always is)
+                // and skips the rest.  (The default instance gained nothing from
+                // skipping its all-padding warps and keeps the full path.)
+                if (ROWS && __all_sync(0xffffffffu, !valid || drop == 0xFFFFu)) {
                     tmem_st32_zero(s_addr);
                     tmem_st32_zero(s_addr + 32);
                 } else {
