@@ -84,3 +84,11 @@ def test_select_mode_names_config_fields():
         for key in over:
             assert hasattr(cfg, key), f"{name}: Config has no field {key}"
     assert bench.SELECT_MODES["per_query_top_k64"] == {"top_k": 64, "per_query": True}
+
+
+def test_cluster_count_overrides_reach_the_config():
+    r = _run(["--impl", "reference", "--workload", SMALL, "--kq", "9", "--kk", "13", "--steps", "1",
+              "--warmup", "0"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    j = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][0])
+    assert j["config"]["kq"] == 9 and j["config"]["kk"] == 13
